@@ -1,0 +1,183 @@
+/*
+ * kvq.h - C ABI of the rotated-INT4 paged KV cache (the data-parallel hot
+ * path of SAW-INT4: token-wise INT4 quantization with a block-diagonal
+ * Hadamard rotation, written into a paged KV cache and read back by a fused
+ * decode-attention kernel).
+ *
+ * Sources (web pages, cited by title and section):
+ *  [SAW]   "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World
+ *          LLM Serving", Abstract (arXiv 2604.19157 mirror): token-wise INT4
+ *          with block-diagonal Hadamard rotation; a fused rotation-quantization
+ *          kernel that writes straight into paged KV-cache layouts; fused
+ *          attention execution over the quantized cache.
+ *  [OSCAR] "OScaR: Occam's Razor for Extreme KV Cache Quantization in LLMs"
+ *          (forum summary), section "The OScaR Framework": V^ = Quant(S.(R.V)),
+ *          rotate first, then scale, then quantize.
+ * The pages fix no layout, rounding rule or API; every such choice below is a
+ * reading of this library and is stated where it is made.
+ *
+ * Conventions shared by every entry point
+ *  - All pointers named "device" are CUDA device pointers; the caller owns
+ *    every buffer, and no entry point allocates device memory.
+ *  - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).
+ *    Every call is asynchronous on that stream.
+ *  - Argument errors are reported synchronously, before anything is launched.
+ *  - Range errors found on the device (a slot or page id outside the pool, a
+ *    context longer than the page table) skip the offending row or page and
+ *    record a status in a per-device error word; a bounded wait that ran out
+ *    records KVQ_ERR_TIMEOUT there. kvq_get_device_error() reads and clears it.
+ *
+ * Data layout (this library's reading; the pages only say "paged"):
+ *  - page size P = 16 tokens (KVQ_PAGE_SIZE).
+ *  - cache : uint8  [num_pages][Hkv][2][P][D/2]  (index 2: 0 = K, 1 = V)
+ *            one row = D 4-bit codes of one (token, kv head, K|V);
+ *            byte j of a row = code[2j] | (code[2j+1] << 4)  (low nibble = even
+ *            channel).
+ *  - scales: fp16   [num_pages][Hkv][2][P]   the per-row step s
+ *  - zeros : fp16   [num_pages][Hkv][2][P]   the per-row offset z
+ *            dequantized value = code * s + z.
+ *  - slot  : page * 16 + offset within the page.
+ */
+#ifndef KVQ_H
+#define KVQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define KVQ_PAGE_SIZE 16
+#define KVQ_ABI_VERSION 1
+
+typedef enum kvq_status {
+  KVQ_OK = 0,
+  KVQ_ERR_INVALID_ARG = 1,  /* null pointer, bad size, misaligned buffer */
+  KVQ_ERR_UNSUPPORTED = 2,  /* head_dim, block size or GQA group not built */
+  KVQ_ERR_OUT_OF_RANGE = 3, /* device-side: slot/page id/context outside the pool */
+  KVQ_ERR_WORKSPACE = 4,    /* workspace missing or smaller than required */
+  KVQ_ERR_TIMEOUT = 5,      /* device-side: a bounded wait ran out */
+  KVQ_ERR_CUDA = 6          /* a CUDA runtime call or launch failed */
+} kvq_status;
+
+/* Shapes of one kv_quant_write call. */
+typedef struct kvq_write_desc {
+  int32_t num_tokens;   /* T >= 0 new tokens */
+  int32_t num_kv_heads; /* Hkv >= 1 */
+  int32_t head_dim;     /* D: 64 or 128 */
+  int32_t page_size;    /* must be KVQ_PAGE_SIZE */
+  int32_t num_pages;    /* pages in the pool; valid slots are [0, num_pages*16) */
+} kvq_write_desc;
+
+/* Shapes of one paged_decode_attn_int4 call. */
+typedef struct kvq_attn_desc {
+  int32_t batch;             /* B sequences, one query token each */
+  int32_t num_q_heads;       /* Hq; query head i reads kv head i / (Hq/Hkv) */
+  int32_t num_kv_heads;      /* Hkv; Hq/Hkv must be 1, 2, 4 or 8 */
+  int32_t head_dim;          /* D: 64 or 128 */
+  int32_t page_size;         /* must be KVQ_PAGE_SIZE */
+  int32_t num_pages;         /* pages in the pool */
+  int32_t max_pages_per_seq; /* columns of page_table */
+  int32_t hadamard_block;    /* the block b the cache was written with (0 = none) */
+  float softmax_scale;       /* 0 means 1/sqrt(head_dim) */
+  int32_t out_dtype;         /* 0 = fp32 output, 1 = bf16 output */
+} kvq_attn_desc;
+
+/*
+ * kv_quant_write - fused rotate + token-wise INT4 quantize + paged store
+ * ([SAW] Abstract: "fused rotation-quantization kernel that integrates
+ * directly into paged KV-cache layouts"; [OSCAR] "The OScaR Framework":
+ * rotate, then quantize).
+ *
+ * For every new token t, kv head h and tensor X in {K, V}, with row x = X[t,h,:]:
+ *   1. y = R x, R = diag(H_b/sqrt(b), ...) over contiguous b-channel blocks,
+ *      H_b the Sylvester Hadamard matrix in natural order
+ *      (H[i][j] = (-1)^popcount(i & j)); b = 0 means R = I (plain INT4).
+ *      y is fp32.
+ *   2. z = the largest fp16 <= min(y); s = the smallest fp16 >= 0 with
+ *      15*s + z >= max(y) (so every element lies in [z, z + 15 s]).
+ *   3. code = round-half-even( fp32(y - z) * fp32(1/s) ), in [0, 15]; s = 0
+ *      gives code 0.
+ *   4. the packed row, s and z go to slot slot_mapping[t]; slot -1 skips t.
+ *
+ * k, v         : device, bf16 [T][Hkv][D], contiguous, 16-byte aligned.
+ * slot_mapping : device, int64 [T]; -1 = skip; any other value outside
+ *                [0, num_pages*16) skips the token and records
+ *                KVQ_ERR_OUT_OF_RANGE in the device error word.
+ * page_table   : accepted for signature compatibility with the decode call and
+ *                not read; placement is decided by slot_mapping alone. May be NULL.
+ * cache, scales, zeros : device, layouts above, 16-byte aligned.
+ * hadamard_block : 0, 32, 64 or 128, and at most D.
+ * desc         : host pointer to the shapes.
+ * Inputs must be finite and their rotated values must lie within the fp16
+ * range (|y| <= 65504); rows outside it get infinite or NaN s/z.
+ * Returns KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED or KVQ_ERR_CUDA.
+ */
+kvq_status kv_quant_write(const void* k, const void* v, const int64_t* slot_mapping,
+                          const int32_t* page_table, uint8_t* cache, void* scales,
+                          void* zeros, int32_t hadamard_block,
+                          const kvq_write_desc* desc, void* stream);
+
+/*
+ * kvq_attn_workspace_size - bytes of device workspace paged_decode_attn_int4
+ * needs for these shapes (0 when the call needs none). The value depends on
+ * the shapes and on the current device's SM count only.
+ */
+size_t kvq_attn_workspace_size(const kvq_attn_desc* desc);
+
+/*
+ * paged_decode_attn_int4 - one decode step of attention over the INT4 cache
+ * ([SAW] Abstract: "fused attention execution"; the rotation is orthogonal,
+ * so q.k = (Rq).(Rk) and the output is R^T sum_t p_t (R v_t), with R^T = R
+ * because H_b/sqrt(b) is symmetric and its own inverse).
+ *
+ * For sequence n and query head i (kv head h = i / (Hq/Hkv)), over the
+ * context_lens[n] cached tokens t with page = page_table[n][t/16]:
+ *   k^_t = code*s + z (per row), likewise v^_t, both in rotated space;
+ *   logit_t = softmax_scale * (R q) . k^_t;  p = softmax(logit);
+ *   out[n][i] = R (sum_t p_t v^_t).      context_lens[n] = 0 gives out = 0.
+ *
+ * q            : device, bf16 [B][Hq][D], contiguous.
+ * cache, scales, zeros : device, as written by kv_quant_write with the same
+ *                hadamard_block.
+ * page_table   : device, int32 [B][max_pages_per_seq]; entries past the
+ *                context are not read. An id outside [0, num_pages) makes the
+ *                page count as empty and records KVQ_ERR_OUT_OF_RANGE.
+ * context_lens : device, int32 [B]; a value above max_pages_per_seq*16 is
+ *                clamped and records KVQ_ERR_OUT_OF_RANGE.
+ * out          : device, [B][Hq][D], fp32 or bf16 (desc->out_dtype).
+ * workspace    : device, at least kvq_attn_workspace_size(desc) bytes, 16-byte
+ *                aligned; may be NULL when that size is 0. It must be all zero
+ *                before its first use; every call leaves it all zero again, so
+ *                one buffer serves any number of calls issued one after
+ *                another on a stream (calls that overlap on the GPU must use
+ *                different workspaces).
+ * Returns KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_WORKSPACE
+ * or KVQ_ERR_CUDA.
+ */
+kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache,
+                                  const void* scales, const void* zeros,
+                                  const int32_t* page_table,
+                                  const int32_t* context_lens, void* out,
+                                  void* workspace, size_t workspace_bytes,
+                                  const kvq_attn_desc* desc, void* stream);
+
+/*
+ * kvq_get_device_error - synchronizes `stream`, then returns and clears the
+ * current device's error word (KVQ_OK when no kernel recorded an error).
+ * Returns KVQ_ERR_CUDA if the synchronization itself fails.
+ */
+kvq_status kvq_get_device_error(void* stream);
+
+/* Static, human-readable name of a status value (never NULL). */
+const char* kvq_status_string(int32_t status);
+
+/* KVQ_ABI_VERSION of the built library. */
+int32_t kvq_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* KVQ_H */

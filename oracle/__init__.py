@@ -1,0 +1,267 @@
+"""CPU oracle of the rotated-INT4 paged KV cache (test infrastructure).
+
+Only the test suite, ``__graft_entry__.smoke()`` and the ``cpu_baseline`` leg
+of ``bench.py`` may import this package. It wraps ``kvq_oracle.c`` (plain C,
+fp64) with numpy marshalling; it never imports the CUDA package.
+
+The arithmetic is in ``kvq_oracle.c``; see its header for the pages it
+follows and the readings it takes.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+import subprocess
+
+import numpy as np
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_SRC = os.path.join(_HERE, "kvq_oracle.c")
+_LIB = os.path.join(_HERE, "libkvq_oracle.so")
+
+_lib = None
+
+
+def build(force: bool = False) -> str:
+    """Compile kvq_oracle.c into libkvq_oracle.so next to it (gcc, OpenMP)."""
+    if force or not os.path.exists(_LIB) or os.path.getmtime(_LIB) < os.path.getmtime(_SRC):
+        tmp = _LIB + f".tmp{os.getpid()}"
+        subprocess.check_call(
+            ["gcc", "-O2", "-std=c11", "-fopenmp", "-shared", "-fPIC", _SRC, "-o", tmp, "-lm"]
+        )
+        os.replace(tmp, _LIB)
+    return _LIB
+
+
+def _p(dtype):
+    return np.ctypeslib.ndpointer(dtype=dtype, flags="C_CONTIGUOUS")
+
+
+def lib():
+    global _lib
+    if _lib is None:
+        L = ctypes.CDLL(build())
+        u16, u8, i8, f32, f64, i64, i32 = (np.uint16, np.uint8, np.int8, np.float32,
+                                            np.float64, np.int64, np.int32)
+        c_int, c_i64, c_d = ctypes.c_int, ctypes.c_int64, ctypes.c_double
+        sig = {
+            "oracle_bf16_to_double": (c_d, [ctypes.c_uint16]),
+            "oracle_half_to_double": (c_d, [ctypes.c_uint16]),
+            "oracle_half_round_down": (ctypes.c_uint16, [c_d]),
+            "oracle_half_round_up": (ctypes.c_uint16, [c_d]),
+            "oracle_half_round_nearest": (ctypes.c_uint16, [c_d]),
+            "oracle_hadamard": (None, [c_int, _p(i8)]),
+            "oracle_rotate_f64": (c_int, [_p(f64), c_int, c_int, _p(f64)]),
+            "oracle_rotate_row": (c_int, [_p(u16), c_int, c_int, _p(f32)]),
+            "oracle_scale_zero": (None, [ctypes.c_float, ctypes.c_float,
+                                         ctypes.POINTER(ctypes.c_uint16),
+                                         ctypes.POINTER(ctypes.c_uint16)]),
+            "oracle_quantize_given": (None, [_p(f32), c_int, ctypes.c_uint16, ctypes.c_uint16, _p(u8)]),
+            "oracle_quotient_given": (None, [_p(f32), c_int, ctypes.c_uint16, ctypes.c_uint16, _p(f64)]),
+            "oracle_quantize_row": (None, [_p(f32), c_int, _p(u8), ctypes.POINTER(ctypes.c_uint16),
+                                           ctypes.POINTER(ctypes.c_uint16)]),
+            "oracle_pack_row": (None, [_p(u8), c_int, _p(u8)]),
+            "oracle_unpack_row": (None, [_p(u8), c_int, _p(u8)]),
+            "oracle_dequant_row": (None, [_p(u8), c_int, ctypes.c_uint16, ctypes.c_uint16, _p(f64)]),
+            "oracle_cache_row_offset": (ctypes.c_size_t, [c_i64, c_int, c_int, c_int, c_int, c_int]),
+            "oracle_scale_offset": (ctypes.c_size_t, [c_i64, c_int, c_int, c_int, c_int]),
+            "oracle_quant_write": (c_int, [_p(u16), _p(u16), _p(i64), c_int, c_int, c_int, c_int, c_i64,
+                                           _p(u8), _p(u16), _p(u16), ctypes.c_void_p]),
+            "oracle_attn_rows": (c_int, [_p(f64), _p(f64), _p(f64), c_int, c_int, c_int, c_d, _p(f64)]),
+            "oracle_decode_one": (c_int, [_p(u16), _p(u8), _p(u16), _p(u16), _p(i32), _p(i32),
+                                          c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_i64,
+                                          c_d, _p(f64)]),
+            "oracle_decode_attn": (c_int, [_p(u16), _p(u8), _p(u16), _p(u16), _p(i32), _p(i32),
+                                           c_int, c_int, c_int, c_int, c_int, c_int, c_i64, c_d,
+                                           _p(f64)]),
+            "oracle_num_threads": (c_int, []),
+        }
+        for name, (res, args) in sig.items():
+            fn = getattr(L, name)
+            fn.restype = res
+            fn.argtypes = args
+        _lib = L
+    return _lib
+
+
+def _c(a, dtype):
+    return np.ascontiguousarray(a, dtype=dtype)
+
+
+# --- number formats -------------------------------------------------------
+
+def half_to_double(bits: int) -> float:
+    return lib().oracle_half_to_double(int(bits))
+
+
+def half_round_down(x: float) -> int:
+    return lib().oracle_half_round_down(float(x))
+
+
+def half_round_up(x: float) -> int:
+    return lib().oracle_half_round_up(float(x))
+
+
+def half_round_nearest(x: float) -> int:
+    return lib().oracle_half_round_nearest(float(x))
+
+
+def bf16_to_double(bits: int) -> float:
+    return lib().oracle_bf16_to_double(int(bits))
+
+
+# --- rotation -------------------------------------------------------------
+
+def hadamard(b: int) -> np.ndarray:
+    H = np.zeros(b * b, np.int8)
+    lib().oracle_hadamard(b, H)
+    return H.reshape(b, b)
+
+
+def rotate_f64(x, b: int) -> np.ndarray:
+    x = _c(x, np.float64)
+    y = np.zeros_like(x)
+    rc = lib().oracle_rotate_f64(x, x.size, b, y)
+    assert rc == 0, rc
+    return y
+
+
+def rotate_row(x_bf16_bits, b: int) -> np.ndarray:
+    x = _c(x_bf16_bits, np.uint16)
+    y = np.zeros(x.size, np.float32)
+    rc = lib().oracle_rotate_row(x, x.size, b, y)
+    assert rc == 0, rc
+    return y
+
+
+# --- quantization ---------------------------------------------------------
+
+def scale_zero(mn: float, mx: float):
+    s, z = ctypes.c_uint16(), ctypes.c_uint16()
+    lib().oracle_scale_zero(float(mn), float(mx), ctypes.byref(s), ctypes.byref(z))
+    return s.value, z.value
+
+
+def quantize_row(y):
+    y = _c(y, np.float32)
+    codes = np.zeros(y.size, np.uint8)
+    s, z = ctypes.c_uint16(), ctypes.c_uint16()
+    lib().oracle_quantize_row(y, y.size, codes, ctypes.byref(s), ctypes.byref(z))
+    return codes, s.value, z.value
+
+
+def quantize_given(y, s: int, z: int) -> np.ndarray:
+    y = _c(y, np.float32)
+    codes = np.zeros(y.size, np.uint8)
+    lib().oracle_quantize_given(y, y.size, int(s), int(z), codes)
+    return codes
+
+
+def quotient_given(y, s: int, z: int) -> np.ndarray:
+    y = _c(y, np.float32)
+    q = np.zeros(y.size, np.float64)
+    lib().oracle_quotient_given(y, y.size, int(s), int(z), q)
+    return q
+
+
+def pack_row(codes) -> np.ndarray:
+    codes = _c(codes, np.uint8)
+    out = np.zeros(codes.size // 2, np.uint8)
+    lib().oracle_pack_row(codes, codes.size, out)
+    return out
+
+
+def unpack_row(packed, D: int) -> np.ndarray:
+    packed = _c(packed, np.uint8)
+    out = np.zeros(D, np.uint8)
+    lib().oracle_unpack_row(packed, D, out)
+    return out
+
+
+def dequant_row(packed, D: int, s: int, z: int) -> np.ndarray:
+    packed = _c(packed, np.uint8)
+    out = np.zeros(D, np.float64)
+    lib().oracle_dequant_row(packed, D, int(s), int(z), out)
+    return out
+
+
+def cache_row_offset(page: int, Hkv: int, D: int, h: int, kv: int, off: int) -> int:
+    return lib().oracle_cache_row_offset(page, Hkv, D, h, kv, off)
+
+
+def scale_offset(page: int, Hkv: int, h: int, kv: int, off: int) -> int:
+    return lib().oracle_scale_offset(page, Hkv, h, kv, off)
+
+
+def quant_write(k_bits, v_bits, slot_mapping, num_pages: int, b: int, cache=None,
+                scales=None, zeros=None, want_y: bool = False):
+    """Rotate, quantize and place every row. k_bits/v_bits: uint16 [T, Hkv, D]
+    bf16 bit patterns. Returns (cache, scales, zeros, y) where y is the fp32
+    rotated rows [T, Hkv, 2, D] (or None). Buffers passed in are updated."""
+    k = _c(k_bits, np.uint16)
+    v = _c(v_bits, np.uint16)
+    T, Hkv, D = k.shape
+    sm = _c(slot_mapping, np.int64)
+    if cache is None:
+        cache = np.zeros(num_pages * Hkv * 2 * 16 * D // 2, np.uint8)
+    if scales is None:
+        scales = np.zeros(num_pages * Hkv * 2 * 16, np.uint16)
+    if zeros is None:
+        zeros = np.zeros(num_pages * Hkv * 2 * 16, np.uint16)
+    assert cache.flags.c_contiguous and scales.flags.c_contiguous and zeros.flags.c_contiguous
+    y = np.zeros((T, Hkv, 2, D), np.float32) if want_y else None
+    rc = lib().oracle_quant_write(k, v, sm, T, Hkv, D, b, num_pages,
+                                  cache.reshape(-1), scales.reshape(-1), zeros.reshape(-1),
+                                  y.ctypes.data if y is not None else None)
+    if rc != 0:
+        raise ValueError(f"oracle_quant_write returned {rc}")
+    return cache, scales, zeros, y
+
+
+# --- attention ------------------------------------------------------------
+
+def attn_rows(q, Krot, Vrot, b: int, scale: float) -> np.ndarray:
+    q = _c(q, np.float64)
+    D = q.size
+    Krot = _c(Krot, np.float64).reshape(-1, D)
+    Vrot = _c(Vrot, np.float64).reshape(-1, D)
+    out = np.zeros(D, np.float64)
+    rc = lib().oracle_attn_rows(q, Krot.reshape(-1), Vrot.reshape(-1), Krot.shape[0], D, b,
+                                float(scale), out)
+    assert rc == 0, rc
+    return out
+
+
+def decode_attn(q_bits, cache, scales, zeros, page_table, context_lens, Hkv: int, b: int,
+                num_pages: int, softmax_scale: float = 0.0) -> np.ndarray:
+    q = _c(q_bits, np.uint16)
+    B, Hq, D = q.shape
+    pt = _c(page_table, np.int32)
+    cl = _c(context_lens, np.int32)
+    out = np.zeros((B, Hq, D), np.float64)
+    rc = lib().oracle_decode_attn(q.reshape(-1), _c(cache, np.uint8).reshape(-1),
+                                  _c(scales, np.uint16).reshape(-1), _c(zeros, np.uint16).reshape(-1),
+                                  pt.reshape(-1), cl, B, Hq, Hkv, D, b, pt.shape[1], num_pages,
+                                  float(softmax_scale), out.reshape(-1))
+    if rc != 0:
+        raise ValueError(f"oracle_decode_attn returned {rc}")
+    return out
+
+
+def decode_one(q_bits, cache, scales, zeros, page_table, context_lens, n: int, hq: int,
+               Hkv: int, b: int, num_pages: int, softmax_scale: float = 0.0) -> np.ndarray:
+    q = _c(q_bits, np.uint16)
+    B, Hq, D = q.shape
+    pt = _c(page_table, np.int32)
+    out = np.zeros(D, np.float64)
+    rc = lib().oracle_decode_one(q.reshape(-1), _c(cache, np.uint8).reshape(-1),
+                                 _c(scales, np.uint16).reshape(-1), _c(zeros, np.uint16).reshape(-1),
+                                 pt.reshape(-1), _c(context_lens, np.int32), n, hq, Hq, Hkv, D, b,
+                                 pt.shape[1], num_pages, float(softmax_scale), out)
+    if rc != 0:
+        raise ValueError(f"oracle_decode_one returned {rc}")
+    return out
+
+
+def num_threads() -> int:
+    return lib().oracle_num_threads()

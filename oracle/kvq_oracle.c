@@ -1,0 +1,424 @@
+/*
+ * kvq_oracle.c - plain, slow CPU statement of the rotated-INT4 paged KV cache.
+ *
+ * TEST INFRASTRUCTURE. Only the test suite, the package smoke check and the
+ * CPU-baseline leg of the benchmark may load this library. It shares no code,
+ * header, table or constant with the CUDA path.
+ *
+ * What it follows (web pages, cited by title and section):
+ *  [SAW]   "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World
+ *          LLM Serving", Abstract: token-wise INT4 quantization with a
+ *          block-diagonal Hadamard rotation, stored in a paged KV cache, read
+ *          back by fused attention.
+ *  [OSCAR] "OScaR: Occam's Razor for Extreme KV Cache Quantization in LLMs",
+ *          section "The OScaR Framework": V^ = Quant(S.(R.V)) - rotate the
+ *          cache, apply the per-token scaling, then quantize.
+ *
+ * Readings where the pages are silent (each is a choice of this library):
+ *  - R = diag(H_b/sqrt(b), ...) over contiguous b-channel blocks, H_b the
+ *    Sylvester Hadamard matrix in natural order, no random signs; b = 0 = I.
+ *  - one (s, z) pair per row = (token, kv head, K or V) over all D channels.
+ *  - z = largest fp16 <= min(y); s = smallest fp16 >= 0 with 15 s + z >= max(y).
+ *  - code = round-half-even(fp32(y - z) * fp32(1/s)); s = 0 gives code 0.
+ *    (The decision is taken in the kernel's fp32 arithmetic on both sides.)
+ *  - byte j of a packed row = code[2j] | code[2j+1] << 4.
+ *  - cache [page][Hkv][2][16][D/2], scales/zeros [page][Hkv][2][16].
+ *  - attention: softmax_scale defaults to 1/sqrt(D); out = R sum_t p_t v^_t.
+ *
+ * Everything here is a direct definition: a dense Hadamard matrix, fp64 sums,
+ * scalar quantize/dequantize, brute-force softmax. Built with
+ *   gcc -O2 -fopenmp -shared -fPIC kvq_oracle.c -o libkvq_oracle.so -lm
+ * (oracle/build_oracle.py does this).
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORACLE_PAGE 16
+
+/* ------------------------------------------------------------------------- */
+/* Number formats, from the IEEE-754 binary16 and bfloat16 bit layouts.      */
+/* ------------------------------------------------------------------------- */
+
+/* bfloat16 is the top 16 bits of an IEEE binary32. */
+double oracle_bf16_to_double(uint16_t b) {
+  uint32_t u = (uint32_t)b << 16;
+  float f;
+  memcpy(&f, &u, 4);
+  return (double)f;
+}
+
+/* binary16: 1 sign bit, 5 exponent bits (bias 15), 10 fraction bits. */
+double oracle_half_to_double(uint16_t h) {
+  int sign = (h >> 15) & 1;
+  int e = (h >> 10) & 31;
+  int m = h & 1023;
+  double v;
+  if (e == 0) {
+    v = ldexp((double)m, -24); /* subnormal: m * 2^-14 * 2^-10 */
+  } else if (e == 31) {
+    v = (m == 0) ? INFINITY : NAN;
+  } else {
+    v = ldexp((double)(1024 + m), e - 25); /* (1 + m/1024) * 2^(e-15) */
+  }
+  return sign ? -v : v;
+}
+
+/* Non-negative binary16 patterns 0x0000..0x7C00 (0 .. +inf) are ordered like
+ * their values; the roundings below search that ordered set. */
+static uint16_t smallest_half_at_least(double x) { /* x >= 0 */
+  uint16_t lo = 0, hi = 0x7C00;
+  while (lo < hi) {
+    uint16_t mid = (uint16_t)((lo + hi) / 2);
+    if (oracle_half_to_double(mid) >= x) hi = mid; else lo = (uint16_t)(mid + 1);
+  }
+  return lo;
+}
+
+static uint16_t largest_half_at_most(double x) { /* x >= 0 */
+  uint16_t lo = 0, hi = 0x7C00;
+  while (lo < hi) {
+    uint16_t mid = (uint16_t)((lo + hi + 1) / 2);
+    if (oracle_half_to_double(mid) <= x) lo = mid; else hi = (uint16_t)(mid - 1);
+  }
+  return lo;
+}
+
+/* Round toward -inf to binary16. */
+uint16_t oracle_half_round_down(double x) {
+  if (!signbit(x)) return largest_half_at_most(x);
+  uint16_t m = smallest_half_at_least(-x);
+  return (uint16_t)(m | 0x8000);
+}
+
+/* Round toward +inf to binary16. */
+uint16_t oracle_half_round_up(double x) {
+  if (!signbit(x)) {
+    uint16_t r = smallest_half_at_least(x);
+    return r;
+  }
+  uint16_t m = largest_half_at_most(-x);
+  return (uint16_t)(m | 0x8000);
+}
+
+/* Round to nearest, ties to even, to binary16 (overflow at >= 65520). */
+uint16_t oracle_half_round_nearest(double x) {
+  double a = fabs(x);
+  uint16_t sign = signbit(x) ? 0x8000 : 0;
+  uint16_t d = largest_half_at_most(a);
+  double dv = oracle_half_to_double(d);
+  if (dv == a) return (uint16_t)(d | sign);
+  /* the next value above 65504 counts as 65536 when judging nearness */
+  double uv = (d == 0x7BFF) ? 65536.0 : oracle_half_to_double((uint16_t)(d + 1));
+  uint16_t u = (uint16_t)(d + 1);
+  uint16_t r;
+  if (a - dv < uv - a) r = d;
+  else if (a - dv > uv - a) r = u;
+  else r = (d & 1) ? u : d;
+  return (uint16_t)(r | sign);
+}
+
+/* ------------------------------------------------------------------------- */
+/* Rotation: block-diagonal Hadamard ([SAW] Abstract; [OSCAR] R.V).          */
+/* ------------------------------------------------------------------------- */
+
+static int popcount_u32(uint32_t v) {
+  int c = 0;
+  while (v) { c += (int)(v & 1u); v >>= 1; }
+  return c;
+}
+
+/* Dense Sylvester Hadamard matrix of order b (a power of two), natural order:
+ * H[i*b + j] = (-1)^popcount(i & j). */
+void oracle_hadamard(int b, int8_t* H) {
+  for (int i = 0; i < b; ++i)
+    for (int j = 0; j < b; ++j)
+      H[i * b + j] = (popcount_u32((uint32_t)(i & j)) & 1) ? -1 : 1;
+}
+
+static int valid_block(int D, int b) {
+  if (b == 0) return 1;
+  if (b != 32 && b != 64 && b != 128) return 0;
+  return (D % b) == 0;
+}
+
+/* y = R x in fp64 for an fp64 row: y[blk + i] = (1/sqrt(b)) sum_j H[i][j] x[blk + j].
+ * b = 0 copies x. */
+int oracle_rotate_f64(const double* x, int D, int b, double* y) {
+  if (!valid_block(D, b)) return -1;
+  if (b == 0) {
+    for (int c = 0; c < D; ++c) y[c] = x[c];
+    return 0;
+  }
+  int8_t* H = (int8_t*)malloc((size_t)b * b);
+  oracle_hadamard(b, H);
+  double norm = 1.0 / sqrt((double)b);
+  for (int blk = 0; blk < D; blk += b) {
+    for (int i = 0; i < b; ++i) {
+      double acc = 0.0;
+      for (int j = 0; j < b; ++j) acc += (double)H[i * b + j] * x[blk + j];
+      y[blk + i] = acc * norm;
+    }
+  }
+  free(H);
+  return 0;
+}
+
+/* The rotated bf16 row, rounded once to fp32 (the precision the kernels keep
+ * between rotation and quantization). */
+int oracle_rotate_row(const uint16_t* x_bf16, int D, int b, float* y) {
+  double xd[256], yd[256];
+  if (D <= 0 || D > 256) return -1;
+  for (int c = 0; c < D; ++c) xd[c] = oracle_bf16_to_double(x_bf16[c]);
+  if (oracle_rotate_f64(xd, D, b, yd) != 0) return -1;
+  for (int c = 0; c < D; ++c) y[c] = (float)yd[c];
+  return 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Token-wise asymmetric INT4 quantization ([SAW] Abstract "token-wise INT4"; */
+/* [OSCAR] Quant(.) after the rotation).                                     */
+/* ------------------------------------------------------------------------- */
+
+/* z = largest fp16 <= mn; s = smallest fp16 >= 0 with 15 s + z >= mx.
+ * 15 s + z is exact in fp64 (both are binary16 values), so the test is exact. */
+void oracle_scale_zero(float mn, float mx, uint16_t* s_out, uint16_t* z_out) {
+  uint16_t z = oracle_half_round_down((double)mn);
+  double zd = oracle_half_to_double(z);
+  double need = ((double)mx - zd) / 15.0;
+  uint16_t s = (need <= 0.0) ? 0 : oracle_half_round_up(need);
+  /* settle the candidate on the exact condition, in either direction */
+  while (s < 0x7C00 && 15.0 * oracle_half_to_double(s) + zd < (double)mx) s = (uint16_t)(s + 1);
+  while (s > 0 && 15.0 * oracle_half_to_double((uint16_t)(s - 1)) + zd >= (double)mx) s = (uint16_t)(s - 1);
+  *s_out = s;
+  *z_out = z;
+}
+
+/* Codes of a row for a given (s, z): code = round-half-even(t * inv) with
+ * t = fp32(y - z) and inv = fp32(1/s); the product of two fp32 values is
+ * exact in fp64, so rint() on it is the one rounding. Clamped to [0, 15]. */
+void oracle_quantize_given(const float* y, int D, uint16_t s, uint16_t z, uint8_t* codes) {
+  float sf = (float)oracle_half_to_double(s);
+  float zf = (float)oracle_half_to_double(z);
+  float inv = (sf > 0.0f) ? 1.0f / sf : 0.0f;
+  for (int c = 0; c < D; ++c) {
+    float t = y[c] - zf;
+    double q = (double)t * (double)inv;
+    double r = nearbyint(q); /* default rounding mode: ties to even */
+    if (r < 0) r = 0;
+    if (r > 15) r = 15;
+    codes[c] = (uint8_t)r;
+  }
+}
+
+/* The quotient fp32(y - z) * fp32(1/s) itself, for classifying elements that
+ * sit next to a rounding boundary. */
+void oracle_quotient_given(const float* y, int D, uint16_t s, uint16_t z, double* qout) {
+  float sf = (float)oracle_half_to_double(s);
+  float zf = (float)oracle_half_to_double(z);
+  float inv = (sf > 0.0f) ? 1.0f / sf : 0.0f;
+  for (int c = 0; c < D; ++c) {
+    float t = y[c] - zf;
+    qout[c] = (double)t * (double)inv;
+  }
+}
+
+void oracle_quantize_row(const float* y, int D, uint8_t* codes, uint16_t* s, uint16_t* z) {
+  float mn = y[0], mx = y[0];
+  for (int c = 1; c < D; ++c) {
+    if (y[c] < mn) mn = y[c];
+    if (y[c] > mx) mx = y[c];
+  }
+  oracle_scale_zero(mn, mx, s, z);
+  oracle_quantize_given(y, D, *s, *z, codes);
+}
+
+/* byte j = code[2j] | code[2j+1] << 4 */
+void oracle_pack_row(const uint8_t* codes, int D, uint8_t* packed) {
+  for (int j = 0; j < D / 2; ++j)
+    packed[j] = (uint8_t)((codes[2 * j] & 15) | ((codes[2 * j + 1] & 15) << 4));
+}
+
+void oracle_unpack_row(const uint8_t* packed, int D, uint8_t* codes) {
+  for (int j = 0; j < D / 2; ++j) {
+    codes[2 * j] = (uint8_t)(packed[j] & 15);
+    codes[2 * j + 1] = (uint8_t)(packed[j] >> 4);
+  }
+}
+
+/* x^ = code * s + z, exact in fp64. */
+void oracle_dequant_row(const uint8_t* packed, int D, uint16_t s, uint16_t z, double* xhat) {
+  double sd = oracle_half_to_double(s), zd = oracle_half_to_double(z);
+  for (int j = 0; j < D / 2; ++j) {
+    xhat[2 * j] = (double)(packed[j] & 15) * sd + zd;
+    xhat[2 * j + 1] = (double)(packed[j] >> 4) * sd + zd;
+  }
+}
+
+/* ------------------------------------------------------------------------- */
+/* Paged placement ([SAW] Abstract: "integrates directly into paged KV-cache  */
+/* layouts").                                                                 */
+/* ------------------------------------------------------------------------- */
+
+static size_t row_index(int64_t page, int Hkv, int h, int kv, int off) {
+  return (((size_t)page * (size_t)Hkv + (size_t)h) * 2 + (size_t)kv) * ORACLE_PAGE + (size_t)off;
+}
+
+/* Byte offset of a packed row inside the cache. */
+size_t oracle_cache_row_offset(int64_t page, int Hkv, int D, int h, int kv, int off) {
+  return row_index(page, Hkv, h, kv, off) * (size_t)(D / 2);
+}
+
+/* Element offset of a row's s (or z) inside scales (or zeros). */
+size_t oracle_scale_offset(int64_t page, int Hkv, int h, int kv, int off) {
+  return row_index(page, Hkv, h, kv, off);
+}
+
+/*
+ * Rotate, quantize and place every (token, kv head, K|V) row.
+ * k, v: bf16 bits [T][Hkv][D]. y_out (optional, may be NULL): the rotated fp32
+ * rows [T][Hkv][2][D]. Rows with slot -1 are skipped (and get no y_out change).
+ * Returns 0, -1 on bad shapes, -2 if a slot lies outside [0, num_pages*16).
+ */
+int oracle_quant_write(const uint16_t* k, const uint16_t* v, const int64_t* slot_mapping,
+                       int T, int Hkv, int D, int b, int64_t num_pages,
+                       uint8_t* cache, uint16_t* scales, uint16_t* zeros, float* y_out) {
+  if (D != 64 && D != 128) return -1;
+  if (!valid_block(D, b)) return -1;
+  for (int t = 0; t < T; ++t) {
+    int64_t slot = slot_mapping[t];
+    if (slot == -1) continue;
+    if (slot < 0 || slot >= num_pages * ORACLE_PAGE) return -2;
+  }
+  int bad = 0;
+#pragma omp parallel for schedule(static)
+  for (int t = 0; t < T; ++t) {
+    int64_t slot = slot_mapping[t];
+    if (slot == -1) continue;
+    int64_t page = slot / ORACLE_PAGE;
+    int off = (int)(slot % ORACLE_PAGE);
+    for (int h = 0; h < Hkv; ++h) {
+      for (int kv = 0; kv < 2; ++kv) {
+        const uint16_t* x = (kv == 0 ? k : v) + ((size_t)t * Hkv + h) * D;
+        float y[128];
+        uint8_t codes[128];
+        uint16_t s, z;
+        if (oracle_rotate_row(x, D, b, y) != 0) { bad = 1; continue; }
+        oracle_quantize_row(y, D, codes, &s, &z);
+        oracle_pack_row(codes, D, cache + oracle_cache_row_offset(page, Hkv, D, h, kv, off));
+        scales[oracle_scale_offset(page, Hkv, h, kv, off)] = s;
+        zeros[oracle_scale_offset(page, Hkv, h, kv, off)] = z;
+        if (y_out) memcpy(y_out + (((size_t)t * Hkv + h) * 2 + kv) * D, y, sizeof(float) * D);
+      }
+    }
+  }
+  return bad ? -1 : 0;
+}
+
+/* ------------------------------------------------------------------------- */
+/* Attention over the quantized cache ([SAW] Abstract: fused attention over  */
+/* the paged INT4 cache). R is orthogonal, so q.k = (Rq).(Rk), and R^T = R.   */
+/* ------------------------------------------------------------------------- */
+
+/* Brute-force softmax attention for one query over n rotated rows:
+ * qr = R q; logit_t = scale * qr . Krot[t]; p = softmax(logit);
+ * out = R (sum_t p_t Vrot[t]). n = 0 gives out = 0. All fp64. */
+int oracle_attn_rows(const double* q, const double* Krot, const double* Vrot, int n,
+                     int D, int b, double scale, double* out) {
+  double qr[256], orot[256];
+  if (D > 256 || !valid_block(D, b)) return -1;
+  if (n == 0) {
+    for (int c = 0; c < D; ++c) out[c] = 0.0;
+    return 0;
+  }
+  oracle_rotate_f64(q, D, b, qr);
+  double* logit = (double*)malloc(sizeof(double) * (size_t)n);
+  double m = -INFINITY;
+  for (int t = 0; t < n; ++t) {
+    double acc = 0.0;
+    for (int c = 0; c < D; ++c) acc += qr[c] * Krot[(size_t)t * D + c];
+    logit[t] = scale * acc;
+    if (logit[t] > m) m = logit[t];
+  }
+  double l = 0.0;
+  for (int c = 0; c < D; ++c) orot[c] = 0.0;
+  for (int t = 0; t < n; ++t) {
+    double p = exp(logit[t] - m);
+    l += p;
+    for (int c = 0; c < D; ++c) orot[c] += p * Vrot[(size_t)t * D + c];
+  }
+  for (int c = 0; c < D; ++c) orot[c] /= l;
+  oracle_rotate_f64(orot, D, b, out);
+  free(logit);
+  return 0;
+}
+
+/* One (sequence, query head): gather the context's rows through the page
+ * table, dequantize them, and run oracle_attn_rows. Returns -2 if a page id
+ * or the context length falls outside the pool or the table. */
+int oracle_decode_one(const uint16_t* q_bf16, const uint8_t* cache, const uint16_t* scales,
+                      const uint16_t* zeros, const int32_t* page_table, const int32_t* context_lens,
+                      int n, int hq, int Hq, int Hkv, int D, int b, int max_pages,
+                      int64_t num_pages, double softmax_scale, double* out) {
+  if (Hkv <= 0 || Hq % Hkv != 0) return -1;
+  int G = Hq / Hkv;
+  int h = hq / G;
+  int ctx = context_lens[n];
+  if (ctx < 0 || ctx > max_pages * ORACLE_PAGE) return -2;
+  double scale = (softmax_scale == 0.0) ? 1.0 / sqrt((double)D) : softmax_scale;
+  double q[256];
+  for (int c = 0; c < D; ++c) q[c] = oracle_bf16_to_double(q_bf16[((size_t)n * Hq + hq) * D + c]);
+  double* K = (double*)malloc(sizeof(double) * (size_t)(ctx > 0 ? ctx : 1) * D);
+  double* V = (double*)malloc(sizeof(double) * (size_t)(ctx > 0 ? ctx : 1) * D);
+  int rc = 0;
+  for (int t = 0; t < ctx; ++t) {
+    int64_t page = page_table[(size_t)n * max_pages + t / ORACLE_PAGE];
+    int off = t % ORACLE_PAGE;
+    if (page < 0 || page >= num_pages) { rc = -2; break; }
+    for (int kv = 0; kv < 2; ++kv) {
+      size_t si = oracle_scale_offset(page, Hkv, h, kv, off);
+      oracle_dequant_row(cache + oracle_cache_row_offset(page, Hkv, D, h, kv, off), D,
+                         scales[si], zeros[si], (kv == 0 ? K : V) + (size_t)t * D);
+    }
+  }
+  if (rc == 0) rc = oracle_attn_rows(q, K, V, ctx, D, b, scale, out);
+  free(K);
+  free(V);
+  return rc;
+}
+
+/* All sequences and query heads; out is fp64 [B][Hq][D]. */
+int oracle_decode_attn(const uint16_t* q_bf16, const uint8_t* cache, const uint16_t* scales,
+                       const uint16_t* zeros, const int32_t* page_table, const int32_t* context_lens,
+                       int B, int Hq, int Hkv, int D, int b, int max_pages, int64_t num_pages,
+                       double softmax_scale, double* out) {
+  if (D != 64 && D != 128) return -1;
+  if (!valid_block(D, b)) return -1;
+  if (Hkv <= 0 || Hq % Hkv != 0) return -1;
+  int rc = 0;
+#pragma omp parallel for schedule(dynamic) collapse(2)
+  for (int n = 0; n < B; ++n)
+    for (int hq = 0; hq < Hq; ++hq) {
+      int r = oracle_decode_one(q_bf16, cache, scales, zeros, page_table, context_lens, n, hq,
+                                Hq, Hkv, D, b, max_pages, num_pages, softmax_scale,
+                                out + ((size_t)n * Hq + hq) * D);
+      if (r != 0) {
+#pragma omp critical
+        rc = r;
+      }
+    }
+  return rc;
+}
+
+/* Threads OpenMP will use (1 when built without it). */
+int oracle_num_threads(void) {
+#ifdef _OPENMP
+  return omp_get_max_threads();
+#else
+  return 1;
+#endif
+}

@@ -1,0 +1,521 @@
+#!/usr/bin/env python
+"""Benchmark of the rotated-INT4 paged KV cache hot path on B200.
+
+One step = one pass of the whole hot path over one batch of the
+Llama-3-8B-shaped workload (8 KV / 32 Q heads, head_dim 128, one sequence of
+32768 tokens, page 16, Hadamard block 128):
+  kv_quant_write      - rotate + quantize + page all 32768 tokens' K and V;
+  paged_decode_attn_int4 - one decode step over the 32768-token INT4 cache.
+The metric is HBM GB/s of algorithmic bytes (the bytes the step must move at
+minimum), whole job over all ranks.
+
+L2 hygiene: the working sets rotate so no kernel reads data still resident in
+L2: two K/V input sets (134 MB each, larger than L2) alternate, and the decode
+of step i reads the cache written at step i-2 (four cache pools), with more
+than 300 MB of traffic in between.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+WORKLOAD = "llama3-8b-32k"
+
+
+def parse_args(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", default=WORKLOAD)
+    ap.add_argument("--block", type=int, default=None, help="override the Hadamard block (0 = plain INT4)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-plain", action="store_true")
+    return ap.parse_args(argv)
+
+
+# ----------------------------------------------------------------------------
+# algorithmic bytes (the minimum a launch must move)
+# ----------------------------------------------------------------------------
+
+def write_bytes(T, Hkv, D):
+    """Per token-head: K and V read (2 x 2D bytes), codes written (2 x D/2),
+    s and z written (4 x 2 bytes); per token: its 8-byte slot."""
+    return T * Hkv * (5 * D + 8) + 8 * T
+
+
+def decode_bytes(context_lens, B, Hq, Hkv, D, out_elem=2):
+    """Per cached token-head: K and V codes (D bytes) + 4 fp16 s/z; per
+    sequence: its page-table entries and context length; q (bf16) and out."""
+    tok = int(sum(int(c) for c in context_lens))
+    pages = int(sum((int(c) + 15) // 16 for c in context_lens))
+    return tok * Hkv * (D + 8) + 4 * pages + 4 * B + B * Hq * D * 2 + B * Hq * D * out_elem
+
+
+def rank_seed(base_seed, rank):
+    """Weak scaling: every rank serves its own, independently drawn batch."""
+    return base_seed + 1000 * rank
+
+
+def aggregate_gbs(bytes_per_step, steps, world, max_ms):
+    """Whole-job GB/s: the bytes all ranks moved over the slowest rank's time."""
+    return bytes_per_step * steps * world / (max_ms / 1e3) / 1e9
+
+
+def source_digest():
+    """Hash of the kernel sources: a committed DRAM-traffic figure is valid
+    only for the kernels it was captured from."""
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "bit_kv_cache_20_b200", "csrc")
+    for name in sorted(os.listdir(csrc)):
+        with open(os.path.join(csrc, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def committed_traffic(kernel):
+    """Per-launch DRAM bytes from profiles/traffic.json if it was captured
+    from the current kernel sources, else None."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            t = json.load(f)
+    except (OSError, ValueError):
+        return None
+    entry = t.get(kernel)
+    if not entry or entry.get("source_digest") != source_digest():
+        return None
+    return entry.get("dram_bytes_per_launch")
+
+
+def measured_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return float(p["hbm_gbs"]), "measured"
+    except (OSError, ValueError, KeyError):
+        return 6650.0, "fallback"
+
+
+# ----------------------------------------------------------------------------
+# clocks during the timed region
+# ----------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except OSError:
+            self.proc = None
+        return self
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+        return False
+
+    def summary(self):
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for line in self.lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                mx = float(parts[2])
+            except ValueError:
+                continue
+            for name, val in zip(names, parts[5:9]):
+                if val.lower() == "active":
+                    reasons.add(name)
+        if not sm:
+            return {"sm_mhz": None, "sm_max_mhz": mx, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(sm), "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------
+# the CUDA arm
+# ----------------------------------------------------------------------------
+
+class Step:
+    """Prepared C-ABI calls for one workload on one device. The timed loop
+    calls the library directly with pre-marshalled arguments (what a C caller
+    does), so Python overhead stays far below the kernels' duration."""
+
+    N_POOLS = 4
+
+    def __init__(self, w, block, dev):
+        import ctypes
+        import torch
+        import bit_kv_cache_20_b200 as kvq
+        from bit_kv_cache_20_b200 import _lib
+
+        self.torch, self.kvq, self.ct = torch, kvq, ctypes
+        self.L = _lib.lib()
+        self.w, self.b, self.dev = w, block, dev
+        k0 = w.k_new.to(dev)
+        v0 = w.v_new.to(dev)
+        self.kv_sets = [(k0, v0), (k0.clone(), v0.clone())]
+        self.slots = torch.as_tensor(w.slots_new).to(dev)
+        self.pools = [kvq.alloc_cache(w.num_pages, w.Hkv, w.D, device=dev) for _ in range(self.N_POOLS)]
+        self.q = w.q.to(dev)
+        self.pt = torch.as_tensor(w.page_table).to(dev)
+        self.ctx = torch.as_tensor(w.context_lens).to(dev)
+        self.out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+        nbytes = kvq.attn_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.num_pages, w.max_pages, block)
+        self.ws = kvq.alloc_workspace(nbytes, device=dev)
+        self.ws_bytes = self.ws.numel()
+        self.stream = torch.cuda.current_stream(dev)
+        self.sh = ctypes.c_void_p(self.stream.cuda_stream)
+        self.wdesc = _lib.WriteDesc(w.tokens_written, w.Hkv, w.D, 16, w.num_pages)
+        self.adesc = _lib.AttnDesc(w.B, w.Hq, w.Hkv, w.D, 16, w.num_pages, w.max_pages, block, 0.0, 1)
+        P = ctypes.c_void_p
+        self.write_args = []
+        for i in range(self.N_POOLS):
+            k, v = self.kv_sets[i % 2]
+            c, s, z = self.pools[i]
+            self.write_args.append((P(k.data_ptr()), P(v.data_ptr()), P(self.slots.data_ptr()), None,
+                                    P(c.data_ptr()), P(s.data_ptr()), P(z.data_ptr()), block,
+                                    ctypes.byref(self.wdesc), self.sh))
+        self.attn_args = []
+        for i in range(self.N_POOLS):
+            c, s, z = self.pools[(i - 2) % self.N_POOLS]
+            self.attn_args.append((P(self.q.data_ptr()), P(c.data_ptr()), P(s.data_ptr()), P(z.data_ptr()),
+                                   P(self.pt.data_ptr()), P(self.ctx.data_ptr()), P(self.out.data_ptr()),
+                                   P(self.ws.data_ptr()), self.ws_bytes, ctypes.byref(self.adesc), self.sh))
+
+    def write(self, i):
+        st = self.L.kv_quant_write(*self.write_args[i % self.N_POOLS])
+        if st:
+            raise RuntimeError(f"kv_quant_write status {st}")
+
+    def decode(self, i):
+        st = self.L.paged_decode_attn_int4(*self.attn_args[i % self.N_POOLS])
+        if st:
+            raise RuntimeError(f"paged_decode_attn_int4 status {st}")
+
+    def fill_pools(self):
+        for i in range(self.N_POOLS):
+            self.write(i)
+        self.torch.cuda.synchronize(self.dev)
+
+    def timed(self, steps, start_index=0):
+        """Run `steps` steps with an event before and after every kernel.
+        Returns (total_ms, [write_ms], [decode_ms])."""
+        torch = self.torch
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3 * steps)]
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(self.stream)
+        for j in range(steps):
+            i = start_index + j
+            evs[3 * j].record(self.stream)
+            self.write(i)
+            evs[3 * j + 1].record(self.stream)
+            self.decode(i)
+            evs[3 * j + 2].record(self.stream)
+        t1.record(self.stream)
+        t1.synchronize()
+        wr = [evs[3 * j].elapsed_time(evs[3 * j + 1]) for j in range(steps)]
+        de = [evs[3 * j + 1].elapsed_time(evs[3 * j + 2]) for j in range(steps)]
+        return t0.elapsed_time(t1), wr, de
+
+
+def e2e_run(w, block, dev, steps, warmup):
+    """The same step through the public API with host inputs: each step copies
+    K, V, the slot mapping, q, the page table and the context lengths from
+    pinned host memory, runs both calls, and copies the output back."""
+    import torch
+    import bit_kv_cache_20_b200 as kvq
+
+    host = {
+        "k": w.k_new.pin_memory(), "v": w.v_new.pin_memory(),
+        "slots": torch.as_tensor(w.slots_new).pin_memory(), "q": w.q.pin_memory(),
+        "pt": torch.as_tensor(w.page_table).pin_memory(),
+        "ctx": torch.as_tensor(w.context_lens).pin_memory(),
+    }
+    devb = {k: torch.empty_like(v, device=dev) for k, v in host.items()}
+    out_d = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+    out_h = torch.empty_like(out_d, device="cpu").pin_memory()
+    cache, scales, zeros = kvq.alloc_cache(w.num_pages, w.Hkv, w.D, device=dev)
+    ws = kvq.alloc_workspace(kvq.attn_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.num_pages,
+                                                     w.max_pages, block), device=dev)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = out_h.numel() * out_h.element_size()
+
+    def step():
+        for key in host:
+            devb[key].copy_(host[key], non_blocking=True)
+        kvq.kv_quant_write(devb["k"], devb["v"], devb["slots"], cache, scales, zeros, block)
+        kvq.paged_decode_attn_int4(devb["q"], cache, scales, zeros, devb["pt"], devb["ctx"], out_d,
+                                   block, ws)
+        out_h.copy_(out_d, non_blocking=True)
+
+    for _ in range(warmup):
+        step()
+    torch.cuda.synchronize(dev)
+    s = torch.cuda.current_stream(dev)
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(s)
+    for _ in range(steps):
+        step()
+    b.record(s)
+    b.synchronize()
+    return a.elapsed_time(b), h2d, d2h
+
+
+# ----------------------------------------------------------------------------
+# the CPU oracle: the cpu_baseline leg and the reference arm
+# ----------------------------------------------------------------------------
+
+def oracle_sample(w, block, n_tokens):
+    """Time the oracle on the first `n_tokens` tokens of the workload: write
+    them (all kv heads, K and V), then one decode step of every query head
+    over that n_tokens-long context. Returns (seconds, algorithmic bytes)."""
+    import numpy as np
+    import oracle
+    from bit_kv_cache_20_b200 import workloads
+
+    n = min(n_tokens, w.tokens_written)
+    kb = workloads.bf16_bits(w.k_new[:n])
+    vb = workloads.bf16_bits(w.v_new[:n])
+    qb = workloads.bf16_bits(w.q)
+    ctx = np.full(w.B, n // w.B, np.int32)
+    t0 = time.perf_counter()
+    cache, scales, zeros, _ = oracle.quant_write(kb, vb, w.slots_new[:n], w.num_pages, block)
+    oracle.decode_attn(qb, cache, scales, zeros, w.page_table, ctx, w.Hkv, block, w.num_pages)
+    dt = time.perf_counter() - t0
+    nbytes = write_bytes(n, w.Hkv, w.D) + decode_bytes(ctx, w.B, w.Hq, w.Hkv, w.D)
+    return dt, nbytes
+
+
+def cpu_baseline(w, block, n_tokens=16384):
+    import oracle
+    dt, nbytes = oracle_sample(w, block, n_tokens)
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"write of the first {min(n_tokens, w.tokens_written)} tokens (all kv heads, K and V) "
+                      f"+ one decode step of all {w.Hq} query heads over them; {dt:.2f} s"}
+
+
+def run_reference(args):
+    """The oracle timed as it stands on the host cores, same metric/config."""
+    import oracle
+    from bit_kv_cache_20_b200 import workloads
+    w = workloads.make(args.config, block=args.block)
+    block = w.block
+    n_tokens = 4096
+    warm = max(args.warmup, 0)
+    for _ in range(warm):
+        oracle_sample(w, block, n_tokens)
+    total_t, total_b = 0.0, 0
+    for _ in range(args.steps):
+        dt, nb = oracle_sample(w, block, n_tokens)
+        total_t += dt
+        total_b += nb
+    value = total_b / total_t / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": warm,
+        "ms_per_step": round(1e3 * total_t / max(args.steps, 1), 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": config_block(w, block),
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+                         "kind": "oracle",
+                         "sample": f"per step: write of {n_tokens} tokens (all kv heads, K and V) + one "
+                                   f"decode step of all {w.Hq} query heads over them"},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    return line
+
+
+METRIC = "fused rot+INT4 KV write & INT4 paged decode attn: HBM GB/s, % of peak"
+
+
+def config_block(w, block):
+    return {
+        "workload": w.cfg.name, "batch": w.B, "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D,
+        "context": int(w.context_lens.max()), "written_tokens": w.tokens_written, "page": 16,
+        "hadamard_block": block, "out_dtype": "bf16",
+        "l2": "inputs larger than L2 alternate; decode reads a cache written two steps earlier",
+    }
+
+
+# ----------------------------------------------------------------------------
+# main
+# ----------------------------------------------------------------------------
+
+def reduce_max(x, world, device):
+    """Max of a per-rank scalar over all ranks (the job's time is the slowest
+    rank's)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def main(argv=None):
+    args = parse_args(argv)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return 0
+
+    import datetime
+    import torch
+    import torch.distributed as dist
+    from bit_kv_cache_20_b200 import workloads
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=180), device_id=dev)
+    warm = max(args.warmup, 3)
+    cfg = workloads.CONFIGS[args.config]
+    # weak scaling: every rank serves its own batch (its own seed)
+    w = workloads.make(args.config, block=args.block, seed=rank_seed(cfg.seed, rank))
+    block = w.block
+    wb = write_bytes(w.tokens_written, w.Hkv, w.D)
+    db = decode_bytes(w.context_lens, w.B, w.Hq, w.Hkv, w.D, out_elem=2)
+
+    def barrier():
+        torch.cuda.synchronize(dev)
+        if world > 1:
+            dist.barrier()
+
+    def max_over_ranks(x):
+        return reduce_max(x, world, dev)
+
+    step = Step(w, block, dev)
+    step.fill_pools()
+    step.timed(warm)                        # warm-up steps (untimed)
+    barrier()
+    with ClockSampler(local) as clocks:
+        total_ms, wr, de = step.timed(args.steps, start_index=warm)
+    barrier()
+    total_ms = max_over_ranks(total_ms)
+    wr_ms = max_over_ranks(statistics.mean(wr))
+    de_ms = max_over_ranks(statistics.mean(de))
+
+    plain = None
+    if not args.no_plain and block != 0:
+        p = Step(w, 0, dev)
+        p.fill_pools()
+        p.timed(warm)
+        barrier()
+        p_total, p_wr, p_de = p.timed(args.steps, start_index=warm)
+        barrier()
+        p_wr_ms = max_over_ranks(statistics.mean(p_wr))
+        p_de_ms = max_over_ranks(statistics.mean(p_de))
+        p_total = max_over_ranks(p_total)
+        plain = {
+            "hadamard_block": 0,
+            "kv_quant_write_us": round(1e3 * p_wr_ms, 3),
+            "paged_decode_attn_int4_us": round(1e3 * p_de_ms, 3),
+            "ms_per_step": round(p_total / args.steps, 5),
+            "rotation_overhead": {
+                "kv_quant_write": round(wr_ms / p_wr_ms - 1, 4),
+                "paged_decode_attn_int4": round(de_ms / p_de_ms - 1, 4),
+                "step": round(total_ms / p_total - 1, 4),
+            },
+        }
+        del p
+
+    e2e = None
+    if not args.no_e2e:
+        e_ms, h2d, d2h = e2e_run(w, block, dev, args.steps, warm)
+        e_ms = max_over_ranks(e_ms)
+        e2e = {"value": round(aggregate_gbs(wb + db, args.steps, world, e_ms), 3), "unit": "GB/s",
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+               "ms_per_step": round(e_ms / args.steps, 4)}
+
+    if world > 1:
+        dist.barrier()
+        dist.destroy_process_group()
+    if rank != 0:
+        return 0
+
+    peak, peak_src = measured_peaks()
+    value = aggregate_gbs(wb + db, args.steps, world, total_ms)
+    w_gbs = wb / (wr_ms / 1e3) / 1e9
+    d_gbs = db / (de_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
+        "steps": args.steps, "warmup": warm, "ms_per_step": round(total_ms / args.steps, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
+        "data": "synthetic", "config": config_block(w, block),
+        "pct_of_peak": round(100 * value / (peak * world), 2),
+        "roofline": {"kernel": "kv_quant_write", "bound": "hbm", "achieved": round(w_gbs, 2),
+                     "peak": peak, "unit": "GB/s", "frac": round(w_gbs / peak, 4),
+                     "traffic": committed_traffic("kv_quant_write"),
+                     "algorithmic_bytes": wb, "peak_source": f"{peak_src} (MEASURED_PEAKS.json hbm_gbs)"
+                     if peak_src == "measured" else "fallback 6.65 TB/s"},
+        "roofline_decode": {"kernel": "paged_decode_attn_int4", "bound": "hbm", "achieved": round(d_gbs, 2),
+                            "peak": peak, "unit": "GB/s", "frac": round(d_gbs / peak, 4),
+                            "traffic": committed_traffic("paged_decode_attn_int4"),
+                            "algorithmic_bytes": db},
+        "kernels": {
+            "kv_quant_write": {"us": round(1e3 * wr_ms, 3), "GB/s": round(w_gbs, 2),
+                               "tokens_per_s": round(w.tokens_written / (wr_ms / 1e3), 1)},
+            "paged_decode_attn_int4": {"us": round(1e3 * de_ms, 3), "GB/s": round(d_gbs, 2),
+                                       "decode_steps_x_batch_per_s": round(w.B / (de_ms / 1e3), 1),
+                                       "cached_tokens_per_s": round(w.tokens_cached / (de_ms / 1e3), 1)},
+        },
+        "plain_int4": plain,
+        "e2e": e2e,
+        "clocks": clocks.summary(),
+        "gpu_launches": 2 * args.steps,
+    }
+    if not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(w, block)
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,160 @@
+"""Rotated-INT4 paged KV cache for B200 (sm_100a).
+
+Python binding of the C ABI in include/kvq.h: torch tensors in, pointers and
+sizes out, the current CUDA stream by default. The two hot-path calls are
+
+    kv_quant_write(k, v, slot_mapping, cache, scales, zeros, hadamard_block)
+    paged_decode_attn_int4(q, cache, scales, zeros, page_table, context_lens,
+                           out, hadamard_block)
+
+Every step runs in the library's kernels; if libkvq.so is missing the calls
+raise (there is no CPU or PyTorch fallback).
+"""
+from __future__ import annotations
+
+import ctypes
+from typing import Optional, Tuple
+
+import torch
+
+from . import _lib
+from ._lib import AttnDesc, KVQError, WriteDesc
+
+PAGE_SIZE = 16
+
+__all__ = [
+    "PAGE_SIZE", "KVQError", "alloc_cache", "kv_quant_write", "paged_decode_attn_int4",
+    "attn_workspace_size", "alloc_workspace", "get_device_error", "library_path",
+]
+
+
+def library_path() -> str:
+    return _lib.LIB_PATH
+
+
+def _stream_handle(stream) -> int:
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return int(stream.cuda_stream) if hasattr(stream, "cuda_stream") else int(stream)
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _need(t: torch.Tensor, name: str, dtype) -> None:
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must live on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def alloc_cache(num_pages: int, num_kv_heads: int, head_dim: int,
+                device="cuda") -> Tuple[torch.Tensor, torch.Tensor, torch.Tensor]:
+    """Empty pool: cache uint8 [pages, Hkv, 2, 16, D/2], scales and zeros
+    fp16 [pages, Hkv, 2, 16]."""
+    cache = torch.zeros((num_pages, num_kv_heads, 2, PAGE_SIZE, head_dim // 2), dtype=torch.uint8,
+                        device=device)
+    scales = torch.zeros((num_pages, num_kv_heads, 2, PAGE_SIZE), dtype=torch.float16, device=device)
+    zeros = torch.zeros_like(scales)
+    return cache, scales, zeros
+
+
+def _pool_shape(cache, scales, zeros):
+    _need(cache, "cache", torch.uint8)
+    _need(scales, "scales", torch.float16)
+    _need(zeros, "zeros", torch.float16)
+    if cache.dim() != 5 or cache.shape[2] != 2 or cache.shape[3] != PAGE_SIZE:
+        raise ValueError("cache must be uint8 [num_pages, Hkv, 2, 16, D/2]")
+    P, Hkv = int(cache.shape[0]), int(cache.shape[1])
+    D = int(cache.shape[4]) * 2
+    if tuple(scales.shape) != (P, Hkv, 2, PAGE_SIZE) or tuple(zeros.shape) != tuple(scales.shape):
+        raise ValueError("scales/zeros must be fp16 [num_pages, Hkv, 2, 16]")
+    return P, Hkv, D
+
+
+def kv_quant_write(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
+                   cache: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
+                   hadamard_block: int, page_table: Optional[torch.Tensor] = None,
+                   stream=None) -> None:
+    """Rotate (block Hadamard), quantize (token-wise INT4) and store new K/V
+    rows [T, Hkv, D] (bf16) at slot_mapping (int64 [T], -1 = skip)."""
+    P, Hkv, D = _pool_shape(cache, scales, zeros)
+    _need(k, "k", torch.bfloat16)
+    _need(v, "v", torch.bfloat16)
+    _need(slot_mapping, "slot_mapping", torch.int64)
+    if k.dim() != 3 or tuple(k.shape[1:]) != (Hkv, D) or k.shape != v.shape:
+        raise ValueError("k and v must be bf16 [T, Hkv, D] matching the cache")
+    T = int(k.shape[0])
+    if slot_mapping.numel() != T:
+        raise ValueError("slot_mapping must hold one slot per token")
+    desc = WriteDesc(T, Hkv, D, PAGE_SIZE, P)
+    st = _lib.lib().kv_quant_write(_ptr(k), _ptr(v), _ptr(slot_mapping), _ptr(page_table),
+                                   _ptr(cache), _ptr(scales), _ptr(zeros), int(hadamard_block),
+                                   ctypes.byref(desc), ctypes.c_void_p(_stream_handle(stream)))
+    _lib.check(st, "kv_quant_write")
+
+
+def _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scale, out_dtype):
+    P, Hkv, D = _pool_shape(cache, scales, zeros)
+    if q.dim() != 3 or int(q.shape[2]) != D:
+        raise ValueError("q must be bf16 [B, Hq, D]")
+    B, Hq = int(q.shape[0]), int(q.shape[1])
+    if page_table.dim() != 2 or int(page_table.shape[0]) != B:
+        raise ValueError("page_table must be int32 [B, max_pages]")
+    return AttnDesc(B, Hq, Hkv, D, PAGE_SIZE, P, int(page_table.shape[1]), int(hadamard_block),
+                    float(softmax_scale), out_dtype)
+
+
+def attn_workspace_size(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
+                        num_pages: int, max_pages_per_seq: int, hadamard_block: int) -> int:
+    """Bytes of workspace paged_decode_attn_int4 needs on the current device."""
+    desc = AttnDesc(batch, num_q_heads, num_kv_heads, head_dim, PAGE_SIZE, num_pages,
+                    max_pages_per_seq, hadamard_block, 0.0, 0)
+    n = _lib.lib().kvq_attn_workspace_size(ctypes.byref(desc))
+    if n == ctypes.c_size_t(-1).value:
+        raise KVQError(1, "kvq_attn_workspace_size (invalid shapes or no device)")
+    return int(n)
+
+
+def alloc_workspace(nbytes: int, device="cuda") -> torch.Tensor:
+    """A zero-filled workspace (the decode call keeps it zero between calls)."""
+    return torch.zeros(max(int(nbytes), 16), dtype=torch.uint8, device=device)
+
+
+def paged_decode_attn_int4(q: torch.Tensor, cache: torch.Tensor, scales: torch.Tensor,
+                           zeros: torch.Tensor, page_table: torch.Tensor,
+                           context_lens: torch.Tensor, out: torch.Tensor, hadamard_block: int,
+                           workspace: Optional[torch.Tensor] = None, softmax_scale: float = 0.0,
+                           stream=None) -> None:
+    """One decode step over the INT4 cache; out is fp32 or bf16 [B, Hq, D]."""
+    _need(q, "q", torch.bfloat16)
+    _need(page_table, "page_table", torch.int32)
+    _need(context_lens, "context_lens", torch.int32)
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("out must be float32 or bfloat16")
+    _need(out, "out", out.dtype)
+    if tuple(out.shape) != tuple(q.shape):
+        raise ValueError("out must have q's shape")
+    desc = _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scale,
+                      0 if out.dtype == torch.float32 else 1)
+    if context_lens.numel() != desc.batch:
+        raise ValueError("context_lens must hold one length per sequence")
+    L = _lib.lib()
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8)
+        ws_ptr, ws_bytes = _ptr(workspace), workspace.numel()
+    st = L.paged_decode_attn_int4(_ptr(q), _ptr(cache), _ptr(scales), _ptr(zeros), _ptr(page_table),
+                                  _ptr(context_lens), _ptr(out), ws_ptr, ws_bytes,
+                                  ctypes.byref(desc), ctypes.c_void_p(_stream_handle(stream)))
+    _lib.check(st, "paged_decode_attn_int4")
+
+
+def get_device_error(stream=None) -> int:
+    """Synchronize the stream and return (and clear) the device error word."""
+    return int(_lib.lib().kvq_get_device_error(ctypes.c_void_p(_stream_handle(stream))))

@@ -1,0 +1,196 @@
+"""Parity of paged_decode_attn_int4 (CUDA, through the C ABI) with the oracle.
+
+The oracle reads the cache bytes the CUDA write produced, so write-path
+differences cannot leak into this check. Bar: fp32 output within 2e-3
+max-abs of the fp64 oracle; bf16 output equal to the round-to-nearest bf16 of
+the fp32 output; guard regions around `out` untouched; the workspace all zero
+again after every call.
+"""
+import numpy as np
+import pytest
+import torch
+
+import bit_kv_cache_20_b200 as kvq
+from bit_kv_cache_20_b200 import workloads
+
+pytestmark = pytest.mark.gpu
+
+TOL = 2e-3
+GUARD = 1024
+
+
+def build_cache(w, b=None):
+    b = w.block if b is None else b
+    cache, scales, zeros = kvq.alloc_cache(w.num_pages, w.Hkv, w.D)
+    for k, v, s in ((w.k_prior, w.v_prior, w.slots_prior), (w.k_new, w.v_new, w.slots_new)):
+        if k.shape[0]:
+            kvq.kv_quant_write(k.cuda(), v.cuda(), torch.as_tensor(s).cuda(), cache, scales, zeros, b)
+    assert kvq.get_device_error() == 0
+    return cache, scales, zeros
+
+
+def host_cache(cache, scales, zeros):
+    return (cache.cpu().numpy().reshape(-1),
+            scales.cpu().view(torch.int16).numpy().view(np.uint16).reshape(-1),
+            zeros.cpu().view(torch.int16).numpy().view(np.uint16).reshape(-1))
+
+
+def gpu_decode(w, pool, b=None, out_dtype=torch.float32, softmax_scale=0.0, ws=None,
+               page_table=None, ctx=None):
+    b = w.block if b is None else b
+    cache, scales, zeros = pool
+    pt = torch.as_tensor(w.page_table if page_table is None else page_table).cuda()
+    cl = torch.as_tensor(w.context_lens if ctx is None else ctx).cuda()
+    n = w.B * w.Hq * w.D
+    big = torch.full((n + 2 * GUARD,), 7.0, dtype=out_dtype, device="cuda")
+    out = big[GUARD:GUARD + n].view(w.B, w.Hq, w.D)
+    if ws is None:
+        nbytes = kvq.attn_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.num_pages, pt.shape[1], b)
+        ws = kvq.alloc_workspace(nbytes)
+    kvq.paged_decode_attn_int4(w.q.cuda(), cache, scales, zeros, pt, cl, out, b, ws,
+                               softmax_scale=softmax_scale)
+    torch.cuda.synchronize()
+    g = big.cpu()
+    assert torch.all(g[:GUARD] == 7.0) and torch.all(g[GUARD + n:] == 7.0), "out guard overwritten"
+    return out.float().cpu().numpy().astype(np.float64), ws
+
+
+def oracle_out(orc, w, pool, b=None, softmax_scale=0.0, pairs=None):
+    b = w.block if b is None else b
+    c, s, z = host_cache(*pool)
+    qb = workloads.bf16_bits(w.q)
+    if pairs is None:
+        return orc.decode_attn(qb, c, s, z, w.page_table, w.context_lens, w.Hkv, b, w.num_pages,
+                               softmax_scale)
+    return {(n, hq): orc.decode_one(qb, c, s, z, w.page_table, w.context_lens, n, hq, w.Hkv, b,
+                                    w.num_pages, softmax_scale) for n, hq in pairs}
+
+
+def assert_close(got, ref, label):
+    err = float(np.abs(got - ref).max()) if ref.size else 0.0
+    print(f"{label}: max|err| = {err:.3e} (max|ref| = {float(np.abs(ref).max(initial=0)):.3e})")
+    assert err <= TOL, (label, err)
+
+
+def test_decode_tiny_config(orc):
+    w = workloads.make("tiny")
+    pool = build_cache(w)
+    got, ws = gpu_decode(w, pool)
+    assert_close(got, oracle_out(orc, w, pool), "tiny")
+    assert int(ws.sum()) == 0
+
+
+@pytest.mark.parametrize("D,b", [(64, 0), (64, 32), (64, 64), (128, 0), (128, 32), (128, 64), (128, 128)])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
+def test_decode_random_shapes(orc, D, b, G):
+    # contexts: empty, a single token, page boundary -1/0/+1, several pages,
+    # and enough pages for several splits
+    ctx = [0, 1, 15, 16, 17, 33, 250, 1000]
+    w = workloads.random_case(seed=D * 3 + b + G, B=len(ctx), Hq=2 * G, Hkv=2, D=D, block=b,
+                              context_lens=ctx, extra_pages=3)
+    pool = build_cache(w)
+    got, ws = gpu_decode(w, pool)
+    ref = oracle_out(orc, w, pool)
+    assert_close(got, ref, f"D={D} b={b} G={G}")
+    assert np.all(got[0] == 0.0), "empty context must give zero output"
+    assert int(ws.sum()) == 0
+
+
+def test_decode_single_split_path(orc):
+    # enough (sequence, kv head) pairs that each is one CTA (no workspace)
+    w = workloads.random_case(seed=21, B=64, Hq=32, Hkv=8, D=128, block=64,
+                              context_lens=list(np.arange(64) * 7 + 1), extra_pages=0)
+    assert kvq.attn_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.num_pages, w.max_pages, 64) == 0
+    pool = build_cache(w)
+    got, _ = gpu_decode(w, pool)
+    assert_close(got, oracle_out(orc, w, pool), "single split")
+
+
+def test_decode_full_size_llama3_8b_32k(orc):
+    # the benchmark's decode launch: 1 sequence of 32768 tokens, 32 q heads
+    w = workloads.make("llama3-8b-32k")
+    pool = build_cache(w)
+    got, _ = gpu_decode(w, pool)
+    ref = oracle_out(orc, w, pool)
+    assert_close(got, ref, "llama3-8b-32k")
+    got16, _ = gpu_decode(w, pool, out_dtype=torch.bfloat16)
+    ref16 = torch.from_numpy(got.astype(np.float32)).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(got16.astype(np.float32), ref16)
+
+
+def test_decode_llama2_70b_b8_sampled(orc):
+    w = workloads.make("llama2-70b-b8")
+    pool = build_cache(w)
+    got, _ = gpu_decode(w, pool)
+    rng = np.random.default_rng(2)
+    pairs = [(int(n), int(h)) for n, h in zip(rng.integers(0, w.B, 12), rng.integers(0, w.Hq, 12))]
+    ref = oracle_out(orc, w, pool, pairs=pairs)
+    for (n, h), r in ref.items():
+        assert_close(got[n, h], r, f"llama2-70b-b8 n={n} hq={h}")
+
+
+def test_decode_serving_b64_sampled(orc):
+    w = workloads.make("serving-b64")
+    pool = build_cache(w)
+    got, _ = gpu_decode(w, pool)
+    rng = np.random.default_rng(3)
+    pairs = [(int(n), int(h)) for n, h in zip(rng.integers(0, w.B, 16), rng.integers(0, w.Hq, 16))]
+    for (n, h), r in oracle_out(orc, w, pool, pairs=pairs).items():
+        assert_close(got[n, h], r, f"serving-b64 n={n} hq={h}")
+
+
+@pytest.mark.parametrize("b", [0, 32, 64, 128])
+def test_decode_stress_lognormal_contexts_sampled(orc, b):
+    w = workloads.make("stress-b256", block=b, batch=24)
+    pool = build_cache(w, b)
+    got, _ = gpu_decode(w, pool, b)
+    rng = np.random.default_rng(4 + b)
+    pairs = [(int(n), int(h)) for n, h in zip(rng.integers(0, w.B, 10), rng.integers(0, w.Hq, 10))]
+    for (n, h), r in oracle_out(orc, w, pool, b, pairs=pairs).items():
+        assert_close(got[n, h], r, f"stress b={b} n={n} hq={h}")
+
+
+def test_decode_explicit_softmax_scale_and_bf16(orc):
+    w = workloads.random_case(seed=8, B=3, Hq=8, Hkv=2, D=128, block=64, context_lens=[70, 3, 400])
+    pool = build_cache(w)
+    got, _ = gpu_decode(w, pool, softmax_scale=0.05)
+    assert_close(got, oracle_out(orc, w, pool, softmax_scale=0.05), "softmax_scale=0.05")
+    got16, _ = gpu_decode(w, pool, out_dtype=torch.bfloat16, softmax_scale=0.05)
+    ref16 = torch.from_numpy(got.astype(np.float32)).to(torch.bfloat16).float().numpy()
+    assert np.array_equal(got16.astype(np.float32), ref16)
+
+
+def test_decode_deterministic_and_workspace_reuse():
+    w = workloads.random_case(seed=9, B=2, Hq=16, Hkv=4, D=128, block=128, context_lens=[3000, 777])
+    pool = build_cache(w)
+    a, ws = gpu_decode(w, pool)
+    assert int(ws.sum()) == 0
+    b_, ws = gpu_decode(w, pool, ws=ws)
+    assert np.array_equal(a, b_)
+    assert int(ws.sum()) == 0
+
+
+def test_decode_bad_page_id_and_long_context_are_reported(orc):
+    w = workloads.random_case(seed=10, B=2, Hq=4, Hkv=2, D=64, block=32, context_lens=[40, 20])
+    pool = build_cache(w)
+    pt = w.page_table.copy()
+    pt[0, 1] = w.num_pages + 5
+    gpu_decode(w, pool, page_table=pt)
+    assert kvq.get_device_error() == 3
+    ctx = w.context_lens.copy()
+    ctx[1] = w.max_pages * 16 + 1
+    gpu_decode(w, pool, ctx=ctx)
+    assert kvq.get_device_error() == 3
+    assert kvq.get_device_error() == 0
+
+
+def test_decode_rejects_missing_workspace():
+    w = workloads.random_case(seed=12, B=1, Hq=8, Hkv=2, D=128, block=128, context_lens=[4000])
+    need = kvq.attn_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.num_pages, w.max_pages, 128)
+    assert need > 0
+    pool = build_cache(w)
+    out = torch.empty((1, 8, 128), device="cuda")
+    with pytest.raises(kvq.KVQError):
+        kvq.paged_decode_attn_int4(w.q.cuda(), *pool, torch.as_tensor(w.page_table).cuda(),
+                                   torch.as_tensor(w.context_lens).cuda(), out, 128,
+                                   kvq.alloc_workspace(need - 16))

@@ -1,0 +1,58 @@
+"""The benchmark's multi-rank logic on two CPU ranks (gloo): weak scaling,
+each rank drawing its own batch, with the job's time the slowest rank's and
+no collective on the data path."""
+import os
+import socket
+
+import numpy as np
+import torch
+import torch.distributed as dist
+import torch.multiprocessing as mp
+
+
+def _free_port():
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def _worker(rank, world, port, results):
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world)
+    import bench
+    from bit_kv_cache_20_b200 import workloads
+    cfg = workloads.CONFIGS["tiny"]
+    w = workloads.make("tiny", seed=bench.rank_seed(cfg.seed, rank))
+    fake_ms = 10.0 + 5.0 * rank                 # rank 1 is the slow one
+    slowest = bench.reduce_max(fake_ms, world, "cpu")
+    digest = float(workloads.bf16_bits(w.k_new).astype(np.int64).sum() % 1000003)
+    t = torch.tensor([digest], dtype=torch.float64)
+    gathered = [torch.zeros(1, dtype=torch.float64) for _ in range(world)]
+    dist.all_gather(gathered, t)
+    results[rank] = (slowest, [float(g.item()) for g in gathered])
+    dist.barrier()
+    dist.destroy_process_group()
+
+
+def test_two_rank_weak_scaling_logic():
+    world = 2
+    mgr = mp.Manager()
+    results = mgr.dict()
+    mp.spawn(_worker, args=(world, _free_port(), results), nprocs=world, join=True)
+    assert results[0][0] == results[1][0] == 15.0          # max over ranks
+    d0, d1 = results[0][1]
+    assert d0 != d1                                         # independent batches
+    import bench
+    from bit_kv_cache_20_b200 import workloads
+    w = workloads.make("tiny")
+    per_step = bench.write_bytes(w.tokens_written, w.Hkv, w.D)
+    # whole-job throughput counts every rank's bytes over the slowest time
+    assert bench.aggregate_gbs(per_step, 10, world, 15.0) == per_step * 10 * 2 / 0.015 / 1e9
+
+
+def test_reference_arm_on_a_non_zero_rank_exits_without_work(monkeypatch, capsys):
+    import bench
+    monkeypatch.setenv("RANK", "1")
+    monkeypatch.setenv("WORLD_SIZE", "2")
+    assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0"]) == 0
+    assert capsys.readouterr().out == ""

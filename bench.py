@@ -38,7 +38,7 @@ WORKLOAD = "llama3-8b-32k"
 def parse_args(argv=None):
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=2000)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", default=WORKLOAD)
@@ -46,6 +46,9 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-plain", action="store_true")
+    ap.add_argument("--only", choices=["write", "decode"], default=None,
+                    help="time one kernel alone (profiling captures); prints its line")
+    ap.add_argument("--e2e-steps", type=int, default=100)
     return ap.parse_args(argv)
 
 
@@ -124,13 +127,14 @@ class ClockSampler:
     def __init__(self, gpu_index):
         self.gpu = gpu_index
         self.proc = None
-        self.lines = []
+        self.lines = []          # (host monotonic time, csv line)
+        self.window = None
 
     def __enter__(self):
         try:
             self.proc = subprocess.Popen(
                 ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "100"],
+                 "--format=csv,noheader,nounits", "-lms", "20"],
                 stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
@@ -140,7 +144,16 @@ class ClockSampler:
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def wait_first_sample(self, timeout=5.0):
+        t_end = time.monotonic() + timeout
+        while self.proc is not None and not self.lines and time.monotonic() < t_end:
+            time.sleep(0.01)
+
+    def mark(self, t0, t1):
+        """The host-time window during which the GPU ran the timed steps."""
+        self.window = (t0, t1)
 
     def __exit__(self, *exc):
         if self.proc is not None:
@@ -154,7 +167,10 @@ class ClockSampler:
     def summary(self):
         sm, mx, reasons = [], None, set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for line in self.lines:
+        lines = self.lines
+        if self.window is not None:
+            lines = [(t, l) for t, l in self.lines if self.window[0] <= t <= self.window[1]]
+        for _, line in lines:
             parts = [p.strip() for p in line.split(",")]
             if len(parts) < 9:
                 continue
@@ -237,6 +253,18 @@ class Step:
         for i in range(self.N_POOLS):
             self.write(i)
         self.torch.cuda.synchronize(self.dev)
+
+    def timed_only(self, kind, steps, start_index=0):
+        """One kernel alone, `steps` launches; returns the per-launch ms."""
+        torch = self.torch
+        evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps)]
+        for j in range(steps):
+            i = start_index + j
+            evs[2 * j].record(self.stream)
+            (self.write if kind == "write" else self.decode)(i)
+            evs[2 * j + 1].record(self.stream)
+        evs[-1].synchronize()
+        return [evs[2 * j].elapsed_time(evs[2 * j + 1]) for j in range(steps)]
 
     def timed(self, steps, start_index=0):
         """Run `steps` steps with an event before and after every kernel.
@@ -433,10 +461,28 @@ def main(argv=None):
 
     step = Step(w, block, dev)
     step.fill_pools()
-    step.timed(warm)                        # warm-up steps (untimed)
-    barrier()
+    if args.only:
+        step.timed_only(args.only, warm)
+        barrier()
+        ms = step.timed_only(args.only, args.steps, start_index=warm)
+        barrier()
+        if rank == 0:
+            nb = wb if args.only == "write" else db
+            mean = statistics.mean(ms)
+            print(json.dumps({"only": args.only, "us": round(1e3 * mean, 3),
+                              "GB/s": round(nb / (mean / 1e3) / 1e9, 2), "launches": args.steps,
+                              "config": config_block(w, block)}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
     with ClockSampler(local) as clocks:
+        clocks.wait_first_sample()
+        step.timed(warm)                    # warm-up steps (untimed)
+        barrier()
+        t_host0 = time.monotonic()
         total_ms, wr, de = step.timed(args.steps, start_index=warm)
+        t_host1 = time.monotonic()
+        clocks.mark(t_host0, t_host1)
     barrier()
     total_ms = max_over_ranks(total_ms)
     wr_ms = max_over_ranks(statistics.mean(wr))
@@ -468,11 +514,12 @@ def main(argv=None):
 
     e2e = None
     if not args.no_e2e:
-        e_ms, h2d, d2h = e2e_run(w, block, dev, args.steps, warm)
+        e_steps = max(1, min(args.steps, args.e2e_steps))
+        e_ms, h2d, d2h = e2e_run(w, block, dev, e_steps, warm)
         e_ms = max_over_ranks(e_ms)
-        e2e = {"value": round(aggregate_gbs(wb + db, args.steps, world, e_ms), 3), "unit": "GB/s",
+        e2e = {"value": round(aggregate_gbs(wb + db, e_steps, world, e_ms), 3), "unit": "GB/s",
                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-               "ms_per_step": round(e_ms / args.steps, 4)}
+               "ms_per_step": round(e_ms / e_steps, 4), "steps": e_steps}
 
     if world > 1:
         dist.barrier()

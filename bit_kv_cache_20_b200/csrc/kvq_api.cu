@@ -130,12 +130,13 @@ struct SplitPlan {
   int pages_per_split;
 };
 
-// Split each (sequence, kv head) over enough CTAs to cover the GPU about three
-// times, keeping at least 8 pages (two per warp) per split.
+// Split each (sequence, kv head) so that all CTAs fit in one wave (three
+// resident CTAs per SM, which the kernel's launch bounds guarantee), keeping
+// at least 8 pages (two per warp) per split.
 SplitPlan plan_splits(const kvq_attn_desc* d, int sms) {
   const long long units = (long long)d->batch * d->num_kv_heads;
   const long long target = 3LL * sms;
-  long long ns = units > 0 ? (target + units - 1) / units : 1;
+  long long ns = units > 0 ? target / units : 1;
   long long most = d->max_pages_per_seq / 8;
   if (most < 1) most = 1;
   if (ns > most) ns = most;
@@ -208,13 +209,13 @@ kvq_status kv_quant_write(const void* k, const void* v, const int64_t* slot_mapp
     return KVQ_ERR_INVALID_ARG;
   if (d.head_dim != 64 && d.head_dim != 128) return KVQ_ERR_UNSUPPORTED;
   if (!valid_block(d.head_dim, hadamard_block)) return KVQ_ERR_UNSUPPORTED;
+  if (d.num_tokens == 0) return KVQ_OK;  // nothing to do; pointers may be NULL
   if (!k || !v || !slot_mapping || !cache || !scales || !zeros) return KVQ_ERR_INVALID_ARG;
   if (!aligned(k, 16) || !aligned(v, 16) || !aligned(cache, 16) || !aligned(scales, 16) ||
       !aligned(zeros, 16) || !aligned(slot_mapping, 8))
     return KVQ_ERR_INVALID_ARG;
   const long long tiles = ((long long)d.num_tokens + 31) / 32 * d.num_kv_heads * 2;
   if (tiles > INT_MAX) return KVQ_ERR_INVALID_ARG;
-  if (d.num_tokens == 0) return KVQ_OK;
   int dev = 0;
   kvq_status st = select_device_of(cache, &dev);
   if (st != KVQ_OK) return st;
@@ -254,12 +255,12 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const voi
   kvq_status st = check_attn_desc(desc);
   if (st != KVQ_OK) return st;
   const kvq_attn_desc& d = *desc;
+  if (d.batch == 0) return KVQ_OK;  // nothing to do; pointers may be NULL
   if (!q || !cache || !scales || !zeros || !page_table || !context_lens || !out)
     return KVQ_ERR_INVALID_ARG;
   if (!aligned(cache, 16) || !aligned(scales, 16) || !aligned(zeros, 16) || !aligned(q, 2) ||
       !aligned(page_table, 4) || !aligned(context_lens, 4) || !aligned(out, d.out_dtype ? 2 : 4))
     return KVQ_ERR_INVALID_ARG;
-  if (d.batch == 0) return KVQ_OK;
   int dev = 0;
   st = select_device_of(cache, &dev);
   if (st != KVQ_OK) return st;

@@ -16,9 +16,11 @@
 //   carries both halves and GQA groups up to 8 share one K/V stream.
 //   QK:  S[16 x 16 tokens] = Qhl[16 x D] * codes^T       (k = channels)
 //   PV:  O[16 x D]        += Phl[16 x 16 tokens] * codes  (k = tokens)
-//   The 4-bit codes enter the MMA unconverted: a nibble masked into the low
-//   bits of an fp16 is the exact subnormal c * 2^-24 (or c * 2^-20 for a
-//   nibble at bits 4..7); the power of two is folded back in fp32.
+//   The 4-bit codes enter the MMA as exact normal fp16 values c (or 16c for a
+//   nibble at bits 4..7, compensated by a factor 1/16 on the other operand or
+//   in the epilogue). Subnormal fp16 operands are avoided on purpose: small
+//   products built from them lost precision in the tensor-core accumulation
+//   (a systematic bias of ~2^-13 relative, measured on B200).
 //   Dequantization is folded into the per-token scalars:
 //     logit_t = s_t * (q~ . code_t) + z_t * sum(q~)
 //     o_rot   = (sum_t p_t s_t code_t + sum_t p_t z_t) / sum_t p_t
@@ -52,7 +54,7 @@ struct AttnParams {
 constexpr int kAttnWarps = 4;
 constexpr int kAttnThreads = kAttnWarps * 32;
 constexpr int kStages = 4;
-constexpr int kMaxSplits = 128;
+constexpr int kMaxSplits = 64;
 
 template <int D>
 struct AttnSmem {
@@ -64,7 +66,7 @@ struct AttnSmem {
   static constexpr int kMergeBytes = kAttnWarps * kMergeFloatsPerWarp * 4;
   static constexpr int kUnionBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
   static constexpr int kQBytes = 8 * D * 4;             // q / output rows, fp32
-  static constexpr int kWeightBytes = (8 * kMaxSplits + 8) * 4;  // split weights + per-head L
+  static constexpr int kWeightBytes = (2 * 8 * kMaxSplits + 8) * 4;  // split maxima/weights, sums, per-head L
   static constexpr int kBarBytes = kAttnWarps * kStages * 8;
   static constexpr int kFlagBytes = kAttnWarps * kStages * 4 + 16;
   static constexpr int kOffQ = kUnionBytes;
@@ -99,7 +101,6 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnP
   constexpr int KS = D / 16;  // QK k-steps
   constexpr int WP = D / 64;  // code words of one token row per thread group (PV)
   constexpr int NT = D / 8;   // PV n-tiles
-  constexpr float kTwo24 = 16777216.0f, kTwo20 = 1048576.0f;
   extern __shared__ __align__(128) uint8_t smem[];
   float* qs = reinterpret_cast<float*>(smem + S::kOffQ);
   float* wts = reinterpret_cast<float*>(smem + S::kOffW);
@@ -153,7 +154,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnP
   int kexp = (amax > 0.0f) ? 13 - ilogbf(amax) : 0;
   kexp = max(-100, min(100, kexp));
   const float up = ldexpf(1.0f, kexp);
-  const float acc_to_true = ldexpf(1.0f, 24 - kexp);
+  const float acc_to_true = ldexpf(1.0f, -kexp);
 
   // A fragments of QK. k-step 2u takes channel pairs (8m, 8m+4), (8m+2, 8m+6)
   // of word m = W tig + u; k-step 2u+1 takes (8m+1, 8m+5), (8m+3, 8m+7) whose
@@ -256,8 +257,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnP
 #pragma unroll
       for (int u = 0; u < W; ++u) {
         const uint32_t w = wk[u], w8 = wk[u] >> 8;
-        mma_f16_16816(acc[nt], aq[2 * u], w & 0x000F000Fu, w8 & 0x000F000Fu);
-        mma_f16_16816(acc[nt], aq[2 * u + 1], w & 0x00F000F0u, w8 & 0x00F000F0u);
+        mma_f16_16816(acc[nt], aq[2 * u], codes_to_half2<false>(w), codes_to_half2<false>(w8));
+        mma_f16_16816(acc[nt], aq[2 * u + 1], codes_to_half2<true>(w), codes_to_half2<true>(w8));
       }
     }
 
@@ -325,8 +326,8 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnP
         const uint32_t sel = k | (k << 4) | ((4 + k) << 8) | ((4 + k) << 12);
         const uint32_t x01 = prmt(wv[0][u], wv[1][u], sel);
         const uint32_t x23 = prmt(wv[2][u], wv[3][u], sel);
-        mma_f16_16816(o[8 * u + 2 * k], ap, x01 & 0x000F000Fu, x23 & 0x000F000Fu);
-        mma_f16_16816(o[8 * u + 2 * k + 1], ap, x01 & 0x00F000F0u, x23 & 0x00F000F0u);
+        mma_f16_16816(o[8 * u + 2 * k], ap, codes_to_half2<false>(x01), codes_to_half2<false>(x23));
+        mma_f16_16816(o[8 * u + 2 * k + 1], ap, codes_to_half2<true>(x01), codes_to_half2<true>(x23));
       }
     }
     __syncwarp();
@@ -349,7 +350,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnP
     if (g < G) {
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
-        const float sc = (nt & 1) ? kTwo20 : kTwo24;  // undo the code's power of two
+        const float sc = (nt & 1) ? 0.0625f : 1.0f;  // odd n-tiles carried 16c
         mw[g * D + (2 * tig) * NT + nt] = (o[nt][0] + o[nt][2]) * sc;
         mw[g * D + (2 * tig + 1) * NT + nt] = (o[nt][1] + o[nt][3]) * sc;
       }
@@ -406,33 +407,52 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnP
     if (!*s_last) return;
     __threadfence();
     const float* base = p.ws_part + (((size_t)n * p.Hkv + h) * p.n_splits) * G * (D + 2);
-    float* Lr = wts + 8 * kMaxSplits;
-    for (int idx = tid; idx < G * p.n_splits; idx += kAttnThreads) {
+    const int ns = p.n_splits;
+    float* lsp = wts + 8 * kMaxSplits;   // per (head, split) sums
+    float* Lr = wts + 16 * kMaxSplits;   // per head total
+    // every (head, split) maximum and sum, loaded in parallel
+    for (int idx = tid; idx < G * ns; idx += kAttnThreads) {
       const int r = idx % G, s = idx / G;
-      wts[r * kMaxSplits + s] = __ldcg(base + ((size_t)s * G + r) * (D + 2) + D);
+      const float* src = base + ((size_t)s * G + r) * (D + 2) + D;
+      wts[r * kMaxSplits + s] = __ldcg(src);
+      lsp[r * kMaxSplits + s] = __ldcg(src + 1);
     }
     __syncthreads();
-    if (tid < G) {
-      const int r = tid;
+    // per head: the global maximum, the split weights and the total sum (one warp per head)
+    for (int r = warp; r < G; r += kAttnWarps) {
       float M = -INFINITY;
-      for (int s = 0; s < p.n_splits; ++s) M = fmaxf(M, wts[r * kMaxSplits + s]);
+      for (int s = lane; s < ns; s += 32) M = fmaxf(M, wts[r * kMaxSplits + s]);
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o));
       float L = 0.0f;
-      for (int s = 0; s < p.n_splits; ++s) {
+      for (int s = lane; s < ns; s += 32) {
         const float ms = wts[r * kMaxSplits + s];
         const float e = (ms == -INFINITY) ? 0.0f : exp2f(ms - M);
         wts[r * kMaxSplits + s] = e;
-        L += e * __ldcg(base + ((size_t)s * G + r) * (D + 2) + D + 1);
+        L += e * lsp[r * kMaxSplits + s];
       }
-      Lr[r] = L;
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(FULL, L, o);
+      if (lane == 0) Lr[r] = L;
     }
     __syncthreads();
+    // weighted sum over splits; independent loads, several in flight
     for (int idx = tid; idx < G * D; idx += kAttnThreads) {
       const int r = idx / D, c = idx % D;
-      float acc = 0.0f;
-      for (int s = 0; s < p.n_splits; ++s) {
-        const float e = wts[r * kMaxSplits + s];
-        if (e != 0.0f) acc += e * __ldcg(base + ((size_t)s * G + r) * (D + 2) + c);
+      const float* src = base + (size_t)r * (D + 2) + c;
+      const size_t stride = (size_t)G * (D + 2);
+      float acc0 = 0.0f, acc1 = 0.0f, acc2 = 0.0f, acc3 = 0.0f;
+      int s = 0;
+      for (; s + 4 <= ns; s += 4) {
+        const float v0 = __ldcg(src + (size_t)s * stride), v1 = __ldcg(src + (size_t)(s + 1) * stride);
+        const float v2 = __ldcg(src + (size_t)(s + 2) * stride), v3 = __ldcg(src + (size_t)(s + 3) * stride);
+        acc0 = fmaf(wts[r * kMaxSplits + s], v0, acc0);
+        acc1 = fmaf(wts[r * kMaxSplits + s + 1], v1, acc1);
+        acc2 = fmaf(wts[r * kMaxSplits + s + 2], v2, acc2);
+        acc3 = fmaf(wts[r * kMaxSplits + s + 3], v3, acc3);
       }
+      for (; s < ns; ++s) acc0 = fmaf(wts[r * kMaxSplits + s], __ldcg(src + (size_t)s * stride), acc0);
+      const float acc = (acc0 + acc1) + (acc2 + acc3);
       qs[r * D + c] = (Lr[r] > 0.0f) ? acc / Lr[r] : 0.0f;
     }
     if (tid == 0) p.ws_count[(size_t)n * p.Hkv + h] = 0;  // leave the workspace zeroed

@@ -118,6 +118,18 @@ __device__ __forceinline__ uint32_t prmt(uint32_t a, uint32_t b, uint32_t sel) {
   return r;
 }
 
+// Two 4-bit codes -> two exact fp16 values. `x` holds a nibble in bits 0..3
+// (and 16..19) or, with `shifted`, in bits 4..7 (and 20..23). OR-ing the bits
+// into 0x6400 (= 1024, whose fp16 ulp is 1) gives 1024 + c (or 1024 + 16c);
+// subtracting 1024 is exact and leaves c (or 16c) as a normal fp16.
+template <bool shifted>
+__device__ __forceinline__ uint32_t codes_to_half2(uint32_t x) {
+  const uint32_t biased = (x & (shifted ? 0x00F000F0u : 0x000F000Fu)) | 0x64006400u;
+  uint32_t r;
+  asm("sub.rn.f16x2 %0, %1, %2;\n" : "=r"(r) : "r"(biased), "r"(0x64006400u));
+  return r;
+}
+
 __device__ __forceinline__ uint32_t pack_half2(__half lo, __half hi) {
   return static_cast<uint32_t>(__half_as_ushort(lo)) |
          (static_cast<uint32_t>(__half_as_ushort(hi)) << 16);

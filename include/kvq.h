@@ -112,6 +112,7 @@ typedef struct kvq_attn_desc {
  * desc         : host pointer to the shapes.
  * Inputs must be finite and their rotated values must lie within the fp16
  * range (|y| <= 65504); rows outside it get infinite or NaN s/z.
+ * num_tokens = 0 launches nothing and returns KVQ_OK (pointers may then be NULL).
  * Returns KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED or KVQ_ERR_CUDA.
  */
 kvq_status kv_quant_write(const void* k, const void* v, const int64_t* slot_mapping,
@@ -122,7 +123,11 @@ kvq_status kv_quant_write(const void* k, const void* v, const int64_t* slot_mapp
 /*
  * kvq_attn_workspace_size - bytes of device workspace paged_decode_attn_int4
  * needs for these shapes (0 when the call needs none). The value depends on
- * the shapes and on the current device's SM count only.
+ * the shapes and on the current device's SM count only. Returns SIZE_MAX when
+ * the shapes are invalid or no device can be queried.
+ *
+ * Layout: the first round_up(batch*num_kv_heads*4, 256) bytes are the split
+ * tickets (int32 counters), the rest holds per-split partial results.
  */
 size_t kvq_attn_workspace_size(const kvq_attn_desc* desc);
 
@@ -148,11 +153,12 @@ size_t kvq_attn_workspace_size(const kvq_attn_desc* desc);
  *                clamped and records KVQ_ERR_OUT_OF_RANGE.
  * out          : device, [B][Hq][D], fp32 or bf16 (desc->out_dtype).
  * workspace    : device, at least kvq_attn_workspace_size(desc) bytes, 16-byte
- *                aligned; may be NULL when that size is 0. It must be all zero
- *                before its first use; every call leaves it all zero again, so
- *                one buffer serves any number of calls issued one after
- *                another on a stream (calls that overlap on the GPU must use
- *                different workspaces).
+ *                aligned; may be NULL when that size is 0. Its ticket counters
+ *                must be zero before its first use (zero the whole buffer
+ *                once); every call returns them to zero, so one buffer serves
+ *                any number of calls issued one after another on a stream.
+ *                Calls that overlap on the GPU must use different workspaces.
+ * batch = 0 launches nothing and returns KVQ_OK (pointers may then be NULL).
  * Returns KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_WORKSPACE
  * or KVQ_ERR_CUDA.
  */

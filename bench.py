@@ -80,12 +80,18 @@ def aggregate_gbs(bytes_per_step, steps, world, max_ms):
     return bytes_per_step * steps * world / (max_ms / 1e3) / 1e9
 
 
-def source_digest():
-    """Hash of the kernel sources: a committed DRAM-traffic figure is valid
-    only for the kernels it was captured from."""
+KERNEL_SOURCES = {
+    "kv_quant_write": ["kvq_write.cuh", "kvq_device.cuh"],
+    "paged_decode_attn_int4": ["kvq_decode.cuh", "kvq_device.cuh"],
+}
+
+
+def source_digest(kernel):
+    """Hash of one kernel's sources: a committed DRAM-traffic figure is valid
+    only for the kernel it was captured from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_kv_cache_20_b200", "csrc")
-    for name in sorted(os.listdir(csrc)):
+    for name in KERNEL_SOURCES[kernel]:
         with open(os.path.join(csrc, name), "rb") as f:
             h.update(name.encode() + f.read())
     return h.hexdigest()[:16]
@@ -101,7 +107,7 @@ def committed_traffic(kernel):
     except (OSError, ValueError):
         return None
     entry = t.get(kernel)
-    if not entry or entry.get("source_digest") != source_digest():
+    if not entry or entry.get("source_digest") != source_digest(kernel):
         return None
     return entry.get("dram_bytes_per_launch")
 

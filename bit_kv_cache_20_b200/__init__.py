@@ -25,6 +25,7 @@ PAGE_SIZE = 16
 __all__ = [
     "PAGE_SIZE", "KVQError", "alloc_cache", "kv_quant_write", "paged_decode_attn_int4",
     "attn_workspace_size", "alloc_workspace", "get_device_error", "library_path",
+    "paged_decode_attn_int4_static_ws",
 ]
 
 
@@ -153,6 +154,34 @@ def paged_decode_attn_int4(q: torch.Tensor, cache: torch.Tensor, scales: torch.T
                                   _ptr(context_lens), _ptr(out), ws_ptr, ws_bytes,
                                   ctypes.byref(desc), ctypes.c_void_p(_stream_handle(stream)))
     _lib.check(st, "paged_decode_attn_int4")
+
+
+def paged_decode_attn_int4_static_ws(q: torch.Tensor, cache: torch.Tensor, scales: torch.Tensor,
+                                     zeros: torch.Tensor, page_table: torch.Tensor,
+                                     context_lens: torch.Tensor, out: torch.Tensor,
+                                     hadamard_block: int, softmax_scale: float = 0.0,
+                                     stream=None) -> None:
+    """paged_decode_attn_int4 for callers that must not allocate device memory
+    (e.g. a plug-in whose host runtime owns all GPU memory): the split-K
+    scratch is a fixed array inside the library, shared by every call on the
+    device, so calls must not overlap on the GPU. The first call on a device
+    looks up that array's address; make it before any stream capture."""
+    _need(q, "q", torch.bfloat16)
+    _need(page_table, "page_table", torch.int32)
+    _need(context_lens, "context_lens", torch.int32)
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("out must be float32 or bfloat16")
+    _need(out, "out", out.dtype)
+    if tuple(out.shape) != tuple(q.shape):
+        raise ValueError("out must have q's shape")
+    desc = _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scale,
+                      0 if out.dtype == torch.float32 else 1)
+    if context_lens.numel() != desc.batch:
+        raise ValueError("context_lens must hold one length per sequence")
+    st = _lib.lib().paged_decode_attn_int4_static_ws(
+        _ptr(q), _ptr(cache), _ptr(scales), _ptr(zeros), _ptr(page_table), _ptr(context_lens),
+        _ptr(out), ctypes.byref(desc), ctypes.c_void_p(_stream_handle(stream)))
+    _lib.check(st, "paged_decode_attn_int4_static_ws")
 
 
 def get_device_error(stream=None) -> int:

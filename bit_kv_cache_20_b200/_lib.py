@@ -47,6 +47,11 @@ SIGNATURES = [
                                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                               ctypes.POINTER(AttnDesc), ctypes.c_void_p]),
+    ("paged_decode_attn_int4_static_ws", ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p,
+                                                        ctypes.c_void_p, ctypes.c_void_p,
+                                                        ctypes.c_void_p, ctypes.c_void_p,
+                                                        ctypes.c_void_p, ctypes.POINTER(AttnDesc),
+                                                        ctypes.c_void_p]),
     ("kvq_get_device_error", ctypes.c_int, [ctypes.c_void_p]),
     ("kvq_status_string", ctypes.c_char_p, [ctypes.c_int32]),
     ("kvq_abi_version", ctypes.c_int32, []),

@@ -5,6 +5,7 @@
 #include <cuda_runtime.h>
 
 #include <atomic>
+#include <mutex>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -335,3 +336,68 @@ const char* kvq_status_string(int32_t status) {
 int32_t kvq_abi_version(void) { return KVQ_ABI_VERSION; }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// paged_decode_attn_int4_static_ws: the decode step without a caller-provided
+// workspace, for callers that cannot allocate device memory. The split-K
+// scratch is this file-scope array (one per device that loads the library).
+// ---------------------------------------------------------------------------
+static __device__ __align__(256) unsigned char g_static_workspace[KVQ_STATIC_WORKSPACE_BYTES];
+
+namespace {
+
+std::mutex g_static_ws_mutex;
+void* g_static_ws_ptr[kMaxDevices] = {};
+
+// Device address of g_static_workspace on `dev` (which must be current). In
+// host code the array's name is only a host-side stand-in, so the address is
+// looked up once per device and cached.
+kvq_status static_workspace_on(int dev, void** out) {
+  std::lock_guard<std::mutex> lock(g_static_ws_mutex);
+  if (!g_static_ws_ptr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return KVQ_ERR_CUDA;
+    }
+    g_static_ws_ptr[dev] = p;
+  }
+  *out = g_static_ws_ptr[dev];
+  return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" kvq_status paged_decode_attn_int4_static_ws(const void* q, const uint8_t* cache,
+                                                       const void* scales, const void* zeros,
+                                                       const int32_t* page_table,
+                                                       const int32_t* context_lens, void* out,
+                                                       const kvq_attn_desc* desc, void* stream) {
+  kvq_status st = check_attn_desc(desc);
+  if (st != KVQ_OK) return st;
+  if (desc->batch == 0) return KVQ_OK;
+  if (!cache || !aligned(cache, 16)) return KVQ_ERR_INVALID_ARG;
+  int dev = 0;
+  st = select_device_of(cache, &dev);  // makes the cache's device current
+  if (st != KVQ_OK) return st;
+  if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
+  const int sms = sm_count(dev);
+  if (sms < 1) return KVQ_ERR_CUDA;
+  const size_t need = workspace_bytes_for(desc, plan_splits(desc, sms));
+  if (need > KVQ_STATIC_WORKSPACE_BYTES) return KVQ_ERR_WORKSPACE;
+  void* ws = nullptr;
+  if (need > 0) {
+    st = static_workspace_on(dev, &ws);
+    if (st != KVQ_OK) return st;
+    // the split tickets must start at zero; a call that stopped early could
+    // have left some of them set
+    const size_t units = (size_t)desc->batch * desc->num_kv_heads;
+    const size_t tickets = ((units * sizeof(int) + 255) / 256) * 256;
+    if (cudaMemsetAsync(ws, 0, tickets, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
+      cudaGetLastError();
+      return KVQ_ERR_CUDA;
+    }
+  }
+  return paged_decode_attn_int4(q, cache, scales, zeros, page_table, context_lens, out, ws,
+                                need > 0 ? (size_t)KVQ_STATIC_WORKSPACE_BYTES : 0, desc, stream);
+}

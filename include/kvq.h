@@ -170,6 +170,37 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache,
                                   const kvq_attn_desc* desc, void* stream);
 
 /*
+ * paged_decode_attn_int4_static_ws - the same decode step as
+ * paged_decode_attn_int4, for callers that are not allowed to allocate device
+ * memory. Examples: a plug-in hosted by a serving runtime that owns all GPU
+ * memory through its own pool and forbids raw cudaMalloc, or a latency-bound
+ * path where an allocation (which may synchronize the device) is unacceptable.
+ * The paper has no counterpart; this is a deployment convenience.
+ *
+ * Instead of a caller-provided workspace, the split-K scratch lives in a
+ * fixed device array of KVQ_STATIC_WORKSPACE_BYTES inside this library (every
+ * GPU that loads the library holds it until the process exits). The caller
+ * still passes all inputs and outputs, exactly as for paged_decode_attn_int4.
+ *  - The first call on a device looks up that array's device address (once
+ *    per device); make that first call before any stream capture.
+ *  - Every call clears the array's ticket counters on `stream` before its
+ *    kernel and otherwise reuses whatever the previous call left there.
+ *  - All calls share the one array per device: calls that overlap on the GPU
+ *    (other streams, other host threads) race and give wrong results.
+ *  - Shapes that would need more scratch than the array holds are rejected
+ *    with KVQ_ERR_WORKSPACE before anything is launched. On a 148-SM B200 every
+ *    accepted shape fits (the library uses at most ~1.9 MB).
+ * No allocation of any kind is made. Returns the same statuses as
+ * paged_decode_attn_int4.
+ */
+#define KVQ_STATIC_WORKSPACE_BYTES (2u * 1024u * 1024u)
+kvq_status paged_decode_attn_int4_static_ws(const void* q, const uint8_t* cache,
+                                            const void* scales, const void* zeros,
+                                            const int32_t* page_table,
+                                            const int32_t* context_lens, void* out,
+                                            const kvq_attn_desc* desc, void* stream);
+
+/*
  * kvq_get_device_error - synchronizes `stream`, then returns and clears the
  * current device's error word (KVQ_OK when no kernel recorded an error).
  * Returns KVQ_ERR_CUDA if the synchronization itself fails.

@@ -112,11 +112,17 @@ def _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scal
 
 
 def attn_workspace_size(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
-                        num_pages: int, max_pages_per_seq: int, hadamard_block: int) -> int:
-    """Bytes of workspace paged_decode_attn_int4 needs on the current device."""
+                        num_pages: int, max_pages_per_seq: int, hadamard_block: int,
+                        device=None) -> int:
+    """Bytes of workspace paged_decode_attn_int4 needs on `device` (default:
+    torch's current CUDA device)."""
+    L = _lib.lib()
+    idx = None if device is None else torch.device(device).index
+    dev = torch.cuda.current_device() if idx is None else idx
+    _lib.check(L.kvq_set_device(int(dev)), "kvq_set_device")
     desc = AttnDesc(batch, num_q_heads, num_kv_heads, head_dim, PAGE_SIZE, num_pages,
                     max_pages_per_seq, hadamard_block, 0.0, 0)
-    n = _lib.lib().kvq_attn_workspace_size(ctypes.byref(desc))
+    n = L.kvq_attn_workspace_size(ctypes.byref(desc))
     if n == ctypes.c_size_t(-1).value:
         raise KVQError(1, "kvq_attn_workspace_size (invalid shapes or no device)")
     return int(n)

@@ -127,25 +127,105 @@ kvq_status dispatch_write(const kvq::WriteParams& p, int b, int dev, cudaStream_
 // paged_decode_attn_int4
 // ---------------------------------------------------------------------------
 struct SplitPlan {
-  int n_splits;
+  int n_splits;         // CTAs per (sequence, kv head)
   int pages_per_split;
+  int cluster;          // CTAs per thread-block cluster (divides n_splits)
+  int n_parts;          // clusters per (sequence, kv head) = partials in the workspace
 };
 
-// Split each (sequence, kv head) so that all CTAs fit in one wave (three
-// resident CTAs per SM, which the kernel's launch bounds guarantee), keeping
-// at least 8 pages (two per warp) per split.
-SplitPlan plan_splits(const kvq_attn_desc* d, int sms) {
+template <int D, int BLK>
+const void* decode_kernel_ptr() {
+  return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK>);
+}
+
+const void* decode_kernel_for(int D, int b) {
+  if (D == 64) {
+    if (b == 0) return decode_kernel_ptr<64, 0>();
+    if (b == 32) return decode_kernel_ptr<64, 32>();
+    if (b == 64) return decode_kernel_ptr<64, 64>();
+    return nullptr;
+  }
+  if (b == 0) return decode_kernel_ptr<128, 0>();
+  if (b == 32) return decode_kernel_ptr<128, 32>();
+  if (b == 64) return decode_kernel_ptr<128, 64>();
+  if (b == 128) return decode_kernel_ptr<128, 128>();
+  return nullptr;
+}
+
+int decode_smem_bytes(int D) {
+  return D == 64 ? kvq::AttnSmem<64>::kTotal : kvq::AttnSmem<128>::kTotal;
+}
+
+// Opt the decode kernel instance into its dynamic shared memory (once per
+// device and instance).
+bool prepare_decode_kernel(int dev, int D, int b) {
+  static std::atomic<int> done[kMaxDevices][8];
+  const int slot = (D == 64 ? 0 : 4) + (b == 0 ? 0 : b == 32 ? 1 : b == 64 ? 2 : 3);
+  if (done[dev][slot].load(std::memory_order_relaxed)) return true;
+  const void* k = decode_kernel_for(D, b);
+  if (!k || cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, decode_smem_bytes(D)) !=
+                cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  done[dev][slot].store(1, std::memory_order_relaxed);
+  return true;
+}
+
+// Clusters of `cs` decode CTAs that can be resident at once on the device.
+int max_active_clusters(int dev, int D, int b, int cs) {
+  static std::atomic<int> cache[kMaxDevices][8][kvq::kMaxCluster + 1];
+  const int slot = (D == 64 ? 0 : 4) + (b == 0 ? 0 : b == 32 ? 1 : b == 64 ? 2 : 3);
+  int v = cache[dev][slot][cs].load(std::memory_order_relaxed);
+  if (v > 0) return v;
+  if (!prepare_decode_kernel(dev, D, b)) return 0;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(cs, 1, 1);
+  cfg.blockDim = dim3(kvq::kAttnThreads, 1, 1);
+  cfg.dynamicSmemBytes = decode_smem_bytes(D);
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = cs;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  int n = 0;
+  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel_for(D, b), &cfg) != cudaSuccess || n < 1) {
+    cudaGetLastError();
+    return 0;
+  }
+  cache[dev][slot][cs].store(n, std::memory_order_relaxed);
+  return n;
+}
+
+// Split each (sequence, kv head) into CTAs grouped in thread-block clusters
+// (which merge on chip), choosing the cluster size and split count so that
+// every CTA of the launch is resident at once (one wave, as the occupancy API
+// reports for clusters of that size) and each split keeps at least 8 pages.
+// Only when a (sequence, kv head) has more than one cluster do partial
+// results go through the workspace.
+SplitPlan plan_splits(const kvq_attn_desc* d, int dev) {
   const long long units = (long long)d->batch * d->num_kv_heads;
-  const long long target = 3LL * sms;
-  long long ns = units > 0 ? target / units : 1;
-  long long most = d->max_pages_per_seq / 8;
-  if (most < 1) most = 1;
-  if (ns > most) ns = most;
-  if (ns > kvq::kMaxSplits) ns = kvq::kMaxSplits;
-  if (ns < 1) ns = 1;
-  const int pps = (int)((d->max_pages_per_seq + ns - 1) / ns);
-  const int n = (d->max_pages_per_seq + pps - 1) / pps;
-  return {n, pps};
+  long long cap = d->max_pages_per_seq / 8;
+  if (cap < 1) cap = 1;
+  if (cap > kvq::kMaxSplits) cap = kvq::kMaxSplits;
+  SplitPlan best = {1, d->max_pages_per_seq, 1, 1};
+  if (units <= 0 || cap == 1) return best;
+  for (int cs = kvq::kMaxCluster; cs >= 1; --cs) {
+    const int mac = max_active_clusters(dev, d->head_dim, d->hadamard_block, cs);
+    const long long per_unit = mac / units;  // clusters per (sequence, kv head) in one wave
+    if (per_unit < 1) continue;
+    long long parts = per_unit;
+    if (parts > cap / cs) parts = cap / cs;
+    if (parts > kvq::kMaxParts) parts = kvq::kMaxParts;
+    if (parts < 1) continue;
+    const long long ns = parts * cs;
+    // larger clusters are tried first; a smaller one must buy > 10 % more splits
+    if (ns * 10 > best.n_splits * 11LL) best = {(int)ns, 0, cs, (int)parts};
+  }
+  best.pages_per_split = (d->max_pages_per_seq + best.n_splits - 1) / best.n_splits;
+  return best;
 }
 
 kvq_status check_attn_desc(const kvq_attn_desc* d) {
@@ -166,31 +246,47 @@ kvq_status check_attn_desc(const kvq_attn_desc* d) {
 }
 
 size_t workspace_bytes_for(const kvq_attn_desc* d, const SplitPlan& plan) {
-  if (plan.n_splits <= 1 || d->batch == 0) return 0;
+  if (plan.n_parts <= 1 || d->batch == 0) return 0;
   const size_t units = (size_t)d->batch * d->num_kv_heads;
   const size_t counters = ((units * sizeof(int) + 255) / 256) * 256;
   const size_t G = (size_t)(d->num_q_heads / d->num_kv_heads);
-  return counters + units * plan.n_splits * G * (d->head_dim + 2) * sizeof(float);
+  return counters + units * plan.n_parts * G * (d->head_dim + 2) * sizeof(float);
 }
 
 template <int D, int BLK>
-kvq_status launch_attn(const kvq::AttnParams& p, cudaStream_t s) {
+kvq_status launch_attn(const kvq::AttnParams& p, int dev, cudaStream_t s) {
   auto kern = kvq::kvq_decode_kernel<D, BLK>;
   constexpr int smem = kvq::AttnSmem<D>::kTotal;
-  static_assert(smem <= 48 * 1024, "decode kernel shared memory exceeds the default limit");
-  dim3 grid(p.n_splits, p.Hkv, p.B);
-  kern<<<grid, kvq::kAttnThreads, smem, s>>>(p);
+  static_assert(3 * (smem + 1024) <= 228 * 1024, "three decode CTAs must fit on one SM");
+  if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
+  if (!prepare_decode_kernel(dev, D, BLK)) return KVQ_ERR_CUDA;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.n_splits, p.Hkv, p.B);
+  cfg.blockDim = dim3(kvq::kAttnThreads, 1, 1);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = p.cluster_size;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
 template <int D>
-kvq_status dispatch_attn(const kvq::AttnParams& p, int b, cudaStream_t s) {
+kvq_status dispatch_attn(const kvq::AttnParams& p, int b, int dev, cudaStream_t s) {
   switch (b) {
-    case 0: return launch_attn<D, 0>(p, s);
-    case 32: return launch_attn<D, 32>(p, s);
-    case 64: return launch_attn<D, 64>(p, s);
+    case 0: return launch_attn<D, 0>(p, dev, s);
+    case 32: return launch_attn<D, 32>(p, dev, s);
+    case 64: return launch_attn<D, 64>(p, dev, s);
     case 128:
-      if constexpr (D >= 128) return launch_attn<D, 128>(p, s);
+      if constexpr (D >= 128) return launch_attn<D, 128>(p, dev, s);
       return KVQ_ERR_UNSUPPORTED;
     default: return KVQ_ERR_UNSUPPORTED;
   }
@@ -244,9 +340,8 @@ size_t kvq_attn_workspace_size(const kvq_attn_desc* desc) {
     cudaGetLastError();
     return SIZE_MAX;
   }
-  const int sms = sm_count(dev);
-  if (sms < 1) return SIZE_MAX;
-  return workspace_bytes_for(desc, plan_splits(desc, sms));
+  if (dev < 0 || dev >= kMaxDevices) return SIZE_MAX;
+  return workspace_bytes_for(desc, plan_splits(desc, dev));
 }
 
 kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const void* scales,
@@ -265,9 +360,8 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const voi
   int dev = 0;
   st = select_device_of(cache, &dev);
   if (st != KVQ_OK) return st;
-  const int sms = sm_count(dev);
-  if (sms < 1) return KVQ_ERR_CUDA;
-  const SplitPlan plan = plan_splits(&d, sms);
+  if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
+  const SplitPlan plan = plan_splits(&d, dev);
   const size_t need = workspace_bytes_for(&d, plan);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16)))
     return KVQ_ERR_WORKSPACE;
@@ -287,6 +381,8 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const voi
   p.max_pages = d.max_pages_per_seq;
   p.n_splits = plan.n_splits;
   p.pages_per_split = plan.pages_per_split;
+  p.cluster_size = plan.cluster;
+  p.n_parts = plan.n_parts;
   p.out_bf16 = d.out_dtype;
   const double cb = d.hadamard_block > 0 ? 1.0 / std::sqrt((double)d.hadamard_block) : 1.0;
   const double scale = d.softmax_scale > 0.0f ? (double)d.softmax_scale : 1.0 / std::sqrt((double)d.head_dim);
@@ -302,8 +398,8 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const voi
     p.ws_part = nullptr;
   }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d.head_dim == 64 ? dispatch_attn<64>(p, d.hadamard_block, s)
-                          : dispatch_attn<128>(p, d.hadamard_block, s);
+  return d.head_dim == 64 ? dispatch_attn<64>(p, d.hadamard_block, dev, s)
+                          : dispatch_attn<128>(p, d.hadamard_block, dev, s);
 }
 
 kvq_status kvq_get_device_error(void* stream) {
@@ -318,6 +414,15 @@ kvq_status kvq_get_device_error(void* stream) {
     return KVQ_ERR_CUDA;
   }
   return static_cast<kvq_status>(v);
+}
+
+kvq_status kvq_set_device(int32_t device) {
+  if (device < 0) return KVQ_ERR_INVALID_ARG;
+  if (cudaSetDevice(device) != cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
+  return KVQ_OK;
 }
 
 const char* kvq_status_string(int32_t status) {
@@ -381,9 +486,7 @@ extern "C" kvq_status paged_decode_attn_int4_static_ws(const void* q, const uint
   st = select_device_of(cache, &dev);  // makes the cache's device current
   if (st != KVQ_OK) return st;
   if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
-  const int sms = sm_count(dev);
-  if (sms < 1) return KVQ_ERR_CUDA;
-  const size_t need = workspace_bytes_for(desc, plan_splits(desc, sms));
+  const size_t need = workspace_bytes_for(desc, plan_splits(desc, dev));
   if (need > KVQ_STATIC_WORKSPACE_BYTES) return KVQ_ERR_WORKSPACE;
   void* ws = nullptr;
   if (need > 0) {

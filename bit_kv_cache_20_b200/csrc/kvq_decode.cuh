@@ -5,29 +5,37 @@
 // rotates q once, runs attention in the rotated space directly on the codes,
 // and rotates the output back: out = R sum_t p_t v^_t.
 //
-// Grid (split, kv head, sequence); 4 warps per CTA. Each warp streams its
-// pages (page p_begin + warp + 4 i) through a private ring of bulk copies
-// (TMA engine, 1-D, completing on an mbarrier): 16*D code bytes (K block then
-// V block) plus 64 B of scales and 64 B of zeros per page.
-//
-// Per page, on the tensor cores (mma.m16n8k16, f16 in, f32 accumulate):
-//   rows 0..7 of the A operand = the "hi" fp16 part of up to 8 query heads,
-//   rows 8..15 = their "lo" part (x = hi + lo keeps ~22 bits), so one MMA
-//   carries both halves and GQA groups up to 8 share one K/V stream.
-//   QK:  S[16 x 16 tokens] = Qhl[16 x D] * codes^T       (k = channels)
-//   PV:  O[16 x D]        += Phl[16 x 16 tokens] * codes  (k = tokens)
-//   The 4-bit codes enter the MMA as exact normal fp16 values c (or 16c for a
-//   nibble at bits 4..7, compensated by a factor 1/16 on the other operand or
-//   in the epilogue). Subnormal fp16 operands are avoided on purpose: small
-//   products built from them lost precision in the tensor-core accumulation
-//   (a systematic bias of ~2^-13 relative, measured on B200).
-//   Dequantization is folded into the per-token scalars:
-//     logit_t = s_t * (q~ . code_t) + z_t * sum(q~)
-//     o_rot   = (sum_t p_t s_t code_t + sum_t p_t z_t) / sum_t p_t
-// Online softmax in base 2 (log2 e folded into q~). Warps merge in shared
-// memory; splits merge through a workspace, the last CTA to arrive (atomic
-// ticket) combining them and applying the inverse rotation.
+// Grid (split, kv head, sequence), 4 warps per CTA; the splits of one
+// (sequence, kv head) form thread-block clusters of up to 8 CTAs.
+//  - Each warp walks its tasks (a task = two consecutive pages of the CTA's
+//    page range) through a private ring of 1-D bulk copies (TMA engine)
+//    completing on mbarriers: 16*D code bytes (K block, V block) + 64 B
+//    scales + 64 B zeros per page. The first copies are issued before q is
+//    rotated, so the rotation overlaps them.
+//  - Per task, on the tensor cores (mma.m16n8k16, f16 in, f32 accumulate):
+//      QK: S[16 rows x 32 tokens] = Qhl[16 x D] * codes^T   (4 n-tiles)
+//      PV: O[16 rows x D]        += Phl[16 x 32 tokens] * codes (2 k-steps)
+//    A rows 0..7 carry the fp16 "hi" part of up to 8 query heads and rows
+//    8..15 the "lo" remainder (x = hi + lo keeps ~22 bits), so one MMA does
+//    both halves and a GQA group of up to 8 shares one K/V stream.
+//    The 4-bit codes enter as exact normal fp16 values c (or 16c for a nibble
+//    at bits 4..7, compensated by 1/16 on the other operand or in the
+//    epilogue). Subnormal fp16 operands are avoided on purpose: small
+//    products built from them lost precision in the tensor-core accumulation
+//    (a systematic bias of ~2^-13 relative, measured on B200).
+//    Dequantization is folded into per-token scalars:
+//      logit_t = s_t * (q~ . code_t) + z_t * sum(q~)
+//      o_rot   = (sum_t p_t s_t code_t + sum_t p_t z_t) / sum_t p_t
+//    Online softmax in base 2 (log2 e folded into q~), rescaling only when
+//    the running maximum grows.
+//  - Warps merge in shared memory; the CTAs of a cluster merge through
+//    distributed shared memory into the cluster's first CTA; when a
+//    (sequence, kv head) has several clusters, their partial results meet in
+//    the workspace and the last cluster to arrive (atomic ticket) combines
+//    them. The final CTA applies the inverse rotation and stores.
 #pragma once
+
+#include <climits>
 
 #include "kvq_device.cuh"
 
@@ -41,11 +49,13 @@ struct AttnParams {
   const int32_t* page_table;  // [B][max_pages]
   const int32_t* ctx_lens;    // [B]
   void* out;                  // [B][Hq][D] fp32 or bf16
-  float* ws_part;             // [B][Hkv][splits][G][D + 2]
+  float* ws_part;             // [B][Hkv][n_parts][G][D + 2]
   int* ws_count;              // [B][Hkv]
   int B, Hq, Hkv, G;
   int num_pages, max_pages;
   int n_splits, pages_per_split;
+  int cluster_size;           // CTAs per cluster along the split axis
+  int n_parts;                // n_splits / cluster_size
   int out_bf16;
   float qmul;                 // c_b * softmax_scale * log2(e)
   float cb;                   // c_b (output rotation), 1 for plain INT4
@@ -53,24 +63,29 @@ struct AttnParams {
 
 constexpr int kAttnWarps = 4;
 constexpr int kAttnThreads = kAttnWarps * 32;
-constexpr int kStages = 4;
-constexpr int kMaxSplits = 64;
+constexpr int kStages = 3;       // ring depth per warp, in tasks of two pages
+constexpr int kMaxSplits = 256;
+constexpr int kMaxParts = 64;    // partial results per (sequence, kv head) in the workspace
+constexpr int kMaxCluster = 8;
 
 template <int D>
 struct AttnSmem {
-  static constexpr int kCodeBytes = 16 * D;             // K block + V block of one page-head
-  static constexpr int kStageBytes = kCodeBytes + 128;  // + 32 scales + 32 zeros (fp16)
+  static constexpr int kCodeBytes = 16 * D;               // K block + V block of one page-head
+  static constexpr int kPageBytes = kCodeBytes + 128;     // + 32 scales + 32 zeros (fp16)
+  static constexpr int kStageBytes = 2 * kPageBytes;      // one task = two pages
   static constexpr int kRingBytes = kAttnWarps * kStages * kStageBytes;
   // per-warp merge area (overlays the ring after the page loop)
   static constexpr int kMergeFloatsPerWarp = 8 * D + 3 * 8;
   static constexpr int kMergeBytes = kAttnWarps * kMergeFloatsPerWarp * 4;
   static constexpr int kUnionBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
-  static constexpr int kQBytes = 8 * D * 4;             // q / output rows, fp32
-  static constexpr int kWeightBytes = (2 * 8 * kMaxSplits + 8) * 4;  // split maxima/weights, sums, per-head L
+  static constexpr int kQBytes = 8 * D * 4;               // q rows, then the CTA's merged O
+  static constexpr int kMLBytes = 8 * 2 * 4;              // the CTA's merged (M, L) per head
+  static constexpr int kWeightBytes = (2 * 8 * kMaxParts + 8) * 4;
   static constexpr int kBarBytes = kAttnWarps * kStages * 8;
   static constexpr int kFlagBytes = kAttnWarps * kStages * 4 + 16;
   static constexpr int kOffQ = kUnionBytes;
-  static constexpr int kOffW = kOffQ + kQBytes;
+  static constexpr int kOffML = kOffQ + kQBytes;
+  static constexpr int kOffW = kOffML + kMLBytes;
   static constexpr int kOffBar = kOffW + kWeightBytes;
   static constexpr int kOffFlag = kOffBar + kBarBytes;
   static constexpr int kTotal = kOffFlag + kFlagBytes;
@@ -94,6 +109,15 @@ __device__ __forceinline__ void smem_fwht_rows(float* rows, int nrows) {
   }
 }
 
+// hi/lo fp16 pair of two floats, packed as the A fragment wants them.
+__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+  const __half2 h = __floats2half2_rn(x0, x1);
+  const float2 hf = __half22float2(h);
+  const __half2 l = __floats2half2_rn(__fsub_rn(x0, hf.x), __fsub_rn(x1, hf.y));
+  hi = *reinterpret_cast<const uint32_t*>(&h);
+  lo = *reinterpret_cast<const uint32_t*>(&l);
+}
+
 template <int D, int BLK>
 __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnParams p) {
   using S = AttnSmem<D>;
@@ -103,6 +127,7 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnP
   constexpr int NT = D / 8;   // PV n-tiles
   extern __shared__ __align__(128) uint8_t smem[];
   float* qs = reinterpret_cast<float*>(smem + S::kOffQ);
+  float* cml = reinterpret_cast<float*>(smem + S::kOffML);
   float* wts = reinterpret_cast<float*>(smem + S::kOffW);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kOffBar);
   int* flags = reinterpret_cast<int*>(smem + S::kOffFlag);
@@ -122,13 +147,76 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnP
   const int n_pages = (ctx + 15) >> 4;
   const int p_begin = split * p.pages_per_split;
   const int p_end = min(p_begin + p.pages_per_split, n_pages);
+  const int n_tasks = (p_end > p_begin) ? (p_end - p_begin + 1) / 2 : 0;
+  const int n_my = (n_tasks > warp) ? (n_tasks - warp + kAttnWarps - 1) / kAttnWarps : 0;
+
+  uint8_t* ring = smem + warp * kStages * S::kStageBytes;
+  const uint32_t ring_s = smem_addr(ring);
+  const uint32_t bar0 = smem_addr(&bars[warp * kStages]);
+  int* wflags = flags + warp * kStages;
+  const int32_t* pt_row = p.page_table + (size_t)n * p.max_pages;
 
   if (lane == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(smem_addr(&bars[warp * kStages + s]), 1);
+    for (int s = 0; s < kStages; ++s) mbar_init(bar0 + 8 * s, 1);
     mbar_init_fence();
   }
+  __syncwarp();
 
-  // ---- q~ = R q * (softmax_scale * log2 e), rows >= G are zero ------------
+  // ---- page ids of this warp's tasks, 32 tasks at a time ---------------------
+  // task i of this warp covers pages p_begin + 2*(warp + 4 i) and the next one;
+  // INT_MIN marks "no page" (past the split's range).
+  int pid_base = 0, pid_a = INT_MIN, pid_b = INT_MIN;
+  auto load_ids = [&](int base) {
+    const int i = base + lane;
+    const int pa = p_begin + 2 * (warp + kAttnWarps * i);
+    pid_a = (i < n_my && pa < p_end) ? pt_row[pa] : INT_MIN;
+    pid_b = (i < n_my && pa + 1 < p_end) ? pt_row[pa + 1] : INT_MIN;
+  };
+  load_ids(0);
+
+  // Issue the copies of task i into its ring stage (all lanes call; i grows by one).
+  auto issue = [&](int i) {
+    if (i - pid_base >= 32) {
+      pid_base += 32;
+      load_ids(pid_base);
+    }
+    const int ia = __shfl_sync(FULL, pid_a, i - pid_base);
+    const int ib = __shfl_sync(FULL, pid_b, i - pid_base);
+    if (lane == 0) {
+      const int st = i % kStages;
+      const uint32_t bar = bar0 + 8 * st;
+      const uint32_t dst = ring_s + st * S::kStageBytes;
+      const bool va = ia >= 0 && ia < p.num_pages;
+      const bool vb = ib >= 0 && ib < p.num_pages;
+      if ((ia != INT_MIN && !va) || (ib != INT_MIN && !vb)) record_error(KVQ_ERR_OUT_OF_RANGE);
+      wflags[st] = (va ? 1 : 0) | (vb ? 2 : 0);
+      const uint32_t bytes = (va ? S::kPageBytes : 0) + (vb ? S::kPageBytes : 0);
+      if (bytes == 0) {
+        mbar_arrive(bar);
+      } else {
+        mbar_arrive_expect_tx(bar, bytes);
+        if (va) {
+          const size_t ph = (size_t)ia * p.Hkv + h;
+          bulk_g2s(dst, p.cache + ph * S::kCodeBytes, S::kCodeBytes, bar);
+          bulk_g2s(dst + S::kCodeBytes, p.scales + ph * 32, 64, bar);
+          bulk_g2s(dst + S::kCodeBytes + 64, p.zeros + ph * 32, 64, bar);
+        }
+        if (vb) {
+          const size_t ph = (size_t)ib * p.Hkv + h;
+          const uint32_t d1 = dst + S::kPageBytes;
+          bulk_g2s(d1, p.cache + ph * S::kCodeBytes, S::kCodeBytes, bar);
+          bulk_g2s(d1 + S::kCodeBytes, p.scales + ph * 32, 64, bar);
+          bulk_g2s(d1 + S::kCodeBytes + 64, p.zeros + ph * 32, 64, bar);
+        }
+      }
+    }
+  };
+
+  const int pre = min(n_my, kStages);
+  for (int i = 0; i < pre; ++i) issue(i);
+  int issued = pre;
+
+  // ---- q~ = R q * (softmax_scale * log2 e), rows >= G are zero --------------
   for (int i = tid; i < 8 * D; i += kAttnThreads) {
     const int r = i / D, c = i % D;
     qs[i] = (r < G) ? bf16_bits_to_float(p.q[((size_t)n * p.Hq + (size_t)h * G + r) * D + c]) : 0.0f;
@@ -165,123 +253,75 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnP
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
       const float f = t ? up * 0.0625f : up;
-      __half h0, l0, h1, l1, h2, l2, h3, l3;
-      split_half(qv[8 * u + t] * f, h0, l0);
-      split_half(qv[8 * u + t + 4] * f, h1, l1);
-      split_half(qv[8 * u + t + 2] * f, h2, l2);
-      split_half(qv[8 * u + t + 6] * f, h3, l3);
-      aq[2 * u + t][0] = pack_half2(h0, h1);
-      aq[2 * u + t][1] = pack_half2(l0, l1);
-      aq[2 * u + t][2] = pack_half2(h2, h3);
-      aq[2 * u + t][3] = pack_half2(l2, l3);
+      split_pair(qv[8 * u + t] * f, qv[8 * u + t + 4] * f, aq[2 * u + t][0], aq[2 * u + t][1]);
+      split_pair(qv[8 * u + t + 2] * f, qv[8 * u + t + 6] * f, aq[2 * u + t][2], aq[2 * u + t][3]);
     }
   }
-  __syncthreads();  // barrier init visible; qs free for reuse later
 
-  // ---- page stream ---------------------------------------------------------
-  const int my_first = p_begin + warp;
-  const int n_my = (my_first < p_end) ? (p_end - my_first + kAttnWarps - 1) / kAttnWarps : 0;
-  uint8_t* ring = smem + warp * kStages * S::kStageBytes;
-  const uint32_t ring_s = smem_addr(ring);
-  const uint32_t bar0 = smem_addr(&bars[warp * kStages]);
-  int* wflags = flags + warp * kStages;
-  const int32_t* pt_row = p.page_table + (size_t)n * p.max_pages;
-
-  int pid_base = 0;
-  int pid_reg = (lane < n_my) ? pt_row[my_first + lane * kAttnWarps] : 0;
-  auto issue = [&](int i) {  // called by all lanes, i increasing by one
-    if (i - pid_base >= 32) {
-      pid_base += 32;
-      const int j = pid_base + lane;
-      pid_reg = (j < n_my) ? pt_row[my_first + j * kAttnWarps] : 0;
-    }
-    const int pid = __shfl_sync(FULL, pid_reg, i - pid_base);
-    if (lane == 0) {
-      const int st = i % kStages;
-      const uint32_t bar = bar0 + st * 8;
-      const uint32_t dst = ring_s + st * S::kStageBytes;
-      if (pid >= 0 && pid < p.num_pages) {
-        wflags[st] = 1;
-        const size_t ph = (size_t)pid * p.Hkv + h;
-        mbar_arrive_expect_tx(bar, S::kStageBytes);
-        bulk_g2s(dst, p.cache + ph * S::kCodeBytes, S::kCodeBytes, bar);
-        bulk_g2s(dst + S::kCodeBytes, p.scales + ph * 32, 64, bar);
-        bulk_g2s(dst + S::kCodeBytes + 64, p.zeros + ph * 32, 64, bar);
-      } else {
-        wflags[st] = 0;
-        record_error(KVQ_ERR_OUT_OF_RANGE);
-        mbar_arrive(bar);
-      }
-    }
-  };
-
-  const int pre = min(n_my, kStages);
-  for (int i = 0; i < pre; ++i) issue(i);
-  int issued = pre, consumed = 0;
-
+  // ---- page stream -------------------------------------------------------------
   float o[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.0f;
   float m_run = -INFINITY, l_run = 0.0f, zs_run = 0.0f;
   bool ok = true;
+  int consumed = 0;
 
   for (int i = 0; i < n_my; ++i) {
     const int st = i % kStages;
-    const bool waited = mbar_wait_bounded(bar0 + st * 8, (i / kStages) & 1);
+    const bool waited = mbar_wait_bounded(bar0 + 8 * st, (i / kStages) & 1);
     if (!__all_sync(FULL, waited)) { ok = false; break; }
     consumed = i + 1;
     const uint8_t* stg = ring + st * S::kStageBytes;
-    const bool valid = wflags[st] != 0;
-    const int page_base = (my_first + i * kAttnWarps) * 16;
-    const uint8_t* kb = stg;
-    const uint8_t* vb = stg + 8 * D;
-    const __half2* sk2 = reinterpret_cast<const __half2*>(stg + S::kCodeBytes);
-    const __half2* sv2 = sk2 + 8;
-    const __half2* zk2 = reinterpret_cast<const __half2*>(stg + S::kCodeBytes + 64);
-    const __half2* zv2 = zk2 + 8;
+    const int fl = wflags[st];
+    const int tok0 = (p_begin + 2 * (warp + kAttnWarps * i)) * 16;  // first token of the task
 
-    // QK on the codes: token rows g and 8 + g
-    float acc[2][4];
+    // QK on the codes: n-tile nt = token rows 8(nt&1) + g of page nt>>1
+    float acc[4][4];
 #pragma unroll
-    for (int nt = 0; nt < 2; ++nt) {
+    for (int nt = 0; nt < 4; ++nt) {
       acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
-      const uint8_t* row = kb + (8 * nt + g) * (D / 2) + tig * (4 * W);
-      uint32_t wk[W];
-      if constexpr (W == 4) {
-        const uint4 t4 = *reinterpret_cast<const uint4*>(row);
-        wk[0] = t4.x; wk[1] = t4.y; wk[2] = t4.z; wk[3] = t4.w;
-      } else {
-        const uint2 t2 = *reinterpret_cast<const uint2*>(row);
-        wk[0] = t2.x; wk[1] = t2.y;
-      }
+      if ((fl >> (nt >> 1)) & 1) {
+        const uint8_t* row = stg + (nt >> 1) * S::kPageBytes + (8 * (nt & 1) + g) * (D / 2) + tig * (4 * W);
+        uint32_t wk[W];
+        if constexpr (W == 4) {
+          const uint4 t4 = *reinterpret_cast<const uint4*>(row);
+          wk[0] = t4.x; wk[1] = t4.y; wk[2] = t4.z; wk[3] = t4.w;
+        } else {
+          const uint2 t2 = *reinterpret_cast<const uint2*>(row);
+          wk[0] = t2.x; wk[1] = t2.y;
+        }
 #pragma unroll
-      for (int u = 0; u < W; ++u) {
-        const uint32_t w = wk[u], w8 = wk[u] >> 8;
-        mma_f16_16816(acc[nt], aq[2 * u], codes_to_half2<false>(w), codes_to_half2<false>(w8));
-        mma_f16_16816(acc[nt], aq[2 * u + 1], codes_to_half2<true>(w), codes_to_half2<true>(w8));
+        for (int u = 0; u < W; ++u) {
+          const uint32_t w = wk[u], w8 = wk[u] >> 8;
+          mma_f16_16816(acc[nt], aq[2 * u], codes_to_half2<false>(w), codes_to_half2<false>(w8));
+          mma_f16_16816(acc[nt], aq[2 * u + 1], codes_to_half2<true>(w), codes_to_half2<true>(w8));
+        }
       }
     }
 
-    // logits (base 2) of this thread's tokens 2tig, 2tig+1, 2tig+8, 2tig+9
-    const float2 skA = __half22float2(sk2[tig]), skB = __half22float2(sk2[tig + 4]);
-    const float2 zkA = __half22float2(zk2[tig]), zkB = __half22float2(zk2[tig + 4]);
-    const int t0 = page_base + 2 * tig;
-    float lg[4];
-    lg[0] = fmaf((acc[0][0] + acc[0][2]) * acc_to_true, skA.x, zkA.x * qsum);
-    lg[1] = fmaf((acc[0][1] + acc[0][3]) * acc_to_true, skA.y, zkA.y * qsum);
-    lg[2] = fmaf((acc[1][0] + acc[1][2]) * acc_to_true, skB.x, zkB.x * qsum);
-    lg[3] = fmaf((acc[1][1] + acc[1][3]) * acc_to_true, skB.y, zkB.y * qsum);
-    if (!valid || t0 >= ctx) lg[0] = -INFINITY;
-    if (!valid || t0 + 1 >= ctx) lg[1] = -INFINITY;
-    if (!valid || t0 + 8 >= ctx) lg[2] = -INFINITY;
-    if (!valid || t0 + 9 >= ctx) lg[3] = -INFINITY;
+    // logits (base 2) of this thread's 8 tokens: 8nt + 2tig + {0, 1}
+    float lg[8];
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const uint8_t* sz = stg + (nt >> 1) * S::kPageBytes + S::kCodeBytes;
+      const int i2 = 4 * (nt & 1) + tig;  // half2 index of tokens 8(nt&1) + 2tig, +1
+      const float2 sk = __half22float2(reinterpret_cast<const __half2*>(sz)[i2]);
+      const float2 zk = __half22float2(reinterpret_cast<const __half2*>(sz + 64)[i2]);
+      lg[2 * nt] = fmaf((acc[nt][0] + acc[nt][2]) * acc_to_true, sk.x, zk.x * qsum);
+      lg[2 * nt + 1] = fmaf((acc[nt][1] + acc[nt][3]) * acc_to_true, sk.y, zk.y * qsum);
+      const int t = tok0 + 8 * nt + 2 * tig;
+      const bool vp = (fl >> (nt >> 1)) & 1;
+      if (!vp || t >= ctx) lg[2 * nt] = -INFINITY;
+      if (!vp || t + 1 >= ctx) lg[2 * nt + 1] = -INFINITY;
+    }
 
     // online softmax, rescaling only when the running maximum grows
-    float pm = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
+    float pm = fmaxf(fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3])),
+                     fmaxf(fmaxf(lg[4], lg[5]), fmaxf(lg[6], lg[7])));
     pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 1));
     pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 2));
     if (pm > m_run) {
-      const float alpha = exp2f(m_run - pm);
+      const float alpha = fast_exp2(m_run - pm);
 #pragma unroll
       for (int nt = 0; nt < NT; ++nt) {
         o[nt][0] *= alpha; o[nt][1] *= alpha; o[nt][2] *= alpha; o[nt][3] *= alpha;
@@ -290,44 +330,54 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnP
       zs_run *= alpha;
       m_run = pm;
     }
-    const float2 svA = __half22float2(sv2[tig]), svB = __half22float2(sv2[tig + 4]);
-    const float2 zvA = __half22float2(zv2[tig]), zvB = __half22float2(zv2[tig + 4]);
-    const float sv[4] = {svA.x, svA.y, svB.x, svB.y};
-    const float zv[4] = {zvA.x, zvA.y, zvB.x, zvB.y};
-    __half ph[4], pl[4];
+    float pv[8];
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const float pr = (lg[j] == -INFINITY) ? 0.0f : exp2f(lg[j] - m_run);
-      l_run += pr;
-      const float pv = (pr > 0.0f) ? pr * sv[j] : 0.0f;
-      zs_run += (pr > 0.0f) ? pr * zv[j] : 0.0f;
-      split_half(pv, ph[j], pl[j]);
+    for (int nt = 0; nt < 4; ++nt) {
+      const uint8_t* sz = stg + (nt >> 1) * S::kPageBytes + S::kCodeBytes;
+      const int i2 = 4 * (nt & 1) + tig;
+      const float2 sv = __half22float2(reinterpret_cast<const __half2*>(sz + 32)[i2]);
+      const float2 zv = __half22float2(reinterpret_cast<const __half2*>(sz + 96)[i2]);
+      const float p0 = (lg[2 * nt] == -INFINITY) ? 0.0f : fast_exp2(lg[2 * nt] - m_run);
+      const float p1 = (lg[2 * nt + 1] == -INFINITY) ? 0.0f : fast_exp2(lg[2 * nt + 1] - m_run);
+      l_run += p0 + p1;
+      pv[2 * nt] = (p0 > 0.0f) ? p0 * sv.x : 0.0f;
+      pv[2 * nt + 1] = (p1 > 0.0f) ? p1 * sv.y : 0.0f;
+      zs_run += ((p0 > 0.0f) ? p0 * zv.x : 0.0f) + ((p1 > 0.0f) ? p1 * zv.y : 0.0f);
     }
-    const uint32_t ap[4] = {pack_half2(ph[0], ph[1]), pack_half2(pl[0], pl[1]),
-                            pack_half2(ph[2], ph[3]), pack_half2(pl[2], pl[3])};
 
-    // PV on the codes: thread group g supplies channels [g*NT, g*NT + NT)
-    uint32_t wv[4][WP];
-    const int rows_v[4] = {2 * tig, 2 * tig + 1, 2 * tig + 8, 2 * tig + 9};
+    // PV on the codes, one k-step per page: A = (p*s_v) hi/lo rows for this
+    // thread's tokens, B = code pairs of token rows (2tig, 2tig+1), (2tig+8,
+    // 2tig+9); thread group g supplies channels [g*NT, g*NT + NT)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const uint8_t* row = vb + rows_v[j] * (D / 2) + g * (4 * WP);
-      if constexpr (WP == 2) {
-        const uint2 t2 = *reinterpret_cast<const uint2*>(row);
-        wv[j][0] = t2.x; wv[j][1] = t2.y;
-      } else {
-        wv[j][0] = *reinterpret_cast<const uint32_t*>(row);
-      }
-    }
+    for (int pg = 0; pg < 2; ++pg) {
+      if ((fl >> pg) & 1) {
+        uint32_t ap[4];
+        split_pair(pv[4 * pg], pv[4 * pg + 1], ap[0], ap[1]);
+        split_pair(pv[4 * pg + 2], pv[4 * pg + 3], ap[2], ap[3]);
+        const uint8_t* vb = stg + pg * S::kPageBytes + 8 * D;
+        uint32_t wv[4][WP];
+        const int rows_v[4] = {2 * tig, 2 * tig + 1, 2 * tig + 8, 2 * tig + 9};
 #pragma unroll
-    for (int u = 0; u < WP; ++u) {
+        for (int j = 0; j < 4; ++j) {
+          const uint8_t* row = vb + rows_v[j] * (D / 2) + g * (4 * WP);
+          if constexpr (WP == 2) {
+            const uint2 t2 = *reinterpret_cast<const uint2*>(row);
+            wv[j][0] = t2.x; wv[j][1] = t2.y;
+          } else {
+            wv[j][0] = *reinterpret_cast<const uint32_t*>(row);
+          }
+        }
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const uint32_t sel = k | (k << 4) | ((4 + k) << 8) | ((4 + k) << 12);
-        const uint32_t x01 = prmt(wv[0][u], wv[1][u], sel);
-        const uint32_t x23 = prmt(wv[2][u], wv[3][u], sel);
-        mma_f16_16816(o[8 * u + 2 * k], ap, codes_to_half2<false>(x01), codes_to_half2<false>(x23));
-        mma_f16_16816(o[8 * u + 2 * k + 1], ap, codes_to_half2<true>(x01), codes_to_half2<true>(x23));
+        for (int u = 0; u < WP; ++u) {
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t sel = k | (k << 4) | ((4 + k) << 8) | ((4 + k) << 12);
+            const uint32_t x01 = prmt(wv[0][u], wv[1][u], sel);
+            const uint32_t x23 = prmt(wv[2][u], wv[3][u], sel);
+            mma_f16_16816(o[8 * u + 2 * k], ap, codes_to_half2<false>(x01), codes_to_half2<false>(x23));
+            mma_f16_16816(o[8 * u + 2 * k + 1], ap, codes_to_half2<true>(x01), codes_to_half2<true>(x23));
+          }
+        }
       }
     }
     __syncwarp();
@@ -335,10 +385,10 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnP
   }
   if (!ok) {
     // a copy never completed: give the ones still outstanding a bounded wait
-    for (int i = consumed; i < issued; ++i) mbar_wait_bounded(bar0 + (i % kStages) * 8, (i / kStages) & 1);
+    for (int i = consumed; i < issued; ++i) mbar_wait_bounded(bar0 + 8 * (i % kStages), (i / kStages) & 1);
   }
 
-  // ---- merge the four warps ------------------------------------------------
+  // ---- merge the four warps into the CTA's (M, L, O + Z) per head --------------
   l_run += __shfl_xor_sync(FULL, l_run, 1);
   l_run += __shfl_xor_sync(FULL, l_run, 2);
   zs_run += __shfl_xor_sync(FULL, zs_run, 1);
@@ -362,9 +412,6 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnP
     }
   }
   __syncthreads();
-  float* part = nullptr;
-  if (p.n_splits > 1)
-    part = p.ws_part + ((((size_t)n * p.Hkv + h) * p.n_splits + split) * G) * (D + 2);
   for (int idx = tid; idx < G * D; idx += kAttnThreads) {
     const int r = idx / D, c = idx % D;
     float M = -INFINITY;
@@ -377,89 +424,146 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnP
         const float* mw = mrg + w * S::kMergeFloatsPerWarp;
         const float mwr = mw[8 * D + r];
         if (mwr == -INFINITY) continue;
-        const float e = exp2f(mwr - M);
+        const float e = fast_exp2(mwr - M);
         O += mw[r * D + c] * e;
         L += mw[8 * D + 8 + r] * e;
         Z += mw[8 * D + 16 + r] * e;
       }
     }
-    if (p.n_splits == 1) {
-      qs[r * D + c] = (L > 0.0f) ? (O + Z) / L : 0.0f;
-    } else {
-      part[r * (D + 2) + c] = O + Z;
-      if (c == 0) {
-        part[r * (D + 2) + D] = M;
-        part[r * (D + 2) + D + 1] = L;
-      }
+    qs[idx] = O + Z;
+    if (c == 0) {
+      cml[2 * r] = M;
+      cml[2 * r + 1] = L;
     }
   }
+  __syncthreads();
 
-  // ---- merge the splits: the last CTA of this (sequence, kv head) ----------
-  if (p.n_splits > 1) {
+  // ---- merge the cluster's CTAs into its first CTA (distributed smem) --------
+  const int cs = p.cluster_size;
+  if (cs > 1) {
+    constexpr int kPer = (8 * D + kAttnThreads - 1) / kAttnThreads;
+    float keepO[kPer], keepM[kPer], keepL[kPer];
+    cluster_sync_all();  // every CTA's merged result is in its shared memory
+    const uint32_t rank = cluster_ctarank();
+    if (rank == 0) {
+#pragma unroll
+      for (int k = 0; k < kPer; ++k) {
+        const int idx = tid + k * kAttnThreads;
+        keepO[k] = keepM[k] = keepL[k] = 0.0f;
+        if (idx < G * D) {
+          const int r = idx / D;
+          float M = -INFINITY;
+          for (int q = 0; q < cs; ++q) M = fmaxf(M, ld_dsmem_f32(&cml[2 * r], q));
+          float O = 0.0f, L = 0.0f;
+          if (M != -INFINITY) {
+            for (int q = 0; q < cs; ++q) {
+              const float mq = ld_dsmem_f32(&cml[2 * r], q);
+              if (mq == -INFINITY) continue;
+              const float e = fast_exp2(mq - M);
+              O += e * ld_dsmem_f32(&qs[idx], q);
+              L += e * ld_dsmem_f32(&cml[2 * r + 1], q);
+            }
+          }
+          keepO[k] = O;
+          keepM[k] = M;
+          keepL[k] = L;
+        }
+      }
+    }
+    cluster_sync_all();  // the first CTA has read every CTA's shared memory
+    if (rank != 0) return;
+#pragma unroll
+    for (int k = 0; k < kPer; ++k) {
+      const int idx = tid + k * kAttnThreads;
+      if (idx < G * D) {
+        qs[idx] = keepO[k];
+        if (idx % D == 0) {
+          cml[2 * (idx / D)] = keepM[k];
+          cml[2 * (idx / D) + 1] = keepL[k];
+        }
+      }
+    }
+    __syncthreads();
+  }
+
+  if (p.n_parts == 1) {
+    for (int idx = tid; idx < G * D; idx += kAttnThreads) {
+      const float L = cml[2 * (idx / D) + 1];
+      qs[idx] = (L > 0.0f) ? qs[idx] / L : 0.0f;
+    }
+  } else {
+    // ---- several clusters per (sequence, kv head): meet in the workspace -----
+    const int part = split / cs;
+    const int np = p.n_parts;
+    float* base = p.ws_part + (((size_t)n * p.Hkv + h) * np) * G * (D + 2);
+    float* dst = base + (size_t)part * G * (D + 2);
+    for (int idx = tid; idx < G * D; idx += kAttnThreads) {
+      const int r = idx / D, c = idx % D;
+      dst[r * (D + 2) + c] = qs[idx];
+      if (c == 0) {
+        dst[r * (D + 2) + D] = cml[2 * r];
+        dst[r * (D + 2) + D + 1] = cml[2 * r + 1];
+      }
+    }
     __threadfence();
     __syncthreads();
     int* s_last = flags + kAttnWarps * kStages;
     if (tid == 0) {
       const int prev = atomicAdd(&p.ws_count[(size_t)n * p.Hkv + h], 1);
-      *s_last = (prev == p.n_splits - 1);
+      *s_last = (prev == np - 1);
     }
     __syncthreads();
     if (!*s_last) return;
     __threadfence();
-    const float* base = p.ws_part + (((size_t)n * p.Hkv + h) * p.n_splits) * G * (D + 2);
-    const int ns = p.n_splits;
-    float* lsp = wts + 8 * kMaxSplits;   // per (head, split) sums
-    float* Lr = wts + 16 * kMaxSplits;   // per head total
-    // every (head, split) maximum and sum, loaded in parallel
-    for (int idx = tid; idx < G * ns; idx += kAttnThreads) {
+    float* lsp = wts + 8 * kMaxParts;  // per (head, part) sums
+    float* Lr = wts + 16 * kMaxParts;  // per head total
+    for (int idx = tid; idx < G * np; idx += kAttnThreads) {
       const int r = idx % G, s = idx / G;
       const float* src = base + ((size_t)s * G + r) * (D + 2) + D;
-      wts[r * kMaxSplits + s] = __ldcg(src);
-      lsp[r * kMaxSplits + s] = __ldcg(src + 1);
+      wts[r * kMaxParts + s] = __ldcg(src);
+      lsp[r * kMaxParts + s] = __ldcg(src + 1);
     }
     __syncthreads();
-    // per head: the global maximum, the split weights and the total sum (one warp per head)
     for (int r = warp; r < G; r += kAttnWarps) {
       float M = -INFINITY;
-      for (int s = lane; s < ns; s += 32) M = fmaxf(M, wts[r * kMaxSplits + s]);
+      for (int s = lane; s < np; s += 32) M = fmaxf(M, wts[r * kMaxParts + s]);
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o));
+      for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o2));
       float L = 0.0f;
-      for (int s = lane; s < ns; s += 32) {
-        const float ms = wts[r * kMaxSplits + s];
-        const float e = (ms == -INFINITY) ? 0.0f : exp2f(ms - M);
-        wts[r * kMaxSplits + s] = e;
-        L += e * lsp[r * kMaxSplits + s];
+      for (int s = lane; s < np; s += 32) {
+        const float ms = wts[r * kMaxParts + s];
+        const float e = (ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
+        wts[r * kMaxParts + s] = e;
+        L += e * lsp[r * kMaxParts + s];
       }
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(FULL, L, o);
+      for (int o2 = 16; o2 > 0; o2 >>= 1) L += __shfl_xor_sync(FULL, L, o2);
       if (lane == 0) Lr[r] = L;
     }
     __syncthreads();
-    // weighted sum over splits; independent loads, several in flight
     for (int idx = tid; idx < G * D; idx += kAttnThreads) {
       const int r = idx / D, c = idx % D;
       const float* src = base + (size_t)r * (D + 2) + c;
       const size_t stride = (size_t)G * (D + 2);
-      float acc0 = 0.0f, acc1 = 0.0f, acc2 = 0.0f, acc3 = 0.0f;
+      float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
       int s = 0;
-      for (; s + 4 <= ns; s += 4) {
+      for (; s + 4 <= np; s += 4) {
         const float v0 = __ldcg(src + (size_t)s * stride), v1 = __ldcg(src + (size_t)(s + 1) * stride);
         const float v2 = __ldcg(src + (size_t)(s + 2) * stride), v3 = __ldcg(src + (size_t)(s + 3) * stride);
-        acc0 = fmaf(wts[r * kMaxSplits + s], v0, acc0);
-        acc1 = fmaf(wts[r * kMaxSplits + s + 1], v1, acc1);
-        acc2 = fmaf(wts[r * kMaxSplits + s + 2], v2, acc2);
-        acc3 = fmaf(wts[r * kMaxSplits + s + 3], v3, acc3);
+        a0 = fmaf(wts[r * kMaxParts + s], v0, a0);
+        a1 = fmaf(wts[r * kMaxParts + s + 1], v1, a1);
+        a2 = fmaf(wts[r * kMaxParts + s + 2], v2, a2);
+        a3 = fmaf(wts[r * kMaxParts + s + 3], v3, a3);
       }
-      for (; s < ns; ++s) acc0 = fmaf(wts[r * kMaxSplits + s], __ldcg(src + (size_t)s * stride), acc0);
-      const float acc = (acc0 + acc1) + (acc2 + acc3);
-      qs[r * D + c] = (Lr[r] > 0.0f) ? acc / Lr[r] : 0.0f;
+      for (; s < np; ++s) a0 = fmaf(wts[r * kMaxParts + s], __ldcg(src + (size_t)s * stride), a0);
+      const float acc = (a0 + a1) + (a2 + a3);
+      qs[idx] = (Lr[r] > 0.0f) ? acc / Lr[r] : 0.0f;
     }
-    if (tid == 0) p.ws_count[(size_t)n * p.Hkv + h] = 0;  // leave the workspace zeroed
+    if (tid == 0) p.ws_count[(size_t)n * p.Hkv + h] = 0;  // leave the tickets at zero
   }
   __syncthreads();
 
-  // ---- out = R o_rot ---------------------------------------------------------
+  // ---- out = R o_rot -------------------------------------------------------------
   if constexpr (BLK > 0) smem_fwht_rows<D, BLK>(qs, G);
   for (int idx = tid; idx < G * D; idx += kAttnThreads) {
     const int r = idx / D, c = idx % D;

@@ -9,8 +9,10 @@
 // block, the row min/max and the packing stay in the thread's registers - no
 // shuffles. Input rows arrive through cp.async into a per-warp shared buffer
 // with an XOR swizzle on 16-byte chunks (conflict-free row reads); the copy of
-// tile i+1 is issued before tile i is computed. Packed rows (D/2 bytes) and
-// the fp16 s, z go straight to their slot.
+// tile i+1 is issued before tile i is computed. The arithmetic runs on packed
+// fp32 pairs (sm_100 f32x2: one issue slot per two lanes) where it can:
+// butterflies, the 1/sqrt(b) scaling, y - z and the rounding fma. Packed rows
+// (D/2 bytes) and the fp16 s, z go straight to their slot.
 #pragma once
 
 #include "kvq_device.cuh"
@@ -38,20 +40,29 @@ __host__ __device__ constexpr int write_smem_bytes() {
   return kWriteWarps * 32 * D * 2;
 }
 
-// In-register fast Walsh-Hadamard transform of each contiguous BLK block
-// (Sylvester natural order: y_i = sum_j (-1)^popcount(i&j) x_j).
+// In-register fast Walsh-Hadamard transform of each contiguous BLK block of a
+// row held as D/2 packed pairs (x[2i], x[2i+1]); Sylvester natural order:
+// y_i = sum_j (-1)^popcount(i&j) x_j. The distance-1 stage pairs the two
+// halves of one register (scalar ops); every other stage pairs whole
+// registers (f32x2 add/sub).
 template <int D, int BLK>
-__device__ __forceinline__ void fwht_blocks(float (&x)[D]) {
+__device__ __forceinline__ void fwht_pairs(uint64_t (&xp)[D / 2]) {
 #pragma unroll
-  for (int base = 0; base < D; base += BLK) {
+  for (int i = 0; i < D / 2; ++i) {
+    float a, b;
+    f2_unpack(xp[i], a, b);
+    xp[i] = f2_pack(__fadd_rn(a, b), __fsub_rn(a, b));
+  }
 #pragma unroll
-    for (int len = 1; len < BLK; len <<= 1) {
+  for (int base = 0; base < D / 2; base += BLK / 2) {
 #pragma unroll
-      for (int i = 0; i < BLK; ++i) {
+    for (int len = 1; len < BLK / 2; len <<= 1) {
+#pragma unroll
+      for (int i = 0; i < BLK / 2; ++i) {
         if ((i & len) == 0) {
-          const float a = x[base + i], b = x[base + i + len];
-          x[base + i] = __fadd_rn(a, b);
-          x[base + i + len] = __fsub_rn(a, b);
+          const uint64_t A = xp[base + i], B = xp[base + i + len];
+          xp[base + i] = f2_add(A, B);
+          xp[base + i + len] = f2_sub(A, B);
         }
       }
     }
@@ -62,6 +73,7 @@ template <int D, int BLK>
 __global__ void __launch_bounds__(kWriteWarps * 32, 3) kvq_write_kernel(const WriteParams p) {
   constexpr int ROWB = D * 2;       // bytes per bf16 input row
   constexpr int CPR = ROWB / 16;    // 16-byte chunks per row (8 or 16)
+  constexpr int RPI = 32 / CPR;     // rows covered by one warp-wide copy instruction
   extern __shared__ __align__(128) uint8_t smem[];
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
@@ -69,24 +81,25 @@ __global__ void __launch_bounds__(kWriteWarps * 32, 3) kvq_write_kernel(const Wr
   const uint32_t wbuf_s = smem_addr(wbuf);
   const int nw = gridDim.x * kWriteWarps;
   int tile = blockIdx.x * kWriteWarps + warp;
+  const size_t row_stride = (size_t)p.Hkv * D;  // elements between consecutive tokens
+  const int lrow = lane / CPR, lchunk = lane % CPR;
 
   auto issue = [&](int tl) {
     const int kv = tl & 1;
     const int h = (tl >> 1) % p.Hkv;
     const int tb = (tl >> 1) / p.Hkv;
-    const uint16_t* src = kv ? p.v : p.k;
+    const uint16_t* src = (kv ? p.v : p.k) + ((size_t)(tb * 32 + lrow) * p.Hkv + h) * D + lchunk * 8;
 #pragma unroll
     for (int j = 0; j < CPR; ++j) {
-      const int idx = j * 32 + lane;
-      const int r = idx / CPR, c = idx % CPR;
-      const int t = tb * 32 + r;
-      if (t < p.T) {
-        const uint16_t* g = src + ((size_t)t * p.Hkv + h) * D + c * 8;
-        cp_async_16(wbuf_s + r * ROWB + ((c ^ (r & (CPR - 1))) * 16), g);
-      }
+      const int r = j * RPI + lrow;
+      if (tb * 32 + r < p.T)
+        cp_async_16(wbuf_s + r * ROWB + ((lchunk ^ (r & (CPR - 1))) * 16), src + (size_t)j * RPI * row_stride);
     }
     cp_async_commit();
   };
+
+  const uint64_t cb2 = f2_pack(p.cb, p.cb);
+  const uint64_t magic2 = f2_pack(8388608.0f, 8388608.0f);
 
   if (tile < p.num_tiles) issue(tile);
   for (; tile < p.num_tiles; tile += nw) {
@@ -98,36 +111,44 @@ __global__ void __launch_bounds__(kWriteWarps * 32, 3) kvq_write_kernel(const Wr
 
     cp_async_wait_all();
     __syncwarp();
-    float x[D];
+    uint64_t xp[D / 2];
 #pragma unroll
     for (int c = 0; c < CPR; ++c) {
       const uint4 u = *reinterpret_cast<const uint4*>(wbuf + lane * ROWB + ((c ^ (lane & (CPR - 1))) * 16));
       const uint32_t w[4] = {u.x, u.y, u.z, u.w};
 #pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        x[c * 8 + 2 * e] = __uint_as_float(w[e] << 16);
-        x[c * 8 + 2 * e + 1] = __uint_as_float(w[e] & 0xffff0000u);
-      }
+      for (int e = 0; e < 4; ++e)
+        xp[c * 4 + e] = f2_pack(__uint_as_float(w[e] << 16), __uint_as_float(w[e] & 0xffff0000u));
     }
     __syncwarp();
     if (tile + nw < p.num_tiles) issue(tile + nw);
 
     // 1. rotation y = (H_b x) * fp32(1/sqrt(b))
     if constexpr (BLK > 0) {
-      fwht_blocks<D, BLK>(x);
+      fwht_pairs<D, BLK>(xp);
 #pragma unroll
-      for (int c = 0; c < D; ++c) x[c] = __fmul_rn(x[c], p.cb);
+      for (int i = 0; i < D / 2; ++i) xp[i] = f2_mul(xp[i], cb2);
     }
-    // 2. row min / max
-    float mn = x[0], mx = x[0];
+    // 2. row min / max (four independent 3-input chains each)
+    float mn4[4], mx4[4];
 #pragma unroll
-    for (int c = 1; c < D; ++c) {
-      mn = fminf(mn, x[c]);
-      mx = fmaxf(mx, x[c]);
+    for (int q = 0; q < 4; ++q) {
+      float a, b;
+      f2_unpack(xp[q * (D / 8)], a, b);
+      mn4[q] = fminf(a, b);
+      mx4[q] = fmaxf(a, b);
+#pragma unroll
+      for (int i = q * (D / 8) + 1; i < (q + 1) * (D / 8); ++i) {
+        f2_unpack(xp[i], a, b);
+        mn4[q] = fmin3(mn4[q], a, b);
+        mx4[q] = fmax3(mx4[q], a, b);
+      }
     }
+    const float mn = fminf(fminf(mn4[0], mn4[1]), fminf(mn4[2], mn4[3]));
+    const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
     // 3. z = largest fp16 <= mn; s = smallest fp16 with 15 s + z >= mx.
-    //    Directed roundings give a candidate at most one fp16 step above the
-    //    smallest; the exact test (fp64: 15 s + z is exact there) settles it.
+    //    Directed roundings give a candidate at most one fp16 step high; the
+    //    exact test (fp64: 15 s + z is exact there) settles it.
     const __half zh = __float2half_rd(mn);
     const float zf = __half2float(zh);
     const float need = __fdiv_ru(__fsub_ru(mx, zf), 15.0f);
@@ -140,16 +161,24 @@ __global__ void __launch_bounds__(kWriteWarps * 32, 3) kvq_write_kernel(const Wr
     const float sf = __half2float(__ushort_as_half(sb));
     const float inv = (sf > 0.0f) ? __frcp_rn(sf) : 0.0f;
     // 4. code = rint(fp32(y - z) * fp32(1/s)): adding 2^23 inside one fma
-    //    rounds the exact product to an integer (ties to even); the code is
-    //    then the low bits of the result.
+    //    rounds the exact product to an integer (ties to even), leaving the
+    //    code in the low 4 bits of the result (above them: the constant
+    //    exponent of 2^23). Eight such words shifted by 4i and summed give the
+    //    packed word plus a known constant, removed by starting the sum at its
+    //    negation.
+    const uint64_t z2 = f2_pack(zf, zf);
+    const uint64_t inv2 = f2_pack(inv, inv);
     uint32_t packed[D / 8];
 #pragma unroll
     for (int wd = 0; wd < D / 8; ++wd) {
-      uint32_t acc = 0;
+      uint32_t acc = 0x05000000u;  // -(0x4B000000 + (0x4B000000 << 4)) mod 2^32
 #pragma unroll
-      for (int i = 0; i < 8; ++i) {
-        const float tq = __fmaf_rn(__fsub_rn(x[wd * 8 + i], zf), inv, 8388608.0f);
-        acc |= (__float_as_uint(tq) & 0xFu) << (4 * i);
+      for (int i = 0; i < 4; ++i) {
+        const uint64_t f = f2_fma(f2_sub(xp[wd * 4 + i], z2), inv2, magic2);
+        float lo, hi;
+        f2_unpack(f, lo, hi);
+        acc += __float_as_uint(lo) << (8 * i);
+        acc += __float_as_uint(hi) << (8 * i + 4);
       }
       packed[wd] = acc;
     }

@@ -122,9 +122,11 @@ kvq_status kv_quant_write(const void* k, const void* v, const int64_t* slot_mapp
 
 /*
  * kvq_attn_workspace_size - bytes of device workspace paged_decode_attn_int4
- * needs for these shapes (0 when the call needs none). The value depends on
- * the shapes and on the current device's SM count only. Returns SIZE_MAX when
- * the shapes are invalid or no device can be queried.
+ * needs for these shapes (0 when the call needs none) on this library's
+ * current device (see kvq_set_device). The value depends on the shapes and on
+ * how many thread-block clusters of the decode kernel that device holds at
+ * once. Returns SIZE_MAX when the shapes are invalid or no device can be
+ * queried.
  *
  * Layout: the first round_up(batch*num_kv_heads*4, 256) bytes are the split
  * tickets (int32 counters), the rest holds per-split partial results.
@@ -206,6 +208,14 @@ kvq_status paged_decode_attn_int4_static_ws(const void* q, const uint8_t* cache,
  * Returns KVQ_ERR_CUDA if the synchronization itself fails.
  */
 kvq_status kvq_get_device_error(void* stream);
+
+/*
+ * kvq_set_device - make `device` this library's current CUDA device (the
+ * device kvq_attn_workspace_size plans for). The other calls select the
+ * device that owns their cache buffer by themselves. Returns KVQ_OK,
+ * KVQ_ERR_INVALID_ARG for a negative ordinal, or KVQ_ERR_CUDA.
+ */
+kvq_status kvq_set_device(int32_t device);
 
 /* Static, human-readable name of a status value (never NULL). */
 const char* kvq_status_string(int32_t status);

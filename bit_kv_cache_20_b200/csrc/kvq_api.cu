@@ -127,28 +127,41 @@ kvq_status dispatch_write(const kvq::WriteParams& p, int b, int dev, cudaStream_
 // paged_decode_attn_int4
 // ---------------------------------------------------------------------------
 struct SplitPlan {
-  int n_splits;         // CTAs per (sequence, kv head)
+  int n_splits;         // CTAs per (sequence, kv-head group)
   int pages_per_split;
   int cluster;          // CTAs per thread-block cluster (divides n_splits)
-  int n_parts;          // clusters per (sequence, kv head) = partials in the workspace
+  int n_parts;          // clusters per (sequence, kv-head group) = partials in the workspace
+  int hg;               // kv heads per CTA
 };
 
+// kv heads served by one CTA: 4, 2 or 1, whichever largest divides Hkv.
+int heads_per_cta(int Hkv) { return (Hkv % 4 == 0) ? 4 : (Hkv % 2 == 0) ? 2 : 1; }
+
+int inst_slot(int D, int b, int hg) {
+  const int bi = (b == 0) ? 0 : (b == 32) ? 1 : (b == 64) ? 2 : 3;
+  const int hi = (hg == 4) ? 2 : (hg == 2) ? 1 : 0;
+  return ((D == 64) ? 0 : 12) + bi * 3 + hi;
+}
+constexpr int kInstSlots = 24;
+
 template <int D, int BLK>
-const void* decode_kernel_ptr() {
-  return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK>);
+const void* decode_kernel_ptr(int hg) {
+  if (hg == 4) return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK, 4>);
+  if (hg == 2) return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK, 2>);
+  return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK, 1>);
 }
 
-const void* decode_kernel_for(int D, int b) {
+const void* decode_kernel_for(int D, int b, int hg) {
   if (D == 64) {
-    if (b == 0) return decode_kernel_ptr<64, 0>();
-    if (b == 32) return decode_kernel_ptr<64, 32>();
-    if (b == 64) return decode_kernel_ptr<64, 64>();
+    if (b == 0) return decode_kernel_ptr<64, 0>(hg);
+    if (b == 32) return decode_kernel_ptr<64, 32>(hg);
+    if (b == 64) return decode_kernel_ptr<64, 64>(hg);
     return nullptr;
   }
-  if (b == 0) return decode_kernel_ptr<128, 0>();
-  if (b == 32) return decode_kernel_ptr<128, 32>();
-  if (b == 64) return decode_kernel_ptr<128, 64>();
-  if (b == 128) return decode_kernel_ptr<128, 128>();
+  if (b == 0) return decode_kernel_ptr<128, 0>(hg);
+  if (b == 32) return decode_kernel_ptr<128, 32>(hg);
+  if (b == 64) return decode_kernel_ptr<128, 64>(hg);
+  if (b == 128) return decode_kernel_ptr<128, 128>(hg);
   return nullptr;
 }
 
@@ -158,11 +171,11 @@ int decode_smem_bytes(int D) {
 
 // Opt the decode kernel instance into its dynamic shared memory (once per
 // device and instance).
-bool prepare_decode_kernel(int dev, int D, int b) {
-  static std::atomic<int> done[kMaxDevices][8];
-  const int slot = (D == 64 ? 0 : 4) + (b == 0 ? 0 : b == 32 ? 1 : b == 64 ? 2 : 3);
+bool prepare_decode_kernel(int dev, int D, int b, int hg) {
+  static std::atomic<int> done[kMaxDevices][kInstSlots];
+  const int slot = inst_slot(D, b, hg);
   if (done[dev][slot].load(std::memory_order_relaxed)) return true;
-  const void* k = decode_kernel_for(D, b);
+  const void* k = decode_kernel_for(D, b, hg);
   if (!k || cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, decode_smem_bytes(D)) !=
                 cudaSuccess) {
     cudaGetLastError();
@@ -173,12 +186,12 @@ bool prepare_decode_kernel(int dev, int D, int b) {
 }
 
 // Clusters of `cs` decode CTAs that can be resident at once on the device.
-int max_active_clusters(int dev, int D, int b, int cs) {
-  static std::atomic<int> cache[kMaxDevices][8][kvq::kMaxCluster + 1];
-  const int slot = (D == 64 ? 0 : 4) + (b == 0 ? 0 : b == 32 ? 1 : b == 64 ? 2 : 3);
+int max_active_clusters(int dev, int D, int b, int hg, int cs) {
+  static std::atomic<int> cache[kMaxDevices][kInstSlots][kvq::kMaxCluster + 1];
+  const int slot = inst_slot(D, b, hg);
   int v = cache[dev][slot][cs].load(std::memory_order_relaxed);
   if (v > 0) return v;
-  if (!prepare_decode_kernel(dev, D, b)) return 0;
+  if (!prepare_decode_kernel(dev, D, b, hg)) return 0;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(cs, 1, 1);
   cfg.blockDim = dim3(kvq::kAttnThreads, 1, 1);
@@ -191,7 +204,7 @@ int max_active_clusters(int dev, int D, int b, int cs) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel_for(D, b), &cfg) != cudaSuccess || n < 1) {
+  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel_for(D, b, hg), &cfg) != cudaSuccess || n < 1) {
     cudaGetLastError();
     return 0;
   }
@@ -199,30 +212,32 @@ int max_active_clusters(int dev, int D, int b, int cs) {
   return n;
 }
 
-// Split each (sequence, kv head) into CTAs grouped in thread-block clusters
-// (which merge on chip), choosing the cluster size and split count so that
-// every CTA of the launch is resident at once (one wave, as the occupancy API
-// reports for clusters of that size) and each split keeps at least 8 pages.
-// Only when a (sequence, kv head) has more than one cluster do partial
-// results go through the workspace.
+// Split each (sequence, kv-head group) into CTAs grouped in thread-block
+// clusters (which merge on chip), choosing the cluster size and the split
+// count so that every CTA of the launch is resident at once (one wave, as the
+// occupancy API reports for clusters of that size) and each split keeps at
+// least 8 pages. Larger clusters are preferred (fewer partial results); a
+// smaller one must buy more than 10 % more splits. Only with more than one
+// cluster per (sequence, head group) do partial results go through the
+// workspace and a combine kernel.
 SplitPlan plan_splits(const kvq_attn_desc* d, int dev) {
-  const long long units = (long long)d->batch * d->num_kv_heads;
+  const int hg = heads_per_cta(d->num_kv_heads);
+  const long long units = (long long)d->batch * (d->num_kv_heads / hg);
   long long cap = d->max_pages_per_seq / 8;
   if (cap < 1) cap = 1;
   if (cap > kvq::kMaxSplits) cap = kvq::kMaxSplits;
-  SplitPlan best = {1, d->max_pages_per_seq, 1, 1};
+  SplitPlan best = {1, d->max_pages_per_seq, 1, 1, hg};
   if (units <= 0 || cap == 1) return best;
   for (int cs = kvq::kMaxCluster; cs >= 1; --cs) {
-    const int mac = max_active_clusters(dev, d->head_dim, d->hadamard_block, cs);
-    const long long per_unit = mac / units;  // clusters per (sequence, kv head) in one wave
+    const int mac = max_active_clusters(dev, d->head_dim, d->hadamard_block, hg, cs);
+    const long long per_unit = mac / units;  // clusters per (sequence, head group) in one wave
     if (per_unit < 1) continue;
     long long parts = per_unit;
     if (parts > cap / cs) parts = cap / cs;
     if (parts > kvq::kMaxParts) parts = kvq::kMaxParts;
     if (parts < 1) continue;
     const long long ns = parts * cs;
-    // larger clusters are tried first; a smaller one must buy > 10 % more splits
-    if (ns * 10 > best.n_splits * 11LL) best = {(int)ns, 0, cs, (int)parts};
+    if (ns * 10 > best.n_splits * 11LL) best = {(int)ns, 0, cs, (int)parts, hg};
   }
   best.pages_per_split = (d->max_pages_per_seq + best.n_splits - 1) / best.n_splits;
   return best;
@@ -247,23 +262,18 @@ kvq_status check_attn_desc(const kvq_attn_desc* d) {
 
 size_t workspace_bytes_for(const kvq_attn_desc* d, const SplitPlan& plan) {
   if (plan.n_parts <= 1 || d->batch == 0) return 0;
-  const size_t units = (size_t)d->batch * d->num_kv_heads;
-  const size_t counters = ((units * sizeof(int) + 255) / 256) * 256;
   const size_t G = (size_t)(d->num_q_heads / d->num_kv_heads);
-  return counters + units * plan.n_parts * G * (d->head_dim + 2) * sizeof(float);
+  return (size_t)d->batch * d->num_kv_heads * plan.n_parts * G * (d->head_dim + 2) * sizeof(float);
 }
 
 template <int D, int BLK>
-kvq_status launch_attn(const kvq::AttnParams& p, int dev, cudaStream_t s) {
-  auto kern = kvq::kvq_decode_kernel<D, BLK>;
-  constexpr int smem = kvq::AttnSmem<D>::kTotal;
-  static_assert(3 * (smem + 1024) <= 228 * 1024, "three decode CTAs must fit on one SM");
+kvq_status launch_attn(const kvq::AttnParams& p, int hg, int dev, cudaStream_t s) {
   if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
-  if (!prepare_decode_kernel(dev, D, BLK)) return KVQ_ERR_CUDA;
+  if (!prepare_decode_kernel(dev, D, BLK, hg)) return KVQ_ERR_CUDA;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.n_splits, p.Hkv, p.B);
+  cfg.gridDim = dim3(p.n_splits, p.Hkv / hg, p.B);
   cfg.blockDim = dim3(kvq::kAttnThreads, 1, 1);
-  cfg.dynamicSmemBytes = smem;
+  cfg.dynamicSmemBytes = kvq::AttnSmem<D>::kTotal;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
@@ -272,21 +282,43 @@ kvq_status launch_attn(const kvq::AttnParams& p, int dev, cudaStream_t s) {
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) {
+  cudaError_t e;
+  if (hg == 4) e = cudaLaunchKernelEx(&cfg, kvq::kvq_decode_kernel<D, BLK, 4>, p);
+  else if (hg == 2) e = cudaLaunchKernelEx(&cfg, kvq::kvq_decode_kernel<D, BLK, 2>, p);
+  else e = cudaLaunchKernelEx(&cfg, kvq::kvq_decode_kernel<D, BLK, 1>, p);
+  if (e != cudaSuccess) {
     cudaGetLastError();
     return KVQ_ERR_CUDA;
+  }
+  if (p.n_parts > 1) {
+    // merge the clusters' partial results; launched as a programmatic
+    // dependent so its CTAs are scheduled while the main grid drains
+    cudaLaunchConfig_t c2 = {};
+    c2.gridDim = dim3(p.G, p.Hkv, p.B);
+    c2.blockDim = dim3(D, 1, 1);
+    c2.dynamicSmemBytes = 0;
+    c2.stream = s;
+    cudaLaunchAttribute a2[1];
+    a2[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    a2[0].val.programmaticStreamSerializationAllowed = 1;
+    c2.attrs = a2;
+    c2.numAttrs = 1;
+    if (cudaLaunchKernelEx(&c2, kvq::kvq_decode_combine_kernel<D, BLK>, p) != cudaSuccess) {
+      cudaGetLastError();
+      return KVQ_ERR_CUDA;
+    }
   }
   return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
 template <int D>
-kvq_status dispatch_attn(const kvq::AttnParams& p, int b, int dev, cudaStream_t s) {
+kvq_status dispatch_attn(const kvq::AttnParams& p, int b, int hg, int dev, cudaStream_t s) {
   switch (b) {
-    case 0: return launch_attn<D, 0>(p, dev, s);
-    case 32: return launch_attn<D, 32>(p, dev, s);
-    case 64: return launch_attn<D, 64>(p, dev, s);
+    case 0: return launch_attn<D, 0>(p, hg, dev, s);
+    case 32: return launch_attn<D, 32>(p, hg, dev, s);
+    case 64: return launch_attn<D, 64>(p, hg, dev, s);
     case 128:
-      if constexpr (D >= 128) return launch_attn<D, 128>(p, dev, s);
+      if constexpr (D >= 128) return launch_attn<D, 128>(p, hg, dev, s);
       return KVQ_ERR_UNSUPPORTED;
     default: return KVQ_ERR_UNSUPPORTED;
   }
@@ -354,7 +386,7 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const voi
   if (d.batch == 0) return KVQ_OK;  // nothing to do; pointers may be NULL
   if (!q || !cache || !scales || !zeros || !page_table || !context_lens || !out)
     return KVQ_ERR_INVALID_ARG;
-  if (!aligned(cache, 16) || !aligned(scales, 16) || !aligned(zeros, 16) || !aligned(q, 2) ||
+  if (!aligned(cache, 16) || !aligned(scales, 16) || !aligned(zeros, 16) || !aligned(q, 16) ||
       !aligned(page_table, 4) || !aligned(context_lens, 4) || !aligned(out, d.out_dtype ? 2 : 4))
     return KVQ_ERR_INVALID_ARG;
   int dev = 0;
@@ -383,23 +415,15 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const voi
   p.pages_per_split = plan.pages_per_split;
   p.cluster_size = plan.cluster;
   p.n_parts = plan.n_parts;
+  p.ws_part = need > 0 ? static_cast<float*>(workspace) : nullptr;
   p.out_bf16 = d.out_dtype;
   const double cb = d.hadamard_block > 0 ? 1.0 / std::sqrt((double)d.hadamard_block) : 1.0;
   const double scale = d.softmax_scale > 0.0f ? (double)d.softmax_scale : 1.0 / std::sqrt((double)d.head_dim);
   p.qmul = (float)(cb * scale * 1.4426950408889634);  // log2(e)
   p.cb = (float)cb;
-  if (need > 0) {
-    const size_t units = (size_t)d.batch * d.num_kv_heads;
-    const size_t counters = ((units * sizeof(int) + 255) / 256) * 256;
-    p.ws_count = static_cast<int*>(workspace);
-    p.ws_part = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + counters);
-  } else {
-    p.ws_count = nullptr;
-    p.ws_part = nullptr;
-  }
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d.head_dim == 64 ? dispatch_attn<64>(p, d.hadamard_block, dev, s)
-                          : dispatch_attn<128>(p, d.hadamard_block, dev, s);
+  return d.head_dim == 64 ? dispatch_attn<64>(p, d.hadamard_block, plan.hg, dev, s)
+                          : dispatch_attn<128>(p, d.hadamard_block, plan.hg, dev, s);
 }
 
 kvq_status kvq_get_device_error(void* stream) {
@@ -492,14 +516,6 @@ extern "C" kvq_status paged_decode_attn_int4_static_ws(const void* q, const uint
   if (need > 0) {
     st = static_workspace_on(dev, &ws);
     if (st != KVQ_OK) return st;
-    // the split tickets must start at zero; a call that stopped early could
-    // have left some of them set
-    const size_t units = (size_t)desc->batch * desc->num_kv_heads;
-    const size_t tickets = ((units * sizeof(int) + 255) / 256) * 256;
-    if (cudaMemsetAsync(ws, 0, tickets, static_cast<cudaStream_t>(stream)) != cudaSuccess) {
-      cudaGetLastError();
-      return KVQ_ERR_CUDA;
-    }
   }
   return paged_decode_attn_int4(q, cache, scales, zeros, page_table, context_lens, out, ws,
                                 need > 0 ? (size_t)KVQ_STATIC_WORKSPACE_BYTES : 0, desc, stream);

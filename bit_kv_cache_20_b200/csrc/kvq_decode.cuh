@@ -5,34 +5,38 @@
 // rotates q once, runs attention in the rotated space directly on the codes,
 // and rotates the output back: out = R sum_t p_t v^_t.
 //
-// Grid (split, kv head, sequence), 4 warps per CTA; the splits of one
-// (sequence, kv head) form thread-block clusters of up to 8 CTAs.
-//  - Each warp walks its tasks (a task = two consecutive pages of the CTA's
-//    page range) through a private ring of 1-D bulk copies (TMA engine)
-//    completing on mbarriers: 16*D code bytes (K block, V block) + 64 B
-//    scales + 64 B zeros per page. The first copies are issued before q is
-//    rotated, so the rotation overlaps them.
-//  - Per task, on the tensor cores (mma.m16n8k16, f16 in, f32 accumulate):
-//      QK: S[16 rows x 32 tokens] = Qhl[16 x D] * codes^T   (4 n-tiles)
-//      PV: O[16 rows x D]        += Phl[16 x 32 tokens] * codes (2 k-steps)
-//    A rows 0..7 carry the fp16 "hi" part of up to 8 query heads and rows
-//    8..15 the "lo" remainder (x = hi + lo keeps ~22 bits), so one MMA does
-//    both halves and a GQA group of up to 8 shares one K/V stream.
-//    The 4-bit codes enter as exact normal fp16 values c (or 16c for a nibble
-//    at bits 4..7, compensated by 1/16 on the other operand or in the
-//    epilogue). Subnormal fp16 operands are avoided on purpose: small
-//    products built from them lost precision in the tensor-core accumulation
-//    (a systematic bias of ~2^-13 relative, measured on B200).
-//    Dequantization is folded into per-token scalars:
-//      logit_t = s_t * (q~ . code_t) + z_t * sum(q~)
-//      o_rot   = (sum_t p_t s_t code_t + sum_t p_t z_t) / sum_t p_t
-//    Online softmax in base 2 (log2 e folded into q~), rescaling only when
-//    the running maximum grows.
-//  - Warps merge in shared memory; the CTAs of a cluster merge through
-//    distributed shared memory into the cluster's first CTA; when a
-//    (sequence, kv head) has several clusters, their partial results meet in
-//    the workspace and the last cluster to arrive (atomic ticket) combines
-//    them. The final CTA applies the inverse rotation and stores.
+// Grid (split, kv-head group, sequence), 4 warps per CTA. A CTA serves HG kv
+// heads (HG = 4, 2 or 1, dividing Hkv); warp w works for head w % HG. Because
+// the cache is laid out [page][kv head][K|V][token][D/2], the HG heads of one
+// page are one contiguous block: each page costs the CTA three 1-D bulk
+// copies (TMA engine) - HG*16*D code bytes, HG*64 B of scales, HG*64 B of
+// zeros - into a CTA-wide ring of stages (a stage = two pages), completing on
+// one mbarrier per stage. The last warp done with a stage refills it.
+//
+// Per page, on the tensor cores (mma.m16n8k16, f16 in, f32 accumulate):
+//   QK: S[16 rows x 16 tokens] = Qhl[16 x D] * codes^T
+//   PV: O[16 rows x D]        += Phl[16 x 16 tokens] * codes
+// A rows 0..7 carry the fp16 "hi" part of up to 8 query heads (the GQA group)
+// and rows 8..15 the "lo" remainder (x = hi + lo keeps ~22 bits), so one MMA
+// does both halves. The 4-bit codes enter as exact normal fp16 values c (or
+// 16c for a nibble at bits 4..7, compensated by 1/16 on the other operand or
+// in the epilogue); subnormal fp16 operands are avoided on purpose - small
+// products built from them lost precision in the tensor-core accumulation (a
+// systematic bias of ~2^-13 relative, measured on B200). Dequantization is
+// folded into per-token scalars:
+//   logit_t = s_t * (q~ . code_t) + z_t * sum(q~)
+//   o_rot   = (sum_t p_t s_t code_t + sum_t p_t z_t) / sum_t p_t
+// with an online softmax in base 2 (log2 e folded into q~) that rescales only
+// when the running maximum grows. q is rotated and the output rotated back in
+// registers: each thread holds a contiguous D/4-channel slice of one query
+// row, and the butterfly stages that cross slices use warp shuffles.
+//
+// The splits of one (sequence, head group) form thread-block clusters (up to
+// 8 CTAs) that merge through distributed shared memory into the cluster's
+// first CTA. With one cluster per (sequence, head group) that CTA writes the
+// output; otherwise each cluster writes a partial result to the workspace and
+// kvq_decode_combine_kernel (chained by programmatic dependent launch) merges
+// them and rotates back.
 #pragma once
 
 #include <climits>
@@ -49,8 +53,7 @@ struct AttnParams {
   const int32_t* page_table;  // [B][max_pages]
   const int32_t* ctx_lens;    // [B]
   void* out;                  // [B][Hq][D] fp32 or bf16
-  float* ws_part;             // [B][Hkv][n_parts][G][D + 2]
-  int* ws_count;              // [B][Hkv]
+  float* ws_part;             // [B][Hkv][n_parts][G][D + 2]: O + Z, then M, L
   int B, Hq, Hkv, G;
   int num_pages, max_pages;
   int n_splits, pages_per_split;
@@ -63,49 +66,53 @@ struct AttnParams {
 
 constexpr int kAttnWarps = 4;
 constexpr int kAttnThreads = kAttnWarps * 32;
-constexpr int kStages = 3;       // ring depth per warp, in tasks of two pages
 constexpr int kMaxSplits = 256;
-constexpr int kMaxParts = 64;    // partial results per (sequence, kv head) in the workspace
+constexpr int kMaxParts = 64;
 constexpr int kMaxCluster = 8;
+constexpr int kMaxPids = 1024;   // page ids of a CTA's range kept in shared memory
 
 template <int D>
 struct AttnSmem {
-  static constexpr int kCodeBytes = 16 * D;               // K block + V block of one page-head
-  static constexpr int kPageBytes = kCodeBytes + 128;     // + 32 scales + 32 zeros (fp16)
-  static constexpr int kStageBytes = 2 * kPageBytes;      // one task = two pages
-  static constexpr int kRingBytes = kAttnWarps * kStages * kStageBytes;
-  // per-warp merge area (overlays the ring after the page loop)
-  static constexpr int kMergeFloatsPerWarp = 8 * D + 3 * 8;
-  static constexpr int kMergeBytes = kAttnWarps * kMergeFloatsPerWarp * 4;
-  static constexpr int kUnionBytes = kRingBytes > kMergeBytes ? kRingBytes : kMergeBytes;
-  static constexpr int kQBytes = 8 * D * 4;               // q rows, then the CTA's merged O
-  static constexpr int kMLBytes = 8 * 2 * 4;              // the CTA's merged (M, L) per head
-  static constexpr int kWeightBytes = (2 * 8 * kMaxParts + 8) * 4;
-  static constexpr int kBarBytes = kAttnWarps * kStages * 8;
-  static constexpr int kFlagBytes = kAttnWarps * kStages * 4 + 16;
-  static constexpr int kOffQ = kUnionBytes;
-  static constexpr int kOffML = kOffQ + kQBytes;
-  static constexpr int kOffW = kOffML + kMLBytes;
-  static constexpr int kOffBar = kOffW + kWeightBytes;
-  static constexpr int kOffFlag = kOffBar + kBarBytes;
-  static constexpr int kTotal = kOffFlag + kFlagBytes;
+  static constexpr int kHeadPageBytes = 16 * D + 128;       // codes + 32 scales + 32 zeros
+  static constexpr int kRingBytes = 24 * kHeadPageBytes;    // 12/HG stages of 2 pages x HG heads
+  // per-warp result slot (overlays the ring once every copy has landed):
+  // O[8 rows][D], then (m, l, zs, unused) per row
+  static constexpr int kSlotFloats = 8 * D + 8 * 4;
+  static constexpr int kSlotBytes = kAttnWarps * kSlotFloats * 4;
+  static constexpr int kUnionBytes = kRingBytes > kSlotBytes ? kRingBytes : kSlotBytes;
+  static constexpr int kOffPid = kUnionBytes;
+  static constexpr int kOffBar = kOffPid + kMaxPids * 4;
+  static constexpr int kOffCnt = kOffBar + 12 * 8;
+  static constexpr int kOffFlag = kOffCnt + 12 * 4;
+  static constexpr int kTotal = kOffFlag + 12 * 4;
 };
 
-// In-place FWHT of rows [0, nrows) of an fp32 [8][D] shared array, blocks of
-// BLK channels; the whole CTA takes part.
-template <int D, int BLK>
-__device__ __forceinline__ void smem_fwht_rows(float* rows, int nrows) {
-#pragma unroll 1
-  for (int len = 1; len < BLK; len <<= 1) {
-    for (int idx = threadIdx.x; idx < nrows * (D / 2); idx += kAttnThreads) {
-      const int r = idx / (D / 2), pi = idx % (D / 2);
-      const int i = (pi / len) * (2 * len) + (pi % len);
-      float* row = rows + r * D;
-      const float a = row[i], b = row[i + len];
-      row[i] = a + b;
-      row[i + len] = a - b;
+// Fast Walsh-Hadamard transform (blocks of BLK, Sylvester natural order) of a
+// row spread over the 4 lanes of a quad: lane tig holds channels
+// [C*tig, C*tig + C). Stages shorter than C stay in the thread; the longer
+// ones pair lanes tig and tig ^ (len / C).
+template <int C, int BLK>
+__device__ __forceinline__ void quad_fwht(float (&v)[C], int tig) {
+#pragma unroll
+  for (int len = 1; len < C && len < BLK; len <<= 1) {
+#pragma unroll
+    for (int i = 0; i < C; ++i) {
+      if ((i & len) == 0) {
+        const float a = v[i], b = v[i + len];
+        v[i] = a + b;
+        v[i + len] = a - b;
+      }
     }
-    __syncthreads();
+  }
+#pragma unroll
+  for (int len = C; len < BLK; len <<= 1) {
+    const int m = len / C;
+    const bool upper = (tig & m) != 0;
+#pragma unroll
+    for (int i = 0; i < C; ++i) {
+      const float other = __shfl_xor_sync(0xffffffffu, v[i], m);
+      v[i] = upper ? (other - v[i]) : (v[i] + other);
+    }
   }
 }
 
@@ -118,25 +125,102 @@ __device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uin
   lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
+__device__ __forceinline__ void store_out(const AttnParams& p, size_t idx, float v) {
+  if (p.out_bf16)
+    reinterpret_cast<__nv_bfloat16*>(p.out)[idx] = __float2bfloat16_rn(v);
+  else
+    reinterpret_cast<float*>(p.out)[idx] = v;
+}
+
+// Merge of the n_parts partial results of one (sequence, kv head, query row)
+// and inverse rotation. Grid (G, Hkv, B), D threads (one per channel).
 template <int D, int BLK>
+__global__ void __launch_bounds__(D) kvq_decode_combine_kernel(const AttnParams p) {
+  __shared__ float sm_m[kMaxParts], sm_w[kMaxParts], sm_row[D];
+  __shared__ float sm_L;
+  asm volatile("griddepcontrol.wait;\n" ::: "memory");  // the partials are complete
+  const int r = blockIdx.x, h = blockIdx.y, n = blockIdx.z, c = threadIdx.x;
+  const int np = p.n_parts, G = p.G;
+  const size_t stride = (size_t)G * (D + 2);
+  const float* base = p.ws_part + (((size_t)n * p.Hkv + h) * np * G + r) * (D + 2);
+  for (int s = c; s < np; s += D) {
+    sm_m[s] = __ldcg(base + s * stride + D);
+    sm_w[s] = __ldcg(base + s * stride + D + 1);
+  }
+  __syncthreads();
+  if (c < 32) {
+    float M = -INFINITY;
+    for (int s = c; s < np; s += 32) M = fmaxf(M, sm_m[s]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    float L = 0.0f;
+    for (int s = c; s < np; s += 32) {
+      const float e = (sm_m[s] == -INFINITY) ? 0.0f : fast_exp2(sm_m[s] - M);
+      L += e * sm_w[s];
+      sm_w[s] = e;
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
+    if (c == 0) sm_L = L;
+  }
+  __syncthreads();
+  // all partials of this channel in flight at once, 16 at a time
+  float acc = 0.0f;
+  for (int s0 = 0; s0 < np; s0 += 16) {
+    float v[16];
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = (s0 + j < np) ? __ldcg(base + (size_t)(s0 + j) * stride + c) : 0.0f;
+#pragma unroll
+    for (int j = 0; j < 16; ++j)
+      if (s0 + j < np) acc = fmaf(sm_w[s0 + j], v[j], acc);
+  }
+  sm_row[c] = (sm_L > 0.0f) ? acc / sm_L : 0.0f;
+  __syncthreads();
+  if constexpr (BLK > 0) {
+#pragma unroll 1
+    for (int len = 1; len < BLK; len <<= 1) {
+      float v = 0.0f;
+      if ((c & len) == 0) v = sm_row[c] + sm_row[c + len];
+      else v = sm_row[c - len] - sm_row[c];
+      __syncthreads();
+      sm_row[c] = v;
+      __syncthreads();
+    }
+  }
+  const float val = (BLK > 0) ? sm_row[c] * p.cb : sm_row[c];
+  store_out(p, ((size_t)n * p.Hq + (size_t)h * G + r) * D + c, val);
+}
+
+template <int D, int BLK, int HG>
 __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnParams p) {
   using S = AttnSmem<D>;
-  constexpr int W = D / 32;   // code words of one token row per thread (QK)
-  constexpr int KS = D / 16;  // QK k-steps
-  constexpr int WP = D / 64;  // code words of one token row per thread group (PV)
-  constexpr int NT = D / 8;   // PV n-tiles
+  constexpr int W = D / 32;    // code words of one token row per thread (QK)
+  constexpr int WP = D / 64;   // code words of one token row per thread group (PV)
+  constexpr int NT = D / 8;    // PV n-tiles
+  constexpr int KS = D / 16;   // QK k-steps
+  constexpr int C = D / 4;     // channels of one query row per thread
+  constexpr int NSUB = kAttnWarps / HG;  // warps per head
+  constexpr int NST = 12 / HG;           // ring stages (a multiple of NSUB)
+  constexpr int HPB = S::kHeadPageBytes;
+  constexpr int PGB = HG * HPB;          // one page of HG heads
+  constexpr int STB = 2 * PGB;           // one stage = two pages
+  static_assert(NST * STB == S::kRingBytes, "ring size");
   extern __shared__ __align__(128) uint8_t smem[];
-  float* qs = reinterpret_cast<float*>(smem + S::kOffQ);
-  float* cml = reinterpret_cast<float*>(smem + S::kOffML);
-  float* wts = reinterpret_cast<float*>(smem + S::kOffW);
+  int* pids = reinterpret_cast<int*>(smem + S::kOffPid);
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kOffBar);
-  int* flags = reinterpret_cast<int*>(smem + S::kOffFlag);
+  int* cnt = reinterpret_cast<int*>(smem + S::kOffCnt);
+  int* sflags = reinterpret_cast<int*>(smem + S::kOffFlag);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tig = lane & 3;
-  const int split = blockIdx.x, h = blockIdx.y, n = blockIdx.z;
+  const int hw = warp % HG, sub = warp / HG;
+  const int split = blockIdx.x, hg = blockIdx.y, n = blockIdx.z;
+  const int h = hg * HG + hw;
   const int G = p.G;
   const unsigned FULL = 0xffffffffu;
+
+  // let a dependent combine kernel get scheduled early; it waits for this grid
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
 
   int ctx = p.ctx_lens[n];
   const int cap = p.max_pages * 16;
@@ -147,89 +231,79 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnP
   const int n_pages = (ctx + 15) >> 4;
   const int p_begin = split * p.pages_per_split;
   const int p_end = min(p_begin + p.pages_per_split, n_pages);
-  const int n_tasks = (p_end > p_begin) ? (p_end - p_begin + 1) / 2 : 0;
-  const int n_my = (n_tasks > warp) ? (n_tasks - warp + kAttnWarps - 1) / kAttnWarps : 0;
+  const int npg = max(p_end - p_begin, 0);
+  const int n_tasks = (npg + 1) / 2;
+  const int32_t* pt_row = p.page_table + (size_t)n * p.max_pages + p_begin;
 
-  uint8_t* ring = smem + warp * kStages * S::kStageBytes;
-  const uint32_t ring_s = smem_addr(ring);
-  const uint32_t bar0 = smem_addr(&bars[warp * kStages]);
-  int* wflags = flags + warp * kStages;
-  const int32_t* pt_row = p.page_table + (size_t)n * p.max_pages;
-
-  if (lane == 0) {
-    for (int s = 0; s < kStages; ++s) mbar_init(bar0 + 8 * s, 1);
+  for (int i = tid; i < npg && i < kMaxPids; i += kAttnThreads) pids[i] = pt_row[i];
+  if (tid == 0) {
+    for (int st = 0; st < NST; ++st) {
+      mbar_init(smem_addr(&bars[st]), 1);
+      cnt[st] = 0;
+    }
     mbar_init_fence();
   }
-  __syncwarp();
+  __syncthreads();
 
-  // ---- page ids of this warp's tasks, 32 tasks at a time ---------------------
-  // task i of this warp covers pages p_begin + 2*(warp + 4 i) and the next one;
-  // INT_MIN marks "no page" (past the split's range).
-  int pid_base = 0, pid_a = INT_MIN, pid_b = INT_MIN;
-  auto load_ids = [&](int base) {
-    const int i = base + lane;
-    const int pa = p_begin + 2 * (warp + kAttnWarps * i);
-    pid_a = (i < n_my && pa < p_end) ? pt_row[pa] : INT_MIN;
-    pid_b = (i < n_my && pa + 1 < p_end) ? pt_row[pa + 1] : INT_MIN;
-  };
-  load_ids(0);
-
-  // Issue the copies of task i into its ring stage (all lanes call; i grows by one).
-  auto issue = [&](int i) {
-    if (i - pid_base >= 32) {
-      pid_base += 32;
-      load_ids(pid_base);
+  // Fill stage t % NST with task t (pages 2t, 2t+1 of the range); one thread.
+  auto issue = [&](int t) {
+    const int st = t % NST;
+    const uint32_t bar = smem_addr(&bars[st]);
+    const uint32_t dst = smem_addr(smem + st * STB);
+    int ids[2];
+    bool ok[2];
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      const int i = 2 * t + j;
+      ids[j] = (i < npg) ? (i < kMaxPids ? pids[i] : pt_row[i]) : INT_MIN;
+      ok[j] = ids[j] >= 0 && ids[j] < p.num_pages;
+      if (ids[j] != INT_MIN && !ok[j]) record_error(KVQ_ERR_OUT_OF_RANGE);
     }
-    const int ia = __shfl_sync(FULL, pid_a, i - pid_base);
-    const int ib = __shfl_sync(FULL, pid_b, i - pid_base);
-    if (lane == 0) {
-      const int st = i % kStages;
-      const uint32_t bar = bar0 + 8 * st;
-      const uint32_t dst = ring_s + st * S::kStageBytes;
-      const bool va = ia >= 0 && ia < p.num_pages;
-      const bool vb = ib >= 0 && ib < p.num_pages;
-      if ((ia != INT_MIN && !va) || (ib != INT_MIN && !vb)) record_error(KVQ_ERR_OUT_OF_RANGE);
-      wflags[st] = (va ? 1 : 0) | (vb ? 2 : 0);
-      const uint32_t bytes = (va ? S::kPageBytes : 0) + (vb ? S::kPageBytes : 0);
-      if (bytes == 0) {
-        mbar_arrive(bar);
-      } else {
-        mbar_arrive_expect_tx(bar, bytes);
-        if (va) {
-          const size_t ph = (size_t)ia * p.Hkv + h;
-          bulk_g2s(dst, p.cache + ph * S::kCodeBytes, S::kCodeBytes, bar);
-          bulk_g2s(dst + S::kCodeBytes, p.scales + ph * 32, 64, bar);
-          bulk_g2s(dst + S::kCodeBytes + 64, p.zeros + ph * 32, 64, bar);
-        }
-        if (vb) {
-          const size_t ph = (size_t)ib * p.Hkv + h;
-          const uint32_t d1 = dst + S::kPageBytes;
-          bulk_g2s(d1, p.cache + ph * S::kCodeBytes, S::kCodeBytes, bar);
-          bulk_g2s(d1 + S::kCodeBytes, p.scales + ph * 32, 64, bar);
-          bulk_g2s(d1 + S::kCodeBytes + 64, p.zeros + ph * 32, 64, bar);
-        }
+    sflags[st] = (ok[0] ? 1 : 0) | (ok[1] ? 2 : 0);
+    const uint32_t bytes = (ok[0] ? PGB : 0) + (ok[1] ? PGB : 0);
+    if (bytes == 0) {
+      mbar_arrive(bar);
+      return;
+    }
+    mbar_arrive_expect_tx(bar, bytes);
+#pragma unroll
+    for (int j = 0; j < 2; ++j) {
+      if (!ok[j]) continue;
+      const size_t ph = (size_t)ids[j] * p.Hkv + (size_t)hg * HG;  // first page-head of the group
+      const uint32_t d = dst + j * PGB;
+      bulk_g2s(d, p.cache + ph * (16 * D), HG * 16 * D, bar);
+      bulk_g2s(d + HG * 16 * D, p.scales + ph * 32, HG * 64, bar);
+      bulk_g2s(d + HG * 16 * D + HG * 64, p.zeros + ph * 32, HG * 64, bar);
+    }
+  };
+  if (tid == 0)
+    for (int t = 0; t < NST && t < n_tasks; ++t) issue(t);
+
+  // ---- q~ = R q * (softmax_scale * log2 e), in registers -------------------
+  // Thread (g, tig) holds query row g (query head h*G + g) channels
+  // [C tig, C tig + C); rows >= G are zero.
+  float qv[C];
+  if (g < G) {
+    const uint4* src = reinterpret_cast<const uint4*>(p.q + ((size_t)n * p.Hq + (size_t)h * G + g) * D + C * tig);
+#pragma unroll
+    for (int i = 0; i < C / 8; ++i) {
+      const uint4 u = src[i];
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        qv[8 * i + 2 * e] = __uint_as_float(w4[e] << 16);
+        qv[8 * i + 2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
       }
     }
-  };
-
-  const int pre = min(n_my, kStages);
-  for (int i = 0; i < pre; ++i) issue(i);
-  int issued = pre;
-
-  // ---- q~ = R q * (softmax_scale * log2 e), rows >= G are zero --------------
-  for (int i = tid; i < 8 * D; i += kAttnThreads) {
-    const int r = i / D, c = i % D;
-    qs[i] = (r < G) ? bf16_bits_to_float(p.q[((size_t)n * p.Hq + (size_t)h * G + r) * D + c]) : 0.0f;
+  } else {
+#pragma unroll
+    for (int i = 0; i < C; ++i) qv[i] = 0.0f;
   }
-  __syncthreads();
-  if constexpr (BLK > 0) smem_fwht_rows<D, BLK>(qs, G);
-
-  // Thread (g, tig) holds head g's channels [8W tig, 8W tig + 8W).
-  float qv[8 * W];
+  if constexpr (BLK > 0) quad_fwht<C, BLK>(qv, tig);
   float amax = 0.0f, qsum = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 8 * W; ++i) {
-    qv[i] = qs[g * D + 8 * W * tig + i] * p.qmul;
+  for (int i = 0; i < C; ++i) {
+    qv[i] *= p.qmul;
     amax = fmaxf(amax, fabsf(qv[i]));
     qsum += qv[i];
   }
@@ -258,30 +332,34 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnP
     }
   }
 
-  // ---- page stream -------------------------------------------------------------
+  // ---- page stream: this warp takes tasks sub, sub + NSUB, ... -------------
   float o[NT][4];
 #pragma unroll
   for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.0f;
   float m_run = -INFINITY, l_run = 0.0f, zs_run = 0.0f;
-  bool ok = true;
-  int consumed = 0;
 
-  for (int i = 0; i < n_my; ++i) {
-    const int st = i % kStages;
-    const bool waited = mbar_wait_bounded(bar0 + 8 * st, (i / kStages) & 1);
-    if (!__all_sync(FULL, waited)) { ok = false; break; }
-    consumed = i + 1;
-    const uint8_t* stg = ring + st * S::kStageBytes;
-    const int fl = wflags[st];
-    const int tok0 = (p_begin + 2 * (warp + kAttnWarps * i)) * 16;  // first token of the task
+  for (int t = sub; t < n_tasks; t += NSUB) {
+    const int st = t % NST;
+    const bool waited = mbar_wait_bounded(smem_addr(&bars[st]), (t / NST) & 1);
+    if (!__all_sync(FULL, waited)) break;
+    const int fl = sflags[st];
+    const uint8_t* stg = smem + st * STB;
+    const int tok0 = (p_begin + 2 * t) * 16;  // first token of the task
 
-    // QK on the codes: n-tile nt = token rows 8(nt&1) + g of page nt>>1
-    float acc[4][4];
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
-      if ((fl >> (nt >> 1)) & 1) {
-        const uint8_t* row = stg + (nt >> 1) * S::kPageBytes + (8 * (nt & 1) + g) * (D / 2) + tig * (4 * W);
+    for (int pg = 0; pg < 2; ++pg) {
+      if (!((fl >> pg) & 1)) continue;
+      const uint8_t* kb = stg + pg * PGB + hw * (16 * D);              // K block, then V block
+      const uint8_t* sz = stg + pg * PGB + HG * 16 * D + hw * 64;      // 16 K then 16 V scales
+      const uint8_t* zz = stg + pg * PGB + HG * 16 * D + HG * 64 + hw * 64;
+      const int tp = tok0 + 16 * pg;
+
+      // QK on the codes: n-tile nt = token rows 8nt + g
+      float acc[2][4];
+#pragma unroll
+      for (int nt = 0; nt < 2; ++nt) {
+        acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
+        const uint8_t* row = kb + (8 * nt + g) * (D / 2) + tig * (4 * W);
         uint32_t wk[W];
         if constexpr (W == 4) {
           const uint4 t4 = *reinterpret_cast<const uint4*>(row);
@@ -297,282 +375,195 @@ __global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnP
           mma_f16_16816(acc[nt], aq[2 * u + 1], codes_to_half2<true>(w), codes_to_half2<true>(w8));
         }
       }
-    }
+      // logits (base 2) of tokens 2tig, 2tig+1 (nt 0) and 2tig+8, 2tig+9 (nt 1)
+      const float2 skA = __half22float2(reinterpret_cast<const __half2*>(sz)[tig]);
+      const float2 skB = __half22float2(reinterpret_cast<const __half2*>(sz)[tig + 4]);
+      const float2 zkA = __half22float2(reinterpret_cast<const __half2*>(zz)[tig]);
+      const float2 zkB = __half22float2(reinterpret_cast<const __half2*>(zz)[tig + 4]);
+      float lg[4];
+      lg[0] = fmaf((acc[0][0] + acc[0][2]) * acc_to_true, skA.x, zkA.x * qsum);
+      lg[1] = fmaf((acc[0][1] + acc[0][3]) * acc_to_true, skA.y, zkA.y * qsum);
+      lg[2] = fmaf((acc[1][0] + acc[1][2]) * acc_to_true, skB.x, zkB.x * qsum);
+      lg[3] = fmaf((acc[1][1] + acc[1][3]) * acc_to_true, skB.y, zkB.y * qsum);
+      const int t0 = tp + 2 * tig;
+      if (t0 >= ctx) lg[0] = -INFINITY;
+      if (t0 + 1 >= ctx) lg[1] = -INFINITY;
+      if (t0 + 8 >= ctx) lg[2] = -INFINITY;
+      if (t0 + 9 >= ctx) lg[3] = -INFINITY;
 
-    // logits (base 2) of this thread's 8 tokens: 8nt + 2tig + {0, 1}
-    float lg[8];
+      // online softmax, rescaling only when the running maximum grows
+      float pm = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
+      pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 1));
+      pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 2));
+      if (pm > m_run) {
+        const float alpha = fast_exp2(m_run - pm);
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      const uint8_t* sz = stg + (nt >> 1) * S::kPageBytes + S::kCodeBytes;
-      const int i2 = 4 * (nt & 1) + tig;  // half2 index of tokens 8(nt&1) + 2tig, +1
-      const float2 sk = __half22float2(reinterpret_cast<const __half2*>(sz)[i2]);
-      const float2 zk = __half22float2(reinterpret_cast<const __half2*>(sz + 64)[i2]);
-      lg[2 * nt] = fmaf((acc[nt][0] + acc[nt][2]) * acc_to_true, sk.x, zk.x * qsum);
-      lg[2 * nt + 1] = fmaf((acc[nt][1] + acc[nt][3]) * acc_to_true, sk.y, zk.y * qsum);
-      const int t = tok0 + 8 * nt + 2 * tig;
-      const bool vp = (fl >> (nt >> 1)) & 1;
-      if (!vp || t >= ctx) lg[2 * nt] = -INFINITY;
-      if (!vp || t + 1 >= ctx) lg[2 * nt + 1] = -INFINITY;
-    }
-
-    // online softmax, rescaling only when the running maximum grows
-    float pm = fmaxf(fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3])),
-                     fmaxf(fmaxf(lg[4], lg[5]), fmaxf(lg[6], lg[7])));
-    pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 1));
-    pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 2));
-    if (pm > m_run) {
-      const float alpha = fast_exp2(m_run - pm);
-#pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        o[nt][0] *= alpha; o[nt][1] *= alpha; o[nt][2] *= alpha; o[nt][3] *= alpha;
-      }
-      l_run *= alpha;
-      zs_run *= alpha;
-      m_run = pm;
-    }
-    float pv[8];
-#pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      const uint8_t* sz = stg + (nt >> 1) * S::kPageBytes + S::kCodeBytes;
-      const int i2 = 4 * (nt & 1) + tig;
-      const float2 sv = __half22float2(reinterpret_cast<const __half2*>(sz + 32)[i2]);
-      const float2 zv = __half22float2(reinterpret_cast<const __half2*>(sz + 96)[i2]);
-      const float p0 = (lg[2 * nt] == -INFINITY) ? 0.0f : fast_exp2(lg[2 * nt] - m_run);
-      const float p1 = (lg[2 * nt + 1] == -INFINITY) ? 0.0f : fast_exp2(lg[2 * nt + 1] - m_run);
-      l_run += p0 + p1;
-      pv[2 * nt] = (p0 > 0.0f) ? p0 * sv.x : 0.0f;
-      pv[2 * nt + 1] = (p1 > 0.0f) ? p1 * sv.y : 0.0f;
-      zs_run += ((p0 > 0.0f) ? p0 * zv.x : 0.0f) + ((p1 > 0.0f) ? p1 * zv.y : 0.0f);
-    }
-
-    // PV on the codes, one k-step per page: A = (p*s_v) hi/lo rows for this
-    // thread's tokens, B = code pairs of token rows (2tig, 2tig+1), (2tig+8,
-    // 2tig+9); thread group g supplies channels [g*NT, g*NT + NT)
-#pragma unroll
-    for (int pg = 0; pg < 2; ++pg) {
-      if ((fl >> pg) & 1) {
-        uint32_t ap[4];
-        split_pair(pv[4 * pg], pv[4 * pg + 1], ap[0], ap[1]);
-        split_pair(pv[4 * pg + 2], pv[4 * pg + 3], ap[2], ap[3]);
-        const uint8_t* vb = stg + pg * S::kPageBytes + 8 * D;
-        uint32_t wv[4][WP];
-        const int rows_v[4] = {2 * tig, 2 * tig + 1, 2 * tig + 8, 2 * tig + 9};
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          const uint8_t* row = vb + rows_v[j] * (D / 2) + g * (4 * WP);
-          if constexpr (WP == 2) {
-            const uint2 t2 = *reinterpret_cast<const uint2*>(row);
-            wv[j][0] = t2.x; wv[j][1] = t2.y;
-          } else {
-            wv[j][0] = *reinterpret_cast<const uint32_t*>(row);
-          }
+        for (int nt = 0; nt < NT; ++nt) {
+          o[nt][0] *= alpha; o[nt][1] *= alpha; o[nt][2] *= alpha; o[nt][3] *= alpha;
         }
+        l_run *= alpha;
+        zs_run *= alpha;
+        m_run = pm;
+      }
+      const float2 svA = __half22float2(reinterpret_cast<const __half2*>(sz + 32)[tig]);
+      const float2 svB = __half22float2(reinterpret_cast<const __half2*>(sz + 32)[tig + 4]);
+      const float2 zvA = __half22float2(reinterpret_cast<const __half2*>(zz + 32)[tig]);
+      const float2 zvB = __half22float2(reinterpret_cast<const __half2*>(zz + 32)[tig + 4]);
+      const float sv[4] = {svA.x, svA.y, svB.x, svB.y};
+      const float zv[4] = {zvA.x, zvA.y, zvB.x, zvB.y};
+      float pv[4];
 #pragma unroll
-        for (int u = 0; u < WP; ++u) {
+      for (int j = 0; j < 4; ++j) {
+        const float pr = (lg[j] == -INFINITY) ? 0.0f : fast_exp2(lg[j] - m_run);
+        l_run += pr;
+        pv[j] = (pr > 0.0f) ? pr * sv[j] : 0.0f;
+        zs_run += (pr > 0.0f) ? pr * zv[j] : 0.0f;
+      }
+      uint32_t ap[4];
+      split_pair(pv[0], pv[1], ap[0], ap[1]);
+      split_pair(pv[2], pv[3], ap[2], ap[3]);
+
+      // PV on the codes: B = code pairs of token rows (2tig, 2tig+1),
+      // (2tig+8, 2tig+9); thread group g supplies channels [g*NT, g*NT + NT)
+      const uint8_t* vb = kb + 8 * D;
+      uint32_t wv[4][WP];
+      const int rows_v[4] = {2 * tig, 2 * tig + 1, 2 * tig + 8, 2 * tig + 9};
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t sel = k | (k << 4) | ((4 + k) << 8) | ((4 + k) << 12);
-            const uint32_t x01 = prmt(wv[0][u], wv[1][u], sel);
-            const uint32_t x23 = prmt(wv[2][u], wv[3][u], sel);
-            mma_f16_16816(o[8 * u + 2 * k], ap, codes_to_half2<false>(x01), codes_to_half2<false>(x23));
-            mma_f16_16816(o[8 * u + 2 * k + 1], ap, codes_to_half2<true>(x01), codes_to_half2<true>(x23));
-          }
+      for (int j = 0; j < 4; ++j) {
+        const uint8_t* row = vb + rows_v[j] * (D / 2) + g * (4 * WP);
+        if constexpr (WP == 2) {
+          const uint2 t2 = *reinterpret_cast<const uint2*>(row);
+          wv[j][0] = t2.x; wv[j][1] = t2.y;
+        } else {
+          wv[j][0] = *reinterpret_cast<const uint32_t*>(row);
+        }
+      }
+#pragma unroll
+      for (int u = 0; u < WP; ++u) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const uint32_t sel = k | (k << 4) | ((4 + k) << 8) | ((4 + k) << 12);
+          const uint32_t x01 = prmt(wv[0][u], wv[1][u], sel);
+          const uint32_t x23 = prmt(wv[2][u], wv[3][u], sel);
+          mma_f16_16816(o[8 * u + 2 * k], ap, codes_to_half2<false>(x01), codes_to_half2<false>(x23));
+          mma_f16_16816(o[8 * u + 2 * k + 1], ap, codes_to_half2<true>(x01), codes_to_half2<true>(x23));
         }
       }
     }
+    // release the stage; the last of its HG consumer warps refills it
     __syncwarp();
-    if (issued < n_my) { issue(issued); ++issued; }
+    if (lane == 0) {
+      const int old = atomicAdd(&cnt[st], 1);
+      if (old == HG - 1) {
+        cnt[st] = 0;
+        if (t + NST < n_tasks) issue(t + NST);
+      }
+    }
   }
-  if (!ok) {
-    // a copy never completed: give the ones still outstanding a bounded wait
-    for (int i = consumed; i < issued; ++i) mbar_wait_bounded(bar0 + 8 * (i % kStages), (i / kStages) & 1);
-  }
+  // (a warp whose wait ran out stops early; the error word records it)
 
-  // ---- merge the four warps into the CTA's (M, L, O + Z) per head --------------
+  // ---- per-warp result: O slice of row g, (m, l, zs) -----------------------
   l_run += __shfl_xor_sync(FULL, l_run, 1);
   l_run += __shfl_xor_sync(FULL, l_run, 2);
   zs_run += __shfl_xor_sync(FULL, zs_run, 1);
   zs_run += __shfl_xor_sync(FULL, zs_run, 2);
-  __syncthreads();  // every warp is past its ring: the merge area may overlay it
-  float* mrg = reinterpret_cast<float*>(smem);
-  {
-    float* mw = mrg + warp * S::kMergeFloatsPerWarp;
-    if (g < G) {
+  float ov[C];
 #pragma unroll
-      for (int nt = 0; nt < NT; ++nt) {
-        const float sc = (nt & 1) ? 0.0625f : 1.0f;  // odd n-tiles carried 16c
-        mw[g * D + (2 * tig) * NT + nt] = (o[nt][0] + o[nt][2]) * sc;
-        mw[g * D + (2 * tig + 1) * NT + nt] = (o[nt][1] + o[nt][3]) * sc;
-      }
-      if (tig == 0) {
-        mw[8 * D + g] = m_run;
-        mw[8 * D + 8 + g] = l_run;
-        mw[8 * D + 16 + g] = zs_run;
-      }
-    }
+  for (int nt = 0; nt < NT; ++nt) {
+    const float sc = (nt & 1) ? 0.0625f : 1.0f;  // odd n-tiles carried 16c
+    ov[nt] = (o[nt][0] + o[nt][2]) * sc;          // channel C tig + nt
+    ov[NT + nt] = (o[nt][1] + o[nt][3]) * sc;     // channel C tig + NT + nt
   }
-  __syncthreads();
-  for (int idx = tid; idx < G * D; idx += kAttnThreads) {
-    const int r = idx / D, c = idx % D;
-    float M = -INFINITY;
-#pragma unroll
-    for (int w = 0; w < kAttnWarps; ++w) M = fmaxf(M, mrg[w * S::kMergeFloatsPerWarp + 8 * D + r]);
-    float O = 0.0f, L = 0.0f, Z = 0.0f;
-    if (M != -INFINITY) {
-#pragma unroll
-      for (int w = 0; w < kAttnWarps; ++w) {
-        const float* mw = mrg + w * S::kMergeFloatsPerWarp;
-        const float mwr = mw[8 * D + r];
-        if (mwr == -INFINITY) continue;
-        const float e = fast_exp2(mwr - M);
-        O += mw[r * D + c] * e;
-        L += mw[8 * D + 8 + r] * e;
-        Z += mw[8 * D + 16 + r] * e;
-      }
-    }
-    qs[idx] = O + Z;
-    if (c == 0) {
-      cml[2 * r] = M;
-      cml[2 * r + 1] = L;
-    }
-  }
-  __syncthreads();
 
-  // ---- merge the cluster's CTAs into its first CTA (distributed smem) --------
+  // Merge (m, l, zs, O) sources into this thread's registers.
+  auto merge_in = [&](float ms, float ls, float zss, const float* os) {
+    const float M = fmaxf(m_run, ms);
+    if (M == -INFINITY) return;
+    const float a = (m_run == -INFINITY) ? 0.0f : fast_exp2(m_run - M);
+    const float b = (ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
+#pragma unroll
+    for (int i = 0; i < C; ++i) ov[i] = ov[i] * a + os[i] * b;
+    l_run = l_run * a + ls * b;
+    zs_run = zs_run * a + zss * b;
+    m_run = M;
+  };
+
+  __syncthreads();  // every copy has landed and been consumed: slots may overlay the ring
+  float* slots = reinterpret_cast<float*>(smem);
+  auto put_local = [&](float* slot) {
+#pragma unroll
+    for (int i = 0; i < C; ++i) slot[g * D + C * tig + i] = ov[i];
+    if (tig == 0) {
+      slot[8 * D + 4 * g] = m_run;
+      slot[8 * D + 4 * g + 1] = l_run;
+      slot[8 * D + 4 * g + 2] = zs_run;
+    }
+  };
+  auto take = [&](const float* slot) {
+    float os[C];
+#pragma unroll
+    for (int i = 0; i < C; ++i) os[i] = slot[g * D + C * tig + i];
+    merge_in(slot[8 * D + 4 * g], slot[8 * D + 4 * g + 1], slot[8 * D + 4 * g + 2], os);
+  };
+  if constexpr (NSUB > 1) {
+    // warps that shared a head hand their results to warp hw
+    if (sub > 0) put_local(slots + warp * S::kSlotFloats);
+    __syncthreads();
+    if (sub == 0)
+      for (int j = 1; j < NSUB; ++j) take(slots + (hw + HG * j) * S::kSlotFloats);
+    __syncthreads();
+  }
   const int cs = p.cluster_size;
   if (cs > 1) {
-    constexpr int kPer = (8 * D + kAttnThreads - 1) / kAttnThreads;
-    float keepO[kPer], keepM[kPer], keepL[kPer];
-    cluster_sync_all();  // every CTA's merged result is in its shared memory
-    const uint32_t rank = cluster_ctarank();
-    if (rank == 0) {
+    // The cluster's CTAs merge into its first CTA along a binary tree: at
+    // level r, CTA rank + 2^r pushes its result into level-r buffer of CTA
+    // rank (remote shared-memory stores, fire and forget); after one cluster
+    // barrier the receiver merges it from its own shared memory.
+    constexpr int kPay = kAttnWarps * S::kSlotFloats;
+    static_assert(3 * kPay * 4 <= S::kUnionBytes, "three merge buffers must fit in the ring");
+    const int rank = (int)cluster_ctarank();
+    cluster_sync_all();  // every CTA of the cluster is past its page loop
+    int level = 0;
+    for (int stride = 1; stride < cs; stride <<= 1, ++level) {
+      float* buf = slots + level * kPay + hw * S::kSlotFloats;
+      const int rel = rank % (2 * stride);
+      if (rel == stride && sub == 0) {
+        const uint32_t to = (uint32_t)(rank - stride);
 #pragma unroll
-      for (int k = 0; k < kPer; ++k) {
-        const int idx = tid + k * kAttnThreads;
-        keepO[k] = keepM[k] = keepL[k] = 0.0f;
-        if (idx < G * D) {
-          const int r = idx / D;
-          float M = -INFINITY;
-          for (int q = 0; q < cs; ++q) M = fmaxf(M, ld_dsmem_f32(&cml[2 * r], q));
-          float O = 0.0f, L = 0.0f;
-          if (M != -INFINITY) {
-            for (int q = 0; q < cs; ++q) {
-              const float mq = ld_dsmem_f32(&cml[2 * r], q);
-              if (mq == -INFINITY) continue;
-              const float e = fast_exp2(mq - M);
-              O += e * ld_dsmem_f32(&qs[idx], q);
-              L += e * ld_dsmem_f32(&cml[2 * r + 1], q);
-            }
-          }
-          keepO[k] = O;
-          keepM[k] = M;
-          keepL[k] = L;
-        }
+        for (int i = 0; i < C; i += 4)
+          st_dsmem_v4(buf + g * D + C * tig + i, to, ov[i], ov[i + 1], ov[i + 2], ov[i + 3]);
+        if (tig == 0) st_dsmem_v4(buf + 8 * D + 4 * g, to, m_run, l_run, zs_run, 0.0f);
       }
+      cluster_sync_all();
+      if (rel == 0 && rank + stride < cs && sub == 0) take(buf);
     }
-    cluster_sync_all();  // the first CTA has read every CTA's shared memory
     if (rank != 0) return;
-#pragma unroll
-    for (int k = 0; k < kPer; ++k) {
-      const int idx = tid + k * kAttnThreads;
-      if (idx < G * D) {
-        qs[idx] = keepO[k];
-        if (idx % D == 0) {
-          cml[2 * (idx / D)] = keepM[k];
-          cml[2 * (idx / D) + 1] = keepL[k];
-        }
-      }
-    }
-    __syncthreads();
   }
+  if (sub != 0) return;
 
   if (p.n_parts == 1) {
-    for (int idx = tid; idx < G * D; idx += kAttnThreads) {
-      const float L = cml[2 * (idx / D) + 1];
-      qs[idx] = (L > 0.0f) ? qs[idx] / L : 0.0f;
+    const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
+#pragma unroll
+    for (int i = 0; i < C; ++i) ov[i] = (l_run > 0.0f) ? (ov[i] + zs_run) * inv_l : 0.0f;
+    if constexpr (BLK > 0) {
+      quad_fwht<C, BLK>(ov, tig);
+#pragma unroll
+      for (int i = 0; i < C; ++i) ov[i] *= p.cb;
     }
-  } else {
-    // ---- several clusters per (sequence, kv head): meet in the workspace -----
+    if (g < G) {
+      const size_t o_base = ((size_t)n * p.Hq + (size_t)h * G + g) * D + C * tig;
+#pragma unroll
+      for (int i = 0; i < C; ++i) store_out(p, o_base + i, ov[i]);
+    }
+  } else if (g < G) {
     const int part = split / cs;
-    const int np = p.n_parts;
-    float* base = p.ws_part + (((size_t)n * p.Hkv + h) * np) * G * (D + 2);
-    float* dst = base + (size_t)part * G * (D + 2);
-    for (int idx = tid; idx < G * D; idx += kAttnThreads) {
-      const int r = idx / D, c = idx % D;
-      dst[r * (D + 2) + c] = qs[idx];
-      if (c == 0) {
-        dst[r * (D + 2) + D] = cml[2 * r];
-        dst[r * (D + 2) + D + 1] = cml[2 * r + 1];
-      }
-    }
-    __threadfence();
-    __syncthreads();
-    int* s_last = flags + kAttnWarps * kStages;
-    if (tid == 0) {
-      const int prev = atomicAdd(&p.ws_count[(size_t)n * p.Hkv + h], 1);
-      *s_last = (prev == np - 1);
-    }
-    __syncthreads();
-    if (!*s_last) return;
-    __threadfence();
-    float* lsp = wts + 8 * kMaxParts;  // per (head, part) sums
-    float* Lr = wts + 16 * kMaxParts;  // per head total
-    for (int idx = tid; idx < G * np; idx += kAttnThreads) {
-      const int r = idx % G, s = idx / G;
-      const float* src = base + ((size_t)s * G + r) * (D + 2) + D;
-      wts[r * kMaxParts + s] = __ldcg(src);
-      lsp[r * kMaxParts + s] = __ldcg(src + 1);
-    }
-    __syncthreads();
-    for (int r = warp; r < G; r += kAttnWarps) {
-      float M = -INFINITY;
-      for (int s = lane; s < np; s += 32) M = fmaxf(M, wts[r * kMaxParts + s]);
+    float* dst = p.ws_part + ((((size_t)n * p.Hkv + h) * p.n_parts + part) * G + g) * (D + 2);
 #pragma unroll
-      for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o2));
-      float L = 0.0f;
-      for (int s = lane; s < np; s += 32) {
-        const float ms = wts[r * kMaxParts + s];
-        const float e = (ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
-        wts[r * kMaxParts + s] = e;
-        L += e * lsp[r * kMaxParts + s];
-      }
-#pragma unroll
-      for (int o2 = 16; o2 > 0; o2 >>= 1) L += __shfl_xor_sync(FULL, L, o2);
-      if (lane == 0) Lr[r] = L;
+    for (int i = 0; i < C; ++i) dst[C * tig + i] = ov[i] + zs_run;
+    if (tig == 0) {
+      dst[D] = m_run;
+      dst[D + 1] = l_run;
     }
-    __syncthreads();
-    for (int idx = tid; idx < G * D; idx += kAttnThreads) {
-      const int r = idx / D, c = idx % D;
-      const float* src = base + (size_t)r * (D + 2) + c;
-      const size_t stride = (size_t)G * (D + 2);
-      float a0 = 0.0f, a1 = 0.0f, a2 = 0.0f, a3 = 0.0f;
-      int s = 0;
-      for (; s + 4 <= np; s += 4) {
-        const float v0 = __ldcg(src + (size_t)s * stride), v1 = __ldcg(src + (size_t)(s + 1) * stride);
-        const float v2 = __ldcg(src + (size_t)(s + 2) * stride), v3 = __ldcg(src + (size_t)(s + 3) * stride);
-        a0 = fmaf(wts[r * kMaxParts + s], v0, a0);
-        a1 = fmaf(wts[r * kMaxParts + s + 1], v1, a1);
-        a2 = fmaf(wts[r * kMaxParts + s + 2], v2, a2);
-        a3 = fmaf(wts[r * kMaxParts + s + 3], v3, a3);
-      }
-      for (; s < np; ++s) a0 = fmaf(wts[r * kMaxParts + s], __ldcg(src + (size_t)s * stride), a0);
-      const float acc = (a0 + a1) + (a2 + a3);
-      qs[idx] = (Lr[r] > 0.0f) ? acc / Lr[r] : 0.0f;
-    }
-    if (tid == 0) p.ws_count[(size_t)n * p.Hkv + h] = 0;  // leave the tickets at zero
-  }
-  __syncthreads();
-
-  // ---- out = R o_rot -------------------------------------------------------------
-  if constexpr (BLK > 0) smem_fwht_rows<D, BLK>(qs, G);
-  for (int idx = tid; idx < G * D; idx += kAttnThreads) {
-    const int r = idx / D, c = idx % D;
-    const float val = (BLK > 0) ? qs[idx] * p.cb : qs[idx];
-    const size_t o_idx = ((size_t)n * p.Hq + (size_t)h * G + r) * D + c;
-    if (p.out_bf16)
-      reinterpret_cast<__nv_bfloat16*>(p.out)[o_idx] = __float2bfloat16_rn(val);
-    else
-      reinterpret_cast<float*>(p.out)[o_idx] = val;
   }
 }
 

@@ -61,24 +61,26 @@ __device__ __forceinline__ void mbar_arrive(uint32_t bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(bar) : "memory");
 }
 
+// One bounded-time wait round: the thread may sleep until the phase completes
+// or about `hint_ns` pass, so a waiting warp does not spin on the issue port.
 __device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
       "{\n"
       ".reg .pred p;\n"
-      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n"
       "selp.u32 %0, 1, 0, p;\n"
       "}\n"
       : "=r"(ok)
-      : "r"(bar), "r"(parity)
+      : "r"(bar), "r"(parity), "r"(1000000u)
       : "memory");
   return ok != 0;
 }
 
-// Upper bound on try_wait rounds before a wait is declared lost. Each round
-// returns after at most a hardware-defined suspend time, so the bound is far
-// above any legitimate copy latency and still ends in well under a minute.
-constexpr uint32_t kMaxWaitRounds = 1u << 22;
+// Upper bound on try_wait rounds before a wait is declared lost. A round lasts
+// at most about a millisecond (its suspend hint), so the bound is far above
+// any legitimate copy latency and ends within a few seconds.
+constexpr uint32_t kMaxWaitRounds = 4096;
 
 // Bounded wait for phase `parity` of an mbarrier. On running out it records
 // KVQ_ERR_TIMEOUT and returns false; the caller abandons its work.
@@ -213,6 +215,15 @@ __device__ __forceinline__ uint32_t cluster_ctarank() {
 __device__ __forceinline__ void cluster_sync_all() {
   asm volatile("barrier.cluster.arrive.release.aligned;\n" ::: "memory");
   asm volatile("barrier.cluster.wait.acquire.aligned;\n" ::: "memory");
+}
+
+// Store four floats into the shared memory of CTA `rank` of this cluster, at
+// the address that `local` has in this CTA (16-byte aligned).
+__device__ __forceinline__ void st_dsmem_v4(float* local, uint32_t rank, float a, float b, float c, float d) {
+  uint32_t remote;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;\n" : "=r"(remote) : "r"(smem_addr(local)), "r"(rank));
+  asm volatile("st.shared::cluster.v4.f32 [%0], {%1, %2, %3, %4};\n" ::"r"(remote), "f"(a), "f"(b), "f"(c), "f"(d)
+               : "memory");
 }
 
 // Load a float from the shared memory of CTA `rank` of this cluster, at the

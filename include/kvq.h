@@ -128,8 +128,8 @@ kvq_status kv_quant_write(const void* k, const void* v, const int64_t* slot_mapp
  * once. Returns SIZE_MAX when the shapes are invalid or no device can be
  * queried.
  *
- * Layout: the first round_up(batch*num_kv_heads*4, 256) bytes are the split
- * tickets (int32 counters), the rest holds per-split partial results.
+ * The workspace holds per-split partial results (fp32); it needs no
+ * initialization.
  */
 size_t kvq_attn_workspace_size(const kvq_attn_desc* desc);
 
@@ -145,7 +145,7 @@ size_t kvq_attn_workspace_size(const kvq_attn_desc* desc);
  *   logit_t = softmax_scale * (R q) . k^_t;  p = softmax(logit);
  *   out[n][i] = R (sum_t p_t v^_t).      context_lens[n] = 0 gives out = 0.
  *
- * q            : device, bf16 [B][Hq][D], contiguous.
+ * q            : device, bf16 [B][Hq][D], contiguous, 16-byte aligned.
  * cache, scales, zeros : device, as written by kv_quant_write with the same
  *                hadamard_block.
  * page_table   : device, int32 [B][max_pages_per_seq]; entries past the
@@ -155,11 +155,10 @@ size_t kvq_attn_workspace_size(const kvq_attn_desc* desc);
  *                clamped and records KVQ_ERR_OUT_OF_RANGE.
  * out          : device, [B][Hq][D], fp32 or bf16 (desc->out_dtype).
  * workspace    : device, at least kvq_attn_workspace_size(desc) bytes, 16-byte
- *                aligned; may be NULL when that size is 0. Its ticket counters
- *                must be zero before its first use (zero the whole buffer
- *                once); every call returns them to zero, so one buffer serves
- *                any number of calls issued one after another on a stream.
- *                Calls that overlap on the GPU must use different workspaces.
+ *                aligned, no initialization needed; may be NULL when that size
+ *                is 0. Calls that overlap on the GPU must use different
+ *                workspaces. When partial results are used, the call launches
+ *                a second, small kernel that merges them (on the same stream).
  * batch = 0 launches nothing and returns KVQ_OK (pointers may then be NULL).
  * Returns KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_WORKSPACE
  * or KVQ_ERR_CUDA.
@@ -185,8 +184,7 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache,
  * still passes all inputs and outputs, exactly as for paged_decode_attn_int4.
  *  - The first call on a device looks up that array's device address (once
  *    per device); make that first call before any stream capture.
- *  - Every call clears the array's ticket counters on `stream` before its
- *    kernel and otherwise reuses whatever the previous call left there.
+ *  - The array needs no clearing: each call overwrites what it reads.
  *  - All calls share the one array per device: calls that overlap on the GPU
  *    (other streams, other host threads) race and give wrong results.
  *  - Shapes that would need more scratch than the array holds are rejected

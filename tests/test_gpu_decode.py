@@ -3,8 +3,8 @@
 The oracle reads the cache bytes the CUDA write produced, so write-path
 differences cannot leak into this check. Bar: fp32 output within 2e-3
 max-abs of the fp64 oracle; bf16 output equal to the round-to-nearest bf16 of
-the fp32 output; guard regions around `out` untouched; the workspace all zero
-again after every call.
+the fp32 output; guard regions around `out` untouched; a workspace reused
+without clearing gives the same result.
 """
 import numpy as np
 import pytest
@@ -66,12 +66,6 @@ def oracle_out(orc, w, pool, b=None, softmax_scale=0.0, pairs=None):
                                     w.num_pages, softmax_scale) for n, hq in pairs}
 
 
-def counters_zero(ws, w):
-    """The split tickets (the workspace's first bytes) are back to zero."""
-    n = ((w.B * w.Hkv * 4 + 255) // 256) * 256
-    return int(ws[:n].sum()) == 0
-
-
 def assert_close(got, ref, label):
     err = float(np.abs(got - ref).max()) if ref.size else 0.0
     print(f"{label}: max|err| = {err:.3e} (max|ref| = {float(np.abs(ref).max(initial=0)):.3e})")
@@ -83,7 +77,6 @@ def test_decode_tiny_config(orc):
     pool = build_cache(w)
     got, ws = gpu_decode(w, pool)
     assert_close(got, oracle_out(orc, w, pool), "tiny")
-    assert counters_zero(ws, w)
 
 
 @pytest.mark.parametrize("D,b", [(64, 0), (64, 32), (64, 64), (128, 0), (128, 32), (128, 64), (128, 128)])
@@ -99,7 +92,6 @@ def test_decode_random_shapes(orc, D, b, G):
     ref = oracle_out(orc, w, pool)
     assert_close(got, ref, f"D={D} b={b} G={G}")
     assert np.all(got[0] == 0.0), "empty context must give zero output"
-    assert counters_zero(ws, w)
 
 
 def test_decode_single_split_path(orc):
@@ -166,14 +158,14 @@ def test_decode_explicit_softmax_scale_and_bf16(orc):
     assert np.array_equal(got16.astype(np.float32), ref16)
 
 
-def test_decode_deterministic_and_workspace_reuse():
+def test_decode_deterministic_and_workspace_needs_no_init():
     w = workloads.random_case(seed=9, B=2, Hq=16, Hkv=4, D=128, block=128, context_lens=[3000, 777])
     pool = build_cache(w)
     a, ws = gpu_decode(w, pool)
-    assert counters_zero(ws, w)
+    assert ws.numel() > 16, "the case must use partial results"
+    ws.fill_(0xFF)  # NaN bytes: the call must not read what it did not write
     b_, ws = gpu_decode(w, pool, ws=ws)
     assert np.array_equal(a, b_)
-    assert counters_zero(ws, w)
 
 
 def test_decode_bad_page_id_and_long_context_are_reported(orc):

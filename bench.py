@@ -261,37 +261,34 @@ class Step:
         self.torch.cuda.synchronize(self.dev)
 
     def timed_only(self, kind, steps, start_index=0):
-        """One kernel alone, `steps` launches; returns the per-launch ms."""
+        """One kernel alone, `steps` back-to-back launches on the stream,
+        bracketed by two events (inputs and outputs rotate through sets
+        larger than L2). Returns the average ms per launch."""
         torch = self.torch
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps)]
+        fn = self.write if kind == "write" else self.decode
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(self.stream)
         for j in range(steps):
-            i = start_index + j
-            evs[2 * j].record(self.stream)
-            (self.write if kind == "write" else self.decode)(i)
-            evs[2 * j + 1].record(self.stream)
-        evs[-1].synchronize()
-        return [evs[2 * j].elapsed_time(evs[2 * j + 1]) for j in range(steps)]
+            fn(start_index + j)
+        t1.record(self.stream)
+        t1.synchronize()
+        return t0.elapsed_time(t1) / steps
 
     def timed(self, steps, start_index=0):
-        """Run `steps` steps with an event before and after every kernel.
-        Returns (total_ms, [write_ms], [decode_ms])."""
+        """Run `steps` whole steps (write, then decode) back to back between
+        two events. Returns the total ms."""
         torch = self.torch
-        evs = [torch.cuda.Event(enable_timing=True) for _ in range(3 * steps)]
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(self.stream)
         for j in range(steps):
             i = start_index + j
-            evs[3 * j].record(self.stream)
             self.write(i)
-            evs[3 * j + 1].record(self.stream)
             self.decode(i)
-            evs[3 * j + 2].record(self.stream)
         t1.record(self.stream)
         t1.synchronize()
-        wr = [evs[3 * j].elapsed_time(evs[3 * j + 1]) for j in range(steps)]
-        de = [evs[3 * j + 1].elapsed_time(evs[3 * j + 2]) for j in range(steps)]
-        return t0.elapsed_time(t1), wr, de
+        return t0.elapsed_time(t1)
 
 
 def e2e_run(w, block, dev, steps, warmup):
@@ -410,7 +407,8 @@ def config_block(w, block):
         "workload": w.cfg.name, "batch": w.B, "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D,
         "context": int(w.context_lens.max()), "written_tokens": w.tokens_written, "page": 16,
         "hadamard_block": block, "out_dtype": "bf16",
-        "l2": "inputs larger than L2 alternate; decode reads a cache written two steps earlier",
+        "l2": "inputs larger than L2 rotate; decode reads a cache written two steps earlier",
+        "timing": "steps back to back between two events; each kernel's line: the same, that kernel alone",
     }
 
 
@@ -470,11 +468,10 @@ def main(argv=None):
     if args.only:
         step.timed_only(args.only, warm)
         barrier()
-        ms = step.timed_only(args.only, args.steps, start_index=warm)
+        mean = step.timed_only(args.only, args.steps, start_index=warm)
         barrier()
         if rank == 0:
             nb = wb if args.only == "write" else db
-            mean = statistics.mean(ms)
             print(json.dumps({"only": args.only, "us": round(1e3 * mean, 3),
                               "GB/s": round(nb / (mean / 1e3) / 1e9, 2), "launches": args.steps,
                               "config": config_block(w, block)}), flush=True)
@@ -486,13 +483,18 @@ def main(argv=None):
         step.timed(warm)                    # warm-up steps (untimed)
         barrier()
         t_host0 = time.monotonic()
-        total_ms, wr, de = step.timed(args.steps, start_index=warm)
+        total_ms = step.timed(args.steps, start_index=warm)
+        barrier()
+        # each kernel alone, back to back, for its own roofline line
+        wr_ms = step.timed_only("write", args.steps, start_index=warm)
+        barrier()
+        de_ms = step.timed_only("decode", args.steps, start_index=warm)
         t_host1 = time.monotonic()
         clocks.mark(t_host0, t_host1)
     barrier()
     total_ms = max_over_ranks(total_ms)
-    wr_ms = max_over_ranks(statistics.mean(wr))
-    de_ms = max_over_ranks(statistics.mean(de))
+    wr_ms = max_over_ranks(wr_ms)
+    de_ms = max_over_ranks(de_ms)
 
     plain = None
     if not args.no_plain and block != 0:
@@ -500,10 +502,12 @@ def main(argv=None):
         p.fill_pools()
         p.timed(warm)
         barrier()
-        p_total, p_wr, p_de = p.timed(args.steps, start_index=warm)
+        p_total = p.timed(args.steps, start_index=warm)
         barrier()
-        p_wr_ms = max_over_ranks(statistics.mean(p_wr))
-        p_de_ms = max_over_ranks(statistics.mean(p_de))
+        p_wr_ms = max_over_ranks(p.timed_only("write", args.steps, start_index=warm))
+        barrier()
+        p_de_ms = max_over_ranks(p.timed_only("decode", args.steps, start_index=warm))
+        barrier()
         p_total = max_over_ranks(p_total)
         plain = {
             "hadamard_block": 0,

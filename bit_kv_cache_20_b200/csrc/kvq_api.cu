@@ -127,119 +127,115 @@ kvq_status dispatch_write(const kvq::WriteParams& p, int b, int dev, cudaStream_
 // paged_decode_attn_int4
 // ---------------------------------------------------------------------------
 struct SplitPlan {
-  int n_splits;         // CTAs per (sequence, kv-head group)
+  int n_splits;         // CTAs per (sequence, kv-head group) = partials in the workspace
   int pages_per_split;
-  int cluster;          // CTAs per thread-block cluster (divides n_splits)
-  int n_parts;          // clusters per (sequence, kv-head group) = partials in the workspace
   int hg;               // kv heads per CTA
+  int nc;               // column tiles of 4 query heads
 };
 
-// kv heads served by one CTA: 4, 2 or 1, whichever largest divides Hkv.
-int heads_per_cta(int Hkv) { return (Hkv % 4 == 0) ? 4 : (Hkv % 2 == 0) ? 2 : 1; }
+int cols_for(int G) { return G > 4 ? 2 : 1; }
 
-int inst_slot(int D, int b, int hg) {
+int inst_slot(int D, int b, int hg, int nc) {
   const int bi = (b == 0) ? 0 : (b == 32) ? 1 : (b == 64) ? 2 : 3;
   const int hi = (hg == 4) ? 2 : (hg == 2) ? 1 : 0;
-  return ((D == 64) ? 0 : 12) + bi * 3 + hi;
+  return (((D == 64) ? 0 : 1) * 4 + bi) * 6 + hi * 2 + (nc - 1);
 }
-constexpr int kInstSlots = 24;
+constexpr int kInstSlots = 48;
 
-template <int D, int BLK>
+// Instances exist for HG * NC <= 4 (the plan never asks for more).
+template <int D, int BLK, int NC>
 const void* decode_kernel_ptr(int hg) {
-  if (hg == 4) return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK, 4>);
-  if (hg == 2) return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK, 2>);
-  return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK, 1>);
-}
-
-const void* decode_kernel_for(int D, int b, int hg) {
-  if (D == 64) {
-    if (b == 0) return decode_kernel_ptr<64, 0>(hg);
-    if (b == 32) return decode_kernel_ptr<64, 32>(hg);
-    if (b == 64) return decode_kernel_ptr<64, 64>(hg);
-    return nullptr;
+  if constexpr (NC == 1) {
+    if (hg == 4) return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK, 4, NC>);
   }
-  if (b == 0) return decode_kernel_ptr<128, 0>(hg);
-  if (b == 32) return decode_kernel_ptr<128, 32>(hg);
-  if (b == 64) return decode_kernel_ptr<128, 64>(hg);
-  if (b == 128) return decode_kernel_ptr<128, 128>(hg);
+  if (hg == 2) return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK, 2, NC>);
+  if (hg == 1) return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK, 1, NC>);
   return nullptr;
 }
 
-int decode_smem_bytes(int D) {
-  return D == 64 ? kvq::AttnSmem<64>::kTotal : kvq::AttnSmem<128>::kTotal;
+template <int D, int BLK>
+const void* decode_kernel_ptr(int hg, int nc) {
+  return nc == 2 ? decode_kernel_ptr<D, BLK, 2>(hg) : decode_kernel_ptr<D, BLK, 1>(hg);
 }
 
-// Opt the decode kernel instance into its dynamic shared memory (once per
-// device and instance).
-bool prepare_decode_kernel(int dev, int D, int b, int hg) {
-  static std::atomic<int> done[kMaxDevices][kInstSlots];
-  const int slot = inst_slot(D, b, hg);
-  if (done[dev][slot].load(std::memory_order_relaxed)) return true;
-  const void* k = decode_kernel_for(D, b, hg);
-  if (!k || cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, decode_smem_bytes(D)) !=
-                cudaSuccess) {
-    cudaGetLastError();
-    return false;
+const void* decode_kernel_for(int D, int b, int hg, int nc) {
+  if (D == 64) {
+    if (b == 0) return decode_kernel_ptr<64, 0>(hg, nc);
+    if (b == 32) return decode_kernel_ptr<64, 32>(hg, nc);
+    if (b == 64) return decode_kernel_ptr<64, 64>(hg, nc);
+    return nullptr;
   }
-  done[dev][slot].store(1, std::memory_order_relaxed);
-  return true;
+  if (b == 0) return decode_kernel_ptr<128, 0>(hg, nc);
+  if (b == 32) return decode_kernel_ptr<128, 32>(hg, nc);
+  if (b == 64) return decode_kernel_ptr<128, 64>(hg, nc);
+  if (b == 128) return decode_kernel_ptr<128, 128>(hg, nc);
+  return nullptr;
 }
 
-// Clusters of `cs` decode CTAs that can be resident at once on the device.
-int max_active_clusters(int dev, int D, int b, int hg, int cs) {
-  static std::atomic<int> cache[kMaxDevices][kInstSlots][kvq::kMaxCluster + 1];
-  const int slot = inst_slot(D, b, hg);
-  int v = cache[dev][slot][cs].load(std::memory_order_relaxed);
+template <int D, int NC>
+int decode_smem_bytes_t(int hg) {
+  if constexpr (NC == 1) {
+    if (hg == 4) return kvq::AttnSmem<D, 4, NC>::kTotal;
+  }
+  if (hg == 2) return kvq::AttnSmem<D, 2, NC>::kTotal;
+  return kvq::AttnSmem<D, 1, NC>::kTotal;
+}
+
+int decode_smem_bytes(int D, int hg, int nc) {
+  if (D == 64) return nc == 2 ? decode_smem_bytes_t<64, 2>(hg) : decode_smem_bytes_t<64, 1>(hg);
+  return nc == 2 ? decode_smem_bytes_t<128, 2>(hg) : decode_smem_bytes_t<128, 1>(hg);
+}
+
+// Opt the decode kernel instance into its dynamic shared memory and return
+// how many of its CTAs one SM holds (once per device and instance; 0 on error).
+int decode_ctas_per_sm(int dev, int D, int b, int hg, int nc) {
+  static std::atomic<int> cache[kMaxDevices][kInstSlots];
+  if (dev < 0 || dev >= kMaxDevices) return 0;
+  const int slot = inst_slot(D, b, hg, nc);
+  int v = cache[dev][slot].load(std::memory_order_relaxed);
   if (v > 0) return v;
-  if (!prepare_decode_kernel(dev, D, b, hg)) return 0;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(cs, 1, 1);
-  cfg.blockDim = dim3(kvq::kAttnThreads, 1, 1);
-  cfg.dynamicSmemBytes = decode_smem_bytes(D);
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = cs;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  int n = 0;
-  if (cudaOccupancyMaxActiveClusters(&n, decode_kernel_for(D, b, hg), &cfg) != cudaSuccess || n < 1) {
+  const void* k = decode_kernel_for(D, b, hg, nc);
+  const int smem = decode_smem_bytes(D, hg, nc);
+  if (!k || cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, k, kvq::kAttnThreads, smem) != cudaSuccess || v < 1) {
     cudaGetLastError();
     return 0;
   }
-  cache[dev][slot][cs].store(n, std::memory_order_relaxed);
-  return n;
+  cache[dev][slot].store(v, std::memory_order_relaxed);
+  return v;
 }
 
-// Split each (sequence, kv-head group) into CTAs grouped in thread-block
-// clusters (which merge on chip), choosing the cluster size and the split
-// count so that every CTA of the launch is resident at once (one wave, as the
-// occupancy API reports for clusters of that size) and each split keeps at
-// least 8 pages. Larger clusters are preferred (fewer partial results); a
-// smaller one must buy more than 10 % more splits. Only with more than one
-// cluster per (sequence, head group) do partial results go through the
-// workspace and a combine kernel.
+// Choose the kv heads per CTA (HG) and the split of each (sequence, head
+// group) into CTAs. For each HG that divides Hkv (with HG * NC <= 4), the
+// split count fills the device's resident CTA slots once (as the occupancy
+// API reports for that instance) with at least 4 pages per split; the plan
+// with the least work per CTA times waves (plus a fixed cost of 8 head-pages
+// per CTA) wins, ties going to the smaller HG (fewer partial results).
 SplitPlan plan_splits(const kvq_attn_desc* d, int dev) {
-  const int hg = heads_per_cta(d->num_kv_heads);
-  const long long units = (long long)d->batch * (d->num_kv_heads / hg);
-  long long cap = d->max_pages_per_seq / 8;
-  if (cap < 1) cap = 1;
-  if (cap > kvq::kMaxSplits) cap = kvq::kMaxSplits;
-  SplitPlan best = {1, d->max_pages_per_seq, 1, 1, hg};
-  if (units <= 0 || cap == 1) return best;
-  for (int cs = kvq::kMaxCluster; cs >= 1; --cs) {
-    const int mac = max_active_clusters(dev, d->head_dim, d->hadamard_block, hg, cs);
-    const long long per_unit = mac / units;  // clusters per (sequence, head group) in one wave
-    if (per_unit < 1) continue;
-    long long parts = per_unit;
-    if (parts > cap / cs) parts = cap / cs;
-    if (parts > kvq::kMaxParts) parts = kvq::kMaxParts;
-    if (parts < 1) continue;
-    const long long ns = parts * cs;
-    if (ns * 10 > best.n_splits * 11LL) best = {(int)ns, 0, cs, (int)parts, hg};
+  const int nc = cols_for(d->num_q_heads / d->num_kv_heads);
+  const int sms = sm_count(dev);
+  SplitPlan best = {1, d->max_pages_per_seq, 1, nc};
+  long long best_cost = LLONG_MAX;
+  for (int hg = 1; hg <= 4; hg <<= 1) {
+    if (d->num_kv_heads % hg != 0 || hg * nc > 4) continue;
+    const int per_sm = decode_ctas_per_sm(dev, d->head_dim, d->hadamard_block, hg, nc);
+    if (per_sm < 1 || sms < 1) continue;
+    const long long slots = (long long)per_sm * sms;
+    const long long units = (long long)d->batch * (d->num_kv_heads / hg);
+    long long ns = units > 0 ? slots / units : 1;
+    long long ns_cap = d->max_pages_per_seq / 4;
+    if (ns_cap > kvq::kMaxSplits) ns_cap = kvq::kMaxSplits;
+    if (ns > ns_cap) ns = ns_cap;
+    if (ns < 1) ns = 1;
+    const long long pps = (d->max_pages_per_seq + ns - 1) / ns;
+    ns = (d->max_pages_per_seq + pps - 1) / pps;  // drop splits that would be empty
+    const long long waves = (units * ns + slots - 1) / slots;
+    const long long cost = (waves < 1 ? 1 : waves) * (pps * hg + 8);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best = {(int)ns, (int)pps, hg, nc};
+    }
   }
-  best.pages_per_split = (d->max_pages_per_seq + best.n_splits - 1) / best.n_splits;
   return best;
 }
 
@@ -260,70 +256,55 @@ kvq_status check_attn_desc(const kvq_attn_desc* d) {
   return KVQ_OK;
 }
 
-size_t workspace_bytes_for(const kvq_attn_desc* d, const SplitPlan& plan) {
-  if (plan.n_parts <= 1 || d->batch == 0) return 0;
+// Workspace: the splits' partial results (fp32 rows of D + 4: O + Z, M, L,
+// padding), then one ticket counter per (sequence, head group).
+size_t partial_bytes_for(const kvq_attn_desc* d, const SplitPlan& plan) {
   const size_t G = (size_t)(d->num_q_heads / d->num_kv_heads);
-  return (size_t)d->batch * d->num_kv_heads * plan.n_parts * G * (d->head_dim + 2) * sizeof(float);
+  return (size_t)d->batch * d->num_kv_heads * plan.n_splits * G * (d->head_dim + 4) * sizeof(float);
+}
+
+size_t workspace_bytes_for(const kvq_attn_desc* d, const SplitPlan& plan) {
+  if (plan.n_splits <= 1 || d->batch == 0) return 0;
+  const size_t counters = (size_t)d->batch * (d->num_kv_heads / plan.hg) * sizeof(int);
+  return partial_bytes_for(d, plan) + (counters + 15) / 16 * 16;
+}
+
+template <int D, int BLK, int NC>
+cudaError_t launch_decode_instance(const kvq::AttnParams& p, int hg, int smem, cudaStream_t s) {
+  const dim3 grid(p.n_splits, p.Hkv / hg, p.B);
+  if constexpr (NC == 1) {
+    if (hg == 4) {
+      kvq::kvq_decode_kernel<D, BLK, 4, NC><<<grid, kvq::kAttnThreads, smem, s>>>(p);
+      return cudaGetLastError();
+    }
+  }
+  if (hg == 2) kvq::kvq_decode_kernel<D, BLK, 2, NC><<<grid, kvq::kAttnThreads, smem, s>>>(p);
+  else if (hg == 1) kvq::kvq_decode_kernel<D, BLK, 1, NC><<<grid, kvq::kAttnThreads, smem, s>>>(p);
+  else return cudaErrorInvalidValue;
+  return cudaGetLastError();
 }
 
 template <int D, int BLK>
-kvq_status launch_attn(const kvq::AttnParams& p, int hg, int dev, cudaStream_t s) {
-  if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
-  if (!prepare_decode_kernel(dev, D, BLK, hg)) return KVQ_ERR_CUDA;
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.n_splits, p.Hkv / hg, p.B);
-  cfg.blockDim = dim3(kvq::kAttnThreads, 1, 1);
-  cfg.dynamicSmemBytes = kvq::AttnSmem<D>::kTotal;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeClusterDimension;
-  attr[0].val.clusterDim.x = p.cluster_size;
-  attr[0].val.clusterDim.y = 1;
-  attr[0].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  cudaError_t e;
-  if (hg == 4) e = cudaLaunchKernelEx(&cfg, kvq::kvq_decode_kernel<D, BLK, 4>, p);
-  else if (hg == 2) e = cudaLaunchKernelEx(&cfg, kvq::kvq_decode_kernel<D, BLK, 2>, p);
-  else e = cudaLaunchKernelEx(&cfg, kvq::kvq_decode_kernel<D, BLK, 1>, p);
-  if (e != cudaSuccess) {
-    cudaGetLastError();
-    return KVQ_ERR_CUDA;
-  }
-  if (p.n_parts > 1) {
-    // merge the clusters' partial results; launched as a programmatic
-    // dependent so its CTAs are scheduled while the main grid drains
-    cudaLaunchConfig_t c2 = {};
-    c2.gridDim = dim3(p.G, p.Hkv, p.B);
-    c2.blockDim = dim3(D, 1, 1);
-    c2.dynamicSmemBytes = 0;
-    c2.stream = s;
-    cudaLaunchAttribute a2[1];
-    a2[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-    a2[0].val.programmaticStreamSerializationAllowed = 1;
-    c2.attrs = a2;
-    c2.numAttrs = 1;
-    if (cudaLaunchKernelEx(&c2, kvq::kvq_decode_combine_kernel<D, BLK>, p) != cudaSuccess) {
-      cudaGetLastError();
-      return KVQ_ERR_CUDA;
-    }
-  }
-  return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+kvq_status launch_attn(const kvq::AttnParams& p, const SplitPlan& plan, int dev, cudaStream_t s) {
+  if (decode_ctas_per_sm(dev, D, BLK, plan.hg, plan.nc) < 1) return KVQ_ERR_CUDA;
+  const int smem = decode_smem_bytes(D, plan.hg, plan.nc);
+  const cudaError_t e = plan.nc == 2 ? launch_decode_instance<D, BLK, 2>(p, plan.hg, smem, s)
+                                     : launch_decode_instance<D, BLK, 1>(p, plan.hg, smem, s);
+  return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
 template <int D>
-kvq_status dispatch_attn(const kvq::AttnParams& p, int b, int hg, int dev, cudaStream_t s) {
+kvq_status dispatch_attn(const kvq::AttnParams& p, int b, const SplitPlan& plan, int dev, cudaStream_t s) {
   switch (b) {
-    case 0: return launch_attn<D, 0>(p, hg, dev, s);
-    case 32: return launch_attn<D, 32>(p, hg, dev, s);
-    case 64: return launch_attn<D, 64>(p, hg, dev, s);
+    case 0: return launch_attn<D, 0>(p, plan, dev, s);
+    case 32: return launch_attn<D, 32>(p, plan, dev, s);
+    case 64: return launch_attn<D, 64>(p, plan, dev, s);
     case 128:
-      if constexpr (D >= 128) return launch_attn<D, 128>(p, hg, dev, s);
+      if constexpr (D >= 128) return launch_attn<D, 128>(p, plan, dev, s);
       return KVQ_ERR_UNSUPPORTED;
     default: return KVQ_ERR_UNSUPPORTED;
   }
 }
-
 }  // namespace
 
 extern "C" {
@@ -413,17 +394,17 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const voi
   p.max_pages = d.max_pages_per_seq;
   p.n_splits = plan.n_splits;
   p.pages_per_split = plan.pages_per_split;
-  p.cluster_size = plan.cluster;
-  p.n_parts = plan.n_parts;
   p.ws_part = need > 0 ? static_cast<float*>(workspace) : nullptr;
+  p.ws_count = need > 0 ? reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + partial_bytes_for(&d, plan))
+                        : nullptr;
   p.out_bf16 = d.out_dtype;
   const double cb = d.hadamard_block > 0 ? 1.0 / std::sqrt((double)d.hadamard_block) : 1.0;
   const double scale = d.softmax_scale > 0.0f ? (double)d.softmax_scale : 1.0 / std::sqrt((double)d.head_dim);
   p.qmul = (float)(cb * scale * 1.4426950408889634);  // log2(e)
   p.cb = (float)cb;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  return d.head_dim == 64 ? dispatch_attn<64>(p, d.hadamard_block, plan.hg, dev, s)
-                          : dispatch_attn<128>(p, d.hadamard_block, plan.hg, dev, s);
+  return d.head_dim == 64 ? dispatch_attn<64>(p, d.hadamard_block, plan, dev, s)
+                          : dispatch_attn<128>(p, d.hadamard_block, plan, dev, s);
 }
 
 kvq_status kvq_get_device_error(void* stream) {

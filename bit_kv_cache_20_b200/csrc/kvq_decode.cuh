@@ -5,38 +5,46 @@
 // rotates q once, runs attention in the rotated space directly on the codes,
 // and rotates the output back: out = R sum_t p_t v^_t.
 //
-// Grid (split, kv-head group, sequence), 4 warps per CTA. A CTA serves HG kv
-// heads (HG = 4, 2 or 1, dividing Hkv); warp w works for head w % HG. Because
-// the cache is laid out [page][kv head][K|V][token][D/2], the HG heads of one
-// page are one contiguous block: each page costs the CTA three 1-D bulk
-// copies (TMA engine) - HG*16*D code bytes, HG*64 B of scales, HG*64 B of
-// zeros - into a CTA-wide ring of stages (a stage = two pages), completing on
-// one mbarrier per stage. The last warp done with a stage refills it.
+// Grid (split, kv-head group, sequence), 8 warps per CTA, every CTA of the
+// launch resident at once. A CTA serves HG kv heads (HG = 1, 2 or 4) over one
+// contiguous range of pages; warp w works for head w % HG and takes every
+// (8/HG)-th page of the range. Each warp streams its own pages into a private
+// ring of kWarpRing page slots in shared memory with 16-byte cp.async copies
+// (the codes of one (page, head) are 16*D contiguous bytes; its 32 scales and
+// 32 zeros 64 B each), kWarpRing - 1 pages ahead of the one it computes on.
+// (Measured on B200 with this page layout: per-warp cp.async streams reach the
+// bandwidth of a contiguous read; a single issuing thread with 1-D bulk copies
+// and mbarriers stayed near a third of it.)
 //
-// Per page, on the tensor cores (mma.m16n8k16, f16 in, f32 accumulate):
-//   QK: S[16 rows x 16 tokens] = Qhl[16 x D] * codes^T
-//   PV: O[16 rows x D]        += Phl[16 x 16 tokens] * codes
-// A rows 0..7 carry the fp16 "hi" part of up to 8 query heads (the GQA group)
-// and rows 8..15 the "lo" remainder (x = hi + lo keeps ~22 bits), so one MMA
-// does both halves. The 4-bit codes enter as exact normal fp16 values c (or
-// 16c for a nibble at bits 4..7, compensated by 1/16 on the other operand or
-// in the epilogue); subnormal fp16 operands are avoided on purpose - small
-// products built from them lost precision in the tensor-core accumulation (a
-// systematic bias of ~2^-13 relative, measured on B200). Dequantization is
-// folded into per-token scalars:
+// Per page (16 tokens) and kv head, on the tensor cores, with the GQA group of
+// up to 4 query heads as 8 columns:
+//   QK (mma.m16n8k32, u8 x s8 -> s32, exact):
+//        S^T[16 tokens x 8] = codes[16 tokens x D] * Q8^T[D x 8]
+//   PV (mma.m16n8k16, f16 -> f32):
+//        O^T[D x 8]        += codes^T[D x 16 tokens] * Phl^T[16 tokens x 8]
+// QK takes the code bytes as they are: byte & 0x0F is the low code, byte &
+// 0xF0 the high code times 16, each product summed in its own accumulator.
+// q~ enters as two int8 limbs per element, q~ = sigma (q0 + q1 / 256) with
+// sigma = max|q~| / 127 per query head (error <= 2^-9 sigma, far below the
+// bf16 input's own precision); columns are (head, limb). PV needs floating
+// weights: p * s_v enters as an fp16 "hi" and "lo" part (hi + lo keeps ~22
+// bits) and the codes as exact normal fp16 values c (or 16c for a nibble at
+// bits 4..7, compensated in the epilogue); subnormal fp16 operands are
+// avoided on purpose - small products built from them lost precision in the
+// tensor-core accumulation (a systematic bias of ~2^-13 relative, measured on
+// B200). QK leaves a thread the logits of 2 tokens for one query head; PV
+// wants 4 tokens of one column, so 4 warp shuffles move the weights across.
+// Dequantization is folded into per-token scalars:
 //   logit_t = s_t * (q~ . code_t) + z_t * sum(q~)
 //   o_rot   = (sum_t p_t s_t code_t + sum_t p_t z_t) / sum_t p_t
 // with an online softmax in base 2 (log2 e folded into q~) that rescales only
-// when the running maximum grows. q is rotated and the output rotated back in
-// registers: each thread holds a contiguous D/4-channel slice of one query
-// row, and the butterfly stages that cross slices use warp shuffles.
+// when the running maximum grows. q is rotated once per CTA in shared memory.
 //
-// The splits of one (sequence, head group) form thread-block clusters (up to
-// 8 CTAs) that merge through distributed shared memory into the cluster's
-// first CTA. With one cluster per (sequence, head group) that CTA writes the
-// output; otherwise each cluster writes a partial result to the workspace and
-// kvq_decode_combine_kernel (chained by programmatic dependent launch) merges
-// them and rotates back.
+// With one split per (sequence, head group) the CTA rotates its output back
+// and writes it; otherwise it writes a partial result (O + Z, M, L) to the
+// workspace and takes a ticket from the group's counter there; the CTA that
+// takes the last ticket merges all splits, rotates back, writes the output and
+// sets the counter back to zero.
 #pragma once
 
 #include <climits>
@@ -53,76 +61,68 @@ struct AttnParams {
   const int32_t* page_table;  // [B][max_pages]
   const int32_t* ctx_lens;    // [B]
   void* out;                  // [B][Hq][D] fp32 or bf16
-  float* ws_part;             // [B][Hkv][n_parts][G][D + 2]: O + Z, then M, L
+  float* ws_part;             // [B][Hkv][n_splits][G][D + 2]: O + Z, then M, L
+  int* ws_count;              // [B][Hkv / HG] tickets, zero between calls
   int B, Hq, Hkv, G;
   int num_pages, max_pages;
   int n_splits, pages_per_split;
-  int cluster_size;           // CTAs per cluster along the split axis
-  int n_parts;                // n_splits / cluster_size
   int out_bf16;
   float qmul;                 // c_b * softmax_scale * log2(e)
   float cb;                   // c_b (output rotation), 1 for plain INT4
 };
 
-constexpr int kAttnWarps = 4;
+constexpr int kAttnWarps = 8;
 constexpr int kAttnThreads = kAttnWarps * 32;
-constexpr int kMaxSplits = 256;
-constexpr int kMaxParts = 64;
-constexpr int kMaxCluster = 8;
-constexpr int kMaxPids = 1024;   // page ids of a CTA's range kept in shared memory
+constexpr int kWarpRing = 4;        // page slots per warp
+constexpr int kMaxSplits = 128;
+constexpr int kMaxPids = 1024;      // page ids of a CTA's range kept in shared memory
 
-template <int D>
+// Shared memory of one decode CTA serving HG kv heads with NC column tiles
+// (4 query heads each).
+template <int D, int HG, int NC>
 struct AttnSmem {
-  static constexpr int kHeadPageBytes = 16 * D + 128;       // codes + 32 scales + 32 zeros
-  static constexpr int kRingBytes = 24 * kHeadPageBytes;    // 12/HG stages of 2 pages x HG heads
-  // per-warp result slot (overlays the ring once every copy has landed):
-  // O[8 rows][D], then (m, l, zs, unused) per row
-  static constexpr int kSlotFloats = 8 * D + 8 * 4;
-  static constexpr int kSlotBytes = kAttnWarps * kSlotFloats * 4;
-  static constexpr int kUnionBytes = kRingBytes > kSlotBytes ? kRingBytes : kSlotBytes;
-  static constexpr int kOffPid = kUnionBytes;
-  static constexpr int kOffBar = kOffPid + kMaxPids * 4;
-  static constexpr int kOffCnt = kOffBar + 12 * 8;
-  static constexpr int kOffFlag = kOffCnt + 12 * 4;
-  static constexpr int kTotal = kOffFlag + 12 * 4;
+  static constexpr int kSlotBytes = 16 * D + 128;               // codes + 32 scales + 32 zeros
+  static constexpr int kRingBytes = kAttnWarps * kWarpRing * kSlotBytes;
+  static constexpr int kRows = HG * 4 * NC;                     // query rows (G padded to 4 NC)
+  // per-warp result: O[4 NC rows][D], then (m, l, zs, unused) per row
+  static constexpr int kResFloats = 4 * NC * (D + 4);
+  static constexpr int kOffRes = kRingBytes;
+  static constexpr int kOffQ = kOffRes + kAttnWarps * kResFloats * 4;  // float [kRows][D]
+  static constexpr int kOffQInfo = kOffQ + kRows * D * 4;       // float [kRows][4]: scale, sum
+  static constexpr int kOffQ8 = kOffQInfo + kRows * 16;         // int8 [kRows][2 limbs][D], B order
+  static constexpr int kOffPid = kOffQ8 + kRows * 2 * D;
+  static constexpr int kOffFlag = kOffPid + kMaxPids * 4;
+  static constexpr int kTotal = kOffFlag + 16;
+  // last-split merge scratch, in the rings (free by then): the weight of
+  // every (row, split), the merged L per row, then the per-thread sums
+  static constexpr int kOffMS = 0;
+  static constexpr int kOffLS = kOffMS + kRows * kMaxSplits * 4;
+  static constexpr int kOffPartO = kOffLS + kRows * 4;
+  static constexpr int kOffML = kOffPartO + 2 * kAttnThreads * 16;  // float2 [kRows][kMaxSplits]: M, L
+  static_assert(kOffML + kRows * kMaxSplits * 8 <= kRingBytes, "merge scratch fits in the rings");
 };
 
-// Fast Walsh-Hadamard transform (blocks of BLK, Sylvester natural order) of a
-// row spread over the 4 lanes of a quad: lane tig holds channels
-// [C*tig, C*tig + C). Stages shorter than C stay in the thread; the longer
-// ones pair lanes tig and tig ^ (len / C).
-template <int C, int BLK>
-__device__ __forceinline__ void quad_fwht(float (&v)[C], int tig) {
-#pragma unroll
-  for (int len = 1; len < C && len < BLK; len <<= 1) {
-#pragma unroll
-    for (int i = 0; i < C; ++i) {
-      if ((i & len) == 0) {
-        const float a = v[i], b = v[i + len];
-        v[i] = a + b;
-        v[i + len] = a - b;
-      }
-    }
-  }
-#pragma unroll
-  for (int len = C; len < BLK; len <<= 1) {
-    const int m = len / C;
-    const bool upper = (tig & m) != 0;
-#pragma unroll
-    for (int i = 0; i < C; ++i) {
-      const float other = __shfl_xor_sync(0xffffffffu, v[i], m);
-      v[i] = upper ? (other - v[i]) : (v[i] + other);
-    }
+template <int N>
+__device__ __forceinline__ void lds_words(const uint8_t* src, uint32_t (&w)[N]) {
+  if constexpr (N == 4) {
+    const uint4 t = *reinterpret_cast<const uint4*>(src);
+    w[0] = t.x; w[1] = t.y; w[2] = t.z; w[3] = t.w;
+  } else if constexpr (N == 2) {
+    const uint2 t = *reinterpret_cast<const uint2*>(src);
+    w[0] = t.x; w[1] = t.y;
+  } else {
+    w[0] = *reinterpret_cast<const uint32_t*>(src);
   }
 }
 
-// hi/lo fp16 pair of two floats, packed as the A fragment wants them.
-__device__ __forceinline__ void split_pair(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+// fp16 pair of (x0, x1): the "hi" rounding, or with `lo` the remainder
+// fp16(x - hi) of each.
+__device__ __forceinline__ uint32_t hilo_pair(float x0, float x1, bool lo) {
   const __half2 h = __floats2half2_rn(x0, x1);
   const float2 hf = __half22float2(h);
   const __half2 l = __floats2half2_rn(__fsub_rn(x0, hf.x), __fsub_rn(x1, hf.y));
-  hi = *reinterpret_cast<const uint32_t*>(&h);
-  lo = *reinterpret_cast<const uint32_t*>(&l);
+  const uint32_t hu = *reinterpret_cast<const uint32_t*>(&h), lu = *reinterpret_cast<const uint32_t*>(&l);
+  return lo ? lu : hu;
 }
 
 __device__ __forceinline__ void store_out(const AttnParams& p, size_t idx, float v) {
@@ -132,438 +132,535 @@ __device__ __forceinline__ void store_out(const AttnParams& p, size_t idx, float
     reinterpret_cast<float*>(p.out)[idx] = v;
 }
 
-// Merge of the n_parts partial results of one (sequence, kv head, query row)
-// and inverse rotation. Grid (G, Hkv, B), D threads (one per channel).
+// Fast Walsh-Hadamard transform (blocks of BLK, Sylvester natural order:
+// y_i = sum_j (-1)^popcount(i & j) x_j) of one row of D values spread over a
+// warp, lane l holding elements [E l, E l + E), E = D / 32. Stages shorter than
+// E stay in the thread; the others pair lanes l and l ^ (len / E).
 template <int D, int BLK>
-__global__ void __launch_bounds__(D) kvq_decode_combine_kernel(const AttnParams p) {
-  __shared__ float sm_m[kMaxParts], sm_w[kMaxParts], sm_row[D];
-  __shared__ float sm_L;
-  asm volatile("griddepcontrol.wait;\n" ::: "memory");  // the partials are complete
-  const int r = blockIdx.x, h = blockIdx.y, n = blockIdx.z, c = threadIdx.x;
-  const int np = p.n_parts, G = p.G;
-  const size_t stride = (size_t)G * (D + 2);
-  const float* base = p.ws_part + (((size_t)n * p.Hkv + h) * np * G + r) * (D + 2);
-  for (int s = c; s < np; s += D) {
-    sm_m[s] = __ldcg(base + s * stride + D);
-    sm_w[s] = __ldcg(base + s * stride + D + 1);
-  }
-  __syncthreads();
-  if (c < 32) {
-    float M = -INFINITY;
-    for (int s = c; s < np; s += 32) M = fmaxf(M, sm_m[s]);
+__device__ __forceinline__ void warp_fwht(float (&v)[D / 32], int lane) {
+  constexpr int E = D / 32;
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
-    float L = 0.0f;
-    for (int s = c; s < np; s += 32) {
-      const float e = (sm_m[s] == -INFINITY) ? 0.0f : fast_exp2(sm_m[s] - M);
-      L += e * sm_w[s];
-      sm_w[s] = e;
-    }
+  for (int len = 1; len < E && len < BLK; len <<= 1) {
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(0xffffffffu, L, o);
-    if (c == 0) sm_L = L;
-  }
-  __syncthreads();
-  // all partials of this channel in flight at once, 16 at a time
-  float acc = 0.0f;
-  for (int s0 = 0; s0 < np; s0 += 16) {
-    float v[16];
-#pragma unroll
-    for (int j = 0; j < 16; ++j) v[j] = (s0 + j < np) ? __ldcg(base + (size_t)(s0 + j) * stride + c) : 0.0f;
-#pragma unroll
-    for (int j = 0; j < 16; ++j)
-      if (s0 + j < np) acc = fmaf(sm_w[s0 + j], v[j], acc);
-  }
-  sm_row[c] = (sm_L > 0.0f) ? acc / sm_L : 0.0f;
-  __syncthreads();
-  if constexpr (BLK > 0) {
-#pragma unroll 1
-    for (int len = 1; len < BLK; len <<= 1) {
-      float v = 0.0f;
-      if ((c & len) == 0) v = sm_row[c] + sm_row[c + len];
-      else v = sm_row[c - len] - sm_row[c];
-      __syncthreads();
-      sm_row[c] = v;
-      __syncthreads();
+    for (int i = 0; i < E; ++i) {
+      if ((i & len) == 0) {
+        const float a = v[i], b = v[i + len];
+        v[i] = a + b;
+        v[i + len] = a - b;
+      }
     }
   }
-  const float val = (BLK > 0) ? sm_row[c] * p.cb : sm_row[c];
-  store_out(p, ((size_t)n * p.Hq + (size_t)h * G + r) * D + c, val);
+#pragma unroll
+  for (int len = E; len < BLK; len <<= 1) {
+    const int m = len / E;
+    const bool upper = (lane & m) != 0;
+#pragma unroll
+    for (int i = 0; i < E; ++i) {
+      const float other = __shfl_xor_sync(0xffffffffu, v[i], m);
+      v[i] = upper ? (other - v[i]) : (v[i] + other);
+    }
+  }
 }
 
-template <int D, int BLK, int HG>
-__global__ void __launch_bounds__(kAttnThreads, 3) kvq_decode_kernel(const AttnParams p) {
-  using S = AttnSmem<D>;
-  constexpr int W = D / 32;    // code words of one token row per thread (QK)
-  constexpr int WP = D / 64;   // code words of one token row per thread group (PV)
-  constexpr int NT = D / 8;    // PV n-tiles
-  constexpr int KS = D / 16;   // QK k-steps
-  constexpr int C = D / 4;     // channels of one query row per thread
+
+template <int D, int BLK, int HG, int NC>
+__global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kernel(const AttnParams p) {
+  using S = AttnSmem<D, HG, NC>;
   constexpr int NSUB = kAttnWarps / HG;  // warps per head
-  constexpr int NST = 12 / HG;           // ring stages (a multiple of NSUB)
-  constexpr int HPB = S::kHeadPageBytes;
-  constexpr int PGB = HG * HPB;          // one page of HG heads
-  constexpr int STB = 2 * PGB;           // one stage = two pages
-  static_assert(NST * STB == S::kRingBytes, "ring size");
+  constexpr int R = kWarpRing;
+  constexpr int SLOT = S::kSlotBytes;
+  constexpr int KW = D / 32;   // K-row words per thread (QK)
+  constexpr int KM = KW / 2;   // QK MMAs per nibble half (32 codes of a row each)
+  constexpr int VW = D / 64;   // V-row words per thread (PV)
+  constexpr int MT = D / 16;   // PV m-tiles (16 channels each)
+  constexpr int NR = 4 * NC;   // query rows per head, padded
+  constexpr int E = D / 32;    // row elements per lane in warp-level row work
   extern __shared__ __align__(128) uint8_t smem[];
+  float* res = reinterpret_cast<float*>(smem + S::kOffRes);
+  float* qs = reinterpret_cast<float*>(smem + S::kOffQ);
+  float* qinfo = reinterpret_cast<float*>(smem + S::kOffQInfo);
+  int8_t* q8 = reinterpret_cast<int8_t*>(smem + S::kOffQ8);
   int* pids = reinterpret_cast<int*>(smem + S::kOffPid);
-  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + S::kOffBar);
-  int* cnt = reinterpret_cast<int*>(smem + S::kOffCnt);
-  int* sflags = reinterpret_cast<int*>(smem + S::kOffFlag);
+  int* sflag = reinterpret_cast<int*>(smem + S::kOffFlag);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tig = lane & 3;
   const int hw = warp % HG, sub = warp / HG;
-  const int split = blockIdx.x, hg = blockIdx.y, n = blockIdx.z;
-  const int h = hg * HG + hw;
+  const int split = blockIdx.x, hgi = blockIdx.y, n = blockIdx.z;
   const int G = p.G;
   const unsigned FULL = 0xffffffffu;
 
-  // let a dependent combine kernel get scheduled early; it waits for this grid
-  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
-
+  // Page ids of the split's range (the page-table row is max_pages long, so
+  // they are read before the context length is known), the context length,
+  // and the query rows of the CTA's heads (fp32, rows >= G zero).
+  const int p_begin = split * p.pages_per_split;
+  const int p_cap = min(p_begin + p.pages_per_split, p.max_pages);
+  const int32_t* pt_row = p.page_table + (size_t)n * p.max_pages + p_begin;
+  for (int i = tid; i < p_cap - p_begin && i < kMaxPids; i += kAttnThreads) pids[i] = pt_row[i];
   int ctx = p.ctx_lens[n];
+  for (int i = tid; i < S::kRows * (D / 8); i += kAttnThreads) {
+    const int row = i / (D / 8), c8 = i % (D / 8);
+    const int hh = row / NR, r = row % NR;
+    float v[8];
+    if (r < G) {
+      const uint4 u = *reinterpret_cast<const uint4*>(
+          p.q + ((size_t)n * p.Hq + (size_t)(hgi * HG + hh) * G + r) * D + 8 * c8);
+      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        v[2 * e] = __uint_as_float(w4[e] << 16);
+        v[2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
+      }
+    } else {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) v[e] = 0.0f;
+    }
+    float4* dst = reinterpret_cast<float4*>(qs + row * D + 8 * c8);
+    dst[0] = make_float4(v[0], v[1], v[2], v[3]);
+    dst[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
   const int cap = p.max_pages * 16;
   if (ctx < 0 || ctx > cap) {
     if (tid == 0) record_error(KVQ_ERR_OUT_OF_RANGE);
     ctx = ctx < 0 ? 0 : cap;
   }
   const int n_pages = (ctx + 15) >> 4;
-  const int p_begin = split * p.pages_per_split;
-  const int p_end = min(p_begin + p.pages_per_split, n_pages);
-  const int npg = max(p_end - p_begin, 0);
-  const int n_tasks = (npg + 1) / 2;
-  const int32_t* pt_row = p.page_table + (size_t)n * p.max_pages + p_begin;
+  const int npg = max(min(p_begin + p.pages_per_split, n_pages) - p_begin, 0);
+  __syncthreads();
 
-  for (int i = tid; i < npg && i < kMaxPids; i += kAttnThreads) pids[i] = pt_row[i];
-  if (tid == 0) {
-    for (int st = 0; st < NST; ++st) {
-      mbar_init(smem_addr(&bars[st]), 1);
-      cnt[st] = 0;
+  // ---- this warp's page stream: pages sub, sub + NSUB, ... of head hw -----
+  // fetch(k) copies the warp's k-th page into ring slot k % R (one commit
+  // group per call, empty past the end); bit k % R of `valid` says whether
+  // the slot holds a page. Lane l copies 16-byte chunks l, l + 32, ... of the
+  // codes; lanes 0..3 one chunk of the scales, lanes 4..7 of the zeros.
+  uint8_t* ring = smem + warp * (R * SLOT);
+  const uint32_t ring_lane = smem_addr(ring) + lane * 16;
+  const size_t head_off = (size_t)hgi * HG + hw;
+  const uint8_t* code_lane = p.cache + head_off * (16 * D) + lane * 16;
+  const uint16_t* sz_lane = (lane < 4 ? p.scales : p.zeros) + head_off * 32 + (lane & 3) * 8;
+  const size_t code_page = (size_t)p.Hkv * (16 * D);  // bytes per page
+  const size_t sz_page = (size_t)p.Hkv * 32;          // fp16 per page
+  uint32_t valid = 0;
+  auto fetch = [&](int k) {
+    const int t = sub + k * NSUB;
+    const int slot = k % R;
+    bool ok = false;
+    if (t < npg) {
+      const int id = (t < kMaxPids) ? pids[t] : pt_row[t];
+      ok = id >= 0 && id < p.num_pages;
+      if (ok) {
+        const uint8_t* src = code_lane + (size_t)id * code_page;
+        const uint32_t dst = ring_lane + slot * SLOT;
+#pragma unroll
+        for (int j = 0; j < D / 32; ++j) cp_async_16(dst + 512 * j, src + 512 * j);
+        cp_async_16_if(dst + 16 * D, sz_lane + (size_t)id * sz_page, lane < 8);
+      } else if (lane == 0) {
+        record_error(KVQ_ERR_OUT_OF_RANGE);
+      }
     }
-    mbar_init_fence();
+    valid = ok ? (valid | (1u << slot)) : (valid & ~(1u << slot));
+    cp_async_commit();
+  };
+#pragma unroll
+  for (int k = 0; k < R - 1; ++k) fetch(k);
+
+  // ---- q~ = R q * (softmax_scale * log2 e) while the first pages land -----
+  // One warp per row. Limbs: q0 = rint(q~ / sigma), q1 = rint((q~ - q0 sigma)
+  // * 256 / sigma), sigma = max|q~| / 127. They are stored in B-fragment
+  // order: element 8w + j goes to byte tig*8KW + ((m*2 + (j&1))*2 + h)*4 +
+  // (j>>1) of its limb's array, w = KW*tig + 2m + h, so that thread tig reads
+  // its fragments as 8KW contiguous bytes.
+  for (int row = warp; row < S::kRows; row += kAttnWarps) {
+    const float* rp = qs + row * D;
+    float v[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) v[e] = rp[E * lane + e];
+    if constexpr (BLK > 0) warp_fwht<D, BLK>(v, lane);
+    float amax = 0.0f, sum = 0.0f;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      v[e] *= p.qmul;
+      amax = fmaxf(amax, fabsf(v[e]));
+      sum += v[e];
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o));
+      sum += __shfl_xor_sync(FULL, sum, o);
+    }
+    const float sigma = amax / 127.0f;
+    const float inv = (amax > 0.0f) ? 127.0f / amax : 0.0f;
+    if (lane == 0) {
+      qinfo[row * 4 + 0] = sigma * (1.0f / 4096.0f);
+      qinfo[row * 4 + 1] = sum;
+    }
+    int8_t* l0 = q8 + row * 2 * D;
+    int8_t* l1 = l0 + D;
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const int el = E * lane + e, w = el >> 3, j = el & 7;
+      const int tw = w / KW, rw = w % KW;
+      const int off = tw * (8 * KW) + (((rw >> 1) * 2 + (j & 1)) * 2 + (rw & 1)) * 4 + (j >> 1);
+      const float a = __fmul_rn(v[e], inv);
+      const float q0 = rintf(a);
+      const float q1 = fminf(fmaxf(rintf(__fmul_rn(__fsub_rn(a, q0), 256.0f)), -127.0f), 127.0f);
+      l0[off] = (int8_t)(int)q0;
+      l1[off] = (int8_t)(int)q1;
+    }
   }
   __syncthreads();
 
-  // Fill stage t % NST with task t (pages 2t, 2t+1 of the range); one thread.
-  auto issue = [&](int t) {
-    const int st = t % NST;
-    const uint32_t bar = smem_addr(&bars[st]);
-    const uint32_t dst = smem_addr(smem + st * STB);
-    int ids[2];
-    bool ok[2];
+  // B fragments of QK: column g is limb g&1 of query row 4c + g/2 of head hw.
+  // MMA (m, half) of thread tig: b0 = bytes of k-group tig, b1 of k-group
+  // 4 + tig; their codes are the low (half 0) or high (half 1) nibbles of K
+  // words KW*tig + 2m (b0) and KW*tig + 2m + 1 (b1).
+  uint32_t bq[NC][KM][2][2];
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      const int i = 2 * t + j;
-      ids[j] = (i < npg) ? (i < kMaxPids ? pids[i] : pt_row[i]) : INT_MIN;
-      ok[j] = ids[j] >= 0 && ids[j] < p.num_pages;
-      if (ids[j] != INT_MIN && !ok[j]) record_error(KVQ_ERR_OUT_OF_RANGE);
-    }
-    sflags[st] = (ok[0] ? 1 : 0) | (ok[1] ? 2 : 0);
-    const uint32_t bytes = (ok[0] ? PGB : 0) + (ok[1] ? PGB : 0);
-    if (bytes == 0) {
-      mbar_arrive(bar);
-      return;
-    }
-    mbar_arrive_expect_tx(bar, bytes);
+  for (int c = 0; c < NC; ++c) {
+    const int row = hw * NR + 4 * c + (g >> 1);
+    const uint8_t* base = reinterpret_cast<const uint8_t*>(q8 + row * 2 * D + (g & 1) * D) + tig * (8 * KW);
 #pragma unroll
-    for (int j = 0; j < 2; ++j) {
-      if (!ok[j]) continue;
-      const size_t ph = (size_t)ids[j] * p.Hkv + (size_t)hg * HG;  // first page-head of the group
-      const uint32_t d = dst + j * PGB;
-      bulk_g2s(d, p.cache + ph * (16 * D), HG * 16 * D, bar);
-      bulk_g2s(d + HG * 16 * D, p.scales + ph * 32, HG * 64, bar);
-      bulk_g2s(d + HG * 16 * D + HG * 64, p.zeros + ph * 32, HG * 64, bar);
-    }
-  };
-  if (tid == 0)
-    for (int t = 0; t < NST && t < n_tasks; ++t) issue(t);
-
-  // ---- q~ = R q * (softmax_scale * log2 e), in registers -------------------
-  // Thread (g, tig) holds query row g (query head h*G + g) channels
-  // [C tig, C tig + C); rows >= G are zero.
-  float qv[C];
-  if (g < G) {
-    const uint4* src = reinterpret_cast<const uint4*>(p.q + ((size_t)n * p.Hq + (size_t)h * G + g) * D + C * tig);
-#pragma unroll
-    for (int i = 0; i < C / 8; ++i) {
-      const uint4 u = src[i];
-      const uint32_t w4[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        qv[8 * i + 2 * e] = __uint_as_float(w4[e] << 16);
-        qv[8 * i + 2 * e + 1] = __uint_as_float(w4[e] & 0xffff0000u);
-      }
-    }
-  } else {
-#pragma unroll
-    for (int i = 0; i < C; ++i) qv[i] = 0.0f;
-  }
-  if constexpr (BLK > 0) quad_fwht<C, BLK>(qv, tig);
-  float amax = 0.0f, qsum = 0.0f;
-#pragma unroll
-  for (int i = 0; i < C; ++i) {
-    qv[i] *= p.qmul;
-    amax = fmaxf(amax, fabsf(qv[i]));
-    qsum += qv[i];
-  }
-  amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 1));
-  amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, 2));
-  qsum += __shfl_xor_sync(FULL, qsum, 1);
-  qsum += __shfl_xor_sync(FULL, qsum, 2);
-  // power-of-two prescale so the largest |q~| lands in [2^13, 2^14): both the
-  // hi and lo fp16 parts stay normal
-  int kexp = (amax > 0.0f) ? 13 - ilogbf(amax) : 0;
-  kexp = max(-100, min(100, kexp));
-  const float up = ldexpf(1.0f, kexp);
-  const float acc_to_true = ldexpf(1.0f, -kexp);
-
-  // A fragments of QK. k-step 2u takes channel pairs (8m, 8m+4), (8m+2, 8m+6)
-  // of word m = W tig + u; k-step 2u+1 takes (8m+1, 8m+5), (8m+3, 8m+7) whose
-  // codes arrive x16, so its q~ is divided by 16.
-  uint32_t aq[KS][4];
-#pragma unroll
-  for (int u = 0; u < W; ++u) {
-#pragma unroll
-    for (int t = 0; t < 2; ++t) {
-      const float f = t ? up * 0.0625f : up;
-      split_pair(qv[8 * u + t] * f, qv[8 * u + t + 4] * f, aq[2 * u + t][0], aq[2 * u + t][1]);
-      split_pair(qv[8 * u + t + 2] * f, qv[8 * u + t + 6] * f, aq[2 * u + t][2], aq[2 * u + t][3]);
+    for (int m = 0; m < KM; ++m) {
+      const uint4 f4 = *reinterpret_cast<const uint4*>(base + 16 * m);
+      bq[c][m][0][0] = f4.x;
+      bq[c][m][0][1] = f4.y;
+      bq[c][m][1][0] = f4.z;
+      bq[c][m][1][1] = f4.w;
     }
   }
-
-  // ---- page stream: this warp takes tasks sub, sub + NSUB, ... -------------
-  float o[NT][4];
+  // this thread's QK results belong to query row 4c + tig of head hw
+  float qsc[NC], qsm[NC];
+  bool hv[NC];
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) o[nt][0] = o[nt][1] = o[nt][2] = o[nt][3] = 0.0f;
-  float m_run = -INFINITY, l_run = 0.0f, zs_run = 0.0f;
+  for (int c = 0; c < NC; ++c) {
+    const int row = hw * NR + 4 * c + tig;
+    qsc[c] = qinfo[row * 4 + 0];
+    qsm[c] = qinfo[row * 4 + 1];
+    hv[c] = 4 * c + tig < G;
+  }
+  // PV B fragments: column g wants tokens 2tig, 2tig+1 (held by lanes
+  // 8tig + g/2 and 8tig + 4 + g/2 as their token g) and 2tig+8, 2tig+9 (the
+  // same lanes' token g+8)
+  const int la = 8 * tig + (g >> 1), lb = la + 4;
 
-  for (int t = sub; t < n_tasks; t += NSUB) {
-    const int st = t % NST;
-    const bool waited = mbar_wait_bounded(smem_addr(&bars[st]), (t / NST) & 1);
-    if (!__all_sync(FULL, waited)) break;
-    const int fl = sflags[st];
-    const uint8_t* stg = smem + st * STB;
-    const int tok0 = (p_begin + 2 * t) * 16;  // first token of the task
+  float o[NC][MT][4];
+#pragma unroll
+  for (int c = 0; c < NC; ++c)
+#pragma unroll
+    for (int i = 0; i < MT; ++i) o[c][i][0] = o[c][i][1] = o[c][i][2] = o[c][i][3] = 0.0f;
+  float m_run[NC], l_run[NC], zs_run[NC];
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+    m_run[c] = -INFINITY;
+    l_run[c] = 0.0f;
+    zs_run[c] = 0.0f;
+  }
+  const int tok_base = p_begin * 16;
 
-#pragma unroll
-    for (int pg = 0; pg < 2; ++pg) {
-      if (!((fl >> pg) & 1)) continue;
-      const uint8_t* kb = stg + pg * PGB + hw * (16 * D);              // K block, then V block
-      const uint8_t* sz = stg + pg * PGB + HG * 16 * D + hw * 64;      // 16 K then 16 V scales
-      const uint8_t* zz = stg + pg * PGB + HG * 16 * D + HG * 64 + hw * 64;
-      const int tp = tok0 + 16 * pg;
-
-      // QK on the codes: n-tile nt = token rows 8nt + g
-      float acc[2][4];
-#pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        acc[nt][0] = acc[nt][1] = acc[nt][2] = acc[nt][3] = 0.0f;
-        const uint8_t* row = kb + (8 * nt + g) * (D / 2) + tig * (4 * W);
-        uint32_t wk[W];
-        if constexpr (W == 4) {
-          const uint4 t4 = *reinterpret_cast<const uint4*>(row);
-          wk[0] = t4.x; wk[1] = t4.y; wk[2] = t4.z; wk[3] = t4.w;
-        } else {
-          const uint2 t2 = *reinterpret_cast<const uint2*>(row);
-          wk[0] = t2.x; wk[1] = t2.y;
-        }
-#pragma unroll
-        for (int u = 0; u < W; ++u) {
-          const uint32_t w = wk[u], w8 = wk[u] >> 8;
-          mma_f16_16816(acc[nt], aq[2 * u], codes_to_half2<false>(w), codes_to_half2<false>(w8));
-          mma_f16_16816(acc[nt], aq[2 * u + 1], codes_to_half2<true>(w), codes_to_half2<true>(w8));
-        }
-      }
-      // logits (base 2) of tokens 2tig, 2tig+1 (nt 0) and 2tig+8, 2tig+9 (nt 1)
-      const float2 skA = __half22float2(reinterpret_cast<const __half2*>(sz)[tig]);
-      const float2 skB = __half22float2(reinterpret_cast<const __half2*>(sz)[tig + 4]);
-      const float2 zkA = __half22float2(reinterpret_cast<const __half2*>(zz)[tig]);
-      const float2 zkB = __half22float2(reinterpret_cast<const __half2*>(zz)[tig + 4]);
-      float lg[4];
-      lg[0] = fmaf((acc[0][0] + acc[0][2]) * acc_to_true, skA.x, zkA.x * qsum);
-      lg[1] = fmaf((acc[0][1] + acc[0][3]) * acc_to_true, skA.y, zkA.y * qsum);
-      lg[2] = fmaf((acc[1][0] + acc[1][2]) * acc_to_true, skB.x, zkB.x * qsum);
-      lg[3] = fmaf((acc[1][1] + acc[1][3]) * acc_to_true, skB.y, zkB.y * qsum);
-      const int t0 = tp + 2 * tig;
-      if (t0 >= ctx) lg[0] = -INFINITY;
-      if (t0 + 1 >= ctx) lg[1] = -INFINITY;
-      if (t0 + 8 >= ctx) lg[2] = -INFINITY;
-      if (t0 + 9 >= ctx) lg[3] = -INFINITY;
-
-      // online softmax, rescaling only when the running maximum grows
-      float pm = fmaxf(fmaxf(lg[0], lg[1]), fmaxf(lg[2], lg[3]));
-      pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 1));
-      pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 2));
-      if (pm > m_run) {
-        const float alpha = fast_exp2(m_run - pm);
-#pragma unroll
-        for (int nt = 0; nt < NT; ++nt) {
-          o[nt][0] *= alpha; o[nt][1] *= alpha; o[nt][2] *= alpha; o[nt][3] *= alpha;
-        }
-        l_run *= alpha;
-        zs_run *= alpha;
-        m_run = pm;
-      }
-      const float2 svA = __half22float2(reinterpret_cast<const __half2*>(sz + 32)[tig]);
-      const float2 svB = __half22float2(reinterpret_cast<const __half2*>(sz + 32)[tig + 4]);
-      const float2 zvA = __half22float2(reinterpret_cast<const __half2*>(zz + 32)[tig]);
-      const float2 zvB = __half22float2(reinterpret_cast<const __half2*>(zz + 32)[tig + 4]);
-      const float sv[4] = {svA.x, svA.y, svB.x, svB.y};
-      const float zv[4] = {zvA.x, zvA.y, zvB.x, zvB.y};
-      float pv[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const float pr = (lg[j] == -INFINITY) ? 0.0f : fast_exp2(lg[j] - m_run);
-        l_run += pr;
-        pv[j] = (pr > 0.0f) ? pr * sv[j] : 0.0f;
-        zs_run += (pr > 0.0f) ? pr * zv[j] : 0.0f;
-      }
-      uint32_t ap[4];
-      split_pair(pv[0], pv[1], ap[0], ap[1]);
-      split_pair(pv[2], pv[3], ap[2], ap[3]);
-
-      // PV on the codes: B = code pairs of token rows (2tig, 2tig+1),
-      // (2tig+8, 2tig+9); thread group g supplies channels [g*NT, g*NT + NT)
+  for (int k = 0; sub + k * NSUB < npg; ++k) {
+    const int t = sub + k * NSUB;
+    fetch(k + R - 1);
+    cp_async_wait<R - 1>();  // page k has landed (this lane's copies)
+    __syncwarp();            // ... and every other lane's
+    if ((valid >> (k % R)) & 1u) {
+      const uint8_t* kb = ring + (k % R) * SLOT;  // K block [16][D/2], then V block
       const uint8_t* vb = kb + 8 * D;
-      uint32_t wv[4][WP];
-      const int rows_v[4] = {2 * tig, 2 * tig + 1, 2 * tig + 8, 2 * tig + 9};
+      const __half* scl = reinterpret_cast<const __half*>(kb + 16 * D);       // 16 K, then 16 V scales
+      const __half* zer = reinterpret_cast<const __half*>(kb + 16 * D + 64);  // zeros, likewise
+
+      // QK: A = code bytes of tokens g (rows 0..7) and g+8 (rows 8..15)
+      uint32_t ka[KW], kc[KW];
+      lds_words<KW>(kb + g * (D / 2) + tig * (4 * KW), ka);
+      lds_words<KW>(kb + (g + 8) * (D / 2) + tig * (4 * KW), kc);
+      int accl[NC][4], acch[NC][4];
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const uint8_t* row = vb + rows_v[j] * (D / 2) + g * (4 * WP);
-        if constexpr (WP == 2) {
-          const uint2 t2 = *reinterpret_cast<const uint2*>(row);
-          wv[j][0] = t2.x; wv[j][1] = t2.y;
-        } else {
-          wv[j][0] = *reinterpret_cast<const uint32_t*>(row);
+      for (int m = 0; m < KM; ++m) {
+        const uint32_t x0 = ka[2 * m], x1 = ka[2 * m + 1], y0 = kc[2 * m], y1 = kc[2 * m + 1];
+        const uint32_t al[4] = {x0 & 0x0F0F0F0Fu, y0 & 0x0F0F0F0Fu, x1 & 0x0F0F0F0Fu, y1 & 0x0F0F0F0Fu};
+        const uint32_t ah[4] = {x0 & 0xF0F0F0F0u, y0 & 0xF0F0F0F0u, x1 & 0xF0F0F0F0u, y1 & 0xF0F0F0F0u};
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          if (m == 0) {
+            mma_u8s8_16832_z(accl[c], al, bq[c][0][0][0], bq[c][0][0][1]);
+            mma_u8s8_16832_z(acch[c], ah, bq[c][0][1][0], bq[c][0][1][1]);
+          } else {
+            mma_u8s8_16832(accl[c], al, bq[c][m][0][0], bq[c][m][0][1]);
+            mma_u8s8_16832(acch[c], ah, bq[c][m][1][0], bq[c][m][1][1]);
+          }
         }
       }
+      const float sk0 = __half2float(scl[g]), sk1 = __half2float(scl[g + 8]);
+      const float zk0 = __half2float(zer[g]), zk1 = __half2float(zer[g + 8]);
+      const float sv0 = __half2float(scl[16 + g]), sv1 = __half2float(scl[24 + g]);
+      const float zv0 = __half2float(zer[16 + g]), zv1 = __half2float(zer[24 + g]);
+      const int tok = tok_base + 16 * t;
+      const bool tail = tok + 16 > ctx;
+
+      uint32_t bp[NC][2];
 #pragma unroll
-      for (int u = 0; u < WP; ++u) {
+      for (int c = 0; c < NC; ++c) {
+        // logits (base 2) of tokens g and g+8 for query row 4c + tig
+        // 16 S_limb = 16 acc_lo + acc_hi; T = 256 (16 S_0) + 16 S_1, exact in s32
+        const int T0 = (accl[c][0] * 16 + acch[c][0]) * 256 + (accl[c][1] * 16 + acch[c][1]);
+        const int T1 = (accl[c][2] * 16 + acch[c][2]) * 256 + (accl[c][3] * 16 + acch[c][3]);
+        float lg0 = fmaf((float)T0 * qsc[c], sk0, zk0 * qsm[c]);
+        float lg1 = fmaf((float)T1 * qsc[c], sk1, zk1 * qsm[c]);
+        if (!hv[c]) lg0 = lg1 = -INFINITY;
+        if (tail) {
+          if (tok + g >= ctx) lg0 = -INFINITY;
+          if (tok + g + 8 >= ctx) lg1 = -INFINITY;
+        }
+        // online softmax, rescaling only when the running maximum grows
+        float pm = fmaxf(lg0, lg1);
+        pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 4));
+        pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 8));
+        pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 16));
+        if (pm > m_run[c]) {
+          const float alpha = (m_run[c] == -INFINITY) ? 0.0f : fast_exp2(m_run[c] - pm);
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {
-          const uint32_t sel = k | (k << 4) | ((4 + k) << 8) | ((4 + k) << 12);
-          const uint32_t x01 = prmt(wv[0][u], wv[1][u], sel);
-          const uint32_t x23 = prmt(wv[2][u], wv[3][u], sel);
-          mma_f16_16816(o[8 * u + 2 * k], ap, codes_to_half2<false>(x01), codes_to_half2<false>(x23));
-          mma_f16_16816(o[8 * u + 2 * k + 1], ap, codes_to_half2<true>(x01), codes_to_half2<true>(x23));
+          for (int i = 0; i < MT; ++i) {
+            o[c][i][0] *= alpha; o[c][i][1] *= alpha; o[c][i][2] *= alpha; o[c][i][3] *= alpha;
+          }
+          l_run[c] *= alpha;
+          zs_run[c] *= alpha;
+          m_run[c] = pm;
+        }
+        const float p0 = (lg0 == -INFINITY) ? 0.0f : fast_exp2(lg0 - m_run[c]);
+        const float p1 = (lg1 == -INFINITY) ? 0.0f : fast_exp2(lg1 - m_run[c]);
+        l_run[c] += p0 + p1;
+        zs_run[c] = fmaf(p0, zv0, fmaf(p1, zv1, zs_run[c]));
+        const float P0 = p0 * sv0, P1 = p1 * sv1;
+        // move p*s_v to the PV B layout (4 tokens of column g)
+        const float q0 = __shfl_sync(FULL, P0, la), q1 = __shfl_sync(FULL, P0, lb);
+        const float q2 = __shfl_sync(FULL, P1, la), q3 = __shfl_sync(FULL, P1, lb);
+        bp[c][0] = hilo_pair(q0, q1, g & 1);
+        bp[c][1] = hilo_pair(q2, q3, g & 1);
+      }
+
+      // PV: A = codes^T; rows g / g+8 of m-tile 4u+j are channels
+      // 8cb + {0,1,4,5}[j] / 8cb + {2,3,6,7}[j] (cb = VW g + u); k-slots
+      // 2tig, 2tig+1, 2tig+8, 2tig+9 are those tokens
+      uint32_t va[VW], vb2[VW], vc[VW], vd[VW];
+      lds_words<VW>(vb + (2 * tig) * (D / 2) + g * (4 * VW), va);
+      lds_words<VW>(vb + (2 * tig + 1) * (D / 2) + g * (4 * VW), vb2);
+      lds_words<VW>(vb + (2 * tig + 8) * (D / 2) + g * (4 * VW), vc);
+      lds_words<VW>(vb + (2 * tig + 9) * (D / 2) + g * (4 * VW), vd);
+#pragma unroll
+      for (int u = 0; u < VW; ++u) {
+        const uint32_t xl = prmt(va[u], vb2[u], 0x5410), xh = prmt(va[u], vb2[u], 0x7632);
+        const uint32_t yl = prmt(vc[u], vd[u], 0x5410), yh = prmt(vc[u], vd[u], 0x7632);
+        const uint32_t xl8 = xl >> 8, xh8 = xh >> 8, yl8 = yl >> 8, yh8 = yh >> 8;
+        const uint32_t m0[4] = {codes_to_half2<false>(xl), codes_to_half2<false>(xl8),
+                                codes_to_half2<false>(yl), codes_to_half2<false>(yl8)};
+        const uint32_t m1[4] = {codes_to_half2<true>(xl), codes_to_half2<true>(xl8),
+                                codes_to_half2<true>(yl), codes_to_half2<true>(yl8)};
+        const uint32_t m2[4] = {codes_to_half2<false>(xh), codes_to_half2<false>(xh8),
+                                codes_to_half2<false>(yh), codes_to_half2<false>(yh8)};
+        const uint32_t m3[4] = {codes_to_half2<true>(xh), codes_to_half2<true>(xh8),
+                                codes_to_half2<true>(yh), codes_to_half2<true>(yh8)};
+#pragma unroll
+        for (int c = 0; c < NC; ++c) {
+          mma_f16_16816(o[c][4 * u + 0], m0, bp[c][0], bp[c][1]);
+          mma_f16_16816(o[c][4 * u + 1], m1, bp[c][0], bp[c][1]);
+          mma_f16_16816(o[c][4 * u + 2], m2, bp[c][0], bp[c][1]);
+          mma_f16_16816(o[c][4 * u + 3], m3, bp[c][0], bp[c][1]);
         }
       }
     }
-    // release the stage; the last of its HG consumer warps refills it
-    __syncwarp();
-    if (lane == 0) {
-      const int old = atomicAdd(&cnt[st], 1);
-      if (old == HG - 1) {
-        cnt[st] = 0;
-        if (t + NST < n_tasks) issue(t + NST);
+    __syncwarp();  // the slot is read out before a later fetch refills it
+  }
+  cp_async_wait<0>();
+
+  // ---- per-warp result: O[row][channel], (m, l, zs) per row -----------------
+#pragma unroll
+  for (int c = 0; c < NC; ++c) {
+#pragma unroll
+    for (int o2 = 4; o2 < 32; o2 <<= 1) {
+      l_run[c] += __shfl_xor_sync(FULL, l_run[c], o2);
+      zs_run[c] += __shfl_xor_sync(FULL, zs_run[c], o2);
+    }
+  }
+  {
+    float* mine = res + warp * S::kResFloats;
+#pragma unroll
+    for (int c = 0; c < NC; ++c) {
+      float* orow = mine + (4 * c + tig) * D;
+#pragma unroll
+      for (int u = 0; u < VW; ++u) {
+        const int cb = VW * g + u;
+        const float* t0 = o[c][4 * u];
+        const float* t1 = o[c][4 * u + 1];
+        const float* t2 = o[c][4 * u + 2];
+        const float* t3 = o[c][4 * u + 3];
+        // hi + lo columns; the odd m-tiles carried 16c
+        float4* dst = reinterpret_cast<float4*>(orow + 8 * cb);
+        dst[0] = make_float4(t0[0] + t0[1], (t1[0] + t1[1]) * 0.0625f, t0[2] + t0[3], (t1[2] + t1[3]) * 0.0625f);
+        dst[1] = make_float4(t2[0] + t2[1], (t3[0] + t3[1]) * 0.0625f, t2[2] + t2[3], (t3[2] + t3[3]) * 0.0625f);
+      }
+      if (g == 0) {
+        float* ml = mine + NR * D + (4 * c + tig) * 4;
+        ml[0] = m_run[c];
+        ml[1] = l_run[c];
+        ml[2] = zs_run[c];
       }
     }
   }
-  // (a warp whose wait ran out stops early; the error word records it)
+  __syncthreads();
 
-  // ---- per-warp result: O slice of row g, (m, l, zs) -----------------------
-  l_run += __shfl_xor_sync(FULL, l_run, 1);
-  l_run += __shfl_xor_sync(FULL, l_run, 2);
-  zs_run += __shfl_xor_sync(FULL, zs_run, 1);
-  zs_run += __shfl_xor_sync(FULL, zs_run, 2);
-  float ov[C];
+  // ---- merge the NSUB warps of each head: output rows or a partial result --
+  const bool single = p.n_splits == 1;
+  for (int e = tid; e < HG * G * (D / 4); e += kAttnThreads) {
+    const int hh = e / (G * (D / 4)), r = (e / (D / 4)) % G, c4 = 4 * (e % (D / 4));
+    float mw[NSUB];
+    float M = -INFINITY;
 #pragma unroll
-  for (int nt = 0; nt < NT; ++nt) {
-    const float sc = (nt & 1) ? 0.0625f : 1.0f;  // odd n-tiles carried 16c
-    ov[nt] = (o[nt][0] + o[nt][2]) * sc;          // channel C tig + nt
-    ov[NT + nt] = (o[nt][1] + o[nt][3]) * sc;     // channel C tig + NT + nt
-  }
-
-  // Merge (m, l, zs, O) sources into this thread's registers.
-  auto merge_in = [&](float ms, float ls, float zss, const float* os) {
-    const float M = fmaxf(m_run, ms);
-    if (M == -INFINITY) return;
-    const float a = (m_run == -INFINITY) ? 0.0f : fast_exp2(m_run - M);
-    const float b = (ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
-#pragma unroll
-    for (int i = 0; i < C; ++i) ov[i] = ov[i] * a + os[i] * b;
-    l_run = l_run * a + ls * b;
-    zs_run = zs_run * a + zss * b;
-    m_run = M;
-  };
-
-  __syncthreads();  // every copy has landed and been consumed: slots may overlay the ring
-  float* slots = reinterpret_cast<float*>(smem);
-  auto put_local = [&](float* slot) {
-#pragma unroll
-    for (int i = 0; i < C; ++i) slot[g * D + C * tig + i] = ov[i];
-    if (tig == 0) {
-      slot[8 * D + 4 * g] = m_run;
-      slot[8 * D + 4 * g + 1] = l_run;
-      slot[8 * D + 4 * g + 2] = zs_run;
+    for (int s2 = 0; s2 < NSUB; ++s2) {
+      mw[s2] = res[(hh + HG * s2) * S::kResFloats + NR * D + r * 4];
+      M = fmaxf(M, mw[s2]);
     }
-  };
-  auto take = [&](const float* slot) {
-    float os[C];
+    float4 O = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    float L = 0.0f, Z = 0.0f;
+    if (M != -INFINITY) {
 #pragma unroll
-    for (int i = 0; i < C; ++i) os[i] = slot[g * D + C * tig + i];
-    merge_in(slot[8 * D + 4 * g], slot[8 * D + 4 * g + 1], slot[8 * D + 4 * g + 2], os);
-  };
-  if constexpr (NSUB > 1) {
-    // warps that shared a head hand their results to warp hw
-    if (sub > 0) put_local(slots + warp * S::kSlotFloats);
-    __syncthreads();
-    if (sub == 0)
-      for (int j = 1; j < NSUB; ++j) take(slots + (hw + HG * j) * S::kSlotFloats);
-    __syncthreads();
-  }
-  const int cs = p.cluster_size;
-  if (cs > 1) {
-    // The cluster's CTAs merge into its first CTA along a binary tree: at
-    // level r, CTA rank + 2^r pushes its result into level-r buffer of CTA
-    // rank (remote shared-memory stores, fire and forget); after one cluster
-    // barrier the receiver merges it from its own shared memory.
-    constexpr int kPay = kAttnWarps * S::kSlotFloats;
-    static_assert(3 * kPay * 4 <= S::kUnionBytes, "three merge buffers must fit in the ring");
-    const int rank = (int)cluster_ctarank();
-    cluster_sync_all();  // every CTA of the cluster is past its page loop
-    int level = 0;
-    for (int stride = 1; stride < cs; stride <<= 1, ++level) {
-      float* buf = slots + level * kPay + hw * S::kSlotFloats;
-      const int rel = rank % (2 * stride);
-      if (rel == stride && sub == 0) {
-        const uint32_t to = (uint32_t)(rank - stride);
-#pragma unroll
-        for (int i = 0; i < C; i += 4)
-          st_dsmem_v4(buf + g * D + C * tig + i, to, ov[i], ov[i + 1], ov[i + 2], ov[i + 3]);
-        if (tig == 0) st_dsmem_v4(buf + 8 * D + 4 * g, to, m_run, l_run, zs_run, 0.0f);
+      for (int s2 = 0; s2 < NSUB; ++s2) {
+        const float* sl = res + (hh + HG * s2) * S::kResFloats;
+        const float wgt = (mw[s2] == -INFINITY) ? 0.0f : fast_exp2(mw[s2] - M);
+        const float4 v = *reinterpret_cast<const float4*>(sl + r * D + c4);
+        O.x = fmaf(wgt, v.x, O.x);
+        O.y = fmaf(wgt, v.y, O.y);
+        O.z = fmaf(wgt, v.z, O.z);
+        O.w = fmaf(wgt, v.w, O.w);
+        L = fmaf(wgt, sl[NR * D + r * 4 + 1], L);
+        Z = fmaf(wgt, sl[NR * D + r * 4 + 2], Z);
       }
-      cluster_sync_all();
-      if (rel == 0 && rank + stride < cs && sub == 0) take(buf);
     }
-    if (rank != 0) return;
+    if (single) {
+      const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
+      *reinterpret_cast<float4*>(qs + (hh * NR + r) * D + c4) =
+          make_float4((O.x + Z) * inv, (O.y + Z) * inv, (O.z + Z) * inv, (O.w + Z) * inv);
+    } else {
+      float* dst = p.ws_part + ((((size_t)n * p.Hkv + hgi * HG + hh) * p.n_splits + split) * G + r) * (D + 4);
+      *reinterpret_cast<float4*>(dst + c4) = make_float4(O.x + Z, O.y + Z, O.z + Z, O.w + Z);
+      if (c4 == 0) *reinterpret_cast<float2*>(dst + D) = make_float2(M, L);
+    }
   }
-  if (sub != 0) return;
 
-  if (p.n_parts == 1) {
-    const float inv_l = (l_run > 0.0f) ? 1.0f / l_run : 0.0f;
+  if (!single) {
+    // ---- ticket: the last split of this (sequence, head group) merges ------
+    // (every thread's partial stores are made visible device-wide before the
+    // barrier and thread 0's atomic; the last CTA reads the partials from L2
+    // with ld.cg, issued after its atomic returned and a barrier)
+    __threadfence();
+    __syncthreads();
+    int* ticket = p.ws_count + (size_t)n * (p.Hkv / HG) + hgi;
+    if (tid == 0) sflag[0] = (atomicAdd(ticket, 1) == p.n_splits - 1) ? 1 : 0;
+    __syncthreads();
+    if (!sflag[0]) return;
+    if (tid == 0) *ticket = 0;  // every split has counted: ready for the next call
+
+    // Merge of the splits. Thread (e, pp) first puts its loads in flight: the
+    // O + Z of output float4 e for splits pp, pp + P, ... (kMergeBatch of them;
+    // more splits take further rounds). Then one warp per query row reads the
+    // (M, L) of every split, reduces M with shuffles and leaves the weights
+    // 2^(M_s - M) and the merged L in shared memory.
+    constexpr int kMergeBatch = 20;
+    const int ns = p.n_splits;
+    const int rows = HG * G;
+    const int e4 = rows * (D / 4);
+    const int P = e4 >= kAttnThreads ? 1 : kAttnThreads / e4;
+    const size_t sstride = (size_t)G * (D + 4);  // floats between consecutive splits
+    float* wS = reinterpret_cast<float*>(smem + S::kOffMS);  // [rows][kMaxSplits] weights
+    float* lS = reinterpret_cast<float*>(smem + S::kOffLS);  // [rows] merged L
+    float4* part_o = reinterpret_cast<float4*>(smem + S::kOffPartO);  // [P][e4]
+    auto head_base = [&](int hh, int r) {
+      return p.ws_part + (((size_t)n * p.Hkv + hgi * HG + hh) * ns * G + r) * (D + 4);
+    };
+    const bool has_e = tid < e4 * P;
+    const int e = tid % e4, pp = tid / e4;
+    const int hh_e = e / (G * (D / 4)), r_e = (e / (D / 4)) % G, c4_e = 4 * (e % (D / 4));
+    const float* base_e = head_base(hh_e, r_e) + c4_e;
+    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    for (int s0 = 0; s0 < ns; s0 += kMergeBatch * P) {
+      // (M, L) of every (row, split) into shared memory first (they are needed
+      // first), then this thread's O + Z into registers (split indices
+      // clamped: the extra loads read a valid split and get weight 0)
+      float2* mlS = reinterpret_cast<float2*>(smem + S::kOffML);  // [rows][kMaxSplits]
+      if (s0 == 0) {
+        for (int i = tid; i < rows * ns; i += kAttnThreads) {
+          const int rr = i / ns, s2 = i % ns;
+          cp_async_8(smem_addr(mlS + rr * kMaxSplits + s2), head_base(rr / G, rr % G) + D + s2 * sstride);
+        }
+        cp_async_commit();
+      }
+      float4 v[kMergeBatch];
 #pragma unroll
-    for (int i = 0; i < C; ++i) ov[i] = (l_run > 0.0f) ? (ov[i] + zs_run) * inv_l : 0.0f;
-    if constexpr (BLK > 0) {
-      quad_fwht<C, BLK>(ov, tig);
+      for (int j = 0; j < kMergeBatch; ++j) {
+        const int s2 = min(s0 + pp + j * P, ns - 1);
+        v[j] = __ldcg(reinterpret_cast<const float4*>(base_e + s2 * sstride));
+      }
+      if (s0 == 0) {
+        cp_async_wait<0>();
+        __syncthreads();
+        // one warp per row: M by shuffles, the weights 2^(M_s - M) and L
+        for (int rr = warp; rr < rows; rr += kAttnWarps) {
+          float M = -INFINITY;
+          for (int s2 = lane; s2 < ns; s2 += 32) M = fmaxf(M, mlS[rr * kMaxSplits + s2].x);
 #pragma unroll
-      for (int i = 0; i < C; ++i) ov[i] *= p.cb;
+          for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o2));
+          float L = 0.0f;
+          for (int s2 = lane; s2 < ns; s2 += 32) {
+            const float2 ml = mlS[rr * kMaxSplits + s2];
+            const float wgt = (ml.x == -INFINITY) ? 0.0f : fast_exp2(ml.x - M);
+            wS[rr * kMaxSplits + s2] = wgt;
+            L = fmaf(wgt, ml.y, L);
+          }
+#pragma unroll
+          for (int o2 = 16; o2 > 0; o2 >>= 1) L += __shfl_xor_sync(FULL, L, o2);
+          if (lane == 0) lS[rr] = L;
+        }
+        __syncthreads();
+      }
+      if (has_e) {
+        const float* wrow = wS + (hh_e * G + r_e) * kMaxSplits;
+#pragma unroll
+        for (int j = 0; j < kMergeBatch; ++j) {
+          const int s2 = s0 + pp + j * P;
+          const float wgt = (s2 < ns) ? wrow[s2] : 0.0f;
+          acc.x = fmaf(wgt, v[j].x, acc.x);
+          acc.y = fmaf(wgt, v[j].y, acc.y);
+          acc.z = fmaf(wgt, v[j].z, acc.z);
+          acc.w = fmaf(wgt, v[j].w, acc.w);
+        }
+      }
     }
-    if (g < G) {
-      const size_t o_base = ((size_t)n * p.Hq + (size_t)h * G + g) * D + C * tig;
-#pragma unroll
-      for (int i = 0; i < C; ++i) store_out(p, o_base + i, ov[i]);
+    if (has_e) part_o[pp * e4 + e] = acc;
+    __syncthreads();
+    for (int i = tid; i < e4; i += kAttnThreads) {
+      const int hh = i / (G * (D / 4)), r = (i / (D / 4)) % G, c4 = 4 * (i % (D / 4));
+      float4 sum = part_o[i];
+      for (int q2 = 1; q2 < P; ++q2) {
+        const float4 w4 = part_o[q2 * e4 + i];
+        sum.x += w4.x; sum.y += w4.y; sum.z += w4.z; sum.w += w4.w;
+      }
+      const float L = lS[hh * G + r];
+      const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
+      *reinterpret_cast<float4*>(qs + (hh * NR + r) * D + c4) =
+          make_float4(sum.x * inv, sum.y * inv, sum.z * inv, sum.w * inv);
     }
-  } else if (g < G) {
-    const int part = split / cs;
-    float* dst = p.ws_part + ((((size_t)n * p.Hkv + h) * p.n_parts + part) * G + g) * (D + 2);
+  }
+  __syncthreads();
+
+  // ---- rotate back (one warp per query row) and store ---------------------
+  for (int rr = warp; rr < HG * G; rr += kAttnWarps) {
+    const int hh = rr / G, r = rr % G;
+    const float* rp = qs + (hh * NR + r) * D;
+    float v[E];
 #pragma unroll
-    for (int i = 0; i < C; ++i) dst[C * tig + i] = ov[i] + zs_run;
-    if (tig == 0) {
-      dst[D] = m_run;
-      dst[D + 1] = l_run;
-    }
+    for (int e2 = 0; e2 < E; ++e2) v[e2] = rp[E * lane + e2];
+    if constexpr (BLK > 0) warp_fwht<D, BLK>(v, lane);
+    const size_t o_base = ((size_t)n * p.Hq + (size_t)(hgi * HG + hh) * G + r) * D + E * lane;
+#pragma unroll
+    for (int e2 = 0; e2 < E; ++e2) store_out(p, o_base + e2, BLK > 0 ? v[e2] * p.cb : v[e2]);
   }
 }
 

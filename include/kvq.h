@@ -124,12 +124,13 @@ kvq_status kv_quant_write(const void* k, const void* v, const int64_t* slot_mapp
  * kvq_attn_workspace_size - bytes of device workspace paged_decode_attn_int4
  * needs for these shapes (0 when the call needs none) on this library's
  * current device (see kvq_set_device). The value depends on the shapes and on
- * how many thread-block clusters of the decode kernel that device holds at
- * once. Returns SIZE_MAX when the shapes are invalid or no device can be
- * queried.
+ * how many decode CTAs that device holds at once (the split count fills them
+ * in one wave). Returns SIZE_MAX when the shapes are invalid or no device can
+ * be queried.
  *
- * The workspace holds per-split partial results (fp32); it needs no
- * initialization.
+ * The workspace holds per-split partial results (fp32) and one ticket counter
+ * per (sequence, head group); it must be zero-filled before its first use,
+ * and every call leaves it zero-filled again.
  */
 size_t kvq_attn_workspace_size(const kvq_attn_desc* desc);
 
@@ -155,10 +156,9 @@ size_t kvq_attn_workspace_size(const kvq_attn_desc* desc);
  *                clamped and records KVQ_ERR_OUT_OF_RANGE.
  * out          : device, [B][Hq][D], fp32 or bf16 (desc->out_dtype).
  * workspace    : device, at least kvq_attn_workspace_size(desc) bytes, 16-byte
- *                aligned, no initialization needed; may be NULL when that size
- *                is 0. Calls that overlap on the GPU must use different
- *                workspaces. When partial results are used, the call launches
- *                a second, small kernel that merges them (on the same stream).
+ *                aligned, zero-filled before its first use (each call leaves
+ *                it zero-filled); may be NULL when that size is 0. Calls that
+ *                overlap on the GPU must use different workspaces.
  * batch = 0 launches nothing and returns KVQ_OK (pointers may then be NULL).
  * Returns KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_WORKSPACE
  * or KVQ_ERR_CUDA.

@@ -13,6 +13,7 @@
 #include "../../include/kvq.h"
 #include "kvq_decode.cuh"
 #include "kvq_write.cuh"
+#include "kvq_write_tc.cuh"
 
 namespace {
 
@@ -110,14 +111,73 @@ kvq_status launch_write(const kvq::WriteParams& p, int dev, cudaStream_t s) {
   return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
+// Tiled tensor maps of K and V ([T][Hkv*D] bf16, boxes of 128 rows x 64
+// elements, 128-byte swizzle) through the driver's encoder, looked up once.
+typedef CUresult (*TmapEncodeFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                 const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                 CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+TmapEncodeFn tmap_encoder() {
+  static std::atomic<TmapEncodeFn> fn{nullptr};
+  TmapEncodeFn f = fn.load(std::memory_order_acquire);
+  if (f) return f;
+  void* raw = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &raw, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !raw) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  f = reinterpret_cast<TmapEncodeFn>(raw);
+  fn.store(f, std::memory_order_release);
+  return f;
+}
+
+bool make_row_tmap(CUtensorMap* m, const void* base, int T, int Hkv, int D) {
+  TmapEncodeFn enc = tmap_encoder();
+  if (!enc) return false;
+  const cuuint64_t dims[2] = {(cuuint64_t)Hkv * D, (cuuint64_t)T};
+  const cuuint64_t strides[1] = {(cuuint64_t)Hkv * D * 2};
+  const cuuint32_t box[2] = {64, (cuuint32_t)kvq::kTcRows};
+  const cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+// Rotated write on the tensor cores: persistent grid, one CTA per SM.
+template <int D, int BLK>
+kvq_status launch_write_tc(const kvq::WriteParams& p, int dev, cudaStream_t s) {
+  if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
+  CUtensorMap tk, tv;
+  if (!make_row_tmap(&tk, p.k, p.T, p.Hkv, D) || !make_row_tmap(&tv, p.v, p.T, p.Hkv, D)) return KVQ_ERR_CUDA;
+  const long long tiles = ((long long)p.T + kvq::kTcRows - 1) / kvq::kTcRows * p.Hkv * 2;
+  if (tiles > INT_MAX) return KVQ_ERR_INVALID_ARG;
+  auto kern = kvq::kvq_write_tc_kernel<D, BLK>;
+  constexpr int smem = kvq::TcSmem<D>::kTotal;
+  static std::atomic<int> ready[kMaxDevices];
+  if (!ready[dev].load(std::memory_order_relaxed)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+      cudaGetLastError();
+      return KVQ_ERR_CUDA;
+    }
+    ready[dev].store(1, std::memory_order_relaxed);
+  }
+  const int sms = sm_count(dev);
+  if (sms < 1) return KVQ_ERR_CUDA;
+  const int grid = (int)(tiles < sms ? tiles : sms);
+  kern<<<grid, kvq::kTcThreads, smem, s>>>(tk, tv, p, (int)tiles);
+  return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+}
+
 template <int D>
 kvq_status dispatch_write(const kvq::WriteParams& p, int b, int dev, cudaStream_t s) {
   switch (b) {
     case 0: return launch_write<D, 0>(p, dev, s);
-    case 32: return launch_write<D, 32>(p, dev, s);
-    case 64: return launch_write<D, 64>(p, dev, s);
+    case 32: return launch_write_tc<D, 32>(p, dev, s);
+    case 64: return launch_write_tc<D, 64>(p, dev, s);
     case 128:
-      if constexpr (D >= 128) return launch_write<D, 128>(p, dev, s);
+      if constexpr (D >= 128) return launch_write_tc<D, 128>(p, dev, s);
       return KVQ_ERR_UNSUPPORTED;
     default: return KVQ_ERR_UNSUPPORTED;
   }

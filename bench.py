@@ -81,7 +81,7 @@ def aggregate_gbs(bytes_per_step, steps, world, max_ms):
 
 
 KERNEL_SOURCES = {
-    "kv_quant_write": ["kvq_write.cuh", "kvq_device.cuh"],
+    "kv_quant_write": ["kvq_write_tc.cuh", "kvq_write.cuh", "kvq_device.cuh"],
     "paged_decode_attn_int4": ["kvq_decode.cuh", "kvq_device.cuh"],
 }
 

@@ -15,14 +15,16 @@
 // and zero-point, the codes and the nibble packing run on the CUDA cores in
 // the epilogue, one thread per row.
 //
-// Persistent grid, one CTA per SM, 10 warps:
-//   warp 0      TMA producer: 2-D tiled loads (128-byte swizzle) of X tiles
-//               into a ring of kTcStages stages;
-//   warp 1      owns the tensor memory and issues the MMAs (one thread) into
-//               one of two accumulator buffers;
-//   warps 2..9  two epilogue groups of 4 warps (one per tensor-memory lane
-//               quarter); group e takes every other tile of the CTA, so one
-//               group's epilogue overlaps the other's and the next MMA.
+// Persistent grid, one CTA per SM, 2 + 4 kTcBufs warps:
+//   warp 0       TMA producer: 2-D tiled loads (128-byte swizzle) of X tiles
+//                into a ring of kTcStages stages;
+//   warp 1       owns the tensor memory and issues the MMAs (one thread) into
+//                one of kTcBufs accumulator buffers;
+//   warps 2..    kTcBufs epilogue groups of 4 warps (one per tensor-memory
+//                lane quarter); group e takes every kTcBufs-th tile of the
+//                CTA, so the groups' epilogues overlap one another and the
+//                MMAs. (Measured on B200: the DRAM traffic, not the epilogue,
+//                bounds the kernel; more groups or stages did not help.)
 // mbarriers hand each stage and each accumulator buffer from one role to the
 // next; every wait is bounded (a lost wait records KVQ_ERR_TIMEOUT and the
 // roles stop), and the CTA waits for its own copies and MMAs before it frees
@@ -37,7 +39,8 @@
 namespace kvq {
 
 constexpr int kTcStages = 4;
-constexpr int kTcWarps = 10;
+constexpr int kTcBufs = 2;  // tensor-memory accumulators = epilogue groups
+constexpr int kTcWarps = 2 + 4 * kTcBufs;
 constexpr int kTcThreads = kTcWarps * 32;
 constexpr int kTcRows = 128;  // rows (tokens) per tile = UMMA M
 
@@ -48,8 +51,8 @@ struct TcSmem {
   static constexpr int kOffH = 0;                              // H as the K-major B operand: D/64 chunks of D x 128 B
   static constexpr int kOffX = D * D * 2;                      // ring of X tiles
   static constexpr int kOffBar = kOffX + kTcStages * kTileBytes;
-  // mbarriers: full[kTcStages], empty[kTcStages], tfull[2], tempty[2], done
-  static constexpr int kBars = 2 * kTcStages + 5;
+  // mbarriers: full[kTcStages], empty[kTcStages], tfull[kTcBufs], tempty[kTcBufs], done
+  static constexpr int kBars = 2 * kTcStages + 2 * kTcBufs + 1;
   static constexpr int kOffTmem = kOffBar + kBars * 8;
   static constexpr int kUsed = kOffTmem + 16;
   static constexpr int kTotal = kUsed + 1024;                  // room to align the base to 1024 B
@@ -87,8 +90,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   auto full = [&](int st) { return bar0 + 8 * st; };
   auto empty = [&](int st) { return bar0 + 8 * (kTcStages + st); };
   auto tfull = [&](int j) { return bar0 + 8 * (2 * kTcStages + j); };
-  auto tempty = [&](int j) { return bar0 + 8 * (2 * kTcStages + 2 + j); };
-  const uint32_t done_bar = bar0 + 8 * (2 * kTcStages + 4);
+  auto tempty = [&](int j) { return bar0 + 8 * (2 * kTcStages + kTcBufs + j); };
+  const uint32_t done_bar = bar0 + 8 * (2 * kTcStages + 2 * kTcBufs);
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + S::kOffTmem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
@@ -105,14 +108,14 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       mbar_init(full(st), 1);
       mbar_init(empty(st), 1);
     }
-    for (int j = 0; j < 2; ++j) {
+    for (int j = 0; j < kTcBufs; ++j) {
       mbar_init(tfull(j), 1);
       mbar_init(tempty(j), 4 * 32);
     }
     mbar_init(done_bar, 1);
     mbar_init_fence();
   }
-  if (warp == 1) tmem_alloc(smem_addr(tslot), 2 * D);
+  if (warp == 1) tmem_alloc(smem_addr(tslot), kTcBufs * D);
   asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // H visible to the tensor cores
   tc_fence_before();
   __syncthreads();
@@ -143,9 +146,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     if (lane == 0) {
       int i = 0;
       for (int tile = first; tile < n_tiles; tile += stride, ++i) {
-        const int st = i % kTcStages, j = i & 1;
+        const int st = i % kTcStages, j = i % kTcBufs;
         if (!mbar_wait_bounded(full(st), (i / kTcStages) & 1)) break;
-        if (i >= 2 && !mbar_wait_bounded(tempty(j), ((i >> 1) - 1) & 1)) break;
+        if (i >= kTcBufs && !mbar_wait_bounded(tempty(j), ((i / kTcBufs) - 1) & 1)) break;
         tc_fence_after();
         const uint32_t xs = sb + S::kOffX + st * S::kTileBytes;
 #pragma unroll
@@ -164,36 +167,37 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ---- epilogue: one thread per row of the tile ---------------------------
-    const int eg = (warp - 2) >> 2;  // epilogue group: takes every other tile
+    const int eg = (warp - 2) >> 2;  // epilogue group: takes every kTcBufs-th tile
     const int q = warp & 3;          // tensor-memory lane quarter this warp may read
     const int r = 32 * q + lane;     // row of the tile
     const uint64_t cb2 = f2_pack(p.cb, p.cb);
     const uint64_t magic2 = f2_pack(8388608.0f, 8388608.0f);
     int i = eg;
-    for (int tile = first + eg * stride; tile < n_tiles; tile += 2 * stride, i += 2) {
+    for (int tile = first + eg * stride; tile < n_tiles; tile += kTcBufs * stride, i += kTcBufs) {
       const int j = eg;
       const int kv = tile & 1, h = (tile >> 1) % p.Hkv, tb = (tile >> 1) / p.Hkv;
       const int t = tb * kTcRows + r;
       const long long slot = (t < p.T) ? p.slots[t] : -1;  // in flight during the wait
-      if (!__all_sync(0xffffffffu, mbar_wait_bounded(tfull(j), (i >> 1) & 1))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait_bounded(tfull(j), (i / kTcBufs) & 1))) break;
       tc_fence_after();
       const uint32_t ta = tmem + ((uint32_t)(32 * q) << 16) + (uint32_t)(j * D);
 
       // 1. min / max of the unnormalized rotation H x; y = fp32(Hx) * c_b is
       //    monotone in Hx, so min y and max y are the scaled extremes
-      float mn = INFINITY, mx = -INFINITY;
+      float mn4[4] = {INFINITY, INFINITY, INFINITY, INFINITY};
+      float mx4[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
       for (int c = 0; c < D / 32; ++c) {
         float v[32];
         tmem_ld32(ta + 32 * c, v);
 #pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          mn = fmin3(mn, v[2 * k], v[2 * k + 1]);
-          mx = fmax3(mx, v[2 * k], v[2 * k + 1]);
+        for (int k = 0; k < 16; ++k) {  // four independent chains
+          mn4[k & 3] = fmin3(mn4[k & 3], v[2 * k], v[2 * k + 1]);
+          mx4[k & 3] = fmax3(mx4[k & 3], v[2 * k], v[2 * k + 1]);
         }
       }
-      mn = __fmul_rn(mn, p.cb);
-      mx = __fmul_rn(mx, p.cb);
+      const float mn = __fmul_rn(fminf(fminf(mn4[0], mn4[1]), fminf(mn4[2], mn4[3])), p.cb);
+      const float mx = __fmul_rn(fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3])), p.cb);
       // 2. z = largest fp16 <= min y; s = smallest fp16 with 15 s + z >= max y
       //    (directed roundings give a candidate at most one fp16 step high;
       //    the exact test in fp64, where 15 s + z is exact, settles it)
@@ -250,7 +254,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 1) tmem_dealloc(tmem, 2 * D);
+  if (warp == 1) tmem_dealloc(tmem, kTcBufs * D);
 }
 
 }  // namespace kvq

@@ -95,14 +95,6 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + S::kOffTmem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
 
-  // H = diag(H_b), unnormalized Sylvester order, as the B operand [n][k]
-  // (symmetric, so B[n][k] = H[k][n])
-  for (int i = tid; i < D * D; i += kTcThreads) {
-    const int n = i / D, k = i % D;
-    float h = 0.0f;
-    if (n / BLK == k / BLK) h = (__popc((n % BLK) & (k % BLK)) & 1) ? -1.0f : 1.0f;
-    *reinterpret_cast<__nv_bfloat16*>(smem + S::kOffH + sw128_offset(n, k, D)) = __float2bfloat16(h);
-  }
   if (tid == 0) {
     for (int st = 0; st < kTcStages; ++st) {
       mbar_init(full(st), 1);
@@ -116,10 +108,34 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     mbar_init_fence();
   }
   if (warp == 1) tmem_alloc(smem_addr(tslot), kTcBufs * D);
-  asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // H visible to the tensor cores
   tc_fence_before();
-  __syncthreads();
+  __syncthreads();  // barriers and the tensor-memory address are in place
   tc_fence_after();
+  // While warp 0 starts the first copies, the other warps build
+  // H = diag(H_b) (unnormalized Sylvester order) as the B operand [n][k]
+  // (symmetric, so B[n][k] = H[k][n]), 16 bytes at a time, then meet on
+  // named barrier 1 before the first MMA.
+  if (warp != 0) {
+    for (int i = tid - 32; i < D * (D / 8); i += kTcThreads - 32) {
+      const int n = i / (D / 8), k0 = 8 * (i % (D / 8));
+      uint32_t w[4];
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        uint32_t pair = 0;
+#pragma unroll
+        for (int hlf = 0; hlf < 2; ++hlf) {
+          const int k = k0 + 2 * e + hlf;
+          uint32_t bits = 0;  // bf16 0
+          if (n / BLK == k / BLK) bits = (__popc((n % BLK) & (k % BLK)) & 1) ? 0xBF80u : 0x3F80u;  // -1, +1
+          pair |= bits << (16 * hlf);
+        }
+        w[e] = pair;
+      }
+      *reinterpret_cast<uint4*>(smem + S::kOffH + sw128_offset(n, k0, D)) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // H visible to the tensor cores
+    named_bar_sync(1, kTcThreads - 32);
+  }
   const uint32_t tmem = *tslot;
   const int first = blockIdx.x, stride = gridDim.x;
 

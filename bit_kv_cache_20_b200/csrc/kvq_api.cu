@@ -317,7 +317,8 @@ kvq_status check_attn_desc(const kvq_attn_desc* d) {
 }
 
 // Workspace: the splits' partial results (fp32 rows of D + 4: O + Z, M, L,
-// padding), then one ticket counter per (sequence, head group).
+// padding), then two counters per (sequence, head group): arrivals and
+// finished merges.
 size_t partial_bytes_for(const kvq_attn_desc* d, const SplitPlan& plan) {
   const size_t G = (size_t)(d->num_q_heads / d->num_kv_heads);
   return (size_t)d->batch * d->num_kv_heads * plan.n_splits * G * (d->head_dim + 4) * sizeof(float);
@@ -325,7 +326,7 @@ size_t partial_bytes_for(const kvq_attn_desc* d, const SplitPlan& plan) {
 
 size_t workspace_bytes_for(const kvq_attn_desc* d, const SplitPlan& plan) {
   if (plan.n_splits <= 1 || d->batch == 0) return 0;
-  const size_t counters = (size_t)d->batch * (d->num_kv_heads / plan.hg) * sizeof(int);
+  const size_t counters = (size_t)d->batch * (d->num_kv_heads / plan.hg) * 2 * sizeof(int);  // arrivals, merges done
   return partial_bytes_for(d, plan) + (counters + 15) / 16 * 16;
 }
 

@@ -93,13 +93,6 @@ struct AttnSmem {
   static constexpr int kOffPid = kOffQ8 + kRows * 2 * D;
   static constexpr int kOffFlag = kOffPid + kMaxPids * 4;
   static constexpr int kTotal = kOffFlag + 16;
-  // last-split merge scratch, in the rings (free by then): the weight of
-  // every (row, split), the merged L per row, then the per-thread sums
-  static constexpr int kOffMS = 0;
-  static constexpr int kOffLS = kOffMS + kRows * kMaxSplits * 4;
-  static constexpr int kOffPartO = kOffLS + kRows * 4;
-  static constexpr int kOffML = kOffPartO + 2 * kAttnThreads * 16;  // float2 [kRows][kMaxSplits]: M, L
-  static_assert(kOffML + kRows * kMaxSplits * 8 <= kRingBytes, "merge scratch fits in the rings");
 };
 
 template <int N>
@@ -546,107 +539,134 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
   }
 
   if (!single) {
-    // ---- ticket: the last split of this (sequence, head group) merges ------
+    // ---- tickets: the last K arrivals each merge some query rows ----------
     // (every thread's partial stores are made visible device-wide before the
-    // barrier and thread 0's atomic; the last CTA reads the partials from L2
-    // with ld.cg, issued after its atomic returned and a barrier)
+    // barrier and thread 0's atomic; a merging CTA reads the partials from L2
+    // with ld.cg once the arrival count shows every split has written)
     __threadfence();
     __syncthreads();
-    int* ticket = p.ws_count + (size_t)n * (p.Hkv / HG) + hgi;
-    if (tid == 0) sflag[0] = (atomicAdd(ticket, 1) == p.n_splits - 1) ? 1 : 0;
-    __syncthreads();
-    if (!sflag[0]) return;
-    if (tid == 0) *ticket = 0;  // every split has counted: ready for the next call
-
-    // Merge of the splits. Thread (e, pp) first puts its loads in flight: the
-    // O + Z of output float4 e for splits pp, pp + P, ... (kMergeBatch of them;
-    // more splits take further rounds). Then one warp per query row reads the
-    // (M, L) of every split, reduces M with shuffles and leaves the weights
-    // 2^(M_s - M) and the merged L in shared memory.
-    constexpr int kMergeBatch = 20;
     const int ns = p.n_splits;
     const int rows = HG * G;
-    const int e4 = rows * (D / 4);
-    const int P = e4 >= kAttnThreads ? 1 : kAttnThreads / e4;
-    const size_t sstride = (size_t)G * (D + 4);  // floats between consecutive splits
-    float* wS = reinterpret_cast<float*>(smem + S::kOffMS);  // [rows][kMaxSplits] weights
-    float* lS = reinterpret_cast<float*>(smem + S::kOffLS);  // [rows] merged L
-    float4* part_o = reinterpret_cast<float4*>(smem + S::kOffPartO);  // [P][e4]
-    auto head_base = [&](int hh, int r) {
-      return p.ws_part + (((size_t)n * p.Hkv + hgi * HG + hh) * ns * G + r) * (D + 4);
-    };
-    const bool has_e = tid < e4 * P;
-    const int e = tid % e4, pp = tid / e4;
-    const int hh_e = e / (G * (D / 4)), r_e = (e / (D / 4)) % G, c4_e = 4 * (e % (D / 4));
-    const float* base_e = head_base(hh_e, r_e) + c4_e;
-    float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-    for (int s0 = 0; s0 < ns; s0 += kMergeBatch * P) {
-      // (M, L) of every (row, split) into shared memory first (they are needed
-      // first), then this thread's O + Z into registers (split indices
-      // clamped: the extra loads read a valid split and get weight 0)
-      float2* mlS = reinterpret_cast<float2*>(smem + S::kOffML);  // [rows][kMaxSplits]
-      if (s0 == 0) {
-        for (int i = tid; i < rows * ns; i += kAttnThreads) {
-          const int rr = i / ns, s2 = i % ns;
-          cp_async_8(smem_addr(mlS + rr * kMaxSplits + s2), head_base(rr / G, rr % G) + D + s2 * sstride);
-        }
-        cp_async_commit();
-      }
-      float4 v[kMergeBatch];
-#pragma unroll
-      for (int j = 0; j < kMergeBatch; ++j) {
-        const int s2 = min(s0 + pp + j * P, ns - 1);
-        v[j] = __ldcg(reinterpret_cast<const float4*>(base_e + s2 * sstride));
-      }
-      if (s0 == 0) {
-        cp_async_wait<0>();
-        __syncthreads();
-        // one warp per row: M by shuffles, the weights 2^(M_s - M) and L
-        for (int rr = warp; rr < rows; rr += kAttnWarps) {
-          float M = -INFINITY;
-          for (int s2 = lane; s2 < ns; s2 += 32) M = fmaxf(M, mlS[rr * kMaxSplits + s2].x);
-#pragma unroll
-          for (int o2 = 16; o2 > 0; o2 >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o2));
-          float L = 0.0f;
-          for (int s2 = lane; s2 < ns; s2 += 32) {
-            const float2 ml = mlS[rr * kMaxSplits + s2];
-            const float wgt = (ml.x == -INFINITY) ? 0.0f : fast_exp2(ml.x - M);
-            wS[rr * kMaxSplits + s2] = wgt;
-            L = fmaf(wgt, ml.y, L);
-          }
-#pragma unroll
-          for (int o2 = 16; o2 > 0; o2 >>= 1) L += __shfl_xor_sync(FULL, L, o2);
-          if (lane == 0) lS[rr] = L;
-        }
-        __syncthreads();
-      }
-      if (has_e) {
-        const float* wrow = wS + (hh_e * G + r_e) * kMaxSplits;
-#pragma unroll
-        for (int j = 0; j < kMergeBatch; ++j) {
-          const int s2 = s0 + pp + j * P;
-          const float wgt = (s2 < ns) ? wrow[s2] : 0.0f;
-          acc.x = fmaf(wgt, v[j].x, acc.x);
-          acc.y = fmaf(wgt, v[j].y, acc.y);
-          acc.z = fmaf(wgt, v[j].z, acc.z);
-          acc.w = fmaf(wgt, v[j].w, acc.w);
-        }
-      }
-    }
-    if (has_e) part_o[pp * e4 + e] = acc;
+    const int K = min(rows, ns);  // merging CTAs; CTA j takes rows j, j + K, ...
+    int* arrive = p.ws_count + ((size_t)n * (p.Hkv / HG) + hgi) * 2;
+    int* done = arrive + 1;
+    if (tid == 0) sflag[0] = atomicAdd(arrive, 1);
     __syncthreads();
-    for (int i = tid; i < e4; i += kAttnThreads) {
-      const int hh = i / (G * (D / 4)), r = (i / (D / 4)) % G, c4 = 4 * (i % (D / 4));
-      float4 sum = part_o[i];
-      for (int q2 = 1; q2 < P; ++q2) {
-        const float4 w4 = part_o[q2 * e4 + i];
-        sum.x += w4.x; sum.y += w4.y; sum.z += w4.z; sum.w += w4.w;
+    const int t = sflag[0];
+    if (t < ns - K) return;
+    if (t < ns - 1) {
+      // not the last arrival: wait (bounded) for the remaining splits; every
+      // CTA of the launch is resident at once, so they are running
+      if (tid == 0) {
+        uint32_t rounds = 0;
+        while (ld_acquire_gpu(arrive) < ns) {
+          __nanosleep(256);
+          if (++rounds > kMaxSpinRounds) {
+            record_error(KVQ_ERR_TIMEOUT);
+            break;
+          }
+        }
       }
-      const float L = lS[hh * G + r];
-      const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
-      *reinterpret_cast<float4*>(qs + (hh * NR + r) * D + c4) =
-          make_float4(sum.x * inv, sum.y * inv, sum.z * inv, sum.w * inv);
+      __syncthreads();
     }
+    const int j = t - (ns - K);
+    // Merge of one row: warp w takes splits w, w + 8, ...; lane l the output
+    // float4 l. Each warp folds its splits into a running (max, l, acc),
+    // every load of a round (up to 8 splits) issued before any is used; the
+    // warps' states are then combined through shared memory.
+    constexpr int kRowBatch = 8;
+    float* mred = reinterpret_cast<float*>(smem);            // [kAttnWarps] (the rings are free)
+    float4* ored = reinterpret_cast<float4*>(smem + 64);     // [kAttnWarps][32]
+    float* lred = reinterpret_cast<float*>(smem + 64 + kAttnWarps * 32 * 16);  // [kAttnWarps]
+    static_assert(64 + kAttnWarps * 32 * 16 + kAttnWarps * 4 <= S::kRingBytes, "row-merge scratch fits in the rings");
+    const size_t sstride = (size_t)G * (D + 4);
+    for (int rr = j; rr < rows; rr += K) {
+      const int hh = rr / G, r = rr % G;
+      const float* base = p.ws_part + (((size_t)n * p.Hkv + hgi * HG + hh) * ns * G + r) * (D + 4);
+      float mw = -INFINITY, L = 0.0f;
+      float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+      for (int s0 = warp; s0 < ns; s0 += kAttnWarps * kRowBatch) {
+        float4 v[kRowBatch];
+        float2 ml[kRowBatch];
+#pragma unroll
+        for (int k = 0; k < kRowBatch; ++k) {
+          const int s2 = min(s0 + k * kAttnWarps, ns - 1);
+          v[k] = (lane < D / 4) ? __ldcg(reinterpret_cast<const float4*>(base + s2 * sstride) + lane)
+                                : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+          ml[k] = __ldcg(reinterpret_cast<const float2*>(base + s2 * sstride + D));
+        }
+        float mb = mw;
+#pragma unroll
+        for (int k = 0; k < kRowBatch; ++k)
+          if (s0 + k * kAttnWarps < ns) mb = fmaxf(mb, ml[k].x);
+        if (mb == -INFINITY) continue;
+        const float a0 = (mw == -INFINITY) ? 0.0f : fast_exp2(mw - mb);
+        acc.x *= a0; acc.y *= a0; acc.z *= a0; acc.w *= a0;
+        L *= a0;
+#pragma unroll
+        for (int k = 0; k < kRowBatch; ++k) {
+          if (s0 + k * kAttnWarps >= ns || ml[k].x == -INFINITY) continue;
+          const float wgt = fast_exp2(ml[k].x - mb);
+          acc.x = fmaf(wgt, v[k].x, acc.x);
+          acc.y = fmaf(wgt, v[k].y, acc.y);
+          acc.z = fmaf(wgt, v[k].z, acc.z);
+          acc.w = fmaf(wgt, v[k].w, acc.w);
+          L = fmaf(wgt, ml[k].y, L);
+        }
+        mw = mb;
+      }
+      if (lane == 0) {
+        mred[warp] = mw;
+        lred[warp] = L;
+      }
+      if (lane < D / 4) ored[warp * 32 + lane] = acc;
+      __syncthreads();
+      if (warp == 0) {
+        float M = mred[0];
+#pragma unroll
+        for (int w2 = 1; w2 < kAttnWarps; ++w2) M = fmaxf(M, mred[w2]);
+        float Lt = 0.0f;
+        float4 sum = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+        if (M != -INFINITY) {
+#pragma unroll
+          for (int w2 = 0; w2 < kAttnWarps; ++w2) {
+            if (mred[w2] == -INFINITY) continue;
+            const float f = fast_exp2(mred[w2] - M);
+            Lt = fmaf(f, lred[w2], Lt);
+            if (lane < D / 4) {
+              const float4 x = ored[w2 * 32 + lane];
+              sum.x = fmaf(f, x.x, sum.x);
+              sum.y = fmaf(f, x.y, sum.y);
+              sum.z = fmaf(f, x.z, sum.z);
+              sum.w = fmaf(f, x.w, sum.w);
+            }
+          }
+        }
+        const float inv = (Lt > 0.0f) ? 1.0f / Lt : 0.0f;
+        if (lane < D / 4)
+          *reinterpret_cast<float4*>(qs + (hh * NR + r) * D + 4 * lane) =
+              make_float4(sum.x * inv, sum.y * inv, sum.z * inv, sum.w * inv);
+      }
+      __syncthreads();
+    }
+    // rotate back this CTA's rows (one warp per row) and store
+    for (int rr = j + K * warp; rr < rows; rr += K * kAttnWarps) {
+      const int hh = rr / G, r = rr % G;
+      const float* rp = qs + (hh * NR + r) * D;
+      float v[E];
+#pragma unroll
+      for (int e2 = 0; e2 < E; ++e2) v[e2] = rp[E * lane + e2];
+      if constexpr (BLK > 0) warp_fwht<D, BLK>(v, lane);
+      const size_t o_base = ((size_t)n * p.Hq + (size_t)(hgi * HG + hh) * G + r) * D + E * lane;
+#pragma unroll
+      for (int e2 = 0; e2 < E; ++e2) store_out(p, o_base + e2, BLK > 0 ? v[e2] * p.cb : v[e2]);
+    }
+    // the last of the K merging CTAs resets both counters for the next call
+    if (tid == 0 && atomicAdd(done, 1) == K - 1) {
+      *arrive = 0;
+      *done = 0;
+    }
+    return;
   }
   __syncthreads();
 

@@ -58,6 +58,17 @@ __device__ __forceinline__ void fence_acq_rel_gpu() {
   asm volatile("fence.acq_rel.gpu;\n" ::: "memory");
 }
 
+// Acquire load of a global int at GPU scope.
+__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
+  int v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Upper bound on the polls of a spin on a global counter (each with a short
+// sleep): far above any legitimate wait, ends within a fraction of a second.
+constexpr uint32_t kMaxSpinRounds = 1u << 20;
+
 // Wait until at most N of this thread's most recent cp.async groups are pending.
 template <int N>
 __device__ __forceinline__ void cp_async_wait() {

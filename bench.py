@@ -199,9 +199,10 @@ class ClockSampler:
 # ----------------------------------------------------------------------------
 
 class Step:
-    """Prepared C-ABI calls for one workload on one device. The timed loop
-    calls the library directly with pre-marshalled arguments (what a C caller
-    does), so Python overhead stays far below the kernels' duration."""
+    """Prepared C-ABI calls for one workload on one device, on a stream of its
+    own. Timed regions replay a CUDA graph captured from those calls (what a
+    serving loop does with its decode step), so the host's launch rate never
+    gates the GPU: the kernels run back to back exactly as launched."""
 
     N_POOLS = 4
 
@@ -226,7 +227,7 @@ class Step:
         nbytes = kvq.attn_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.num_pages, w.max_pages, block)
         self.ws = kvq.alloc_workspace(nbytes, device=dev)
         self.ws_bytes = self.ws.numel()
-        self.stream = torch.cuda.current_stream(dev)
+        self.stream = torch.cuda.Stream(dev)
         self.sh = ctypes.c_void_p(self.stream.cuda_stream)
         self.wdesc = _lib.WriteDesc(w.tokens_written, w.Hkv, w.D, 16, w.num_pages)
         self.adesc = _lib.AttnDesc(w.B, w.Hq, w.Hkv, w.D, 16, w.num_pages, w.max_pages, block, 0.0, 1)
@@ -244,6 +245,7 @@ class Step:
             self.attn_args.append((P(self.q.data_ptr()), P(c.data_ptr()), P(s.data_ptr()), P(z.data_ptr()),
                                    P(self.pt.data_ptr()), P(self.ctx.data_ptr()), P(self.out.data_ptr()),
                                    P(self.ws.data_ptr()), self.ws_bytes, ctypes.byref(self.adesc), self.sh))
+        torch.cuda.synchronize(dev)  # allocations above ran on the default stream
 
     def write(self, i):
         st = self.L.kv_quant_write(*self.write_args[i % self.N_POOLS])
@@ -260,35 +262,44 @@ class Step:
             self.write(i)
         self.torch.cuda.synchronize(self.dev)
 
-    def timed_only(self, kind, steps, start_index=0):
-        """One kernel alone, `steps` back-to-back launches on the stream,
-        bracketed by two events (inputs and outputs rotate through sets
-        larger than L2). Returns the average ms per launch."""
+    def capture(self, kinds, steps, start_index=0):
+        """A CUDA graph of `steps` steps, each the calls named in `kinds`
+        ("write", "decode") in that order, inputs and outputs rotating through
+        the pools as in the direct calls. It is replayed once, untimed, so the
+        first timed replay does not include the graph's upload."""
         torch = self.torch
-        fn = self.write if kind == "write" else self.decode
-        t0 = torch.cuda.Event(enable_timing=True)
-        t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(self.stream)
-        for j in range(steps):
-            fn(start_index + j)
-        t1.record(self.stream)
-        t1.synchronize()
-        return t0.elapsed_time(t1) / steps
+        fns = [self.write if k == "write" else self.decode for k in kinds]
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=self.stream, capture_error_mode="thread_local"):
+            for j in range(steps):
+                for fn in fns:
+                    fn(start_index + j)
+        with torch.cuda.stream(self.stream):
+            g.replay()
+        self.stream.synchronize()
+        return g
 
-    def timed(self, steps, start_index=0):
-        """Run `steps` whole steps (write, then decode) back to back between
-        two events. Returns the total ms."""
+    def replay_ms(self, g):
+        """Device time of one replay of `g` between two events on the stream."""
         torch = self.torch
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
-        t0.record(self.stream)
-        for j in range(steps):
-            i = start_index + j
-            self.write(i)
-            self.decode(i)
-        t1.record(self.stream)
+        with torch.cuda.stream(self.stream):
+            t0.record(self.stream)
+            g.replay()
+            t1.record(self.stream)
         t1.synchronize()
         return t0.elapsed_time(t1)
+
+    def timed_only(self, kind, steps, start_index=0):
+        """One kernel alone, `steps` back-to-back launches (inputs and outputs
+        rotate through sets larger than L2). Returns the average ms per launch."""
+        return self.replay_ms(self.capture((kind,), steps, start_index)) / steps
+
+    def timed(self, steps, start_index=0):
+        """`steps` whole steps (write, then decode) back to back. Returns the
+        total ms."""
+        return self.replay_ms(self.capture(("write", "decode"), steps, start_index))
 
 
 def e2e_run(w, block, dev, steps, warmup):
@@ -408,7 +419,7 @@ def config_block(w, block):
         "context": int(w.context_lens.max()), "written_tokens": w.tokens_written, "page": 16,
         "hadamard_block": block, "out_dtype": "bf16",
         "l2": "inputs larger than L2 rotate; decode reads a cache written two steps earlier",
-        "timing": "steps back to back between two events; each kernel's line: the same, that kernel alone",
+        "timing": "the K steps as one CUDA graph (replayed once untimed, then once between two events); each kernel's line: the same, that kernel alone",
     }
 
 

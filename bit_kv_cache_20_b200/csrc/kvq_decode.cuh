@@ -24,9 +24,12 @@
 //        O^T[D x 8]        += codes^T[D x 16 tokens] * Phl^T[16 tokens x 8]
 // QK takes the code bytes as they are: byte & 0x0F is the low code, byte &
 // 0xF0 the high code times 16, each product summed in its own accumulator.
-// q~ enters as two int8 limbs per element, q~ = sigma (q0 + q1 / 256) with
-// sigma = max|q~| / 127 per query head (error <= 2^-9 sigma, far below the
-// bf16 input's own precision); columns are (head, limb). PV needs floating
+// q~ enters as three int8 limbs per element, q~ = sigma (q0 + q1 / 256 +
+// q2 / 32768) with sigma = max|q~| / 127 per query head (error <= 2^-16 sigma;
+// with two limbs the logit error, ~sigma / 512 times |k|, reached 1.7e-3 of
+// output on keys with x10 outlier channels and large token norms); columns
+// are (head, limb 0 / 1) in one 8-column tile and (head, limb 2) in the even
+// columns of a second. PV needs floating
 // weights: p * s_v enters as an fp16 "hi" and "lo" part (hi + lo keeps ~22
 // bits) and the codes as exact normal fp16 values c (or 16c for a nibble at
 // bits 4..7, compensated in the epilogue); subnormal fp16 operands are
@@ -89,8 +92,8 @@ struct AttnSmem {
   static constexpr int kOffRes = kRingBytes;
   static constexpr int kOffQ = kOffRes + kAttnWarps * kResFloats * 4;  // float [kRows][D]
   static constexpr int kOffQInfo = kOffQ + kRows * D * 4;       // float [kRows][4]: scale, sum
-  static constexpr int kOffQ8 = kOffQInfo + kRows * 16;         // int8 [kRows][2 limbs][D], B order
-  static constexpr int kOffPid = kOffQ8 + kRows * 2 * D;
+  static constexpr int kOffQ8 = kOffQInfo + kRows * 16;         // int8 [kRows][3 limbs][D], B order
+  static constexpr int kOffPid = kOffQ8 + kRows * 3 * D;
   static constexpr int kOffFlag = kOffPid + kMaxPids * 4;
   static constexpr int kTotal = kOffFlag + 16;
 };
@@ -258,8 +261,10 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
   for (int k = 0; k < R - 1; ++k) fetch(k);
 
   // ---- q~ = R q * (softmax_scale * log2 e) while the first pages land -----
-  // One warp per row. Limbs: q0 = rint(q~ / sigma), q1 = rint((q~ - q0 sigma)
-  // * 256 / sigma), sigma = max|q~| / 127. They are stored in B-fragment
+  // One warp per row. Limbs, with a = q~ / sigma and sigma = max|q~| / 127:
+  // q0 = rint(a), r1 = 256 (a - q0), q1 = rint(r1), q2 = rint(128 (r1 - q1))
+  // (every step exact in fp32; |q1|, |q2| <= 64 except at exact ties, where
+  // the +-127 clamp costs at most sigma / 32768). They are stored in B-fragment
   // order: element 8w + j goes to byte tig*8KW + ((m*2 + (j&1))*2 + h)*4 +
   // (j>>1) of its limb's array, w = KW*tig + 2m + h, so that thread tig reads
   // its fragments as 8KW contiguous bytes.
@@ -284,11 +289,12 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
     const float sigma = amax / 127.0f;
     const float inv = (amax > 0.0f) ? 127.0f / amax : 0.0f;
     if (lane == 0) {
-      qinfo[row * 4 + 0] = sigma * (1.0f / 4096.0f);
+      qinfo[row * 4 + 0] = sigma * (1.0f / 16.0f);
       qinfo[row * 4 + 1] = sum;
     }
-    int8_t* l0 = q8 + row * 2 * D;
+    int8_t* l0 = q8 + row * 3 * D;
     int8_t* l1 = l0 + D;
+    int8_t* l2 = l1 + D;
 #pragma unroll
     for (int e = 0; e < E; ++e) {
       const int el = E * lane + e, w = el >> 3, j = el & 7;
@@ -296,29 +302,38 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
       const int off = tw * (8 * KW) + (((rw >> 1) * 2 + (j & 1)) * 2 + (rw & 1)) * 4 + (j >> 1);
       const float a = __fmul_rn(v[e], inv);
       const float q0 = rintf(a);
-      const float q1 = fminf(fmaxf(rintf(__fmul_rn(__fsub_rn(a, q0), 256.0f)), -127.0f), 127.0f);
+      const float r1 = __fmul_rn(__fsub_rn(a, q0), 256.0f);
+      const float q1 = fminf(fmaxf(rintf(r1), -127.0f), 127.0f);
+      const float q2 = fminf(fmaxf(rintf(__fmul_rn(__fsub_rn(r1, q1), 128.0f)), -127.0f), 127.0f);
       l0[off] = (int8_t)(int)q0;
       l1[off] = (int8_t)(int)q1;
+      l2[off] = (int8_t)(int)q2;
     }
   }
   __syncthreads();
 
-  // B fragments of QK: column g is limb g&1 of query row 4c + g/2 of head hw.
+  // B fragments of QK. Tile 0: column g is limb g&1 of query row 4c + g/2 of
+  // head hw; tile 1: column g is limb 2 of that row for even g, zero for odd.
   // MMA (m, half) of thread tig: b0 = bytes of k-group tig, b1 of k-group
   // 4 + tig; their codes are the low (half 0) or high (half 1) nibbles of K
   // words KW*tig + 2m (b0) and KW*tig + 2m + 1 (b1).
-  uint32_t bq[NC][KM][2][2];
+  uint32_t bq[NC][KM][2][2], bq2[NC][KM][2][2];
 #pragma unroll
   for (int c = 0; c < NC; ++c) {
     const int row = hw * NR + 4 * c + (g >> 1);
-    const uint8_t* base = reinterpret_cast<const uint8_t*>(q8 + row * 2 * D + (g & 1) * D) + tig * (8 * KW);
+    const uint8_t* base = reinterpret_cast<const uint8_t*>(q8 + row * 3 * D) + tig * (8 * KW);
 #pragma unroll
     for (int m = 0; m < KM; ++m) {
-      const uint4 f4 = *reinterpret_cast<const uint4*>(base + 16 * m);
+      const uint4 f4 = *reinterpret_cast<const uint4*>(base + (g & 1) * D + 16 * m);
+      const uint4 h4 = (g & 1) ? make_uint4(0u, 0u, 0u, 0u) : *reinterpret_cast<const uint4*>(base + 2 * D + 16 * m);
       bq[c][m][0][0] = f4.x;
       bq[c][m][0][1] = f4.y;
       bq[c][m][1][0] = f4.z;
       bq[c][m][1][1] = f4.w;
+      bq2[c][m][0][0] = h4.x;
+      bq2[c][m][0][1] = h4.y;
+      bq2[c][m][1][0] = h4.z;
+      bq2[c][m][1][1] = h4.w;
     }
   }
   // this thread's QK results belong to query row 4c + tig of head hw
@@ -365,7 +380,7 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
       uint32_t ka[KW], kc[KW];
       lds_words<KW>(kb + g * (D / 2) + tig * (4 * KW), ka);
       lds_words<KW>(kb + (g + 8) * (D / 2) + tig * (4 * KW), kc);
-      int accl[NC][4], acch[NC][4];
+      int accl[NC][4], acch[NC][4], accl2[NC][4], acch2[NC][4];
 #pragma unroll
       for (int m = 0; m < KM; ++m) {
         const uint32_t x0 = ka[2 * m], x1 = ka[2 * m + 1], y0 = kc[2 * m], y1 = kc[2 * m + 1];
@@ -376,9 +391,13 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
           if (m == 0) {
             mma_u8s8_16832_z(accl[c], al, bq[c][0][0][0], bq[c][0][0][1]);
             mma_u8s8_16832_z(acch[c], ah, bq[c][0][1][0], bq[c][0][1][1]);
+            mma_u8s8_16832_z(accl2[c], al, bq2[c][0][0][0], bq2[c][0][0][1]);
+            mma_u8s8_16832_z(acch2[c], ah, bq2[c][0][1][0], bq2[c][0][1][1]);
           } else {
             mma_u8s8_16832(accl[c], al, bq[c][m][0][0], bq[c][m][0][1]);
             mma_u8s8_16832(acch[c], ah, bq[c][m][1][0], bq[c][m][1][1]);
+            mma_u8s8_16832(accl2[c], al, bq2[c][m][0][0], bq2[c][m][0][1]);
+            mma_u8s8_16832(acch2[c], ah, bq2[c][m][1][0], bq2[c][m][1][1]);
           }
         }
       }
@@ -393,11 +412,17 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
 #pragma unroll
       for (int c = 0; c < NC; ++c) {
         // logits (base 2) of tokens g and g+8 for query row 4c + tig
-        // 16 S_limb = 16 acc_lo + acc_hi; T = 256 (16 S_0) + 16 S_1, exact in s32
-        const int T0 = (accl[c][0] * 16 + acch[c][0]) * 256 + (accl[c][1] * 16 + acch[c][1]);
-        const int T1 = (accl[c][2] * 16 + acch[c][2]) * 256 + (accl[c][3] * 16 + acch[c][3]);
-        float lg0 = fmaf((float)T0 * qsc[c], sk0, zk0 * qsm[c]);
-        float lg1 = fmaf((float)T1 * qsc[c], sk1, zk1 * qsm[c]);
+        // X_l = 16 S_l = 16 acc_lo + acc_hi of limb l, an integer below 2^22
+        // in magnitude (exact in fp32); q~ . code = sigma / 16 (X_0 + X_1 / 256
+        // + X_2 / 32768), summed in fp32
+        const float T0 = fmaf(fmaf((float)(accl2[c][0] * 16 + acch2[c][0]), 1.0f / 128.0f,
+                                   (float)(accl[c][1] * 16 + acch[c][1])),
+                              1.0f / 256.0f, (float)(accl[c][0] * 16 + acch[c][0]));
+        const float T1 = fmaf(fmaf((float)(accl2[c][2] * 16 + acch2[c][2]), 1.0f / 128.0f,
+                                   (float)(accl[c][3] * 16 + acch[c][3])),
+                              1.0f / 256.0f, (float)(accl[c][2] * 16 + acch[c][2]));
+        float lg0 = fmaf(T0 * qsc[c], sk0, zk0 * qsm[c]);
+        float lg1 = fmaf(T1 * qsc[c], sk1, zk1 * qsm[c]);
         if (!hv[c]) lg0 = lg1 = -INFINITY;
         if (tail) {
           if (tok + g >= ctx) lg0 = -INFINITY;

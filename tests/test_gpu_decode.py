@@ -6,6 +6,8 @@ max-abs of the fp64 oracle; bf16 output equal to the round-to-nearest bf16 of
 the fp32 output; guard regions around `out` untouched; a workspace reused
 without clearing gives the same result.
 """
+import dataclasses
+
 import numpy as np
 import pytest
 import torch
@@ -170,6 +172,33 @@ def test_decode_deterministic_and_workspace_left_zeroed():
     for _ in range(3):
         b_, ws = gpu_decode(w, pool, ws=ws)
         assert np.array_equal(a, b_)
+
+
+@pytest.mark.parametrize("ctx,Hq,Hkv", [([40000 - 7], 8, 2), ([36001, 2000], 8, 2), ([1, 17, 900], 8, 2),
+                                        ([60000] + [16] * 39, 8, 8)])
+def test_decode_counts_every_page_once(ctx, Hq, Hkv):
+    """q = 0 makes the softmax uniform, and on a plain INT4 cache a constant V
+    row c is stored exactly (s = 0, z = c). With c = a different integer per
+    page, the output is the mean page value over the context: a page skipped
+    or counted twice by the split plan moves it by ~16 |c - mean| / ctx, far
+    above fp32 rounding. In the last case 320 (sequence, kv head) pairs leave
+    at most 3 splits per pair on 148 SMs, so a split of the long sequence
+    holds more pages than the kernel keeps page ids for in shared memory."""
+    B = len(ctx)
+    w = workloads.random_case(seed=31, B=B, Hq=Hq, Hkv=Hkv, D=128, block=0, context_lens=ctx)
+    vals = []
+    for n in range(B):
+        pos = np.arange(ctx[n])
+        vals.append(((pos // 16) % 97 - 48).astype(np.float64))
+    c = torch.as_tensor(np.concatenate(vals), dtype=torch.bfloat16)
+    v_new = c[:, None, None].expand(-1, w.Hkv, w.D).contiguous()
+    w = dataclasses.replace(w, v_new=v_new, q=torch.zeros_like(w.q))
+    pool = build_cache(w)
+    got, _ = gpu_decode(w, pool)
+    for n in range(B):
+        ref = vals[n].mean()
+        err = float(np.abs(got[n] - ref).max())
+        assert err <= 1e-5 * max(1.0, abs(ref)), (ctx, n, err)
 
 
 def test_decode_bad_page_id_and_long_context_are_reported(orc):

@@ -316,18 +316,12 @@ kvq_status check_attn_desc(const kvq_attn_desc* d) {
   return KVQ_OK;
 }
 
-// Workspace: the splits' partial results (fp32 rows of D + 4: O + Z, M, L,
-// padding), then two counters per (sequence, head group): arrivals and
-// finished merges.
-size_t partial_bytes_for(const kvq_attn_desc* d, const SplitPlan& plan) {
-  const size_t G = (size_t)(d->num_q_heads / d->num_kv_heads);
-  return (size_t)d->batch * d->num_kv_heads * plan.n_splits * G * (d->head_dim + 4) * sizeof(float);
-}
-
+// Workspace: the splits' partial results, rows of D + 4 words (O + Z, M, L,
+// padding), each word stored as ~bits so that zero means "not written".
 size_t workspace_bytes_for(const kvq_attn_desc* d, const SplitPlan& plan) {
   if (plan.n_splits <= 1 || d->batch == 0) return 0;
-  const size_t counters = (size_t)d->batch * (d->num_kv_heads / plan.hg) * 2 * sizeof(int);  // arrivals, merges done
-  return partial_bytes_for(d, plan) + (counters + 15) / 16 * 16;
+  const size_t G = (size_t)(d->num_q_heads / d->num_kv_heads);
+  return (size_t)d->batch * d->num_kv_heads * plan.n_splits * G * (d->head_dim + 4) * sizeof(uint32_t);
 }
 
 template <int D, int BLK, int NC>
@@ -455,9 +449,7 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const voi
   p.max_pages = d.max_pages_per_seq;
   p.n_splits = plan.n_splits;
   p.pages_per_split = plan.pages_per_split;
-  p.ws_part = need > 0 ? static_cast<float*>(workspace) : nullptr;
-  p.ws_count = need > 0 ? reinterpret_cast<int*>(static_cast<uint8_t*>(workspace) + partial_bytes_for(&d, plan))
-                        : nullptr;
+  p.ws_part = need > 0 ? static_cast<uint32_t*>(workspace) : nullptr;
   p.out_bf16 = d.out_dtype;
   const double cb = d.hadamard_block > 0 ? 1.0 / std::sqrt((double)d.hadamard_block) : 1.0;
   const double scale = d.softmax_scale > 0.0f ? (double)d.softmax_scale : 1.0 / std::sqrt((double)d.head_dim);

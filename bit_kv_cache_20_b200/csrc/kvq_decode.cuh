@@ -44,10 +44,10 @@
 // when the running maximum grows. q is rotated once per CTA in shared memory.
 //
 // With one split per (sequence, head group) the CTA rotates its output back
-// and writes it; otherwise it writes a partial result (O + Z, M, L) to the
-// workspace and takes a ticket from the group's counter there; the CTA that
-// takes the last ticket merges all splits, rotates back, writes the output and
-// sets the counter back to zero.
+// and writes it; otherwise every split writes a partial result (O + Z, M, L)
+// to the workspace in a self-validating encoding, and the first few splits
+// each gather, merge, rotate back and write some of the group's query rows
+// (details at the merge below).
 #pragma once
 
 #include <climits>
@@ -64,8 +64,8 @@ struct AttnParams {
   const int32_t* page_table;  // [B][max_pages]
   const int32_t* ctx_lens;    // [B]
   void* out;                  // [B][Hq][D] fp32 or bf16
-  float* ws_part;             // [B][Hkv][n_splits][G][D + 2]: O + Z, then M, L
-  int* ws_count;              // [B][Hkv / HG] tickets, zero between calls
+  uint32_t* ws_part;          // [B][Hkv][n_splits][G][D + 4]: ~bits of O + Z, M, L, 2 unused;
+                              // zero between calls
   int B, Hq, Hkv, G;
   int num_pages, max_pages;
   int n_splits, pages_per_split;
@@ -94,8 +94,7 @@ struct AttnSmem {
   static constexpr int kOffQInfo = kOffQ + kRows * D * 4;       // float [kRows][4]: scale, sum
   static constexpr int kOffQ8 = kOffQInfo + kRows * 16;         // int8 [kRows][3 limbs][D], B order
   static constexpr int kOffPid = kOffQ8 + kRows * 3 * D;
-  static constexpr int kOffFlag = kOffPid + kMaxPids * 4;
-  static constexpr int kTotal = kOffFlag + 16;
+  static constexpr int kTotal = kOffPid + kMaxPids * 4;
 };
 
 template <int N>
@@ -177,7 +176,6 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
   float* qinfo = reinterpret_cast<float*>(smem + S::kOffQInfo);
   int8_t* q8 = reinterpret_cast<int8_t*>(smem + S::kOffQ8);
   int* pids = reinterpret_cast<int*>(smem + S::kOffPid);
-  int* sflag = reinterpret_cast<int*>(smem + S::kOffFlag);
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tig = lane & 3;
@@ -557,86 +555,93 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
       *reinterpret_cast<float4*>(qs + (hh * NR + r) * D + c4) =
           make_float4((O.x + Z) * inv, (O.y + Z) * inv, (O.z + Z) * inv, (O.w + Z) * inv);
     } else {
-      float* dst = p.ws_part + ((((size_t)n * p.Hkv + hgi * HG + hh) * p.n_splits + split) * G + r) * (D + 4);
-      *reinterpret_cast<float4*>(dst + c4) = make_float4(O.x + Z, O.y + Z, O.z + Z, O.w + Z);
-      if (c4 == 0) *reinterpret_cast<float2*>(dst + D) = make_float2(M, L);
+      // the split's partial result, every word stored as ~bits (see below)
+      uint32_t* dst = p.ws_part + ((((size_t)n * p.Hkv + hgi * HG + hh) * p.n_splits + split) * G + r) * (D + 4);
+      *reinterpret_cast<uint4*>(dst + c4) = make_uint4(~__float_as_uint(O.x + Z), ~__float_as_uint(O.y + Z),
+                                                       ~__float_as_uint(O.z + Z), ~__float_as_uint(O.w + Z));
+      if (c4 == 0) *reinterpret_cast<uint2*>(dst + D) = make_uint2(~__float_as_uint(M), ~__float_as_uint(L));
     }
   }
 
   if (!single) {
-    // ---- tickets: the last K arrivals each merge some query rows ----------
-    // (every thread's partial stores are made visible device-wide before the
-    // barrier and thread 0's atomic; a merging CTA reads the partials from L2
-    // with ld.cg once the arrival count shows every split has written)
-    __threadfence();
-    __syncthreads();
+    // ---- split merge: CTA j < K merges query rows j, j + K, ... ------------
+    // Each 32-bit word of a partial result is stored as ~bits(x). fp32
+    // arithmetic never yields the bits 0xFFFFFFFF (a NaN payload it does not
+    // produce), so no stored word is zero, and a zero word of the zero-filled
+    // workspace means that split has not written it yet. A merger polls the
+    // words of its rows in L2 until none is zero - no fence, ticket or counter
+    // between writer and reader, each word validates itself - folds them and
+    // zeroes them again for the next call. Every CTA of the launch is resident
+    // at once, so the splits a merger waits for are running.
     const int ns = p.n_splits;
     const int rows = HG * G;
-    const int K = min(rows, ns);  // merging CTAs; CTA j takes rows j, j + K, ...
-    int* arrive = p.ws_count + ((size_t)n * (p.Hkv / HG) + hgi) * 2;
-    int* done = arrive + 1;
-    if (tid == 0) sflag[0] = atomicAdd(arrive, 1);
-    __syncthreads();
-    const int t = sflag[0];
-    if (t < ns - K) return;
-    if (t < ns - 1) {
-      // not the last arrival: wait (bounded) for the remaining splits; every
-      // CTA of the launch is resident at once, so they are running
-      if (tid == 0) {
-        uint32_t rounds = 0;
-        while (ld_acquire_gpu(arrive) < ns) {
-          __nanosleep(256);
-          if (++rounds > kMaxSpinRounds) {
-            record_error(KVQ_ERR_TIMEOUT);
-            break;
-          }
-        }
-      }
-      __syncthreads();
-    }
-    const int j = t - (ns - K);
+    const int K = min(rows, ns);
+    if (split >= K) return;
     // Merge of one row: warp w takes splits w, w + 8, ...; lane l the output
-    // float4 l. Each warp folds its splits into a running (max, l, acc),
-    // every load of a round (up to 8 splits) issued before any is used; the
-    // warps' states are then combined through shared memory.
+    // float4 l. Each warp folds its splits into a running (max, l, acc), all
+    // loads of a round (up to 8 splits) issued before any is used; the warps'
+    // states are then combined through shared memory.
     constexpr int kRowBatch = 8;
     float* mred = reinterpret_cast<float*>(smem);            // [kAttnWarps] (the rings are free)
     float4* ored = reinterpret_cast<float4*>(smem + 64);     // [kAttnWarps][32]
     float* lred = reinterpret_cast<float*>(smem + 64 + kAttnWarps * 32 * 16);  // [kAttnWarps]
     static_assert(64 + kAttnWarps * 32 * 16 + kAttnWarps * 4 <= S::kRingBytes, "row-merge scratch fits in the rings");
     const size_t sstride = (size_t)G * (D + 4);
-    for (int rr = j; rr < rows; rr += K) {
+    for (int rr = split; rr < rows; rr += K) {
       const int hh = rr / G, r = rr % G;
-      const float* base = p.ws_part + (((size_t)n * p.Hkv + hgi * HG + hh) * ns * G + r) * (D + 4);
+      uint32_t* base = p.ws_part + (((size_t)n * p.Hkv + hgi * HG + hh) * ns * G + r) * (D + 4);
       float mw = -INFINITY, L = 0.0f;
       float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       for (int s0 = warp; s0 < ns; s0 += kAttnWarps * kRowBatch) {
-        float4 v[kRowBatch];
-        float2 ml[kRowBatch];
+        uint4 v[kRowBatch];
+        uint2 ml[kRowBatch];
+        for (uint32_t rounds = 0;; ++rounds) {
+          bool ok = true;
+#pragma unroll
+          for (int k = 0; k < kRowBatch; ++k) {
+            const int s2 = s0 + k * kAttnWarps;
+            v[k] = make_uint4(1u, 1u, 1u, 1u);
+            ml[k] = make_uint2(1u, 1u);
+            if (s2 < ns) {
+              if (lane < D / 4) v[k] = ld_relaxed_gpu_v4(base + s2 * sstride + 4 * lane);
+              ml[k] = ld_relaxed_gpu_v2(base + s2 * sstride + D);
+            }
+            ok = ok && v[k].x && v[k].y && v[k].z && v[k].w && ml[k].x && ml[k].y;
+          }
+          if (__all_sync(FULL, ok)) break;
+          if (rounds >= kMaxSpinRounds) {
+            if (lane == 0) record_error(KVQ_ERR_TIMEOUT);
+            break;
+          }
+          __nanosleep(64);
+        }
+        __syncwarp();  // every lane holds its words: zero them for the next call
 #pragma unroll
         for (int k = 0; k < kRowBatch; ++k) {
-          const int s2 = min(s0 + k * kAttnWarps, ns - 1);
-          v[k] = (lane < D / 4) ? __ldcg(reinterpret_cast<const float4*>(base + s2 * sstride) + lane)
-                                : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
-          ml[k] = __ldcg(reinterpret_cast<const float2*>(base + s2 * sstride + D));
+          const int s2 = s0 + k * kAttnWarps;
+          if (s2 < ns) {
+            if (lane < D / 4) *reinterpret_cast<uint4*>(base + s2 * sstride + 4 * lane) = make_uint4(0u, 0u, 0u, 0u);
+            if (lane == 0) *reinterpret_cast<uint2*>(base + s2 * sstride + D) = make_uint2(0u, 0u);
+          }
         }
         float mb = mw;
 #pragma unroll
         for (int k = 0; k < kRowBatch; ++k)
-          if (s0 + k * kAttnWarps < ns) mb = fmaxf(mb, ml[k].x);
+          if (s0 + k * kAttnWarps < ns) mb = fmaxf(mb, __uint_as_float(~ml[k].x));
         if (mb == -INFINITY) continue;
         const float a0 = (mw == -INFINITY) ? 0.0f : fast_exp2(mw - mb);
         acc.x *= a0; acc.y *= a0; acc.z *= a0; acc.w *= a0;
         L *= a0;
 #pragma unroll
         for (int k = 0; k < kRowBatch; ++k) {
-          if (s0 + k * kAttnWarps >= ns || ml[k].x == -INFINITY) continue;
-          const float wgt = fast_exp2(ml[k].x - mb);
-          acc.x = fmaf(wgt, v[k].x, acc.x);
-          acc.y = fmaf(wgt, v[k].y, acc.y);
-          acc.z = fmaf(wgt, v[k].z, acc.z);
-          acc.w = fmaf(wgt, v[k].w, acc.w);
-          L = fmaf(wgt, ml[k].y, L);
+          const float mk = __uint_as_float(~ml[k].x);
+          if (s0 + k * kAttnWarps >= ns || mk == -INFINITY) continue;
+          const float wgt = fast_exp2(mk - mb);
+          acc.x = fmaf(wgt, __uint_as_float(~v[k].x), acc.x);
+          acc.y = fmaf(wgt, __uint_as_float(~v[k].y), acc.y);
+          acc.z = fmaf(wgt, __uint_as_float(~v[k].z), acc.z);
+          acc.w = fmaf(wgt, __uint_as_float(~v[k].w), acc.w);
+          L = fmaf(wgt, __uint_as_float(~ml[k].y), L);
         }
         mw = mb;
       }
@@ -675,7 +680,7 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
       __syncthreads();
     }
     // rotate back this CTA's rows (one warp per row) and store
-    for (int rr = j + K * warp; rr < rows; rr += K * kAttnWarps) {
+    for (int rr = split + K * warp; rr < rows; rr += K * kAttnWarps) {
       const int hh = rr / G, r = rr % G;
       const float* rp = qs + (hh * NR + r) * D;
       float v[E];
@@ -685,11 +690,6 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
       const size_t o_base = ((size_t)n * p.Hq + (size_t)(hgi * HG + hh) * G + r) * D + E * lane;
 #pragma unroll
       for (int e2 = 0; e2 < E; ++e2) store_out(p, o_base + e2, BLK > 0 ? v[e2] * p.cb : v[e2]);
-    }
-    // the last of the K merging CTAs resets both counters for the next call
-    if (tid == 0 && atomicAdd(done, 1) == K - 1) {
-      *arrive = 0;
-      *done = 0;
     }
     return;
   }

@@ -52,20 +52,21 @@ __device__ __forceinline__ void cp_async_16_if(uint32_t dst, const void* src, bo
       : "memory");
 }
 
-// Acquire-release fence at GPU scope: orders this thread's earlier memory
-// operations before its later ones as seen by every thread of the device.
-__device__ __forceinline__ void fence_acq_rel_gpu() {
-  asm volatile("fence.acq_rel.gpu;\n" ::: "memory");
+// Relaxed GPU-scope vector loads of global words (served by L2, never by a
+// stale L1 line): polls of words another CTA writes.
+__device__ __forceinline__ uint4 ld_relaxed_gpu_v4(const uint32_t* p) {
+  uint4 v;
+  asm volatile("ld.relaxed.gpu.global.v4.b32 {%0, %1, %2, %3}, [%4];\n"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p) : "memory");
+  return v;
 }
-
-// Acquire load of a global int at GPU scope.
-__device__ __forceinline__ int ld_acquire_gpu(const int* p) {
-  int v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
+__device__ __forceinline__ uint2 ld_relaxed_gpu_v2(const uint32_t* p) {
+  uint2 v;
+  asm volatile("ld.relaxed.gpu.global.v2.b32 {%0, %1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "l"(p) : "memory");
   return v;
 }
 
-// Upper bound on the polls of a spin on a global counter (each with a short
+// Upper bound on the polls of a spin on global words (each with a short
 // sleep): far above any legitimate wait, ends within a fraction of a second.
 constexpr uint32_t kMaxSpinRounds = 1u << 20;
 

@@ -128,9 +128,10 @@ kvq_status kv_quant_write(const void* k, const void* v, const int64_t* slot_mapp
  * in one wave). Returns SIZE_MAX when the shapes are invalid or no device can
  * be queried.
  *
- * The workspace holds per-split partial results (fp32) and one ticket counter
- * per (sequence, head group); it must be zero-filled before its first use,
- * and every call leaves it zero-filled again.
+ * The workspace holds the per-split partial results (fp32, each word stored
+ * bit-inverted so that a zero word means "not written yet"); it must be
+ * zero-filled before its first use, and every call leaves it zero-filled
+ * again.
  */
 size_t kvq_attn_workspace_size(const kvq_attn_desc* desc);
 

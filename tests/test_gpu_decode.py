@@ -161,17 +161,19 @@ def test_decode_explicit_softmax_scale_and_bf16(orc):
 
 
 def test_decode_deterministic_and_workspace_left_zeroed():
-    """Repeated calls on one workspace give identical outputs. Each call must
-    leave the ticket counters at zero: a stale counter would leave no split
-    holding the last ticket, and the output (a fresh buffer of 7.0 per call)
-    would not be written."""
+    """Repeated calls on one workspace give identical outputs, and each call
+    leaves every workspace word at zero: partial results are stored
+    bit-inverted and a merger takes a non-zero word as written, so a stale
+    word would be merged in place of the next call's value."""
     w = workloads.random_case(seed=9, B=2, Hq=16, Hkv=4, D=128, block=128, context_lens=[3000, 777])
     pool = build_cache(w)
     a, ws = gpu_decode(w, pool)
     assert ws.numel() > 16, "the case must use partial results"
+    assert int(torch.count_nonzero(ws)) == 0
     for _ in range(3):
         b_, ws = gpu_decode(w, pool, ws=ws)
         assert np.array_equal(a, b_)
+        assert int(torch.count_nonzero(ws)) == 0
 
 
 @pytest.mark.parametrize("ctx,Hq,Hkv", [([40000 - 7], 8, 2), ([36001, 2000], 8, 2), ([1, 17, 900], 8, 2),

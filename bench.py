@@ -46,6 +46,8 @@ def parse_args(argv=None):
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-plain", action="store_true")
+    ap.add_argument("--no-graph", action="store_true",
+                    help="time direct launches instead of CUDA graph replays (for profilers)")
     ap.add_argument("--only", choices=["write", "decode"], default=None,
                     help="time one kernel alone (profiling captures); prints its line")
     ap.add_argument("--e2e-steps", type=int, default=100)
@@ -206,7 +208,7 @@ class Step:
 
     N_POOLS = 4
 
-    def __init__(self, w, block, dev):
+    def __init__(self, w, block, dev, graph=True):
         import ctypes
         import torch
         import bit_kv_cache_20_b200 as kvq
@@ -214,7 +216,7 @@ class Step:
 
         self.torch, self.kvq, self.ct = torch, kvq, ctypes
         self.L = _lib.lib()
-        self.w, self.b, self.dev = w, block, dev
+        self.w, self.b, self.dev, self.graph = w, block, dev, graph
         k0 = w.k_new.to(dev)
         v0 = w.v_new.to(dev)
         self.kv_sets = [(k0, v0), (k0.clone(), v0.clone())]
@@ -291,15 +293,34 @@ class Step:
         t1.synchronize()
         return t0.elapsed_time(t1)
 
+    def direct_ms(self, kinds, steps, start_index=0):
+        """The same launches issued directly on the stream between two events."""
+        torch = self.torch
+        fns = [self.write if k == "write" else self.decode for k in kinds]
+        t0 = torch.cuda.Event(enable_timing=True)
+        t1 = torch.cuda.Event(enable_timing=True)
+        t0.record(self.stream)
+        for j in range(steps):
+            for fn in fns:
+                fn(start_index + j)
+        t1.record(self.stream)
+        t1.synchronize()
+        return t0.elapsed_time(t1)
+
+    def run_ms(self, kinds, steps, start_index=0):
+        if not self.graph:
+            return self.direct_ms(kinds, steps, start_index)
+        return self.replay_ms(self.capture(kinds, steps, start_index))
+
     def timed_only(self, kind, steps, start_index=0):
         """One kernel alone, `steps` back-to-back launches (inputs and outputs
         rotate through sets larger than L2). Returns the average ms per launch."""
-        return self.replay_ms(self.capture((kind,), steps, start_index)) / steps
+        return self.run_ms((kind,), steps, start_index) / steps
 
     def timed(self, steps, start_index=0):
         """`steps` whole steps (write, then decode) back to back. Returns the
         total ms."""
-        return self.replay_ms(self.capture(("write", "decode"), steps, start_index))
+        return self.run_ms(("write", "decode"), steps, start_index)
 
 
 def e2e_run(w, block, dev, steps, warmup):
@@ -400,7 +421,7 @@ def run_reference(args):
         "n_gpus": args.gpus, "steps": args.steps, "warmup": warm,
         "ms_per_step": round(1e3 * total_t / max(args.steps, 1), 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": config_block(w, block),
+        "config": config_block(w, block, not args.no_graph),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": oracle.num_threads(),
                          "kind": "oracle",
                          "sample": f"per step: write of {n_tokens} tokens (all kv heads, K and V) + one "
@@ -413,13 +434,16 @@ def run_reference(args):
 METRIC = "fused rot+INT4 KV write & INT4 paged decode attn: HBM GB/s, % of peak"
 
 
-def config_block(w, block):
+def config_block(w, block, graph=True):
+    timing = ("the K steps as one CUDA graph (replayed once untimed, then once between two events)"
+              if graph else "the K steps launched directly, back to back between two events")
     return {
         "workload": w.cfg.name, "batch": w.B, "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D,
         "context": int(w.context_lens.max()), "written_tokens": w.tokens_written, "page": 16,
         "hadamard_block": block, "out_dtype": "bf16",
         "l2": "inputs larger than L2 rotate; decode reads a cache written two steps earlier",
-        "timing": "the K steps as one CUDA graph (replayed once untimed, then once between two events); each kernel's line: the same, that kernel alone",
+        "timing": timing + "; each kernel's line: the same, that kernel alone, median of 3 "
+                           "(alternating with the plain-INT4 kernel)",
     }
 
 
@@ -474,7 +498,7 @@ def main(argv=None):
     def max_over_ranks(x):
         return reduce_max(x, world, dev)
 
-    step = Step(w, block, dev)
+    step = Step(w, block, dev, graph=not args.no_graph)
     step.fill_pools()
     if args.only:
         step.timed_only(args.only, warm)
@@ -485,41 +509,51 @@ def main(argv=None):
             nb = wb if args.only == "write" else db
             print(json.dumps({"only": args.only, "us": round(1e3 * mean, 3),
                               "GB/s": round(nb / (mean / 1e3) / 1e9, 2), "launches": args.steps,
-                              "config": config_block(w, block)}), flush=True)
+                              "config": config_block(w, block, not args.no_graph)}), flush=True)
         if world > 1:
             dist.destroy_process_group()
         return 0
+    # the plain-INT4 comparator (block 0) on the same workload; its kernels are
+    # timed in alternation with the rotated ones, so that drifting clocks or
+    # power cannot bias the rotation overhead
+    p = None
+    if not args.no_plain and block != 0:
+        p = Step(w, 0, dev, graph=not args.no_graph)
+        p.fill_pools()
+    rounds = 3
     with ClockSampler(local) as clocks:
         clocks.wait_first_sample()
         step.timed(warm)                    # warm-up steps (untimed)
+        if p is not None:
+            p.timed(warm)
         barrier()
         t_host0 = time.monotonic()
         total_ms = step.timed(args.steps, start_index=warm)
         barrier()
-        # each kernel alone, back to back, for its own roofline line
-        wr_ms = step.timed_only("write", args.steps, start_index=warm)
+        p_total = p.timed(args.steps, start_index=warm) if p is not None else None
         barrier()
-        de_ms = step.timed_only("decode", args.steps, start_index=warm)
+        # each kernel alone, back to back, for its own line: the median of
+        # `rounds` measurements, rotated and plain alternating
+        ms = {k: [] for k in ("write", "decode", "p_write", "p_decode")}
+        for _ in range(rounds):
+            for kind in ("write", "decode"):
+                ms[kind].append(step.timed_only(kind, args.steps, start_index=warm))
+                barrier()
+                if p is not None:
+                    ms["p_" + kind].append(p.timed_only(kind, args.steps, start_index=warm))
+                    barrier()
         t_host1 = time.monotonic()
         clocks.mark(t_host0, t_host1)
     barrier()
     total_ms = max_over_ranks(total_ms)
-    wr_ms = max_over_ranks(wr_ms)
-    de_ms = max_over_ranks(de_ms)
+    wr_ms = max_over_ranks(statistics.median(ms["write"]))
+    de_ms = max_over_ranks(statistics.median(ms["decode"]))
 
     plain = None
-    if not args.no_plain and block != 0:
-        p = Step(w, 0, dev)
-        p.fill_pools()
-        p.timed(warm)
-        barrier()
-        p_total = p.timed(args.steps, start_index=warm)
-        barrier()
-        p_wr_ms = max_over_ranks(p.timed_only("write", args.steps, start_index=warm))
-        barrier()
-        p_de_ms = max_over_ranks(p.timed_only("decode", args.steps, start_index=warm))
-        barrier()
+    if p is not None:
         p_total = max_over_ranks(p_total)
+        p_wr_ms = max_over_ranks(statistics.median(ms["p_write"]))
+        p_de_ms = max_over_ranks(statistics.median(ms["p_decode"]))
         plain = {
             "hadamard_block": 0,
             "kv_quant_write_us": round(1e3 * p_wr_ms, 3),
@@ -556,7 +590,7 @@ def main(argv=None):
         "metric": METRIC, "value": round(value, 3), "unit": "GB/s", "n_gpus": world,
         "steps": args.steps, "warmup": warm, "ms_per_step": round(total_ms / args.steps, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "fp32",
-        "data": "synthetic", "config": config_block(w, block),
+        "data": "synthetic", "config": config_block(w, block, not args.no_graph),
         "pct_of_peak": round(100 * value / (peak * world), 2),
         "roofline": {"kernel": "kv_quant_write", "bound": "hbm", "achieved": round(w_gbs, 2),
                      "peak": peak, "unit": "GB/s", "frac": round(w_gbs / peak, 4),

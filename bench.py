@@ -232,7 +232,10 @@ class Step:
         self.stream = torch.cuda.Stream(dev)
         self.sh = ctypes.c_void_p(self.stream.cuda_stream)
         self.wdesc = _lib.WriteDesc(w.tokens_written, w.Hkv, w.D, 16, w.num_pages)
-        self.adesc = _lib.AttnDesc(w.B, w.Hq, w.Hkv, w.D, 16, w.num_pages, w.max_pages, block, 0.0, 1)
+        # q, the page table and the context lengths are set up once, never
+        # written by the write kernel that precedes each decode
+        self.adesc = _lib.AttnDesc(w.B, w.Hq, w.Hkv, w.D, 16, w.num_pages, w.max_pages, block, 0.0, 1,
+                                   _lib.ATTN_INPUTS_READY)
         P = ctypes.c_void_p
         self.write_args = []
         for i in range(self.N_POOLS):

@@ -18,7 +18,7 @@ from typing import Optional, Tuple
 import torch
 
 from . import _lib
-from ._lib import AttnDesc, KVQError, WriteDesc
+from ._lib import ATTN_INPUTS_READY, AttnDesc, KVQError, WriteDesc
 
 PAGE_SIZE = 16
 
@@ -100,7 +100,8 @@ def kv_quant_write(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
     _lib.check(st, "kv_quant_write")
 
 
-def _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scale, out_dtype):
+def _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scale, out_dtype,
+               inputs_ready=False):
     P, Hkv, D = _pool_shape(cache, scales, zeros)
     if q.dim() != 3 or int(q.shape[2]) != D:
         raise ValueError("q must be bf16 [B, Hq, D]")
@@ -108,7 +109,7 @@ def _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scal
     if page_table.dim() != 2 or int(page_table.shape[0]) != B:
         raise ValueError("page_table must be int32 [B, max_pages]")
     return AttnDesc(B, Hq, Hkv, D, PAGE_SIZE, P, int(page_table.shape[1]), int(hadamard_block),
-                    float(softmax_scale), out_dtype)
+                    float(softmax_scale), out_dtype, ATTN_INPUTS_READY if inputs_ready else 0)
 
 
 def attn_workspace_size(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
@@ -121,7 +122,7 @@ def attn_workspace_size(batch: int, num_q_heads: int, num_kv_heads: int, head_di
     dev = torch.cuda.current_device() if idx is None else idx
     _lib.check(L.kvq_set_device(int(dev)), "kvq_set_device")
     desc = AttnDesc(batch, num_q_heads, num_kv_heads, head_dim, PAGE_SIZE, num_pages,
-                    max_pages_per_seq, hadamard_block, 0.0, 0)
+                    max_pages_per_seq, hadamard_block, 0.0, 0, 0)
     n = L.kvq_attn_workspace_size(ctypes.byref(desc))
     if n == ctypes.c_size_t(-1).value:
         raise KVQError(1, "kvq_attn_workspace_size (invalid shapes or no device)")
@@ -137,8 +138,11 @@ def paged_decode_attn_int4(q: torch.Tensor, cache: torch.Tensor, scales: torch.T
                            zeros: torch.Tensor, page_table: torch.Tensor,
                            context_lens: torch.Tensor, out: torch.Tensor, hadamard_block: int,
                            workspace: Optional[torch.Tensor] = None, softmax_scale: float = 0.0,
-                           stream=None) -> None:
-    """One decode step over the INT4 cache; out is fp32 or bf16 [B, Hq, D]."""
+                           stream=None, inputs_ready: bool = False) -> None:
+    """One decode step over the INT4 cache; out is fp32 or bf16 [B, Hq, D].
+    inputs_ready: q, page_table and context_lens were not written by the
+    kernel launched just before this call on the stream (KVQ_ATTN_INPUTS_READY),
+    so the call may read them while that kernel finishes."""
     _need(q, "q", torch.bfloat16)
     _need(page_table, "page_table", torch.int32)
     _need(context_lens, "context_lens", torch.int32)
@@ -148,7 +152,7 @@ def paged_decode_attn_int4(q: torch.Tensor, cache: torch.Tensor, scales: torch.T
     if tuple(out.shape) != tuple(q.shape):
         raise ValueError("out must have q's shape")
     desc = _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scale,
-                      0 if out.dtype == torch.float32 else 1)
+                      0 if out.dtype == torch.float32 else 1, inputs_ready)
     if context_lens.numel() != desc.batch:
         raise ValueError("context_lens must hold one length per sequence")
     L = _lib.lib()

@@ -26,7 +26,11 @@ class AttnDesc(ctypes.Structure):
                 ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32),
                 ("max_pages_per_seq", ctypes.c_int32), ("hadamard_block", ctypes.c_int32),
-                ("softmax_scale", ctypes.c_float), ("out_dtype", ctypes.c_int32)]
+                ("softmax_scale", ctypes.c_float), ("out_dtype", ctypes.c_int32),
+                ("flags", ctypes.c_int32)]
+
+
+ATTN_INPUTS_READY = 1  # KVQ_ATTN_INPUTS_READY
 
 
 class KVQError(RuntimeError):

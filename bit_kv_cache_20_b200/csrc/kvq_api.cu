@@ -6,6 +6,7 @@
 
 #include <atomic>
 #include <mutex>
+#include <utility>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -16,6 +17,27 @@
 #include "kvq_write_tc.cuh"
 
 namespace {
+
+// Launch with programmatic stream serialization (see KVQ_ATTN_INPUTS_READY in
+// kvq.h): the kernel's CTAs may start while the previous kernel on the stream
+// drains; every kernel here waits for it (griddepcontrol.wait) before
+// touching memory that kernel may have written.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, int smem, cudaStream_t s,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = (size_t)smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+}
+
 
 constexpr int kMaxDevices = 64;
 
@@ -107,8 +129,11 @@ kvq_status launch_write(const kvq::WriteParams& p, int dev, cudaStream_t s) {
   const long long need = (p.num_tiles + kvq::kWriteWarps - 1) / kvq::kWriteWarps;
   const long long cap = (long long)per_sm * sm_count(dev);
   const int blocks = (int)(need < cap ? need : cap);
-  kern<<<blocks, threads, smem, s>>>(p);
-  return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+  if (launch_pdl(kern, dim3(blocks), dim3(threads), smem, s, p) != cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
+  return KVQ_OK;
 }
 
 // Tiled tensor maps of K and V ([T][Hkv*D] bf16, boxes of 128 rows x 64
@@ -166,8 +191,11 @@ kvq_status launch_write_tc(const kvq::WriteParams& p, int dev, cudaStream_t s) {
   const int sms = sm_count(dev);
   if (sms < 1) return KVQ_ERR_CUDA;
   const int grid = (int)(tiles < sms ? tiles : sms);
-  kern<<<grid, kvq::kTcThreads, smem, s>>>(tk, tv, p, (int)tiles);
-  return cudaGetLastError() == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
+  if (launch_pdl(kern, dim3(grid), dim3(kvq::kTcThreads), smem, s, tk, tv, p, (int)tiles) != cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
+  return KVQ_OK;
 }
 
 template <int D>
@@ -309,6 +337,7 @@ kvq_status check_attn_desc(const kvq_attn_desc* d) {
   if (d->max_pages_per_seq > INT_MAX / KVQ_PAGE_SIZE) return KVQ_ERR_INVALID_ARG;
   if (!(d->softmax_scale >= 0.0f) || !std::isfinite(d->softmax_scale)) return KVQ_ERR_INVALID_ARG;
   if (d->out_dtype != 0 && d->out_dtype != 1) return KVQ_ERR_INVALID_ARG;
+  if ((d->flags & ~KVQ_ATTN_INPUTS_READY) != 0) return KVQ_ERR_INVALID_ARG;
   const int G = d->num_q_heads / d->num_kv_heads;
   if (d->head_dim != 64 && d->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
   if (G != 1 && G != 2 && G != 4 && G != 8) return KVQ_ERR_UNSUPPORTED;
@@ -327,16 +356,15 @@ size_t workspace_bytes_for(const kvq_attn_desc* d, const SplitPlan& plan) {
 template <int D, int BLK, int NC>
 cudaError_t launch_decode_instance(const kvq::AttnParams& p, int hg, int smem, cudaStream_t s) {
   const dim3 grid(p.n_splits, p.Hkv / hg, p.B);
+  const dim3 block(kvq::kAttnThreads);
+  cudaError_t e = cudaErrorInvalidValue;
   if constexpr (NC == 1) {
-    if (hg == 4) {
-      kvq::kvq_decode_kernel<D, BLK, 4, NC><<<grid, kvq::kAttnThreads, smem, s>>>(p);
-      return cudaGetLastError();
-    }
+    if (hg == 4) e = launch_pdl(kvq::kvq_decode_kernel<D, BLK, 4, NC>, grid, block, smem, s, p);
   }
-  if (hg == 2) kvq::kvq_decode_kernel<D, BLK, 2, NC><<<grid, kvq::kAttnThreads, smem, s>>>(p);
-  else if (hg == 1) kvq::kvq_decode_kernel<D, BLK, 1, NC><<<grid, kvq::kAttnThreads, smem, s>>>(p);
-  else return cudaErrorInvalidValue;
-  return cudaGetLastError();
+  if (hg == 2) e = launch_pdl(kvq::kvq_decode_kernel<D, BLK, 2, NC>, grid, block, smem, s, p);
+  else if (hg == 1) e = launch_pdl(kvq::kvq_decode_kernel<D, BLK, 1, NC>, grid, block, smem, s, p);
+  if (e != cudaSuccess) cudaGetLastError();
+  return e;
 }
 
 template <int D, int BLK>
@@ -451,6 +479,7 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const voi
   p.pages_per_split = plan.pages_per_split;
   p.ws_part = need > 0 ? static_cast<uint32_t*>(workspace) : nullptr;
   p.out_bf16 = d.out_dtype;
+  p.inputs_ready = (d.flags & KVQ_ATTN_INPUTS_READY) ? 1 : 0;
   const double cb = d.hadamard_block > 0 ? 1.0 / std::sqrt((double)d.hadamard_block) : 1.0;
   const double scale = d.softmax_scale > 0.0f ? (double)d.softmax_scale : 1.0 / std::sqrt((double)d.head_dim);
   p.qmul = (float)(cb * scale * 1.4426950408889634);  // log2(e)

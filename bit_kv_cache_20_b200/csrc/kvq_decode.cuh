@@ -72,6 +72,7 @@ struct AttnParams {
   int out_bf16;
   float qmul;                 // c_b * softmax_scale * log2(e)
   float cb;                   // c_b (output rotation), 1 for plain INT4
+  int inputs_ready;           // q, page_table, ctx_lens not written by the previous kernel
 };
 
 constexpr int kAttnWarps = 8;
@@ -184,6 +185,16 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
   const int G = p.G;
   const unsigned FULL = 0xffffffffu;
 
+  // The launch may overlap the previous kernel on the stream (programmatic
+  // dependent launch). By default everything waits for it here; with
+  // inputs_ready the page ids, context length and q are read and q is
+  // rotated first, and the wait comes before the first cache read.
+  const bool early = p.inputs_ready != 0;
+  if (!early) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
+
   // Page ids of the split's range (the page-table row is max_pages long, so
   // they are read before the context length is known), the context length,
   // and the query rows of the CTA's heads (fp32, rows >= G zero).
@@ -255,10 +266,7 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
     valid = ok ? (valid | (1u << slot)) : (valid & ~(1u << slot));
     cp_async_commit();
   };
-#pragma unroll
-  for (int k = 0; k < R - 1; ++k) fetch(k);
-
-  // ---- q~ = R q * (softmax_scale * log2 e) while the first pages land -----
+  // ---- q~ = R q * (softmax_scale * log2 e) -----------------------------------
   // One warp per row. Limbs, with a = q~ / sigma and sigma = max|q~| / 127:
   // q0 = rint(a), r1 = 256 (a - q0), q1 = rint(r1), q2 = rint(128 (r1 - q1))
   // (every step exact in fp32; |q1|, |q2| <= 64 except at exact ties, where
@@ -266,49 +274,62 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
   // order: element 8w + j goes to byte tig*8KW + ((m*2 + (j&1))*2 + h)*4 +
   // (j>>1) of its limb's array, w = KW*tig + 2m + h, so that thread tig reads
   // its fragments as 8KW contiguous bytes.
-  for (int row = warp; row < S::kRows; row += kAttnWarps) {
-    const float* rp = qs + row * D;
-    float v[E];
+  auto prep_q = [&]() {
+    for (int row = warp; row < S::kRows; row += kAttnWarps) {
+      const float* rp = qs + row * D;
+      float v[E];
 #pragma unroll
-    for (int e = 0; e < E; ++e) v[e] = rp[E * lane + e];
-    if constexpr (BLK > 0) warp_fwht<D, BLK>(v, lane);
-    float amax = 0.0f, sum = 0.0f;
+      for (int e = 0; e < E; ++e) v[e] = rp[E * lane + e];
+      if constexpr (BLK > 0) warp_fwht<D, BLK>(v, lane);
+      float amax = 0.0f, sum = 0.0f;
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      v[e] *= p.qmul;
-      amax = fmaxf(amax, fabsf(v[e]));
-      sum += v[e];
-    }
+      for (int e = 0; e < E; ++e) {
+        v[e] *= p.qmul;
+        amax = fmaxf(amax, fabsf(v[e]));
+        sum += v[e];
+      }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o));
-      sum += __shfl_xor_sync(FULL, sum, o);
-    }
-    const float sigma = amax / 127.0f;
-    const float inv = (amax > 0.0f) ? 127.0f / amax : 0.0f;
-    if (lane == 0) {
-      qinfo[row * 4 + 0] = sigma * (1.0f / 16.0f);
-      qinfo[row * 4 + 1] = sum;
-    }
-    int8_t* l0 = q8 + row * 3 * D;
-    int8_t* l1 = l0 + D;
-    int8_t* l2 = l1 + D;
+      for (int o = 16; o > 0; o >>= 1) {
+        amax = fmaxf(amax, __shfl_xor_sync(FULL, amax, o));
+        sum += __shfl_xor_sync(FULL, sum, o);
+      }
+      const float sigma = amax / 127.0f;
+      const float inv = (amax > 0.0f) ? 127.0f / amax : 0.0f;
+      if (lane == 0) {
+        qinfo[row * 4 + 0] = sigma * (1.0f / 16.0f);
+        qinfo[row * 4 + 1] = sum;
+      }
+      int8_t* l0 = q8 + row * 3 * D;
+      int8_t* l1 = l0 + D;
+      int8_t* l2 = l1 + D;
 #pragma unroll
-    for (int e = 0; e < E; ++e) {
-      const int el = E * lane + e, w = el >> 3, j = el & 7;
-      const int tw = w / KW, rw = w % KW;
-      const int off = tw * (8 * KW) + (((rw >> 1) * 2 + (j & 1)) * 2 + (rw & 1)) * 4 + (j >> 1);
-      const float a = __fmul_rn(v[e], inv);
-      const float q0 = rintf(a);
-      const float r1 = __fmul_rn(__fsub_rn(a, q0), 256.0f);
-      const float q1 = fminf(fmaxf(rintf(r1), -127.0f), 127.0f);
-      const float q2 = fminf(fmaxf(rintf(__fmul_rn(__fsub_rn(r1, q1), 128.0f)), -127.0f), 127.0f);
-      l0[off] = (int8_t)(int)q0;
-      l1[off] = (int8_t)(int)q1;
-      l2[off] = (int8_t)(int)q2;
+      for (int e = 0; e < E; ++e) {
+        const int el = E * lane + e, w = el >> 3, j = el & 7;
+        const int tw = w / KW, rw = w % KW;
+        const int off = tw * (8 * KW) + (((rw >> 1) * 2 + (j & 1)) * 2 + (rw & 1)) * 4 + (j >> 1);
+        const float a = __fmul_rn(v[e], inv);
+        const float q0 = rintf(a);
+        const float r1 = __fmul_rn(__fsub_rn(a, q0), 256.0f);
+        const float q1 = fminf(fmaxf(rintf(r1), -127.0f), 127.0f);
+        const float q2 = fminf(fmaxf(rintf(__fmul_rn(__fsub_rn(r1, q1), 128.0f)), -127.0f), 127.0f);
+        l0[off] = (int8_t)(int)q0;
+        l1[off] = (int8_t)(int)q1;
+        l2[off] = (int8_t)(int)q2;
+      }
     }
+    __syncthreads();
+  };
+  if (early) {
+    prep_q();    // overlaps the previous kernel's last CTAs
+    pdl_wait();  // the cache may be what that kernel wrote
+    pdl_launch_dependents();
+#pragma unroll
+    for (int k = 0; k < R - 1; ++k) fetch(k);
+  } else {
+#pragma unroll
+    for (int k = 0; k < R - 1; ++k) fetch(k);
+    prep_q();    // while the first pages land
   }
-  __syncthreads();
 
   // B fragments of QK. Tile 0: column g is limb g&1 of query row 4c + g/2 of
   // head hw; tile 1: column g is limb 2 of that row for even g, zero for odd.

@@ -52,6 +52,17 @@ __device__ __forceinline__ void cp_async_16_if(uint32_t dst, const void* src, bo
       : "memory");
 }
 
+// Programmatic dependent launch. Kernels are launched so that their CTAs may
+// start while the previous kernel on the stream drains; pdl_wait() returns
+// once that kernel has completed and its memory operations are visible (at
+// once when the launch was not programmatic). After its own wait a kernel
+// lets the next one start launching: what ran before this kernel is then
+// complete as well, so chains stay ordered.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory");
+}
+
 // Relaxed GPU-scope vector loads of global words (served by L2, never by a
 // stale L1 line): polls of words another CTA writes.
 __device__ __forceinline__ uint4 ld_relaxed_gpu_v4(const uint32_t* p) {

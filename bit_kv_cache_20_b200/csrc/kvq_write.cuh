@@ -75,6 +75,8 @@ __global__ void __launch_bounds__(kWriteWarps * 32, 3) kvq_write_kernel(const Wr
   constexpr int CPR = ROWB / 16;    // 16-byte chunks per row (8 or 16)
   constexpr int RPI = 32 / CPR;     // rows covered by one warp-wide copy instruction
   extern __shared__ __align__(128) uint8_t smem[];
+  pdl_wait();  // the previous kernel on the stream may still read the cache or write K, V
+  pdl_launch_dependents();
   const int lane = threadIdx.x & 31;
   const int warp = threadIdx.x >> 5;
   uint8_t* wbuf = smem + warp * 32 * ROWB;

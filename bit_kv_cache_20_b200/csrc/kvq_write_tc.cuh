@@ -138,6 +138,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   }
   const uint32_t tmem = *tslot;
   const int first = blockIdx.x, stride = gridDim.x;
+  // Everything above touched only this CTA's shared and tensor memory, so it
+  // overlaps the previous kernel's last CTAs; global memory waits for it.
+  pdl_wait();
+  pdl_launch_dependents();
 
   if (warp == 0) {
     // ---- TMA producer --------------------------------------------------------

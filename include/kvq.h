@@ -49,7 +49,7 @@ extern "C" {
 #endif
 
 #define KVQ_PAGE_SIZE 16
-#define KVQ_ABI_VERSION 1
+#define KVQ_ABI_VERSION 2
 
 typedef enum kvq_status {
   KVQ_OK = 0,
@@ -82,7 +82,23 @@ typedef struct kvq_attn_desc {
   int32_t hadamard_block;    /* the block b the cache was written with (0 = none) */
   float softmax_scale;       /* 0 means 1/sqrt(head_dim) */
   int32_t out_dtype;         /* 0 = fp32 output, 1 = bf16 output */
+  int32_t flags;             /* 0 or KVQ_ATTN_INPUTS_READY */
 } kvq_attn_desc;
+
+/*
+ * Every kernel of this library is launched as a programmatic dependent
+ * launch: its CTAs may start while the previous kernel on the stream is
+ * finishing, and wait for that kernel to complete before touching memory it
+ * may have written. KVQ_ATTN_INPUTS_READY tells paged_decode_attn_int4 that
+ * q, page_table and context_lens were not written by the kernel launched
+ * just before it on the stream (they may be written by anything earlier:
+ * every kernel of this library waits for its predecessor before letting its
+ * own successor start), so it may read them and rotate q while that kernel
+ * is still running. kv_quant_write followed by paged_decode_attn_int4 on
+ * the same stream qualifies when q, the page table and the context lengths
+ * came from before the write.
+ */
+#define KVQ_ATTN_INPUTS_READY 1
 
 /*
  * kv_quant_write - fused rotate + token-wise INT4 quantize + paged store

@@ -47,7 +47,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_version_and_status_strings(L):
-    assert L.kvq_abi_version() == 1
+    assert L.kvq_abi_version() == 2
     assert L.kvq_status_string(0) == b"KVQ_OK"
     assert L.kvq_status_string(5) == b"KVQ_ERR_TIMEOUT"
     assert L.kvq_status_string(99) == b"KVQ_ERR_UNKNOWN"
@@ -88,7 +88,7 @@ def attn_call(L, desc, ws=None, ws_bytes=0, out=FAKE):
 def test_decode_argument_errors(L):
     from bit_kv_cache_20_b200._lib import AttnDesc
     ok = dict(batch=2, num_q_heads=8, num_kv_heads=2, head_dim=128, page_size=16, num_pages=10,
-              max_pages_per_seq=5, hadamard_block=128, softmax_scale=0.0, out_dtype=0)
+              max_pages_per_seq=5, hadamard_block=128, softmax_scale=0.0, out_dtype=0, flags=0)
 
     def d(**kw):
         a = dict(ok)
@@ -103,6 +103,7 @@ def test_decode_argument_errors(L):
     assert attn_call(L, d(page_size=32)) == 1
     assert attn_call(L, d(softmax_scale=-1.0)) == 1
     assert attn_call(L, d(out_dtype=3)) == 1
+    assert attn_call(L, d(flags=2)) == 1                            # unknown flag bit
     assert attn_call(L, d(max_pages_per_seq=0)) == 1
     assert attn_call(L, d(), out=FAKE + 2) == 1                     # fp32 out misaligned
     assert attn_call(L, d(batch=0)) == 0                            # nothing to do

@@ -210,6 +210,7 @@ class Step:
 
     def __init__(self, w, block, dev, graph=True):
         import ctypes
+        import numpy as np
         import torch
         import bit_kv_cache_20_b200 as kvq
         from bit_kv_cache_20_b200 import _lib
@@ -226,7 +227,8 @@ class Step:
         self.pt = torch.as_tensor(w.page_table).to(dev)
         self.ctx = torch.as_tensor(w.context_lens).to(dev)
         self.out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
-        nbytes = kvq.attn_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.num_pages, w.max_pages, block)
+        nbytes = kvq.attn_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.num_pages, w.max_pages, block,
+                                         host_lengths=True)
         self.ws = kvq.alloc_workspace(nbytes, device=dev)
         self.ws_bytes = self.ws.numel()
         self.stream = torch.cuda.Stream(dev)
@@ -234,8 +236,12 @@ class Step:
         self.wdesc = _lib.WriteDesc(w.tokens_written, w.Hkv, w.D, 16, w.num_pages)
         # q, the page table and the context lengths are set up once, never
         # written by the write kernel that precedes each decode
+        # with the host copy of the context lengths (a serving engine has it)
+        # the work is split per sequence in proportion to its length
+        self.lens_host = np.ascontiguousarray(w.context_lens, dtype=np.int32)
         self.adesc = _lib.AttnDesc(w.B, w.Hq, w.Hkv, w.D, 16, w.num_pages, w.max_pages, block, 0.0, 1,
-                                   _lib.ATTN_INPUTS_READY)
+                                   _lib.ATTN_INPUTS_READY,
+                                   self.lens_host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
         P = ctypes.c_void_p
         self.write_args = []
         for i in range(self.N_POOLS):

@@ -15,6 +15,7 @@ from __future__ import annotations
 import ctypes
 from typing import Optional, Tuple
 
+import numpy as np
 import torch
 
 from . import _lib
@@ -100,8 +101,19 @@ def kv_quant_write(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
     _lib.check(st, "kv_quant_write")
 
 
+def _host_lengths(context_lens_host, batch):
+    """int32 host array of the context lengths (kept alive by the caller) and
+    its pointer, or (None, None)."""
+    if context_lens_host is None:
+        return None, None
+    arr = np.ascontiguousarray(np.asarray(context_lens_host, dtype=np.int32))
+    if arr.shape != (batch,):
+        raise ValueError("context_lens_host must hold one length per sequence")
+    return arr, arr.ctypes.data_as(ctypes.POINTER(ctypes.c_int32))
+
+
 def _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scale, out_dtype,
-               inputs_ready=False):
+               inputs_ready=False, lens_ptr=None):
     P, Hkv, D = _pool_shape(cache, scales, zeros)
     if q.dim() != 3 or int(q.shape[2]) != D:
         raise ValueError("q must be bf16 [B, Hq, D]")
@@ -109,20 +121,24 @@ def _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scal
     if page_table.dim() != 2 or int(page_table.shape[0]) != B:
         raise ValueError("page_table must be int32 [B, max_pages]")
     return AttnDesc(B, Hq, Hkv, D, PAGE_SIZE, P, int(page_table.shape[1]), int(hadamard_block),
-                    float(softmax_scale), out_dtype, ATTN_INPUTS_READY if inputs_ready else 0)
+                    float(softmax_scale), out_dtype, ATTN_INPUTS_READY if inputs_ready else 0,
+                    lens_ptr)
 
 
 def attn_workspace_size(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
                         num_pages: int, max_pages_per_seq: int, hadamard_block: int,
-                        device=None) -> int:
+                        device=None, host_lengths: bool = False) -> int:
     """Bytes of workspace paged_decode_attn_int4 needs on `device` (default:
-    torch's current CUDA device)."""
+    torch's current CUDA device); with host_lengths, enough for calls that pass
+    context_lens_host (a per-sequence plan), whatever the lengths."""
     L = _lib.lib()
     idx = None if device is None else torch.device(device).index
     dev = torch.cuda.current_device() if idx is None else idx
     _lib.check(L.kvq_set_device(int(dev)), "kvq_set_device")
+    dummy = (ctypes.c_int32 * 1)(0)
     desc = AttnDesc(batch, num_q_heads, num_kv_heads, head_dim, PAGE_SIZE, num_pages,
-                    max_pages_per_seq, hadamard_block, 0.0, 0, 0)
+                    max_pages_per_seq, hadamard_block, 0.0, 0, 0,
+                    ctypes.cast(dummy, ctypes.POINTER(ctypes.c_int32)) if host_lengths else None)
     n = L.kvq_attn_workspace_size(ctypes.byref(desc))
     if n == ctypes.c_size_t(-1).value:
         raise KVQError(1, "kvq_attn_workspace_size (invalid shapes or no device)")
@@ -138,11 +154,15 @@ def paged_decode_attn_int4(q: torch.Tensor, cache: torch.Tensor, scales: torch.T
                            zeros: torch.Tensor, page_table: torch.Tensor,
                            context_lens: torch.Tensor, out: torch.Tensor, hadamard_block: int,
                            workspace: Optional[torch.Tensor] = None, softmax_scale: float = 0.0,
-                           stream=None, inputs_ready: bool = False) -> None:
+                           stream=None, inputs_ready: bool = False,
+                           context_lens_host=None) -> None:
     """One decode step over the INT4 cache; out is fp32 or bf16 [B, Hq, D].
     inputs_ready: q, page_table and context_lens were not written by the
     kernel launched just before this call on the stream (KVQ_ATTN_INPUTS_READY),
-    so the call may read them while that kernel finishes."""
+    so the call may read them while that kernel finishes.
+    context_lens_host: an optional host copy of the context lengths; the work
+    is then split per sequence in proportion to its length (size the workspace
+    with attn_workspace_size(..., host_lengths=True))."""
     _need(q, "q", torch.bfloat16)
     _need(page_table, "page_table", torch.int32)
     _need(context_lens, "context_lens", torch.int32)
@@ -151,8 +171,9 @@ def paged_decode_attn_int4(q: torch.Tensor, cache: torch.Tensor, scales: torch.T
     _need(out, "out", out.dtype)
     if tuple(out.shape) != tuple(q.shape):
         raise ValueError("out must have q's shape")
+    lens_arr, lens_ptr = _host_lengths(context_lens_host, int(q.shape[0]) if q.dim() == 3 else -1)
     desc = _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scale,
-                      0 if out.dtype == torch.float32 else 1, inputs_ready)
+                      0 if out.dtype == torch.float32 else 1, inputs_ready, lens_ptr)
     if context_lens.numel() != desc.batch:
         raise ValueError("context_lens must hold one length per sequence")
     L = _lib.lib()
@@ -170,7 +191,7 @@ def paged_decode_attn_int4_static_ws(q: torch.Tensor, cache: torch.Tensor, scale
                                      zeros: torch.Tensor, page_table: torch.Tensor,
                                      context_lens: torch.Tensor, out: torch.Tensor,
                                      hadamard_block: int, softmax_scale: float = 0.0,
-                                     stream=None) -> None:
+                                     stream=None, context_lens_host=None) -> None:
     """paged_decode_attn_int4 for callers that must not allocate device memory
     (e.g. a plug-in whose host runtime owns all GPU memory): the split-K
     scratch is a fixed array inside the library, shared by every call on the
@@ -184,8 +205,9 @@ def paged_decode_attn_int4_static_ws(q: torch.Tensor, cache: torch.Tensor, scale
     _need(out, "out", out.dtype)
     if tuple(out.shape) != tuple(q.shape):
         raise ValueError("out must have q's shape")
+    lens_arr, lens_ptr = _host_lengths(context_lens_host, int(q.shape[0]) if q.dim() == 3 else -1)
     desc = _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scale,
-                      0 if out.dtype == torch.float32 else 1)
+                      0 if out.dtype == torch.float32 else 1, False, lens_ptr)
     if context_lens.numel() != desc.batch:
         raise ValueError("context_lens must hold one length per sequence")
     st = _lib.lib().paged_decode_attn_int4_static_ws(

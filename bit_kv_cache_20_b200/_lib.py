@@ -27,7 +27,7 @@ class AttnDesc(ctypes.Structure):
                 ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32),
                 ("max_pages_per_seq", ctypes.c_int32), ("hadamard_block", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("out_dtype", ctypes.c_int32),
-                ("flags", ctypes.c_int32)]
+                ("flags", ctypes.c_int32), ("context_lens_host", ctypes.POINTER(ctypes.c_int32))]
 
 
 ATTN_INPUTS_READY = 1  # KVQ_ATTN_INPUTS_READY

@@ -4,9 +4,11 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <atomic>
 #include <mutex>
 #include <utility>
+#include <vector>
 #include <climits>
 #include <cmath>
 #include <cstdint>
@@ -215,10 +217,12 @@ kvq_status dispatch_write(const kvq::WriteParams& p, int b, int dev, cudaStream_
 // paged_decode_attn_int4
 // ---------------------------------------------------------------------------
 struct SplitPlan {
-  int n_splits;         // CTAs per (sequence, kv-head group) = partials in the workspace
+  int n_splits;         // uniform plan: CTAs per (sequence, kv-head group)
   int pages_per_split;
   int hg;               // kv heads per CTA
   int nc;               // column tiles of 4 query heads
+  int n_items;          // per-sequence plan: entries of AttnParams::items (0 = uniform plan)
+  int part_slots;       // per-sequence plan: partial-result slots it writes
 };
 
 int cols_for(int G) { return G > 4 ? 2 : 1; }
@@ -302,7 +306,7 @@ int decode_ctas_per_sm(int dev, int D, int b, int hg, int nc) {
 SplitPlan plan_splits(const kvq_attn_desc* d, int dev) {
   const int nc = cols_for(d->num_q_heads / d->num_kv_heads);
   const int sms = sm_count(dev);
-  SplitPlan best = {1, d->max_pages_per_seq, 1, nc};
+  SplitPlan best = {1, d->max_pages_per_seq, 1, nc, 0, 0};
   long long best_cost = LLONG_MAX;
   for (int hg = 1; hg <= 4; hg <<= 1) {
     if (d->num_kv_heads % hg != 0 || hg * nc > 4) continue;
@@ -321,8 +325,151 @@ SplitPlan plan_splits(const kvq_attn_desc* d, int dev) {
     const long long cost = (waves < 1 ? 1 : waves) * (pps * hg + 8);
     if (cost < best_cost) {
       best_cost = cost;
-      best = {(int)ns, (int)pps, hg, nc};
+      best = {(int)ns, (int)pps, hg, nc, 0, 0};
     }
+  }
+  return best;
+}
+
+// Per-sequence plan from a host copy of the context lengths. Sequence n
+// (np_n pages) gets ns_n splits so that no CTA holds much more than T
+// head-pages, T the smallest value (not below the average per resident CTA)
+// for which the CTAs of split sequences fit in one wave: those CTAs wait for
+// one another in the split merge, the others never wait, so the launch may
+// take several waves and cannot deadlock. Items (one per (sequence, split),
+// each launched for every kv-head group) are ordered longest first, so that
+// the block scheduler's waves balance (longest-processing-time order). Cost
+// of a plan: max(total work / resident CTAs, the largest CTA) in head-pages
+// plus a fixed 8 per CTA; the cheapest kv-head group size wins. Returns false
+// when the plan does not fit the parameter block (then the uniform plan runs).
+bool plan_lengths(const kvq_attn_desc* d, int dev, SplitPlan* out, uint2* items) {
+  const int B = d->batch;
+  const int32_t* lens = d->context_lens_host;
+  if (!lens || B < 1 || B > kvq::kMaxPlanItems) return false;
+  const int nc = cols_for(d->num_q_heads / d->num_kv_heads);
+  const int sms = sm_count(dev);
+  if (sms < 1) return false;
+  static thread_local std::vector<int> np, ns;
+  static thread_local std::vector<std::pair<long long, int>> order;
+  np.assign(B, 0);
+  ns.assign(B, 1);
+  long long max_np = 0;
+  for (int n = 0; n < B; ++n) {
+    long long c = lens[n];
+    if (c < 0) c = 0;
+    if (c > (long long)d->max_pages_per_seq * KVQ_PAGE_SIZE) c = (long long)d->max_pages_per_seq * KVQ_PAGE_SIZE;
+    np[n] = (int)((c + KVQ_PAGE_SIZE - 1) / KVQ_PAGE_SIZE);
+    if (np[n] > max_np) max_np = np[n];
+  }
+  long long best_cost = LLONG_MAX;
+  int best_hg = 0;
+  long long best_T = 0;
+  for (int hg = 1; hg <= 4; hg <<= 1) {
+    if (d->num_kv_heads % hg != 0 || hg * nc > 4) continue;
+    const int per_sm = decode_ctas_per_sm(dev, d->head_dim, d->hadamard_block, hg, nc);
+    if (per_sm < 1) continue;
+    const long long slots = (long long)per_sm * sms;
+    const long long groups = d->num_kv_heads / hg;
+    long long total = 0;
+    for (int n = 0; n < B; ++n) total += groups * ((long long)np[n] * hg + 8);
+    // splits of sequence n at threshold T; the merge waits need their CTAs in one wave
+    auto splits = [&](int n, long long T) {
+      const long long w = (long long)np[n] * hg;
+      long long k = (w + T - 1) / T;
+      long long cap = np[n] / 4;  // at least 4 pages per split
+      if (cap > kvq::kMaxSplits) cap = kvq::kMaxSplits;
+      if (k > cap) k = cap;
+      return k < 1 ? 1LL : k;
+    };
+    auto fits = [&](long long T) {
+      long long in_merges = 0, n_items = 0;
+      for (int n = 0; n < B; ++n) {
+        const long long k = splits(n, T);
+        n_items += k;
+        if (k > 1) in_merges += k;
+      }
+      return groups * in_merges <= slots && n_items <= kvq::kMaxPlanItems;
+    };
+    long long lo = total / slots, hi = max_np * hg + 1;
+    if (lo < 1) lo = 1;
+    if (lo > hi) lo = hi;
+    if (!fits(hi)) continue;
+    while (lo < hi) {
+      const long long mid = lo + (hi - lo) / 2;
+      if (fits(mid)) hi = mid;
+      else lo = mid + 1;
+    }
+    long long largest = 0;
+    for (int n = 0; n < B; ++n) {
+      const long long k = splits(n, lo);
+      const long long w = ((long long)np[n] + k - 1) / k * hg + 8;
+      if (w > largest) largest = w;
+    }
+    const long long cost = std::max((total + slots - 1) / slots, largest);
+    if (cost < best_cost) {
+      best_cost = cost;
+      best_hg = hg;
+      best_T = lo;
+    }
+  }
+  if (best_hg == 0) return false;
+  const int hg = best_hg;
+  order.clear();
+  int part_slots = 0;
+  for (int n = 0; n < B; ++n) {
+    const long long w = (long long)np[n] * hg;
+    long long k = (w + best_T - 1) / best_T;
+    long long cap = np[n] / 4;
+    if (cap > kvq::kMaxSplits) cap = kvq::kMaxSplits;
+    if (k > cap) k = cap;
+    ns[n] = (int)(k < 1 ? 1 : k);
+    const int pps = np[n] > 0 ? (np[n] + ns[n] - 1) / ns[n] : 1;
+    if (pps > 0xFFFF) return false;
+    for (int sp = 0; sp < ns[n]; ++sp) {
+      const long long pages = std::min<long long>(pps, std::max<long long>(np[n] - (long long)sp * pps, 0));
+      order.push_back({pages, (n << 8) | sp});
+    }
+  }
+  if ((int)order.size() > kvq::kMaxPlanItems) return false;
+  std::stable_sort(order.begin(), order.end(),
+                   [](const std::pair<long long, int>& a, const std::pair<long long, int>& b) { return a.first > b.first; });
+  // partial-result slots: the splits of one sequence take consecutive slots
+  static thread_local std::vector<int> base;
+  base.assign(B, 0);
+  for (int n = 0; n < B; ++n)
+    if (ns[n] > 1) {
+      base[n] = part_slots;
+      part_slots += ns[n];
+    }
+  if (part_slots > 0xFFFF) return false;
+  for (size_t i = 0; i < order.size(); ++i) {
+    const int n = order[i].second >> 8, sp = order[i].second & 0xFF;
+    const int pps = np[n] > 0 ? (np[n] + ns[n] - 1) / ns[n] : 1;
+    items[i] = make_uint2((uint32_t)n | ((uint32_t)sp << 16) | ((uint32_t)ns[n] << 24),
+                          (uint32_t)base[n] | ((uint32_t)pps << 16));
+  }
+  *out = {0, 0, hg, nc, (int)order.size(), part_slots};
+  return true;
+}
+
+// Workspace of a per-sequence plan: its partial slots, each holding every
+// query head's row.
+size_t planned_workspace_bytes(const kvq_attn_desc* d, const SplitPlan& plan) {
+  return (size_t)plan.part_slots * d->num_q_heads * (d->head_dim + 4) * sizeof(uint32_t);
+}
+
+// Bound on planned_workspace_bytes over every context-length vector: the
+// CTAs of split sequences fit in one wave, so at most resident/groups slots.
+size_t planned_workspace_bound(const kvq_attn_desc* d, int dev) {
+  const int nc = cols_for(d->num_q_heads / d->num_kv_heads);
+  const int sms = sm_count(dev);
+  size_t best = 0;
+  for (int hg = 1; hg <= 4; hg <<= 1) {
+    if (d->num_kv_heads % hg != 0 || hg * nc > 4) continue;
+    const int per_sm = decode_ctas_per_sm(dev, d->head_dim, d->hadamard_block, hg, nc);
+    if (per_sm < 1 || sms < 1) continue;
+    const size_t slots = (size_t)per_sm * sms * hg / d->num_kv_heads;
+    best = std::max(best, slots * d->num_q_heads * (d->head_dim + 4) * sizeof(uint32_t));
   }
   return best;
 }
@@ -345,9 +492,12 @@ kvq_status check_attn_desc(const kvq_attn_desc* d) {
   return KVQ_OK;
 }
 
-// Workspace: the splits' partial results, rows of D + 4 words (O + Z, M, L,
-// padding), each word stored as ~bits so that zero means "not written".
+// Workspace: the splits' partial results, slot-major ([slot][Hq] rows of
+// D + 4 words: O + Z, M, L, padding; the uniform plan's slot of split j of
+// sequence n is n * n_splits + j), each word stored as ~bits so that zero
+// means "not written".
 size_t workspace_bytes_for(const kvq_attn_desc* d, const SplitPlan& plan) {
+  if (plan.n_items > 0) return planned_workspace_bytes(d, plan);
   if (plan.n_splits <= 1 || d->batch == 0) return 0;
   const size_t G = (size_t)(d->num_q_heads / d->num_kv_heads);
   return (size_t)d->batch * d->num_kv_heads * plan.n_splits * G * (d->head_dim + 4) * sizeof(uint32_t);
@@ -355,7 +505,7 @@ size_t workspace_bytes_for(const kvq_attn_desc* d, const SplitPlan& plan) {
 
 template <int D, int BLK, int NC>
 cudaError_t launch_decode_instance(const kvq::AttnParams& p, int hg, int smem, cudaStream_t s) {
-  const dim3 grid(p.n_splits, p.Hkv / hg, p.B);
+  const dim3 grid = p.n_items > 0 ? dim3(p.Hkv / hg, p.n_items, 1) : dim3(p.n_splits, p.Hkv / hg, p.B);
   const dim3 block(kvq::kAttnThreads);
   cudaError_t e = cudaErrorInvalidValue;
   if constexpr (NC == 1) {
@@ -437,7 +587,8 @@ size_t kvq_attn_workspace_size(const kvq_attn_desc* desc) {
     return SIZE_MAX;
   }
   if (dev < 0 || dev >= kMaxDevices) return SIZE_MAX;
-  return workspace_bytes_for(desc, plan_splits(desc, dev));
+  const size_t uniform = workspace_bytes_for(desc, plan_splits(desc, dev));
+  return desc->context_lens_host ? std::max(uniform, planned_workspace_bound(desc, dev)) : uniform;
 }
 
 kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const void* scales,
@@ -457,11 +608,22 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const voi
   st = select_device_of(cache, &dev);
   if (st != KVQ_OK) return st;
   if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
-  const SplitPlan plan = plan_splits(&d, dev);
+  // kernel parameters (with the per-sequence plan's items) live in static
+  // storage per thread rather than on the stack: the item table is 8 KB
+  static thread_local kvq::AttnParams p;
+  SplitPlan plan;
+  SplitPlan lp;
+  if (d.context_lens_host && plan_lengths(&d, dev, &lp, p.items) &&
+      (lp.part_slots == 0 || (workspace && aligned(workspace, 16) &&
+                              workspace_bytes >= planned_workspace_bytes(&d, lp)))) {
+    plan = lp;
+  } else {
+    plan = plan_splits(&d, dev);
+  }
   const size_t need = workspace_bytes_for(&d, plan);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16)))
     return KVQ_ERR_WORKSPACE;
-  kvq::AttnParams p;
+  p.n_items = plan.n_items;
   p.q = static_cast<const uint16_t*>(q);
   p.cache = cache;
   p.scales = static_cast<const uint16_t*>(scales);
@@ -576,10 +738,9 @@ extern "C" kvq_status paged_decode_attn_int4_static_ws(const void* q, const uint
   const size_t need = workspace_bytes_for(desc, plan_splits(desc, dev));
   if (need > KVQ_STATIC_WORKSPACE_BYTES) return KVQ_ERR_WORKSPACE;
   void* ws = nullptr;
-  if (need > 0) {
-    st = static_workspace_on(dev, &ws);
-    if (st != KVQ_OK) return st;
-  }
+  st = static_workspace_on(dev, &ws);
+  if (st != KVQ_OK) return st;
+  // a per-sequence plan (host lengths given) runs when its partials fit too
   return paged_decode_attn_int4(q, cache, scales, zeros, page_table, context_lens, out, ws,
-                                need > 0 ? (size_t)KVQ_STATIC_WORKSPACE_BYTES : 0, desc, stream);
+                                (size_t)KVQ_STATIC_WORKSPACE_BYTES, desc, stream);
 }

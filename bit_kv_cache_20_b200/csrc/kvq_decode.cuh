@@ -5,10 +5,13 @@
 // rotates q once, runs attention in the rotated space directly on the codes,
 // and rotates the output back: out = R sum_t p_t v^_t.
 //
-// Grid (split, kv-head group, sequence), 8 warps per CTA, every CTA of the
-// launch resident at once. A CTA serves HG kv heads (HG = 1, 2 or 4) over one
-// contiguous range of pages; warp w works for head w % HG and takes every
-// (8/HG)-th page of the range. Each warp streams its own pages into a private
+// 8 warps per CTA. A CTA serves HG kv heads (HG = 1, 2 or 4) over one
+// contiguous range of one sequence's pages; warp w works for head w % HG and
+// takes every (8/HG)-th page of the range. Grid: (split, kv-head group,
+// sequence) with the same number of splits for every sequence, or, when the
+// host passed its copy of the context lengths, (kv-head group, item) over a
+// per-sequence item table (splits in proportion to length, longest first).
+// The CTAs that take part in split merges are all resident at once. Each warp streams its own pages into a private
 // ring of kWarpRing page slots in shared memory with 16-byte cp.async copies
 // (the codes of one (page, head) are 16*D contiguous bytes; its 32 scales and
 // 32 zeros 64 B each), kWarpRing - 1 pages ahead of the one it computes on.
@@ -56,6 +59,8 @@
 
 namespace kvq {
 
+constexpr int kMaxPlanItems = 1024;  // (sequence, split) entries of a per-sequence plan
+
 struct AttnParams {
   const uint16_t* q;          // bf16 [B][Hq][D]
   const uint8_t* cache;       // [pages][Hkv][2][16][D/2]
@@ -64,7 +69,7 @@ struct AttnParams {
   const int32_t* page_table;  // [B][max_pages]
   const int32_t* ctx_lens;    // [B]
   void* out;                  // [B][Hq][D] fp32 or bf16
-  uint32_t* ws_part;          // [B][Hkv][n_splits][G][D + 4]: ~bits of O + Z, M, L, 2 unused;
+  uint32_t* ws_part;          // [slots][Hkv][G][D + 4]: ~bits of O + Z, M, L, 2 unused;
                               // zero between calls
   int B, Hq, Hkv, G;
   int num_pages, max_pages;
@@ -73,6 +78,12 @@ struct AttnParams {
   float qmul;                 // c_b * softmax_scale * log2(e)
   float cb;                   // c_b (output rotation), 1 for plain INT4
   int inputs_ready;           // q, page_table, ctx_lens not written by the previous kernel
+  // Per-sequence plan (n_items > 0; grid = (Hkv / HG, n_items)): item i is
+  // x = sequence | split << 16 | splits << 24, y = first partial slot of the
+  // sequence | pages per split << 16. Otherwise the grid is (n_splits,
+  // Hkv / HG, B) with pages_per_split pages each and slot n * n_splits + split.
+  int n_items;
+  uint2 items[kMaxPlanItems];
 };
 
 constexpr int kAttnWarps = 8;
@@ -160,7 +171,7 @@ __device__ __forceinline__ void warp_fwht(float (&v)[D / 32], int lane) {
 
 
 template <int D, int BLK, int HG, int NC>
-__global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kernel(const AttnParams p) {
+__global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kernel(const __grid_constant__ AttnParams p) {
   using S = AttnSmem<D, HG, NC>;
   constexpr int NSUB = kAttnWarps / HG;  // warps per head
   constexpr int R = kWarpRing;
@@ -181,7 +192,23 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, tig = lane & 3;
   const int hw = warp % HG, sub = warp / HG;
-  const int split = blockIdx.x, hgi = blockIdx.y, n = blockIdx.z;
+  int n, split, ns, slot_base, pps, hgi;
+  if (p.n_items > 0) {
+    const uint2 it = p.items[blockIdx.y];
+    hgi = blockIdx.x;
+    n = it.x & 0xFFFF;
+    split = (it.x >> 16) & 0xFF;
+    ns = it.x >> 24;
+    slot_base = it.y & 0xFFFF;
+    pps = it.y >> 16;
+  } else {
+    split = blockIdx.x;
+    hgi = blockIdx.y;
+    n = blockIdx.z;
+    ns = p.n_splits;
+    slot_base = n * ns;
+    pps = p.pages_per_split;
+  }
   const int G = p.G;
   const unsigned FULL = 0xffffffffu;
 
@@ -198,10 +225,10 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
   // Page ids of the split's range (the page-table row is max_pages long, so
   // they are read before the context length is known), the context length,
   // and the query rows of the CTA's heads (fp32, rows >= G zero).
-  const int p_begin = split * p.pages_per_split;
-  const int p_cap = min(p_begin + p.pages_per_split, p.max_pages);
+  int p_begin = split * pps;
   const int32_t* pt_row = p.page_table + (size_t)n * p.max_pages + p_begin;
-  for (int i = tid; i < p_cap - p_begin && i < kMaxPids; i += kAttnThreads) pids[i] = pt_row[i];
+  for (int i = tid; i < min(p_begin + pps, p.max_pages) - p_begin && i < kMaxPids; i += kAttnThreads)
+    pids[i] = pt_row[i];
   int ctx = p.ctx_lens[n];
   for (int i = tid; i < S::kRows * (D / 8); i += kAttnThreads) {
     const int row = i / (D / 8), c8 = i % (D / 8);
@@ -230,7 +257,16 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
     ctx = ctx < 0 ? 0 : cap;
   }
   const int n_pages = (ctx + 15) >> 4;
-  const int npg = max(min(p_begin + p.pages_per_split, n_pages) - p_begin, 0);
+  if (n_pages > ns * pps) {
+    // only a per-sequence plan made from host lengths shorter than these:
+    // re-split so that every page is still covered once
+    pps = (n_pages + ns - 1) / ns;
+    p_begin = split * pps;
+    pt_row = p.page_table + (size_t)n * p.max_pages + p_begin;
+    for (int i = tid; i < min(p_begin + pps, p.max_pages) - p_begin && i < kMaxPids; i += kAttnThreads)
+      pids[i] = pt_row[i];
+  }
+  const int npg = max(min(p_begin + pps, n_pages) - p_begin, 0);
   __syncthreads();
 
   // ---- this warp's page stream: pages sub, sub + NSUB, ... of head hw -----
@@ -545,7 +581,7 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
   __syncthreads();
 
   // ---- merge the NSUB warps of each head: output rows or a partial result --
-  const bool single = p.n_splits == 1;
+  const bool single = ns == 1;
   for (int e = tid; e < HG * G * (D / 4); e += kAttnThreads) {
     const int hh = e / (G * (D / 4)), r = (e / (D / 4)) % G, c4 = 4 * (e % (D / 4));
     float mw[NSUB];
@@ -577,7 +613,7 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
           make_float4((O.x + Z) * inv, (O.y + Z) * inv, (O.z + Z) * inv, (O.w + Z) * inv);
     } else {
       // the split's partial result, every word stored as ~bits (see below)
-      uint32_t* dst = p.ws_part + ((((size_t)n * p.Hkv + hgi * HG + hh) * p.n_splits + split) * G + r) * (D + 4);
+      uint32_t* dst = p.ws_part + ((((size_t)slot_base + split) * p.Hkv + hgi * HG + hh) * G + r) * (D + 4);
       *reinterpret_cast<uint4*>(dst + c4) = make_uint4(~__float_as_uint(O.x + Z), ~__float_as_uint(O.y + Z),
                                                        ~__float_as_uint(O.z + Z), ~__float_as_uint(O.w + Z));
       if (c4 == 0) *reinterpret_cast<uint2*>(dst + D) = make_uint2(~__float_as_uint(M), ~__float_as_uint(L));
@@ -594,7 +630,6 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
     // between writer and reader, each word validates itself - folds them and
     // zeroes them again for the next call. Every CTA of the launch is resident
     // at once, so the splits a merger waits for are running.
-    const int ns = p.n_splits;
     const int rows = HG * G;
     const int K = min(rows, ns);
     if (split >= K) return;
@@ -607,10 +642,10 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
     float4* ored = reinterpret_cast<float4*>(smem + 64);     // [kAttnWarps][32]
     float* lred = reinterpret_cast<float*>(smem + 64 + kAttnWarps * 32 * 16);  // [kAttnWarps]
     static_assert(64 + kAttnWarps * 32 * 16 + kAttnWarps * 4 <= S::kRingBytes, "row-merge scratch fits in the rings");
-    const size_t sstride = (size_t)G * (D + 4);
+    const size_t sstride = (size_t)p.Hkv * G * (D + 4);  // between consecutive slots
     for (int rr = split; rr < rows; rr += K) {
       const int hh = rr / G, r = rr % G;
-      uint32_t* base = p.ws_part + (((size_t)n * p.Hkv + hgi * HG + hh) * ns * G + r) * (D + 4);
+      uint32_t* base = p.ws_part + (((size_t)slot_base * p.Hkv + hgi * HG + hh) * G + r) * (D + 4);
       float mw = -INFINITY, L = 0.0f;
       float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       for (int s0 = warp; s0 < ns; s0 += kAttnWarps * kRowBatch) {

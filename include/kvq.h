@@ -49,7 +49,7 @@ extern "C" {
 #endif
 
 #define KVQ_PAGE_SIZE 16
-#define KVQ_ABI_VERSION 2
+#define KVQ_ABI_VERSION 3
 
 typedef enum kvq_status {
   KVQ_OK = 0,
@@ -83,6 +83,12 @@ typedef struct kvq_attn_desc {
   float softmax_scale;       /* 0 means 1/sqrt(head_dim) */
   int32_t out_dtype;         /* 0 = fp32 output, 1 = bf16 output */
   int32_t flags;             /* 0 or KVQ_ATTN_INPUTS_READY */
+  /* Optional host copy of context_lens (B values), or NULL. When given, the
+   * work is split per sequence in proportion to its length (longer sequences
+   * get more CTAs, the longest start first) instead of evenly; the kernel
+   * still reads the lengths from the device array, so a host copy that is
+   * out of date costs balance, never correctness. Read during the call only. */
+  const int32_t* context_lens_host;
 } kvq_attn_desc;
 
 /*

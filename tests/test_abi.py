@@ -47,7 +47,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_version_and_status_strings(L):
-    assert L.kvq_abi_version() == 2
+    assert L.kvq_abi_version() == 3
     assert L.kvq_status_string(0) == b"KVQ_OK"
     assert L.kvq_status_string(5) == b"KVQ_ERR_TIMEOUT"
     assert L.kvq_status_string(99) == b"KVQ_ERR_UNKNOWN"
@@ -88,7 +88,8 @@ def attn_call(L, desc, ws=None, ws_bytes=0, out=FAKE):
 def test_decode_argument_errors(L):
     from bit_kv_cache_20_b200._lib import AttnDesc
     ok = dict(batch=2, num_q_heads=8, num_kv_heads=2, head_dim=128, page_size=16, num_pages=10,
-              max_pages_per_seq=5, hadamard_block=128, softmax_scale=0.0, out_dtype=0, flags=0)
+              max_pages_per_seq=5, hadamard_block=128, softmax_scale=0.0, out_dtype=0, flags=0,
+              context_lens_host=None)
 
     def d(**kw):
         a = dict(ok)

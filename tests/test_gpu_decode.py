@@ -38,7 +38,7 @@ def host_cache(cache, scales, zeros):
 
 
 def gpu_decode(w, pool, b=None, out_dtype=torch.float32, softmax_scale=0.0, ws=None,
-               page_table=None, ctx=None):
+               page_table=None, ctx=None, host_lens=None):
     b = w.block if b is None else b
     cache, scales, zeros = pool
     pt = torch.as_tensor(w.page_table if page_table is None else page_table).cuda()
@@ -47,10 +47,11 @@ def gpu_decode(w, pool, b=None, out_dtype=torch.float32, softmax_scale=0.0, ws=N
     big = torch.full((n + 2 * GUARD,), 7.0, dtype=out_dtype, device="cuda")
     out = big[GUARD:GUARD + n].view(w.B, w.Hq, w.D)
     if ws is None:
-        nbytes = kvq.attn_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.num_pages, pt.shape[1], b)
+        nbytes = kvq.attn_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.num_pages, pt.shape[1], b,
+                                         host_lengths=host_lens is not None)
         ws = kvq.alloc_workspace(nbytes)
     kvq.paged_decode_attn_int4(w.q.cuda(), cache, scales, zeros, pt, cl, out, b, ws,
-                               softmax_scale=softmax_scale)
+                               softmax_scale=softmax_scale, context_lens_host=host_lens)
     torch.cuda.synchronize()
     g = big.cpu()
     assert torch.all(g[:GUARD] == 7.0) and torch.all(g[GUARD + n:] == 7.0), "out guard overwritten"
@@ -176,9 +177,10 @@ def test_decode_deterministic_and_workspace_left_zeroed():
         assert int(torch.count_nonzero(ws)) == 0
 
 
+@pytest.mark.parametrize("host", [False, True])
 @pytest.mark.parametrize("ctx,Hq,Hkv", [([40000 - 7], 8, 2), ([36001, 2000], 8, 2), ([1, 17, 900], 8, 2),
                                         ([60000] + [16] * 39, 8, 8)])
-def test_decode_counts_every_page_once(ctx, Hq, Hkv):
+def test_decode_counts_every_page_once(ctx, Hq, Hkv, host):
     """q = 0 makes the softmax uniform, and on a plain INT4 cache a constant V
     row c is stored exactly (s = 0, z = c). With c = a different integer per
     page, the output is the mean page value over the context: a page skipped
@@ -196,7 +198,7 @@ def test_decode_counts_every_page_once(ctx, Hq, Hkv):
     v_new = c[:, None, None].expand(-1, w.Hkv, w.D).contiguous()
     w = dataclasses.replace(w, v_new=v_new, q=torch.zeros_like(w.q))
     pool = build_cache(w)
-    got, _ = gpu_decode(w, pool)
+    got, _ = gpu_decode(w, pool, host_lens=np.asarray(ctx, np.int32) if host else None)
     for n in range(B):
         ref = vals[n].mean()
         err = float(np.abs(got[n] - ref).max())
@@ -227,3 +229,45 @@ def test_decode_rejects_missing_workspace():
         kvq.paged_decode_attn_int4(w.q.cuda(), *pool, torch.as_tensor(w.page_table).cuda(),
                                    torch.as_tensor(w.context_lens).cuda(), out, 128,
                                    kvq.alloc_workspace(need - 16))
+
+
+@pytest.mark.parametrize("case", ["mixed-g4", "mixed-g8", "many-short"])
+def test_decode_per_sequence_plan_matches_oracle(orc, case):
+    """With the host copy of the context lengths the launch is planned per
+    sequence: long sequences get several splits, short ones one CTA, the
+    longest start first, and a batch with more (sequence, head) pairs than
+    resident CTAs runs in several waves."""
+    if case == "mixed-g4":
+        ctx = [1, 17, 900, 4000, 12000, 0, 250, 33, 20000, 5]
+        w = workloads.random_case(seed=51, B=len(ctx), Hq=32, Hkv=8, D=128, block=64, context_lens=ctx)
+    elif case == "mixed-g8":
+        ctx = [30000, 100, 7000, 16, 2500]
+        w = workloads.random_case(seed=52, B=len(ctx), Hq=64, Hkv=8, D=128, block=128, context_lens=ctx)
+    else:
+        rng = np.random.default_rng(53)
+        ctx = [int(x) for x in rng.integers(1, 3000, size=300)]
+        ctx[7] = 9000
+        w = workloads.random_case(seed=53, B=len(ctx), Hq=8, Hkv=2, D=64, block=32, context_lens=ctx)
+    pool = build_cache(w)
+    got, _ = gpu_decode(w, pool, host_lens=np.asarray(ctx, np.int32))
+    if w.B <= 16:
+        assert_close(got, oracle_out(orc, w, pool), case)
+    else:
+        rng = np.random.default_rng(54)
+        pairs = [(7, 0)] + [(int(n), int(h)) for n, h in zip(rng.integers(0, w.B, 20), rng.integers(0, w.Hq, 20))]
+        for (n, h), r in oracle_out(orc, w, pool, pairs=pairs).items():
+            assert_close(got[n, h], r, f"{case} n={n} hq={h}")
+
+
+@pytest.mark.parametrize("factor", [0.5, 2.0])
+def test_decode_out_of_date_host_lengths_stay_correct(orc, factor):
+    """A host copy that no longer matches the device lengths (the plan of a
+    captured graph replayed a step later) changes only the balance: shorter
+    host lengths make the kernel re-split the affected sequences itself."""
+    ctx = [9000, 300, 17, 4100]
+    w = workloads.random_case(seed=55, B=len(ctx), Hq=32, Hkv=8, D=128, block=128, context_lens=ctx)
+    pool = build_cache(w)
+    host = np.maximum((np.asarray(ctx) * factor).astype(np.int32), 1)
+    got, _ = gpu_decode(w, pool, host_lens=host)
+    assert_close(got, oracle_out(orc, w, pool), f"host lengths x{factor}")
+    assert kvq.get_device_error() == 0

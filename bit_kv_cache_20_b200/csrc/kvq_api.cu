@@ -289,7 +289,8 @@ int decode_ctas_per_sm(int dev, int D, int b, int hg, int nc) {
   const void* k = decode_kernel_for(D, b, hg, nc);
   const int smem = decode_smem_bytes(D, hg, nc);
   if (!k || cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
-      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, k, kvq::kAttnThreads, smem) != cudaSuccess || v < 1) {
+      cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, k, 32 * kvq::attn_warps(nc), smem) != cudaSuccess ||
+      v < 1) {
     cudaGetLastError();
     return 0;
   }
@@ -506,7 +507,7 @@ size_t workspace_bytes_for(const kvq_attn_desc* d, const SplitPlan& plan) {
 template <int D, int BLK, int NC>
 cudaError_t launch_decode_instance(const kvq::AttnParams& p, int hg, int smem, cudaStream_t s) {
   const dim3 grid = p.n_items > 0 ? dim3(p.Hkv / hg, p.n_items, 1) : dim3(p.n_splits, p.Hkv / hg, p.B);
-  const dim3 block(kvq::kAttnThreads);
+  const dim3 block(32 * kvq::attn_warps(NC));
   cudaError_t e = cudaErrorInvalidValue;
   if constexpr (NC == 1) {
     if (hg == 4) e = launch_pdl(kvq::kvq_decode_kernel<D, BLK, 4, NC>, grid, block, smem, s, p);

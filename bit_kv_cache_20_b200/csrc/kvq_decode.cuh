@@ -86,8 +86,11 @@ struct AttnParams {
   uint2 items[kMaxPlanItems];
 };
 
-constexpr int kAttnWarps = 8;
-constexpr int kAttnThreads = kAttnWarps * 32;
+// Warps per CTA: 8 for up to 4 query heads per kv head (two CTAs per SM);
+// 12 for 8 query heads, whose doubled accumulators leave room for one CTA per
+// SM only, so that SM still runs 12 page streams to hide each warp's
+// per-page dependency chain.
+__host__ __device__ constexpr int attn_warps(int nc) { return nc == 2 ? 12 : 8; }
 constexpr int kWarpRing = 4;        // page slots per warp
 constexpr int kMaxSplits = 128;
 constexpr int kMaxPids = 1024;      // page ids of a CTA's range kept in shared memory
@@ -96,13 +99,14 @@ constexpr int kMaxPids = 1024;      // page ids of a CTA's range kept in shared 
 // (4 query heads each).
 template <int D, int HG, int NC>
 struct AttnSmem {
+  static constexpr int kWarps = attn_warps(NC);
   static constexpr int kSlotBytes = 16 * D + 128;               // codes + 32 scales + 32 zeros
-  static constexpr int kRingBytes = kAttnWarps * kWarpRing * kSlotBytes;
+  static constexpr int kRingBytes = kWarps * kWarpRing * kSlotBytes;
   static constexpr int kRows = HG * 4 * NC;                     // query rows (G padded to 4 NC)
   // per-warp result: O[4 NC rows][D], then (m, l, zs, unused) per row
   static constexpr int kResFloats = 4 * NC * (D + 4);
   static constexpr int kOffRes = kRingBytes;
-  static constexpr int kOffQ = kOffRes + kAttnWarps * kResFloats * 4;  // float [kRows][D]
+  static constexpr int kOffQ = kOffRes + kWarps * kResFloats * 4;  // float [kRows][D]
   static constexpr int kOffQInfo = kOffQ + kRows * D * 4;       // float [kRows][4]: scale, sum
   static constexpr int kOffQ8 = kOffQInfo + kRows * 16;         // int8 [kRows][3 limbs][D], B order
   static constexpr int kOffPid = kOffQ8 + kRows * 3 * D;
@@ -171,8 +175,11 @@ __device__ __forceinline__ void warp_fwht(float (&v)[D / 32], int lane) {
 
 
 template <int D, int BLK, int HG, int NC>
-__global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kernel(const __grid_constant__ AttnParams p) {
+__global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
+    kvq_decode_kernel(const __grid_constant__ AttnParams p) {
   using S = AttnSmem<D, HG, NC>;
+  constexpr int kAttnWarps = S::kWarps;
+  constexpr int kAttnThreads = 32 * kAttnWarps;
   constexpr int NSUB = kAttnWarps / HG;  // warps per head
   constexpr int R = kWarpRing;
   constexpr int SLOT = S::kSlotBytes;
@@ -371,26 +378,23 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
   // head hw; tile 1: column g is limb 2 of that row for even g, zero for odd.
   // MMA (m, half) of thread tig: b0 = bytes of k-group tig, b1 of k-group
   // 4 + tig; their codes are the low (half 0) or high (half 1) nibbles of K
-  // words KW*tig + 2m (b0) and KW*tig + 2m + 1 (b1).
-  uint32_t bq[NC][KM][2][2], bq2[NC][KM][2][2];
+  // words KW*tig + 2m (b0) and KW*tig + 2m + 1 (b1). With one column tile
+  // they stay in registers; with two they are read from shared memory for
+  // every page (registers for a third CTA-wide warp group instead).
+  const uint8_t* qfb[NC];
 #pragma unroll
-  for (int c = 0; c < NC; ++c) {
-    const int row = hw * NR + 4 * c + (g >> 1);
-    const uint8_t* base = reinterpret_cast<const uint8_t*>(q8 + row * 3 * D) + tig * (8 * KW);
+  for (int c = 0; c < NC; ++c)
+    qfb[c] = reinterpret_cast<const uint8_t*>(q8 + (hw * NR + 4 * c + (g >> 1)) * 3 * D) + tig * (8 * KW);
+  auto qfrag = [&](int c, int m, uint4& f4, uint4& h4) {
+    f4 = *reinterpret_cast<const uint4*>(qfb[c] + (g & 1) * D + 16 * m);
+    h4 = (g & 1) ? make_uint4(0u, 0u, 0u, 0u) : *reinterpret_cast<const uint4*>(qfb[c] + 2 * D + 16 * m);
+  };
+  constexpr int NCR = NC == 1 ? 1 : 0;  // column tiles whose fragments stay in registers
+  uint4 bqf[NCR > 0 ? NCR : 1][KM], bqh[NCR > 0 ? NCR : 1][KM];
 #pragma unroll
-    for (int m = 0; m < KM; ++m) {
-      const uint4 f4 = *reinterpret_cast<const uint4*>(base + (g & 1) * D + 16 * m);
-      const uint4 h4 = (g & 1) ? make_uint4(0u, 0u, 0u, 0u) : *reinterpret_cast<const uint4*>(base + 2 * D + 16 * m);
-      bq[c][m][0][0] = f4.x;
-      bq[c][m][0][1] = f4.y;
-      bq[c][m][1][0] = f4.z;
-      bq[c][m][1][1] = f4.w;
-      bq2[c][m][0][0] = h4.x;
-      bq2[c][m][0][1] = h4.y;
-      bq2[c][m][1][0] = h4.z;
-      bq2[c][m][1][1] = h4.w;
-    }
-  }
+  for (int c = 0; c < NCR; ++c)
+#pragma unroll
+    for (int m = 0; m < KM; ++m) qfrag(c, m, bqf[c][m], bqh[c][m]);
   // this thread's QK results belong to query row 4c + tig of head hw
   float qsc[NC], qsm[NC];
   bool hv[NC];
@@ -443,16 +447,23 @@ __global__ void __launch_bounds__(kAttnThreads, NC == 1 ? 2 : 1) kvq_decode_kern
         const uint32_t ah[4] = {x0 & 0xF0F0F0F0u, y0 & 0xF0F0F0F0u, x1 & 0xF0F0F0F0u, y1 & 0xF0F0F0F0u};
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
-          if (m == 0) {
-            mma_u8s8_16832_z(accl[c], al, bq[c][0][0][0], bq[c][0][0][1]);
-            mma_u8s8_16832_z(acch[c], ah, bq[c][0][1][0], bq[c][0][1][1]);
-            mma_u8s8_16832_z(accl2[c], al, bq2[c][0][0][0], bq2[c][0][0][1]);
-            mma_u8s8_16832_z(acch2[c], ah, bq2[c][0][1][0], bq2[c][0][1][1]);
+          uint4 f4, h4;
+          if constexpr (NCR > 0) {
+            f4 = bqf[c][m];
+            h4 = bqh[c][m];
           } else {
-            mma_u8s8_16832(accl[c], al, bq[c][m][0][0], bq[c][m][0][1]);
-            mma_u8s8_16832(acch[c], ah, bq[c][m][1][0], bq[c][m][1][1]);
-            mma_u8s8_16832(accl2[c], al, bq2[c][m][0][0], bq2[c][m][0][1]);
-            mma_u8s8_16832(acch2[c], ah, bq2[c][m][1][0], bq2[c][m][1][1]);
+            qfrag(c, m, f4, h4);
+          }
+          if (m == 0) {
+            mma_u8s8_16832_z(accl[c], al, f4.x, f4.y);
+            mma_u8s8_16832_z(acch[c], ah, f4.z, f4.w);
+            mma_u8s8_16832_z(accl2[c], al, h4.x, h4.y);
+            mma_u8s8_16832_z(acch2[c], ah, h4.z, h4.w);
+          } else {
+            mma_u8s8_16832(accl[c], al, f4.x, f4.y);
+            mma_u8s8_16832(acch[c], ah, f4.z, f4.w);
+            mma_u8s8_16832(accl2[c], al, h4.x, h4.y);
+            mma_u8s8_16832(acch2[c], ah, h4.z, h4.w);
           }
         }
       }

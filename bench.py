@@ -256,6 +256,26 @@ class Step:
             self.attn_args.append((P(self.q.data_ptr()), P(c.data_ptr()), P(s.data_ptr()), P(z.data_ptr()),
                                    P(self.pt.data_ptr()), P(self.ctx.data_ptr()), P(self.out.data_ptr()),
                                    P(self.ws.data_ptr()), self.ws_bytes, ctypes.byref(self.adesc), self.sh))
+        # decode-append: each sequence's last context token is the step's
+        # new token (rewritten in place every step, so every step does the
+        # same work); separate = a 1-token-per-sequence write + the decode,
+        # fused = one paged_decode_append_attn_int4 launch
+        ends = np.cumsum(np.asarray(w.context_lens, np.int64))
+        last = torch.as_tensor(ends - 1)
+        self.k1 = w.k_new[last].contiguous().to(dev)
+        self.v1 = w.v_new[last].contiguous().to(dev)
+        self.s1 = torch.as_tensor(np.asarray(w.slots_new)[ends - 1]).to(dev)
+        self.wdesc1 = _lib.WriteDesc(w.B, w.Hkv, w.D, 16, w.num_pages)
+        self.write1_args, self.app_args = [], []
+        for i in range(self.N_POOLS):
+            c, s, z = self.pools[(i - 2) % self.N_POOLS]
+            self.write1_args.append((P(self.k1.data_ptr()), P(self.v1.data_ptr()), P(self.s1.data_ptr()), None,
+                                     P(c.data_ptr()), P(s.data_ptr()), P(z.data_ptr()), block,
+                                     ctypes.byref(self.wdesc1), self.sh))
+            self.app_args.append((P(self.q.data_ptr()), P(self.k1.data_ptr()), P(self.v1.data_ptr()),
+                                  P(self.s1.data_ptr()), P(c.data_ptr()), P(s.data_ptr()), P(z.data_ptr()),
+                                  P(self.pt.data_ptr()), P(self.ctx.data_ptr()), P(self.out.data_ptr()),
+                                  P(self.ws.data_ptr()), self.ws_bytes, ctypes.byref(self.adesc), self.sh))
         torch.cuda.synchronize(dev)  # allocations above ran on the default stream
 
     def write(self, i):
@@ -268,6 +288,17 @@ class Step:
         if st:
             raise RuntimeError(f"paged_decode_attn_int4 status {st}")
 
+    def append_separate(self, i):
+        st = self.L.kv_quant_write(*self.write1_args[i % self.N_POOLS])
+        if st:
+            raise RuntimeError(f"kv_quant_write status {st}")
+        self.decode(i)
+
+    def append_fused(self, i):
+        st = self.L.paged_decode_append_attn_int4(*self.app_args[i % self.N_POOLS])
+        if st:
+            raise RuntimeError(f"paged_decode_append_attn_int4 status {st}")
+
     def fill_pools(self):
         for i in range(self.N_POOLS):
             self.write(i)
@@ -279,7 +310,7 @@ class Step:
         the pools as in the direct calls. It is replayed once, untimed, so the
         first timed replay does not include the graph's upload."""
         torch = self.torch
-        fns = [self.write if k == "write" else self.decode for k in kinds]
+        fns = [getattr(self, k) for k in kinds]
         g = torch.cuda.CUDAGraph()
         with torch.cuda.graph(g, stream=self.stream, capture_error_mode="thread_local"):
             for j in range(steps):
@@ -305,7 +336,7 @@ class Step:
     def direct_ms(self, kinds, steps, start_index=0):
         """The same launches issued directly on the stream between two events."""
         torch = self.torch
-        fns = [self.write if k == "write" else self.decode for k in kinds]
+        fns = [getattr(self, k) for k in kinds]
         t0 = torch.cuda.Event(enable_timing=True)
         t1 = torch.cuda.Event(enable_timing=True)
         t0.record(self.stream)
@@ -543,7 +574,7 @@ def main(argv=None):
         barrier()
         # each kernel alone, back to back, for its own line: the median of
         # `rounds` measurements, rotated and plain alternating
-        ms = {k: [] for k in ("write", "decode", "p_write", "p_decode")}
+        ms = {k: [] for k in ("write", "decode", "p_write", "p_decode", "append_separate", "append_fused")}
         for _ in range(rounds):
             for kind in ("write", "decode"):
                 ms[kind].append(step.timed_only(kind, args.steps, start_index=warm))
@@ -551,12 +582,18 @@ def main(argv=None):
                 if p is not None:
                     ms["p_" + kind].append(p.timed_only(kind, args.steps, start_index=warm))
                     barrier()
+            # decode with a 1-token append per sequence: two launches or one
+            for kind in ("append_separate", "append_fused"):
+                ms[kind].append(step.timed_only(kind, args.steps, start_index=warm))
+                barrier()
         t_host1 = time.monotonic()
         clocks.mark(t_host0, t_host1)
     barrier()
     total_ms = max_over_ranks(total_ms)
     wr_ms = max_over_ranks(statistics.median(ms["write"]))
     de_ms = max_over_ranks(statistics.median(ms["decode"]))
+    ap_sep_ms = max_over_ranks(statistics.median(ms["append_separate"]))
+    ap_fus_ms = max_over_ranks(statistics.median(ms["append_fused"]))
 
     plain = None
     if p is not None:
@@ -618,6 +655,11 @@ def main(argv=None):
                                        "cached_tokens_per_s": round(w.tokens_cached / (de_ms / 1e3), 1)},
         },
         "plain_int4": plain,
+        "decode_append": {
+            "what": "each sequence's new token stored, then a decode step over contexts that include it",
+            "separate_us": round(1e3 * ap_sep_ms, 3),  # kv_quant_write (B tokens) + paged_decode_attn_int4
+            "fused_us": round(1e3 * ap_fus_ms, 3),     # paged_decode_append_attn_int4
+        },
         "e2e": e2e,
         "clocks": clocks.summary(),
         "gpu_launches": 2 * args.steps,

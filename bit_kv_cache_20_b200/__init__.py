@@ -187,6 +187,48 @@ def paged_decode_attn_int4(q: torch.Tensor, cache: torch.Tensor, scales: torch.T
     _lib.check(st, "paged_decode_attn_int4")
 
 
+def paged_decode_append_attn_int4(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,
+                                  slot_mapping: torch.Tensor, cache: torch.Tensor,
+                                  scales: torch.Tensor, zeros: torch.Tensor,
+                                  page_table: torch.Tensor, context_lens: torch.Tensor,
+                                  out: torch.Tensor, hadamard_block: int,
+                                  workspace: Optional[torch.Tensor] = None,
+                                  softmax_scale: float = 0.0, stream=None,
+                                  inputs_ready: bool = False, context_lens_host=None) -> None:
+    """One decode step that first appends each sequence's new token: k_new,
+    v_new bf16 [B, Hkv, D] are rotated, quantized and stored at slot_mapping
+    (int64 [B], -1 = no new token), position context_lens - 1 of their
+    sequence, and the attention runs over contexts that include them - one
+    launch instead of kv_quant_write + paged_decode_attn_int4."""
+    _need(q, "q", torch.bfloat16)
+    _need(k_new, "k_new", torch.bfloat16)
+    _need(v_new, "v_new", torch.bfloat16)
+    _need(slot_mapping, "slot_mapping", torch.int64)
+    _need(page_table, "page_table", torch.int32)
+    _need(context_lens, "context_lens", torch.int32)
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("out must be float32 or bfloat16")
+    _need(out, "out", out.dtype)
+    if tuple(out.shape) != tuple(q.shape):
+        raise ValueError("out must have q's shape")
+    lens_arr, lens_ptr = _host_lengths(context_lens_host, int(q.shape[0]) if q.dim() == 3 else -1)
+    desc = _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scale,
+                      0 if out.dtype == torch.float32 else 1, inputs_ready, lens_ptr)
+    if context_lens.numel() != desc.batch or slot_mapping.numel() != desc.batch:
+        raise ValueError("context_lens and slot_mapping must hold one entry per sequence")
+    if tuple(k_new.shape) != (desc.batch, desc.num_kv_heads, desc.head_dim) or k_new.shape != v_new.shape:
+        raise ValueError("k_new and v_new must be bf16 [B, Hkv, D]")
+    ws_ptr, ws_bytes = None, 0
+    if workspace is not None:
+        _need(workspace, "workspace", torch.uint8)
+        ws_ptr, ws_bytes = _ptr(workspace), workspace.numel()
+    st = _lib.lib().paged_decode_append_attn_int4(
+        _ptr(q), _ptr(k_new), _ptr(v_new), _ptr(slot_mapping), _ptr(cache), _ptr(scales), _ptr(zeros),
+        _ptr(page_table), _ptr(context_lens), _ptr(out), ws_ptr, ws_bytes, ctypes.byref(desc),
+        ctypes.c_void_p(_stream_handle(stream)))
+    _lib.check(st, "paged_decode_append_attn_int4")
+
+
 def paged_decode_attn_int4_static_ws(q: torch.Tensor, cache: torch.Tensor, scales: torch.Tensor,
                                      zeros: torch.Tensor, page_table: torch.Tensor,
                                      context_lens: torch.Tensor, out: torch.Tensor,

@@ -227,40 +227,41 @@ struct SplitPlan {
 
 int cols_for(int G) { return G > 4 ? 2 : 1; }
 
-int inst_slot(int D, int b, int hg, int nc) {
+int inst_slot(int D, int b, int hg, int nc, int app) {
   const int bi = (b == 0) ? 0 : (b == 32) ? 1 : (b == 64) ? 2 : 3;
   const int hi = (hg == 4) ? 2 : (hg == 2) ? 1 : 0;
-  return (((D == 64) ? 0 : 1) * 4 + bi) * 6 + hi * 2 + (nc - 1);
+  return ((((D == 64) ? 0 : 1) * 4 + bi) * 6 + hi * 2 + (nc - 1)) * 2 + (app ? 1 : 0);
 }
-constexpr int kInstSlots = 48;
+constexpr int kInstSlots = 96;
 
 // Instances exist for HG * NC <= 4 (the plan never asks for more).
-template <int D, int BLK, int NC>
+template <int D, int BLK, int NC, bool APP>
 const void* decode_kernel_ptr(int hg) {
   if constexpr (NC == 1) {
-    if (hg == 4) return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK, 4, NC>);
+    if (hg == 4) return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK, 4, NC, APP>);
   }
-  if (hg == 2) return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK, 2, NC>);
-  if (hg == 1) return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK, 1, NC>);
+  if (hg == 2) return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK, 2, NC, APP>);
+  if (hg == 1) return reinterpret_cast<const void*>(kvq::kvq_decode_kernel<D, BLK, 1, NC, APP>);
   return nullptr;
 }
 
 template <int D, int BLK>
-const void* decode_kernel_ptr(int hg, int nc) {
-  return nc == 2 ? decode_kernel_ptr<D, BLK, 2>(hg) : decode_kernel_ptr<D, BLK, 1>(hg);
+const void* decode_kernel_ptr(int hg, int nc, int app) {
+  if (app) return nc == 2 ? decode_kernel_ptr<D, BLK, 2, true>(hg) : decode_kernel_ptr<D, BLK, 1, true>(hg);
+  return nc == 2 ? decode_kernel_ptr<D, BLK, 2, false>(hg) : decode_kernel_ptr<D, BLK, 1, false>(hg);
 }
 
-const void* decode_kernel_for(int D, int b, int hg, int nc) {
+const void* decode_kernel_for(int D, int b, int hg, int nc, int app) {
   if (D == 64) {
-    if (b == 0) return decode_kernel_ptr<64, 0>(hg, nc);
-    if (b == 32) return decode_kernel_ptr<64, 32>(hg, nc);
-    if (b == 64) return decode_kernel_ptr<64, 64>(hg, nc);
+    if (b == 0) return decode_kernel_ptr<64, 0>(hg, nc, app);
+    if (b == 32) return decode_kernel_ptr<64, 32>(hg, nc, app);
+    if (b == 64) return decode_kernel_ptr<64, 64>(hg, nc, app);
     return nullptr;
   }
-  if (b == 0) return decode_kernel_ptr<128, 0>(hg, nc);
-  if (b == 32) return decode_kernel_ptr<128, 32>(hg, nc);
-  if (b == 64) return decode_kernel_ptr<128, 64>(hg, nc);
-  if (b == 128) return decode_kernel_ptr<128, 128>(hg, nc);
+  if (b == 0) return decode_kernel_ptr<128, 0>(hg, nc, app);
+  if (b == 32) return decode_kernel_ptr<128, 32>(hg, nc, app);
+  if (b == 64) return decode_kernel_ptr<128, 64>(hg, nc, app);
+  if (b == 128) return decode_kernel_ptr<128, 128>(hg, nc, app);
   return nullptr;
 }
 
@@ -280,13 +281,13 @@ int decode_smem_bytes(int D, int hg, int nc) {
 
 // Opt the decode kernel instance into its dynamic shared memory and return
 // how many of its CTAs one SM holds (once per device and instance; 0 on error).
-int decode_ctas_per_sm(int dev, int D, int b, int hg, int nc) {
+int decode_ctas_per_sm(int dev, int D, int b, int hg, int nc, int app) {
   static std::atomic<int> cache[kMaxDevices][kInstSlots];
   if (dev < 0 || dev >= kMaxDevices) return 0;
-  const int slot = inst_slot(D, b, hg, nc);
+  const int slot = inst_slot(D, b, hg, nc, app);
   int v = cache[dev][slot].load(std::memory_order_relaxed);
   if (v > 0) return v;
-  const void* k = decode_kernel_for(D, b, hg, nc);
+  const void* k = decode_kernel_for(D, b, hg, nc, app);
   const int smem = decode_smem_bytes(D, hg, nc);
   if (!k || cudaFuncSetAttribute(k, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
       cudaOccupancyMaxActiveBlocksPerMultiprocessor(&v, k, 32 * kvq::attn_warps(nc), smem) != cudaSuccess ||
@@ -304,14 +305,14 @@ int decode_ctas_per_sm(int dev, int D, int b, int hg, int nc) {
 // API reports for that instance) with at least 4 pages per split; the plan
 // with the least work per CTA times waves (plus a fixed cost of 8 head-pages
 // per CTA) wins, ties going to the smaller HG (fewer partial results).
-SplitPlan plan_splits(const kvq_attn_desc* d, int dev) {
+SplitPlan plan_splits(const kvq_attn_desc* d, int dev, int app) {
   const int nc = cols_for(d->num_q_heads / d->num_kv_heads);
   const int sms = sm_count(dev);
   SplitPlan best = {1, d->max_pages_per_seq, 1, nc, 0, 0};
   long long best_cost = LLONG_MAX;
   for (int hg = 1; hg <= 4; hg <<= 1) {
     if (d->num_kv_heads % hg != 0 || hg * nc > 4) continue;
-    const int per_sm = decode_ctas_per_sm(dev, d->head_dim, d->hadamard_block, hg, nc);
+    const int per_sm = decode_ctas_per_sm(dev, d->head_dim, d->hadamard_block, hg, nc, app);
     if (per_sm < 1 || sms < 1) continue;
     const long long slots = (long long)per_sm * sms;
     const long long units = (long long)d->batch * (d->num_kv_heads / hg);
@@ -343,7 +344,7 @@ SplitPlan plan_splits(const kvq_attn_desc* d, int dev) {
 // of a plan: max(total work / resident CTAs, the largest CTA) in head-pages
 // plus a fixed 8 per CTA; the cheapest kv-head group size wins. Returns false
 // when the plan does not fit the parameter block (then the uniform plan runs).
-bool plan_lengths(const kvq_attn_desc* d, int dev, SplitPlan* out, uint2* items) {
+bool plan_lengths(const kvq_attn_desc* d, int dev, int app, SplitPlan* out, uint2* items) {
   const int B = d->batch;
   const int32_t* lens = d->context_lens_host;
   if (!lens || B < 1 || B > kvq::kMaxPlanItems) return false;
@@ -367,7 +368,7 @@ bool plan_lengths(const kvq_attn_desc* d, int dev, SplitPlan* out, uint2* items)
   long long best_T = 0;
   for (int hg = 1; hg <= 4; hg <<= 1) {
     if (d->num_kv_heads % hg != 0 || hg * nc > 4) continue;
-    const int per_sm = decode_ctas_per_sm(dev, d->head_dim, d->hadamard_block, hg, nc);
+    const int per_sm = decode_ctas_per_sm(dev, d->head_dim, d->hadamard_block, hg, nc, app);
     if (per_sm < 1) continue;
     const long long slots = (long long)per_sm * sms;
     const long long groups = d->num_kv_heads / hg;
@@ -461,13 +462,13 @@ size_t planned_workspace_bytes(const kvq_attn_desc* d, const SplitPlan& plan) {
 
 // Bound on planned_workspace_bytes over every context-length vector: the
 // CTAs of split sequences fit in one wave, so at most resident/groups slots.
-size_t planned_workspace_bound(const kvq_attn_desc* d, int dev) {
+size_t planned_workspace_bound(const kvq_attn_desc* d, int dev, int app) {
   const int nc = cols_for(d->num_q_heads / d->num_kv_heads);
   const int sms = sm_count(dev);
   size_t best = 0;
   for (int hg = 1; hg <= 4; hg <<= 1) {
     if (d->num_kv_heads % hg != 0 || hg * nc > 4) continue;
-    const int per_sm = decode_ctas_per_sm(dev, d->head_dim, d->hadamard_block, hg, nc);
+    const int per_sm = decode_ctas_per_sm(dev, d->head_dim, d->hadamard_block, hg, nc, app);
     if (per_sm < 1 || sms < 1) continue;
     const size_t slots = (size_t)per_sm * sms * hg / d->num_kv_heads;
     best = std::max(best, slots * d->num_q_heads * (d->head_dim + 4) * sizeof(uint32_t));
@@ -504,26 +505,32 @@ size_t workspace_bytes_for(const kvq_attn_desc* d, const SplitPlan& plan) {
   return (size_t)d->batch * d->num_kv_heads * plan.n_splits * G * (d->head_dim + 4) * sizeof(uint32_t);
 }
 
-template <int D, int BLK, int NC>
+template <int D, int BLK, int NC, bool APP>
 cudaError_t launch_decode_instance(const kvq::AttnParams& p, int hg, int smem, cudaStream_t s) {
   const dim3 grid = p.n_items > 0 ? dim3(p.Hkv / hg, p.n_items, 1) : dim3(p.n_splits, p.Hkv / hg, p.B);
   const dim3 block(32 * kvq::attn_warps(NC));
   cudaError_t e = cudaErrorInvalidValue;
   if constexpr (NC == 1) {
-    if (hg == 4) e = launch_pdl(kvq::kvq_decode_kernel<D, BLK, 4, NC>, grid, block, smem, s, p);
+    if (hg == 4) e = launch_pdl(kvq::kvq_decode_kernel<D, BLK, 4, NC, APP>, grid, block, smem, s, p);
   }
-  if (hg == 2) e = launch_pdl(kvq::kvq_decode_kernel<D, BLK, 2, NC>, grid, block, smem, s, p);
-  else if (hg == 1) e = launch_pdl(kvq::kvq_decode_kernel<D, BLK, 1, NC>, grid, block, smem, s, p);
+  if (hg == 2) e = launch_pdl(kvq::kvq_decode_kernel<D, BLK, 2, NC, APP>, grid, block, smem, s, p);
+  else if (hg == 1) e = launch_pdl(kvq::kvq_decode_kernel<D, BLK, 1, NC, APP>, grid, block, smem, s, p);
   if (e != cudaSuccess) cudaGetLastError();
   return e;
 }
 
 template <int D, int BLK>
 kvq_status launch_attn(const kvq::AttnParams& p, const SplitPlan& plan, int dev, cudaStream_t s) {
-  if (decode_ctas_per_sm(dev, D, BLK, plan.hg, plan.nc) < 1) return KVQ_ERR_CUDA;
+  const int app = p.slots_new != nullptr;
+  if (decode_ctas_per_sm(dev, D, BLK, plan.hg, plan.nc, app) < 1) return KVQ_ERR_CUDA;
   const int smem = decode_smem_bytes(D, plan.hg, plan.nc);
-  const cudaError_t e = plan.nc == 2 ? launch_decode_instance<D, BLK, 2>(p, plan.hg, smem, s)
-                                     : launch_decode_instance<D, BLK, 1>(p, plan.hg, smem, s);
+  cudaError_t e;
+  if (app)
+    e = plan.nc == 2 ? launch_decode_instance<D, BLK, 2, true>(p, plan.hg, smem, s)
+                     : launch_decode_instance<D, BLK, 1, true>(p, plan.hg, smem, s);
+  else
+    e = plan.nc == 2 ? launch_decode_instance<D, BLK, 2, false>(p, plan.hg, smem, s)
+                     : launch_decode_instance<D, BLK, 1, false>(p, plan.hg, smem, s);
   return e == cudaSuccess ? KVQ_OK : KVQ_ERR_CUDA;
 }
 
@@ -588,14 +595,28 @@ size_t kvq_attn_workspace_size(const kvq_attn_desc* desc) {
     return SIZE_MAX;
   }
   if (dev < 0 || dev >= kMaxDevices) return SIZE_MAX;
-  const size_t uniform = workspace_bytes_for(desc, plan_splits(desc, dev));
-  return desc->context_lens_host ? std::max(uniform, planned_workspace_bound(desc, dev)) : uniform;
+  // the same workspace serves paged_decode_attn_int4 and the decode-append
+  // entry point (their kernels may hold different numbers of CTAs per SM)
+  size_t need = 0;
+  for (int app = 0; app < 2; ++app) {
+    need = std::max(need, workspace_bytes_for(desc, plan_splits(desc, dev, app)));
+    if (desc->context_lens_host) need = std::max(need, planned_workspace_bound(desc, dev, app));
+  }
+  return need;
 }
 
-kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const void* scales,
-                                  const void* zeros, const int32_t* page_table,
-                                  const int32_t* context_lens, void* out, void* workspace,
-                                  size_t workspace_bytes, const kvq_attn_desc* desc, void* stream) {
+namespace {
+
+// The new tokens of a decode-append call (all null for a plain decode).
+struct AppendArgs {
+  const void* k_new;
+  const void* v_new;
+  const int64_t* slot_mapping;
+};
+
+kvq_status decode_impl(const void* q, const uint8_t* cache, const void* scales, const void* zeros,
+                       const int32_t* page_table, const int32_t* context_lens, void* out, void* workspace,
+                       size_t workspace_bytes, const kvq_attn_desc* desc, void* stream, const AppendArgs& app) {
   kvq_status st = check_attn_desc(desc);
   if (st != KVQ_OK) return st;
   const kvq_attn_desc& d = *desc;
@@ -614,12 +635,13 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const voi
   static thread_local kvq::AttnParams p;
   SplitPlan plan;
   SplitPlan lp;
-  if (d.context_lens_host && plan_lengths(&d, dev, &lp, p.items) &&
+  const int app_mode = app.slot_mapping != nullptr;
+  if (d.context_lens_host && plan_lengths(&d, dev, app_mode, &lp, p.items) &&
       (lp.part_slots == 0 || (workspace && aligned(workspace, 16) &&
                               workspace_bytes >= planned_workspace_bytes(&d, lp)))) {
     plan = lp;
   } else {
-    plan = plan_splits(&d, dev);
+    plan = plan_splits(&d, dev, app_mode);
   }
   const size_t need = workspace_bytes_for(&d, plan);
   if (need > 0 && (!workspace || workspace_bytes < need || !aligned(workspace, 16)))
@@ -643,6 +665,12 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const voi
   p.ws_part = need > 0 ? static_cast<uint32_t*>(workspace) : nullptr;
   p.out_bf16 = d.out_dtype;
   p.inputs_ready = (d.flags & KVQ_ATTN_INPUTS_READY) ? 1 : 0;
+  p.k_new = static_cast<const uint16_t*>(app.k_new);
+  p.v_new = static_cast<const uint16_t*>(app.v_new);
+  p.slots_new = app.slot_mapping;
+  p.cache_w = const_cast<uint8_t*>(cache);
+  p.scales_w = static_cast<uint16_t*>(const_cast<void*>(scales));
+  p.zeros_w = static_cast<uint16_t*>(const_cast<void*>(zeros));
   const double cb = d.hadamard_block > 0 ? 1.0 / std::sqrt((double)d.hadamard_block) : 1.0;
   const double scale = d.softmax_scale > 0.0f ? (double)d.softmax_scale : 1.0 / std::sqrt((double)d.head_dim);
   p.qmul = (float)(cb * scale * 1.4426950408889634);  // log2(e)
@@ -650,6 +678,28 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const voi
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d.head_dim == 64 ? dispatch_attn<64>(p, d.hadamard_block, plan, dev, s)
                           : dispatch_attn<128>(p, d.hadamard_block, plan, dev, s);
+}
+
+}  // namespace
+
+kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache, const void* scales,
+                                  const void* zeros, const int32_t* page_table,
+                                  const int32_t* context_lens, void* out, void* workspace,
+                                  size_t workspace_bytes, const kvq_attn_desc* desc, void* stream) {
+  return decode_impl(q, cache, scales, zeros, page_table, context_lens, out, workspace, workspace_bytes,
+                     desc, stream, AppendArgs{nullptr, nullptr, nullptr});
+}
+
+kvq_status paged_decode_append_attn_int4(const void* q, const void* k_new, const void* v_new,
+                                         const int64_t* slot_mapping, uint8_t* cache, void* scales,
+                                         void* zeros, const int32_t* page_table,
+                                         const int32_t* context_lens, void* out, void* workspace,
+                                         size_t workspace_bytes, const kvq_attn_desc* desc, void* stream) {
+  if (desc && desc->batch > 0 &&
+      (!k_new || !v_new || !slot_mapping || !aligned(k_new, 16) || !aligned(v_new, 16) || !aligned(slot_mapping, 8)))
+    return KVQ_ERR_INVALID_ARG;
+  return decode_impl(q, cache, scales, zeros, page_table, context_lens, out, workspace, workspace_bytes,
+                     desc, stream, AppendArgs{k_new, v_new, slot_mapping});
 }
 
 kvq_status kvq_get_device_error(void* stream) {
@@ -736,7 +786,7 @@ extern "C" kvq_status paged_decode_attn_int4_static_ws(const void* q, const uint
   st = select_device_of(cache, &dev);  // makes the cache's device current
   if (st != KVQ_OK) return st;
   if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
-  const size_t need = workspace_bytes_for(desc, plan_splits(desc, dev));
+  const size_t need = workspace_bytes_for(desc, plan_splits(desc, dev, 0));
   if (need > KVQ_STATIC_WORKSPACE_BYTES) return KVQ_ERR_WORKSPACE;
   void* ws = nullptr;
   st = static_workspace_on(dev, &ws);

@@ -78,6 +78,16 @@ struct AttnParams {
   float qmul;                 // c_b * softmax_scale * log2(e)
   float cb;                   // c_b (output rotation), 1 for plain INT4
   int inputs_ready;           // q, page_table, ctx_lens not written by the previous kernel
+  // Decode-append (slots_new != nullptr): sequence n's new token, k_new /
+  // v_new bf16 [B][Hkv][D], is quantized and stored at slots_new[n] (-1: none)
+  // as position ctx_lens[n] - 1 of the sequence, through cache_w, scales_w,
+  // zeros_w (the same buffers as cache, scales, zeros).
+  const uint16_t* k_new;
+  const uint16_t* v_new;
+  const int64_t* slots_new;
+  uint8_t* cache_w;
+  uint16_t* scales_w;
+  uint16_t* zeros_w;
   // Per-sequence plan (n_items > 0; grid = (Hkv / HG, n_items)): item i is
   // x = sequence | split << 16 | splits << 24, y = first partial slot of the
   // sequence | pages per split << 16. Otherwise the grid is (n_splits,
@@ -110,7 +120,11 @@ struct AttnSmem {
   static constexpr int kOffQInfo = kOffQ + kRows * D * 4;       // float [kRows][4]: scale, sum
   static constexpr int kOffQ8 = kOffQInfo + kRows * 16;         // int8 [kRows][3 limbs][D], B order
   static constexpr int kOffPid = kOffQ8 + kRows * 3 * D;
-  static constexpr int kTotal = kOffPid + kMaxPids * 4;
+  // decode-append: per (kv head of the CTA, K|V) the new token's packed row,
+  // then its fp16 scale and zero
+  static constexpr int kAppRow = D / 2 + 16;
+  static constexpr int kOffApp = kOffPid + kMaxPids * 4;
+  static constexpr int kTotal = kOffApp + HG * 2 * kAppRow;
 };
 
 template <int N>
@@ -174,7 +188,7 @@ __device__ __forceinline__ void warp_fwht(float (&v)[D / 32], int lane) {
 }
 
 
-template <int D, int BLK, int HG, int NC>
+template <int D, int BLK, int HG, int NC, bool APP>
 __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
     kvq_decode_kernel(const __grid_constant__ AttnParams p) {
   using S = AttnSmem<D, HG, NC>;
@@ -237,6 +251,8 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
   for (int i = tid; i < min(p_begin + pps, p.max_pages) - p_begin && i < kMaxPids; i += kAttnThreads)
     pids[i] = pt_row[i];
   int ctx = p.ctx_lens[n];
+  long long app_slot = -1;
+  if constexpr (APP) app_slot = p.slots_new[n];
   for (int i = tid; i < S::kRows * (D / 8); i += kAttnThreads) {
     const int row = i / (D / 8), c8 = i % (D / 8);
     const int hh = row / NR, r = row % NR;
@@ -275,6 +291,25 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
   }
   const int npg = max(min(p_begin + pps, n_pages) - p_begin, 0);
   __syncthreads();
+
+  // Decode-append: the CTA whose range holds position ctx - 1 owns the new
+  // token; its slot must be that position's (page-table entry, offset).
+  int app_t = -1, app_off = 0;  // the token's page within the range, and row
+  if (APP && app_slot >= 0) {
+    const int tn = ctx - 1, pl = tn >> 4;
+    if (tn >= 0 && pl >= p_begin && pl < p_begin + npg) {
+      const int t = pl - p_begin;
+      const int id = (t < kMaxPids) ? pids[t] : pt_row[t];
+      if (app_slot < (long long)p.num_pages * 16 && (app_slot >> 4) == id && (int)(app_slot & 15) == (tn & 15)) {
+        app_t = t;
+        app_off = tn & 15;
+      } else if (tid == 0) {
+        record_error(KVQ_ERR_OUT_OF_RANGE);
+      }
+    } else if (tn < 0 && tid == 0) {
+      record_error(KVQ_ERR_OUT_OF_RANGE);  // a new token for an empty context
+    }
+  }
 
   // ---- this warp's page stream: pages sub, sub + NSUB, ... of head hw -----
   // fetch(k) copies the warp's k-th page into ring slot k % R (one commit
@@ -362,16 +397,83 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
     }
     __syncthreads();
   };
+  // Decode-append, in the owner CTA: warp 2 hh + kv rotates, quantizes and
+  // packs the new token's K (kv = 0) or V row of head hh exactly as
+  // kv_quant_write defines it (z = RD16(min y), s = the smallest fp16 with
+  // 15 s + z >= max y, code = rint(fp32(y - z) * fp32(1/s))), stores it in the
+  // cache and keeps a copy in shared memory; the warp that computes on that
+  // page patches its copy of the page with it (the cp.async copy may predate
+  // the store), so the attention sees the row as stored.
+  auto append = [&]() {
+    if (!APP || app_t < 0 || warp >= 2 * HG) return;
+    const int hh = warp >> 1, kv = warp & 1;
+    const size_t head = (size_t)hgi * HG + hh;
+    const uint16_t* src = (kv ? p.v_new : p.k_new) + ((size_t)n * p.Hkv + head) * D + E * lane;
+    float v[E];
+#pragma unroll
+    for (int e = 0; e < E; ++e) v[e] = bf16_bits_to_float(src[e]);
+    if constexpr (BLK > 0) warp_fwht<D, BLK>(v, lane);
+    float mn = v[0], mx = v[0];
+#pragma unroll
+    for (int e = 1; e < E; ++e) {
+      mn = fminf(mn, v[e]);
+      mx = fmaxf(mx, v[e]);
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      mn = fminf(mn, __shfl_xor_sync(FULL, mn, o));
+      mx = fmaxf(mx, __shfl_xor_sync(FULL, mx, o));
+    }
+    mn = __fmul_rn(mn, p.cb);  // y = fp32(H x) * c_b is monotone in H x
+    mx = __fmul_rn(mx, p.cb);
+    const __half zh = __float2half_rd(mn);
+    const float zf = __half2float(zh);
+    const float need = __fdiv_ru(__fsub_ru(mx, zf), 15.0f);
+    unsigned short sbits = __half_as_ushort(__float2half_ru(need));
+    if (sbits != 0 && sbits < 0x7C00) {  // one fp16 step lower may still cover max y
+      const unsigned short pb = (unsigned short)(sbits - 1);
+      if (fma(15.0, (double)__half2float(__ushort_as_half(pb)), (double)zf) >= (double)mx) sbits = pb;
+    }
+    const float sf = __half2float(__ushort_as_half(sbits));
+    const float inv = (sf > 0.0f) ? __frcp_rn(sf) : 0.0f;
+    uint32_t packed = 0;  // E codes, two per byte, low nibble first
+#pragma unroll
+    for (int e = 0; e < E; ++e) {
+      const float y = __fmul_rn(v[e], p.cb);
+      const uint32_t code = __float_as_uint(__fmaf_rn(__fsub_rn(y, zf), inv, 8388608.0f)) & 0xFu;
+      packed |= code << (4 * e);
+    }
+    const long long row = (((app_slot >> 4) * p.Hkv + (long long)head) * 2 + kv) * 16 + app_off;
+    uint8_t* sdst = smem + S::kOffApp + (hh * 2 + kv) * S::kAppRow;
+    if constexpr (E == 4) {
+      *reinterpret_cast<uint16_t*>(p.cache_w + row * (D / 2) + 2 * lane) = (uint16_t)packed;
+      *reinterpret_cast<uint16_t*>(sdst + 2 * lane) = (uint16_t)packed;
+    } else {
+      p.cache_w[row * (D / 2) + lane] = (uint8_t)packed;
+      sdst[lane] = (uint8_t)packed;
+    }
+    if (lane == 0) {
+      p.scales_w[row] = sbits;
+      p.zeros_w[row] = __half_as_ushort(zh);
+      reinterpret_cast<uint16_t*>(sdst + D / 2)[0] = sbits;
+      reinterpret_cast<uint16_t*>(sdst + D / 2)[1] = __half_as_ushort(zh);
+    }
+  };
+  static_assert(E == 2 || E == 4, "row elements per lane");
+
   if (early) {
     prep_q();    // overlaps the previous kernel's last CTAs
     pdl_wait();  // the cache may be what that kernel wrote
     pdl_launch_dependents();
 #pragma unroll
     for (int k = 0; k < R - 1; ++k) fetch(k);
+    append();
+    if (APP && app_t >= 0) __syncthreads();  // the shared copy of the new rows
   } else {
 #pragma unroll
     for (int k = 0; k < R - 1; ++k) fetch(k);
-    prep_q();    // while the first pages land
+    append();
+    prep_q();    // while the first pages land (ends with a barrier)
   }
 
   // B fragments of QK. Tile 0: column g is limb g&1 of query row 4c + g/2 of
@@ -430,6 +532,23 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
     cp_async_wait<R - 1>();  // page k has landed (this lane's copies)
     __syncwarp();            // ... and every other lane's
     if ((valid >> (k % R)) & 1u) {
+      if (APP && t == app_t) {
+        // the new token's rows replace this page's copy of that position
+        uint8_t* pg = ring + (k % R) * SLOT;
+        const uint8_t* a = smem + S::kOffApp + hw * 2 * S::kAppRow;  // K row, then V row
+        constexpr int CH = D / 32;  // 16-byte chunks of a packed row
+        if (lane < 2 * CH) {
+          const int kvp = lane / CH, c = lane % CH;
+          *reinterpret_cast<uint4*>(pg + kvp * 8 * D + app_off * (D / 2) + 16 * c) =
+              *reinterpret_cast<const uint4*>(a + kvp * S::kAppRow + 16 * c);
+        } else if (lane < 2 * CH + 2) {
+          const int kvp = lane - 2 * CH;
+          const uint16_t* sz = reinterpret_cast<const uint16_t*>(a + kvp * S::kAppRow + D / 2);
+          reinterpret_cast<uint16_t*>(pg + 16 * D)[16 * kvp + app_off] = sz[0];
+          reinterpret_cast<uint16_t*>(pg + 16 * D + 64)[16 * kvp + app_off] = sz[1];
+        }
+        __syncwarp();
+      }
       const uint8_t* kb = ring + (k % R) * SLOT;  // K block [16][D/2], then V block
       const uint8_t* vb = kb + 8 * D;
       const __half* scl = reinterpret_cast<const __half*>(kb + 16 * D);       // 16 K, then 16 V scales
@@ -469,10 +588,17 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
       }
       const float sk0 = __half2float(scl[g]), sk1 = __half2float(scl[g + 8]);
       const float zk0 = __half2float(zer[g]), zk1 = __half2float(zer[g + 8]);
-      const float sv0 = __half2float(scl[16 + g]), sv1 = __half2float(scl[24 + g]);
-      const float zv0 = __half2float(zer[16 + g]), zv1 = __half2float(zer[24 + g]);
+      float sv0 = __half2float(scl[16 + g]), sv1 = __half2float(scl[24 + g]);
+      float zv0 = __half2float(zer[16 + g]), zv1 = __half2float(zer[24 + g]);
       const int tok = tok_base + 16 * t;
       const bool tail = tok + 16 > ctx;
+      if (tail) {
+        // rows past the context may hold anything, NaN scales included: they
+        // get p = 0 below, and V scale and offset 0 so that 0 * garbage
+        // cannot reach the sums
+        if (tok + g >= ctx) sv0 = zv0 = 0.0f;
+        if (tok + g + 8 >= ctx) sv1 = zv1 = 0.0f;
+      }
 
       uint32_t bp[NC][2];
 #pragma unroll

@@ -194,6 +194,40 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache,
                                   const kvq_attn_desc* desc, void* stream);
 
 /*
+ * paged_decode_append_attn_int4 - one decode step that also appends the
+ * step's new token: kv_quant_write of k_new/v_new at slot_mapping followed by
+ * paged_decode_attn_int4 over the contexts that include it, in one launch
+ * ([SAW] Abstract: the rotation-quantization kernel "integrates directly
+ * into paged KV-cache layouts" and attention execution is fused).
+ *
+ * For sequence n the new token is position context_lens[n] - 1: its slot
+ * (page * 16 + offset) must be page_table[n][(ctx - 1) / 16] * 16 +
+ * (ctx - 1) % 16, or -1 for "no new token" (the sequence is then decoded as
+ * paged_decode_attn_int4 would). Its K and V rows are rotated, quantized
+ * and stored exactly as kv_quant_write defines them (codes may differ from
+ * a kv_quant_write call only where both are within the rounding of a code
+ * boundary: this path rotates with fp32 butterflies), and the attention uses
+ * the stored values.
+ *
+ * k_new, v_new : device, bf16 [B][Hkv][D], contiguous, 16-byte aligned.
+ * slot_mapping : device, int64 [B], 8-byte aligned.
+ * cache, scales, zeros : device, written at the new slots, read as in
+ *                paged_decode_attn_int4.
+ * Every other argument as for paged_decode_attn_int4 (the same workspace
+ * size applies). A slot that does not match its sequence's last position,
+ * or a new token with context length 0, is not stored and records
+ * KVQ_ERR_OUT_OF_RANGE. Returns as paged_decode_attn_int4.
+ */
+kvq_status paged_decode_append_attn_int4(const void* q, const void* k_new,
+                                         const void* v_new,
+                                         const int64_t* slot_mapping,
+                                         uint8_t* cache, void* scales, void* zeros,
+                                         const int32_t* page_table,
+                                         const int32_t* context_lens, void* out,
+                                         void* workspace, size_t workspace_bytes,
+                                         const kvq_attn_desc* desc, void* stream);
+
+/*
  * paged_decode_attn_int4_static_ws - the same decode step as
  * paged_decode_attn_int4, for callers that are not allowed to allocate device
  * memory. Examples: a plug-in hosted by a serving runtime that owns all GPU

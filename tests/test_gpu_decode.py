@@ -271,3 +271,21 @@ def test_decode_out_of_date_host_lengths_stay_correct(orc, factor):
     got, _ = gpu_decode(w, pool, host_lens=host)
     assert_close(got, oracle_out(orc, w, pool), f"host lengths x{factor}")
     assert kvq.get_device_error() == 0
+
+
+def test_decode_ignores_garbage_past_the_context(orc):
+    """Rows of a sequence's last page past its context may hold anything (a
+    freed sequence's data, never-written memory): filled here with NaN scales
+    and offsets and random code bytes, they must not reach the output."""
+    ctx = [1, 17, 250, 31]
+    w = workloads.random_case(seed=71, B=len(ctx), Hq=16, Hkv=2, D=128, block=64, context_lens=ctx)
+    cache, scales, zeros = kvq.alloc_cache(w.num_pages, w.Hkv, w.D)
+    g = torch.Generator(device="cuda").manual_seed(72)
+    cache.copy_(torch.randint(0, 256, cache.shape, generator=g, device="cuda", dtype=torch.int32).to(torch.uint8))
+    scales.view(torch.int16).fill_(0x7E00)  # fp16 NaN
+    zeros.view(torch.int16).fill_(0x7E00)
+    pool = (cache, scales, zeros)
+    kvq.kv_quant_write(w.k_new.cuda(), w.v_new.cuda(), torch.as_tensor(w.slots_new).cuda(), *pool, w.block)
+    got, _ = gpu_decode(w, pool)
+    assert np.all(np.isfinite(got))
+    assert_close(got, oracle_out(orc, w, pool), "garbage past the context")

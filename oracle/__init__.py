@@ -52,7 +52,10 @@ def lib():
             "oracle_half_round_nearest": (ctypes.c_uint16, [c_d]),
             "oracle_hadamard": (None, [c_int, _p(i8)]),
             "oracle_rotate_f64": (c_int, [_p(f64), c_int, c_int, _p(f64)]),
+            "oracle_rotate_f64_signed": (c_int, [_p(f64), c_int, c_int, ctypes.c_void_p, _p(f64)]),
+            "oracle_unrotate_f64_signed": (c_int, [_p(f64), c_int, c_int, ctypes.c_void_p, _p(f64)]),
             "oracle_rotate_row": (c_int, [_p(u16), c_int, c_int, _p(f32)]),
+            "oracle_rotate_row_signed": (c_int, [_p(u16), c_int, c_int, ctypes.c_void_p, _p(f32)]),
             "oracle_scale_zero": (None, [ctypes.c_float, ctypes.c_float,
                                          ctypes.POINTER(ctypes.c_uint16),
                                          ctypes.POINTER(ctypes.c_uint16)]),
@@ -65,15 +68,17 @@ def lib():
             "oracle_dequant_row": (None, [_p(u8), c_int, ctypes.c_uint16, ctypes.c_uint16, _p(f64)]),
             "oracle_cache_row_offset": (ctypes.c_size_t, [c_i64, c_int, c_int, c_int, c_int, c_int]),
             "oracle_scale_offset": (ctypes.c_size_t, [c_i64, c_int, c_int, c_int, c_int]),
-            "oracle_quant_write": (c_int, [_p(u16), _p(u16), _p(i64), c_int, c_int, c_int, c_int, c_i64,
-                                           _p(u8), _p(u16), _p(u16), ctypes.c_void_p]),
-            "oracle_attn_rows": (c_int, [_p(f64), _p(f64), _p(f64), c_int, c_int, c_int, c_d, _p(f64)]),
+            "oracle_quant_write": (c_int, [_p(u16), _p(u16), _p(i64), c_int, c_int, c_int, c_int,
+                                           ctypes.c_void_p, c_i64, _p(u8), _p(u16), _p(u16),
+                                           ctypes.c_void_p]),
+            "oracle_attn_rows": (c_int, [_p(f64), _p(f64), _p(f64), c_int, c_int, c_int, ctypes.c_void_p,
+                                         c_d, _p(f64)]),
             "oracle_decode_one": (c_int, [_p(u16), _p(u8), _p(u16), _p(u16), _p(i32), _p(i32),
-                                          c_int, c_int, c_int, c_int, c_int, c_int, c_int, c_i64,
-                                          c_d, _p(f64)]),
+                                          c_int, c_int, c_int, c_int, c_int, c_int, ctypes.c_void_p,
+                                          c_int, c_i64, c_d, _p(f64)]),
             "oracle_decode_attn": (c_int, [_p(u16), _p(u8), _p(u16), _p(u16), _p(i32), _p(i32),
-                                           c_int, c_int, c_int, c_int, c_int, c_int, c_i64, c_d,
-                                           _p(f64)]),
+                                           c_int, c_int, c_int, c_int, c_int, ctypes.c_void_p, c_int,
+                                           c_i64, c_d, _p(f64)]),
             "oracle_num_threads": (c_int, []),
         }
         for name, (res, args) in sig.items():
@@ -118,18 +123,51 @@ def hadamard(b: int) -> np.ndarray:
     return H.reshape(b, b)
 
 
-def rotate_f64(x, b: int) -> np.ndarray:
+def sign_mask(signs, D: int):
+    """The 4-word sign mask of a per-channel +-1 vector (bit c set: channel c
+    negated; a bool / 0-1 array of D entries, or 4 words), or None."""
+    if signs is None:
+        return None
+    a = np.asarray(signs)
+    if a.dtype == np.uint32 and a.shape == (4,):
+        return np.ascontiguousarray(a)
+    a = a.astype(bool).reshape(-1)
+    assert a.size == D
+    words = np.zeros(4, np.uint32)
+    for c in np.nonzero(a)[0]:
+        words[c // 32] |= np.uint32(1) << np.uint32(c % 32)
+    return words
+
+
+def _sp(mask):
+    return None if mask is None else mask.ctypes.data
+
+
+def rotate_f64(x, b: int, signs=None) -> np.ndarray:
+    """y = R x, R = H_b diag(sigma) / sqrt(b) per block (sigma = +1 without signs)."""
     x = _c(x, np.float64)
     y = np.zeros_like(x)
-    rc = lib().oracle_rotate_f64(x, x.size, b, y)
+    m = sign_mask(signs, x.size)
+    rc = lib().oracle_rotate_f64_signed(x, x.size, b, _sp(m), y)
     assert rc == 0, rc
     return y
 
 
-def rotate_row(x_bf16_bits, b: int) -> np.ndarray:
+def unrotate_f64(x, b: int, signs=None) -> np.ndarray:
+    """y = R^T x."""
+    x = _c(x, np.float64)
+    y = np.zeros_like(x)
+    m = sign_mask(signs, x.size)
+    rc = lib().oracle_unrotate_f64_signed(x, x.size, b, _sp(m), y)
+    assert rc == 0, rc
+    return y
+
+
+def rotate_row(x_bf16_bits, b: int, signs=None) -> np.ndarray:
     x = _c(x_bf16_bits, np.uint16)
     y = np.zeros(x.size, np.float32)
-    rc = lib().oracle_rotate_row(x, x.size, b, y)
+    m = sign_mask(signs, x.size)
+    rc = lib().oracle_rotate_row_signed(x, x.size, b, _sp(m), y)
     assert rc == 0, rc
     return y
 
@@ -194,7 +232,7 @@ def scale_offset(page: int, Hkv: int, h: int, kv: int, off: int) -> int:
 
 
 def quant_write(k_bits, v_bits, slot_mapping, num_pages: int, b: int, cache=None,
-                scales=None, zeros=None, want_y: bool = False):
+                scales=None, zeros=None, want_y: bool = False, signs=None):
     """Rotate, quantize and place every row. k_bits/v_bits: uint16 [T, Hkv, D]
     bf16 bit patterns. Returns (cache, scales, zeros, y) where y is the fp32
     rotated rows [T, Hkv, 2, D] (or None). Buffers passed in are updated."""
@@ -210,7 +248,8 @@ def quant_write(k_bits, v_bits, slot_mapping, num_pages: int, b: int, cache=None
         zeros = np.zeros(num_pages * Hkv * 2 * 16, np.uint16)
     assert cache.flags.c_contiguous and scales.flags.c_contiguous and zeros.flags.c_contiguous
     y = np.zeros((T, Hkv, 2, D), np.float32) if want_y else None
-    rc = lib().oracle_quant_write(k, v, sm, T, Hkv, D, b, num_pages,
+    m = sign_mask(signs, D)
+    rc = lib().oracle_quant_write(k, v, sm, T, Hkv, D, b, _sp(m), num_pages,
                                   cache.reshape(-1), scales.reshape(-1), zeros.reshape(-1),
                                   y.ctypes.data if y is not None else None)
     if rc != 0:
@@ -220,20 +259,21 @@ def quant_write(k_bits, v_bits, slot_mapping, num_pages: int, b: int, cache=None
 
 # --- attention ------------------------------------------------------------
 
-def attn_rows(q, Krot, Vrot, b: int, scale: float) -> np.ndarray:
+def attn_rows(q, Krot, Vrot, b: int, scale: float, signs=None) -> np.ndarray:
     q = _c(q, np.float64)
     D = q.size
     Krot = _c(Krot, np.float64).reshape(-1, D)
     Vrot = _c(Vrot, np.float64).reshape(-1, D)
     out = np.zeros(D, np.float64)
-    rc = lib().oracle_attn_rows(q, Krot.reshape(-1), Vrot.reshape(-1), Krot.shape[0], D, b,
+    m = sign_mask(signs, D)
+    rc = lib().oracle_attn_rows(q, Krot.reshape(-1), Vrot.reshape(-1), Krot.shape[0], D, b, _sp(m),
                                 float(scale), out)
     assert rc == 0, rc
     return out
 
 
 def decode_attn(q_bits, cache, scales, zeros, page_table, context_lens, Hkv: int, b: int,
-                num_pages: int, softmax_scale: float = 0.0) -> np.ndarray:
+                num_pages: int, softmax_scale: float = 0.0, signs=None) -> np.ndarray:
     q = _c(q_bits, np.uint16)
     B, Hq, D = q.shape
     pt = _c(page_table, np.int32)
@@ -241,15 +281,15 @@ def decode_attn(q_bits, cache, scales, zeros, page_table, context_lens, Hkv: int
     out = np.zeros((B, Hq, D), np.float64)
     rc = lib().oracle_decode_attn(q.reshape(-1), _c(cache, np.uint8).reshape(-1),
                                   _c(scales, np.uint16).reshape(-1), _c(zeros, np.uint16).reshape(-1),
-                                  pt.reshape(-1), cl, B, Hq, Hkv, D, b, pt.shape[1], num_pages,
-                                  float(softmax_scale), out.reshape(-1))
+                                  pt.reshape(-1), cl, B, Hq, Hkv, D, b, _sp(sign_mask(signs, D)),
+                                  pt.shape[1], num_pages, float(softmax_scale), out.reshape(-1))
     if rc != 0:
         raise ValueError(f"oracle_decode_attn returned {rc}")
     return out
 
 
 def decode_one(q_bits, cache, scales, zeros, page_table, context_lens, n: int, hq: int,
-               Hkv: int, b: int, num_pages: int, softmax_scale: float = 0.0) -> np.ndarray:
+               Hkv: int, b: int, num_pages: int, softmax_scale: float = 0.0, signs=None) -> np.ndarray:
     q = _c(q_bits, np.uint16)
     B, Hq, D = q.shape
     pt = _c(page_table, np.int32)
@@ -257,7 +297,8 @@ def decode_one(q_bits, cache, scales, zeros, page_table, context_lens, n: int, h
     rc = lib().oracle_decode_one(q.reshape(-1), _c(cache, np.uint8).reshape(-1),
                                  _c(scales, np.uint16).reshape(-1), _c(zeros, np.uint16).reshape(-1),
                                  pt.reshape(-1), _c(context_lens, np.int32), n, hq, Hq, Hkv, D, b,
-                                 pt.shape[1], num_pages, float(softmax_scale), out)
+                                 _sp(sign_mask(signs, D)), pt.shape[1], num_pages, float(softmax_scale),
+                                 out)
     if rc != 0:
         raise ValueError(f"oracle_decode_one returned {rc}")
     return out

@@ -146,9 +146,18 @@ static int valid_block(int D, int b) {
   return (D % b) == 0;
 }
 
-/* y = R x in fp64 for an fp64 row: y[blk + i] = (1/sqrt(b)) sum_j H[i][j] x[blk + j].
- * b = 0 copies x. */
-int oracle_rotate_f64(const double* x, int D, int b, double* y) {
+/* The +-1 of channel c under a sign mask (NULL: all +1): bit c of
+ * signs[c / 32] set means -1. Randomized Hadamard: R = (1/sqrt(b)) H_b
+ * diag(sigma) per block, orthogonal for any signs, R^T = diag(sigma) H_b /
+ * sqrt(b) (H_b is symmetric). */
+static double sign_of(const uint32_t* signs, int c) {
+  return (signs && ((signs[c >> 5] >> (c & 31)) & 1u)) ? -1.0 : 1.0;
+}
+
+/* y = R x in fp64 for an fp64 row: with x' = sigma * x (elementwise),
+ * y[blk + i] = (1/sqrt(b)) sum_j H[i][j] x'[blk + j]. b = 0 copies x (signs
+ * must then be NULL or zero). */
+int oracle_rotate_f64_signed(const double* x, int D, int b, const uint32_t* signs, double* y) {
   if (!valid_block(D, b)) return -1;
   if (b == 0) {
     for (int c = 0; c < D; ++c) y[c] = x[c];
@@ -160,7 +169,7 @@ int oracle_rotate_f64(const double* x, int D, int b, double* y) {
   for (int blk = 0; blk < D; blk += b) {
     for (int i = 0; i < b; ++i) {
       double acc = 0.0;
-      for (int j = 0; j < b; ++j) acc += (double)H[i * b + j] * x[blk + j];
+      for (int j = 0; j < b; ++j) acc += (double)H[i * b + j] * (sign_of(signs, blk + j) * x[blk + j]);
       y[blk + i] = acc * norm;
     }
   }
@@ -168,15 +177,32 @@ int oracle_rotate_f64(const double* x, int D, int b, double* y) {
   return 0;
 }
 
+int oracle_rotate_f64(const double* x, int D, int b, double* y) {
+  return oracle_rotate_f64_signed(x, D, b, NULL, y);
+}
+
+/* y = R^T x = sigma * ((1/sqrt(b)) H_b x) (elementwise sign after the
+ * transform); with no signs R^T = R. */
+int oracle_unrotate_f64_signed(const double* x, int D, int b, const uint32_t* signs, double* y) {
+  if (oracle_rotate_f64_signed(x, D, b, NULL, y) != 0) return -1;
+  if (b > 0)
+    for (int c = 0; c < D; ++c) y[c] *= sign_of(signs, c);
+  return 0;
+}
+
 /* The rotated bf16 row, rounded once to fp32 (the precision the kernels keep
  * between rotation and quantization). */
-int oracle_rotate_row(const uint16_t* x_bf16, int D, int b, float* y) {
+int oracle_rotate_row_signed(const uint16_t* x_bf16, int D, int b, const uint32_t* signs, float* y) {
   double xd[256], yd[256];
   if (D <= 0 || D > 256) return -1;
   for (int c = 0; c < D; ++c) xd[c] = oracle_bf16_to_double(x_bf16[c]);
-  if (oracle_rotate_f64(xd, D, b, yd) != 0) return -1;
+  if (oracle_rotate_f64_signed(xd, D, b, signs, yd) != 0) return -1;
   for (int c = 0; c < D; ++c) y[c] = (float)yd[c];
   return 0;
+}
+
+int oracle_rotate_row(const uint16_t* x_bf16, int D, int b, float* y) {
+  return oracle_rotate_row_signed(x_bf16, D, b, NULL, y);
 }
 
 /* ------------------------------------------------------------------------- */
@@ -285,7 +311,7 @@ size_t oracle_scale_offset(int64_t page, int Hkv, int h, int kv, int off) {
  * Returns 0, -1 on bad shapes, -2 if a slot lies outside [0, num_pages*16).
  */
 int oracle_quant_write(const uint16_t* k, const uint16_t* v, const int64_t* slot_mapping,
-                       int T, int Hkv, int D, int b, int64_t num_pages,
+                       int T, int Hkv, int D, int b, const uint32_t* signs, int64_t num_pages,
                        uint8_t* cache, uint16_t* scales, uint16_t* zeros, float* y_out) {
   if (D != 64 && D != 128) return -1;
   if (!valid_block(D, b)) return -1;
@@ -307,7 +333,7 @@ int oracle_quant_write(const uint16_t* k, const uint16_t* v, const int64_t* slot
         float y[128];
         uint8_t codes[128];
         uint16_t s, z;
-        if (oracle_rotate_row(x, D, b, y) != 0) { bad = 1; continue; }
+        if (oracle_rotate_row_signed(x, D, b, signs, y) != 0) { bad = 1; continue; }
         oracle_quantize_row(y, D, codes, &s, &z);
         oracle_pack_row(codes, D, cache + oracle_cache_row_offset(page, Hkv, D, h, kv, off));
         scales[oracle_scale_offset(page, Hkv, h, kv, off)] = s;
@@ -326,16 +352,16 @@ int oracle_quant_write(const uint16_t* k, const uint16_t* v, const int64_t* slot
 
 /* Brute-force softmax attention for one query over n rotated rows:
  * qr = R q; logit_t = scale * qr . Krot[t]; p = softmax(logit);
- * out = R (sum_t p_t Vrot[t]). n = 0 gives out = 0. All fp64. */
+ * out = R^T (sum_t p_t Vrot[t]). n = 0 gives out = 0. All fp64. */
 int oracle_attn_rows(const double* q, const double* Krot, const double* Vrot, int n,
-                     int D, int b, double scale, double* out) {
+                     int D, int b, const uint32_t* signs, double scale, double* out) {
   double qr[256], orot[256];
   if (D > 256 || !valid_block(D, b)) return -1;
   if (n == 0) {
     for (int c = 0; c < D; ++c) out[c] = 0.0;
     return 0;
   }
-  oracle_rotate_f64(q, D, b, qr);
+  oracle_rotate_f64_signed(q, D, b, signs, qr);
   double* logit = (double*)malloc(sizeof(double) * (size_t)n);
   double m = -INFINITY;
   for (int t = 0; t < n; ++t) {
@@ -352,7 +378,7 @@ int oracle_attn_rows(const double* q, const double* Krot, const double* Vrot, in
     for (int c = 0; c < D; ++c) orot[c] += p * Vrot[(size_t)t * D + c];
   }
   for (int c = 0; c < D; ++c) orot[c] /= l;
-  oracle_rotate_f64(orot, D, b, out);
+  oracle_unrotate_f64_signed(orot, D, b, signs, out);
   free(logit);
   return 0;
 }
@@ -362,7 +388,7 @@ int oracle_attn_rows(const double* q, const double* Krot, const double* Vrot, in
  * or the context length falls outside the pool or the table. */
 int oracle_decode_one(const uint16_t* q_bf16, const uint8_t* cache, const uint16_t* scales,
                       const uint16_t* zeros, const int32_t* page_table, const int32_t* context_lens,
-                      int n, int hq, int Hq, int Hkv, int D, int b, int max_pages,
+                      int n, int hq, int Hq, int Hkv, int D, int b, const uint32_t* signs, int max_pages,
                       int64_t num_pages, double softmax_scale, double* out) {
   if (Hkv <= 0 || Hq % Hkv != 0) return -1;
   int G = Hq / Hkv;
@@ -385,7 +411,7 @@ int oracle_decode_one(const uint16_t* q_bf16, const uint8_t* cache, const uint16
                          scales[si], zeros[si], (kv == 0 ? K : V) + (size_t)t * D);
     }
   }
-  if (rc == 0) rc = oracle_attn_rows(q, K, V, ctx, D, b, scale, out);
+  if (rc == 0) rc = oracle_attn_rows(q, K, V, ctx, D, b, signs, scale, out);
   free(K);
   free(V);
   return rc;
@@ -394,8 +420,8 @@ int oracle_decode_one(const uint16_t* q_bf16, const uint8_t* cache, const uint16
 /* All sequences and query heads; out is fp64 [B][Hq][D]. */
 int oracle_decode_attn(const uint16_t* q_bf16, const uint8_t* cache, const uint16_t* scales,
                        const uint16_t* zeros, const int32_t* page_table, const int32_t* context_lens,
-                       int B, int Hq, int Hkv, int D, int b, int max_pages, int64_t num_pages,
-                       double softmax_scale, double* out) {
+                       int B, int Hq, int Hkv, int D, int b, const uint32_t* signs, int max_pages,
+                       int64_t num_pages, double softmax_scale, double* out) {
   if (D != 64 && D != 128) return -1;
   if (!valid_block(D, b)) return -1;
   if (Hkv <= 0 || Hq % Hkv != 0) return -1;
@@ -404,7 +430,7 @@ int oracle_decode_attn(const uint16_t* q_bf16, const uint8_t* cache, const uint1
   for (int n = 0; n < B; ++n)
     for (int hq = 0; hq < Hq; ++hq) {
       int r = oracle_decode_one(q_bf16, cache, scales, zeros, page_table, context_lens, n, hq,
-                                Hq, Hkv, D, b, max_pages, num_pages, softmax_scale,
+                                Hq, Hkv, D, b, signs, max_pages, num_pages, softmax_scale,
                                 out + ((size_t)n * Hq + hq) * D);
       if (r != 0) {
 #pragma omp critical

@@ -444,3 +444,93 @@ def test_quantization_moves_each_logit_within_the_step_bound(orc):
         exact = orc.rotate_f64(xd[i], 64)
         gap = abs(qr @ (khat - exact))
         assert gap <= np.abs(qr).sum() * f16(s) * (0.5 + 1e-5) + 1e-6 * np.abs(qr).sum() * np.abs(exact).max()
+
+
+# --- randomized Hadamard: R = H_b diag(sigma) / sqrt(b) ------------------------
+
+def _random_sign_vector(D, seed):
+    return np.random.default_rng(seed).integers(0, 2, D).astype(bool)
+
+
+@pytest.mark.parametrize("b,D", [(32, 64), (64, 128), (128, 128)])
+def test_signed_rotation_columns_closed_form(orc, b, D):
+    """R e_i = sigma_i * (column i of H_b within i's block) / sqrt(b), with
+    H_b[j][i] = (-1)^popcount(i & j): a sign applied after the transform, or
+    to the wrong index, fails here."""
+    sig = _random_sign_vector(D, 3 * b + D)
+    for i in range(D):
+        e = np.zeros(D)
+        e[i] = 1.0
+        y = orc.rotate_f64(e, b, signs=sig)
+        blk, ii = (i // b) * b, i % b
+        ref = np.zeros(D)
+        for j in range(b):
+            ref[blk + j] = (-1.0 if bin(ii & j).count("1") % 2 else 1.0) / math.sqrt(b)
+        ref *= -1.0 if sig[i] else 1.0
+        assert np.array_equal(y, ref) or np.allclose(y, ref, rtol=0, atol=1e-15), i
+
+
+@pytest.mark.parametrize("b,D", [(32, 64), (64, 128), (128, 128)])
+def test_signed_rotation_is_orthogonal_and_unrotate_is_its_transpose(orc, b, D):
+    sig = _random_sign_vector(D, b + D)
+    rng = np.random.default_rng(b)
+    for i in range(D):  # R^T R = I on every basis vector
+        e = np.zeros(D)
+        e[i] = 1.0
+        assert np.allclose(orc.unrotate_f64(orc.rotate_f64(e, b, signs=sig), b, signs=sig), e,
+                           rtol=0, atol=1e-14)
+    for _ in range(20):
+        x = rng.standard_normal(D) * 10
+        y = orc.rotate_f64(x, b, signs=sig)
+        assert abs(np.linalg.norm(y) / np.linalg.norm(x) - 1) < 1e-12
+        # <R x, z> = <x, R^T z> for a second vector
+        z = rng.standard_normal(D)
+        assert abs(y @ z - x @ orc.unrotate_f64(z, b, signs=sig)) < 1e-10 * np.linalg.norm(x) * np.linalg.norm(z)
+
+
+def test_zero_sign_mask_is_the_plain_rotation(orc):
+    from bit_kv_cache_20_b200 import workloads
+    rng = np.random.default_rng(8)
+    x = rng.standard_normal(128)
+    xb = workloads.bf16_bits(torch.from_numpy(x.astype(np.float32)).to(torch.bfloat16))
+    for b in (32, 64, 128):
+        assert np.array_equal(orc.rotate_f64(x, b, signs=np.zeros(128, bool)), orc.rotate_f64(x, b))
+        assert np.array_equal(orc.rotate_row(xb, b, signs=np.zeros(128, bool)), orc.rotate_row(xb, b))
+
+
+@pytest.mark.parametrize("b", [32, 128])
+def test_attention_invariance_with_random_signs(orc, b):
+    """Attention in the randomized-rotated space (q by R, rows by R, output
+    back by R^T) equals plain attention."""
+    rng = np.random.default_rng(50 + b)
+    D, n = 128, 29
+    sig = _random_sign_vector(D, 60 + b)
+    R = blockdiag_hadamard(D, b) @ np.diag(np.where(sig, -1.0, 1.0))
+    for _ in range(4):
+        q = rng.standard_normal(D) / 8
+        K = rng.standard_normal((n, D)) * np.exp(rng.standard_normal((n, 1)))
+        V = rng.standard_normal((n, D)) * np.exp(rng.standard_normal((n, 1)))
+        got = orc.attn_rows(q, K @ R.T, V @ R.T, b, 1 / math.sqrt(D), signs=sig)
+        ref = textbook_attention(q, K, V, 1 / math.sqrt(D))
+        assert np.allclose(got, ref, rtol=1e-11, atol=1e-11 * np.abs(ref).max())
+
+
+def test_quant_write_with_signs_rotates_each_row(orc):
+    """The write's placement with signs: each stored row is the quantization
+    of that row's signed rotation."""
+    from bit_kv_cache_20_b200 import workloads
+    rng = np.random.default_rng(9)
+    T, Hkv, D, b = 5, 2, 128, 64
+    sig = _random_sign_vector(D, 10)
+    k = workloads.bf16_bits(torch.from_numpy(rng.standard_normal((T, Hkv, D)).astype(np.float32)).to(torch.bfloat16))
+    v = workloads.bf16_bits(torch.from_numpy(rng.standard_normal((T, Hkv, D)).astype(np.float32)).to(torch.bfloat16))
+    slots = np.array([3, 17, 0, 40, 31], np.int64)
+    cache, scales, zeros, _ = orc.quant_write(k, v, slots, 4, b, signs=sig)
+    for t in range(T):
+        page, off = divmod(int(slots[t]), 16)
+        for h in range(Hkv):
+            for kv, src in enumerate((k, v)):
+                codes, s_, z_ = orc.quantize_row(orc.rotate_row(src[t, h], b, signs=sig))
+                row = ((page * Hkv + h) * 2 + kv) * 16 + off
+                assert np.array_equal(cache.reshape(-1, D // 2)[row], orc.pack_row(codes))
+                assert scales[row] == s_ and zeros[row] == z_

@@ -82,9 +82,11 @@ def _pool_shape(cache, scales, zeros):
 def kv_quant_write(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
                    cache: torch.Tensor, scales: torch.Tensor, zeros: torch.Tensor,
                    hadamard_block: int, page_table: Optional[torch.Tensor] = None,
-                   stream=None) -> None:
+                   stream=None, hadamard_signs=None) -> None:
     """Rotate (block Hadamard), quantize (token-wise INT4) and store new K/V
-    rows [T, Hkv, D] (bf16) at slot_mapping (int64 [T], -1 = skip)."""
+    rows [T, Hkv, D] (bf16) at slot_mapping (int64 [T], -1 = skip).
+    hadamard_signs: optional per-channel booleans for the randomized rotation
+    H_b diag(sigma) / sqrt(b) (decode with the same signs)."""
     P, Hkv, D = _pool_shape(cache, scales, zeros)
     _need(k, "k", torch.bfloat16)
     _need(v, "v", torch.bfloat16)
@@ -94,11 +96,26 @@ def kv_quant_write(k: torch.Tensor, v: torch.Tensor, slot_mapping: torch.Tensor,
     T = int(k.shape[0])
     if slot_mapping.numel() != T:
         raise ValueError("slot_mapping must hold one slot per token")
-    desc = WriteDesc(T, Hkv, D, PAGE_SIZE, P)
+    desc = WriteDesc(T, Hkv, D, PAGE_SIZE, P, sign_words(hadamard_signs, D))
     st = _lib.lib().kv_quant_write(_ptr(k), _ptr(v), _ptr(slot_mapping), _ptr(page_table),
                                    _ptr(cache), _ptr(scales), _ptr(zeros), int(hadamard_block),
                                    ctypes.byref(desc), ctypes.c_void_p(_stream_handle(stream)))
     _lib.check(st, "kv_quant_write")
+
+
+def sign_words(signs, head_dim: int):
+    """The 4-word mask of a randomized-Hadamard sign vector: `signs` holds
+    head_dim booleans (True negates that channel before the transform), or is
+    None (no signs)."""
+    words = (ctypes.c_uint32 * 4)(0, 0, 0, 0)
+    if signs is None:
+        return words
+    a = np.asarray(signs.cpu() if isinstance(signs, torch.Tensor) else signs).astype(bool).reshape(-1)
+    if a.size != head_dim:
+        raise ValueError("hadamard_signs must hold one entry per channel")
+    for c in np.nonzero(a)[0]:
+        words[int(c) // 32] |= 1 << (int(c) % 32)
+    return words
 
 
 def _host_lengths(context_lens_host, batch):
@@ -113,7 +130,7 @@ def _host_lengths(context_lens_host, batch):
 
 
 def _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scale, out_dtype,
-               inputs_ready=False, lens_ptr=None):
+               inputs_ready=False, lens_ptr=None, signs=None):
     P, Hkv, D = _pool_shape(cache, scales, zeros)
     if q.dim() != 3 or int(q.shape[2]) != D:
         raise ValueError("q must be bf16 [B, Hq, D]")
@@ -122,7 +139,7 @@ def _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scal
         raise ValueError("page_table must be int32 [B, max_pages]")
     return AttnDesc(B, Hq, Hkv, D, PAGE_SIZE, P, int(page_table.shape[1]), int(hadamard_block),
                     float(softmax_scale), out_dtype, ATTN_INPUTS_READY if inputs_ready else 0,
-                    lens_ptr)
+                    lens_ptr, sign_words(signs, D))
 
 
 def attn_workspace_size(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int,
@@ -155,7 +172,7 @@ def paged_decode_attn_int4(q: torch.Tensor, cache: torch.Tensor, scales: torch.T
                            context_lens: torch.Tensor, out: torch.Tensor, hadamard_block: int,
                            workspace: Optional[torch.Tensor] = None, softmax_scale: float = 0.0,
                            stream=None, inputs_ready: bool = False,
-                           context_lens_host=None) -> None:
+                           context_lens_host=None, hadamard_signs=None) -> None:
     """One decode step over the INT4 cache; out is fp32 or bf16 [B, Hq, D].
     inputs_ready: q, page_table and context_lens were not written by the
     kernel launched just before this call on the stream (KVQ_ATTN_INPUTS_READY),
@@ -173,7 +190,7 @@ def paged_decode_attn_int4(q: torch.Tensor, cache: torch.Tensor, scales: torch.T
         raise ValueError("out must have q's shape")
     lens_arr, lens_ptr = _host_lengths(context_lens_host, int(q.shape[0]) if q.dim() == 3 else -1)
     desc = _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scale,
-                      0 if out.dtype == torch.float32 else 1, inputs_ready, lens_ptr)
+                      0 if out.dtype == torch.float32 else 1, inputs_ready, lens_ptr, hadamard_signs)
     if context_lens.numel() != desc.batch:
         raise ValueError("context_lens must hold one length per sequence")
     L = _lib.lib()
@@ -194,7 +211,8 @@ def paged_decode_append_attn_int4(q: torch.Tensor, k_new: torch.Tensor, v_new: t
                                   out: torch.Tensor, hadamard_block: int,
                                   workspace: Optional[torch.Tensor] = None,
                                   softmax_scale: float = 0.0, stream=None,
-                                  inputs_ready: bool = False, context_lens_host=None) -> None:
+                                  inputs_ready: bool = False, context_lens_host=None,
+                                  hadamard_signs=None) -> None:
     """One decode step that first appends each sequence's new token: k_new,
     v_new bf16 [B, Hkv, D] are rotated, quantized and stored at slot_mapping
     (int64 [B], -1 = no new token), position context_lens - 1 of their
@@ -213,7 +231,7 @@ def paged_decode_append_attn_int4(q: torch.Tensor, k_new: torch.Tensor, v_new: t
         raise ValueError("out must have q's shape")
     lens_arr, lens_ptr = _host_lengths(context_lens_host, int(q.shape[0]) if q.dim() == 3 else -1)
     desc = _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scale,
-                      0 if out.dtype == torch.float32 else 1, inputs_ready, lens_ptr)
+                      0 if out.dtype == torch.float32 else 1, inputs_ready, lens_ptr, hadamard_signs)
     if context_lens.numel() != desc.batch or slot_mapping.numel() != desc.batch:
         raise ValueError("context_lens and slot_mapping must hold one entry per sequence")
     if tuple(k_new.shape) != (desc.batch, desc.num_kv_heads, desc.head_dim) or k_new.shape != v_new.shape:
@@ -233,7 +251,7 @@ def paged_decode_attn_int4_static_ws(q: torch.Tensor, cache: torch.Tensor, scale
                                      zeros: torch.Tensor, page_table: torch.Tensor,
                                      context_lens: torch.Tensor, out: torch.Tensor,
                                      hadamard_block: int, softmax_scale: float = 0.0,
-                                     stream=None, context_lens_host=None) -> None:
+                                     stream=None, context_lens_host=None, hadamard_signs=None) -> None:
     """paged_decode_attn_int4 for callers that must not allocate device memory
     (e.g. a plug-in whose host runtime owns all GPU memory): the split-K
     scratch is a fixed array inside the library, shared by every call on the
@@ -249,7 +267,7 @@ def paged_decode_attn_int4_static_ws(q: torch.Tensor, cache: torch.Tensor, scale
         raise ValueError("out must have q's shape")
     lens_arr, lens_ptr = _host_lengths(context_lens_host, int(q.shape[0]) if q.dim() == 3 else -1)
     desc = _attn_desc(q, cache, scales, zeros, page_table, hadamard_block, softmax_scale,
-                      0 if out.dtype == torch.float32 else 1, False, lens_ptr)
+                      0 if out.dtype == torch.float32 else 1, False, lens_ptr, hadamard_signs)
     if context_lens.numel() != desc.batch:
         raise ValueError("context_lens must hold one length per sequence")
     st = _lib.lib().paged_decode_attn_int4_static_ws(

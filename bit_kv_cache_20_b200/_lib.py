@@ -18,7 +18,7 @@ STATUS_NAMES = {
 class WriteDesc(ctypes.Structure):
     _fields_ = [("num_tokens", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
                 ("head_dim", ctypes.c_int32), ("page_size", ctypes.c_int32),
-                ("num_pages", ctypes.c_int32)]
+                ("num_pages", ctypes.c_int32), ("hadamard_signs", ctypes.c_uint32 * 4)]
 
 
 class AttnDesc(ctypes.Structure):
@@ -27,7 +27,8 @@ class AttnDesc(ctypes.Structure):
                 ("page_size", ctypes.c_int32), ("num_pages", ctypes.c_int32),
                 ("max_pages_per_seq", ctypes.c_int32), ("hadamard_block", ctypes.c_int32),
                 ("softmax_scale", ctypes.c_float), ("out_dtype", ctypes.c_int32),
-                ("flags", ctypes.c_int32), ("context_lens_host", ctypes.POINTER(ctypes.c_int32))]
+                ("flags", ctypes.c_int32), ("context_lens_host", ctypes.POINTER(ctypes.c_int32)),
+                ("hadamard_signs", ctypes.c_uint32 * 4)]
 
 
 ATTN_INPUTS_READY = 1  # KVQ_ATTN_INPUTS_READY

@@ -476,6 +476,17 @@ size_t planned_workspace_bound(const kvq_attn_desc* d, int dev, int app) {
   return best;
 }
 
+// A randomized-Hadamard sign mask: zero without a rotation, no bit at or
+// above D.
+bool valid_signs(const uint32_t (&sg)[4], int D, int b) {
+  for (int w = 0; w < 4; ++w) {
+    const uint32_t allowed = (b == 0) ? 0u : (D >= 32 * (w + 1)) ? 0xFFFFFFFFu : (D <= 32 * w) ? 0u
+                                                                  : ((1u << (D - 32 * w)) - 1u);
+    if (sg[w] & ~allowed) return false;
+  }
+  return true;
+}
+
 kvq_status check_attn_desc(const kvq_attn_desc* d) {
   if (!d) return KVQ_ERR_INVALID_ARG;
   if (d->batch < 0 || d->num_q_heads < 1 || d->num_kv_heads < 1 || d->num_pages < 1 ||
@@ -491,6 +502,7 @@ kvq_status check_attn_desc(const kvq_attn_desc* d) {
   if (d->head_dim != 64 && d->head_dim != 128) return KVQ_ERR_UNSUPPORTED;
   if (G != 1 && G != 2 && G != 4 && G != 8) return KVQ_ERR_UNSUPPORTED;
   if (!valid_block(d->head_dim, d->hadamard_block)) return KVQ_ERR_UNSUPPORTED;
+  if (!valid_signs(d->hadamard_signs, d->head_dim, d->hadamard_block)) return KVQ_ERR_INVALID_ARG;
   return KVQ_OK;
 }
 
@@ -560,6 +572,7 @@ kvq_status kv_quant_write(const void* k, const void* v, const int64_t* slot_mapp
     return KVQ_ERR_INVALID_ARG;
   if (d.head_dim != 64 && d.head_dim != 128) return KVQ_ERR_UNSUPPORTED;
   if (!valid_block(d.head_dim, hadamard_block)) return KVQ_ERR_UNSUPPORTED;
+  if (!valid_signs(d.hadamard_signs, d.head_dim, hadamard_block)) return KVQ_ERR_INVALID_ARG;
   if (d.num_tokens == 0) return KVQ_OK;  // nothing to do; pointers may be NULL
   if (!k || !v || !slot_mapping || !cache || !scales || !zeros) return KVQ_ERR_INVALID_ARG;
   if (!aligned(k, 16) || !aligned(v, 16) || !aligned(cache, 16) || !aligned(scales, 16) ||
@@ -582,6 +595,7 @@ kvq_status kv_quant_write(const void* k, const void* v, const int64_t* slot_mapp
   p.num_slots = (long long)d.num_pages * KVQ_PAGE_SIZE;
   p.num_tiles = (int)tiles;
   p.cb = hadamard_block > 0 ? (float)(1.0 / std::sqrt((double)hadamard_block)) : 1.0f;
+  for (int w = 0; w < 4; ++w) p.signs[w] = d.hadamard_signs[w];
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d.head_dim == 64 ? dispatch_write<64>(p, hadamard_block, dev, s)
                           : dispatch_write<128>(p, hadamard_block, dev, s);
@@ -675,6 +689,7 @@ kvq_status decode_impl(const void* q, const uint8_t* cache, const void* scales, 
   const double scale = d.softmax_scale > 0.0f ? (double)d.softmax_scale : 1.0 / std::sqrt((double)d.head_dim);
   p.qmul = (float)(cb * scale * 1.4426950408889634);  // log2(e)
   p.cb = (float)cb;
+  for (int w = 0; w < 4; ++w) p.signs[w] = d.hadamard_signs[w];
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   return d.head_dim == 64 ? dispatch_attn<64>(p, d.hadamard_block, plan, dev, s)
                           : dispatch_attn<128>(p, d.hadamard_block, plan, dev, s);

@@ -77,6 +77,7 @@ struct AttnParams {
   int out_bf16;
   float qmul;                 // c_b * softmax_scale * log2(e)
   float cb;                   // c_b (output rotation), 1 for plain INT4
+  uint32_t signs[4];          // randomized Hadamard signs (bit c: channel c), as written
   int inputs_ready;           // q, page_table, ctx_lens not written by the previous kernel
   // Decode-append (slots_new != nullptr): sequence n's new token, k_new /
   // v_new bf16 [B][Hkv][D], is quantized and stored at slots_new[n] (-1: none)
@@ -187,6 +188,19 @@ __device__ __forceinline__ void warp_fwht(float (&v)[D / 32], int lane) {
   }
 }
 
+
+// Randomized Hadamard: negate the lane's elements (channels E lane + e) whose
+// sign bit is set. R = H_b diag(sigma) / sqrt(b): applied before the
+// transform to rotate, after it for R^T.
+template <int D>
+__device__ __forceinline__ void apply_signs(float (&v)[D / 32], const uint32_t (&sg)[4], int lane) {
+  constexpr int E = D / 32;
+#pragma unroll
+  for (int e = 0; e < E; ++e) {
+    const int c = E * lane + e;
+    v[e] = __uint_as_float(__float_as_uint(v[e]) ^ (((sg[c >> 5] >> (c & 31)) & 1u) << 31));
+  }
+}
 
 template <int D, int BLK, int HG, int NC, bool APP>
 __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
@@ -358,7 +372,10 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
       float v[E];
 #pragma unroll
       for (int e = 0; e < E; ++e) v[e] = rp[E * lane + e];
-      if constexpr (BLK > 0) warp_fwht<D, BLK>(v, lane);
+      if constexpr (BLK > 0) {
+        apply_signs<D>(v, p.signs, lane);
+        warp_fwht<D, BLK>(v, lane);
+      }
       float amax = 0.0f, sum = 0.0f;
 #pragma unroll
       for (int e = 0; e < E; ++e) {
@@ -412,7 +429,10 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
     float v[E];
 #pragma unroll
     for (int e = 0; e < E; ++e) v[e] = bf16_bits_to_float(src[e]);
-    if constexpr (BLK > 0) warp_fwht<D, BLK>(v, lane);
+    if constexpr (BLK > 0) {
+      apply_signs<D>(v, p.signs, lane);
+      warp_fwht<D, BLK>(v, lane);
+    }
     float mn = v[0], mx = v[0];
 #pragma unroll
     for (int e = 1; e < E; ++e) {
@@ -879,7 +899,10 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
       float v[E];
 #pragma unroll
       for (int e2 = 0; e2 < E; ++e2) v[e2] = rp[E * lane + e2];
-      if constexpr (BLK > 0) warp_fwht<D, BLK>(v, lane);
+      if constexpr (BLK > 0) {
+        warp_fwht<D, BLK>(v, lane);
+        apply_signs<D>(v, p.signs, lane);
+      }
       const size_t o_base = ((size_t)n * p.Hq + (size_t)(hgi * HG + hh) * G + r) * D + E * lane;
 #pragma unroll
       for (int e2 = 0; e2 < E; ++e2) store_out(p, o_base + e2, BLK > 0 ? v[e2] * p.cb : v[e2]);
@@ -895,7 +918,10 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
     float v[E];
 #pragma unroll
     for (int e2 = 0; e2 < E; ++e2) v[e2] = rp[E * lane + e2];
-    if constexpr (BLK > 0) warp_fwht<D, BLK>(v, lane);
+    if constexpr (BLK > 0) {
+      warp_fwht<D, BLK>(v, lane);
+      apply_signs<D>(v, p.signs, lane);
+    }
     const size_t o_base = ((size_t)n * p.Hq + (size_t)(hgi * HG + hh) * G + r) * D + E * lane;
 #pragma unroll
     for (int e2 = 0; e2 < E; ++e2) store_out(p, o_base + e2, BLK > 0 ? v[e2] * p.cb : v[e2]);

@@ -31,6 +31,7 @@ struct WriteParams {
   long long num_slots;      // num_pages * 16
   int num_tiles;            // ceil(T/32) * Hkv * 2
   float cb;                 // fp32(1/sqrt(b)), 1 for b = 0
+  uint32_t signs[4];        // randomized Hadamard: bit c negates channel c before the transform
 };
 
 constexpr int kWriteWarps = 4;

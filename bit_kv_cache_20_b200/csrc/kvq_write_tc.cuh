@@ -111,13 +111,16 @@ __global__ void __launch_bounds__(kTcThreads, 1)
   tc_fence_before();
   __syncthreads();  // barriers and the tensor-memory address are in place
   tc_fence_after();
-  // While warp 0 starts the first copies, the other warps build
-  // H = diag(H_b) (unnormalized Sylvester order) as the B operand [n][k]
-  // (symmetric, so B[n][k] = H[k][n]), 16 bytes at a time, then meet on
-  // named barrier 1 before the first MMA.
+  // While warp 0 starts the first copies, the other warps build the B
+  // operand [n][k] = H[n][k] sigma_k (H = diag(H_b), unnormalized Sylvester
+  // order, symmetric; sigma the randomized signs, all +1 by default), so that
+  // Y = X B^T = (R X^T)^T sqrt(b), 16 bytes at a time, then meet on named
+  // barrier 1 before the first MMA.
   if (warp != 0) {
     for (int i = tid - 32; i < D * (D / 8); i += kTcThreads - 32) {
       const int n = i / (D / 8), k0 = 8 * (i % (D / 8));
+      // sign word of channels k0 .. k0 + 7 (constant indices: no local copy of p)
+      const uint32_t sw = k0 < 32 ? p.signs[0] : k0 < 64 ? p.signs[1] : k0 < 96 ? p.signs[2] : p.signs[3];
       uint32_t w[4];
 #pragma unroll
       for (int e = 0; e < 4; ++e) {
@@ -126,7 +129,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         for (int hlf = 0; hlf < 2; ++hlf) {
           const int k = k0 + 2 * e + hlf;
           uint32_t bits = 0;  // bf16 0
-          if (n / BLK == k / BLK) bits = (__popc((n % BLK) & (k % BLK)) & 1) ? 0xBF80u : 0x3F80u;  // -1, +1
+          if (n / BLK == k / BLK) {
+            bits = (__popc((n % BLK) & (k % BLK)) & 1) ? 0xBF80u : 0x3F80u;  // -1, +1
+            bits ^= ((sw >> (k & 31)) & 1u) << 15;  // times sigma_k
+          }
           pair |= bits << (16 * hlf);
         }
         w[e] = pair;

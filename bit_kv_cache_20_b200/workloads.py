@@ -231,3 +231,10 @@ def bf16_bits(t: torch.Tensor) -> np.ndarray:
 
 def page_count(context_lens) -> int:
     return int(sum(math.ceil(int(c) / PAGE) for c in context_lens))
+
+
+def random_signs(seed: int, D: int) -> np.ndarray:
+    """A seeded randomized-Hadamard sign vector: D booleans, True = negate
+    that channel before the transform."""
+    g = torch.Generator().manual_seed(seed)
+    return (torch.rand(D, generator=g) < 0.5).numpy()

@@ -49,7 +49,7 @@ extern "C" {
 #endif
 
 #define KVQ_PAGE_SIZE 16
-#define KVQ_ABI_VERSION 3
+#define KVQ_ABI_VERSION 4
 
 typedef enum kvq_status {
   KVQ_OK = 0,
@@ -68,6 +68,11 @@ typedef struct kvq_write_desc {
   int32_t head_dim;     /* D: 64 or 128 */
   int32_t page_size;    /* must be KVQ_PAGE_SIZE */
   int32_t num_pages;    /* pages in the pool; valid slots are [0, num_pages*16) */
+  /* Randomized Hadamard: bit c of hadamard_signs[c / 32] set negates channel
+   * c before the transform, R = H_b diag(sigma) / sqrt(b) (orthogonal for any
+   * signs). All zero: the plain rotation. Must be zero when hadamard_block is
+   * 0 and above bit D - 1; a decode of the cache must use the same mask. */
+  uint32_t hadamard_signs[4];
 } kvq_write_desc;
 
 /* Shapes of one paged_decode_attn_int4 call. */
@@ -89,6 +94,9 @@ typedef struct kvq_attn_desc {
    * still reads the lengths from the device array, so a host copy that is
    * out of date costs balance, never correctness. Read during the call only. */
   const int32_t* context_lens_host;
+  /* The sign mask the cache was written with (see kvq_write_desc): q is
+   * rotated by R and the output by R^T = diag(sigma) H_b / sqrt(b). */
+  uint32_t hadamard_signs[4];
 } kvq_attn_desc;
 
 /*
@@ -130,7 +138,8 @@ typedef struct kvq_attn_desc {
  * page_table   : accepted for signature compatibility with the decode call and
  *                not read; placement is decided by slot_mapping alone. May be NULL.
  * cache, scales, zeros : device, layouts above, 16-byte aligned.
- * hadamard_block : 0, 32, 64 or 128, and at most D.
+ * hadamard_block : 0, 32, 64 or 128, and at most D (with desc->hadamard_signs,
+ *                the randomized rotation H_b diag(sigma) / sqrt(b)).
  * desc         : host pointer to the shapes.
  * Inputs must be finite and their rotated values must lie within the fp16
  * range (|y| <= 65504); rows outside it get infinite or NaN s/z.

@@ -47,7 +47,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_version_and_status_strings(L):
-    assert L.kvq_abi_version() == 3
+    assert L.kvq_abi_version() == 4
     assert L.kvq_status_string(0) == b"KVQ_OK"
     assert L.kvq_status_string(5) == b"KVQ_ERR_TIMEOUT"
     assert L.kvq_status_string(99) == b"KVQ_ERR_UNKNOWN"
@@ -76,6 +76,9 @@ def test_write_argument_errors(L):
     assert write_call(L, WriteDesc(4, 2, 64, 16, 4), k=0) == 1      # null
     assert write_call(L, WriteDesc(4, 2, 64, 16, 4), cache=FAKE + 8) == 1  # misaligned
     assert write_call(L, WriteDesc(0, 2, 64, 16, 4)) == 0           # nothing to do
+    sg = ctypes.c_uint32 * 4
+    assert write_call(L, WriteDesc(4, 2, 64, 16, 4, sg(0, 0, 2, 0)), b=64) == 1  # sign of channel 65 > D
+    assert write_call(L, WriteDesc(4, 2, 64, 16, 4, sg(1, 0, 0, 0)), b=0) == 1   # signs without a rotation
 
 
 def attn_call(L, desc, ws=None, ws_bytes=0, out=FAKE):
@@ -89,7 +92,7 @@ def test_decode_argument_errors(L):
     from bit_kv_cache_20_b200._lib import AttnDesc
     ok = dict(batch=2, num_q_heads=8, num_kv_heads=2, head_dim=128, page_size=16, num_pages=10,
               max_pages_per_seq=5, hadamard_block=128, softmax_scale=0.0, out_dtype=0, flags=0,
-              context_lens_host=None)
+              context_lens_host=None, hadamard_signs=(ctypes.c_uint32 * 4)(0, 0, 0, 0))
 
     def d(**kw):
         a = dict(ok)
@@ -105,6 +108,9 @@ def test_decode_argument_errors(L):
     assert attn_call(L, d(softmax_scale=-1.0)) == 1
     assert attn_call(L, d(out_dtype=3)) == 1
     assert attn_call(L, d(flags=2)) == 1                            # unknown flag bit
+    assert attn_call(L, d(hadamard_block=0, hadamard_signs=(ctypes.c_uint32 * 4)(1, 0, 0, 0))) == 1
+    assert attn_call(L, d(head_dim=64, hadamard_block=64,
+                          hadamard_signs=(ctypes.c_uint32 * 4)(0, 0, 1, 0))) == 1  # channel 64 of D = 64
     assert attn_call(L, d(max_pages_per_seq=0)) == 1
     assert attn_call(L, d(), out=FAKE + 2) == 1                     # fp32 out misaligned
     assert attn_call(L, d(batch=0)) == 0                            # nothing to do

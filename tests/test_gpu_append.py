@@ -28,13 +28,13 @@ def _split_last(w):
     return last, rest
 
 
-def _run(orc, w, b, host_lens=False, slots_override=None, out_dtype=torch.float32):
+def _run(orc, w, b, host_lens=False, slots_override=None, out_dtype=torch.float32, signs=None):
     last, rest = _split_last(w)
     pool = Pool(w.num_pages, w.Hkv, w.D)
     slots = torch.as_tensor(w.slots_new)
     if rest.size:
         kvq.kv_quant_write(w.k_new[rest].cuda(), w.v_new[rest].cuda(), slots[rest].cuda(),
-                           pool.cache, pool.scales, pool.zeros, b)
+                           pool.cache, pool.scales, pool.zeros, b, hadamard_signs=signs)
     step_slots = slots[last].clone() if slots_override is None else torch.as_tensor(slots_override)
     pt = torch.as_tensor(w.page_table).cuda()
     cl = torch.as_tensor(w.context_lens).cuda()
@@ -44,15 +44,15 @@ def _run(orc, w, b, host_lens=False, slots_override=None, out_dtype=torch.float3
     kvq.paged_decode_append_attn_int4(
         w.q.cuda(), w.k_new[last].contiguous().cuda(), w.v_new[last].contiguous().cuda(),
         step_slots.to(torch.int64).cuda(), pool.cache, pool.scales, pool.zeros, pt, cl, out, b, ws,
-        context_lens_host=w.context_lens if host_lens else None)
+        context_lens_host=w.context_lens if host_lens else None, hadamard_signs=signs)
     torch.cuda.synchronize()
     return pool, last, step_slots.numpy(), out.float().cpu().numpy().astype(np.float64), ws
 
 
-def _oracle(orc, w, pool, b):
+def _oracle(orc, w, pool, b, signs=None):
     c, s, z = pool.host()
     return orc.decode_attn(workloads.bf16_bits(w.q), c.reshape(-1), s, z, w.page_table, w.context_lens,
-                           w.Hkv, b, w.num_pages)
+                           w.Hkv, b, w.num_pages, signs=signs)
 
 
 @pytest.mark.parametrize("b", [0, 64, 128])
@@ -107,3 +107,13 @@ def test_append_slot_minus_one_and_a_mismatched_slot(orc):
     check_tokens(orc, pool, w.k_new, w.v_new, w.slots_new, 32, tokens=[last[1]])
     ref = _oracle(orc, w, pool, 32)
     assert_close(got[1], ref[1], "appended sequence")
+
+
+def test_append_with_randomized_hadamard_signs(orc):
+    ctx = [700, 18, 4100]
+    w = workloads.random_case(seed=66, B=len(ctx), Hq=16, Hkv=4, D=128, block=64, context_lens=ctx)
+    sig = workloads.random_signs(67, 128)
+    pool, last, _, got, _ = _run(orc, w, 64, signs=sig)
+    assert kvq.get_device_error() == 0
+    check_tokens(orc, pool, w.k_new, w.v_new, w.slots_new, 64, tokens=last, signs=sig)
+    assert_close(got, _oracle(orc, w, pool, 64, signs=sig), "append with signs")

@@ -289,3 +289,26 @@ def test_decode_ignores_garbage_past_the_context(orc):
     got, _ = gpu_decode(w, pool)
     assert np.all(np.isfinite(got))
     assert_close(got, oracle_out(orc, w, pool), "garbage past the context")
+
+
+@pytest.mark.parametrize("D,b,G", [(64, 32, 4), (128, 64, 8), (128, 128, 4)])
+def test_decode_randomized_hadamard_signs(orc, D, b, G):
+    """q rotated by R = H_b diag(sigma)/sqrt(b), the output by R^T, over a
+    cache written with the same signs; several splits (long context)."""
+    ctx = [5000, 33, 1]
+    w = workloads.random_case(seed=91 + D + b + G, B=len(ctx), Hq=2 * G, Hkv=2, D=D, block=b, context_lens=ctx)
+    sig = workloads.random_signs(92 + D, D)
+    cache, scales, zeros = kvq.alloc_cache(w.num_pages, w.Hkv, w.D)
+    kvq.kv_quant_write(w.k_new.cuda(), w.v_new.cuda(), torch.as_tensor(w.slots_new).cuda(), cache, scales,
+                       zeros, b, hadamard_signs=sig)
+    pool = (cache, scales, zeros)
+    pt = torch.as_tensor(w.page_table).cuda()
+    cl = torch.as_tensor(w.context_lens).cuda()
+    out = torch.empty((w.B, w.Hq, w.D), device="cuda")
+    ws = kvq.alloc_workspace(kvq.attn_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.num_pages, w.max_pages, b))
+    kvq.paged_decode_attn_int4(w.q.cuda(), cache, scales, zeros, pt, cl, out, b, ws, hadamard_signs=sig)
+    got = out.cpu().numpy().astype(np.float64)
+    c, s_, z_ = host_cache(*pool)
+    ref = orc.decode_attn(workloads.bf16_bits(w.q), c, s_, z_, w.page_table, w.context_lens, w.Hkv, b,
+                          w.num_pages, signs=sig)
+    assert_close(got, ref, f"signs D={D} b={b} G={G}")

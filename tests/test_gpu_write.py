@@ -71,7 +71,7 @@ def gpu_write(pool, k, v, slots, b):
     assert kvq.get_device_error() == 0
 
 
-def check_tokens(orc, pool, k, v, slots, b, tokens=None, written_rows=None):
+def check_tokens(orc, pool, k, v, slots, b, tokens=None, written_rows=None, signs=None):
     """Compare the rows of `tokens` (default: all) with the oracle."""
     cache, scales, zeros = pool.host()
     kb = workloads.bf16_bits(k)
@@ -85,7 +85,7 @@ def check_tokens(orc, pool, k, v, slots, b, tokens=None, written_rows=None):
         for h in range(Hkv):
             for kv, src in enumerate((kb, vb)):
                 rows.append(((page * Hkv + h) * 2 + kv) * 16 + off)
-                ys.append(orc.rotate_row(src[t, h], b))
+                ys.append(orc.rotate_row(src[t, h], b, signs=signs))
                 xs.append(src[t, h].view(np.int16).astype(np.int32) << 16)
     rows = np.asarray(rows, np.int64)
     x_rows = np.asarray(xs, np.int32).view(np.float32).astype(np.float64) if xs else np.zeros((0, D))
@@ -220,3 +220,22 @@ def test_write_prior_then_append(orc):
                  tokens=rng.choice(w.k_prior.shape[0], 200, replace=False))
     check_tokens(orc, pool, w.k_new, w.v_new, w.slots_new, w.block,
                  tokens=rng.choice(w.tokens_written, 200, replace=False))
+
+
+@pytest.mark.parametrize("D,b", [(64, 32), (64, 64), (128, 64), (128, 128)])
+def test_write_randomized_hadamard_signs(orc, D, b):
+    """R = H_b diag(sigma) / sqrt(b) with seeded random signs: the tensor-core
+    operand carries the signs; codes, s and z against the oracle's signed
+    rotation."""
+    w = workloads.random_case(seed=81 + D + b, B=2, Hq=4, Hkv=2, D=D, block=b, context_lens=[300, 77])
+    sig = workloads.random_signs(82 + b, D)
+    pool = Pool(w.num_pages, w.Hkv, D)
+    kvq.kv_quant_write(w.k_new.cuda(), w.v_new.cuda(), torch.as_tensor(w.slots_new).cuda(),
+                       pool.cache, pool.scales, pool.zeros, b, hadamard_signs=sig)
+    assert kvq.get_device_error() == 0
+    check_tokens(orc, pool, w.k_new, w.v_new, w.slots_new, b, signs=sig)
+    # the signs matter: the unsigned rotation stores other codes
+    plain = Pool(w.num_pages, w.Hkv, D)
+    kvq.kv_quant_write(w.k_new.cuda(), w.v_new.cuda(), torch.as_tensor(w.slots_new).cuda(),
+                       plain.cache, plain.scales, plain.zeros, b)
+    assert not np.array_equal(pool.host()[0], plain.host()[0])

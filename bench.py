@@ -260,11 +260,8 @@ class Step:
         # new token (rewritten in place every step, so every step does the
         # same work); separate = a 1-token-per-sequence write + the decode,
         # fused = one paged_decode_append_attn_int4 launch
-        ends = np.cumsum(np.asarray(w.context_lens, np.int64))
-        last = torch.as_tensor(ends - 1)
-        self.k1 = w.k_new[last].contiguous().to(dev)
-        self.v1 = w.v_new[last].contiguous().to(dev)
-        self.s1 = torch.as_tensor(np.asarray(w.slots_new)[ends - 1]).to(dev)
+        k1, v1, s1 = self.last_tokens(w)
+        self.k1, self.v1, self.s1 = k1.to(dev), v1.to(dev), s1.to(dev)
         self.wdesc1 = _lib.WriteDesc(w.B, w.Hkv, w.D, 16, w.num_pages)
         self.write1_args, self.app_args = [], []
         for i in range(self.N_POOLS):
@@ -277,6 +274,34 @@ class Step:
                                   P(self.pt.data_ptr()), P(self.ctx.data_ptr()), P(self.out.data_ptr()),
                                   P(self.ws.data_ptr()), self.ws_bytes, ctypes.byref(self.adesc), self.sh))
         torch.cuda.synchronize(dev)  # allocations above ran on the default stream
+
+    @staticmethod
+    def last_tokens(w):
+        """K, V ([B, Hkv, D]) and slot of every sequence's last context token,
+        wherever the workload holds it (the step's new tokens or the prior
+        context); a sequence with an empty context gets slot -1."""
+        import numpy as np
+        import torch
+        where = {}
+        for src, (k, v, slots) in enumerate(((w.k_prior, w.v_prior, w.slots_prior),
+                                              (w.k_new, w.v_new, w.slots_new))):
+            for i, sl in enumerate(np.asarray(slots).tolist()):
+                if sl >= 0:
+                    where[sl] = (src, i)
+        k1 = torch.zeros((w.B, w.Hkv, w.D), dtype=torch.bfloat16)
+        v1 = torch.zeros_like(k1)
+        s1 = np.full(w.B, -1, np.int64)
+        for n in range(w.B):
+            c = int(w.context_lens[n])
+            if c == 0:
+                continue
+            sl = int(w.page_table[n][(c - 1) // 16]) * 16 + (c - 1) % 16
+            if sl not in where:
+                continue
+            src, i = where[sl]
+            k, v = (w.k_prior, w.v_prior) if src == 0 else (w.k_new, w.v_new)
+            k1[n], v1[n], s1[n] = k[i], v[i], sl
+        return k1, v1, torch.as_tensor(s1)
 
     def write(self, i):
         st = self.L.kv_quant_write(*self.write_args[i % self.N_POOLS])

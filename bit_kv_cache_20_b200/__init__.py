@@ -247,6 +247,37 @@ def paged_decode_append_attn_int4(q: torch.Tensor, k_new: torch.Tensor, v_new: t
     _lib.check(st, "paged_decode_append_attn_int4")
 
 
+def paged_prefill_attn_int4(q: torch.Tensor, cache: torch.Tensor, scales: torch.Tensor,
+                            zeros: torch.Tensor, page_table: torch.Tensor, context_lens: torch.Tensor,
+                            q_start: torch.Tensor, max_q_len: int, out: torch.Tensor, hadamard_block: int,
+                            softmax_scale: float = 0.0, stream=None, hadamard_signs=None) -> None:
+    """Chunked-prefill attention over the INT4 cache (head_dim 128): q, bf16
+    [Tq, Hq, D], holds for sequence n the queries of its last
+    q_start[n + 1] - q_start[n] context tokens (q_start int32 [B + 1]), which
+    the cache already holds; each attends causally to its own position and
+    everything before it. out: fp32 or bf16 [Tq, Hq, D]."""
+    _need(q, "q", torch.bfloat16)
+    _need(page_table, "page_table", torch.int32)
+    _need(context_lens, "context_lens", torch.int32)
+    _need(q_start, "q_start", torch.int32)
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("out must be float32 or bfloat16")
+    _need(out, "out", out.dtype)
+    if tuple(out.shape) != tuple(q.shape) or q.dim() != 3:
+        raise ValueError("q and out must be [Tq, Hq, D]")
+    P, Hkv, D = _pool_shape(cache, scales, zeros)
+    B = int(context_lens.numel())
+    if q_start.numel() != B + 1 or page_table.dim() != 2 or int(page_table.shape[0]) != B:
+        raise ValueError("q_start must hold B + 1 offsets and page_table B rows")
+    desc = AttnDesc(B, int(q.shape[1]), Hkv, D, PAGE_SIZE, P, int(page_table.shape[1]), int(hadamard_block),
+                    float(softmax_scale), 0 if out.dtype == torch.float32 else 1, 0, None,
+                    sign_words(hadamard_signs, D))
+    st = _lib.lib().paged_prefill_attn_int4(
+        _ptr(q), _ptr(cache), _ptr(scales), _ptr(zeros), _ptr(page_table), _ptr(context_lens),
+        _ptr(q_start), int(max_q_len), _ptr(out), ctypes.byref(desc), ctypes.c_void_p(_stream_handle(stream)))
+    _lib.check(st, "paged_prefill_attn_int4")
+
+
 def paged_decode_attn_int4_static_ws(q: torch.Tensor, cache: torch.Tensor, scales: torch.Tensor,
                                      zeros: torch.Tensor, page_table: torch.Tensor,
                                      context_lens: torch.Tensor, out: torch.Tensor,

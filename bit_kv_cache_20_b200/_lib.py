@@ -57,6 +57,10 @@ SIGNATURES = [
                                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                                      ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                                      ctypes.POINTER(AttnDesc), ctypes.c_void_p]),
+    ("paged_prefill_attn_int4", ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_int32, ctypes.c_void_p,
+                                               ctypes.POINTER(AttnDesc), ctypes.c_void_p]),
     ("paged_decode_attn_int4_static_ws", ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p,
                                                         ctypes.c_void_p, ctypes.c_void_p,
                                                         ctypes.c_void_p, ctypes.c_void_p,

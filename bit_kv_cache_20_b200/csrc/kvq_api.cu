@@ -17,6 +17,7 @@
 #include "kvq_decode.cuh"
 #include "kvq_write.cuh"
 #include "kvq_write_tc.cuh"
+#include "kvq_prefill.cuh"
 
 namespace {
 
@@ -558,6 +559,29 @@ kvq_status dispatch_attn(const kvq::AttnParams& p, int b, const SplitPlan& plan,
     default: return KVQ_ERR_UNSUPPORTED;
   }
 }
+// Chunked prefill on the tensor cores (D = 128).
+template <int BLK>
+kvq_status launch_prefill(const kvq::PrefillParams& p, int max_q_len, int dev, cudaStream_t s) {
+  if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
+  auto kern = kvq::kvq_prefill_kernel<128, BLK>;
+  constexpr int smem = kvq::PfSmem<128>::kTotal;
+  static std::atomic<int> ready[kMaxDevices];
+  if (!ready[dev].load(std::memory_order_relaxed)) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
+      cudaGetLastError();
+      return KVQ_ERR_CUDA;
+    }
+    ready[dev].store(1, std::memory_order_relaxed);
+  }
+  const int tq = kvq::kPfRows / p.G;
+  const dim3 grid((unsigned)(((long long)max_q_len + tq - 1) / tq), p.Hkv, p.B);
+  if (launch_pdl(kern, grid, dim3(kvq::kPfThreads), smem, s, p) != cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
+  return KVQ_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -715,6 +739,56 @@ kvq_status paged_decode_append_attn_int4(const void* q, const void* k_new, const
     return KVQ_ERR_INVALID_ARG;
   return decode_impl(q, cache, scales, zeros, page_table, context_lens, out, workspace, workspace_bytes,
                      desc, stream, AppendArgs{k_new, v_new, slot_mapping});
+}
+
+kvq_status paged_prefill_attn_int4(const void* q, const uint8_t* cache, const void* scales,
+                                   const void* zeros, const int32_t* page_table,
+                                   const int32_t* context_lens, const int32_t* q_start, int32_t max_q_len,
+                                   void* out, const kvq_attn_desc* desc, void* stream) {
+  kvq_status st = check_attn_desc(desc);
+  if (st != KVQ_OK) return st;
+  const kvq_attn_desc& d = *desc;
+  if (d.head_dim != 128) return KVQ_ERR_UNSUPPORTED;
+  if (max_q_len < 0) return KVQ_ERR_INVALID_ARG;
+  if (d.batch == 0 || max_q_len == 0) return KVQ_OK;
+  if (!q || !cache || !scales || !zeros || !page_table || !context_lens || !q_start || !out)
+    return KVQ_ERR_INVALID_ARG;
+  if (!aligned(cache, 16) || !aligned(scales, 16) || !aligned(zeros, 16) || !aligned(q, 16) ||
+      !aligned(page_table, 4) || !aligned(context_lens, 4) || !aligned(q_start, 4) ||
+      !aligned(out, d.out_dtype ? 2 : 4))
+    return KVQ_ERR_INVALID_ARG;
+  int dev = 0;
+  st = select_device_of(cache, &dev);
+  if (st != KVQ_OK) return st;
+  kvq::PrefillParams p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.cache = cache;
+  p.scales = static_cast<const uint16_t*>(scales);
+  p.zeros = static_cast<const uint16_t*>(zeros);
+  p.page_table = page_table;
+  p.ctx_lens = context_lens;
+  p.q_start = q_start;
+  p.out = out;
+  p.B = d.batch;
+  p.Hq = d.num_q_heads;
+  p.Hkv = d.num_kv_heads;
+  p.G = d.num_q_heads / d.num_kv_heads;
+  p.num_pages = d.num_pages;
+  p.max_pages = d.max_pages_per_seq;
+  p.out_bf16 = d.out_dtype;
+  const double cb = d.hadamard_block > 0 ? 1.0 / std::sqrt((double)d.hadamard_block) : 1.0;
+  const double scale = d.softmax_scale > 0.0f ? (double)d.softmax_scale : 1.0 / std::sqrt((double)d.head_dim);
+  p.qmul = (float)(cb * scale * 1.4426950408889634);  // log2(e)
+  p.cb = (float)cb;
+  for (int w = 0; w < 4; ++w) p.signs[w] = d.hadamard_signs[w];
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (d.hadamard_block) {
+    case 0: return launch_prefill<0>(p, max_q_len, dev, s);
+    case 32: return launch_prefill<32>(p, max_q_len, dev, s);
+    case 64: return launch_prefill<64>(p, max_q_len, dev, s);
+    case 128: return launch_prefill<128>(p, max_q_len, dev, s);
+    default: return KVQ_ERR_UNSUPPORTED;
+  }
 }
 
 kvq_status kvq_get_device_error(void* stream) {

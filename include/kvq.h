@@ -237,6 +237,39 @@ kvq_status paged_decode_append_attn_int4(const void* q, const void* k_new,
                                          const kvq_attn_desc* desc, void* stream);
 
 /*
+ * paged_prefill_attn_int4 - chunked-prefill attention over the INT4 cache
+ * ([SAW] Abstract: fused attention over the quantized paged cache, for
+ * "high-throughput concurrent workloads"): many queries per sequence, so
+ * QK^T and PV run as dense tcgen05 MMAs.
+ *
+ * Sequence n's chunk is its last L_n = q_start[n+1] - q_start[n] context
+ * tokens, already stored by kv_quant_write; query token i of the chunk (row
+ * q_start[n] + i of q) is position context_lens[n] - L_n + i and attends to
+ * positions 0 .. that position (causal):
+ *   out[row][head] = R^T sum_t p_t v^_t, p = softmax over those positions of
+ *   softmax_scale * (R q[row][head]) . k^_t      (k^, v^ as in paged_decode_attn_int4).
+ *
+ * q            : device, bf16 [Tq][Hq][D], D = 128 (other head sizes return
+ *                KVQ_ERR_UNSUPPORTED), 16-byte aligned.
+ * cache, scales, zeros, page_table, desc : as for paged_decode_attn_int4
+ *                (desc->context_lens_host and desc->flags are not used).
+ * context_lens : device, int32 [B], each >= its chunk length.
+ * q_start      : device, int32 [B + 1], non-decreasing, q_start[0] = 0.
+ * max_q_len    : host, the largest chunk length (sizes the grid).
+ * out          : device, [Tq][Hq][D], fp32 or bf16 (desc->out_dtype).
+ * A context shorter than its chunk or longer than max_pages_per_seq * 16, or a
+ * chunk longer than max_q_len, records KVQ_ERR_OUT_OF_RANGE and leaves that
+ * sequence's rows unwritten.
+ * Returns KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED or KVQ_ERR_CUDA.
+ */
+kvq_status paged_prefill_attn_int4(const void* q, const uint8_t* cache,
+                                   const void* scales, const void* zeros,
+                                   const int32_t* page_table,
+                                   const int32_t* context_lens,
+                                   const int32_t* q_start, int32_t max_q_len,
+                                   void* out, const kvq_attn_desc* desc, void* stream);
+
+/*
  * paged_decode_attn_int4_static_ws - the same decode step as
  * paged_decode_attn_int4, for callers that are not allowed to allocate device
  * memory. Examples: a plug-in hosted by a serving runtime that owns all GPU

@@ -48,7 +48,7 @@ def parse_args(argv=None):
     ap.add_argument("--no-plain", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="time direct launches instead of CUDA graph replays (for profilers)")
-    ap.add_argument("--only", choices=["write", "decode"], default=None,
+    ap.add_argument("--only", choices=["write", "decode", "prefill"], default=None,
                     help="time one kernel alone (profiling captures); prints its line")
     ap.add_argument("--e2e-steps", type=int, default=100)
     return ap.parse_args(argv)
@@ -85,6 +85,7 @@ def aggregate_gbs(bytes_per_step, steps, world, max_ms):
 KERNEL_SOURCES = {
     "kv_quant_write": ["kvq_write_tc.cuh", "kvq_write.cuh", "kvq_device.cuh"],
     "paged_decode_attn_int4": ["kvq_decode.cuh", "kvq_device.cuh"],
+    "paged_prefill_attn_int4": ["kvq_prefill.cuh", "kvq_decode.cuh", "kvq_write_tc.cuh", "kvq_device.cuh"],
 }
 
 
@@ -114,13 +115,85 @@ def committed_traffic(kernel):
     return entry.get("dram_bytes_per_launch")
 
 
-def measured_peaks():
+def measured_peaks(key="hbm_gbs"):
+    """(peak, "measured" | "fallback"): HBM GB/s, or with key="bf16_tflops"
+    the dense bf16 tensor TFLOP/s (burst: the kernels it is used for are
+    timed alone)."""
     try:
         with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
             p = json.load(f)
-        return float(p["hbm_gbs"]), "measured"
+        return float(p[key]), "measured"
     except (OSError, ValueError, KeyError):
-        return 6650.0, "fallback"
+        return (6650.0 if key == "hbm_gbs" else 1590.0), "fallback"
+
+
+# chunked prefill: every sequence's last PREFILL_CHUNK context tokens (all of
+# it when shorter) are one chunk of queries over the cache that holds them
+PREFILL_CHUNK = 2048
+
+
+def prefill_flops(context_lens, chunk, Hq, D):
+    """Algorithmic FLOPs of a causal chunked prefill: query token i of a chunk
+    of L at context c attends to c - L + i + 1 positions, and each (query
+    head, position) pair costs 2D for q.k and 2D for p.v."""
+    pairs = 0
+    for c in context_lens:
+        c = int(c)
+        L = min(chunk, c)
+        pairs += L * (c - L) + L * (L + 1) // 2
+    return 4 * D * Hq * pairs
+
+
+def prefill_run(step, launches, warm):
+    """paged_prefill_attn_int4 over the cache of pool 0: each launch preceded
+    by an L2 flush (a 256 MB write), timed alone with CUDA events on the
+    launching stream. Returns (mean ms per launch, FLOPs per launch)."""
+    import numpy as np
+    import torch
+    kvq, w, dev = step.kvq, step.w, step.dev
+    lens = np.minimum(np.asarray(w.context_lens, np.int64), PREFILL_CHUNK)
+    q_start = np.concatenate([[0], np.cumsum(lens)]).astype(np.int32)
+    g = torch.Generator().manual_seed(w.cfg.seed + 7)
+    q = (torch.randn((int(q_start[-1]), w.Hq, w.D), generator=g) / 8).to(torch.bfloat16).to(dev)
+    out = torch.empty(q.shape, dtype=torch.bfloat16, device=dev)
+    qs = torch.as_tensor(q_start).to(dev)
+    c, s, z = step.pools[0]
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    max_q = int(lens.max())
+
+    def launch():
+        kvq.paged_prefill_attn_int4(q, c, s, z, step.pt, step.ctx, qs, max_q, out, step.b, stream=step.stream)
+
+    total = 0.0
+    with torch.cuda.stream(step.stream):
+        for k in range(warm + launches):
+            flush.zero_()
+            e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            e0.record(step.stream)
+            launch()
+            e1.record(step.stream)
+            e1.synchronize()
+            if k >= warm:
+                total += e0.elapsed_time(e1)
+    if kvq.get_device_error(step.stream) != 0:
+        raise RuntimeError("paged_prefill_attn_int4 recorded a device error")
+    return total / launches, prefill_flops(w.context_lens, PREFILL_CHUNK, w.Hq, w.D)
+
+
+def prefill_line(ms, flops):
+    peak, src = measured_peaks("bf16_tflops")
+    tf = flops / (ms / 1e3) / 1e12
+    return {
+        "what": f"chunked prefill: each sequence's last {PREFILL_CHUNK} context tokens (all when shorter) "
+                "as queries, causal, over the INT4 cache; L2 flushed before each launch",
+        "us": round(1e3 * ms, 1), "TFLOP/s": round(tf, 2),
+        "roofline": {"kernel": "paged_prefill_attn_int4", "bound": "tensor", "achieved": round(tf, 2),
+                     "peak": peak, "unit": "TFLOP/s", "frac": round(tf / peak, 4),
+                     "traffic": committed_traffic("paged_prefill_attn_int4"),
+                     "algorithmic_flops": flops,
+                     "peak_source": "measured (MEASURED_PEAKS.json bf16_tflops, burst)" if src == "measured"
+                     else "fallback 1.59 PFLOP/s"},
+    }
 
 
 # ----------------------------------------------------------------------------
@@ -565,6 +638,15 @@ def main(argv=None):
 
     step = Step(w, block, dev, graph=not args.no_graph)
     step.fill_pools()
+    if args.only == "prefill":
+        ms_pf, fl = prefill_run(step, args.steps, warm)
+        ms_pf = max_over_ranks(ms_pf)
+        if rank == 0:
+            print(json.dumps({"only": "prefill", **prefill_line(ms_pf, fl * world), "launches": args.steps,
+                              "config": config_block(w, block, not args.no_graph)}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
     if args.only:
         step.timed_only(args.only, warm)
         barrier()
@@ -638,6 +720,10 @@ def main(argv=None):
         }
         del p
 
+    # chunked prefill (a row beside the step, not part of it): a few launches
+    pf_ms, pf_flops = prefill_run(step, 3, 1)
+    pf_ms = max_over_ranks(pf_ms)
+
     e2e = None
     if not args.no_e2e:
         e_steps = max(1, min(args.steps, args.e2e_steps))
@@ -685,6 +771,7 @@ def main(argv=None):
             "separate_us": round(1e3 * ap_sep_ms, 3),  # kv_quant_write (B tokens) + paged_decode_attn_int4
             "fused_us": round(1e3 * ap_fus_ms, 3),     # paged_decode_append_attn_int4
         },
+        "prefill": prefill_line(pf_ms, pf_flops * world),
         "e2e": e2e,
         "clocks": clocks.summary(),
         "gpu_launches": 2 * args.steps,

@@ -10,9 +10,12 @@
 // ctx - 1), already written to the cache by kv_quant_write; query token i of
 // the chunk attends causally to positions 0 .. ctx - qlen + i.
 //
-// One CTA (4 warps) per (tile of 128 / G chunk tokens x the G query heads of
+// One CTA (8 warps) per (tile of 128 / G chunk tokens x the G query heads of
 // one kv head, kv head, sequence): 128 query rows = the MMA's M, row
-// r = token (r / G) x head (r % G), one thread (= tensor-memory lane) per row.
+// r = token (r / G) x head (r % G) = tensor-memory lane r. Two threads share a
+// row: warps w and w + 4 (the lane quarter w mod 4 is all that a warp may
+// read of tensor memory), each with half of the row's logits and of its
+// output columns; they meet once per block to agree on the running maximum.
 // The cache is read in blocks of 64 tokens (4 pages), up to the tile's last
 // position:
 //   - 16-byte cp.async copies of the block's codes, scales and zeros into a
@@ -66,7 +69,7 @@ struct PrefillParams {
   uint32_t signs[4];          // randomized Hadamard signs, as written
 };
 
-constexpr int kPfThreads = 128;
+constexpr int kPfThreads = 256;  // two threads per query row
 constexpr int kPfRows = 128;   // query rows per CTA (MMA M)
 constexpr int kPfBlock = 64;   // cache tokens per block (N of S, K of PV)
 constexpr int kPfTmemCols = 512;  // S [0, 64), O_blk [64, 192), O [192, 320)
@@ -84,7 +87,8 @@ struct PfSmem {
   static constexpr int kStage = kPlo + kPfRows * kPfBlock * 2;
   static constexpr int kSz = kStage + 2 * kStageBytes;       // float [4][64]: s_k, z_k, s_v, z_v
   static constexpr int kPageOk = kSz + 4 * kPfBlock * 4;     // int [4]
-  static constexpr int kQsum = kPageOk + 16;                 // float [128]
+  static constexpr int kXch = kPageOk + 16;                  // float [2][128]: the two halves' block maxima
+  static constexpr int kQsum = kXch + 2 * kPfRows * 4;       // float [128]
   static constexpr int kQinv = kQsum + kPfRows * 4;          // float [128]: 2^-e of each row
   static constexpr int kBar = kQinv + kPfRows * 4;           // 2 mbarriers
   static constexpr int kTmem = kBar + 16;
@@ -129,6 +133,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
   int* page_ok = reinterpret_cast<int*>(smem + S::kPageOk);
   float* qsum = reinterpret_cast<float*>(smem + S::kQsum);
   float* qinv = reinterpret_cast<float*>(smem + S::kQinv);
+  float* xch = reinterpret_cast<float*>(smem + S::kXch);
   const uint32_t bar_s = sb + S::kBar, bar_pv = bar_s + 8;
   uint32_t* tslot = reinterpret_cast<uint32_t*>(smem + S::kTmem);
 
@@ -162,8 +167,11 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tslot;
-  const uint32_t lane_base = (uint32_t)(32 * warp) << 16;
-  const uint32_t tS = tmem + lane_base, tOb = tmem + lane_base + kPfBlock, tO = tOb + D;
+  const int quarter = warp & 3, half = warp >> 2;  // tensor-memory lanes; half of the row
+  const uint32_t lane_base = (uint32_t)(32 * quarter) << 16;
+  // this thread's columns: S [32 half, +32), O_blk and O [D/2 half, +D/2)
+  const uint32_t tS = tmem + lane_base + 32 * half;
+  const uint32_t tOb = tmem + lane_base + kPfBlock + (D / 2) * half, tO = tOb + D;
 
   // ---- block fetch: 4 pages of kv head h into staging buffer b & 1 --------
   const int32_t* pt_row = p.page_table + (size_t)n * p.max_pages;
@@ -186,7 +194,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
   fetch(0);
 
   // ---- q~ = R q * (softmax_scale * log2 e) as fp16 hi + lo, sum(q~) per row -
-  for (int r = warp; r < kPfRows; r += 4) {
+  for (int r = warp; r < kPfRows; r += kPfThreads / 32) {
     const int i = r / G, j = r % G;
     float v[E];
     if (i < ntok) {
@@ -236,7 +244,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
   }
 
   // this thread's row (= tensor-memory lane)
-  const int row = tid, ri = row / G;
+  const int row = 32 * quarter + lane, ri = row / G;
   const bool row_ok = ri < ntok;
   const int pos_r = pos0 + ri;  // the last position this row attends to
   float m_used = -INFINITY, l_sum = 0.0f, zs = 0.0f;
@@ -245,7 +253,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
   // tensor-memory loads and stores; `first`: O := O_blk)
   auto fold = [&](bool first, float alpha) {
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
+    for (int c0 = 0; c0 < D / 2; c0 += 32) {
       float ob[32];
       tmem_ld32(tOb + c0, ob);
       if (!first) {
@@ -343,38 +351,48 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
     mbar_wait_bounded(bar_s, b & 1);
     tc_fence_after();
 
-    // ---- online softmax over this row's 64 logits ----------------------------
-    float sv[64];
-    {
-      float a[32], c[32];
-      tmem_ld32(tS, a);
-      tmem_ld32(tS + 32, c);
+    // ---- online softmax: this thread's 32 of the row's 64 logits ------------
+    constexpr int kH = kPfBlock / 2;
+    const int t0 = kH * half;  // first token of this thread's half
+    float sv[kH];
+    tmem_ld32(tS, sv);
+    const float qs = qsum[row], qi = qinv[row];
+    // every row sees the whole block, every page is valid: no masks
+    const bool open = kPfBlock * b + kPfBlock - 1 <= pos0 &&
+                      (page_ok[0] & page_ok[1] & page_ok[2] & page_ok[3]) != 0;
+    float mb = -INFINITY;
+    if (open) {
 #pragma unroll
-      for (int k = 0; k < 32; ++k) {
-        sv[k] = a[k];
-        sv[32 + k] = c[k];
+      for (int t = 0; t < kH; ++t) {
+        sv[t] = fmaf(sv[t] * qi, sz[t0 + t], sz[kPfBlock + t0 + t] * qs);
+        mb = fmaxf(mb, sv[t]);
+      }
+    } else {
+#pragma unroll
+      for (int t = 0; t < kH; ++t) {
+        const int pos = kPfBlock * b + t0 + t;
+        const bool live = row_ok && pos <= pos_r && page_ok[(t0 + t) >> 4];
+        const float lg = fmaf(sv[t] * qi, sz[t0 + t], sz[kPfBlock + t0 + t] * qs);
+        sv[t] = live ? lg : -INFINITY;
+        mb = fmaxf(mb, sv[t]);
       }
     }
-    const float qs = qsum[row], qi = qinv[row];
-    float mb = -INFINITY;
-#pragma unroll
-    for (int t = 0; t < kPfBlock; ++t) {
-      const int pos = kPfBlock * b + t;
-      const bool live = row_ok && pos <= pos_r && page_ok[t >> 4];
-      const float lg = fmaf(sv[t] * qi, sz[t], sz[kPfBlock + t] * qs);
-      sv[t] = live ? lg : -INFINITY;
-      mb = fmaxf(mb, sv[t]);
-    }
+    // the row's block maximum: the two halves meet (warps quarter and
+    // quarter + 4, 64 threads, named barrier 1 + quarter)
+    xch[half * kPfRows + row] = mb;
+    named_bar_sync(1 + quarter, 64);
+    mb = fmaxf(mb, xch[(half ^ 1) * kPfRows + row]);
     // online softmax: the running maximum, and the factor for what came before
+    // (both halves compute the same values)
     const float m_new = fmaxf(m_used, mb);
     const float alpha = (m_new == -INFINITY || m_used == -INFINITY) ? 0.0f : fast_exp2(m_used - m_new);
     l_sum *= alpha;
     zs *= alpha;
     alpha_prev = alpha;
     m_used = m_new;
-    // p and P' = p s_v as fp16 hi + lo, row `row` of the A operands
+    // p and P' = p * s_v as bf16 hi + lo, this half of row `row` of the A operands
 #pragma unroll
-    for (int t8 = 0; t8 < kPfBlock; t8 += 8) {
+    for (int t8 = 0; t8 < kH; t8 += 8) {
       uint32_t hw[4], lw[4];
 #pragma unroll
       for (int k = 0; k < 8; k += 2) {
@@ -382,13 +400,13 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
         const float p0 = (sv[t] == -INFINITY) ? 0.0f : fast_exp2(sv[t] - m_used);
         const float p1 = (sv[t + 1] == -INFINITY) ? 0.0f : fast_exp2(sv[t + 1] - m_used);
         l_sum += p0 + p1;
-        zs = fmaf(p0, sz[3 * kPfBlock + t], fmaf(p1, sz[3 * kPfBlock + t + 1], zs));
-        const float P0 = p0 * sz[2 * kPfBlock + t], P1 = p1 * sz[2 * kPfBlock + t + 1];
+        zs = fmaf(p0, sz[3 * kPfBlock + t0 + t], fmaf(p1, sz[3 * kPfBlock + t0 + t + 1], zs));
+        const float P0 = p0 * sz[2 * kPfBlock + t0 + t], P1 = p1 * sz[2 * kPfBlock + t0 + t + 1];
         hw[k / 2] = hilo_pair_bf16(P0, P1, false);
         lw[k / 2] = hilo_pair_bf16(P0, P1, true);
       }
-      *reinterpret_cast<uint4*>(smem + S::kPhi + sw128_offset(row, t8, kPfRows)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
-      *reinterpret_cast<uint4*>(smem + S::kPlo + sw128_offset(row, t8, kPfRows)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+      *reinterpret_cast<uint4*>(smem + S::kPhi + sw128_offset(row, t0 + t8, kPfRows)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
+      *reinterpret_cast<uint4*>(smem + S::kPlo + sw128_offset(row, t0 + t8, kPfRows)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
     }
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
     tc_fence_before();
@@ -412,22 +430,32 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
   fold(n_blocks == 1, alpha_prev);
 
   // ---- epilogue: o~ = (O + Z) / L, then R^T per row --------------------------
+  // the halves' sums of p and p z: each thread adds its partner's
+  xch[half * kPfRows + row] = l_sum;
+  named_bar_sync(1 + quarter, 64);
+  const float l_all = l_sum + xch[(half ^ 1) * kPfRows + row];
+  named_bar_sync(1 + quarter, 64);
+  xch[half * kPfRows + row] = zs;
+  named_bar_sync(1 + quarter, 64);
+  const float z_all = zs + xch[(half ^ 1) * kPfRows + row];
   float* orow = reinterpret_cast<float*>(smem + S::kQhi);  // [128][D] fp32 over the Q tiles
   {
-    const float inv = (l_sum > 0.0f) ? 1.0f / l_sum : 0.0f;
+    const float inv = (l_all > 0.0f) ? 1.0f / l_all : 0.0f;
 #pragma unroll
-    for (int c0 = 0; c0 < D; c0 += 32) {
+    for (int c0 = 0; c0 < D / 2; c0 += 32) {
       float o[32];
       tmem_ld32(tO + c0, o);
+      const int cb = (D / 2) * half + c0;  // column of o[0]
 #pragma unroll
       for (int k = 0; k < 32; k += 4)
-        *reinterpret_cast<float4*>(orow + row * D + ((c0 + k + 4 * row) & (D - 1))) =
-            make_float4((o[k] + zs) * inv, (o[k + 1] + zs) * inv, (o[k + 2] + zs) * inv, (o[k + 3] + zs) * inv);
+        *reinterpret_cast<float4*>(orow + row * D + ((cb + k + 4 * row) & (D - 1))) =
+            make_float4((o[k] + z_all) * inv, (o[k + 1] + z_all) * inv, (o[k + 2] + z_all) * inv,
+                        (o[k + 3] + z_all) * inv);
     }
   }
   tc_fence_before();
   __syncthreads();
-  for (int r = warp; r < kPfRows; r += 4) {
+  for (int r = warp; r < kPfRows; r += kPfThreads / 32) {
     const int i = r / G, j = r % G;
     if (i >= ntok) continue;
     float v[E];

@@ -56,3 +56,15 @@ def test_reference_arm_on_a_non_zero_rank_exits_without_work(monkeypatch, capsys
     monkeypatch.setenv("WORLD_SIZE", "2")
     assert bench.main(["--impl", "reference", "--steps", "1", "--warmup", "0"]) == 0
     assert capsys.readouterr().out == ""
+
+
+def test_prefill_flops_counts_every_causal_pair():
+    # brute force: query i of a chunk of L at context c sees positions 0 .. c - L + i
+    import bench
+    for ctx, chunk in (([1, 5, 40], 16), ([3000, 70, 2048], 2048), ([0, 9], 4)):
+        pairs = 0
+        for c in ctx:
+            L = min(chunk, c)
+            for i in range(L):
+                pairs += sum(1 for pos in range(c) if pos <= c - L + i)
+        assert bench.prefill_flops(ctx, chunk, Hq=3, D=8) == 4 * 8 * 3 * pairs

@@ -175,15 +175,29 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
 
   // ---- block fetch: 4 pages of kv head h into staging buffer b & 1 --------
   const int32_t* pt_row = p.page_table + (size_t)n * p.max_pages;
+  // The page ids a block needs are read from the page table one block ahead
+  // (into registers), so that no fetch waits for that load: pid[k] for this
+  // thread's k-th 16-byte chunk of the next fetch, sid for the scales and
+  // zeros of token tid (tid < 64).
+  constexpr int kChunks = D + 8;  // 16-byte chunks per page: codes, then scales, zeros
+  constexpr int kPerThread = (4 * kChunks + kPfThreads - 1) / kPfThreads;
+  auto page_id = [&](int lp) { return (lp * 16 < ctx) ? pt_row[lp] : -1; };
+  int pid[kPerThread];
+  auto load_ids = [&](int b) {
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k) {
+      const int i = tid + k * kPfThreads;
+      pid[k] = (i < 4 * kChunks) ? page_id(4 * b + i / kChunks) : -1;
+    }
+  };
   auto fetch = [&](int b) {
     uint8_t* st = smem + S::kStage + (b & 1) * S::kStageBytes;
-    constexpr int kChunks = D + 8;  // 16-byte chunks per page: codes, then scales, zeros
-    for (int i = tid; i < 4 * kChunks; i += kPfThreads) {
+#pragma unroll
+    for (int k = 0; k < kPerThread; ++k) {
+      const int i = tid + k * kPfThreads;
+      const int id = pid[k];
+      if (i >= 4 * kChunks || id < 0 || id >= p.num_pages) continue;
       const int pg = i / kChunks, c = i % kChunks;
-      const int lp = 4 * b + pg;
-      if (lp * 16 >= ctx) continue;
-      const int id = pt_row[lp];
-      if (id < 0 || id >= p.num_pages) continue;
       const size_t head = (size_t)id * p.Hkv + h;
       const void* src = (c < D) ? static_cast<const void*>(p.cache + head * (16 * D) + 16 * c)
                                 : static_cast<const void*>((c < D + 4 ? p.scales : p.zeros) + head * 32 + 8 * ((c - D) & 3));
@@ -191,7 +205,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
     }
     cp_async_commit();
   };
+  load_ids(0);
   fetch(0);
+  if (n_blocks > 1) load_ids(1);
+  int sid = (tid < kPfBlock) ? page_id(tid >> 4) : -1;  // block 0
 
   // ---- q~ = R q * (softmax_scale * log2 e) as fp16 hi + lo, sum(q~) per row -
   for (int r = warp; r < kPfRows; r += kPfThreads / 32) {
@@ -267,7 +284,10 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
   };
 
   for (int b = 0; b < n_blocks; ++b) {
-    if (b + 1 < n_blocks) fetch(b + 1);
+    if (b + 1 < n_blocks) {
+      fetch(b + 1);
+      if (b + 2 < n_blocks) load_ids(b + 2);
+    }
     else cp_async_commit();
     cp_async_wait<1>();  // block b has landed (this thread's copies)
     // the previous PV MMA read the K, V and P' tiles and wrote O_blk: done
@@ -317,7 +337,8 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
     }
     if (tid < kPfBlock) {  // token tid of the block
       const int t = tid, pg = t >> 4, lp = 4 * b + pg;
-      const int id = (lp * 16 < ctx) ? pt_row[lp] : -1;
+      const int id = sid;
+      if (b + 1 < n_blocks) sid = page_id(lp + 4);  // the next block's, read ahead
       const bool ok = id >= 0 && id < p.num_pages;
       if (!ok && lp * 16 < ctx && (t & 15) == 0) record_error(KVQ_ERR_OUT_OF_RANGE);
       const __half* scl = reinterpret_cast<const __half*>(st + pg * S::kSlot + 16 * D);

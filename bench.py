@@ -529,13 +529,24 @@ def oracle_sample(w, block, n_tokens):
     return dt, nbytes
 
 
-def cpu_baseline(w, block, n_tokens=16384):
+def cpu_baseline(w, block, n_tokens=32768, min_seconds=10.0, max_passes=20):
+    """The oracle on a bounded sample of the workload, repeated until it has
+    run for `min_seconds` (at most `max_passes` passes)."""
     import oracle
-    dt, nbytes = oracle_sample(w, block, n_tokens)
-    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
+    passes, total_t, total_b = 0, 0.0, 0
+    while passes < max_passes and total_t < min_seconds:
+        dt, nbytes = oracle_sample(w, block, n_tokens)
+        passes += 1
+        total_t += dt
+        total_b += nbytes
+    return {"value": round(total_b / total_t / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
             "kind": "oracle",
-            "sample": f"write of the first {min(n_tokens, w.tokens_written)} tokens (all kv heads, K and V) "
-                      f"+ one decode step of all {w.Hq} query heads over them; {dt:.2f} s"}
+            "sample": f"{passes} passes of: write of the first {min(n_tokens, w.tokens_written)} tokens "
+                      f"(all kv heads, K and V) + one decode step of all {w.Hq} query heads over them; "
+                      f"{total_t:.1f} s in all"}
+
+
+REFERENCE_BUDGET_S = 120.0
 
 
 def run_reference(args):
@@ -544,8 +555,12 @@ def run_reference(args):
     from bit_kv_cache_20_b200 import workloads
     w = workloads.make(args.config, block=args.block)
     block = w.block
-    n_tokens = 4096
     warm = max(args.warmup, 0)
+    # each step's sample is sized so that the whole run takes about
+    # REFERENCE_BUDGET_S: 256 .. 4096 tokens, from a timed 1024-token sample
+    dt_cal, _ = oracle_sample(w, block, 1024)
+    per_step = REFERENCE_BUDGET_S / (max(args.steps, 1) + warm)
+    n_tokens = max(256, min(4096, int(per_step / (dt_cal / 1024)) // 256 * 256))
     for _ in range(warm):
         oracle_sample(w, block, n_tokens)
     total_t, total_b = 0.0, 0

@@ -118,6 +118,50 @@ def test_decode_argument_errors(L):
     assert L.kvq_attn_workspace_size(ctypes.byref(d(head_dim=96))) == size_max
 
 
+def _desc(**kw):
+    from bit_kv_cache_20_b200._lib import AttnDesc
+    a = dict(batch=2, num_q_heads=8, num_kv_heads=2, head_dim=128, page_size=16, num_pages=10,
+             max_pages_per_seq=5, hadamard_block=128, softmax_scale=0.0, out_dtype=0, flags=0,
+             context_lens_host=None, hadamard_signs=(ctypes.c_uint32 * 4)(0, 0, 0, 0))
+    a.update(kw)
+    return AttnDesc(*a.values())
+
+
+def append_call(L, desc, k=FAKE, v=FAKE, slots=FAKE):
+    P = ctypes.c_void_p
+    return L.paged_decode_append_attn_int4(P(FAKE), P(k), P(v), P(slots), P(FAKE), P(FAKE), P(FAKE),
+                                           P(FAKE), P(FAKE), P(FAKE), None, 0,
+                                           ctypes.byref(desc) if desc is not None else None, None)
+
+
+def test_append_argument_errors(L):
+    assert append_call(L, None) == 1
+    assert append_call(L, _desc(), k=0) == 1                        # no new K
+    assert append_call(L, _desc(), v=FAKE + 8) == 1                 # misaligned V
+    assert append_call(L, _desc(), slots=FAKE + 4) == 1             # misaligned slot_mapping
+    assert append_call(L, _desc(head_dim=96)) == 2                  # as the decode
+    assert append_call(L, _desc(batch=0), k=0, v=0, slots=0) == 0   # nothing to do
+
+
+def prefill_call(L, desc, max_q=64, q=FAKE, q_start=FAKE, out=FAKE):
+    P = ctypes.c_void_p
+    return L.paged_prefill_attn_int4(P(q), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(FAKE), P(q_start), max_q,
+                                     P(out), ctypes.byref(desc) if desc is not None else None, None)
+
+
+def test_prefill_argument_errors(L):
+    assert prefill_call(L, None) == 1
+    assert prefill_call(L, _desc(head_dim=64, hadamard_block=64)) == 2   # prefill instances: D = 128
+    assert prefill_call(L, _desc(num_q_heads=32, num_kv_heads=2)) == 2   # GQA group 16
+    assert prefill_call(L, _desc(hadamard_block=48)) == 2
+    assert prefill_call(L, _desc(), max_q=-1) == 1
+    assert prefill_call(L, _desc(), q_start=0) == 1                      # null
+    assert prefill_call(L, _desc(), q=FAKE + 8) == 1                     # misaligned q
+    assert prefill_call(L, _desc(out_dtype=1), out=FAKE + 1) == 1        # misaligned bf16 out
+    assert prefill_call(L, _desc(batch=0)) == 0                          # nothing to do
+    assert prefill_call(L, _desc(), max_q=0) == 0
+
+
 def test_binding_fails_loudly_without_the_library(tmp_path, monkeypatch):
     from bit_kv_cache_20_b200 import _lib
     monkeypatch.setattr(_lib, "LIB_PATH", str(tmp_path / "missing.so"))

@@ -559,12 +559,12 @@ kvq_status dispatch_attn(const kvq::AttnParams& p, int b, const SplitPlan& plan,
     default: return KVQ_ERR_UNSUPPORTED;
   }
 }
-// Chunked prefill on the tensor cores (D = 128).
-template <int BLK>
+// Chunked prefill on the tensor cores (D = 64, 128).
+template <int D, int BLK>
 kvq_status launch_prefill(const kvq::PrefillParams& p, int max_q_len, int dev, cudaStream_t s) {
   if (dev < 0 || dev >= kMaxDevices) return KVQ_ERR_UNSUPPORTED;
-  auto kern = kvq::kvq_prefill_kernel<128, BLK>;
-  constexpr int smem = kvq::PfSmem<128>::kTotal;
+  auto kern = kvq::kvq_prefill_kernel<D, BLK>;
+  constexpr int smem = kvq::PfSmem<D>::kTotal;
   static std::atomic<int> ready[kMaxDevices];
   if (!ready[dev].load(std::memory_order_relaxed)) {
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess) {
@@ -748,7 +748,6 @@ kvq_status paged_prefill_attn_int4(const void* q, const uint8_t* cache, const vo
   kvq_status st = check_attn_desc(desc);
   if (st != KVQ_OK) return st;
   const kvq_attn_desc& d = *desc;
-  if (d.head_dim != 128) return KVQ_ERR_UNSUPPORTED;
   if (max_q_len < 0) return KVQ_ERR_INVALID_ARG;
   if (d.batch == 0 || max_q_len == 0) return KVQ_OK;
   if (!q || !cache || !scales || !zeros || !page_table || !context_lens || !q_start || !out)
@@ -783,10 +782,13 @@ kvq_status paged_prefill_attn_int4(const void* q, const uint8_t* cache, const vo
   for (int w = 0; w < 4; ++w) p.signs[w] = d.hadamard_signs[w];
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (d.hadamard_block) {
-    case 0: return launch_prefill<0>(p, max_q_len, dev, s);
-    case 32: return launch_prefill<32>(p, max_q_len, dev, s);
-    case 64: return launch_prefill<64>(p, max_q_len, dev, s);
-    case 128: return launch_prefill<128>(p, max_q_len, dev, s);
+    case 0: return d.head_dim == 64 ? launch_prefill<64, 0>(p, max_q_len, dev, s)
+                                    : launch_prefill<128, 0>(p, max_q_len, dev, s);
+    case 32: return d.head_dim == 64 ? launch_prefill<64, 32>(p, max_q_len, dev, s)
+                                     : launch_prefill<128, 32>(p, max_q_len, dev, s);
+    case 64: return d.head_dim == 64 ? launch_prefill<64, 64>(p, max_q_len, dev, s)
+                                     : launch_prefill<128, 64>(p, max_q_len, dev, s);
+    case 128: return launch_prefill<128, 128>(p, max_q_len, dev, s);
     default: return KVQ_ERR_UNSUPPORTED;
   }
 }

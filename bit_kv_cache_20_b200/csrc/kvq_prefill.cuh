@@ -72,7 +72,9 @@ struct PrefillParams {
 constexpr int kPfThreads = 256;  // two threads per query row
 constexpr int kPfRows = 128;   // query rows per CTA (MMA M)
 constexpr int kPfBlock = 64;   // cache tokens per block (N of S, K of PV)
-constexpr int kPfTmemCols = 512;  // S [0, 64), O_blk [64, 192), O [192, 320)
+// tensor-memory columns: S [0, 64), O_blk [64, 64 + D), O [64 + D, 64 + 2D),
+// rounded up to a power of two
+__host__ __device__ constexpr uint32_t pf_tmem_cols(int d) { return 64 + 2 * d <= 256 ? 256 : 512; }
 
 template <int D>
 struct PfSmem {
@@ -119,7 +121,7 @@ __device__ __forceinline__ uint32_t byte_to_half2(uint32_t w, uint32_t w4, uint3
 
 template <int D, int BLK>
 __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid_constant__ PrefillParams p) {
-  static_assert(D == 128, "prefill instances exist for D = 128");
+  static_assert(D == 64 || D == 128, "prefill instances exist for D = 64 and 128");
   using S = PfSmem<D>;
   constexpr int E = D / 32;
   constexpr uint32_t kIdescS = (1u << 4) | ((uint32_t)(kPfBlock >> 3) << 17) | ((uint32_t)(kPfRows >> 4) << 24);
@@ -162,7 +164,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
     mbar_init(bar_pv, 1);
     mbar_init_fence();
   }
-  if (warp == 0) tmem_alloc(smem_addr(tslot), kPfTmemCols);
+  if (warp == 0) tmem_alloc(smem_addr(tslot), pf_tmem_cols(D));
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -256,8 +258,14 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
       lo2[e / 2] = hilo_pair(v[e] * up, v[e + 1] * up, true);
     }
     // E = 4 consecutive elements = 8 bytes of one 16-byte swizzle unit
-    *reinterpret_cast<uint2*>(smem + S::kQhi + sw128_offset(r, E * lane, kPfRows)) = make_uint2(hi2[0], hi2[1]);
-    *reinterpret_cast<uint2*>(smem + S::kQlo + sw128_offset(r, E * lane, kPfRows)) = make_uint2(lo2[0], lo2[1]);
+    // E consecutive elements = 2E bytes of one 16-byte swizzle unit
+    if constexpr (E == 4) {
+      *reinterpret_cast<uint2*>(smem + S::kQhi + sw128_offset(r, E * lane, kPfRows)) = make_uint2(hi2[0], hi2[1]);
+      *reinterpret_cast<uint2*>(smem + S::kQlo + sw128_offset(r, E * lane, kPfRows)) = make_uint2(lo2[0], lo2[1]);
+    } else {
+      *reinterpret_cast<uint32_t*>(smem + S::kQhi + sw128_offset(r, E * lane, kPfRows)) = hi2[0];
+      *reinterpret_cast<uint32_t*>(smem + S::kQlo + sw128_offset(r, E * lane, kPfRows)) = lo2[0];
+    }
   }
 
   // this thread's row (= tensor-memory lane)
@@ -499,7 +507,7 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  if (warp == 0) tmem_dealloc(tmem, kPfTmemCols);
+  if (warp == 0) tmem_dealloc(tmem, pf_tmem_cols(D));
 }
 
 }  // namespace kvq

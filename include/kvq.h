@@ -249,8 +249,8 @@ kvq_status paged_decode_append_attn_int4(const void* q, const void* k_new,
  *   out[row][head] = R^T sum_t p_t v^_t, p = softmax over those positions of
  *   softmax_scale * (R q[row][head]) . k^_t      (k^, v^ as in paged_decode_attn_int4).
  *
- * q            : device, bf16 [Tq][Hq][D], D = 128 (other head sizes return
- *                KVQ_ERR_UNSUPPORTED), 16-byte aligned.
+ * q            : device, bf16 [Tq][Hq][D], D = 64 or 128 (as for the decode),
+ *                16-byte aligned.
  * cache, scales, zeros, page_table, desc : as for paged_decode_attn_int4
  *                (desc->context_lens_host and desc->flags are not used).
  * context_lens : device, int32 [B], each >= its chunk length.

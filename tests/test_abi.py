@@ -151,7 +151,7 @@ def prefill_call(L, desc, max_q=64, q=FAKE, q_start=FAKE, out=FAKE):
 
 def test_prefill_argument_errors(L):
     assert prefill_call(L, None) == 1
-    assert prefill_call(L, _desc(head_dim=64, hadamard_block=64)) == 2   # prefill instances: D = 128
+    assert prefill_call(L, _desc(head_dim=96)) == 2                      # as the decode
     assert prefill_call(L, _desc(num_q_heads=32, num_kv_heads=2)) == 2   # GQA group 16
     assert prefill_call(L, _desc(hadamard_block=48)) == 2
     assert prefill_call(L, _desc(), max_q=-1) == 1

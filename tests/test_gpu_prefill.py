@@ -13,14 +13,14 @@ from test_gpu_decode import assert_close, host_cache
 pytestmark = pytest.mark.gpu
 
 
-def _case(seed, ctx, qlen, Hq, Hkv, b, signs=None):
-    w = workloads.random_case(seed=seed, B=len(ctx), Hq=Hq, Hkv=Hkv, D=128, block=b, context_lens=ctx)
+def _case(seed, ctx, qlen, Hq, Hkv, b, signs=None, D=128):
+    w = workloads.random_case(seed=seed, B=len(ctx), Hq=Hq, Hkv=Hkv, D=D, block=b, context_lens=ctx)
     cache, scales, zeros = kvq.alloc_cache(w.num_pages, w.Hkv, w.D)
     kvq.kv_quant_write(w.k_new.cuda(), w.v_new.cuda(), torch.as_tensor(w.slots_new).cuda(), cache, scales,
                        zeros, b, hadamard_signs=signs)
     g = torch.Generator().manual_seed(seed + 1)
     qstart = np.concatenate([[0], np.cumsum(qlen)]).astype(np.int32)
-    q = (torch.randn((int(qstart[-1]), Hq, 128), generator=g) / 8).to(torch.bfloat16)
+    q = (torch.randn((int(qstart[-1]), Hq, D), generator=g) / 8).to(torch.bfloat16)
     out = torch.full(q.shape, 7.0, dtype=torch.float32, device="cuda")
     kvq.paged_prefill_attn_int4(q.cuda(), cache, scales, zeros, torch.as_tensor(w.page_table).cuda(),
                                 torch.as_tensor(w.context_lens).cuda(), torch.as_tensor(qstart).cuda(),
@@ -49,6 +49,15 @@ def test_prefill_matches_the_oracle(orc, G, b):
     qlen = [1, 17, 128 // G, 300]
     got, ref = _case(100 + G + b, ctx, qlen, Hq=2 * G, Hkv=2, b=b)
     assert_close(got, ref, f"prefill G={G} b={b}")
+
+
+@pytest.mark.parametrize("b", [0, 32, 64])
+def test_prefill_head_dim_64(orc, b):
+    ctx = [1, 70, 1000 + 32, 300]
+    qlen = [1, 17, 32, 300]
+    sig = workloads.random_signs(9, 64) if b else None
+    got, ref = _case(140 + b, ctx, qlen, Hq=8, Hkv=2, b=b, signs=sig, D=64)
+    assert_close(got, ref, f"prefill D=64 b={b}")
 
 
 def test_prefill_long_context_and_signs(orc):
@@ -86,3 +95,21 @@ def test_prefill_out_of_range_sequence_is_reported_and_left_unwritten(orc, bad):
     ref = orc_decode(q[:32], c, s, z, w.page_table[np.zeros(32, int)], (pos + 1).astype(np.int32), 2, 128,
                      w.num_pages, None)
     assert_close(got[:32], ref, "prefill valid sequence beside an invalid one")
+
+
+def test_prefill_bf16_output_is_the_rounded_fp32_output(orc):
+    ctx, qlen = [600, 90], [130, 90]
+    w = workloads.random_case(seed=150, B=2, Hq=8, Hkv=2, D=128, block=64, context_lens=ctx)
+    cache, scales, zeros = kvq.alloc_cache(w.num_pages, w.Hkv, w.D)
+    kvq.kv_quant_write(w.k_new.cuda(), w.v_new.cuda(), torch.as_tensor(w.slots_new).cuda(), cache, scales,
+                       zeros, 64)
+    qstart = torch.tensor([0, 130, 220], dtype=torch.int32).cuda()
+    q = (torch.randn((220, 8, 128), generator=torch.Generator().manual_seed(4)) / 8).to(torch.bfloat16).cuda()
+    args = (cache, scales, zeros, torch.as_tensor(w.page_table).cuda(), torch.as_tensor(w.context_lens).cuda(),
+            qstart, 130)
+    o32 = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    o16 = torch.empty(q.shape, dtype=torch.bfloat16, device="cuda")
+    kvq.paged_prefill_attn_int4(q, *args, o32, 64)
+    kvq.paged_prefill_attn_int4(q, *args, o16, 64)
+    assert kvq.get_device_error() == 0
+    assert torch.equal(o16, o32.to(torch.bfloat16))

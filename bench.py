@@ -281,7 +281,7 @@ class Step:
 
     N_POOLS = 4
 
-    def __init__(self, w, block, dev, graph=True):
+    def __init__(self, w, block, dev, graph=True, signs=None):
         import ctypes
         import numpy as np
         import torch
@@ -306,7 +306,9 @@ class Step:
         self.ws_bytes = self.ws.numel()
         self.stream = torch.cuda.Stream(dev)
         self.sh = ctypes.c_void_p(self.stream.cuda_stream)
-        self.wdesc = _lib.WriteDesc(w.tokens_written, w.Hkv, w.D, 16, w.num_pages)
+        # randomized Hadamard: the same sign mask in both descriptors
+        sw = kvq.sign_words(signs, w.D)
+        self.wdesc = _lib.WriteDesc(w.tokens_written, w.Hkv, w.D, 16, w.num_pages, sw)
         # q, the page table and the context lengths are set up once, never
         # written by the write kernel that precedes each decode
         # with the host copy of the context lengths (a serving engine has it)
@@ -314,7 +316,7 @@ class Step:
         self.lens_host = np.ascontiguousarray(w.context_lens, dtype=np.int32)
         self.adesc = _lib.AttnDesc(w.B, w.Hq, w.Hkv, w.D, 16, w.num_pages, w.max_pages, block, 0.0, 1,
                                    _lib.ATTN_INPUTS_READY,
-                                   self.lens_host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)))
+                                   self.lens_host.ctypes.data_as(ctypes.POINTER(ctypes.c_int32)), sw)
         P = ctypes.c_void_p
         self.write_args = []
         for i in range(self.N_POOLS):
@@ -335,7 +337,7 @@ class Step:
         # fused = one paged_decode_append_attn_int4 launch
         k1, v1, s1 = self.last_tokens(w)
         self.k1, self.v1, self.s1 = k1.to(dev), v1.to(dev), s1.to(dev)
-        self.wdesc1 = _lib.WriteDesc(w.B, w.Hkv, w.D, 16, w.num_pages)
+        self.wdesc1 = _lib.WriteDesc(w.B, w.Hkv, w.D, 16, w.num_pages, sw)
         self.write1_args, self.app_args = [], []
         for i in range(self.N_POOLS):
             c, s, z = self.pools[(i - 2) % self.N_POOLS]
@@ -682,6 +684,11 @@ def main(argv=None):
     if not args.no_plain and block != 0:
         p = Step(w, 0, dev, graph=not args.no_graph)
         p.fill_pools()
+    # randomized Hadamard (a seeded sign mask) on the same workload
+    r = None
+    if not args.no_plain and block != 0:
+        r = Step(w, block, dev, graph=not args.no_graph, signs=workloads.random_signs(cfg.seed + 11, w.D))
+        r.fill_pools()
     rounds = 3
     with ClockSampler(local) as clocks:
         clocks.wait_first_sample()
@@ -696,13 +703,17 @@ def main(argv=None):
         barrier()
         # each kernel alone, back to back, for its own line: the median of
         # `rounds` measurements, rotated and plain alternating
-        ms = {k: [] for k in ("write", "decode", "p_write", "p_decode", "append_separate", "append_fused")}
+        ms = {k: [] for k in ("write", "decode", "p_write", "p_decode", "r_write", "r_decode",
+                              "append_separate", "append_fused")}
         for _ in range(rounds):
             for kind in ("write", "decode"):
                 ms[kind].append(step.timed_only(kind, args.steps, start_index=warm))
                 barrier()
                 if p is not None:
                     ms["p_" + kind].append(p.timed_only(kind, args.steps, start_index=warm))
+                    barrier()
+                if r is not None:
+                    ms["r_" + kind].append(r.timed_only(kind, args.steps, start_index=warm))
                     barrier()
             # decode with a 1-token append per sequence: two launches or one
             for kind in ("append_separate", "append_fused"):
@@ -734,6 +745,18 @@ def main(argv=None):
             },
         }
         del p
+    randomized = None
+    if r is not None:
+        r_wr_ms = max_over_ranks(statistics.median(ms["r_write"]))
+        r_de_ms = max_over_ranks(statistics.median(ms["r_decode"]))
+        randomized = {
+            "what": "R = H_b diag(sigma) / sqrt(b), a seeded sign mask in both descriptors",
+            "kv_quant_write_us": round(1e3 * r_wr_ms, 3),
+            "paged_decode_attn_int4_us": round(1e3 * r_de_ms, 3),
+            "vs_plain_rotation": {"kv_quant_write": round(r_wr_ms / wr_ms - 1, 4),
+                                  "paged_decode_attn_int4": round(r_de_ms / de_ms - 1, 4)},
+        }
+        del r
 
     # chunked prefill (a row beside the step, not part of it): a few launches
     pf_ms, pf_flops = prefill_run(step, 3, 1)
@@ -781,6 +804,7 @@ def main(argv=None):
                                        "cached_tokens_per_s": round(w.tokens_cached / (de_ms / 1e3), 1)},
         },
         "plain_int4": plain,
+        "randomized_hadamard": randomized,
         "decode_append": {
             "what": "each sequence's new token stored, then a decode step over contexts that include it",
             "separate_us": round(1e3 * ap_sep_ms, 3),  # kv_quant_write (B tokens) + paged_decode_attn_int4

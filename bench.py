@@ -89,14 +89,23 @@ KERNEL_SOURCES = {
 }
 
 
+def strip_comments(src):
+    """C/C++ source without its // and /* */ comments and trailing blanks
+    (string literals in these kernels hold no comment markers)."""
+    import re
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    src = re.sub(r"//[^\n]*", "", src)
+    return "\n".join(line.rstrip() for line in src.splitlines() if line.strip())
+
+
 def source_digest(kernel):
-    """Hash of one kernel's sources: a committed DRAM-traffic figure is valid
-    only for the kernel it was captured from."""
+    """Hash of one kernel's sources, comments excluded: a committed
+    DRAM-traffic figure is valid only for the code it was captured from."""
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "bit_kv_cache_20_b200", "csrc")
     for name in KERNEL_SOURCES[kernel]:
-        with open(os.path.join(csrc, name), "rb") as f:
-            h.update(name.encode() + f.read())
+        with open(os.path.join(csrc, name)) as f:
+            h.update(name.encode() + strip_comments(f.read()).encode())
     return h.hexdigest()[:16]
 
 

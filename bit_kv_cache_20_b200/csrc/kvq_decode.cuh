@@ -1,7 +1,7 @@
 // kvq_decode.cuh - split-K paged decode attention over the rotated INT4 cache.
 //
-// SAW-INT4 (Abstract): "fused attention execution" over the quantized paged
-// cache. The rotation R is orthogonal and its own inverse, so the kernel
+// SAW-INT4 (Abstract): attention is computed by the kernel that reads the
+// quantized paged cache, with no separate dequantization pass. The rotation R is orthogonal and its own inverse, so the kernel
 // rotates q once, runs attention in the rotated space directly on the codes,
 // and rotates the output back: out = R sum_t p_t v^_t.
 //

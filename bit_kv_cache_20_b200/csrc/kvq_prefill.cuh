@@ -1,10 +1,10 @@
 // kvq_prefill.cuh - chunked-prefill attention over the rotated INT4 cache on
 // the 5th-generation tensor cores.
 //
-// SAW-INT4 (Abstract): attention executes directly on the quantized paged
-// cache ("fused attention execution") for "high-throughput concurrent
-// workloads". A prefill chunk brings many queries per sequence, so QK^T and
-// PV become dense products and run as tcgen05 MMAs.
+// SAW-INT4 (Abstract): attention is computed directly on the quantized paged
+// cache, and the method targets serving many requests at once. A prefill
+// chunk brings many queries per sequence, so QK^T and PV become dense
+// products and run as tcgen05 MMAs.
 //
 // Sequence n's chunk is its last qlen context tokens (positions ctx - qlen ..
 // ctx - 1), already written to the cache by kv_quant_write; query token i of

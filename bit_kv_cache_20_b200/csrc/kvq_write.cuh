@@ -1,8 +1,8 @@
 // kvq_write.cuh - fused rotation + token-wise INT4 quantization + paged store.
 //
-// SAW-INT4 (Abstract): "a fused rotation-quantization kernel that integrates
-// directly into paged KV-cache layouts"; OScaR (forum summary, "The OScaR
-// Framework"): rotate, then quantize.
+// SAW-INT4 (Abstract): a single kernel rotates, quantizes and stores each
+// row straight into the paged cache; OScaR (forum summary, "The OScaR
+// Framework"): rotate first, then quantize.
 //
 // Work unit: a warp tile = 32 consecutive tokens of one (kv head, K|V). One
 // thread owns one row (token, head, K|V) of D values, so the whole Hadamard

@@ -1,9 +1,9 @@
 // kvq_write_tc.cuh - fused rotation + token-wise INT4 quantization + paged
 // store, with the rotation on the 5th-generation tensor cores.
 //
-// SAW-INT4 (Abstract): "a fused rotation-quantization kernel that integrates
-// directly into paged KV-cache layouts"; OScaR (forum summary, "The OScaR
-// Framework"): rotate, then quantize.
+// SAW-INT4 (Abstract): a single kernel rotates, quantizes and stores each
+// row straight into the paged cache; OScaR (forum summary, "The OScaR
+// Framework"): rotate first, then quantize.
 //
 // The block-diagonal Hadamard rotation of a tile of 128 rows (128 consecutive
 // tokens of one kv head, K or V) is one dense product Y = X H with X [128 x D]

@@ -7,9 +7,9 @@
  * Sources (web pages, cited by title and section):
  *  [SAW]   "SAW-INT4: System-Aware 4-Bit KV-Cache Quantization for Real-World
  *          LLM Serving", Abstract (arXiv 2604.19157 mirror): token-wise INT4
- *          with block-diagonal Hadamard rotation; a fused rotation-quantization
- *          kernel that writes straight into paged KV-cache layouts; fused
- *          attention execution over the quantized cache.
+ *          after a Hadamard rotation applied block by block; one kernel
+ *          rotates, quantizes and stores into the paged cache; attention
+ *          is computed on the quantized cache in the kernel that reads it.
  *  [OSCAR] "OScaR: Occam's Razor for Extreme KV Cache Quantization in LLMs"
  *          (forum summary), section "The OScaR Framework": V^ = Quant(S.(R.V)),
  *          rotate first, then scale, then quantize.
@@ -116,9 +116,8 @@ typedef struct kvq_attn_desc {
 
 /*
  * kv_quant_write - fused rotate + token-wise INT4 quantize + paged store
- * ([SAW] Abstract: "fused rotation-quantization kernel that integrates
- * directly into paged KV-cache layouts"; [OSCAR] "The OScaR Framework":
- * rotate, then quantize).
+ * ([SAW] Abstract: one kernel rotates, quantizes and stores into the paged
+ * cache; [OSCAR] "The OScaR Framework": rotate first, then quantize).
  *
  * For every new token t, kv head h and tensor X in {K, V}, with row x = X[t,h,:]:
  *   1. y = R x, R = diag(H_b/sqrt(b), ...) over contiguous b-channel blocks,
@@ -168,7 +167,8 @@ size_t kvq_attn_workspace_size(const kvq_attn_desc* desc);
 
 /*
  * paged_decode_attn_int4 - one decode step of attention over the INT4 cache
- * ([SAW] Abstract: "fused attention execution"; the rotation is orthogonal,
+ * ([SAW] Abstract: attention computed on the quantized cache in the kernel
+ * that reads it; the rotation is orthogonal,
  * so q.k = (Rq).(Rk) and the output is R^T sum_t p_t (R v_t), with R^T = R
  * because H_b/sqrt(b) is symmetric and its own inverse).
  *
@@ -206,8 +206,8 @@ kvq_status paged_decode_attn_int4(const void* q, const uint8_t* cache,
  * paged_decode_append_attn_int4 - one decode step that also appends the
  * step's new token: kv_quant_write of k_new/v_new at slot_mapping followed by
  * paged_decode_attn_int4 over the contexts that include it, in one launch
- * ([SAW] Abstract: the rotation-quantization kernel "integrates directly
- * into paged KV-cache layouts" and attention execution is fused).
+ * ([SAW] Abstract: the rotate-quantize-store step and the attention over
+ * the paged cache, here in a single kernel).
  *
  * For sequence n the new token is position context_lens[n] - 1: its slot
  * (page * 16 + offset) must be page_table[n][(ctx - 1) / 16] * 16 +
@@ -238,8 +238,8 @@ kvq_status paged_decode_append_attn_int4(const void* q, const void* k_new,
 
 /*
  * paged_prefill_attn_int4 - chunked-prefill attention over the INT4 cache
- * ([SAW] Abstract: fused attention over the quantized paged cache, for
- * "high-throughput concurrent workloads"): many queries per sequence, so
+ * ([SAW] Abstract: attention on the quantized paged cache, aimed at serving
+ * many requests at once): many queries per sequence, so
  * QK^T and PV run as dense tcgen05 MMAs.
  *
  * Sequence n's chunk is its last L_n = q_start[n+1] - q_start[n] context

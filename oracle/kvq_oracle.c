@@ -206,7 +206,7 @@ int oracle_rotate_row(const uint16_t* x_bf16, int D, int b, float* y) {
 }
 
 /* ------------------------------------------------------------------------- */
-/* Token-wise asymmetric INT4 quantization ([SAW] Abstract "token-wise INT4"; */
+/* Asymmetric INT4 quantization, one scale per token ([SAW] Abstract;       */
 /* [OSCAR] Quant(.) after the rotation).                                     */
 /* ------------------------------------------------------------------------- */
 
@@ -286,8 +286,8 @@ void oracle_dequant_row(const uint8_t* packed, int D, uint16_t s, uint16_t z, do
 }
 
 /* ------------------------------------------------------------------------- */
-/* Paged placement ([SAW] Abstract: "integrates directly into paged KV-cache  */
-/* layouts").                                                                 */
+/* Paged placement ([SAW] Abstract: the quantized rows are stored straight   */
+/* into the paged cache).                                                     */
 /* ------------------------------------------------------------------------- */
 
 static size_t row_index(int64_t page, int Hkv, int h, int kv, int off) {

@@ -98,14 +98,18 @@ struct PfSmem {
   static constexpr int kTotal = kUsed + 1024;                // room to align the base to 1024 B
 };
 
-// bf16 pair of (x0, x1): the "hi" rounding, or with `lo` the remainder
-// bf16(x - hi) of each (hi + lo keeps 16 significant bits).
-__device__ __forceinline__ uint32_t hilo_pair_bf16(float x0, float x1, bool lo) {
+// The pair (x0, x1) as bf16 hi = RN(x) and lo = RN(x - hi), each packed in
+// one word (hi + lo keeps 16 significant bits).
+__device__ __forceinline__ void hilo_split_bf16(uint64_t x2, uint32_t& hw, uint32_t& lw) {
+  float x0, x1;
+  f2_unpack(x2, x0, x1);
   const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
   const float2 hf = __bfloat1622float2(h);
-  const __nv_bfloat162 l = __floats2bfloat162_rn(__fsub_rn(x0, hf.x), __fsub_rn(x1, hf.y));
-  const uint32_t hu = *reinterpret_cast<const uint32_t*>(&h), lu = *reinterpret_cast<const uint32_t*>(&l);
-  return lo ? lu : hu;
+  float r0, r1;
+  f2_unpack(f2_sub(x2, f2_pack(hf.x, hf.y)), r0, r1);
+  const __nv_bfloat162 l = __floats2bfloat162_rn(r0, r1);
+  hw = *reinterpret_cast<const uint32_t*>(&h);
+  lw = *reinterpret_cast<const uint32_t*>(&l);
 }
 
 // Two 4-bit codes of byte k of w -> half2 (low nibble, high nibble) as exact
@@ -389,23 +393,26 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
     // every row sees the whole block, every page is valid: no masks
     const bool open = kPfBlock * b + kPfBlock - 1 <= pos0 &&
                       (page_ok[0] & page_ok[1] & page_ok[2] & page_ok[3]) != 0;
-    float mb = -INFINITY;
-    if (open) {
+    // logits two at a time (f32x2): fma(S qi, s_k, z_k qs)
+    const uint64_t qi2 = f2_pack(qi, qi), qs2 = f2_pack(qs, qs);
 #pragma unroll
-      for (int t = 0; t < kH; ++t) {
-        sv[t] = fmaf(sv[t] * qi, sz[t0 + t], sz[kPfBlock + t0 + t] * qs);
-        mb = fmaxf(mb, sv[t]);
-      }
-    } else {
+    for (int t = 0; t < kH; t += 2) {
+      const float2 sk = *reinterpret_cast<const float2*>(sz + t0 + t);
+      const float2 zk = *reinterpret_cast<const float2*>(sz + kPfBlock + t0 + t);
+      f2_unpack(f2_fma(f2_mul(f2_pack(sv[t], sv[t + 1]), qi2), f2_pack(sk.x, sk.y), f2_mul(f2_pack(zk.x, zk.y), qs2)),
+                sv[t], sv[t + 1]);
+    }
+    if (!open) {
 #pragma unroll
       for (int t = 0; t < kH; ++t) {
         const int pos = kPfBlock * b + t0 + t;
         const bool live = row_ok && pos <= pos_r && page_ok[(t0 + t) >> 4];
-        const float lg = fmaf(sv[t] * qi, sz[t0 + t], sz[kPfBlock + t0 + t] * qs);
-        sv[t] = live ? lg : -INFINITY;
-        mb = fmaxf(mb, sv[t]);
+        sv[t] = live ? sv[t] : -INFINITY;
       }
     }
+    float mb = -INFINITY;
+#pragma unroll
+    for (int t = 0; t < kH; t += 2) mb = fmax3(mb, sv[t], sv[t + 1]);
     // the row's block maximum: the two halves meet (warps quarter and
     // quarter + 4, 64 threads, named barrier 1 + quarter)
     xch[half * kPfRows + row] = mb;
@@ -419,23 +426,36 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
     zs *= alpha;
     alpha_prev = alpha;
     m_used = m_new;
-    // p and P' = p * s_v as bf16 hi + lo, this half of row `row` of the A operands
+    // p and P' = p * s_v as bf16 hi + lo, this half of row `row` of the A
+    // operands, two at a time; a masked logit (-inf) gives exp2 = 0, and a
+    // row with no visible position yet (m = -inf) subtracts 0 instead
+    const float msub = (m_used == -INFINITY) ? 0.0f : m_used;
+    const uint64_t m2 = f2_pack(msub, msub);
+    uint64_t l2 = f2_pack(0.0f, 0.0f), z2 = l2;
 #pragma unroll
     for (int t8 = 0; t8 < kH; t8 += 8) {
       uint32_t hw[4], lw[4];
 #pragma unroll
       for (int k = 0; k < 8; k += 2) {
         const int t = t8 + k;
-        const float p0 = (sv[t] == -INFINITY) ? 0.0f : fast_exp2(sv[t] - m_used);
-        const float p1 = (sv[t + 1] == -INFINITY) ? 0.0f : fast_exp2(sv[t + 1] - m_used);
-        l_sum += p0 + p1;
-        zs = fmaf(p0, sz[3 * kPfBlock + t0 + t], fmaf(p1, sz[3 * kPfBlock + t0 + t + 1], zs));
-        const float P0 = p0 * sz[2 * kPfBlock + t0 + t], P1 = p1 * sz[2 * kPfBlock + t0 + t + 1];
-        hw[k / 2] = hilo_pair_bf16(P0, P1, false);
-        lw[k / 2] = hilo_pair_bf16(P0, P1, true);
+        float d0, d1;
+        f2_unpack(f2_sub(f2_pack(sv[t], sv[t + 1]), m2), d0, d1);
+        const uint64_t p2 = f2_pack(fast_exp2(d0), fast_exp2(d1));
+        const float2 s_v = *reinterpret_cast<const float2*>(sz + 2 * kPfBlock + t0 + t);
+        const float2 z_v = *reinterpret_cast<const float2*>(sz + 3 * kPfBlock + t0 + t);
+        l2 = f2_add(l2, p2);
+        z2 = f2_fma(p2, f2_pack(z_v.x, z_v.y), z2);
+        hilo_split_bf16(f2_mul(p2, f2_pack(s_v.x, s_v.y)), hw[k / 2], lw[k / 2]);
       }
       *reinterpret_cast<uint4*>(smem + S::kPhi + sw128_offset(row, t0 + t8, kPfRows)) = make_uint4(hw[0], hw[1], hw[2], hw[3]);
       *reinterpret_cast<uint4*>(smem + S::kPlo + sw128_offset(row, t0 + t8, kPfRows)) = make_uint4(lw[0], lw[1], lw[2], lw[3]);
+    }
+    {
+      float a0, a1, c0, c1;
+      f2_unpack(l2, a0, a1);
+      f2_unpack(z2, c0, c1);
+      l_sum += a0 + a1;
+      zs += c0 + c1;
     }
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");
     tc_fence_before();

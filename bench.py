@@ -189,6 +189,35 @@ def prefill_run(step, launches, warm):
     return total / launches, prefill_flops(w.context_lens, PREFILL_CHUNK, w.Hq, w.D)
 
 
+def prefill_cpu_baseline(w, block, n_ctx=4096, n_q=64):
+    """The oracle's attention for a chunk of `n_q` queries at the end of an
+    `n_ctx`-token context of sequence 0 (its cache written by the oracle from
+    the workload's first tokens, untimed), on the host cores. None when the
+    workload's new tokens do not start with sequence 0's positions 0, 1, ..."""
+    import numpy as np
+    import torch
+    import oracle
+    from bit_kv_cache_20_b200 import workloads
+    n = min(n_ctx, int(w.context_lens[0]), w.tokens_written)
+    want = np.array([int(w.page_table[0][p // 16]) * 16 + p % 16 for p in range(n)], np.int64)
+    if int(w.prior_lens[0]) != 0 or n < n_q or not np.array_equal(np.asarray(w.slots_new[:n]), want):
+        return None
+    cache, scales, zeros, _ = oracle.quant_write(workloads.bf16_bits(w.k_new[:n]), workloads.bf16_bits(w.v_new[:n]),
+                                                 w.slots_new[:n], w.num_pages, block)
+    g = torch.Generator().manual_seed(w.cfg.seed + 7)
+    q = (torch.randn((n_q, w.Hq, w.D), generator=g) / 8).to(torch.bfloat16)
+    ctx = np.arange(n - n_q + 1, n + 1).astype(np.int32)
+    pt = np.repeat(np.asarray(w.page_table)[:1], n_q, axis=0)
+    t0 = time.perf_counter()
+    oracle.decode_attn(workloads.bf16_bits(q), cache, scales, zeros, pt, ctx, w.Hkv, block, w.num_pages)
+    dt = time.perf_counter() - t0
+    flops = 4 * w.D * w.Hq * int(ctx.sum())
+    return {"value": round(flops / dt / 1e12, 6), "unit": "TFLOP/s", "cores": oracle.num_threads(),
+            "kind": "oracle",
+            "sample": f"{n_q} causal chunk queries x {w.Hq} heads at the end of a {n}-token context; "
+                      f"{dt:.2f} s"}
+
+
 def prefill_line(ms, flops):
     peak, src = measured_peaks("bf16_tflops")
     tf = flops / (ms / 1e3) / 1e12
@@ -826,6 +855,7 @@ def main(argv=None):
     }
     if not args.no_cpu_baseline:
         line["cpu_baseline"] = cpu_baseline(w, block)
+        line["prefill"]["cpu_baseline"] = prefill_cpu_baseline(w, block)
     print(json.dumps(line), flush=True)
     return 0
 

@@ -40,7 +40,7 @@ def orc_decode(q, c, s, z, pt, ctx, Hkv, b, num_pages, signs):
     return oracle.decode_attn(workloads.bf16_bits(q), c, s, z, pt, ctx, Hkv, b, num_pages, signs=signs)
 
 
-@pytest.mark.parametrize("G", [1, 4, 8])
+@pytest.mark.parametrize("G", [1, 2, 4, 8])
 @pytest.mark.parametrize("b", [0, 64, 128])
 def test_prefill_matches_the_oracle(orc, G, b):
     # chunks: 1 token, a ragged tile, exactly one tile of 128 / G tokens, several tiles;

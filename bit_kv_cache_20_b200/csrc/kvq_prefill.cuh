@@ -355,12 +355,15 @@ __global__ void __launch_bounds__(kPfThreads, 1) kvq_prefill_kernel(const __grid
       if (!ok && lp * 16 < ctx && (t & 15) == 0) record_error(KVQ_ERR_OUT_OF_RANGE);
       const __half* scl = reinterpret_cast<const __half*>(st + pg * S::kSlot + 16 * D);
       const __half* zer = reinterpret_cast<const __half*>(st + pg * S::kSlot + 16 * D + 64);
-      // scales, and the zero points of the centred codes: z + 8 s
+      // scales, and the zero points of the centred codes: z + 8 s. Rows past
+      // the context may hold anything (NaN scales included): they get 0, so
+      // that their zero weights cannot turn 0 * garbage into NaN
+      const bool live = ok && lp * 16 + (t & 15) < ctx;
       const float s_k = __half2float(scl[t & 15]), s_v = __half2float(scl[16 + (t & 15)]);
-      sz[0 * kPfBlock + t] = ok ? s_k : 0.0f;
-      sz[1 * kPfBlock + t] = ok ? fmaf(8.0f, s_k, __half2float(zer[t & 15])) : 0.0f;
-      sz[2 * kPfBlock + t] = ok ? s_v : 0.0f;
-      sz[3 * kPfBlock + t] = ok ? fmaf(8.0f, s_v, __half2float(zer[16 + (t & 15)])) : 0.0f;
+      sz[0 * kPfBlock + t] = live ? s_k : 0.0f;
+      sz[1 * kPfBlock + t] = live ? fmaf(8.0f, s_k, __half2float(zer[t & 15])) : 0.0f;
+      sz[2 * kPfBlock + t] = live ? s_v : 0.0f;
+      sz[3 * kPfBlock + t] = live ? fmaf(8.0f, s_v, __half2float(zer[16 + (t & 15)])) : 0.0f;
       if ((t & 15) == 0) page_ok[pg] = ok ? 1 : 0;
     }
     asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");  // operands visible to the MMAs

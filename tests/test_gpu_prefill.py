@@ -113,3 +113,50 @@ def test_prefill_bf16_output_is_the_rounded_fp32_output(orc):
     kvq.paged_prefill_attn_int4(q, *args, o16, 64)
     assert kvq.get_device_error() == 0
     assert torch.equal(o16, o32.to(torch.bfloat16))
+
+
+def test_prefill_ignores_garbage_past_the_context(orc):
+    """Rows of a sequence's last page past its context may hold anything
+    (filled here with NaN scales and offsets and random code bytes); they
+    must not reach the output."""
+    ctx, qlen = [250, 31, 100], [60, 31, 1]
+    w = workloads.random_case(seed=160, B=3, Hq=8, Hkv=2, D=128, block=64, context_lens=ctx)
+    cache, scales, zeros = kvq.alloc_cache(w.num_pages, w.Hkv, w.D)
+    g = torch.Generator(device="cuda").manual_seed(161)
+    cache.copy_(torch.randint(0, 256, cache.shape, generator=g, device="cuda", dtype=torch.int32).to(torch.uint8))
+    scales.view(torch.int16).fill_(0x7E00)  # fp16 NaN
+    zeros.view(torch.int16).fill_(0x7E00)
+    kvq.kv_quant_write(w.k_new.cuda(), w.v_new.cuda(), torch.as_tensor(w.slots_new).cuda(), cache, scales,
+                       zeros, 64)
+    qstart = np.concatenate([[0], np.cumsum(qlen)]).astype(np.int32)
+    q = (torch.randn((int(qstart[-1]), 8, 128), generator=torch.Generator().manual_seed(162)) / 8).to(torch.bfloat16)
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    kvq.paged_prefill_attn_int4(q.cuda(), cache, scales, zeros, torch.as_tensor(w.page_table).cuda(),
+                                torch.as_tensor(w.context_lens).cuda(), torch.as_tensor(qstart).cuda(),
+                                max(qlen), out, 64)
+    assert kvq.get_device_error() == 0
+    got = out.cpu().numpy().astype(np.float64)
+    assert np.all(np.isfinite(got))
+    rows_n = np.repeat(np.arange(3), qlen)
+    pos = np.concatenate([np.arange(c - l, c) for c, l in zip(ctx, qlen)])
+    c, s, z = host_cache(cache, scales, zeros)
+    ref = orc_decode(q, c, s, z, w.page_table[rows_n], (pos + 1).astype(np.int32), 2, 64, w.num_pages, None)
+    assert_close(got, ref, "prefill with garbage past the context")
+
+
+def test_prefill_bad_page_id_is_reported(orc):
+    ctx, qlen = [100, 40], [30, 40]
+    w = workloads.random_case(seed=170, B=2, Hq=4, Hkv=2, D=64, block=32, context_lens=ctx)
+    cache, scales, zeros = kvq.alloc_cache(w.num_pages, w.Hkv, w.D)
+    kvq.kv_quant_write(w.k_new.cuda(), w.v_new.cuda(), torch.as_tensor(w.slots_new).cuda(), cache, scales,
+                       zeros, 32)
+    pt = w.page_table.copy()
+    pt[0, 2] = w.num_pages + 5
+    qstart = torch.tensor([0, 30, 70], dtype=torch.int32).cuda()
+    q = (torch.randn((70, 4, 64), generator=torch.Generator().manual_seed(171)) / 8).to(torch.bfloat16).cuda()
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    kvq.paged_prefill_attn_int4(q, cache, scales, zeros, torch.as_tensor(pt).cuda(),
+                                torch.as_tensor(w.context_lens).cuda(), qstart, 40, out, 32)
+    assert kvq.get_device_error() == 3  # KVQ_ERR_OUT_OF_RANGE
+    assert kvq.get_device_error() == 0
+    assert np.all(np.isfinite(out.cpu().numpy()))

@@ -25,8 +25,9 @@ PAGE_SIZE = 16
 
 __all__ = [
     "PAGE_SIZE", "KVQError", "alloc_cache", "kv_quant_write", "paged_decode_attn_int4",
-    "attn_workspace_size", "alloc_workspace", "get_device_error", "library_path",
-    "paged_decode_attn_int4_static_ws",
+    "attn_workspace_size", "alloc_workspace", "get_device_error", "selftest_bounded_wait", "library_path",
+    "paged_decode_attn_int4_static_ws", "paged_decode_append_attn_int4", "paged_prefill_attn_int4",
+    "sign_words",
 ]
 
 
@@ -305,6 +306,15 @@ def paged_decode_attn_int4_static_ws(q: torch.Tensor, cache: torch.Tensor, scale
         _ptr(q), _ptr(cache), _ptr(scales), _ptr(zeros), _ptr(page_table), _ptr(context_lens),
         _ptr(out), ctypes.byref(desc), ctypes.c_void_p(_stream_handle(stream)))
     _lib.check(st, "paged_decode_attn_int4_static_ws")
+
+
+def selftest_bounded_wait(which: int, stream=None) -> None:
+    """Run one of the library's bounded waits on a condition that nothing
+    completes (0: an mbarrier wait, 1: the split-merge poll): it runs out
+    within seconds and records KVQ_ERR_TIMEOUT (read it with
+    get_device_error). For tests of the failure path."""
+    _lib.check(_lib.lib().kvq_selftest_bounded_wait(int(which), ctypes.c_void_p(_stream_handle(stream))),
+               "kvq_selftest_bounded_wait")
 
 
 def get_device_error(stream=None) -> int:

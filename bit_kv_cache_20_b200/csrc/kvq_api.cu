@@ -18,6 +18,7 @@
 #include "kvq_write.cuh"
 #include "kvq_write_tc.cuh"
 #include "kvq_prefill.cuh"
+#include "kvq_selftest.cuh"
 
 namespace {
 
@@ -805,6 +806,13 @@ kvq_status kvq_get_device_error(void* stream) {
     return KVQ_ERR_CUDA;
   }
   return static_cast<kvq_status>(v);
+}
+
+kvq_status kvq_selftest_bounded_wait(int32_t which, void* stream) {
+  if (which != 0 && which != 1) return KVQ_ERR_INVALID_ARG;
+  kvq::kvq_selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(which);
+  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+  return KVQ_OK;
 }
 
 kvq_status kvq_set_device(int32_t device) {

@@ -314,6 +314,20 @@ kvq_status kvq_get_device_error(void* stream);
  */
 kvq_status kvq_set_device(int32_t device);
 
+/*
+ * kvq_selftest_bounded_wait - the failure path of the library's bounded
+ * waits, for tests: on the current device, one warp runs a wait on a
+ * condition that nothing completes, which = 0: an mbarrier wait as in the
+ * write and prefill pipelines (gives up after ~4096 rounds of at most ~1 ms);
+ * which = 1: the decode's split-merge poll of a word that stays zero (gives
+ * up after 2^20 polls 64 ns apart). The wait runs out, records
+ * KVQ_ERR_TIMEOUT in the device error word and the kernel returns; nothing
+ * faults and the context stays usable. Not part of the hot path. Returns
+ * KVQ_OK once launched, KVQ_ERR_INVALID_ARG for another `which`, or
+ * KVQ_ERR_CUDA.
+ */
+kvq_status kvq_selftest_bounded_wait(int32_t which, void* stream);
+
 /* Static, human-readable name of a status value (never NULL). */
 const char* kvq_status_string(int32_t status);
 

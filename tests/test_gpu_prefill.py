@@ -160,3 +160,29 @@ def test_prefill_bad_page_id_is_reported(orc):
     assert kvq.get_device_error() == 3  # KVQ_ERR_OUT_OF_RANGE
     assert kvq.get_device_error() == 0
     assert np.all(np.isfinite(out.cpu().numpy()))
+
+
+def test_prefill_bench_workload_sampled(orc):
+    """The call bench.py times (llama3-8b-32k: the last 2048 tokens of the
+    32768-token context as one chunk, bf16 queries drawn as there), with 8
+    query tokens (all 32 heads) checked one by one against the oracle."""
+    import bench
+    w = workloads.make("llama3-8b-32k")
+    cache, scales, zeros = kvq.alloc_cache(w.num_pages, w.Hkv, w.D)
+    kvq.kv_quant_write(w.k_new.cuda(), w.v_new.cuda(), torch.as_tensor(w.slots_new).cuda(), cache, scales,
+                       zeros, w.block)
+    L = min(bench.PREFILL_CHUNK, int(w.context_lens[0]))
+    g = torch.Generator().manual_seed(w.cfg.seed + 7)
+    q = (torch.randn((L, w.Hq, w.D), generator=g) / 8).to(torch.bfloat16)
+    out = torch.empty(q.shape, dtype=torch.float32, device="cuda")
+    kvq.paged_prefill_attn_int4(q.cuda(), cache, scales, zeros, torch.as_tensor(w.page_table).cuda(),
+                                torch.as_tensor(w.context_lens).cuda(),
+                                torch.tensor([0, L], dtype=torch.int32, device="cuda"), L, out, w.block)
+    assert kvq.get_device_error() == 0
+    ctx = int(w.context_lens[0])
+    rows = np.array([0, 1, 31, 32, 777, 1500, L - 2, L - 1])
+    pos = ctx - L + rows
+    c, s, z = host_cache(cache, scales, zeros)
+    ref = orc_decode(q[rows], c, s, z, np.repeat(w.page_table, len(rows), axis=0), (pos + 1).astype(np.int32),
+                     w.Hkv, w.block, w.num_pages, None)
+    assert_close(out.cpu().numpy().astype(np.float64)[rows], ref, "prefill, bench workload, sampled rows")

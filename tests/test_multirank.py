@@ -68,3 +68,11 @@ def test_prefill_flops_counts_every_causal_pair():
             for i in range(L):
                 pairs += sum(1 for pos in range(c) if pos <= c - L + i)
         assert bench.prefill_flops(ctx, chunk, Hq=3, D=8) == 4 * 8 * 3 * pairs
+
+
+def test_source_digest_ignores_comments_only():
+    import bench
+    src = "int a; // one\n/* two\n three */ int b;\n\n  int c;  // four\n"
+    assert bench.strip_comments(src) == "int a;\n int b;\n  int c;"
+    assert bench.strip_comments(src) == bench.strip_comments(src.replace("one", "changed wording"))
+    assert bench.strip_comments(src) != bench.strip_comments(src.replace("int b", "int bb"))

@@ -76,3 +76,19 @@ def test_source_digest_ignores_comments_only():
     assert bench.strip_comments(src) == "int a;\n int b;\n  int c;"
     assert bench.strip_comments(src) == bench.strip_comments(src.replace("one", "changed wording"))
     assert bench.strip_comments(src) != bench.strip_comments(src.replace("int b", "int bb"))
+
+
+def test_reference_arm_prints_one_contract_line(monkeypatch, capsys):
+    import json
+    import bench
+    monkeypatch.setenv("RANK", "0")
+    monkeypatch.setenv("WORLD_SIZE", "1")
+    assert bench.main(["--impl", "reference", "--config", "tiny", "--steps", "2", "--warmup", "1"]) == 0
+    lines = [l for l in capsys.readouterr().out.splitlines() if l.strip()]
+    assert len(lines) == 1
+    d = json.loads(lines[0])
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "GB/s"
+    assert d["value"] > 0 and d["steps"] == 2 and d["higher_is_better"] is True
+    assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+    assert d["config"]["workload"] == "tiny"

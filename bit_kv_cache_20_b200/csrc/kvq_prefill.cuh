@@ -19,7 +19,8 @@
 // The cache is read in blocks of 64 tokens (4 pages), up to the tile's last
 // position:
 //   - 16-byte cp.async copies of the block's codes, scales and zeros into a
-//     double-buffered staging area (the next block loads while this one runs);
+//     double-buffered staging area (the next block loads while this one runs;
+//     its page ids were read from the page table a block earlier);
 //   - the codes become exact centred integers c - 8 in shared memory: K as
 //     fp16, the MMA's B operand [64 tokens][D], and V transposed as bf16,
 //     [D][64 tokens], both K-major with the 128-byte swizzle; the 8 moves into
@@ -34,9 +35,11 @@
 //     alone would move logits on keys with x10 outlier channels), codes are
 //     exact, the fp32 accumulator lands in tensor memory:
 //     logit = s_t 2^-e (q~ 2^e . (code_t - 8)) + (z_t + 8 s_t) sum(q~);
-//   - each thread takes its row of S from tensor memory, masks positions past
-//     its own, and runs an online softmax (running maximum, sum p, sum p z_v
-//     in registers);
+//   - each thread takes its half of the row's S from tensor memory, masks
+//     positions past its own, and runs its share of the online softmax two
+//     logits at a time (f32x2; sum p and sum p z_v in registers, the running
+//     maximum agreed with the partner thread); rows past the context get scale
+//     and offset 0, so that garbage there cannot reach the sums;
 //   - P' = p * s_v as bf16 hi + lo (16 significant bits over the fp32 exponent
 //     range: small weights never become subnormal) is written to shared memory
 //     as the A operand and O_blk = P' V (V codes as exact bf16 integers) goes

@@ -14,7 +14,19 @@ L2: two K/V input sets (134 MB each, larger than L2) alternate, and the decode
 of step i reads the cache written at step i-2 (four cache pools), with more
 than 300 MB of traffic in between.
 
+Besides the step, the JSON line carries:
+  - each kernel timed alone, and a roofline object for each;
+  - the plain-INT4 comparator (rotation overhead);
+  - the randomized-sign rotation;
+  - the decode step with a fused 1-token append;
+  - a chunked prefill (the last 2048 context tokens as one chunk, L2 flushed
+    before each launch);
+  - an end-to-end figure through the public API with host buffers;
+  - the SM clocks sampled during the timed regions;
+  - the oracle's throughput on the host cores.
+
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                    [--config NAME] [--only write|decode|prefill] [--no-graph]
 """
 from __future__ import annotations
 

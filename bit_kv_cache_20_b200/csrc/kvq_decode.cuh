@@ -34,11 +34,13 @@
 // are (head, limb 0 / 1) in one 8-column tile and (head, limb 2) in the even
 // columns of a second. PV needs floating
 // weights: p * s_v enters as an fp16 "hi" and "lo" part (hi + lo keeps ~22
-// bits) and the codes as exact normal fp16 values c (or 16c for a nibble at
-// bits 4..7, compensated in the epilogue); subnormal fp16 operands are
-// avoided on purpose - small products built from them lost precision in the
-// tensor-core accumulation (a systematic bias of ~2^-13 relative, measured on
-// B200). QK leaves a thread the logits of 2 tokens for one query head; PV
+// bits) and the codes as exact normal fp16 values c * 2^-9: a byte holding a
+// code in its low nibble, read as e4m3, is exactly c * 2^-9 (subnormal e4m3
+// for c < 8, normal fp16 after the conversion), so one cvt turns two bytes
+// into an A-operand register and the epilogue multiplies by 2^9. Subnormal
+// fp16 operands are avoided on purpose - small products built from them lost
+// precision in the tensor-core accumulation (a systematic bias of ~2^-13
+// relative, measured on B200). QK leaves a thread the logits of 2 tokens for one query head; PV
 // wants 4 tokens of one column, so 4 warp shuffles move the weights across.
 // Dequantization is folded into per-token scalars:
 //   logit_t = s_t * (q~ . code_t) + z_t * sum(q~)
@@ -677,17 +679,23 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
       lds_words<VW>(vb + (2 * tig + 9) * (D / 2) + g * (4 * VW), vd);
 #pragma unroll
       for (int u = 0; u < VW; ++u) {
-        const uint32_t xl = prmt(va[u], vb2[u], 0x5410), xh = prmt(va[u], vb2[u], 0x7632);
-        const uint32_t yl = prmt(vc[u], vd[u], 0x5410), yh = prmt(vc[u], vd[u], 0x7632);
-        const uint32_t xl8 = xl >> 8, xh8 = xh >> 8, yl8 = yl >> 8, yh8 = yh >> 8;
-        const uint32_t m0[4] = {codes_to_half2<false>(xl), codes_to_half2<false>(xl8),
-                                codes_to_half2<false>(yl), codes_to_half2<false>(yl8)};
-        const uint32_t m1[4] = {codes_to_half2<true>(xl), codes_to_half2<true>(xl8),
-                                codes_to_half2<true>(yl), codes_to_half2<true>(yl8)};
-        const uint32_t m2[4] = {codes_to_half2<false>(xh), codes_to_half2<false>(xh8),
-                                codes_to_half2<false>(yh), codes_to_half2<false>(yh8)};
-        const uint32_t m3[4] = {codes_to_half2<true>(xh), codes_to_half2<true>(xh8),
-                                codes_to_half2<true>(yh), codes_to_half2<true>(yh8)};
+        // bytes [tok0.b0, tok1.b0, tok0.b1, tok1.b1] (and b2, b3); a code in a
+        // byte's low nibble, read as e4m3, is exactly code * 2^-9
+        const uint32_t x0 = prmt(va[u], vb2[u], 0x5140), x1 = prmt(va[u], vb2[u], 0x7362);
+        const uint32_t y0 = prmt(vc[u], vd[u], 0x5140), y1 = prmt(vc[u], vd[u], 0x7362);
+        auto cv = [](uint32_t x, uint32_t& lo, uint32_t& hi) {
+          asm("{\n .reg .b16 a, b;\n mov.b32 {a, b}, %2;\n cvt.rn.f16x2.e4m3x2 %0, a;\n"
+              " cvt.rn.f16x2.e4m3x2 %1, b;\n}\n" : "=r"(lo), "=r"(hi) : "r"(x));
+        };
+        uint32_t m0[4], m1[4], m2[4], m3[4];
+        cv(x0 & 0x0F0F0F0Fu, m0[0], m0[1]);
+        cv((x0 >> 4) & 0x0F0F0F0Fu, m1[0], m1[1]);
+        cv(y0 & 0x0F0F0F0Fu, m0[2], m0[3]);
+        cv((y0 >> 4) & 0x0F0F0F0Fu, m1[2], m1[3]);
+        cv(x1 & 0x0F0F0F0Fu, m2[0], m2[1]);
+        cv((x1 >> 4) & 0x0F0F0F0Fu, m3[0], m3[1]);
+        cv(y1 & 0x0F0F0F0Fu, m2[2], m2[3]);
+        cv((y1 >> 4) & 0x0F0F0F0Fu, m3[2], m3[3]);
 #pragma unroll
         for (int c = 0; c < NC; ++c) {
           mma_f16_16816(o[c][4 * u + 0], m0, bp[c][0], bp[c][1]);
@@ -722,10 +730,12 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
         const float* t1 = o[c][4 * u + 1];
         const float* t2 = o[c][4 * u + 2];
         const float* t3 = o[c][4 * u + 3];
-        // hi + lo columns; the odd m-tiles carried 16c
+        // hi + lo columns; the codes entered as c * 2^-9
         float4* dst = reinterpret_cast<float4*>(orow + 8 * cb);
-        dst[0] = make_float4(t0[0] + t0[1], (t1[0] + t1[1]) * 0.0625f, t0[2] + t0[3], (t1[2] + t1[3]) * 0.0625f);
-        dst[1] = make_float4(t2[0] + t2[1], (t3[0] + t3[1]) * 0.0625f, t2[2] + t2[3], (t3[2] + t3[3]) * 0.0625f);
+        dst[0] = make_float4((t0[0] + t0[1]) * 512.0f, (t1[0] + t1[1]) * 512.0f, (t0[2] + t0[3]) * 512.0f,
+                             (t1[2] + t1[3]) * 512.0f);
+        dst[1] = make_float4((t2[0] + t2[1]) * 512.0f, (t3[0] + t3[1]) * 512.0f, (t2[2] + t2[3]) * 512.0f,
+                             (t3[2] + t3[3]) * 512.0f);
       }
       if (g == 0) {
         float* ml = mine + NR * D + (4 * c + tig) * 4;

@@ -27,7 +27,7 @@ __all__ = [
     "PAGE_SIZE", "KVQError", "alloc_cache", "kv_quant_write", "paged_decode_attn_int4",
     "attn_workspace_size", "alloc_workspace", "get_device_error", "selftest_bounded_wait", "library_path",
     "paged_decode_attn_int4_static_ws", "paged_decode_append_attn_int4", "paged_prefill_attn_int4",
-    "sign_words",
+    "sign_words", "selftest_occupy",
 ]
 
 
@@ -203,6 +203,14 @@ def paged_decode_attn_int4(q: torch.Tensor, cache: torch.Tensor, scales: torch.T
                                   _ptr(context_lens), _ptr(out), ws_ptr, ws_bytes,
                                   ctypes.byref(desc), ctypes.c_void_p(_stream_handle(stream)))
     _lib.check(st, "paged_decode_attn_int4")
+
+
+def selftest_occupy(ctas: int, microseconds: int, stream=None) -> None:
+    """Test hook: `ctas` CTAs that each hold most of an SM's shared memory and
+    end on their own after `microseconds`, launched on `stream`."""
+    _lib.check(_lib.lib().kvq_selftest_occupy(int(ctas), int(microseconds),
+                                              ctypes.c_void_p(_stream_handle(stream))),
+               "kvq_selftest_occupy")
 
 
 def paged_decode_append_attn_int4(q: torch.Tensor, k_new: torch.Tensor, v_new: torch.Tensor,

@@ -68,6 +68,8 @@ SIGNATURES = [
                                                         ctypes.c_void_p]),
     ("kvq_get_device_error", ctypes.c_int, [ctypes.c_void_p]),
     ("kvq_selftest_bounded_wait", ctypes.c_int, [ctypes.c_int32, ctypes.c_void_p]),
+    ("kvq_selftest_occupy", ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p]),
+    ("kvq_static_workspace_nonzero", ctypes.c_size_t, []),
     ("kvq_set_device", ctypes.c_int, [ctypes.c_int32]),
     ("kvq_status_string", ctypes.c_char_p, [ctypes.c_int32]),
     ("kvq_abi_version", ctypes.c_int32, []),

@@ -794,23 +794,33 @@ kvq_status paged_prefill_attn_int4(const void* q, const uint8_t* cache, const vo
   }
 }
 
-kvq_status kvq_get_device_error(void* stream) {
-  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) {
-    cudaGetLastError();
-    return KVQ_ERR_CUDA;
-  }
-  int v = 0, zero = 0;
-  if (cudaMemcpyFromSymbol(&v, kvq::g_device_error, sizeof(int)) != cudaSuccess ||
-      cudaMemcpyToSymbol(kvq::g_device_error, &zero, sizeof(int)) != cudaSuccess) {
-    cudaGetLastError();
-    return KVQ_ERR_CUDA;
-  }
-  return static_cast<kvq_status>(v);
-}
-
 kvq_status kvq_selftest_bounded_wait(int32_t which, void* stream) {
   if (which != 0 && which != 1) return KVQ_ERR_INVALID_ARG;
   kvq::kvq_selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(which);
+  if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
+  return KVQ_OK;
+}
+
+kvq_status kvq_selftest_occupy(int32_t ctas, int32_t microseconds, void* stream) {
+  if (ctas < 1 || ctas > 65535 || microseconds < 0 || microseconds > 1000000) return KVQ_ERR_INVALID_ARG;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
+  int smem_max = 0;
+  if (cudaDeviceGetAttribute(&smem_max, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
+  const int smem = smem_max - 8 * 1024;  // most of an SM's shared memory
+  if (cudaFuncSetAttribute(kvq::kvq_selftest_occupy_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) !=
+      cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
+  kvq::kvq_selftest_occupy_kernel<<<ctas, 32, smem, static_cast<cudaStream_t>(stream)>>>(
+      1000ull * (unsigned long long)microseconds);
   if (cudaGetLastError() != cudaSuccess) return KVQ_ERR_CUDA;
   return KVQ_OK;
 }
@@ -852,19 +862,44 @@ namespace {
 
 std::mutex g_static_ws_mutex;
 void* g_static_ws_ptr[kMaxDevices] = {};
+CUcontext g_static_ws_ctx[kMaxDevices] = {};
+
+typedef CUresult (*CtxGetFn)(CUcontext*);
+
+CtxGetFn ctx_query() {
+  static std::atomic<CtxGetFn> fn{nullptr};
+  CtxGetFn f = fn.load(std::memory_order_acquire);
+  if (f) return f;
+  void* raw = nullptr;
+  cudaDriverEntryPointQueryResult q;
+  if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &raw, cudaEnableDefault, &q) != cudaSuccess ||
+      q != cudaDriverEntryPointSuccess || !raw) {
+    cudaGetLastError();
+    return nullptr;
+  }
+  f = reinterpret_cast<CtxGetFn>(raw);
+  fn.store(f, std::memory_order_release);
+  return f;
+}
 
 // Device address of g_static_workspace on `dev` (which must be current). In
 // host code the array's name is only a host-side stand-in, so the address is
-// looked up once per device and cached.
+// looked up with cudaGetSymbolAddress once per device - again whenever the
+// device's current context is another one than at the last lookup (after a
+// cudaDeviceReset the module, and the array, may be loaded elsewhere).
 kvq_status static_workspace_on(int dev, void** out) {
   std::lock_guard<std::mutex> lock(g_static_ws_mutex);
-  if (!g_static_ws_ptr[dev]) {
+  CtxGetFn get = ctx_query();
+  CUcontext ctx = nullptr;
+  if (get && get(&ctx) != CUDA_SUCCESS) ctx = nullptr;
+  if (!g_static_ws_ptr[dev] || ctx != g_static_ws_ctx[dev]) {
     void* p = nullptr;
     if (cudaGetSymbolAddress(&p, g_static_workspace) != cudaSuccess || p == nullptr) {
       cudaGetLastError();
       return KVQ_ERR_CUDA;
     }
     g_static_ws_ptr[dev] = p;
+    g_static_ws_ctx[dev] = ctx;
   }
   *out = g_static_ws_ptr[dev];
   return KVQ_OK;
@@ -893,4 +928,45 @@ extern "C" kvq_status paged_decode_attn_int4_static_ws(const void* q, const uint
   // a per-sequence plan (host lengths given) runs when its partials fit too
   return paged_decode_attn_int4(q, cache, scales, zeros, page_table, context_lens, out, ws,
                                 (size_t)KVQ_STATIC_WORKSPACE_BYTES, desc, stream);
+}
+
+extern "C" kvq_status kvq_get_device_error(void* stream) {
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(st) != cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
+  int v = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&v, kvq::g_device_error, sizeof(int)) != cudaSuccess ||
+      cudaMemcpyToSymbol(kvq::g_device_error, &zero, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
+  if (v == KVQ_ERR_TIMEOUT) {
+    // words that arrived after a merge gave up may remain in the static
+    // split-K array, which no caller can reach: clear it
+    int dev = 0;
+    void* ws = nullptr;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices ||
+        static_workspace_on(dev, &ws) != KVQ_OK ||
+        cudaMemsetAsync(ws, 0, KVQ_STATIC_WORKSPACE_BYTES, st) != cudaSuccess ||
+        cudaStreamSynchronize(st) != cudaSuccess) {
+      cudaGetLastError();
+      return KVQ_ERR_CUDA;
+    }
+  }
+  return static_cast<kvq_status>(v);
+}
+
+extern "C" size_t kvq_static_workspace_nonzero(void) {
+  static unsigned char host[KVQ_STATIC_WORKSPACE_BYTES];
+  static std::mutex m;
+  std::lock_guard<std::mutex> lock(m);
+  if (cudaMemcpyFromSymbol(host, g_static_workspace, KVQ_STATIC_WORKSPACE_BYTES) != cudaSuccess) {
+    cudaGetLastError();
+    return SIZE_MAX;
+  }
+  size_t n = 0;
+  for (size_t i = 0; i < KVQ_STATIC_WORKSPACE_BYTES; ++i) n += host[i] != 0;
+  return n;
 }

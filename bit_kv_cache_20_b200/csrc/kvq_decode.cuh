@@ -71,8 +71,8 @@ struct AttnParams {
   const int32_t* page_table;  // [B][max_pages]
   const int32_t* ctx_lens;    // [B]
   void* out;                  // [B][Hq][D] fp32 or bf16
-  uint32_t* ws_part;          // [slots][Hkv][G][D + 4]: ~bits of O + Z, M, L, 2 unused;
-                              // zero between calls
+  uint32_t* ws_part;          // [slots][Hkv][G][D + 4]: ~bits of O + Z, M, L; a hand-over
+                              // word; 1 unused. Zero between calls
   int B, Hq, Hkv, G;
   int num_pages, max_pages;
   int n_splits, pages_per_split;
@@ -107,6 +107,11 @@ __host__ __device__ constexpr int attn_warps(int nc) { return nc == 2 ? 12 : 8; 
 constexpr int kWarpRing = 4;        // page slots per warp
 constexpr int kMaxSplits = 128;
 constexpr int kMaxPids = 1024;      // page ids of a CTA's range kept in shared memory
+// states of a partial-result row's word D + 2 (zero: not written yet)
+constexpr uint32_t kRowWritten = 1u;
+constexpr uint32_t kRowHandedOver = 2u;
+constexpr float kHead = 3.0f;        // log2 headroom of the lazy softmax reference
+constexpr float kBigScale = 8188.0f; // 65504 / 2^kHead: larger V scales force p <= 1
 
 // Shared memory of one decode CTA serving HG kv heads with NC column tiles
 // (4 query heads each).
@@ -127,7 +132,9 @@ struct AttnSmem {
   // then its fp16 scale and zero
   static constexpr int kAppRow = D / 2 + 16;
   static constexpr int kOffApp = kOffPid + kMaxPids * 4;
-  static constexpr int kTotal = kOffApp + HG * 2 * kAppRow;
+  // split-merge control words (see the merge at the end)
+  static constexpr int kOffCtl = (kOffApp + HG * 2 * kAppRow + 15) / 16 * 16;
+  static constexpr int kTotal = kOffCtl + 16;
 };
 
 template <int N>
@@ -248,6 +255,10 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
   }
   const int G = p.G;
   const unsigned FULL = 0xffffffffu;
+  // Split-merge control words: [0] a merger's hand-over decision (0 none yet,
+  // 3 being taken, 1 kept every row, 2 handed rows over), [1] rows handed
+  // over by this CTA, [2] rows handed over to this CTA.
+  uint32_t* sctl = reinterpret_cast<uint32_t*>(smem + S::kOffCtl);
 
   // The launch may overlap the previous kernel on the stream (programmatic
   // dependent launch). By default everything waits for it here; with
@@ -306,6 +317,7 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
       pids[i] = pt_row[i];
   }
   const int npg = max(min(p_begin + pps, n_pages) - p_begin, 0);
+  if (tid < 4) sctl[tid] = 0;
   __syncthreads();
 
   // Decode-append: the CTA whose range holds position ctx - 1 owns the new
@@ -340,8 +352,7 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
   const size_t code_page = (size_t)p.Hkv * (16 * D);  // bytes per page
   const size_t sz_page = (size_t)p.Hkv * 32;          // fp16 per page
   uint32_t valid = 0;
-  auto fetch = [&](int k) {
-    const int t = sub + k * NSUB;
+  auto fetch_t = [&](int k, int t) {
     const int slot = k % R;
     bool ok = false;
     if (t < npg) {
@@ -360,6 +371,7 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
     valid = ok ? (valid | (1u << slot)) : (valid & ~(1u << slot));
     cp_async_commit();
   };
+  auto fetch = [&](int k) { fetch_t(k, sub + k * NSUB); };
   // ---- q~ = R q * (softmax_scale * log2 e) -----------------------------------
   // One warp per row. Limbs, with a = q~ / sigma and sigma = max|q~| / 127:
   // q0 = rint(a), r1 = 256 (a - q0), q1 = rint(r1), q2 = rint(128 (r1 - q1))
@@ -485,7 +497,7 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
 
   if (early) {
     prep_q();    // overlaps the previous kernel's last CTAs
-    pdl_wait();  // the cache may be what that kernel wrote
+    pdl_wait();  // the cache (and the workspace) may be what that kernel wrote
     pdl_launch_dependents();
 #pragma unroll
     for (int k = 0; k < R - 1; ++k) fetch(k);
@@ -542,7 +554,7 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
   float m_run[NC], l_run[NC], zs_run[NC];
 #pragma unroll
   for (int c = 0; c < NC; ++c) {
-    m_run[c] = -INFINITY;
+    m_run[c] = hv[c] ? -INFINITY : 0.0f;  // padding rows: p = exp2(-inf - 0) = 0
     l_run[c] = 0.0f;
     zs_run[c] = 0.0f;
   }
@@ -614,6 +626,7 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
       float zv0 = __half2float(zer[16 + g]), zv1 = __half2float(zer[24 + g]);
       const int tok = tok_base + 16 * t;
       const bool tail = tok + 16 > ctx;
+      const bool sv_big = fmaxf(sv0, sv1) > kBigScale;
       if (tail) {
         // rows past the context may hold anything, NaN scales included: they
         // get p = 0 below, and V scale and offset 0 so that 0 * garbage
@@ -642,23 +655,29 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
           if (tok + g >= ctx) lg0 = -INFINITY;
           if (tok + g + 8 >= ctx) lg1 = -INFINITY;
         }
-        // online softmax, rescaling only when the running maximum grows
-        float pm = fmaxf(lg0, lg1);
-        pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 4));
-        pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 8));
-        pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 16));
-        if (pm > m_run[c]) {
-          const float alpha = (m_run[c] == -INFINITY) ? 0.0f : fast_exp2(m_run[c] - pm);
+        // lazy online softmax: p = exp2(logit - m) with m the reference the
+        // sums are kept in; it moves only when a logit exceeds m + kHead
+        // (or a huge V scale could overflow the fp16 weight), so most pages
+        // need neither a max reduction nor a rescale
+        const bool need = (lg0 > m_run[c] + kHead) || (lg1 > m_run[c] + kHead) || sv_big;
+        if (__any_sync(FULL, need)) {
+          float pm = fmaxf(lg0, lg1);
+          pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 4));
+          pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 8));
+          pm = fmaxf(pm, __shfl_xor_sync(FULL, pm, 16));
+          const bool big = __any_sync(FULL, sv_big);
+          const float mn = (pm > m_run[c] + kHead || (big && pm > m_run[c])) ? pm : m_run[c];
+          const float alpha = fast_exp2(m_run[c] - mn);
 #pragma unroll
           for (int i = 0; i < MT; ++i) {
             o[c][i][0] *= alpha; o[c][i][1] *= alpha; o[c][i][2] *= alpha; o[c][i][3] *= alpha;
           }
           l_run[c] *= alpha;
           zs_run[c] *= alpha;
-          m_run[c] = pm;
+          m_run[c] = mn;
         }
-        const float p0 = (lg0 == -INFINITY) ? 0.0f : fast_exp2(lg0 - m_run[c]);
-        const float p1 = (lg1 == -INFINITY) ? 0.0f : fast_exp2(lg1 - m_run[c]);
+        const float p0 = fast_exp2(lg0 - m_run[c]);
+        const float p1 = fast_exp2(lg1 - m_run[c]);
         l_run[c] += p0 + p1;
         zs_run[c] = fmaf(p0, zv0, fmaf(p1, zv1, zs_run[c]));
         const float P0 = p0 * sv0, P1 = p1 * sv1;
@@ -783,36 +802,61 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
       uint32_t* dst = p.ws_part + ((((size_t)slot_base + split) * p.Hkv + hgi * HG + hh) * G + r) * (D + 4);
       *reinterpret_cast<uint4*>(dst + c4) = make_uint4(~__float_as_uint(O.x + Z), ~__float_as_uint(O.y + Z),
                                                        ~__float_as_uint(O.z + Z), ~__float_as_uint(O.w + Z));
-      if (c4 == 0) *reinterpret_cast<uint2*>(dst + D) = make_uint2(~__float_as_uint(M), ~__float_as_uint(L));
+      if (c4 == 0) {
+        *reinterpret_cast<uint2*>(dst + D) = make_uint2(~__float_as_uint(M), ~__float_as_uint(L));
+        // mark the row written; a merger may have handed the row to this
+        // split meanwhile (see the split merge)
+        if (atomicExch(dst + D + 2, kRowWritten) == kRowHandedOver) atomicOr(&sctl[2], 1u << (hh * G + r));
+      }
     }
   }
 
   if (!single) {
+    __syncthreads();  // the rows handed over to this split are known
     // ---- split merge: CTA j < K merges query rows j, j + K, ... ------------
     // Each 32-bit word of a partial result is stored as ~bits(x). fp32
     // arithmetic never yields the bits 0xFFFFFFFF (a NaN payload it does not
     // produce), so no stored word is zero, and a zero word of the zero-filled
     // workspace means that split has not written it yet. A merger polls the
-    // words of its rows in L2 until none is zero - no fence, ticket or counter
-    // between writer and reader, each word validates itself - folds them and
-    // zeroes them again for the next call. Every CTA of the launch is resident
-    // at once, so the splits a merger waits for are running.
+    // words of its rows in L2 until none is zero - no fence or ticket between
+    // writer and reader, each word validates itself - folds them and zeroes
+    // them again for the next call.
+    //
+    // The splits a merger waits for have to get to run, and nothing
+    // guarantees that all CTAs of a launch are resident at once (other
+    // streams' kernels may hold SMs). So a merger never waits for long on a
+    // split that has not written: after a while it hands its rows over to
+    // such a split through a compare-and-swap of that split's row word D + 2
+    // (0 -> handed over) and exits. Every split, when it writes a row of its
+    // partial result, exchanges that word for "written"; finding "handed
+    // over", it merges the row itself once its partial is written. The word
+    // changes once either way, so each row is merged exactly once, and a CTA
+    // only ever waits for splits that have written (their stores are in
+    // flight) or hands over and leaves.
     const int rows = HG * G;
     const int K = min(rows, ns);
-    if (split >= K) return;
+    uint32_t todo = sctl[2];  // rows handed over to this split
+    if (split < K)
+      for (int rr = split; rr < rows; rr += K) todo |= 1u << rr;
+    if (todo == 0u) return;
     // Merge of one row: warp w takes splits w, w + 8, ...; lane l the output
     // float4 l. Each warp folds its splits into a running (max, l, acc), all
     // loads of a round (up to 8 splits) issued before any is used; the warps'
     // states are then combined through shared memory.
     constexpr int kRowBatch = 8;
+    constexpr uint32_t kHandOverRounds = 256;  // polls (~0.2 ms) before a merger hands over
     float* mred = reinterpret_cast<float*>(smem);            // [kAttnWarps] (the rings are free)
     float4* ored = reinterpret_cast<float4*>(smem + 64);     // [kAttnWarps][32]
     float* lred = reinterpret_cast<float*>(smem + 64 + kAttnWarps * 32 * 16);  // [kAttnWarps]
     static_assert(64 + kAttnWarps * 32 * 16 + kAttnWarps * 4 <= S::kRingBytes, "row-merge scratch fits in the rings");
     const size_t sstride = (size_t)p.Hkv * G * (D + 4);  // between consecutive slots
-    for (int rr = split; rr < rows; rr += K) {
+    uint32_t* row0 = p.ws_part + ((size_t)slot_base * p.Hkv + (size_t)hgi * HG) * G * (D + 4);
+    const int first = __ffs(todo) - 1;  // the hand-over window is this row's poll
+    for (uint32_t rest = todo; rest != 0u; rest &= rest - 1u) {
+      const int rr = __ffs(rest) - 1;
+      if ((sctl[1] >> rr) & 1u) continue;  // handed over
       const int hh = rr / G, r = rr % G;
-      uint32_t* base = p.ws_part + (((size_t)slot_base * p.Hkv + hgi * HG + hh) * G + r) * (D + 4);
+      uint32_t* base = row0 + (size_t)rr * (D + 4);
       float mw = -INFINITY, L = 0.0f;
       float4 acc = make_float4(0.0f, 0.0f, 0.0f, 0.0f);
       for (int s0 = warp; s0 < ns; s0 += kAttnWarps * kRowBatch) {
@@ -820,6 +864,7 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
         uint2 ml[kRowBatch];
         for (uint32_t rounds = 0;; ++rounds) {
           bool ok = true;
+          uint32_t miss = 0u;  // this lane's splits (bit k) with a word not written
 #pragma unroll
           for (int k = 0; k < kRowBatch; ++k) {
             const int s2 = s0 + k * kAttnWarps;
@@ -829,24 +874,38 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
               if (lane < D / 4) v[k] = ld_relaxed_gpu_v4(base + s2 * sstride + 4 * lane);
               ml[k] = ld_relaxed_gpu_v2(base + s2 * sstride + D);
             }
-            ok = ok && v[k].x && v[k].y && v[k].z && v[k].w && ml[k].x && ml[k].y;
+            const bool okk = v[k].x && v[k].y && v[k].z && v[k].w && ml[k].x && ml[k].y;
+            ok = ok && okk;
+            miss |= okk ? 0u : 1u << k;
           }
           if (__all_sync(FULL, ok)) break;
           if (rounds >= kMaxSpinRounds) {
             if (lane == 0) record_error(KVQ_ERR_TIMEOUT);
             break;
           }
+          if (rounds == kHandOverRounds && rr == first) {
+            const uint32_t wmiss = __reduce_or_sync(FULL, miss);
+            if (lane == 0 && wmiss != 0u && atomicCAS(&sctl[0], 0u, 3u) == 0u) {
+              // this warp decides for the CTA: hand every row of `todo` to
+              // one split that has not written; a row whose word already
+              // says "written" stays here (that split's stores are landing)
+              const int sj = s0 + (__ffs(wmiss) - 1) * kAttnWarps;
+              uint32_t gone = 0u;
+              for (uint32_t t2 = todo; t2 != 0u; t2 &= t2 - 1u) {
+                const int r2 = __ffs(t2) - 1;
+                if (atomicCAS(row0 + (size_t)sj * sstride + (size_t)r2 * (D + 4) + D + 2, 0u, kRowHandedOver) == 0u)
+                  gone |= 1u << r2;
+              }
+              atomicOr(&sctl[1], gone);
+              atomicExch(&sctl[0], gone ? 2u : 1u);
+            }
+          }
+          if (__shfl_sync(FULL, lane == 0 ? (*reinterpret_cast<volatile uint32_t*>(&sctl[1]) >> rr) & 1u : 0u, 0))
+            break;  // the row was handed over
           __nanosleep(64);
         }
-        __syncwarp();  // every lane holds its words: zero them for the next call
-#pragma unroll
-        for (int k = 0; k < kRowBatch; ++k) {
-          const int s2 = s0 + k * kAttnWarps;
-          if (s2 < ns) {
-            if (lane < D / 4) *reinterpret_cast<uint4*>(base + s2 * sstride + 4 * lane) = make_uint4(0u, 0u, 0u, 0u);
-            if (lane == 0) *reinterpret_cast<uint2*>(base + s2 * sstride + D) = make_uint2(0u, 0u);
-          }
-        }
+        __syncwarp();
+        if ((*reinterpret_cast<volatile uint32_t*>(&sctl[1]) >> rr) & 1u) break;  // handed over: the words stay
         float mb = mw;
 #pragma unroll
         for (int k = 0; k < kRowBatch; ++k)
@@ -874,6 +933,13 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
       }
       if (lane < D / 4) ored[warp * 32 + lane] = acc;
       __syncthreads();
+      if ((sctl[1] >> rr) & 1u) continue;  // this row went to another split
+      // the row's words are all read: zero them (and its word D + 2) for the
+      // next call
+      for (int s2 = warp; s2 < ns; s2 += kAttnWarps) {
+        if (lane < D / 4) *reinterpret_cast<uint4*>(base + s2 * sstride + 4 * lane) = make_uint4(0u, 0u, 0u, 0u);
+        if (lane == 0) *reinterpret_cast<uint4*>(base + s2 * sstride + D) = make_uint4(0u, 0u, 0u, 0u);
+      }
       if (warp == 0) {
         float M = mred[0];
 #pragma unroll
@@ -902,8 +968,12 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
       }
       __syncthreads();
     }
-    // rotate back this CTA's rows (one warp per row) and store
-    for (int rr = split + K * warp; rr < rows; rr += K * kAttnWarps) {
+    // rotate back the merged rows (one warp per row) and store
+    const uint32_t done = todo & ~sctl[1];
+    int nth = 0;
+    for (uint32_t rest = done; rest != 0u; rest &= rest - 1u, ++nth) {
+      if (nth % kAttnWarps != warp) continue;
+      const int rr = __ffs(rest) - 1;
       const int hh = rr / G, r = rr % G;
       const float* rp = qs + (hh * NR + r) * D;
       float v[E];

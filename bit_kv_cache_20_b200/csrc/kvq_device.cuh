@@ -71,6 +71,11 @@ __device__ __forceinline__ uint4 ld_relaxed_gpu_v4(const uint32_t* p) {
                : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "l"(p) : "memory");
   return v;
 }
+__device__ __forceinline__ uint32_t ld_relaxed_gpu_u32(const uint32_t* p) {
+  uint32_t v;
+  asm volatile("ld.relaxed.gpu.global.b32 %0, [%1];\n" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
 __device__ __forceinline__ uint2 ld_relaxed_gpu_v2(const uint32_t* p) {
   uint2 v;
   asm volatile("ld.relaxed.gpu.global.v2.b32 {%0, %1}, [%2];\n" : "=r"(v.x), "=r"(v.y) : "l"(p) : "memory");

@@ -40,4 +40,21 @@ __global__ void __launch_bounds__(32, 1) kvq_selftest_wait_kernel(int which) {
   }
 }
 
+// A kernel that holds SMs for a while and then ends on its own: each CTA
+// (given most of an SM's shared memory, so that little else fits beside it)
+// waits until `ns` nanoseconds of the global timer have passed, with a cap
+// on its polls. Tests use it to fill SMs while a decode is launched on
+// another stream.
+__global__ void __launch_bounds__(32, 1) kvq_selftest_occupy_kernel(unsigned long long ns) {
+  extern __shared__ uint8_t hold[];
+  unsigned long long t0, t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t0));
+  for (uint32_t i = 0; i < (1u << 22); ++i) {
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    if (t - t0 >= ns) break;
+    __nanosleep(256);
+  }
+  if (threadIdx.x == 0 && ns == ~0ull) hold[0] = 0;  // never: keeps the allocation
+}
+
 }  // namespace kvq

@@ -49,7 +49,7 @@ extern "C" {
 #endif
 
 #define KVQ_PAGE_SIZE 16
-#define KVQ_ABI_VERSION 4
+#define KVQ_ABI_VERSION 5
 
 typedef enum kvq_status {
   KVQ_OK = 0,
@@ -159,9 +159,17 @@ kvq_status kv_quant_write(const void* k, const void* v, const int64_t* slot_mapp
  * be queried.
  *
  * The workspace holds the per-split partial results (fp32, each word stored
- * bit-inverted so that a zero word means "not written yet"); it must be
+ * bit-inverted so that a zero word means "not written yet", plus one state
+ * word per row used to hand a merge over to another split); it must be
  * zero-filled before its first use, and every call leaves it zero-filled
- * again.
+ * again - except after a call whose bounded waits ran out (kvq_get_device_error
+ * returns KVQ_ERR_TIMEOUT): words that arrived after the wait gave up may
+ * remain, so clear the workspace before using it again.
+ *
+ * The split merge needs no co-residency of the launch's CTAs: a merger that
+ * waits long (about 0.2 ms) for a split that has not written hands its rows
+ * over to that split and exits, so a decode also completes when other
+ * streams' kernels hold most SMs.
  */
 size_t kvq_attn_workspace_size(const kvq_attn_desc* desc);
 
@@ -189,8 +197,9 @@ size_t kvq_attn_workspace_size(const kvq_attn_desc* desc);
  * out          : device, [B][Hq][D], fp32 or bf16 (desc->out_dtype).
  * workspace    : device, at least kvq_attn_workspace_size(desc) bytes, 16-byte
  *                aligned, zero-filled before its first use (each call leaves
- *                it zero-filled); may be NULL when that size is 0. Calls that
- *                overlap on the GPU must use different workspaces.
+ *                it zero-filled; after KVQ_ERR_TIMEOUT clear it again); may be
+ *                NULL when that size is 0. Calls that overlap on the GPU must
+ *                use different workspaces.
  * batch = 0 launches nothing and returns KVQ_OK (pointers may then be NULL).
  * Returns KVQ_OK, KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_WORKSPACE
  * or KVQ_ERR_CUDA.
@@ -281,14 +290,23 @@ kvq_status paged_prefill_attn_int4(const void* q, const uint8_t* cache,
  * fixed device array of KVQ_STATIC_WORKSPACE_BYTES inside this library (every
  * GPU that loads the library holds it until the process exits). The caller
  * still passes all inputs and outputs, exactly as for paged_decode_attn_int4.
- *  - The first call on a device looks up that array's device address (once
- *    per device); make that first call before any stream capture.
- *  - The array needs no clearing: each call overwrites what it reads.
+ *  - The first call on a device (and the first after that device's context
+ *    changed, e.g. after cudaDeviceReset) looks up that array's device
+ *    address; make that first call before any stream capture.
+ *  - The array starts zeroed and every call leaves it zeroed (each merge
+ *    clears the words it read). After a call whose bounded waits ran out,
+ *    kvq_get_device_error (which reports KVQ_ERR_TIMEOUT) clears the array on
+ *    that device with an asynchronous memset on its stream - nothing else
+ *    can, since callers cannot reach the array.
  *  - All calls share the one array per device: calls that overlap on the GPU
  *    (other streams, other host threads) race and give wrong results.
- *  - Shapes that would need more scratch than the array holds are rejected
- *    with KVQ_ERR_WORKSPACE before anything is launched. On a 148-SM B200 every
- *    accepted shape fits (the library uses at most ~1.9 MB).
+ *  - The uniform split plan needs up to resident CTAs x (query rows per CTA)
+ *    x (D + 4) x 4 bytes; shapes whose plan needs more than the array holds
+ *    are rejected with KVQ_ERR_WORKSPACE before anything is launched (on a
+ *    148-SM B200: up to 2.5 MB when 4 kv heads of GQA 4 share a CTA, so such
+ *    shapes are rejected; the benchmark's shapes need at most 0.6 MB). With
+ *    desc->context_lens_host, the per-sequence plan runs when its partials
+ *    fit, else the uniform plan.
  * No allocation of any kind is made. Returns the same statuses as
  * paged_decode_attn_int4.
  */
@@ -302,9 +320,20 @@ kvq_status paged_decode_attn_int4_static_ws(const void* q, const uint8_t* cache,
 /*
  * kvq_get_device_error - synchronizes `stream`, then returns and clears the
  * current device's error word (KVQ_OK when no kernel recorded an error).
+ * When the word is KVQ_ERR_TIMEOUT it also clears the static split-K array
+ * of paged_decode_attn_int4_static_ws on that device (a memset on `stream`,
+ * waited for), since late words may remain there.
  * Returns KVQ_ERR_CUDA if the synchronization itself fails.
  */
 kvq_status kvq_get_device_error(void* stream);
+
+/*
+ * kvq_static_workspace_nonzero - a test hook with no counterpart in the
+ * pages: the number of non-zero bytes in the static split-K array of
+ * paged_decode_attn_int4_static_ws on the current device (copied to the host,
+ * synchronously), or SIZE_MAX when it cannot be read.
+ */
+size_t kvq_static_workspace_nonzero(void);
 
 /*
  * kvq_set_device - make `device` this library's current CUDA device (the
@@ -327,6 +356,17 @@ kvq_status kvq_set_device(int32_t device);
  * KVQ_ERR_CUDA.
  */
 kvq_status kvq_selftest_bounded_wait(int32_t which, void* stream);
+
+/*
+ * kvq_selftest_occupy - a test hook with no counterpart in the pages: launch
+ * `ctas` CTAs (1..65535) on `stream`, each holding most of an SM's shared
+ * memory, that wait on the global timer for `microseconds` (0..1000000) and
+ * then end on their own. Tests use it to keep SMs busy while a decode runs on
+ * another stream. No hot-path call uses it.
+ * Returns KVQ_ERR_INVALID_ARG on out-of-range arguments, KVQ_ERR_CUDA when
+ * the launch fails.
+ */
+kvq_status kvq_selftest_occupy(int32_t ctas, int32_t microseconds, void* stream);
 
 /* Static, human-readable name of a status value (never NULL). */
 const char* kvq_status_string(int32_t status);

@@ -11,8 +11,8 @@ minimum), whole job over all ranks.
 
 L2 hygiene: the working sets rotate so no kernel reads data still resident in
 L2: two K/V input sets (134 MB each, larger than L2) alternate, and the decode
-of step i reads the cache written at step i-2 (four cache pools), with more
-than 300 MB of traffic in between.
+of step i reads the cache written at step i-2 (six cache pools, 214 MB in
+all), with more than 300 MB of traffic in between.
 
 Besides the step, the JSON line carries:
   - each kernel timed alone, and a roofline object for each;
@@ -63,6 +63,10 @@ def parse_args(argv=None):
     ap.add_argument("--only", choices=["write", "decode", "prefill"], default=None,
                     help="time one kernel alone (profiling captures); prints its line")
     ap.add_argument("--e2e-steps", type=int, default=100)
+    ap.add_argument("--no-configs", action="store_true",
+                    help="skip the other workloads' write and decode lines")
+    ap.add_argument("--launch-check", action="store_true",
+                    help="start the ranks, count them over gloo on the CPU and print n_gpus (no GPU work)")
     return ap.parse_args(argv)
 
 
@@ -329,7 +333,7 @@ class Step:
     serving loop does with its decode step), so the host's launch rate never
     gates the GPU: the kernels run back to back exactly as launched."""
 
-    N_POOLS = 4
+    N_POOLS = 6
 
     def __init__(self, w, block, dev, graph=True, signs=None):
         import ctypes
@@ -497,20 +501,24 @@ class Step:
         t1.synchronize()
         return t0.elapsed_time(t1)
 
-    def run_ms(self, kinds, steps, start_index=0):
+    def run_ms(self, kinds, steps, start_index=0, rounds=1):
+        """Device ms of `steps` steps of `kinds`: the median of `rounds`
+        measurements (replays of one captured graph, or direct launches)."""
         if not self.graph:
-            return self.direct_ms(kinds, steps, start_index)
-        return self.replay_ms(self.capture(kinds, steps, start_index))
+            return statistics.median(self.direct_ms(kinds, steps, start_index) for _ in range(rounds))
+        g = self.capture(kinds, steps, start_index)
+        return statistics.median(self.replay_ms(g) for _ in range(rounds))
 
-    def timed_only(self, kind, steps, start_index=0):
+    def timed_only(self, kind, steps, start_index=0, rounds=1):
         """One kernel alone, `steps` back-to-back launches (inputs and outputs
-        rotate through sets larger than L2). Returns the average ms per launch."""
-        return self.run_ms((kind,), steps, start_index) / steps
+        rotate through sets larger than L2). Returns the average ms per launch
+        (median of `rounds` measurements)."""
+        return self.run_ms((kind,), steps, start_index, rounds) / steps
 
-    def timed(self, steps, start_index=0):
+    def timed(self, steps, start_index=0, rounds=3):
         """`steps` whole steps (write, then decode) back to back. Returns the
-        total ms."""
-        return self.run_ms(("write", "decode"), steps, start_index)
+        total ms (median of `rounds` measurements)."""
+        return self.run_ms(("write", "decode"), steps, start_index, rounds)
 
 
 def e2e_run(w, block, dev, steps, warmup):
@@ -581,9 +589,22 @@ def oracle_sample(w, block, n_tokens):
     return dt, nbytes
 
 
-def cpu_baseline(w, block, n_tokens=32768, min_seconds=10.0, max_passes=20):
+def cpu_model():
+    """The host CPU's model name (lscpu), or None."""
+    try:
+        out = subprocess.run(["lscpu"], capture_output=True, text=True, timeout=10).stdout
+    except (OSError, subprocess.SubprocessError):
+        return None
+    for line in out.splitlines():
+        if line.strip().startswith("Model name:"):
+            return line.split(":", 1)[1].strip()
+    return None
+
+
+def cpu_baseline(w, block, n_tokens=32768, min_seconds=10.0, max_passes=20, single_tokens=2048):
     """The oracle on a bounded sample of the workload, repeated until it has
-    run for `min_seconds` (at most `max_passes` passes)."""
+    run for `min_seconds` (at most `max_passes` passes), on all host cores;
+    then once on a smaller sample with one thread."""
     import oracle
     passes, total_t, total_b = 0, 0.0, 0
     while passes < max_passes and total_t < min_seconds:
@@ -591,11 +612,21 @@ def cpu_baseline(w, block, n_tokens=32768, min_seconds=10.0, max_passes=20):
         passes += 1
         total_t += dt
         total_b += nbytes
-    return {"value": round(total_b / total_t / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(),
-            "kind": "oracle",
+    cores = oracle.num_threads()
+    oracle.set_num_threads(1)
+    try:
+        dt1, nb1 = oracle_sample(w, block, single_tokens)
+    finally:
+        oracle.set_num_threads(cores)
+    n1 = min(single_tokens, w.tokens_written)
+    return {"value": round(total_b / total_t / 1e9, 4), "unit": "GB/s", "cores": cores,
+            "kind": "oracle", "cpu_model": cpu_model(),
             "sample": f"{passes} passes of: write of the first {min(n_tokens, w.tokens_written)} tokens "
                       f"(all kv heads, K and V) + one decode step of all {w.Hq} query heads over them; "
-                      f"{total_t:.1f} s in all"}
+                      f"{total_t:.1f} s in all",
+            "single_thread": {"value": round(nb1 / dt1 / 1e9, 5), "unit": "GB/s", "cores": 1,
+                              "sample": f"write of the first {n1} tokens + one decode step over them; "
+                                        f"{dt1:.1f} s"}}
 
 
 REFERENCE_BUDGET_S = 120.0
@@ -653,8 +684,95 @@ def config_block(w, block, graph=True):
 
 
 # ----------------------------------------------------------------------------
+# the other workloads: each kernel alone, at each Hadamard block and plain
+# ----------------------------------------------------------------------------
+
+SWEEP = (("serving-b64", None), ("llama2-70b-b8", None), ("stress-b256", (32, 64, 128)))
+
+
+def config_sweep(dev, steps, warm, rank, world, max_over_ranks):
+    """For every other workload: kv_quant_write and paged_decode_attn_int4
+    alone (graph replays of `steps` back-to-back launches, median of 3), at
+    its Hadamard block(s) and at 0 (plain INT4), with GB/s, the fraction of
+    the HBM peak and the rotation overhead."""
+    import torch
+    from bit_kv_cache_20_b200 import workloads
+    peak, _ = measured_peaks()
+    out = {}
+    for name, blocks in SWEEP:
+        cfg = workloads.CONFIGS[name]
+        w = workloads.make(name, seed=rank_seed(cfg.seed, rank))
+        blocks = tuple(blocks or (w.block,))
+        wb = write_bytes(w.tokens_written, w.Hkv, w.D)
+        db = decode_bytes(w.context_lens, w.B, w.Hq, w.Hkv, w.D, out_elem=2)
+        times = {}
+        for b in (0,) + blocks:
+            st = Step(w, b, dev, graph=True)
+            st.fill_pools()
+            st.timed_only("write", warm)
+            st.timed_only("decode", warm)
+            wr = max_over_ranks(st.timed_only("write", steps, start_index=warm, rounds=3))
+            de = max_over_ranks(st.timed_only("decode", steps, start_index=warm, rounds=3))
+            times[b] = (wr, de)
+            del st
+            torch.cuda.empty_cache()
+
+        def line(b):
+            wr, de = times[b]
+            w_gbs, d_gbs = wb * world / (wr / 1e3) / 1e9, db * world / (de / 1e3) / 1e9
+            entry = {"write_us": round(1e3 * wr, 2), "write_GB/s": round(w_gbs, 1),
+                     "write_frac": round(w_gbs / (peak * world), 4),
+                     "decode_us": round(1e3 * de, 2), "decode_GB/s": round(d_gbs, 1),
+                     "decode_frac": round(d_gbs / (peak * world), 4)}
+            if b != 0:
+                entry["rotation_overhead"] = {"kv_quant_write": round(wr / times[0][0] - 1, 4),
+                                              "paged_decode_attn_int4": round(de / times[0][1] - 1, 4)}
+            return entry
+
+        out[name] = {"batch": w.B, "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D,
+                     "context_tokens": int(w.context_lens.sum()), "written_tokens": w.tokens_written,
+                     "write_bytes": wb, "decode_bytes": db,
+                     "blocks": {str(b): line(b) for b in (0,) + blocks}}
+        del w
+    return out
+
+
+# ----------------------------------------------------------------------------
 # main
 # ----------------------------------------------------------------------------
+
+def free_port():
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def launch_local_ranks(n, argv):
+    """`python bench.py --gpus N` without torchrun: start N ranks of this
+    script on this node (RANK / LOCAL_RANK / WORLD_SIZE / MASTER_* set), one
+    per GPU; rank 0 prints the line. Returns the worst exit code."""
+    env = dict(os.environ, WORLD_SIZE=str(n), MASTER_ADDR="127.0.0.1", MASTER_PORT=str(free_port()))
+    procs = [subprocess.Popen([sys.executable, os.path.abspath(__file__)] + list(argv),
+                              env=dict(env, RANK=str(r), LOCAL_RANK=str(r))) for r in range(n)]
+    return max(p.wait() for p in procs)
+
+
+def launch_check(rank, world):
+    """Count the ranks over gloo (CPU) and print what the line would report."""
+    import datetime
+    import torch
+    import torch.distributed as dist
+    t = torch.ones(1)
+    if world > 1:
+        dist.init_process_group("gloo", timeout=datetime.timedelta(seconds=60))
+        dist.all_reduce(t)
+    if rank == 0:
+        print(json.dumps({"launch_check": True, "n_gpus": world, "ranks_seen": int(t.item())}), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
 
 def reduce_max(x, world, device):
     """Max of a per-rank scalar over all ranks (the job's time is the slowest
@@ -669,10 +787,15 @@ def reduce_max(x, world, device):
 
 
 def main(argv=None):
+    argv = sys.argv[1:] if argv is None else list(argv)
     args = parse_args(argv)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        return launch_local_ranks(args.gpus, argv)
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.launch_check:
+        return launch_check(rank, world)
     if args.impl == "reference":
         if rank == 0:
             print(json.dumps(run_reference(args)), flush=True)
@@ -785,6 +908,10 @@ def main(argv=None):
         p_de_ms = max_over_ranks(statistics.median(ms["p_decode"]))
         plain = {
             "hadamard_block": 0,
+            "kernels": {"kv_quant_write": "kvq_write_kernel<D> (CUDA cores, no rotation) vs the rotated "
+                                          "kvq_write_tc_kernel<D, b> (tcgen05 rotation)",
+                        "paged_decode_attn_int4": "kvq_decode_kernel with b = 0 (the same template, "
+                                                  "rotations compiled out)"},
             "kv_quant_write_us": round(1e3 * p_wr_ms, 3),
             "paged_decode_attn_int4_us": round(1e3 * p_de_ms, 3),
             "ms_per_step": round(p_total / args.steps, 5),
@@ -811,6 +938,12 @@ def main(argv=None):
     # chunked prefill (a row beside the step, not part of it): a few launches
     pf_ms, pf_flops = prefill_run(step, 3, 1)
     pf_ms = max_over_ranks(pf_ms)
+    del step
+
+    # the other workloads, each kernel alone (not part of the step)
+    configs = None
+    if not args.no_configs:
+        configs = config_sweep(dev, min(args.steps, 50), warm, rank, world, max_over_ranks)
 
     e2e = None
     if not args.no_e2e:
@@ -861,6 +994,7 @@ def main(argv=None):
             "fused_us": round(1e3 * ap_fus_ms, 3),     # paged_decode_append_attn_int4
         },
         "prefill": prefill_line(pf_ms, pf_flops * world),
+        "configs": configs,
         "e2e": e2e,
         "clocks": clocks.summary(),
         "gpu_launches": 2 * args.steps,

@@ -123,9 +123,9 @@ int resident_ctas(K kernel, std::atomic<int>* cache, int dev, int threads, int s
 // ---------------------------------------------------------------------------
 // kv_quant_write
 // ---------------------------------------------------------------------------
-template <int D, int BLK>
+template <int D>
 kvq_status launch_write(const kvq::WriteParams& p, int dev, cudaStream_t s) {
-  auto kern = kvq::kvq_write_kernel<D, BLK>;
+  auto kern = kvq::kvq_write_kernel<D>;
   constexpr int smem = kvq::write_smem_bytes<D>();
   const int threads = kvq::kWriteWarps * 32;
   static std::atomic<int> occ[kMaxDevices];
@@ -205,7 +205,7 @@ kvq_status launch_write_tc(const kvq::WriteParams& p, int dev, cudaStream_t s) {
 template <int D>
 kvq_status dispatch_write(const kvq::WriteParams& p, int b, int dev, cudaStream_t s) {
   switch (b) {
-    case 0: return launch_write<D, 0>(p, dev, s);
+    case 0: return launch_write<D>(p, dev, s);
     case 32: return launch_write_tc<D, 32>(p, dev, s);
     case 64: return launch_write_tc<D, 64>(p, dev, s);
     case 128:

@@ -1,18 +1,19 @@
-// kvq_write.cuh - fused rotation + token-wise INT4 quantization + paged store.
+// kvq_write.cuh - token-wise INT4 quantization + paged store without a
+// rotation: kv_quant_write with hadamard_block = 0 (plain INT4, the
+// comparator of the rotated path). The rotated write (b = 32/64/128) is the
+// tensor-core kernel in kvq_write_tc.cuh.
 //
-// SAW-INT4 (Abstract): a single kernel rotates, quantizes and stores each
-// row straight into the paged cache; OScaR (forum summary, "The OScaR
-// Framework"): rotate first, then quantize.
+// SAW-INT4 (Abstract): one scale per token, codes stored straight into the
+// paged cache by the kernel that quantizes them.
 //
 // Work unit: a warp tile = 32 consecutive tokens of one (kv head, K|V). One
-// thread owns one row (token, head, K|V) of D values, so the whole Hadamard
-// block, the row min/max and the packing stay in the thread's registers - no
-// shuffles. Input rows arrive through cp.async into a per-warp shared buffer
-// with an XOR swizzle on 16-byte chunks (conflict-free row reads); the copy of
-// tile i+1 is issued before tile i is computed. The arithmetic runs on packed
-// fp32 pairs (sm_100 f32x2: one issue slot per two lanes) where it can:
-// butterflies, the 1/sqrt(b) scaling, y - z and the rounding fma. Packed rows
-// (D/2 bytes) and the fp16 s, z go straight to their slot.
+// thread owns one row (token, head, K|V) of D values, so the row min/max and
+// the packing stay in the thread's registers - no shuffles. Input rows arrive
+// through cp.async into a per-warp shared buffer with an XOR swizzle on
+// 16-byte chunks (conflict-free row reads); the copy of tile i+1 is issued
+// before tile i is computed. The arithmetic runs on packed fp32 pairs (sm_100
+// f32x2: one issue slot per two lanes) where it can: y - z and the rounding
+// fma. Packed rows (D/2 bytes) and the fp16 s, z go straight to their slot.
 #pragma once
 
 #include "kvq_device.cuh"
@@ -41,36 +42,7 @@ __host__ __device__ constexpr int write_smem_bytes() {
   return kWriteWarps * 32 * D * 2;
 }
 
-// In-register fast Walsh-Hadamard transform of each contiguous BLK block of a
-// row held as D/2 packed pairs (x[2i], x[2i+1]); Sylvester natural order:
-// y_i = sum_j (-1)^popcount(i&j) x_j. The distance-1 stage pairs the two
-// halves of one register (scalar ops); every other stage pairs whole
-// registers (f32x2 add/sub).
-template <int D, int BLK>
-__device__ __forceinline__ void fwht_pairs(uint64_t (&xp)[D / 2]) {
-#pragma unroll
-  for (int i = 0; i < D / 2; ++i) {
-    float a, b;
-    f2_unpack(xp[i], a, b);
-    xp[i] = f2_pack(__fadd_rn(a, b), __fsub_rn(a, b));
-  }
-#pragma unroll
-  for (int base = 0; base < D / 2; base += BLK / 2) {
-#pragma unroll
-    for (int len = 1; len < BLK / 2; len <<= 1) {
-#pragma unroll
-      for (int i = 0; i < BLK / 2; ++i) {
-        if ((i & len) == 0) {
-          const uint64_t A = xp[base + i], B = xp[base + i + len];
-          xp[base + i] = f2_add(A, B);
-          xp[base + i + len] = f2_sub(A, B);
-        }
-      }
-    }
-  }
-}
-
-template <int D, int BLK>
+template <int D>
 __global__ void __launch_bounds__(kWriteWarps * 32, 3) kvq_write_kernel(const WriteParams p) {
   constexpr int ROWB = D * 2;       // bytes per bf16 input row
   constexpr int CPR = ROWB / 16;    // 16-byte chunks per row (8 or 16)
@@ -101,7 +73,6 @@ __global__ void __launch_bounds__(kWriteWarps * 32, 3) kvq_write_kernel(const Wr
     cp_async_commit();
   };
 
-  const uint64_t cb2 = f2_pack(p.cb, p.cb);
   const uint64_t magic2 = f2_pack(8388608.0f, 8388608.0f);
 
   if (tile < p.num_tiles) issue(tile);
@@ -126,13 +97,7 @@ __global__ void __launch_bounds__(kWriteWarps * 32, 3) kvq_write_kernel(const Wr
     __syncwarp();
     if (tile + nw < p.num_tiles) issue(tile + nw);
 
-    // 1. rotation y = (H_b x) * fp32(1/sqrt(b))
-    if constexpr (BLK > 0) {
-      fwht_pairs<D, BLK>(xp);
-#pragma unroll
-      for (int i = 0; i < D / 2; ++i) xp[i] = f2_mul(xp[i], cb2);
-    }
-    // 2. row min / max (four independent 3-input chains each)
+    // 1. row min / max (y = x: no rotation) (four independent 3-input chains each)
     float mn4[4], mx4[4];
 #pragma unroll
     for (int q = 0; q < 4; ++q) {
@@ -149,7 +114,7 @@ __global__ void __launch_bounds__(kWriteWarps * 32, 3) kvq_write_kernel(const Wr
     }
     const float mn = fminf(fminf(mn4[0], mn4[1]), fminf(mn4[2], mn4[3]));
     const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
-    // 3. z = largest fp16 <= mn; s = smallest fp16 with 15 s + z >= mx.
+    // 2. z = largest fp16 <= mn; s = smallest fp16 with 15 s + z >= mx.
     //    Directed roundings give a candidate at most one fp16 step high; the
     //    exact test (fp64: 15 s + z is exact there) settles it.
     const __half zh = __float2half_rd(mn);
@@ -163,7 +128,7 @@ __global__ void __launch_bounds__(kWriteWarps * 32, 3) kvq_write_kernel(const Wr
     }
     const float sf = __half2float(__ushort_as_half(sb));
     const float inv = (sf > 0.0f) ? __frcp_rn(sf) : 0.0f;
-    // 4. code = rint(fp32(y - z) * fp32(1/s)): adding 2^23 inside one fma
+    // 3. code = rint(fp32(y - z) * fp32(1/s)): adding 2^23 inside one fma
     //    rounds the exact product to an integer (ties to even), leaving the
     //    code in the low 4 bits of the result (above them: the constant
     //    exponent of 2^23). Eight such words shifted by 4i and summed give the
@@ -185,7 +150,7 @@ __global__ void __launch_bounds__(kWriteWarps * 32, 3) kvq_write_kernel(const Wr
       }
       packed[wd] = acc;
     }
-    // 5. paged store
+    // 4. paged store
     if (slot >= 0 && slot < p.num_slots) {
       const long long page = slot >> 4;
       const int off = (int)(slot & 15);

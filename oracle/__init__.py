@@ -80,6 +80,7 @@ def lib():
                                            c_int, c_int, c_int, c_int, c_int, ctypes.c_void_p, c_int,
                                            c_i64, c_d, _p(f64)]),
             "oracle_num_threads": (c_int, []),
+            "oracle_set_num_threads": (None, [c_int]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -306,3 +307,8 @@ def decode_one(q_bits, cache, scales, zeros, page_table, context_lens, n: int, h
 
 def num_threads() -> int:
     return lib().oracle_num_threads()
+
+
+def set_num_threads(n: int) -> None:
+    """Threads of the oracle's OpenMP loops from now on (timing legs only)."""
+    lib().oracle_set_num_threads(int(n))

@@ -92,3 +92,19 @@ def test_reference_arm_prints_one_contract_line(monkeypatch, capsys):
     assert d["cpu_baseline"]["kind"] == "oracle" and d["cpu_baseline"]["value"] == d["value"]
     assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
     assert d["config"]["workload"] == "tiny"
+
+
+def test_bench_gpus_n_starts_n_ranks():
+    """`python bench.py --gpus 2` with no torchrun starts two ranks itself;
+    with --launch-check they count themselves over gloo on the CPU and rank 0
+    prints the n_gpus the line would report."""
+    import json
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = {k: v for k, v in os.environ.items() if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK")}
+    out = subprocess.run([sys.executable, os.path.join(root, "bench.py"), "--gpus", "2", "--launch-check"],
+                         capture_output=True, text=True, timeout=120, env=env, check=True).stdout
+    lines = [json.loads(l) for l in out.splitlines() if l.startswith("{")]
+    assert len(lines) == 1, out
+    assert lines[0]["n_gpus"] == 2 and lines[0]["ranks_seen"] == 2

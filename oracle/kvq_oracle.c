@@ -19,9 +19,11 @@
  *    Sylvester Hadamard matrix in natural order, no random signs; b = 0 = I.
  *  - one (s, z) pair per row = (token, kv head, K or V) over all D channels.
  *  - z = largest fp16 <= min(y); s = smallest fp16 >= 0 with 15 s + z >= max(y).
- *  - code = round-half-even((y - z) / s), the exact quotient (fp64 holds it
- *    to far below the 1e-6 boundary band the acceptance allows); s = 0 gives
- *    code 0.
+ *  - code = round-half-even(fp32(y - z) * fp32(1/s)); s = 0 gives code 0.
+ *    (The pages fix no rounding rule for this step; with bf16 inputs the
+ *    exact quotient often lands exactly on a half-integer, where the rule
+ *    decides, so the rule is stated here and computed in fp64 from those
+ *    two fp32 operands.)
  *  - byte j of a packed row = code[2j] | code[2j+1] << 4.
  *  - cache [page][Hkv][2][16][D/2], scales/zeros [page][Hkv][2][16].
  *  - attention: softmax_scale defaults to 1/sqrt(D); out = R sum_t p_t v^_t.
@@ -225,28 +227,32 @@ void oracle_scale_zero(float mn, float mx, uint16_t* s_out, uint16_t* z_out) {
   *z_out = z;
 }
 
-/* The quotient (y - z) / s of each element for a given (s, z), in fp64 (y is
- * an fp32 value, s and z fp16 values: y - z is exact in fp64 and the division
- * rounds once, far below any rounding boundary band); 0 when s = 0. */
-void oracle_quotient_given(const float* y, int D, uint16_t s, uint16_t z, double* qout) {
-  const double sd = oracle_half_to_double(s);
-  const double zd = oracle_half_to_double(z);
-  for (int c = 0; c < D; ++c) qout[c] = (sd > 0.0) ? ((double)y[c] - zd) / sd : 0.0;
+/* Codes of a row for a given (s, z): code = round-half-even(t * inv) with
+ * t = fp32(y - z) and inv = fp32(1/s); the product of two fp32 values is
+ * exact in fp64, so rint() on it is the one rounding. Clamped to [0, 15]. */
+void oracle_quantize_given(const float* y, int D, uint16_t s, uint16_t z, uint8_t* codes) {
+  float sf = (float)oracle_half_to_double(s);
+  float zf = (float)oracle_half_to_double(z);
+  float inv = (sf > 0.0f) ? 1.0f / sf : 0.0f;
+  for (int c = 0; c < D; ++c) {
+    float t = y[c] - zf;
+    double q = (double)t * (double)inv;
+    double r = nearbyint(q); /* default rounding mode: ties to even */
+    if (r < 0) r = 0;
+    if (r > 15) r = 15;
+    codes[c] = (uint8_t)r;
+  }
 }
 
-/* Codes of a row for a given (s, z): code = round-half-even((y - z) / s),
- * clamped to [0, 15]. */
-void oracle_quantize_given(const float* y, int D, uint16_t s, uint16_t z, uint8_t* codes) {
-  double q[128];
-  for (int c0 = 0; c0 < D; c0 += 128) {
-    const int n = (D - c0) < 128 ? (D - c0) : 128;
-    oracle_quotient_given(y + c0, n, s, z, q);
-    for (int c = 0; c < n; ++c) {
-      double r = nearbyint(q[c]); /* default rounding mode: ties to even */
-      if (r < 0) r = 0;
-      if (r > 15) r = 15;
-      codes[c0 + c] = (uint8_t)r;
-    }
+/* The quotient fp32(y - z) * fp32(1/s) itself, for classifying elements that
+ * sit next to a rounding boundary. */
+void oracle_quotient_given(const float* y, int D, uint16_t s, uint16_t z, double* qout) {
+  float sf = (float)oracle_half_to_double(s);
+  float zf = (float)oracle_half_to_double(z);
+  float inv = (sf > 0.0f) ? 1.0f / sf : 0.0f;
+  for (int c = 0; c < D; ++c) {
+    float t = y[c] - zf;
+    qout[c] = (double)t * (double)inv;
   }
 }
 

@@ -54,31 +54,22 @@ def f16_bits_to_float(bits):
     return _np.asarray(bits, _np.uint16).view(_np.float16).astype(_np.float64)
 
 
-# The kernel decides a code from fp32(y - z) and fp32(1/s) (two roundings of
-# at most 2^-24 relative on a quotient of at most 15: < 2^-19.1 code units);
-# the oracle from the exact quotient. Both lie within 2^-18 code units of
-# each other - inside the benchmark spec's band, which at 1e-6 of the row's largest
-# magnitude (>= 7.5 s) is at least 7.5e-6 code units.
-QUOTIENT_BAND = 2.0 ** -18
-
-
 def write_window(x_rows, b, s_bits):
     """Per-row width (in code units) of the band around a rounding boundary in
-    which the kernel may legitimately land on the other code than the
-    oracle's exact quotient of its once-rounded fp64 rotation: the quotient
-    band, plus for b > 0 the fp32 butterfly's rounding error bound
-    (log2(b) + 1 roundings of at most 2^-24 times the block's sum of |x|,
-    times 1/sqrt(b)) divided by the step s. With b = 0 the rotated row is
-    the bf16 input itself on both sides, so only the quotient band remains."""
+    which the kernel's fp32 butterfly may legitimately land on the other code
+    than the oracle's once-rounded fp64 rotation: the butterfly's rounding
+    error bound (log2(b) + 1 roundings of at most 2^-24 times the block's sum
+    of |x|, times 1/sqrt(b)), divided by the step s. Zero when b = 0: then
+    the rotated row is the bf16 input itself on both sides."""
     if b == 0:
-        return _np.full(x_rows.shape[0], QUOTIENT_BAND)
+        return _np.zeros(x_rows.shape[0])
     n, D = x_rows.shape
     blocks = _np.abs(x_rows).reshape(n, D // b, b).sum(axis=2).max(axis=1)
     bound_y = (_math.log2(b) + 2) * 2.0 ** -24 * blocks / _math.sqrt(b)
     s = f16_bits_to_float(s_bits)
     with _np.errstate(divide="ignore", invalid="ignore"):
         w = _np.where(s > 0, bound_y / s, 0.0)
-    return w + QUOTIENT_BAND
+    return w + 2.0 ** -19
 
 
 def compare_write_rows(orc, y_oracle, x_rows, b, gpu_packed, gpu_s, gpu_z, D):

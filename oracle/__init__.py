@@ -81,6 +81,23 @@ def lib():
                                            c_i64, c_d, _p(f64)]),
             "oracle_num_threads": (c_int, []),
             "oracle_set_num_threads": (None, [c_int]),
+            "oracle_scale_zero_levels": (None, [ctypes.c_float, ctypes.c_float, c_int,
+                                                ctypes.POINTER(ctypes.c_uint16),
+                                                ctypes.POINTER(ctypes.c_uint16)]),
+            "oracle_oscar_token_norm": (ctypes.c_uint16, [_p(f32), c_int, _p(f32)]),
+            "oracle_oscar_quant_channels": (None, [_p(f32), c_int, _p(u8), _p(u16), _p(u16)]),
+            "oracle_oscar_quant_page": (c_int, [_p(u16), _p(u16), c_int, c_int, _p(u8), _p(u8), _p(u16),
+                                                _p(u16), _p(u16), _p(u16), _p(u16)]),
+            "oracle_oscar_write": (c_int, [_p(u16), _p(u16), _p(i32), c_int, c_int, c_int, c_int, c_i64,
+                                           _p(u8), _p(u16), _p(u16)]),
+            "oracle_oscar_dequant_page": (None, [_p(u8), _p(u16), _p(u16), c_i64, c_int, c_int, c_int,
+                                                 _p(f64), _p(f64)]),
+            "oracle_oscar_decode_one": (c_int, [_p(u16), _p(u8), _p(u16), _p(u16), _p(i32), _p(i32),
+                                                _p(u16), _p(u16), c_int, c_int, c_int, c_int, c_int, c_int,
+                                                c_int, c_i64, c_d, _p(f64)]),
+            "oracle_oscar_decode_attn": (c_int, [_p(u16), _p(u8), _p(u16), _p(u16), _p(i32), _p(i32),
+                                                 _p(u16), _p(u16), c_int, c_int, c_int, c_int, c_int, c_int,
+                                                 c_i64, c_d, _p(f64)]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -312,3 +329,110 @@ def num_threads() -> int:
 def set_num_threads(n: int) -> None:
     """Threads of the oracle's OpenMP loops from now on (timing legs only)."""
     lib().oracle_set_num_threads(int(n))
+
+
+# --- OScaR (forum summary, "The OScaR Framework": V^ = Quant(S (R V))) -------
+
+OSCAR_TOP = 3  # INT2 codes 0..3
+
+
+def scale_zero_levels(mn: float, mx: float, top: int):
+    """(s, z) fp16 bits: z = largest fp16 <= mn, s = smallest fp16 >= 0 with
+    top * s + z >= mx."""
+    s_, z_ = ctypes.c_uint16(), ctypes.c_uint16()
+    lib().oracle_scale_zero_levels(float(mn), float(mx), int(top), ctypes.byref(s_), ctypes.byref(z_))
+    return int(s_.value), int(z_.value)
+
+
+def oscar_token_norm(y):
+    """(n fp16 bits, u fp32 row): the Omni-Token factor of a rotated row."""
+    y = _c(y, np.float32)
+    u = np.zeros_like(y)
+    n = lib().oracle_oscar_token_norm(y, y.size, u)
+    return int(n), u
+
+
+def oscar_quant_channels(u):
+    """Per-channel INT2 quantization of 16 normalized rows u (fp32 [16, D]):
+    (codes uint8 [16, D/4], ks, kz fp16 bits [D])."""
+    u = _c(u, np.float32)
+    D = u.shape[1]
+    codes = np.zeros((16, D // 4), np.uint8)
+    ks = np.zeros(D, np.uint16)
+    kz = np.zeros(D, np.uint16)
+    lib().oracle_oscar_quant_channels(u.reshape(-1), D, codes.reshape(-1), ks, kz)
+    return codes, ks, kz
+
+
+def oscar_quant_page(k_bits, v_bits, b: int):
+    """One page-head: k_bits, v_bits uint16 [16, D] (bf16). Returns a dict of
+    kcodes, vcodes (uint8 [16, D/4]), ks, kz (fp16 bits [D]), kn, vs, vz
+    (fp16 bits [16])."""
+    k = _c(k_bits, np.uint16)
+    v = _c(v_bits, np.uint16)
+    D = k.shape[1]
+    out = {"kcodes": np.zeros((16, D // 4), np.uint8), "vcodes": np.zeros((16, D // 4), np.uint8),
+           "ks": np.zeros(D, np.uint16), "kz": np.zeros(D, np.uint16), "kn": np.zeros(16, np.uint16),
+           "vs": np.zeros(16, np.uint16), "vz": np.zeros(16, np.uint16)}
+    rc = lib().oracle_oscar_quant_page(k.reshape(-1), v.reshape(-1), D, b, out["kcodes"].reshape(-1),
+                                       out["vcodes"].reshape(-1), out["ks"], out["kz"], out["kn"], out["vs"],
+                                       out["vz"])
+    assert rc == 0, rc
+    return out
+
+
+def oscar_alloc(num_pages: int, Hkv: int, D: int):
+    """Zeroed host OScaR pool: cache uint8 [pages][Hkv][2][16][D/4], kmeta
+    fp16 bits [pages][Hkv][2][D] (K per-channel s, z), tmeta fp16 bits
+    [pages][Hkv][3][16] (K token norm, V s, V z)."""
+    return (np.zeros((num_pages, Hkv, 2, 16, D // 4), np.uint8), np.zeros((num_pages, Hkv, 2, D), np.uint16),
+            np.zeros((num_pages, Hkv, 3, 16), np.uint16))
+
+
+def oscar_write(k_bits, v_bits, page_ids, num_pages: int, b: int, pool=None):
+    """Token group g (rows 16 g .. 16 g + 15 of k_bits, v_bits: uint16
+    [T, Hkv, D]) fills page page_ids[g]. Returns (cache, kmeta, tmeta)."""
+    k = _c(k_bits, np.uint16)
+    v = _c(v_bits, np.uint16)
+    T, Hkv, D = k.shape
+    ids = _c(page_ids, np.int32)
+    assert T == 16 * ids.size
+    cache, kmeta, tmeta = pool if pool is not None else oscar_alloc(num_pages, Hkv, D)
+    rc = lib().oracle_oscar_write(k.reshape(-1), v.reshape(-1), ids, ids.size, Hkv, D, b, num_pages,
+                                  cache.reshape(-1), kmeta.reshape(-1), tmeta.reshape(-1))
+    if rc != 0:
+        raise ValueError(f"oracle_oscar_write returned {rc}")
+    return cache, kmeta, tmeta
+
+
+def oscar_dequant_page(cache, kmeta, tmeta, page: int, h: int):
+    """Dequantized rotated K, V rows [16, D] (fp64) of one page-head."""
+    P, Hkv, _, _, Dq = cache.shape
+    D = 4 * Dq
+    K = np.zeros((16, D), np.float64)
+    V = np.zeros((16, D), np.float64)
+    lib().oracle_oscar_dequant_page(_c(cache, np.uint8).reshape(-1), _c(kmeta, np.uint16).reshape(-1),
+                                    _c(tmeta, np.uint16).reshape(-1), page, Hkv, D, h, K.reshape(-1),
+                                    V.reshape(-1))
+    return K, V
+
+
+def oscar_decode_attn(q_bits, cache, kmeta, tmeta, page_table, context_lens, k_tail_bits, v_tail_bits,
+                      b: int, softmax_scale: float = 0.0) -> np.ndarray:
+    """The OScaR decode: full pages from the INT2 pool, the last ctx % 16
+    tokens of each sequence from k_tail / v_tail (uint16 [B, Hkv, 16, D]
+    bf16). Returns fp64 [B, Hq, D]."""
+    q = _c(q_bits, np.uint16)
+    B, Hq, D = q.shape
+    P, Hkv = cache.shape[0], cache.shape[1]
+    pt = _c(page_table, np.int32)
+    out = np.zeros((B, Hq, D), np.float64)
+    rc = lib().oracle_oscar_decode_attn(q.reshape(-1), _c(cache, np.uint8).reshape(-1),
+                                        _c(kmeta, np.uint16).reshape(-1), _c(tmeta, np.uint16).reshape(-1),
+                                        pt.reshape(-1), _c(context_lens, np.int32),
+                                        _c(k_tail_bits, np.uint16).reshape(-1),
+                                        _c(v_tail_bits, np.uint16).reshape(-1), B, Hq, Hkv, D, b, pt.shape[1],
+                                        P, float(softmax_scale), out.reshape(-1))
+    if rc != 0:
+        raise ValueError(f"oracle_oscar_decode_attn returned {rc}")
+    return out

@@ -215,16 +215,22 @@ int oracle_rotate_row(const uint16_t* x_bf16, int D, int b, float* y) {
 
 /* z = largest fp16 <= mn; s = smallest fp16 >= 0 with 15 s + z >= mx.
  * 15 s + z is exact in fp64 (both are binary16 values), so the test is exact. */
-void oracle_scale_zero(float mn, float mx, uint16_t* s_out, uint16_t* z_out) {
+/* z = largest fp16 <= mn; s = smallest fp16 >= 0 with top * s + z >= mx,
+ * top the largest code (15 for INT4, 3 for INT2). */
+void oracle_scale_zero_levels(float mn, float mx, int top, uint16_t* s_out, uint16_t* z_out) {
   uint16_t z = oracle_half_round_down((double)mn);
   double zd = oracle_half_to_double(z);
-  double need = ((double)mx - zd) / 15.0;
+  double need = ((double)mx - zd) / (double)top;
   uint16_t s = (need <= 0.0) ? 0 : oracle_half_round_up(need);
   /* settle the candidate on the exact condition, in either direction */
-  while (s < 0x7C00 && 15.0 * oracle_half_to_double(s) + zd < (double)mx) s = (uint16_t)(s + 1);
-  while (s > 0 && 15.0 * oracle_half_to_double((uint16_t)(s - 1)) + zd >= (double)mx) s = (uint16_t)(s - 1);
+  while (s < 0x7C00 && top * oracle_half_to_double(s) + zd < (double)mx) s = (uint16_t)(s + 1);
+  while (s > 0 && top * oracle_half_to_double((uint16_t)(s - 1)) + zd >= (double)mx) s = (uint16_t)(s - 1);
   *s_out = s;
   *z_out = z;
+}
+
+void oracle_scale_zero(float mn, float mx, uint16_t* s_out, uint16_t* z_out) {
+  oracle_scale_zero_levels(mn, mx, 15, s_out, z_out);
 }
 
 /* Codes of a row for a given (s, z): code = round-half-even(t * inv) with
@@ -459,4 +465,217 @@ void oracle_set_num_threads(int n) {
 #else
   (void)n;
 #endif
+}
+
+/* ------------------------------------------------------------------------- */
+/* OScaR (forum summary, "The OScaR Framework": V^ = Quant(S (R V)); the     */
+/* OScaR abstract: per-channel quantization of K, Token Norm Imbalance, INT2) */
+/* Readings: R the same block Hadamard; S the per-token factor 1 / ||R k||_2  */
+/* (the norm kept as fp16, so K^ = n * dequant); K quantized per channel over */
+/* the 16 tokens of a page; V token-wise (S cancels there); codes 0..3, four  */
+/* per byte, lowest channel in the lowest bits; a page is quantized whole.    */
+/* ------------------------------------------------------------------------- */
+
+#define OSCAR_TOP 3
+
+static size_t oscar_code_row(int64_t page, int Hkv, int D, int h, int kv, int t) {
+  return ((((size_t)page * Hkv + h) * 2 + kv) * ORACLE_PAGE + t) * (size_t)(D / 4);
+}
+static size_t oscar_kmeta(int64_t page, int Hkv, int D, int h, int which) { /* which 0: s, 1: z */
+  return (((size_t)page * Hkv + h) * 2 + which) * (size_t)D;
+}
+static size_t oscar_tmeta(int64_t page, int Hkv, int h, int which) { /* 0: K norm, 1: V s, 2: V z */
+  return (((size_t)page * Hkv + h) * 3 + which) * ORACLE_PAGE;
+}
+
+/* Codes of values u for a given (s, z): round-half-even(fp32(u - z) * fp32(1/s))
+ * clamped to [0, top], the same decision rule as the INT4 path. */
+static uint8_t oscar_code(float u, uint16_t s, uint16_t z, int top) {
+  float sf = (float)oracle_half_to_double(s);
+  float zf = (float)oracle_half_to_double(z);
+  float inv = (sf > 0.0f) ? 1.0f / sf : 0.0f;
+  double r = nearbyint((double)(u - zf) * (double)inv);
+  if (r < 0) r = 0;
+  if (r > top) r = top;
+  return (uint8_t)r;
+}
+
+/* The Omni-Token factor of a rotated row: n = ||y||_2 rounded to the nearest
+ * fp16 (saturating at the largest finite one); u = fp32(y / n), 0 when n = 0. */
+uint16_t oracle_oscar_token_norm(const float* y, int D, float* u) {
+  double ss = 0.0;
+  for (int c = 0; c < D; ++c) ss += (double)y[c] * (double)y[c];
+  uint16_t n = oracle_half_round_nearest(sqrt(ss));
+  if ((n & 0x7FFF) >= 0x7C00) n = 0x7BFF;
+  double nd = oracle_half_to_double(n);
+  for (int c = 0; c < D; ++c) u[c] = (nd > 0.0) ? (float)((double)y[c] / nd) : 0.0f;
+  return n;
+}
+
+/* Per-channel INT2 quantization of 16 normalized rows u[16][D]: (s_c, z_c)
+ * from the channel's min and max over the 16 rows, codes packed four per byte. */
+void oracle_oscar_quant_channels(const float* u, int D, uint8_t* kcodes, uint16_t* ks, uint16_t* kz) {
+  uint8_t codes[256];
+  for (int c = 0; c < D; ++c) {
+    float mn = u[c], mx = u[c];
+    for (int t = 1; t < ORACLE_PAGE; ++t) {
+      if (u[t * D + c] < mn) mn = u[t * D + c];
+      if (u[t * D + c] > mx) mx = u[t * D + c];
+    }
+    oracle_scale_zero_levels(mn, mx, OSCAR_TOP, &ks[c], &kz[c]);
+  }
+  for (int t = 0; t < ORACLE_PAGE; ++t) {
+    for (int c = 0; c < D; ++c) codes[c] = oscar_code(u[t * D + c], ks[c], kz[c], OSCAR_TOP);
+    for (int j = 0; j < D / 4; ++j)
+      kcodes[(size_t)t * (D / 4) + j] = (uint8_t)(codes[4 * j] | codes[4 * j + 1] << 2 |
+                                                  codes[4 * j + 2] << 4 | codes[4 * j + 3] << 6);
+  }
+}
+
+/* One page of one kv head: K rows k[16][D], V rows v[16][D] (bf16) -> codes,
+ * per-channel (s, z) of K, token norms of K, per-token (s, z) of V. */
+int oracle_oscar_quant_page(const uint16_t* k, const uint16_t* v, int D, int b, uint8_t* kcodes,
+                            uint8_t* vcodes, uint16_t* ks, uint16_t* kz, uint16_t* kn, uint16_t* vs,
+                            uint16_t* vz) {
+  float y[ORACLE_PAGE][256], u[ORACLE_PAGE][256];
+  uint8_t codes[256];
+  if (D > 256 || !valid_block(D, b)) return -1;
+  float uf[ORACLE_PAGE * 256];
+  for (int t = 0; t < ORACLE_PAGE; ++t) {
+    oracle_rotate_row(k + (size_t)t * D, D, b, y[t]);
+    kn[t] = oracle_oscar_token_norm(y[t], D, u[t]);
+    for (int c = 0; c < D; ++c) uf[t * D + c] = u[t][c];
+  }
+  oracle_oscar_quant_channels(uf, D, kcodes, ks, kz);
+  for (int t = 0; t < ORACLE_PAGE; ++t) {
+    float yv[256];
+    oracle_rotate_row(v + (size_t)t * D, D, b, yv);
+    float mn = yv[0], mx = yv[0];
+    for (int c = 1; c < D; ++c) {
+      if (yv[c] < mn) mn = yv[c];
+      if (yv[c] > mx) mx = yv[c];
+    }
+    oracle_scale_zero_levels(mn, mx, OSCAR_TOP, &vs[t], &vz[t]);
+    for (int c = 0; c < D; ++c) codes[c] = oscar_code(yv[c], vs[t], vz[t], OSCAR_TOP);
+    for (int j = 0; j < D / 4; ++j)
+      vcodes[(size_t)t * (D / 4) + j] = (uint8_t)(codes[4 * j] | codes[4 * j + 1] << 2 |
+                                                  codes[4 * j + 2] << 4 | codes[4 * j + 3] << 6);
+  }
+  return 0;
+}
+
+/* The write: token group g (rows 16 g .. 16 g + 15 of k and v, [T][Hkv][D]
+ * bf16) fills page page_ids[g] whole, for every kv head. A page id outside
+ * [0, num_pages) is skipped and makes the return -2. */
+int oracle_oscar_write(const uint16_t* k, const uint16_t* v, const int32_t* page_ids, int P, int Hkv,
+                       int D, int b, int64_t num_pages, uint8_t* cache, uint16_t* kmeta, uint16_t* tmeta) {
+  if ((D != 64 && D != 128) || !valid_block(D, b)) return -1;
+  int rc = 0;
+#pragma omp parallel for schedule(static) collapse(2)
+  for (int g = 0; g < P; ++g)
+    for (int h = 0; h < Hkv; ++h) {
+      int64_t page = page_ids[g];
+      if (page < 0 || page >= num_pages) {
+#pragma omp critical
+        rc = -2;
+        continue;
+      }
+      uint16_t kr[ORACLE_PAGE * 256], vr[ORACLE_PAGE * 256];
+      for (int t = 0; t < ORACLE_PAGE; ++t)
+        for (int c = 0; c < D; ++c) {
+          size_t src = (((size_t)g * ORACLE_PAGE + t) * Hkv + h) * D + c;
+          kr[t * D + c] = k[src];
+          vr[t * D + c] = v[src];
+        }
+      oracle_oscar_quant_page(kr, vr, D, b, cache + oscar_code_row(page, Hkv, D, h, 0, 0),
+                              cache + oscar_code_row(page, Hkv, D, h, 1, 0),
+                              kmeta + oscar_kmeta(page, Hkv, D, h, 0), kmeta + oscar_kmeta(page, Hkv, D, h, 1),
+                              tmeta + oscar_tmeta(page, Hkv, h, 0), tmeta + oscar_tmeta(page, Hkv, h, 1),
+                              tmeta + oscar_tmeta(page, Hkv, h, 2));
+    }
+  return rc;
+}
+
+/* Dequantized rotated rows of one page-head: K^ = n (code s_c + z_c),
+ * V^ = code s + z, [16][D] each, fp64. */
+void oracle_oscar_dequant_page(const uint8_t* cache, const uint16_t* kmeta, const uint16_t* tmeta,
+                               int64_t page, int Hkv, int D, int h, double* K, double* V) {
+  const uint8_t* kc = cache + oscar_code_row(page, Hkv, D, h, 0, 0);
+  const uint8_t* vc = cache + oscar_code_row(page, Hkv, D, h, 1, 0);
+  const uint16_t* ks = kmeta + oscar_kmeta(page, Hkv, D, h, 0);
+  const uint16_t* kz = kmeta + oscar_kmeta(page, Hkv, D, h, 1);
+  const uint16_t* kn = tmeta + oscar_tmeta(page, Hkv, h, 0);
+  const uint16_t* vs = tmeta + oscar_tmeta(page, Hkv, h, 1);
+  const uint16_t* vz = tmeta + oscar_tmeta(page, Hkv, h, 2);
+  for (int t = 0; t < ORACLE_PAGE; ++t) {
+    const double n = oracle_half_to_double(kn[t]);
+    for (int c = 0; c < D; ++c) {
+      const int ck = (kc[(size_t)t * (D / 4) + c / 4] >> (2 * (c % 4))) & 3;
+      const int cv = (vc[(size_t)t * (D / 4) + c / 4] >> (2 * (c % 4))) & 3;
+      K[(size_t)t * D + c] = n * (ck * oracle_half_to_double(ks[c]) + oracle_half_to_double(kz[c]));
+      V[(size_t)t * D + c] = cv * oracle_half_to_double(vs[t]) + oracle_half_to_double(vz[t]);
+    }
+  }
+}
+
+/* One (sequence, query head) of the OScaR decode: the context's first
+ * 16 * (ctx / 16) tokens from the INT2 pages of page_table[n], the last
+ * ctx % 16 from the bf16 rows of the unfinished page, k_tail / v_tail
+ * [B][Hkv][16][D]; brute-force fp64 softmax attention as for INT4. */
+int oracle_oscar_decode_one(const uint16_t* q_bf16, const uint8_t* cache, const uint16_t* kmeta,
+                            const uint16_t* tmeta, const int32_t* page_table, const int32_t* context_lens,
+                            const uint16_t* k_tail, const uint16_t* v_tail, int n, int hq, int Hq, int Hkv,
+                            int D, int b, int max_pages, int64_t num_pages, double softmax_scale,
+                            double* out) {
+  if (Hkv <= 0 || Hq % Hkv != 0) return -1;
+  const int G = Hq / Hkv, h = hq / G;
+  const int ctx = context_lens[n];
+  const int full = ctx / ORACLE_PAGE, tail = ctx % ORACLE_PAGE;
+  if (ctx < 0 || full > max_pages) return -2;
+  const double scale = (softmax_scale == 0.0) ? 1.0 / sqrt((double)D) : softmax_scale;
+  double q[256];
+  for (int c = 0; c < D; ++c) q[c] = oracle_bf16_to_double(q_bf16[((size_t)n * Hq + hq) * D + c]);
+  const size_t rows = (size_t)(ctx > 0 ? ctx : 1);
+  double* K = (double*)malloc(sizeof(double) * rows * D);
+  double* V = (double*)malloc(sizeof(double) * rows * D);
+  int rc = 0;
+  for (int p = 0; p < full && rc == 0; ++p) {
+    const int64_t page = page_table[(size_t)n * max_pages + p];
+    if (page < 0 || page >= num_pages) { rc = -2; break; }
+    oracle_oscar_dequant_page(cache, kmeta, tmeta, page, Hkv, D, h, K + (size_t)p * ORACLE_PAGE * D,
+                              V + (size_t)p * ORACLE_PAGE * D);
+  }
+  for (int t = 0; t < tail && rc == 0; ++t) {
+    double x[256];
+    const size_t src = (((size_t)n * Hkv + h) * ORACLE_PAGE + t) * D;
+    const size_t dst = ((size_t)full * ORACLE_PAGE + t) * D;
+    for (int c = 0; c < D; ++c) x[c] = oracle_bf16_to_double(k_tail[src + c]);
+    oracle_rotate_f64(x, D, b, K + dst);
+    for (int c = 0; c < D; ++c) x[c] = oracle_bf16_to_double(v_tail[src + c]);
+    oracle_rotate_f64(x, D, b, V + dst);
+  }
+  if (rc == 0) rc = oracle_attn_rows(q, K, V, ctx, D, b, NULL, scale, out);
+  free(K);
+  free(V);
+  return rc;
+}
+
+int oracle_oscar_decode_attn(const uint16_t* q_bf16, const uint8_t* cache, const uint16_t* kmeta,
+                             const uint16_t* tmeta, const int32_t* page_table, const int32_t* context_lens,
+                             const uint16_t* k_tail, const uint16_t* v_tail, int B, int Hq, int Hkv, int D,
+                             int b, int max_pages, int64_t num_pages, double softmax_scale, double* out) {
+  if ((D != 64 && D != 128) || !valid_block(D, b) || Hkv <= 0 || Hq % Hkv != 0) return -1;
+  int rc = 0;
+#pragma omp parallel for schedule(dynamic) collapse(2)
+  for (int n = 0; n < B; ++n)
+    for (int hq = 0; hq < Hq; ++hq) {
+      int r = oracle_oscar_decode_one(q_bf16, cache, kmeta, tmeta, page_table, context_lens, k_tail, v_tail,
+                                      n, hq, Hq, Hkv, D, b, max_pages, num_pages, softmax_scale,
+                                      out + ((size_t)n * Hq + hq) * D);
+      if (r != 0) {
+#pragma omp critical
+        rc = r;
+      }
+    }
+  return rc;
 }

@@ -19,7 +19,7 @@ import numpy as np
 import torch
 
 from . import _lib
-from ._lib import ATTN_INPUTS_READY, AttnDesc, KVQError, WriteDesc
+from ._lib import ATTN_INPUTS_READY, AttnDesc, KVQError, OscarAttnDesc, OscarWriteDesc, WriteDesc
 
 PAGE_SIZE = 16
 
@@ -27,7 +27,8 @@ __all__ = [
     "PAGE_SIZE", "KVQError", "alloc_cache", "kv_quant_write", "paged_decode_attn_int4",
     "attn_workspace_size", "alloc_workspace", "get_device_error", "selftest_bounded_wait", "library_path",
     "paged_decode_attn_int4_static_ws", "paged_decode_append_attn_int4", "paged_prefill_attn_int4",
-    "sign_words", "selftest_occupy",
+    "sign_words", "selftest_occupy", "alloc_oscar_cache", "kv_quant_write_oscar", "oscar_workspace_size",
+    "paged_decode_attn_oscar",
 ]
 
 
@@ -328,3 +329,85 @@ def selftest_bounded_wait(which: int, stream=None) -> None:
 def get_device_error(stream=None) -> int:
     """Synchronize the stream and return (and clear) the device error word."""
     return int(_lib.lib().kvq_get_device_error(ctypes.c_void_p(_stream_handle(stream))))
+
+
+# --- OScaR variant: INT2, K per channel after a per-token scale -------------
+
+def alloc_oscar_cache(num_pages: int, num_kv_heads: int, head_dim: int, device="cuda"):
+    """Empty OScaR pool: cache uint8 [pages, Hkv, 2, 16, D/4] (K then V
+    codes), kmeta fp16 [pages, Hkv, 2, D] (K per-channel s, z), tmeta fp16
+    [pages, Hkv, 3, 16] (K token norms, V s, V z)."""
+    return (torch.zeros((num_pages, num_kv_heads, 2, PAGE_SIZE, head_dim // 4), dtype=torch.uint8, device=device),
+            torch.zeros((num_pages, num_kv_heads, 2, head_dim), dtype=torch.float16, device=device),
+            torch.zeros((num_pages, num_kv_heads, 3, PAGE_SIZE), dtype=torch.float16, device=device))
+
+
+def _oscar_pool(cache, kmeta, tmeta):
+    _need(cache, "cache", torch.uint8)
+    _need(kmeta, "kmeta", torch.float16)
+    _need(tmeta, "tmeta", torch.float16)
+    if cache.dim() != 5 or cache.shape[2] != 2 or cache.shape[3] != PAGE_SIZE:
+        raise ValueError("cache must be uint8 [num_pages, Hkv, 2, 16, D/4]")
+    P, Hkv, D = int(cache.shape[0]), int(cache.shape[1]), 4 * int(cache.shape[4])
+    if tuple(kmeta.shape) != (P, Hkv, 2, D) or tuple(tmeta.shape) != (P, Hkv, 3, PAGE_SIZE):
+        raise ValueError("kmeta must be fp16 [pages, Hkv, 2, D] and tmeta fp16 [pages, Hkv, 3, 16]")
+    return P, Hkv, D
+
+
+def kv_quant_write_oscar(k: torch.Tensor, v: torch.Tensor, page_ids: torch.Tensor, cache: torch.Tensor,
+                         kmeta: torch.Tensor, tmeta: torch.Tensor, hadamard_block: int, stream=None) -> None:
+    """OScaR write: rows 16 g .. 16 g + 15 of k, v (bf16 [16 P, Hkv, D]) fill
+    page page_ids[g] (int32 [P]) whole."""
+    P, Hkv, D = _oscar_pool(cache, kmeta, tmeta)
+    _need(k, "k", torch.bfloat16)
+    _need(v, "v", torch.bfloat16)
+    _need(page_ids, "page_ids", torch.int32)
+    if k.dim() != 3 or tuple(k.shape[1:]) != (Hkv, D) or k.shape != v.shape or k.shape[0] != 16 * page_ids.numel():
+        raise ValueError("k and v must be bf16 [16 * len(page_ids), Hkv, D] matching the pool")
+    desc = OscarWriteDesc(int(page_ids.numel()), Hkv, D, P)
+    st = _lib.lib().kv_quant_write_oscar(_ptr(k), _ptr(v), _ptr(page_ids), _ptr(cache), _ptr(kmeta), _ptr(tmeta),
+                                         int(hadamard_block), ctypes.byref(desc),
+                                         ctypes.c_void_p(_stream_handle(stream)))
+    _lib.check(st, "kv_quant_write_oscar")
+
+
+def oscar_workspace_size(batch: int, num_q_heads: int, num_kv_heads: int, head_dim: int, num_pages: int,
+                         max_pages_per_seq: int, hadamard_block: int, device=None) -> int:
+    L = _lib.lib()
+    idx = None if device is None else torch.device(device).index
+    _lib.check(L.kvq_set_device(int(torch.cuda.current_device() if idx is None else idx)), "kvq_set_device")
+    desc = OscarAttnDesc(batch, num_q_heads, num_kv_heads, head_dim, num_pages, max_pages_per_seq,
+                         hadamard_block, 0.0, 0)
+    n = L.kvq_oscar_workspace_size(ctypes.byref(desc))
+    if n == ctypes.c_size_t(-1).value:
+        raise KVQError(1, "kvq_oscar_workspace_size (invalid shapes or no device)")
+    return int(n)
+
+
+def paged_decode_attn_oscar(q: torch.Tensor, cache: torch.Tensor, kmeta: torch.Tensor, tmeta: torch.Tensor,
+                            page_table: torch.Tensor, context_lens: torch.Tensor, k_tail: torch.Tensor,
+                            v_tail: torch.Tensor, out: torch.Tensor, hadamard_block: int,
+                            workspace: torch.Tensor, softmax_scale: float = 0.0, stream=None) -> None:
+    """OScaR decode step: full pages from the INT2 pool, each sequence's last
+    context_lens % 16 tokens from k_tail / v_tail (bf16 [B, Hkv, 16, D])."""
+    P, Hkv, D = _oscar_pool(cache, kmeta, tmeta)
+    _need(q, "q", torch.bfloat16)
+    _need(page_table, "page_table", torch.int32)
+    _need(context_lens, "context_lens", torch.int32)
+    _need(k_tail, "k_tail", torch.bfloat16)
+    _need(v_tail, "v_tail", torch.bfloat16)
+    _need(workspace, "workspace", torch.uint8)
+    if out.dtype not in (torch.float32, torch.bfloat16):
+        raise TypeError("out must be float32 or bfloat16")
+    _need(out, "out", out.dtype)
+    B, Hq = int(q.shape[0]), int(q.shape[1])
+    if tuple(out.shape) != tuple(q.shape) or tuple(k_tail.shape) != (B, Hkv, PAGE_SIZE, D) or \
+            k_tail.shape != v_tail.shape or page_table.dim() != 2 or int(page_table.shape[0]) != B:
+        raise ValueError("shapes: q/out [B, Hq, D], k_tail/v_tail [B, Hkv, 16, D], page_table [B, max_pages]")
+    desc = OscarAttnDesc(B, Hq, Hkv, D, P, int(page_table.shape[1]), int(hadamard_block), float(softmax_scale),
+                         0 if out.dtype == torch.float32 else 1)
+    st = _lib.lib().paged_decode_attn_oscar(
+        _ptr(q), _ptr(cache), _ptr(kmeta), _ptr(tmeta), _ptr(page_table), _ptr(context_lens), _ptr(k_tail),
+        _ptr(v_tail), _ptr(out), _ptr(workspace), workspace.numel(), ctypes.byref(desc),
+        ctypes.c_void_p(_stream_handle(stream)))
+    _lib.check(st, "paged_decode_attn_oscar")

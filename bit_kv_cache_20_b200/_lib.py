@@ -31,6 +31,19 @@ class AttnDesc(ctypes.Structure):
                 ("hadamard_signs", ctypes.c_uint32 * 4)]
 
 
+class OscarWriteDesc(ctypes.Structure):
+    _fields_ = [("num_groups", ctypes.c_int32), ("num_kv_heads", ctypes.c_int32),
+                ("head_dim", ctypes.c_int32), ("num_pages", ctypes.c_int32)]
+
+
+class OscarAttnDesc(ctypes.Structure):
+    _fields_ = [("batch", ctypes.c_int32), ("num_q_heads", ctypes.c_int32),
+                ("num_kv_heads", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("num_pages", ctypes.c_int32), ("max_pages_per_seq", ctypes.c_int32),
+                ("hadamard_block", ctypes.c_int32), ("softmax_scale", ctypes.c_float),
+                ("out_dtype", ctypes.c_int32)]
+
+
 ATTN_INPUTS_READY = 1  # KVQ_ATTN_INPUTS_READY
 
 
@@ -66,6 +79,15 @@ SIGNATURES = [
                                                         ctypes.c_void_p, ctypes.c_void_p,
                                                         ctypes.c_void_p, ctypes.POINTER(AttnDesc),
                                                         ctypes.c_void_p]),
+    ("kv_quant_write_oscar", ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_int32,
+                                            ctypes.POINTER(OscarWriteDesc), ctypes.c_void_p]),
+    ("kvq_oscar_workspace_size", ctypes.c_size_t, [ctypes.POINTER(OscarAttnDesc)]),
+    ("paged_decode_attn_oscar", ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                               ctypes.c_void_p, ctypes.c_size_t, ctypes.POINTER(OscarAttnDesc),
+                                               ctypes.c_void_p]),
     ("kvq_get_device_error", ctypes.c_int, [ctypes.c_void_p]),
     ("kvq_selftest_bounded_wait", ctypes.c_int, [ctypes.c_int32, ctypes.c_void_p]),
     ("kvq_selftest_occupy", ctypes.c_int, [ctypes.c_int32, ctypes.c_int32, ctypes.c_void_p]),

@@ -18,6 +18,7 @@
 #include "kvq_write.cuh"
 #include "kvq_write_tc.cuh"
 #include "kvq_prefill.cuh"
+#include "kvq_oscar.cuh"
 #include "kvq_selftest.cuh"
 
 namespace {
@@ -791,6 +792,192 @@ kvq_status paged_prefill_attn_int4(const void* q, const uint8_t* cache, const vo
                                      : launch_prefill<128, 64>(p, max_q_len, dev, s);
     case 128: return launch_prefill<128, 128>(p, max_q_len, dev, s);
     default: return KVQ_ERR_UNSUPPORTED;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// OScaR variant
+// ---------------------------------------------------------------------------
+}  // extern "C"
+
+namespace {
+
+// Persistent write grid: at most one wave of resident CTAs.
+template <int BLK>
+kvq_status launch_oscar_write(const kvq::OscarWriteParams& p, int dev, cudaStream_t s) {
+  static std::atomic<int> occ[kMaxDevices];
+  constexpr int smem = kvq::OscarWriteSmem::kTotal;
+  auto kern = kvq::kvq_oscar_write_kernel<128, BLK>;
+  const int per_sm = resident_ctas(kern, occ, dev, kvq::kOscarWriteWarps * 32, smem);
+  const long long units = (long long)p.P * p.Hkv;
+  const long long need = (units + kvq::kOscarWriteWarps - 1) / kvq::kOscarWriteWarps;
+  const long long wave = (long long)per_sm * std::max(sm_count(dev), 1);
+  const dim3 grid((unsigned)std::min(need, wave));
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+      launch_pdl(kern, grid, dim3(kvq::kOscarWriteWarps * 32), smem, s, p) != cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
+  return KVQ_OK;
+}
+
+kvq_status check_oscar_desc(const kvq_oscar_attn_desc* d) {
+  if (!d) return KVQ_ERR_INVALID_ARG;
+  if (d->batch < 0 || d->batch > 65535 || d->num_q_heads < 1 || d->num_kv_heads < 1 ||
+      d->num_kv_heads > 65535 || d->num_pages < 1 || d->max_pages_per_seq < 1 ||
+      d->max_pages_per_seq > INT_MAX / KVQ_PAGE_SIZE - 1)
+    return KVQ_ERR_INVALID_ARG;
+  if (d->num_q_heads % d->num_kv_heads != 0) return KVQ_ERR_INVALID_ARG;
+  if (!(d->softmax_scale >= 0.0f) || !std::isfinite(d->softmax_scale)) return KVQ_ERR_INVALID_ARG;
+  if (d->out_dtype != 0 && d->out_dtype != 1) return KVQ_ERR_INVALID_ARG;
+  const int G = d->num_q_heads / d->num_kv_heads;
+  if (d->head_dim != 128 || (G != 1 && G != 2 && G != 4)) return KVQ_ERR_UNSUPPORTED;
+  if (!valid_block(d->head_dim, d->hadamard_block)) return KVQ_ERR_UNSUPPORTED;
+  return KVQ_OK;
+}
+
+// Splits per (sequence, kv head): enough to fill the device's resident decode
+// CTAs once, and at most 64 pages per split (short CTAs balance sequences of
+// different lengths over several waves); at least two pages per split.
+void oscar_plan(const kvq_oscar_attn_desc* d, int dev, int* ns, int* pps) {
+  static std::atomic<int> occ[kMaxDevices];
+  int per_sm = 1;
+  if (dev >= 0 && dev < kMaxDevices)
+    per_sm = resident_ctas(kvq::kvq_oscar_decode_kernel<128, 128>, occ, dev, kvq::kOscarWarps * 32,
+                           kvq::OscarSmem<128>::kTotal);
+  const long long slots = (long long)per_sm * std::max(sm_count(dev), 1);
+  const long long units = std::max<long long>((long long)d->batch * d->num_kv_heads, 1);
+  long long n = std::max<long long>(slots / units, (d->max_pages_per_seq + 63) / 64);
+  const long long cap = std::max<long long>(d->max_pages_per_seq / 2, 1);
+  if (n > cap) n = cap;
+  if (n > kvq::kMaxSplits) n = kvq::kMaxSplits;
+  if (n < 1) n = 1;
+  const long long p = (d->max_pages_per_seq + n - 1) / n;
+  *ns = (int)((d->max_pages_per_seq + p - 1) / p);
+  *pps = (int)p;
+}
+
+size_t oscar_ws_bytes(const kvq_oscar_attn_desc* d, int ns) {
+  const size_t G = (size_t)(d->num_q_heads / d->num_kv_heads);
+  return (size_t)d->batch * d->num_kv_heads * ns * G * (d->head_dim + 2) * sizeof(float);
+}
+
+template <int BLK>
+kvq_status launch_oscar_decode(const kvq::OscarAttnParams& p, cudaStream_t s) {
+  constexpr int smem = kvq::OscarSmem<128>::kTotal;
+  auto kern = kvq::kvq_oscar_decode_kernel<128, BLK>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
+      launch_pdl(kern, dim3(p.n_splits, p.Hkv, p.B), dim3(kvq::kOscarWarps * 32), smem, s, p) != cudaSuccess ||
+      launch_pdl(kvq::kvq_oscar_combine_kernel<128, BLK>, dim3((unsigned)(((long long)p.B * p.Hq + 3) / 4)),
+                 dim3(128), 0, s, p) != cudaSuccess) {
+    cudaGetLastError();
+    return KVQ_ERR_CUDA;
+  }
+  return KVQ_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+kvq_status kv_quant_write_oscar(const void* k, const void* v, const int32_t* page_ids, uint8_t* cache,
+                                void* kmeta, void* tmeta, int32_t hadamard_block,
+                                const kvq_oscar_write_desc* desc, void* stream) {
+  if (!desc) return KVQ_ERR_INVALID_ARG;
+  const kvq_oscar_write_desc& d = *desc;
+  if (d.num_groups < 0 || d.num_kv_heads < 1 || d.num_pages < 1) return KVQ_ERR_INVALID_ARG;
+  if ((long long)d.num_groups * d.num_kv_heads > INT_MAX) return KVQ_ERR_INVALID_ARG;
+  if (d.head_dim != 128 || !valid_block(d.head_dim, hadamard_block)) return KVQ_ERR_UNSUPPORTED;
+  if (d.num_groups == 0) return KVQ_OK;
+  if (!k || !v || !page_ids || !cache || !kmeta || !tmeta) return KVQ_ERR_INVALID_ARG;
+  if (!aligned(k, 16) || !aligned(v, 16) || !aligned(cache, 16) || !aligned(kmeta, 16) || !aligned(tmeta, 16) ||
+      !aligned(page_ids, 4))
+    return KVQ_ERR_INVALID_ARG;
+  int dev = 0;
+  kvq_status st = select_device_of(cache, &dev);
+  if (st != KVQ_OK) return st;
+  kvq::OscarWriteParams p;
+  p.k = static_cast<const uint16_t*>(k);
+  p.v = static_cast<const uint16_t*>(v);
+  p.page_ids = page_ids;
+  p.cache = cache;
+  p.kmeta = static_cast<uint16_t*>(kmeta);
+  p.tmeta = static_cast<uint16_t*>(tmeta);
+  p.P = d.num_groups;
+  p.Hkv = d.num_kv_heads;
+  p.num_pages = d.num_pages;
+  p.cb = hadamard_block > 0 ? (float)(1.0 / std::sqrt((double)hadamard_block)) : 1.0f;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (hadamard_block) {
+    case 0: return launch_oscar_write<0>(p, dev, s);
+    case 32: return launch_oscar_write<32>(p, dev, s);
+    case 64: return launch_oscar_write<64>(p, dev, s);
+    default: return launch_oscar_write<128>(p, dev, s);
+  }
+}
+
+size_t kvq_oscar_workspace_size(const kvq_oscar_attn_desc* desc) {
+  if (check_oscar_desc(desc) != KVQ_OK) return SIZE_MAX;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return SIZE_MAX;
+  }
+  int ns = 1, pps = 1;
+  oscar_plan(desc, dev, &ns, &pps);
+  return oscar_ws_bytes(desc, ns);
+}
+
+kvq_status paged_decode_attn_oscar(const void* q, const uint8_t* cache, const void* kmeta, const void* tmeta,
+                                   const int32_t* page_table, const int32_t* context_lens, const void* k_tail,
+                                   const void* v_tail, void* out, void* workspace, size_t workspace_bytes,
+                                   const kvq_oscar_attn_desc* desc, void* stream) {
+  kvq_status st = check_oscar_desc(desc);
+  if (st != KVQ_OK) return st;
+  const kvq_oscar_attn_desc& d = *desc;
+  if (d.batch == 0) return KVQ_OK;
+  if (!q || !cache || !kmeta || !tmeta || !page_table || !context_lens || !k_tail || !v_tail || !out)
+    return KVQ_ERR_INVALID_ARG;
+  if (!aligned(q, 16) || !aligned(cache, 16) || !aligned(kmeta, 16) || !aligned(tmeta, 16) ||
+      !aligned(k_tail, 16) || !aligned(v_tail, 16) || !aligned(page_table, 4) || !aligned(context_lens, 4) ||
+      !aligned(out, d.out_dtype ? 8 : 16))
+    return KVQ_ERR_INVALID_ARG;
+  int dev = 0;
+  st = select_device_of(cache, &dev);
+  if (st != KVQ_OK) return st;
+  int ns = 1, pps = 1;
+  oscar_plan(&d, dev, &ns, &pps);
+  if (!workspace || !aligned(workspace, 16) || workspace_bytes < oscar_ws_bytes(&d, ns)) return KVQ_ERR_WORKSPACE;
+  kvq::OscarAttnParams p;
+  p.q = static_cast<const uint16_t*>(q);
+  p.cache = cache;
+  p.kmeta = static_cast<const uint16_t*>(kmeta);
+  p.tmeta = static_cast<const uint16_t*>(tmeta);
+  p.page_table = page_table;
+  p.ctx_lens = context_lens;
+  p.k_tail = static_cast<const uint16_t*>(k_tail);
+  p.v_tail = static_cast<const uint16_t*>(v_tail);
+  p.ws = static_cast<float*>(workspace);
+  p.out = out;
+  p.B = d.batch;
+  p.Hq = d.num_q_heads;
+  p.Hkv = d.num_kv_heads;
+  p.G = d.num_q_heads / d.num_kv_heads;
+  p.num_pages = d.num_pages;
+  p.max_pages = d.max_pages_per_seq;
+  p.n_splits = ns;
+  p.pages_per_split = pps;
+  p.out_bf16 = d.out_dtype;
+  const double cb = d.hadamard_block > 0 ? 1.0 / std::sqrt((double)d.hadamard_block) : 1.0;
+  const double scale = d.softmax_scale > 0.0f ? (double)d.softmax_scale : 1.0 / std::sqrt((double)d.head_dim);
+  p.qmul = (float)(cb * scale * 1.4426950408889634);
+  p.cb = (float)cb;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (d.hadamard_block) {
+    case 0: return launch_oscar_decode<0>(p, s);
+    case 32: return launch_oscar_decode<32>(p, s);
+    case 64: return launch_oscar_decode<64>(p, s);
+    default: return launch_oscar_decode<128>(p, s);
   }
 }
 

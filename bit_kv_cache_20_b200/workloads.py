@@ -238,3 +238,31 @@ def random_signs(seed: int, D: int) -> np.ndarray:
     that channel before the transform."""
     g = torch.Generator().manual_seed(seed)
     return (torch.rand(D, generator=g) < 0.5).numpy()
+
+
+def oscar_rows(w: Workload):
+    """The rows of a workload arranged for the OScaR layout, where a page is
+    quantized whole: each sequence's full pages as write groups of 16 rows
+    (k, v bf16 [16 P, Hkv, D], page ids int32 [P] from its page table), and
+    its last ctx % 16 rows as the bf16 unfinished page k_tail, v_tail
+    [B, Hkv, 16, D] (rows past the tail zero)."""
+    B, Hkv, D = w.B, w.Hkv, w.D
+    ks, vs, ids = [], [], []
+    k_tail = torch.zeros((B, Hkv, PAGE, D), dtype=torch.bfloat16)
+    v_tail = torch.zeros((B, Hkv, PAGE, D), dtype=torch.bfloat16)
+    op = on = 0
+    for n in range(B):
+        npr, ctx = int(w.prior_lens[n]), int(w.context_lens[n])
+        k = torch.cat([w.k_prior[op:op + npr], w.k_new[on:on + ctx - npr]])
+        v = torch.cat([w.v_prior[op:op + npr], w.v_new[on:on + ctx - npr]])
+        op += npr
+        on += ctx - npr
+        full = ctx // PAGE
+        ks.append(k[:full * PAGE])
+        vs.append(v[:full * PAGE])
+        ids.append(w.page_table[n, :full].astype(np.int32))
+        tail = ctx - full * PAGE
+        k_tail[n, :, :tail] = k[full * PAGE:].transpose(0, 1)
+        v_tail[n, :, :tail] = v[full * PAGE:].transpose(0, 1)
+    return (torch.cat(ks), torch.cat(vs), np.concatenate(ids) if ids else np.zeros(0, np.int32),
+            k_tail, v_tail)

@@ -49,7 +49,7 @@ extern "C" {
 #endif
 
 #define KVQ_PAGE_SIZE 16
-#define KVQ_ABI_VERSION 5
+#define KVQ_ABI_VERSION 6
 
 typedef enum kvq_status {
   KVQ_OK = 0,
@@ -316,6 +316,94 @@ kvq_status paged_decode_attn_int4_static_ws(const void* q, const uint8_t* cache,
                                             const int32_t* page_table,
                                             const int32_t* context_lens, void* out,
                                             const kvq_attn_desc* desc, void* stream);
+
+/* ------------------------------------------------------------------------ */
+/* OScaR variant: INT2 codes, K quantized per channel after a per-token scale */
+/* ------------------------------------------------------------------------ */
+
+/* Shapes of one kv_quant_write_oscar call. */
+typedef struct kvq_oscar_write_desc {
+  int32_t num_groups;   /* P >= 0 token groups of 16, each filling one whole page */
+  int32_t num_kv_heads; /* Hkv >= 1 */
+  int32_t head_dim;     /* D: 128 */
+  int32_t num_pages;    /* pages in the pool */
+} kvq_oscar_write_desc;
+
+/*
+ * kv_quant_write_oscar - the OScaR write (OScaR forum summary, "The OScaR
+ * Framework": V^ = Quant(S (R V)); OScaR abstract: per-channel quantization
+ * of K, Token Norm Imbalance, INT2): for every token group g and kv head h,
+ * rows 16 g .. 16 g + 15 of k and v become page page_ids[g]:
+ *   K: y_t = R k_t; n_t = fp16(||y_t||_2) (saturating); S_t = fp32(1/n_t)
+ *      (0 when n_t = 0), u_t = fp32(y_t * S_t); per channel c over the
+ *      page's 16 tokens z_c = RD16(min_t u_tc), s_c = the smallest fp16 with
+ *      3 s_c + z_c >= max_t u_tc; code = rint(fp32(u - z_c) * fp32(1/s_c))
+ *      in 0..3;
+ *      dequantized K^_tc = n_t (code s_c + z_c).
+ *   V: y_t = R v_t, per token z = RD16(min), s = the smallest fp16 with
+ *      3 s + z >= max, codes as for K; V^ = code s + z.
+ * A sequence's unfinished last page is not written here: the caller keeps
+ * its rows in bf16 and passes them to paged_decode_attn_oscar.
+ *
+ * k, v         : device, bf16 [16 P][Hkv][D], contiguous, 16-byte aligned.
+ * page_ids     : device, int32 [P]; an id outside [0, num_pages) skips that
+ *                group and records KVQ_ERR_OUT_OF_RANGE.
+ * cache        : device, uint8 [num_pages][Hkv][2][16][D/4]: K codes, then V
+ *                codes, four per byte, the lowest channel in the lowest bits.
+ * kmeta        : device, fp16 [num_pages][Hkv][2][D]: K per-channel s, then z.
+ * tmeta        : device, fp16 [num_pages][Hkv][3][16]: K token norms, V s, V z.
+ * hadamard_block : 0, 32, 64 or 128.
+ * Returns KVQ_OK, KVQ_ERR_INVALID_ARG (null or misaligned pointers, bad
+ * shapes), KVQ_ERR_UNSUPPORTED (D != 128, bad block) or KVQ_ERR_CUDA.
+ */
+kvq_status kv_quant_write_oscar(const void* k, const void* v, const int32_t* page_ids, uint8_t* cache,
+                                void* kmeta, void* tmeta, int32_t hadamard_block,
+                                const kvq_oscar_write_desc* desc, void* stream);
+
+/* Shapes of one paged_decode_attn_oscar call (fields as in kvq_attn_desc). */
+typedef struct kvq_oscar_attn_desc {
+  int32_t batch;
+  int32_t num_q_heads;       /* Hq / Hkv must be 1, 2 or 4 */
+  int32_t num_kv_heads;
+  int32_t head_dim;          /* 128 */
+  int32_t num_pages;
+  int32_t max_pages_per_seq; /* columns of page_table: full pages only */
+  int32_t hadamard_block;
+  float softmax_scale;       /* 0 means 1/sqrt(head_dim) */
+  int32_t out_dtype;         /* 0 = fp32, 1 = bf16 */
+} kvq_oscar_attn_desc;
+
+/*
+ * kvq_oscar_workspace_size - bytes of device workspace paged_decode_attn_oscar
+ * needs on this library's current device (the splits' partial results; no
+ * zero-filling needed). SIZE_MAX for invalid shapes.
+ */
+size_t kvq_oscar_workspace_size(const kvq_oscar_attn_desc* desc);
+
+/*
+ * paged_decode_attn_oscar - one decode step over the OScaR cache. For
+ * sequence n with ctx = context_lens[n]: tokens 0 .. 16 (ctx / 16) - 1 are
+ * the INT2 pages page_table[n][0 .. ctx / 16 - 1]; the last ctx % 16 tokens
+ * are rows 0 .. ctx % 16 - 1 of k_tail[n][h] / v_tail[n][h] (bf16, exact).
+ *   logit_t = softmax_scale * q . k_t, p = softmax(logit),
+ *   out[n][i] = sum_t p_t v_t, with k_t, v_t the dequantized rows rotated
+ *   back (R^T K^, R^T V^) or the bf16 rows of the unfinished page.
+ * q            : device, bf16 [B][Hq][D], 16-byte aligned.
+ * cache, kmeta, tmeta : as written by kv_quant_write_oscar with the same block.
+ * page_table   : device, int32 [B][max_pages_per_seq].
+ * context_lens : device, int32 [B]; above max_pages_per_seq * 16 + 15 it is
+ *                clamped and records KVQ_ERR_OUT_OF_RANGE.
+ * k_tail, v_tail : device, bf16 [B][Hkv][16][D].
+ * out          : device, [B][Hq][D] fp32 or bf16.
+ * workspace    : device, >= kvq_oscar_workspace_size(desc) bytes, 16-byte
+ *                aligned (contents need not be zero).
+ * Two launches (the split decode, then a merge kernel). Returns KVQ_OK,
+ * KVQ_ERR_INVALID_ARG, KVQ_ERR_UNSUPPORTED, KVQ_ERR_WORKSPACE or KVQ_ERR_CUDA.
+ */
+kvq_status paged_decode_attn_oscar(const void* q, const uint8_t* cache, const void* kmeta, const void* tmeta,
+                                   const int32_t* page_table, const int32_t* context_lens, const void* k_tail,
+                                   const void* v_tail, void* out, void* workspace, size_t workspace_bytes,
+                                   const kvq_oscar_attn_desc* desc, void* stream);
 
 /*
  * kvq_get_device_error - synchronizes `stream`, then returns and clears the

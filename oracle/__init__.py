@@ -85,6 +85,7 @@ def lib():
                                                 ctypes.POINTER(ctypes.c_uint16),
                                                 ctypes.POINTER(ctypes.c_uint16)]),
             "oracle_oscar_token_norm": (ctypes.c_uint16, [_p(f32), c_int, _p(f32)]),
+            "oracle_oscar_codes_given": (None, [_p(f32), c_int, ctypes.c_uint16, ctypes.c_uint16, _p(u8)]),
             "oracle_oscar_quant_channels": (None, [_p(f32), c_int, _p(u8), _p(u16), _p(u16)]),
             "oracle_oscar_quant_page": (c_int, [_p(u16), _p(u16), c_int, c_int, _p(u8), _p(u8), _p(u16),
                                                 _p(u16), _p(u16), _p(u16), _p(u16)]),
@@ -352,6 +353,15 @@ def oscar_token_norm(y):
     return int(n), u
 
 
+def oscar_codes_given(u, s: int, z: int) -> np.ndarray:
+    """INT2 codes (uint8, one per value) of the fp32 values u under the given
+    (s, z) fp16 bits: round-half-even(fp32(u - z) * fp32(1/s)) in 0..3."""
+    u = _c(u, np.float32)
+    out = np.zeros(u.size, np.uint8)
+    lib().oracle_oscar_codes_given(u.reshape(-1), u.size, int(s), int(z), out)
+    return out.reshape(u.shape)
+
+
 def oscar_quant_channels(u):
     """Per-channel INT2 quantization of 16 normalized rows u (fp32 [16, D]):
     (codes uint8 [16, D/4], ks, kz fp16 bits [D])."""
@@ -415,6 +425,25 @@ def oscar_dequant_page(cache, kmeta, tmeta, page: int, h: int):
                                     _c(tmeta, np.uint16).reshape(-1), page, Hkv, D, h, K.reshape(-1),
                                     V.reshape(-1))
     return K, V
+
+
+def oscar_decode_one(q_bits, cache, kmeta, tmeta, page_table, context_lens, k_tail_bits, v_tail_bits,
+                     n: int, hq: int, b: int, softmax_scale: float = 0.0) -> np.ndarray:
+    """One (sequence n, query head hq) of the OScaR decode, fp64 [D]."""
+    q = _c(q_bits, np.uint16)
+    B, Hq, D = q.shape
+    P, Hkv = cache.shape[0], cache.shape[1]
+    pt = _c(page_table, np.int32)
+    out = np.zeros(D, np.float64)
+    rc = lib().oracle_oscar_decode_one(q.reshape(-1), _c(cache, np.uint8).reshape(-1),
+                                       _c(kmeta, np.uint16).reshape(-1), _c(tmeta, np.uint16).reshape(-1),
+                                       pt.reshape(-1), _c(context_lens, np.int32),
+                                       _c(k_tail_bits, np.uint16).reshape(-1),
+                                       _c(v_tail_bits, np.uint16).reshape(-1), n, hq, Hq, Hkv, D, b,
+                                       pt.shape[1], P, float(softmax_scale), out)
+    if rc != 0:
+        raise ValueError(f"oracle_oscar_decode_one returned {rc}")
+    return out
 
 
 def oscar_decode_attn(q_bits, cache, kmeta, tmeta, page_table, context_lens, k_tail_bits, v_tail_bits,

@@ -500,15 +500,26 @@ static uint8_t oscar_code(float u, uint16_t s, uint16_t z, int top) {
   return (uint8_t)r;
 }
 
+/* Codes (one per byte, unpacked) of n values for a given (s, z), by the rule
+ * of oscar_code; used to compare another implementation's codes under that
+ * implementation's own (s, z). */
+void oracle_oscar_codes_given(const float* u, int n, uint16_t s, uint16_t z, uint8_t* codes) {
+  for (int i = 0; i < n; ++i) codes[i] = oscar_code(u[i], s, z, OSCAR_TOP);
+}
+
 /* The Omni-Token factor of a rotated row: n = ||y||_2 rounded to the nearest
- * fp16 (saturating at the largest finite one); u = fp32(y / n), 0 when n = 0. */
+ * fp16 (saturating at the largest finite one) is stored; the row is scaled
+ * by S = fp32(1/n) (0 when n = 0): u = fp32(y * S). 1/n in fp64 rounded to
+ * fp32 is the correctly rounded fp32 quotient, and the product of two fp32
+ * values is exact in fp64, so each step rounds once. */
 uint16_t oracle_oscar_token_norm(const float* y, int D, float* u) {
   double ss = 0.0;
   for (int c = 0; c < D; ++c) ss += (double)y[c] * (double)y[c];
   uint16_t n = oracle_half_round_nearest(sqrt(ss));
   if ((n & 0x7FFF) >= 0x7C00) n = 0x7BFF;
   double nd = oracle_half_to_double(n);
-  for (int c = 0; c < D; ++c) u[c] = (nd > 0.0) ? (float)((double)y[c] / nd) : 0.0f;
+  float S = (nd > 0.0) ? (float)(1.0 / nd) : 0.0f;
+  for (int c = 0; c < D; ++c) u[c] = (float)((double)y[c] * (double)S);
   return n;
 }
 

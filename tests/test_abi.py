@@ -47,7 +47,7 @@ def test_library_exports_every_declared_symbol(L):
 
 
 def test_version_and_status_strings(L):
-    assert L.kvq_abi_version() == 5
+    assert L.kvq_abi_version() == 6
     assert L.kvq_status_string(0) == b"KVQ_OK"
     assert L.kvq_status_string(5) == b"KVQ_ERR_TIMEOUT"
     assert L.kvq_status_string(99) == b"KVQ_ERR_UNKNOWN"

@@ -61,9 +61,15 @@ def test_token_norm_is_the_fp16_rounded_l2_norm():
         n, u = oracle.oscar_token_norm(y)
         ref = np.float16(np.linalg.norm(y.astype(np.float64)))
         assert n == ref.view(np.uint16)
-        assert np.array_equal(u, (y.astype(np.float64) / float(ref)).astype(np.float32))
+        S = np.float32(1.0) / np.float32(ref)                       # numpy's fp32 quotient
+        assert np.array_equal(u, (y.astype(np.float64) * np.float64(S)).astype(np.float32))
+        # the scaled row has unit norm up to the fp16 rounding of n (2^-11)
+        assert abs(np.linalg.norm(u.astype(np.float64)) - 1.0) <= 2.0 ** -11 + 2.0 ** -20
     n, u = oracle.oscar_token_norm(np.zeros(64, np.float32))
     assert n == 0 and not u.any()
+    # a norm above the fp16 range saturates at 65504
+    n, u = oracle.oscar_token_norm(np.full(128, 7000.0, np.float32))
+    assert n == 0x7BFF and np.allclose(u, 7000.0 / 65504.0, rtol=2.0 ** -22)
 
 
 def test_per_channel_round_trip_on_the_int2_grid():

@@ -828,6 +828,7 @@ kvq_status check_oscar_desc(const kvq_oscar_attn_desc* d) {
       d->max_pages_per_seq > INT_MAX / KVQ_PAGE_SIZE - 1)
     return KVQ_ERR_INVALID_ARG;
   if (d->num_q_heads % d->num_kv_heads != 0) return KVQ_ERR_INVALID_ARG;
+  if ((long long)d->batch * d->num_q_heads > INT_MAX) return KVQ_ERR_INVALID_ARG;  // one merge CTA per row
   if (!(d->softmax_scale >= 0.0f) || !std::isfinite(d->softmax_scale)) return KVQ_ERR_INVALID_ARG;
   if (d->out_dtype != 0 && d->out_dtype != 1) return KVQ_ERR_INVALID_ARG;
   const int G = d->num_q_heads / d->num_kv_heads;
@@ -868,8 +869,8 @@ kvq_status launch_oscar_decode(const kvq::OscarAttnParams& p, cudaStream_t s) {
   auto kern = kvq::kvq_oscar_decode_kernel<128, BLK>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem) != cudaSuccess ||
       launch_pdl(kern, dim3(p.n_splits, p.Hkv, p.B), dim3(kvq::kOscarWarps * 32), smem, s, p) != cudaSuccess ||
-      launch_pdl(kvq::kvq_oscar_combine_kernel<128, BLK>, dim3((unsigned)(((long long)p.B * p.Hq + 3) / 4)),
-                 dim3(128), 0, s, p) != cudaSuccess) {
+      launch_pdl(kvq::kvq_oscar_combine_kernel<128, BLK>, dim3((unsigned)((long long)p.B * p.Hq)), dim3(128), 0,
+                 s, p) != cudaSuccess) {
     cudaGetLastError();
     return KVQ_ERR_CUDA;
   }
@@ -971,6 +972,7 @@ kvq_status paged_decode_attn_oscar(const void* q, const uint8_t* cache, const vo
   const double cb = d.hadamard_block > 0 ? 1.0 / std::sqrt((double)d.hadamard_block) : 1.0;
   const double scale = d.softmax_scale > 0.0f ? (double)d.softmax_scale : 1.0 / std::sqrt((double)d.head_dim);
   p.qmul = (float)(cb * scale * 1.4426950408889634);
+  p.qraw = (float)(scale * 1.4426950408889634);
   p.cb = (float)cb;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (d.hadamard_block) {

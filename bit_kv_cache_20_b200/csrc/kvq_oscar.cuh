@@ -27,14 +27,15 @@
 //  tmeta fp16 [pages][Hkv][3][16]  K token norms, V s, V z (96 B)
 //
 // Decode: split-K over pages, each warp streaming its own pages through a
-// cp.async ring. QK on the tensor cores (mma.m16n8k16 f16): A = the K codes
-// of 16 tokens, each 2-bit code moved to its own byte and read as e4m3,
-// which is exactly code * 2^-9; B = q~ (.) s_c for the page (the
-// per-channel scale folds into q~, as fp16 hi + lo), columns = (query head,
-// hi/lo); logit_t = n_t (2^9 dot + sum_c q~_c z_c). PV as in the INT4 path
-// with the V codes of two tokens paired per channel. The splits' partial
-// results go to the workspace; a second kernel (programmatic dependent
-// launch) merges them, rotates back and stores.
+// cp.async ring. QK on the tensor cores (mma.m16n8k16 f16) by bit planes of
+// the codes: A = b0 * s_c, then b1 * (2 s_c), for 16 tokens (each entry s_c
+// or 0, exact in fp16), B = q~ as fp16 hi + lo columns (query head, hi/lo),
+// built once per CTA; sum_c q~_c z_c comes from one more MMA whose A holds z
+// in row 0; logit_t = n_t (dot + sum_c q~_c z_c). PV with the V codes of two
+// tokens paired per channel, each 2-bit code moved to its own byte and read
+// as e4m3 (exactly code * 2^-9), against p * s_t as hi + lo. The splits'
+// partial results go to the workspace; a second kernel (programmatic
+// dependent launch) merges them, rotates back and stores.
 #pragma once
 
 #include "kvq_decode.cuh"
@@ -89,17 +90,17 @@ __device__ __forceinline__ void int2_scale_zero(float mn, float mx, unsigned sho
   sf = __half2float(__ushort_as_half(s));
 }
 
-// Two codes rint(fp32(u - z) * fp32(1/s)) (ties to even), clamped to 0..3,
-// as one nibble (the first code in bits 0-1): adding 2^23 inside one fma
-// rounds the exact product to an integer, read back as the distance of the
-// sum's bit pattern from that of 2^23.
+// Two codes rint(fp32(u - z) * fp32(1/s)) (ties to even) as a nibble in
+// bits 0-3 of the result (the first code in bits 0-1; the bits above are not
+// cleared). Adding 2^23 inside one fma rounds the exact product to an
+// integer c in the low mantissa bits of 2^23 + c. No clamp is needed: z <= u
+// gives c >= 0, and u - z <= 3 s exactly, so fp32(u - z) * fp32(1/s) <=
+// 3 (1 + 2^-24) gives c <= 3 (s = 0 has 1/s read as 0, c = 0).
 __device__ __forceinline__ uint32_t int2_code_pair(uint64_t u2, uint64_t z2, uint64_t inv2) {
   const uint64_t r = f2_fma(f2_sub(u2, z2), inv2, f2_pack(8388608.0f, 8388608.0f));
   float r0, r1;
   f2_unpack(r, r0, r1);
-  const uint32_t c0 = min(__float_as_uint(r0) - 0x4B000000u, 3u);
-  const uint32_t c1 = min(__float_as_uint(r1) - 0x4B000000u, 3u);
-  return c0 | (c1 << 2);
+  return (__float_as_uint(r1) << 2) + __float_as_uint(r0);
 }
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t (&r)[4]) {
@@ -269,23 +270,56 @@ __global__ void __launch_bounds__(kOscarWriteWarps * 32) kvq_oscar_write_kernel(
     oscar_rotate_rows<BLK>(rows_s, hb, p.cb, y);
     __syncwarp();
     stage(unit + stride, 0);
-    double ss[2] = {0.0, 0.0};
+    // token norms: an fp32 sum of the squares (no path through its tree has
+    // more than 9 roundings, so ||y||^2 is within 2^-20.8 relative and n
+    // within 2^-21.5); when n (1 -+ 2^-19) round to different fp16 values
+    // for any token of the warp, the warp sums again in fp64, where the
+    // squares of fp32 values are exact
+    unsigned short nb[2];
+    {
+      float sq[2];
 #pragma unroll
-    for (int G = 0; G < 8; ++G)
+      for (int t = 0; t < 2; ++t) {
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt)
+        for (int G = 0; G < 8; ++G)
+#pragma unroll
+          for (int nt = 0; nt < 2; ++nt) acc[(2 * G + nt) & 3] = f2_fma(y[G][nt][t], y[G][nt][t], acc[(2 * G + nt) & 3]);
+        const uint64_t a2 = f2_add(f2_add(acc[0], acc[1]), f2_add(acc[2], acc[3]));
+        float lo, hi;
+        f2_unpack(a2, lo, hi);
+        sq[t] = lo + hi;
+        sq[t] += __shfl_xor_sync(FULL, sq[t], 1);
+        sq[t] += __shfl_xor_sync(FULL, sq[t], 2);
+      }
+      bool unsure = false;
+#pragma unroll
+      for (int t = 0; t < 2; ++t) {
+        const float n32 = __fsqrt_rn(sq[t]);
+        nb[t] = __half_as_ushort(__float2half_rn(n32));
+        unsure |= __half_as_ushort(__float2half_rn(n32 * (1.0f - 0x1p-19f))) !=
+                  __half_as_ushort(__float2half_rn(n32 * (1.0f + 0x1p-19f)));
+      }
+      if (__any_sync(FULL, unsure)) {
 #pragma unroll
         for (int t = 0; t < 2; ++t) {
-          float a, b;
-          f2_unpack(y[G][nt][t], a, b);
-          ss[t] = fma((double)a, (double)a, fma((double)b, (double)b, ss[t]));
+          double ss = 0.0;
+#pragma unroll
+          for (int G = 0; G < 8; ++G)
+#pragma unroll
+            for (int nt = 0; nt < 2; ++nt) {
+              float a, b;
+              f2_unpack(y[G][nt][t], a, b);
+              ss = fma((double)a, (double)a, fma((double)b, (double)b, ss));
+            }
+          ss += __shfl_xor_sync(FULL, ss, 1);
+          ss += __shfl_xor_sync(FULL, ss, 2);
+          nb[t] = __half_as_ushort(__double2half(sqrt(ss)));
         }
-    unsigned short nb[2];
+      }
+    }
 #pragma unroll
     for (int t = 0; t < 2; ++t) {
-      ss[t] += __shfl_xor_sync(FULL, ss[t], 1);
-      ss[t] += __shfl_xor_sync(FULL, ss[t], 2);
-      nb[t] = __half_as_ushort(__double2half(sqrt(ss[t])));
       if ((nb[t] & 0x7FFF) >= 0x7C00) nb[t] = 0x7BFF;  // saturate at the largest finite fp16
       const float nf = __half2float(__ushort_as_half(nb[t]));
       const float S = nf > 0.0f ? __frcp_rn(nf) : 0.0f;
@@ -354,7 +388,7 @@ __global__ void __launch_bounds__(kOscarWriteWarps * 32) kvq_oscar_write_kernel(
           const float2 iv = *reinterpret_cast<const float2*>(smax + ch);
           const uint64_t z2 = f2_pack(z.x, z.y), i2 = f2_pack(iv.x, iv.y);
 #pragma unroll
-          for (int t = 0; t < 2; ++t) nib[t][k >> 2] |= int2_code_pair(y[G][nt][t], z2, i2) << (8 * (k & 3));
+          for (int t = 0; t < 2; ++t) nib[t][k >> 2] |= (int2_code_pair(y[G][nt][t], z2, i2) & 0xFu) << (8 * (k & 3));
         }
       oscar_store_codes(nib, kc, ok);
     }
@@ -404,7 +438,7 @@ __global__ void __launch_bounds__(kOscarWriteWarps * 32) kvq_oscar_write_kernel(
 #pragma unroll
           for (int nt = 0; nt < 2; ++nt) {
             const int k = 2 * G + nt;
-            nib[t][k >> 2] |= int2_code_pair(y[G][nt][t], z2, i2) << (8 * (k & 3));
+            nib[t][k >> 2] |= (int2_code_pair(y[G][nt][t], z2, i2) & 0xFu) << (8 * (k & 3));
           }
       }
       oscar_store_codes(nib, vc, ok);
@@ -432,6 +466,7 @@ struct OscarAttnParams {
   int n_splits, pages_per_split;
   int out_bf16;
   float qmul;                 // c_b * softmax_scale * log2(e)
+  float qraw;                 // softmax_scale * log2(e)
   float cb;
 };
 
@@ -453,6 +488,7 @@ struct OscarSmem {
   static constexpr int kOffRes = kOffQ + 4 * kQRow * 4;         // states: the warps', then the tail's
   static constexpr int kTotal = kOffRes + (kOscarWarps + 1) * kRes * 4;
 };
+
 
 __device__ __forceinline__ void e4m3x2_to_f16x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
   asm("{\n .reg .b16 a, b;\n mov.b32 {a, b}, %2;\n cvt.rn.f16x2.e4m3x2 %0, a;\n"
@@ -490,6 +526,9 @@ __global__ void __launch_bounds__(kOscarWarps * 32) kvq_oscar_decode_kernel(cons
   const int n_full = ctx >> 4, tail = ctx & 15;
   const int p0 = split * p.pages_per_split;
   const int p1 = min(p0 + p.pages_per_split, n_full);
+  // a split past the sequence's pages (and not holding its unfinished page)
+  // has nothing to add; the merge kernel does not read its workspace rows
+  if (p0 >= n_full && !(split == 0 && tail > 0)) return;
 
   // q~ = R q * qmul for the G query heads of kv head h (rows >= G zero)
   for (int r = warp; r < 4; r += kOscarWarps) {
@@ -513,12 +552,17 @@ __global__ void __launch_bounds__(kOscarWarps * 32) kvq_oscar_decode_kernel(cons
   uint8_t* ring = smem + warp * (R * SLOT);
   const uint32_t ring_s = smem_addr(ring);
   uint32_t valid = 0;
+  int ids = -1;  // page ids of this warp's pages 32 c .. 32 c + 31 (lane i: page 32 c + i)
   auto fetch = [&](int k) {
+    if ((k & 31) == 0) {
+      const int pl = p0 + warp + (k + lane) * kOscarWarps;
+      ids = pl < p1 ? p.page_table[(size_t)n * p.max_pages + pl] : -1;
+    }
+    const int id = __shfl_sync(FULL, ids, k & 31);
     const int pg = p0 + warp + k * kOscarWarps;
     const int slot = k % R;
     bool ok = false;
     if (pg < p1) {
-      const int id = p.page_table[(size_t)n * p.max_pages + pg];
       ok = id >= 0 && id < p.num_pages;
       if (ok) {
         const size_t ph = (size_t)id * p.Hkv + h;
@@ -545,8 +589,20 @@ __global__ void __launch_bounds__(kOscarWarps * 32) kvq_oscar_decode_kernel(cons
   const bool hv = tig < G;                 // this thread's logits belong to query head tig
   float m_run = hv ? -INFINITY : 0.0f, l_run = 0.0f, zs_run = 0.0f;
   const int hd = g >> 1, part = g & 1;     // this thread's B column: head hd, hi (0) or lo (1)
-  const float* qrow = qs + hd * S::kQRow + tig * S::kQSeg;  // channels 32 tig .. + 31 of head hd
   const int la = 8 * tig + (g >> 1), lb = la + 4;
+  // B = q~ of head hd as fp16 hi or lo, the same for every page: k-step j
+  // covers channels 32 tig + 4 j .. + 3 (rows 2 tig, + 1 -> channels + 0,
+  // + 1; rows 2 tig + 8, + 9 -> + 2, + 3)
+  uint32_t bq0[NJ], bq1[NJ];
+  {
+    const float* qrow = qs + hd * S::kQRow + tig * S::kQSeg;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      const float4 qv = *reinterpret_cast<const float4*>(qrow + 4 * j);
+      bq0[j] = hilo_pair(qv.x, qv.y, part);
+      bq1[j] = hilo_pair(qv.z, qv.w, part);
+    }
+  }
 
 #pragma unroll
   for (int k = 0; k < R - 1; ++k) fetch(k);
@@ -564,58 +620,46 @@ __global__ void __launch_bounds__(kOscarWarps * 32) kvq_oscar_decode_kernel(cons
       const __half* vsc = kno + 16;
       const __half* vze = kno + 32;
 
-      // B = q~ (.) s_c of head hd over channels 32 tig .. + 31 (k-step j:
-      // channels 32 tig + 4 j .. + 3), and this head's sum_c q~_c z_c part
-      uint32_t bq0[NJ], bq1[NJ];
-      float zpart = 0.0f;
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) {
-        const float4 qv = *reinterpret_cast<const float4*>(qrow + 4 * j);
-        const uint2 sw = *reinterpret_cast<const uint2*>(ksc + 32 * tig + 4 * j);
-        const uint2 zw = *reinterpret_cast<const uint2*>(kze + 32 * tig + 4 * j);
-        const float2 s01 = __half22float2(*reinterpret_cast<const __half2*>(&sw.x));
-        const float2 s23 = __half22float2(*reinterpret_cast<const __half2*>(&sw.y));
-        const float2 z01 = __half22float2(*reinterpret_cast<const __half2*>(&zw.x));
-        const float2 z23 = __half22float2(*reinterpret_cast<const __half2*>(&zw.y));
-        bq0[j] = hilo_pair(qv.x * s01.x, qv.y * s01.y, part);
-        bq1[j] = hilo_pair(qv.z * s23.x, qv.w * s23.y, part);
-        zpart = fmaf(qv.x, z01.x, fmaf(qv.y, z01.y, fmaf(qv.z, z23.x, fmaf(qv.w, z23.y, zpart))));
-      }
-      zpart += __shfl_xor_sync(FULL, zpart, 1);
-      zpart += __shfl_xor_sync(FULL, zpart, 2);
-      const float zsum = __shfl_sync(FULL, zpart, 8 * tig);  // the lane of head tig (g = 2 tig)
-
-      // A = K codes of tokens g and g + 8: bytes 8 tig .. 8 tig + 7 of each
-      // row; byte 8 tig + j is k-step j (codes 0, 1 -> columns 2 tig, +1;
-      // codes 2, 3 -> columns 2 tig + 8, + 9)
+      // QK by bit planes, code = b0 + 2 b1: A = b0 s_c, then b1 (2 s_c), both
+      // exact in fp16 (a select of s_c or 0). The bits of tokens g and g + 8
+      // come from K code bytes 8 tig .. 8 tig + 7 (byte 8 tig + j: k-step j,
+      // channels 32 tig + 4 j + c' at bits 2 c', 2 c' + 1); each shifted copy
+      // of a code word brings one bit position of every byte to bit 7, which
+      // prmt (in its sign mode) replicates across a half. sum_c q~_c z_c: an
+      // extra MMA whose A holds z in row 0 only.
       const uint2 ra = *reinterpret_cast<const uint2*>(kcode + g * (D / 4) + 8 * tig);
       const uint2 rc = *reinterpret_cast<const uint2*>(kcode + (g + 8) * (D / 4) + 8 * tig);
       float acc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
+      float zacc[4] = {0.0f, 0.0f, 0.0f, 0.0f};
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
         const uint32_t xa = half ? ra.y : ra.x, xc = half ? rc.y : rc.x;
-        uint32_t a01[4], a23[4], c01[4], c23[4];
-        auto split4 = [](uint32_t x, uint32_t (&lo4)[4], uint32_t (&hi4)[4]) {
-          const uint32_t e0 = x & 0x03030303u, e1 = (x >> 2) & 0x03030303u;
-          const uint32_t e2 = (x >> 4) & 0x03030303u, e3 = (x >> 6) & 0x03030303u;
-          e4m3x2_to_f16x2(prmt(e0, e1, 0x5140), lo4[0], lo4[1]);
-          e4m3x2_to_f16x2(prmt(e0, e1, 0x7362), lo4[2], lo4[3]);
-          e4m3x2_to_f16x2(prmt(e2, e3, 0x5140), hi4[0], hi4[1]);
-          e4m3x2_to_f16x2(prmt(e2, e3, 0x7362), hi4[2], hi4[3]);
-        };
-        split4(xa, a01, a23);
-        split4(xc, c01, c23);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int j = 4 * half + i;
-          const uint32_t a[4] = {a01[i], c01[i], a23[i], c23[i]};
-          mma_f16_16816(acc, a, bq0[j], bq1[j]);
+          // output bytes 0, 1 <- bit 7 of byte i of the first word, 2, 3 <- of the second
+          const uint32_t sel = (8u + i) | ((8u + i) << 4) | ((12u + i) << 8) | ((12u + i) << 12);
+          const uint2 sw = *reinterpret_cast<const uint2*>(ksc + 32 * tig + 4 * j);
+          const uint2 zw = *reinterpret_cast<const uint2*>(kze + 32 * tig + 4 * j);
+          uint32_t s2x, s2y;
+          asm("add.rn.f16x2 %0, %1, %1;\n" : "=r"(s2x) : "r"(sw.x));
+          asm("add.rn.f16x2 %0, %1, %1;\n" : "=r"(s2y) : "r"(sw.y));
+          const uint32_t a0[4] = {prmt(xa << 7, xa << 5, sel) & sw.x, prmt(xc << 7, xc << 5, sel) & sw.x,
+                                  prmt(xa << 3, xa << 1, sel) & sw.y, prmt(xc << 3, xc << 1, sel) & sw.y};
+          mma_f16_16816(acc, a0, bq0[j], bq1[j]);
+          const uint32_t a1[4] = {prmt(xa << 6, xa << 4, sel) & s2x, prmt(xc << 6, xc << 4, sel) & s2x,
+                                  prmt(xa << 2, xa, sel) & s2y, prmt(xc << 2, xc, sel) & s2y};
+          mma_f16_16816(acc, a1, bq0[j], bq1[j]);
+          const uint32_t az[4] = {g == 0 ? zw.x : 0u, 0u, g == 0 ? zw.y : 0u, 0u};
+          mma_f16_16816(zacc, az, bq0[j], bq1[j]);
         }
       }
+      const float zsum = __shfl_sync(FULL, zacc[0] + zacc[1], tig);  // row 0 = lane tig: head tig
+
       // logits (base 2) of tokens g and g + 8 for query head tig
       const float n0 = __half2float(kno[g]), n1 = __half2float(kno[g + 8]);
-      float lg0 = n0 * fmaf(acc[0] + acc[1], 512.0f, zsum);
-      float lg1 = n1 * fmaf(acc[2] + acc[3], 512.0f, zsum);
+      float lg0 = n0 * (acc[0] + acc[1] + zsum);
+      float lg1 = n1 * (acc[2] + acc[3] + zsum);
       if (!hv) lg0 = lg1 = -INFINITY;
       const float sv0 = __half2float(vsc[g]), sv1 = __half2float(vsc[g + 8]);
       const float zv0 = __half2float(vze[g]), zv1 = __half2float(vze[g + 8]);
@@ -700,14 +744,22 @@ __global__ void __launch_bounds__(kOscarWarps * 32) kvq_oscar_decode_kernel(cons
       mine[D + 2] = zs_run;
     }
   }
-  // ---- the unfinished page (split 0, warp 0): bf16 rows, rotated here -------
+  // ---- the unfinished page (split 0, warp 0): bf16 rows as they are -------
+  // q . k = (R q) . (R k), so the logits take the unrotated q and k; the
+  // weighted sum of the unrotated v is rotated once at the end.
   const bool has_tail = split == 0 && tail > 0;
   if (has_tail && warp == 0) {
-    float mt[4], lt[4], ot[4][E];
+    float mt[4], lt[4], ot[4][E], qr[4][E];
 #pragma unroll
     for (int r = 0; r < 4; ++r) {
       mt[r] = -INFINITY;
       lt[r] = 0.0f;
+      const int rr = r < G ? r : 0;
+      const uint2 w = *reinterpret_cast<const uint2*>(p.q + ((size_t)n * p.Hq + (size_t)h * G + rr) * D + E * lane);
+      qr[r][0] = __uint_as_float(w.x << 16) * p.qraw;
+      qr[r][1] = __uint_as_float(w.x & 0xffff0000u) * p.qraw;
+      qr[r][2] = __uint_as_float(w.y << 16) * p.qraw;
+      qr[r][3] = __uint_as_float(w.y & 0xffff0000u) * p.qraw;
 #pragma unroll
       for (int e = 0; e < E; ++e) ot[r][e] = 0.0f;
     }
@@ -720,20 +772,11 @@ __global__ void __launch_bounds__(kOscarWarps * 32) kvq_oscar_decode_kernel(cons
       kr[2] = __uint_as_float(kw.y << 16); kr[3] = __uint_as_float(kw.y & 0xffff0000u);
       vr[0] = __uint_as_float(vw.x << 16); vr[1] = __uint_as_float(vw.x & 0xffff0000u);
       vr[2] = __uint_as_float(vw.y << 16); vr[3] = __uint_as_float(vw.y & 0xffff0000u);
-      if constexpr (BLK > 0) {
-        warp_fwht<D, BLK>(kr, lane);
-        warp_fwht<D, BLK>(vr, lane);
-#pragma unroll
-        for (int e = 0; e < E; ++e) {
-          kr[e] *= p.cb;
-          vr[e] *= p.cb;
-        }
-      }
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         float d = 0.0f;
 #pragma unroll
-        for (int e = 0; e < E; ++e) d = fmaf(qs[r * S::kQRow + (lane >> 3) * S::kQSeg + E * (lane & 7) + e], kr[e], d);
+        for (int e = 0; e < E; ++e) d = fmaf(qr[r][e], kr[e], d);
 #pragma unroll
         for (int o2 = 16; o2 > 0; o2 >>= 1) d += __shfl_xor_sync(FULL, d, o2);
         const float mn = fmaxf(mt[r], d);
@@ -742,6 +785,14 @@ __global__ void __launch_bounds__(kOscarWarps * 32) kvq_oscar_decode_kernel(cons
 #pragma unroll
         for (int e = 0; e < E; ++e) ot[r][e] = fmaf(ot[r][e], a, pw * vr[e]);
         mt[r] = mn;
+      }
+    }
+    if constexpr (BLK > 0) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        warp_fwht<D, BLK>(ot[r], lane);
+#pragma unroll
+        for (int e = 0; e < E; ++e) ot[r][e] *= p.cb;
       }
     }
     float* st = res + kOscarWarps * S::kRes;
@@ -791,51 +842,75 @@ __global__ void __launch_bounds__(kOscarWarps * 32) kvq_oscar_decode_kernel(cons
 }
 
 // Merge the splits of each (sequence, query head), rotate back, store: one
-// warp per query row. The lanes first take the splits' maxima and weights
-// (split s on lane s % 32); then every lane sums its 4 channels over the
-// splits, eight splits' loads in flight at a time, with the weights read
-// back from shared memory.
+// CTA per query row, warp w taking splits 32 w .. 32 w + 31 (lane i: split
+// 32 w + i), so that every load of a row is in flight at once but for the
+// channel sums, sixteen splits deep.
 template <int D, int BLK>
 __global__ void __launch_bounds__(128) kvq_oscar_combine_kernel(const __grid_constant__ OscarAttnParams p) {
   constexpr int E = D / 32;
-  __shared__ float wts[4][kMaxSplits];
+  static_assert(kMaxSplits <= 128, "four warps of 32 splits");
+  __shared__ __align__(16) float part[4][D + 4];
+  __shared__ float wmax[4];
   pdl_wait();  // the decode kernel's partial results
   pdl_launch_dependents();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const unsigned FULL = 0xffffffffu;
-  const int row = blockIdx.x * 4 + warp;  // n * Hq + hq
-  if (row >= p.B * p.Hq) return;
+  const int row = blockIdx.x;  // n * Hq + hq
   const int n = row / p.Hq, hq = row % p.Hq, h = hq / p.G, r = hq % p.G;
-  const float* base = p.ws + (((size_t)n * p.Hkv + h) * p.n_splits * p.G + r) * (D + 2);
   const size_t sstride = (size_t)p.G * (D + 2);
-  const int ns = p.n_splits;
-  float M = -INFINITY;
-  for (int s = lane; s < ns; s += 32) M = fmaxf(M, base[s * sstride + D]);
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(FULL, M, o));
-  float L = 0.0f;
-  for (int s = lane; s < ns; s += 32) {
-    const float ms = base[s * sstride + D];
-    const float w = (ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
-    wts[warp][s] = w;
-    L = fmaf(w, base[s * sstride + D + 1], L);
+  const float* base = p.ws + (((size_t)n * p.Hkv + h) * p.n_splits * p.G + r) * (D + 2);
+  // splits that hold a part of this sequence (the decode kernel returns
+  // early from the others and leaves their rows unwritten)
+  int ctx = p.ctx_lens[n];
+  const int cap = p.max_pages * 16 + 15;
+  ctx = ctx < 0 ? 0 : (ctx > cap ? cap : ctx);
+  const int ns = ctx == 0 ? 0 : max(1, ((ctx >> 4) + p.pages_per_split - 1) / p.pages_per_split);
+  const int s = 32 * warp + lane;
+  float ms = -INFINITY, ls = 0.0f;
+  if (s < ns) {
+    ms = base[s * sstride + D];
+    ls = base[s * sstride + D + 1];
   }
+  float m = ms;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(FULL, m, o));
+  if (lane == 0) wmax[warp] = m;
+  __syncthreads();
+  const float M = fmaxf(fmaxf(wmax[0], wmax[1]), fmaxf(wmax[2], wmax[3]));
+  const float w = (ms == -INFINITY) ? 0.0f : fast_exp2(ms - M);
+  float L = w * ls;
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) L += __shfl_xor_sync(FULL, L, o);
-  __syncwarp();
   float v[E] = {0.0f, 0.0f, 0.0f, 0.0f};
-#pragma unroll 8
-  for (int s = 0; s < ns; ++s) {
-    const float w = wts[warp][s];
-    const float* sl = base + s * sstride + E * lane;
-    const float2 a = *reinterpret_cast<const float2*>(sl);
-    const float2 b = *reinterpret_cast<const float2*>(sl + 2);
-    v[0] = fmaf(w, a.x, v[0]);
-    v[1] = fmaf(w, a.y, v[1]);
-    v[2] = fmaf(w, b.x, v[2]);
-    v[3] = fmaf(w, b.y, v[3]);
+  const int cnt = max(0, min(32, ns - 32 * warp));
+  const float* sb = base + (size_t)(32 * warp) * sstride + E * lane;
+#pragma unroll 16
+  for (int i = 0; i < cnt; ++i) {
+    const float wi = __shfl_sync(FULL, w, i);
+    const float2 a = *reinterpret_cast<const float2*>(sb + i * sstride);
+    const float2 b = *reinterpret_cast<const float2*>(sb + i * sstride + 2);
+    v[0] = fmaf(wi, a.x, v[0]);
+    v[1] = fmaf(wi, a.y, v[1]);
+    v[2] = fmaf(wi, b.x, v[2]);
+    v[3] = fmaf(wi, b.y, v[3]);
   }
-  const float inv = (L > 0.0f) ? 1.0f / L : 0.0f;
+  *reinterpret_cast<float4*>(&part[warp][E * lane]) = make_float4(v[0], v[1], v[2], v[3]);
+  if (lane == 0) part[warp][D] = L;
+  __syncthreads();
+  if (warp != 0) return;
+  float Lt = 0.0f;
+#pragma unroll
+  for (int e = 0; e < E; ++e) v[e] = 0.0f;
+#pragma unroll
+  for (int w2 = 0; w2 < 4; ++w2) {
+    const float4 a = *reinterpret_cast<const float4*>(&part[w2][E * lane]);
+    v[0] += a.x;
+    v[1] += a.y;
+    v[2] += a.z;
+    v[3] += a.w;
+    Lt += part[w2][D];
+  }
+  const float inv = (Lt > 0.0f) ? 1.0f / Lt : 0.0f;
 #pragma unroll
   for (int e = 0; e < E; ++e) v[e] *= inv;
   if constexpr (BLK > 0) {

@@ -60,8 +60,10 @@ def parse_args(argv=None):
     ap.add_argument("--no-plain", action="store_true")
     ap.add_argument("--no-graph", action="store_true",
                     help="time direct launches instead of CUDA graph replays (for profilers)")
-    ap.add_argument("--only", choices=["write", "decode", "prefill"], default=None,
-                    help="time one kernel alone (profiling captures); prints its line")
+    ap.add_argument("--only", choices=["write", "decode", "prefill", "oscar"], default=None,
+                    help="time one kernel alone (profiling captures; oscar: the OScaR write and decode); "
+                         "prints its line")
+    ap.add_argument("--no-oscar", action="store_true", help="skip the OScaR variant's line")
     ap.add_argument("--e2e-steps", type=int, default=100)
     ap.add_argument("--no-configs", action="store_true",
                     help="skip the other workloads' write and decode lines")
@@ -738,6 +740,97 @@ def config_sweep(dev, steps, warm, rank, world, max_over_ranks):
 
 
 # ----------------------------------------------------------------------------
+# the OScaR variant (INT2: per-token norm scaling, K per channel) on the same
+# workload: each kernel alone, graph replays of back-to-back launches
+# ----------------------------------------------------------------------------
+
+OSCAR_PAGE_HEAD_BYTES = 2 * 16 * 128 // 4 + 2 * 2 * 128 + 3 * 2 * 16   # codes + K (s, z) + (n, V s, V z)
+
+
+def oscar_run(w, block, dev, steps, warm, max_over_ranks):
+    """kv_quant_write_oscar and paged_decode_attn_oscar on the workload's
+    full pages (each sequence's unfinished last page stays bf16 and is read
+    by the decode), each alone: a CUDA graph of `steps` launches rotating
+    through pools larger than L2, median of 3 replays."""
+    import numpy as np
+    import torch
+    import bit_kv_cache_20_b200 as kvq
+    from bit_kv_cache_20_b200 import workloads
+    k, v, ids, k_tail, v_tail = workloads.oscar_rows(w)
+    P = int(ids.size)
+    pool_bytes = max(P * w.Hkv * OSCAR_PAGE_HEAD_BYTES, 1)
+    n_pools = int(min(16, max(2, -(-300_000_000 // pool_bytes))))
+    pools = [kvq.alloc_oscar_cache(w.num_pages, w.Hkv, w.D, device=dev) for _ in range(n_pools)]
+    kc, vc, idc = k.to(dev), v.to(dev), torch.as_tensor(ids).to(dev)
+    full = max(1, int(max(int(c) // 16 for c in w.context_lens)))
+    pt = torch.as_tensor(np.ascontiguousarray(w.page_table[:, :full])).to(dev)
+    cl = torch.as_tensor(w.context_lens).to(dev)
+    q, ktc, vtc = w.q.to(dev), k_tail.to(dev), v_tail.to(dev)
+    out = torch.empty((w.B, w.Hq, w.D), dtype=torch.bfloat16, device=dev)
+    ws = torch.empty(kvq.oscar_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.num_pages, full, block, device=dev),
+                     dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(dev)
+    for pool in pools:
+        kvq.kv_quant_write_oscar(kc, vc, idc, *pool, block)
+    torch.cuda.synchronize(dev)
+
+    def graph_ms(fn):
+        with torch.cuda.stream(stream):
+            for j in range(warm):
+                fn(j)
+        stream.synchronize()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream, capture_error_mode="thread_local"):
+            for j in range(steps):
+                fn(warm + j)
+        with torch.cuda.stream(stream):
+            g.replay()
+        stream.synchronize()
+        ts = []
+        for _ in range(3):
+            t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            with torch.cuda.stream(stream):
+                t0.record(stream)
+                g.replay()
+                t1.record(stream)
+            t1.synchronize()
+            ts.append(t0.elapsed_time(t1) / steps)
+        del g
+        return statistics.median(ts)
+
+    def wr(j):
+        kvq.kv_quant_write_oscar(kc, vc, idc, *pools[j % n_pools], block, stream=stream)
+
+    def de(j):
+        kvq.paged_decode_attn_oscar(q, *pools[j % n_pools], pt, cl, ktc, vtc, out, block, ws, stream=stream)
+
+    wr_ms = max_over_ranks(graph_ms(wr))
+    de_ms = max_over_ranks(graph_ms(de))
+    assert kvq.get_device_error() == 0
+    tails = int(sum(int(c) % 16 for c in w.context_lens))
+    wbytes = P * w.Hkv * (16 * w.D * 2 * 2 + OSCAR_PAGE_HEAD_BYTES)
+    dbytes = P * w.Hkv * OSCAR_PAGE_HEAD_BYTES + tails * w.Hkv * w.D * 2 * 2 + 2 * w.B * w.Hq * w.D * 2
+    peak, _ = measured_peaks()
+    w_gbs, d_gbs = wbytes / (wr_ms / 1e3) / 1e9, dbytes / (de_ms / 1e3) / 1e9
+    del pools, kc, vc, ws
+    torch.cuda.empty_cache()
+    return {
+        "what": "OScaR: R, then each K token scaled to unit norm (fp16 norm kept), K INT2 per channel over "
+                "each 16-token page, V INT2 per token; the unfinished last page in bf16",
+        "hadamard_block": block, "pages": P, "bytes_per_page_head": OSCAR_PAGE_HEAD_BYTES,
+        "timing": f"each kernel alone: a CUDA graph of {steps} launches over {n_pools} pools (larger than "
+                  "L2), median of 3 replays",
+        "kernels": {
+            "kv_quant_write_oscar": {"us": round(1e3 * wr_ms, 3), "GB/s": round(w_gbs, 1),
+                                     "algorithmic_bytes": wbytes, "frac": round(w_gbs / peak, 4)},
+            "paged_decode_attn_oscar": {"us": round(1e3 * de_ms, 3), "GB/s": round(d_gbs, 1),
+                                        "algorithmic_bytes": dbytes, "frac": round(d_gbs / peak, 4),
+                                        "launches": 2},
+        },
+    }
+
+
+# ----------------------------------------------------------------------------
 # main
 # ----------------------------------------------------------------------------
 
@@ -826,6 +919,13 @@ def main(argv=None):
     def max_over_ranks(x):
         return reduce_max(x, world, dev)
 
+    if args.only == "oscar":
+        line = oscar_run(w, block, dev, args.steps, warm, max_over_ranks)
+        if rank == 0:
+            print(json.dumps({"only": "oscar", **line, "config": config_block(w, block)}), flush=True)
+        if world > 1:
+            dist.destroy_process_group()
+        return 0
     step = Step(w, block, dev, graph=not args.no_graph)
     step.fill_pools()
     if args.only == "prefill":
@@ -939,6 +1039,10 @@ def main(argv=None):
     pf_ms, pf_flops = prefill_run(step, 3, 1)
     pf_ms = max_over_ranks(pf_ms)
     del step
+    torch.cuda.empty_cache()
+
+    # the OScaR variant on the same workload (not part of the step)
+    oscar = None if args.no_oscar else oscar_run(w, block, dev, min(args.steps, 50), warm, max_over_ranks)
 
     # the other workloads, each kernel alone (not part of the step)
     configs = None
@@ -994,6 +1098,7 @@ def main(argv=None):
             "fused_us": round(1e3 * ap_fus_ms, 3),     # paged_decode_append_attn_int4
         },
         "prefill": prefill_line(pf_ms, pf_flops * world),
+        "oscar": oscar,
         "configs": configs,
         "e2e": e2e,
         "clocks": clocks.summary(),

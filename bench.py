@@ -694,9 +694,10 @@ SWEEP = (("serving-b64", None), ("llama2-70b-b8", None), ("stress-b256", (32, 64
 
 def config_sweep(dev, steps, warm, rank, world, max_over_ranks):
     """For every other workload: kv_quant_write and paged_decode_attn_int4
-    alone (graph replays of `steps` back-to-back launches, median of 3), at
-    its Hadamard block(s) and at 0 (plain INT4), with GB/s, the fraction of
-    the HBM peak and the rotation overhead."""
+    alone (graph replays of `steps` back-to-back launches), at its Hadamard
+    block(s) and at 0 (plain INT4), the blocks taking turns over three rounds
+    (median of 3), with GB/s, the fraction of the HBM peak and the rotation
+    overhead."""
     import torch
     from bit_kv_cache_20_b200 import workloads
     peak, _ = measured_peaks()
@@ -707,17 +708,24 @@ def config_sweep(dev, steps, warm, rank, world, max_over_ranks):
         blocks = tuple(blocks or (w.block,))
         wb = write_bytes(w.tokens_written, w.Hkv, w.D)
         db = decode_bytes(w.context_lens, w.B, w.Hq, w.Hkv, w.D, out_elem=2)
-        times = {}
+        # every block's Step set up first, then three rounds in which the
+        # blocks take turns: one block measured after the others would run
+        # on a hotter, more power-capped GPU than the first
+        sts = {}
         for b in (0,) + blocks:
-            st = Step(w, b, dev, graph=True)
-            st.fill_pools()
-            st.timed_only("write", warm)
-            st.timed_only("decode", warm)
-            wr = max_over_ranks(st.timed_only("write", steps, start_index=warm, rounds=3))
-            de = max_over_ranks(st.timed_only("decode", steps, start_index=warm, rounds=3))
-            times[b] = (wr, de)
-            del st
-            torch.cuda.empty_cache()
+            sts[b] = Step(w, b, dev, graph=True)
+            sts[b].fill_pools()
+            sts[b].timed_only("write", warm)
+            sts[b].timed_only("decode", warm)
+        ms = {b: ([], []) for b in sts}
+        for _ in range(3):
+            for b, st in sts.items():
+                ms[b][0].append(st.timed_only("write", steps, start_index=warm))
+                ms[b][1].append(st.timed_only("decode", steps, start_index=warm))
+        times = {b: (max_over_ranks(statistics.median(ms[b][0])), max_over_ranks(statistics.median(ms[b][1])))
+                 for b in sts}
+        del sts
+        torch.cuda.empty_cache()
 
         def line(b):
             wr, de = times[b]

@@ -61,12 +61,13 @@ constexpr int kOscarWriteWarps = 4;
 // Shared memory of one write warp: the 16 K and 16 V rows of its (group,
 // head) unit as bf16, each row padded by 16 bytes so that the eight row
 // addresses of an ldmatrix fall on distinct banks; then per-channel minimum
-// and maximum scratch, [8][136] floats each (a row stride of 544 bytes keeps
-// the float2 stores of one instruction within two wavefronts).
+// and maximum scratch for 64 channels, [8][72] floats each (a row stride of
+// 288 bytes keeps the float2 stores of one instruction within two
+// wavefronts). 13 KB a warp: four 4-warp CTAs fit on an SM.
 struct OscarWriteSmem {
   static constexpr int kRowBytes = 2 * 128 + 16;
   static constexpr int kRows = 32 * kRowBytes;
-  static constexpr int kStatStride = 136;
+  static constexpr int kStatStride = 72;
   static constexpr int kStats = 2 * 8 * kStatStride * 4;
   static constexpr int kWarp = kRows + kStats;
   static constexpr int kTotal = kOscarWriteWarps * kWarp;
@@ -202,7 +203,7 @@ __device__ __forceinline__ void oscar_store_codes(const uint32_t (&nib)[2][4], u
 // The next unit's K rows are fetched while this unit's K is quantized, its V
 // rows while this unit's V is.
 template <int D, int BLK>
-__global__ void __launch_bounds__(kOscarWriteWarps * 32) kvq_oscar_write_kernel(const OscarWriteParams p) {
+__global__ void __launch_bounds__(kOscarWriteWarps * 32, 4) kvq_oscar_write_kernel(const OscarWriteParams p) {
   static_assert(D == 128, "the OScaR path is built for head_dim 128");
   using SM = OscarWriteSmem;
   extern __shared__ __align__(128) uint8_t smem[];
@@ -334,65 +335,61 @@ __global__ void __launch_bounds__(kOscarWriteWarps * 32) kvq_oscar_write_kernel(
       tm[g + 8] = nb[1];
     }
     // per-channel min / max over the 16 tokens: tokens g, g + 8 here, then
-    // the 8 lanes of each tig through shared memory
+    // the 8 lanes of each tig through shared memory, 64 channels (groups
+    // 4 hc .. 4 hc + 3) at a time
+    uint32_t nib[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
 #pragma unroll
-    for (int G = 0; G < 8; ++G)
+    for (int hc = 0; hc < 2; ++hc) {
 #pragma unroll
-      for (int nt = 0; nt < 2; ++nt) {
-        float a0, a1, c0, c1;
-        f2_unpack(y[G][nt][0], a0, a1);
-        f2_unpack(y[G][nt][1], c0, c1);
-        const int ch = 16 * G + 8 * nt + 2 * tig;
-        *reinterpret_cast<float2*>(smin + g * SM::kStatStride + ch) = make_float2(fminf(a0, c0), fminf(a1, c1));
-        *reinterpret_cast<float2*>(smax + g * SM::kStatStride + ch) = make_float2(fmaxf(a0, c0), fmaxf(a1, c1));
-      }
-    __syncwarp();
-    {
-      float4 mn = *reinterpret_cast<const float4*>(smin + 4 * lane);
-      float4 mx = *reinterpret_cast<const float4*>(smax + 4 * lane);
-#pragma unroll
-      for (int r = 1; r < 8; ++r) {
-        const float4 a = *reinterpret_cast<const float4*>(smin + r * SM::kStatStride + 4 * lane);
-        const float4 b = *reinterpret_cast<const float4*>(smax + r * SM::kStatStride + 4 * lane);
-        mn = make_float4(fminf(mn.x, a.x), fminf(mn.y, a.y), fminf(mn.z, a.z), fminf(mn.w, a.w));
-        mx = make_float4(fmaxf(mx.x, b.x), fmaxf(mx.y, b.y), fmaxf(mx.z, b.z), fmaxf(mx.w, b.w));
-      }
-      const float lo[4] = {mn.x, mn.y, mn.z, mn.w}, up[4] = {mx.x, mx.y, mx.z, mx.w};
-      unsigned short sb[4], zb[4];
-      float zf[4], inv[4];
-#pragma unroll
-      for (int e = 0; e < 4; ++e) {
-        float sf;
-        int2_scale_zero(lo[e], up[e], sb[e], zb[e], sf, zf[e]);
-        inv[e] = (sf > 0.0f) ? __frcp_rn(sf) : 0.0f;
-      }
-      if (ok) {
-        *reinterpret_cast<uint2*>(kmeta + 4 * lane) =
-            make_uint2(sb[0] | ((uint32_t)sb[1] << 16), sb[2] | ((uint32_t)sb[3] << 16));
-        *reinterpret_cast<uint2*>(kmeta + D + 4 * lane) =
-            make_uint2(zb[0] | ((uint32_t)zb[1] << 16), zb[2] | ((uint32_t)zb[3] << 16));
-      }
-      // this lane's columns of row 0 now hold z and 1/s
-      *reinterpret_cast<float4*>(smin + 4 * lane) = make_float4(zf[0], zf[1], zf[2], zf[3]);
-      *reinterpret_cast<float4*>(smax + 4 * lane) = make_float4(inv[0], inv[1], inv[2], inv[3]);
-    }
-    __syncwarp();
-    {
-      uint32_t nib[2][4] = {{0u, 0u, 0u, 0u}, {0u, 0u, 0u, 0u}};
-#pragma unroll
-      for (int G = 0; G < 8; ++G)
+      for (int G = 4 * hc; G < 4 * hc + 4; ++G)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-          const int ch = 16 * G + 8 * nt + 2 * tig, k = 2 * G + nt;
+          float a0, a1, c0, c1;
+          f2_unpack(y[G][nt][0], a0, a1);
+          f2_unpack(y[G][nt][1], c0, c1);
+          const int ch = 16 * (G - 4 * hc) + 8 * nt + 2 * tig;
+          *reinterpret_cast<float2*>(smin + g * SM::kStatStride + ch) = make_float2(fminf(a0, c0), fminf(a1, c1));
+          *reinterpret_cast<float2*>(smax + g * SM::kStatStride + ch) = make_float2(fmaxf(a0, c0), fmaxf(a1, c1));
+        }
+      __syncwarp();
+      {
+        float2 mn = *reinterpret_cast<const float2*>(smin + 2 * lane);
+        float2 mx = *reinterpret_cast<const float2*>(smax + 2 * lane);
+#pragma unroll
+        for (int r = 1; r < 8; ++r) {
+          const float2 a = *reinterpret_cast<const float2*>(smin + r * SM::kStatStride + 2 * lane);
+          const float2 b = *reinterpret_cast<const float2*>(smax + r * SM::kStatStride + 2 * lane);
+          mn = make_float2(fminf(mn.x, a.x), fminf(mn.y, a.y));
+          mx = make_float2(fmaxf(mx.x, b.x), fmaxf(mx.y, b.y));
+        }
+        unsigned short sb0, zb0, sb1, zb1;
+        float sf0, sf1, zf0, zf1;
+        int2_scale_zero(mn.x, mx.x, sb0, zb0, sf0, zf0);
+        int2_scale_zero(mn.y, mx.y, sb1, zb1, sf1, zf1);
+        if (ok) {
+          *reinterpret_cast<uint32_t*>(kmeta + 64 * hc + 2 * lane) = sb0 | ((uint32_t)sb1 << 16);
+          *reinterpret_cast<uint32_t*>(kmeta + D + 64 * hc + 2 * lane) = zb0 | ((uint32_t)zb1 << 16);
+        }
+        // this lane's columns of row 0 now hold z and 1/s
+        *reinterpret_cast<float2*>(smin + 2 * lane) = make_float2(zf0, zf1);
+        *reinterpret_cast<float2*>(smax + 2 * lane) =
+            make_float2(sf0 > 0.0f ? __frcp_rn(sf0) : 0.0f, sf1 > 0.0f ? __frcp_rn(sf1) : 0.0f);
+      }
+      __syncwarp();
+#pragma unroll
+      for (int G = 4 * hc; G < 4 * hc + 4; ++G)
+#pragma unroll
+        for (int nt = 0; nt < 2; ++nt) {
+          const int ch = 16 * (G - 4 * hc) + 8 * nt + 2 * tig, k = 2 * G + nt;
           const float2 z = *reinterpret_cast<const float2*>(smin + ch);
           const float2 iv = *reinterpret_cast<const float2*>(smax + ch);
           const uint64_t z2 = f2_pack(z.x, z.y), i2 = f2_pack(iv.x, iv.y);
 #pragma unroll
           for (int t = 0; t < 2; ++t) nib[t][k >> 2] |= (int2_code_pair(y[G][nt][t], z2, i2) & 0xFu) << (8 * (k & 3));
         }
-      oscar_store_codes(nib, kc, ok);
+      __syncwarp();  // row 0 of the scratch is read before it is rewritten
     }
-    __syncwarp();  // row 0 of the scratch is read before the next unit rewrites it
+    oscar_store_codes(nib, kc, ok);
 
     // ---- V: rotate, token-wise INT2 ------------------------------------------
     cp_async_wait<1>();

@@ -104,6 +104,8 @@ KERNEL_SOURCES = {
     "kv_quant_write": ["kvq_write_tc.cuh", "kvq_write.cuh", "kvq_device.cuh"],
     "paged_decode_attn_int4": ["kvq_decode.cuh", "kvq_device.cuh"],
     "paged_prefill_attn_int4": ["kvq_prefill.cuh", "kvq_decode.cuh", "kvq_write_tc.cuh", "kvq_device.cuh"],
+    "kv_quant_write_oscar": ["kvq_oscar.cuh", "kvq_decode.cuh", "kvq_device.cuh"],
+    "paged_decode_attn_oscar": ["kvq_oscar.cuh", "kvq_decode.cuh", "kvq_device.cuh"],
 }
 
 
@@ -830,9 +832,11 @@ def oscar_run(w, block, dev, steps, warm, max_over_ranks):
                   "L2), median of 3 replays",
         "kernels": {
             "kv_quant_write_oscar": {"us": round(1e3 * wr_ms, 3), "GB/s": round(w_gbs, 1),
-                                     "algorithmic_bytes": wbytes, "frac": round(w_gbs / peak, 4)},
+                                     "algorithmic_bytes": wbytes, "frac": round(w_gbs / peak, 4),
+                                     "traffic": committed_traffic("kv_quant_write_oscar")},
             "paged_decode_attn_oscar": {"us": round(1e3 * de_ms, 3), "GB/s": round(d_gbs, 1),
                                         "algorithmic_bytes": dbytes, "frac": round(d_gbs / peak, 4),
+                                        "traffic": committed_traffic("paged_decode_attn_oscar"),
                                         "launches": 2},
         },
     }

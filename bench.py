@@ -712,7 +712,10 @@ def config_sweep(dev, steps, warm, rank, world, max_over_ranks):
         db = decode_bytes(w.context_lens, w.B, w.Hq, w.Hkv, w.D, out_elem=2)
         # every block's Step set up first, then three rounds in which the
         # blocks take turns: one block measured after the others would run
-        # on a hotter, more power-capped GPU than the first
+        # on a hotter, more power-capped GPU than the first. All writes come
+        # before all decodes: a decode timed right after a burst of the
+        # tensor-core write (b > 0) would start at the lower clock that
+        # burst leaves, one after the CUDA-core write (b = 0) would not
         sts = {}
         for b in (0,) + blocks:
             sts[b] = Step(w, b, dev, graph=True)
@@ -720,10 +723,10 @@ def config_sweep(dev, steps, warm, rank, world, max_over_ranks):
             sts[b].timed_only("write", warm)
             sts[b].timed_only("decode", warm)
         ms = {b: ([], []) for b in sts}
-        for _ in range(3):
-            for b, st in sts.items():
-                ms[b][0].append(st.timed_only("write", steps, start_index=warm))
-                ms[b][1].append(st.timed_only("decode", steps, start_index=warm))
+        for kind in (0, 1):
+            for _ in range(3):
+                for b, st in sts.items():
+                    ms[b][kind].append(st.timed_only(("write", "decode")[kind], steps, start_index=warm))
         times = {b: (max_over_ranks(statistics.median(ms[b][0])), max_over_ranks(statistics.median(ms[b][1])))
                  for b in sts}
         del sts

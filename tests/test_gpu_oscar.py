@@ -317,3 +317,49 @@ def test_oscar_argument_errors():
     with pytest.raises(kvq.KVQError) as e:
         kvq.paged_decode_attn_oscar(q, cache, kmeta, tmeta, pt, cl, tail, tail, out, 48, ws)
     assert e.value.status == 2
+
+
+def test_oscar_decode_out_of_range_inputs(orc):
+    """A page id outside the pool skips that page and records
+    KVQ_ERR_OUT_OF_RANGE; a context length above the table's capacity is
+    clamped (and recorded); the rest of the batch is unaffected."""
+    ctx = [90, 50]
+    w = workloads.random_case(61, 2, 4, 2, 128, 64, ctx)
+    pool, _, rows = write_both(orc, w, 64)
+    good, pt = gpu_decode(w, pool, rows, 64)
+    # sequence 1: a bad id in its page table
+    bad_pt = pt.copy()
+    bad_pt[1, 1] = w.num_pages + 5
+    _, _, ids, k_tail, v_tail = rows
+    out = torch.zeros((w.B, w.Hq, w.D), dtype=torch.float32, device="cuda")
+    nb = kvq.oscar_workspace_size(w.B, w.Hq, w.Hkv, w.D, w.num_pages, pt.shape[1], 64)
+    ws = torch.zeros(nb, dtype=torch.uint8, device="cuda")
+    kvq.paged_decode_attn_oscar(w.q.cuda(), *pool, torch.as_tensor(bad_pt).cuda(),
+                                torch.as_tensor(w.context_lens).cuda(), k_tail.cuda(), v_tail.cuda(), out, 64, ws)
+    torch.cuda.synchronize()
+    assert kvq.get_device_error() == 3
+    assert kvq.get_device_error() == 0
+    got = out.cpu().numpy()
+    assert np.array_equal(got[0], good[0].astype(np.float32))  # sequence 0 untouched
+    # a context length beyond max_pages * 16 + 15 is clamped to it
+    big = np.array(ctx, np.int32)
+    big[0] = pt.shape[1] * 16 + 100
+    kvq.paged_decode_attn_oscar(w.q.cuda(), *pool, torch.as_tensor(pt).cuda(), torch.as_tensor(big).cuda(),
+                                k_tail.cuda(), v_tail.cuda(), out, 64, ws)
+    torch.cuda.synchronize()
+    assert kvq.get_device_error() == 3
+    assert np.all(np.isfinite(out.cpu().numpy()))
+
+
+def test_oscar_empty_calls():
+    cache, kmeta, tmeta = kvq.alloc_oscar_cache(2, 2, 128)
+    e = torch.zeros((0, 2, 128), dtype=torch.bfloat16, device="cuda")
+    kvq.kv_quant_write_oscar(e, e, torch.zeros(0, dtype=torch.int32, device="cuda"), cache, kmeta, tmeta, 128)
+    q = torch.zeros((0, 4, 128), dtype=torch.bfloat16, device="cuda")
+    tail = torch.zeros((0, 2, 16, 128), dtype=torch.bfloat16, device="cuda")
+    out = torch.zeros((0, 4, 128), dtype=torch.float32, device="cuda")
+    ws = torch.zeros(16, dtype=torch.uint8, device="cuda")
+    kvq.paged_decode_attn_oscar(q, cache, kmeta, tmeta, torch.zeros((0, 1), dtype=torch.int32, device="cuda"),
+                                torch.zeros(0, dtype=torch.int32, device="cuda"), tail, tail, out, 128, ws)
+    torch.cuda.synchronize()
+    assert kvq.get_device_error() == 0

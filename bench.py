@@ -722,11 +722,22 @@ def config_sweep(dev, steps, warm, rank, world, max_over_ranks):
             sts[b].fill_pools()
             sts[b].timed_only("write", warm)
             sts[b].timed_only("decode", warm)
+        # Each kind starts with an untimed pass over every block (the clock
+        # settles at that kind's power level), and the block order rotates
+        # from round to round, so that no block always follows the heaviest
         ms = {b: ([], []) for b in sts}
-        for kind in (0, 1):
-            for _ in range(3):
-                for b, st in sts.items():
-                    ms[b][kind].append(st.timed_only(("write", "decode")[kind], steps, start_index=warm))
+        order = list(sts)
+        with ClockSampler(dev.index if dev.index is not None else 0) as clocks:
+            clocks.wait_first_sample()
+            t0 = time.monotonic()
+            for kind in (0, 1):
+                kname = ("write", "decode")[kind]
+                for b in order:
+                    sts[b].timed_only(kname, steps, start_index=warm)
+                for r in range(3):
+                    for b in order[r % len(order):] + order[:r % len(order)]:
+                        ms[b][kind].append(sts[b].timed_only(kname, steps, start_index=warm))
+            clocks.mark(t0, time.monotonic())
         times = {b: (max_over_ranks(statistics.median(ms[b][0])), max_over_ranks(statistics.median(ms[b][1])))
                  for b in sts}
         del sts
@@ -747,7 +758,7 @@ def config_sweep(dev, steps, warm, rank, world, max_over_ranks):
         out[name] = {"batch": w.B, "kv_heads": w.Hkv, "q_heads": w.Hq, "head_dim": w.D,
                      "context_tokens": int(w.context_lens.sum()), "written_tokens": w.tokens_written,
                      "write_bytes": wb, "decode_bytes": db,
-                     "blocks": {str(b): line(b) for b in (0,) + blocks}}
+                     "blocks": {str(b): line(b) for b in (0,) + blocks}, "clocks": clocks.summary()}
         del w
     return out
 

@@ -476,8 +476,8 @@ struct OscarSmem {
   static constexpr int kSlot = kCodes + 2 * D * 2 + 3 * 16 * 2; // + kmeta + tmeta
   static constexpr int kRing = kOscarWarps * kOscarRing * kSlot;
   // q~ rows: row r, channels 32 j .. 32 j + 31 at float r * kQRow + j * kQSeg;
-  // the padding puts the 16 (row, j) float4 reads of one k-step in 8
-  // distinct 16-byte bank groups (two wavefronts instead of sixteen)
+  // the padding puts the 16 (row, j) float4 reads of one k-step (when the
+  // B fragments are built, once per CTA) in 8 distinct 16-byte bank groups
   static constexpr int kQSeg = 36;
   static constexpr int kQRow = 4 * kQSeg;
   static constexpr int kOffQ = kRing;
@@ -486,7 +486,9 @@ struct OscarSmem {
   static constexpr int kTotal = kOffRes + (kOscarWarps + 1) * kRes * 4;
 };
 
-
+// Four bytes read as e4m3 -> two f16x2 registers (bytes 0, 1 and 2, 3). A
+// byte holding a 2-bit code c (bits 0-1, the rest zero) is the e4m3
+// subnormal c * 2^-9, which fp16 holds exactly.
 __device__ __forceinline__ void e4m3x2_to_f16x2(uint32_t x, uint32_t& lo, uint32_t& hi) {
   asm("{\n .reg .b16 a, b;\n mov.b32 {a, b}, %2;\n cvt.rn.f16x2.e4m3x2 %0, a;\n"
       " cvt.rn.f16x2.e4m3x2 %1, b;\n}\n"

@@ -682,8 +682,9 @@ def config_block(w, block, graph=True):
         "context": int(w.context_lens.max()), "written_tokens": w.tokens_written, "page": 16,
         "hadamard_block": block, "out_dtype": "bf16",
         "l2": "inputs larger than L2 rotate; decode reads a cache written two steps earlier",
-        "timing": timing + "; each kernel's line: the same, that kernel alone, median of 3 "
-                           "(alternating with the plain-INT4 kernel)",
+        "timing": timing + "; each kernel's line: the same, that kernel alone, median of 3 rounds "
+                           "in which the rotated, plain-INT4 and randomized-sign kernels take turns "
+                           "(all writes before all decodes, each kind after an untimed pass)",
     }
 
 
@@ -1001,21 +1002,26 @@ def main(argv=None):
         p_total = p.timed(args.steps, start_index=warm) if p is not None else None
         barrier()
         # each kernel alone, back to back, for its own line: the median of
-        # `rounds` measurements, rotated and plain alternating
+        # `rounds` measurements. Rotated, plain and randomized-sign variants
+        # take turns, their order rotating from round to round; all writes
+        # come first, then all decodes, each kind after an untimed pass of
+        # every variant, so that no decode is timed right after a burst of
+        # the power-hungrier tensor-core write and the clock it leaves
         ms = {k: [] for k in ("write", "decode", "p_write", "p_decode", "r_write", "r_decode",
                               "append_separate", "append_fused")}
-        for _ in range(rounds):
-            for kind in ("write", "decode"):
-                ms[kind].append(step.timed_only(kind, args.steps, start_index=warm))
+        variants = [("", step)] + ([("p_", p)] if p is not None else []) + ([("r_", r)] if r is not None else [])
+        for kind in ("write", "decode"):
+            for _, obj in variants:
+                obj.timed_only(kind, args.steps, start_index=warm)
                 barrier()
-                if p is not None:
-                    ms["p_" + kind].append(p.timed_only(kind, args.steps, start_index=warm))
+            for rd in range(rounds):
+                k0 = rd % len(variants)
+                for pre, obj in variants[k0:] + variants[:k0]:
+                    ms[pre + kind].append(obj.timed_only(kind, args.steps, start_index=warm))
                     barrier()
-                if r is not None:
-                    ms["r_" + kind].append(r.timed_only(kind, args.steps, start_index=warm))
-                    barrier()
-            # decode with a 1-token append per sequence: two launches or one
-            for kind in ("append_separate", "append_fused"):
+        # decode with a 1-token append per sequence: two launches or one
+        for rd in range(rounds):
+            for kind in (("append_separate", "append_fused") if rd % 2 == 0 else ("append_fused", "append_separate")):
                 ms[kind].append(step.timed_only(kind, args.steps, start_index=warm))
                 barrier()
         t_host1 = time.monotonic()

@@ -363,3 +363,28 @@ def test_oscar_empty_calls():
                                 torch.zeros(0, dtype=torch.int32, device="cuda"), tail, tail, out, 128, ws)
     torch.cuda.synchronize()
     assert kvq.get_device_error() == 0
+
+
+def test_oscar_write_full_size_plain_bit_exact(orc):
+    """The full 32768-token write at b = 0: every byte of every page-head
+    equal to the oracle's."""
+    w = workloads.make("llama3-8b-32k", block=0)
+    k, v, ids, _, _ = workloads.oscar_rows(w)
+    pool = gpu_pool(w.num_pages, w.Hkv, w.D)
+    kvq.kv_quant_write_oscar(k.cuda(), v.cuda(), torch.as_tensor(ids).cuda(), *pool, 0)
+    assert kvq.get_device_error() == 0
+    ora = orc.oscar_write(workloads.bf16_bits(k), workloads.bf16_bits(v), ids, w.num_pages, 0)
+    compare_oscar_write(orc, host(pool), ora, k, v, ids, 0)
+
+
+def test_oscar_decode_batched_gqa4(orc):
+    """Eight sequences of mixed lengths (tails of every size, one sequence
+    shorter than a page) in one call, GQA 4, b = 64, bf16 and fp32 out."""
+    ctx = [3000, 17, 1024, 2500, 15, 777, 4096, 1601]
+    w = workloads.random_case(77, len(ctx), 32, 8, 128, 64, ctx, n_outliers=4)
+    pool, _, rows = write_both(orc, w, 64)
+    got, pt = gpu_decode(w, pool, rows, 64)
+    ref = oracle_decode(orc, w, host(pool), rows, pt, 64)
+    assert_close(got, ref, "oscar decode batched")
+    got16, _ = gpu_decode(w, pool, rows, 64, out_dtype=torch.bfloat16)
+    assert float((np.abs(got16 - ref) - 2.0 ** -8 * np.abs(ref)).max()) <= TOL

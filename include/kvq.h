@@ -390,7 +390,10 @@ size_t kvq_oscar_workspace_size(const kvq_oscar_attn_desc* desc);
  *   back (R^T K^, R^T V^) or the bf16 rows of the unfinished page.
  * q            : device, bf16 [B][Hq][D], 16-byte aligned.
  * cache, kmeta, tmeta : as written by kv_quant_write_oscar with the same block.
- * page_table   : device, int32 [B][max_pages_per_seq].
+ * page_table   : device, int32 [B][max_pages_per_seq]; only the first
+ *                ctx / 16 entries of row n are read. An id outside
+ *                [0, num_pages) skips that page (its tokens get no weight)
+ *                and records KVQ_ERR_OUT_OF_RANGE.
  * context_lens : device, int32 [B]; above max_pages_per_seq * 16 + 15 it is
  *                clamped and records KVQ_ERR_OUT_OF_RANGE.
  * k_tail, v_tail : device, bf16 [B][Hkv][16][D].

@@ -74,21 +74,30 @@ struct OscarWriteSmem {
 };
 
 // INT2 (s, z) of a range: z = RD16(mn); s = the smallest fp16 with
-// 3 s + z >= mx (directed fp32 roundings give a candidate at most one fp16
-// step high; an exact fp64 test settles it).
+// 3 s + z >= mx. need = RU(RU(mx - z) * RU(1/3)) is at least (mx - z) / 3 and
+// within a few fp32 ulps of it, so RU16(need) is the answer or one fp16 step
+// above it. The step below, pb, is tested exactly in fp32: 3 pb is exact,
+// and 3 pb >= mx - z holds exactly when 3 pb >= RU(mx - z) (no fp32 value
+// lies strictly between the rounded-down and rounded-up difference).
 __device__ __forceinline__ void int2_scale_zero(float mn, float mx, unsigned short& sb, unsigned short& zb,
                                                 float& sf, float& zf) {
   const __half zh = __float2half_rd(mn);
   zf = __half2float(zh);
-  const float need = __fdiv_ru(__fsub_ru(mx, zf), 3.0f);
+  const float d = __fsub_ru(mx, zf);
+  const float need = __fmul_ru(d, 0.333333343f);  // RU(1/3)
   unsigned short s = __half_as_ushort(__float2half_ru(need));
   if (s != 0 && s < 0x7C00) {
     const unsigned short pb = (unsigned short)(s - 1);
-    if (fma(3.0, (double)__half2float(__ushort_as_half(pb)), (double)zf) >= (double)mx) s = pb;
+    if (__fmul_rn(3.0f, __half2float(__ushort_as_half(pb))) >= d) s = pb;
   }
   sb = s;
   zb = __half_as_ushort(zh);
   sf = __half2float(__ushort_as_half(s));
+}
+
+// Bytes 0 of four words, in order, as one word.
+__device__ __forceinline__ uint32_t gather_low_bytes(uint32_t a, uint32_t b, uint32_t c, uint32_t d) {
+  return prmt(prmt(a, b, 0x0040u), prmt(c, d, 0x0040u), 0x5410u);
 }
 
 // Two codes rint(fp32(u - z) * fp32(1/s)) (ties to even) as a nibble in
@@ -376,17 +385,24 @@ __global__ void __launch_bounds__(kOscarWriteWarps * 32, 4) kvq_oscar_write_kern
             make_float2(sf0 > 0.0f ? __frcp_rn(sf0) : 0.0f, sf1 > 0.0f ? __frcp_rn(sf1) : 0.0f);
       }
       __syncwarp();
+      uint32_t pk[2][8];  // [token][k - 8 hc]: a nibble in bits 0-3
 #pragma unroll
       for (int G = 4 * hc; G < 4 * hc + 4; ++G)
 #pragma unroll
         for (int nt = 0; nt < 2; ++nt) {
-          const int ch = 16 * (G - 4 * hc) + 8 * nt + 2 * tig, k = 2 * G + nt;
+          const int ch = 16 * (G - 4 * hc) + 8 * nt + 2 * tig, k = 2 * (G - 4 * hc) + nt;
           const float2 z = *reinterpret_cast<const float2*>(smin + ch);
           const float2 iv = *reinterpret_cast<const float2*>(smax + ch);
           const uint64_t z2 = f2_pack(z.x, z.y), i2 = f2_pack(iv.x, iv.y);
 #pragma unroll
-          for (int t = 0; t < 2; ++t) nib[t][k >> 2] |= (int2_code_pair(y[G][nt][t], z2, i2) & 0xFu) << (8 * (k & 3));
+          for (int t = 0; t < 2; ++t) pk[t][k] = int2_code_pair(y[G][nt][t], z2, i2);
         }
+#pragma unroll
+      for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int q = 0; q < 2; ++q)
+          nib[t][2 * hc + q] =
+              gather_low_bytes(pk[t][4 * q], pk[t][4 * q + 1], pk[t][4 * q + 2], pk[t][4 * q + 3]) & 0x0F0F0F0Fu;
       __syncwarp();  // row 0 of the scratch is read before it is rewritten
     }
     oscar_store_codes(nib, kc, ok);
@@ -430,13 +446,14 @@ __global__ void __launch_bounds__(kOscarWriteWarps * 32, 4) kvq_oscar_write_kern
           tm[32 + g + 8 * t] = zb;
         }
         const uint64_t z2 = f2_pack(zf, zf), i2 = f2_pack(iv, iv);
+        uint32_t pk[16];  // [k = 2 G + nt]: a nibble in bits 0-3
 #pragma unroll
         for (int G = 0; G < 8; ++G)
 #pragma unroll
-          for (int nt = 0; nt < 2; ++nt) {
-            const int k = 2 * G + nt;
-            nib[t][k >> 2] |= (int2_code_pair(y[G][nt][t], z2, i2) & 0xFu) << (8 * (k & 3));
-          }
+          for (int nt = 0; nt < 2; ++nt) pk[2 * G + nt] = int2_code_pair(y[G][nt][t], z2, i2);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          nib[t][q] = gather_low_bytes(pk[4 * q], pk[4 * q + 1], pk[4 * q + 2], pk[4 * q + 3]) & 0x0F0F0F0Fu;
       }
       oscar_store_codes(nib, vc, ok);
     }

@@ -462,11 +462,12 @@ __global__ void __launch_bounds__(32 * attn_warps(NC), NC == 1 ? 2 : 1)
     mx = __fmul_rn(mx, p.cb);
     const __half zh = __float2half_rd(mn);
     const float zf = __half2float(zh);
-    const float need = __fdiv_ru(__fsub_ru(mx, zf), 15.0f);
+    const float dz = __fsub_ru(mx, zf);
+    const float need = __fmul_ru(dz, 0.0666666701f);  // RU(1/15): a candidate at most one step high
     unsigned short sbits = __half_as_ushort(__float2half_ru(need));
-    if (sbits != 0 && sbits < 0x7C00) {  // one fp16 step lower may still cover max y
+    if (sbits != 0 && sbits < 0x7C00) {  // one fp16 step lower may still cover max y (exact fp32 test)
       const unsigned short pb = (unsigned short)(sbits - 1);
-      if (fma(15.0, (double)__half2float(__ushort_as_half(pb)), (double)zf) >= (double)mx) sbits = pb;
+      if (__fmul_rn(15.0f, __half2float(__ushort_as_half(pb))) >= dz) sbits = pb;
     }
     const float sf = __half2float(__ushort_as_half(sbits));
     const float inv = (sf > 0.0f) ? __frcp_rn(sf) : 0.0f;

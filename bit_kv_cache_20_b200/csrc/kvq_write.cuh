@@ -116,15 +116,16 @@ __global__ void __launch_bounds__(kWriteWarps * 32, 3) kvq_write_kernel(const Wr
     const float mx = fmaxf(fmaxf(mx4[0], mx4[1]), fmaxf(mx4[2], mx4[3]));
     // 2. z = largest fp16 <= mn; s = smallest fp16 with 15 s + z >= mx.
     //    Directed roundings give a candidate at most one fp16 step high; the
-    //    exact test (fp64: 15 s + z is exact there) settles it.
+    //    step below is tested exactly in fp32 (15 s is exact, and
+    //    15 s >= mx - z holds exactly when 15 s >= RU(mx - z)).
     const __half zh = __float2half_rd(mn);
     const float zf = __half2float(zh);
-    const float need = __fdiv_ru(__fsub_ru(mx, zf), 15.0f);
+    const float dz = __fsub_ru(mx, zf);
+    const float need = __fmul_ru(dz, 0.0666666701f);  // RU(1/15)
     unsigned short sb = __half_as_ushort(__float2half_ru(need));
     if (sb != 0 && sb < 0x7C00) {
       const unsigned short pb = (unsigned short)(sb - 1);
-      const float sp = __half2float(__ushort_as_half(pb));
-      if (fma(15.0, (double)sp, (double)zf) >= (double)mx) sb = pb;
+      if (__fmul_rn(15.0f, __half2float(__ushort_as_half(pb))) >= dz) sb = pb;
     }
     const float sf = __half2float(__ushort_as_half(sb));
     const float inv = (sf > 0.0f) ? __frcp_rn(sf) : 0.0f;

@@ -887,7 +887,8 @@ kvq_status kv_quant_write_oscar(const void* k, const void* v, const int32_t* pag
   if (!desc) return KVQ_ERR_INVALID_ARG;
   const kvq_oscar_write_desc& d = *desc;
   if (d.num_groups < 0 || d.num_kv_heads < 1 || d.num_pages < 1) return KVQ_ERR_INVALID_ARG;
-  if ((long long)d.num_groups * d.num_kv_heads > INT_MAX) return KVQ_ERR_INVALID_ARG;
+  // units (group, head) and unit + grid stride must stay in int
+  if ((long long)d.num_groups * d.num_kv_heads > INT_MAX / 2) return KVQ_ERR_INVALID_ARG;
   if (d.head_dim != 128 || !valid_block(d.head_dim, hadamard_block)) return KVQ_ERR_UNSUPPORTED;
   if (d.num_groups == 0) return KVQ_OK;
   if (!k || !v || !page_ids || !cache || !kmeta || !tmeta) return KVQ_ERR_INVALID_ARG;

@@ -36,7 +36,7 @@ def _worker(rank, world, port, results):
 
 def test_two_rank_weak_scaling_logic():
     world = 2
-    mgr = mp.Manager()
+    mgr = mp.get_context("spawn").Manager()  # no fork of a process that has threads
     results = mgr.dict()
     mp.spawn(_worker, args=(world, _free_port(), results), nprocs=world, join=True)
     assert results[0][0] == results[1][0] == 15.0          # max over ranks

@@ -229,10 +229,20 @@ __global__ void __launch_bounds__(kOscarWriteWarps * 32, 4) kvq_oscar_write_kern
   const int stride = gridDim.x * kOscarWriteWarps;
   const size_t row_stride = (size_t)p.Hkv * D;
 
+  // (group, head) of a unit, and of the unit one grid stride later, without
+  // a division per unit: unit = grp * Hkv + h
+  const int sg = stride / p.Hkv, sh = stride - sg * p.Hkv;
+  auto advance = [&](int& grp, int& h) {
+    grp += sg;
+    h += sh;
+    if (h >= p.Hkv) {
+      h -= p.Hkv;
+      ++grp;
+    }
+  };
   // one matrix (0: K, 1: V) of a unit: 16 rows of 256 bytes, 8 chunks a lane
-  auto stage = [&](int unit, int which) {
+  auto stage = [&](int unit, int grp, int h, int which) {
     if (unit < units) {
-      const int grp = unit / p.Hkv, h = unit - grp * p.Hkv;
       const uint16_t* src = (which ? p.v : p.k) + ((size_t)grp * 16 * p.Hkv + h) * D;
 #pragma unroll
       for (int j = 0; j < 8; ++j) {
@@ -260,10 +270,12 @@ __global__ void __launch_bounds__(kOscarWriteWarps * 32, 4) kvq_oscar_write_kern
   }
 
   int unit = blockIdx.x * kOscarWriteWarps + warp;
-  stage(unit, 0);
-  stage(unit, 1);
-  for (; unit < units; unit += stride) {
-    const int grp = unit / p.Hkv, h = unit - grp * p.Hkv;
+  int grp = unit / p.Hkv, h = unit - grp * p.Hkv;
+  stage(unit, grp, h, 0);
+  stage(unit, grp, h, 1);
+  for (; unit < units; unit += stride, advance(grp, h)) {
+    int ngrp = grp, nh = h;  // the next unit's
+    advance(ngrp, nh);
     const int page = p.page_ids[grp];
     const bool ok = page >= 0 && page < p.num_pages;
     if (!ok && lane == 0) record_error(KVQ_ERR_OUT_OF_RANGE);
@@ -279,7 +291,7 @@ __global__ void __launch_bounds__(kOscarWriteWarps * 32, 4) kvq_oscar_write_kern
     uint64_t y[8][2][2];
     oscar_rotate_rows<BLK>(rows_s, hb, p.cb, y);
     __syncwarp();
-    stage(unit + stride, 0);
+    stage(unit + stride, ngrp, nh, 0);
     // token norms: an fp32 sum of the squares (no path through its tree has
     // more than 9 roundings, so ||y||^2 is within 2^-20.8 relative and n
     // within 2^-21.5); when n (1 -+ 2^-19) round to different fp16 values
@@ -412,7 +424,7 @@ __global__ void __launch_bounds__(kOscarWriteWarps * 32, 4) kvq_oscar_write_kern
     __syncwarp();
     oscar_rotate_rows<BLK>(rows_s + 16 * SM::kRowBytes, hb, p.cb, y);
     __syncwarp();
-    stage(unit + stride, 1);
+    stage(unit + stride, ngrp, nh, 1);
     {
       float mn[2], mx[2];
 #pragma unroll
